@@ -1,0 +1,257 @@
+"""DualQuant dual-scale solver, written out step by step in float64.
+
+TEST INFRASTRUCTURE.  Plain, slow and meant to be read against the pages; only
+the tests, the smoke check and the benchmark's CPU-baseline leg use it.
+
+The method (DualQuant pages):
+* Model of a weight matrix, daiwk reproduction note, section "核心公式",
+  eq. (1):  W ~= D_a Q(D_a^-1 W D_b^-1) D_b  with outer inverse scales
+  a = alpha^-1 (one per row) and b = beta^-1 (one per column).
+* Closed-form updates with the codes held fixed, same section, eq. (2):
+  a_i <- Pi_Fa( sum_j W_ij R_ij / sum_j R_ij^2 ),  R = Qhat D_b,
+  b_j <- Pi_Fb( sum_i W_ij S_ij / sum_i S_ij^2 ),  S = D_a Qhat.
+* Order and conventions, text under eq. (2): re-quantize after the row update,
+  then solve the column update and re-quantize again; a slice whose codes are
+  all zero keeps scale 1; what is projected is the inverse scale.
+* The solver's inputs are only the weights, the format's quantizer and scale
+  set, an iteration count T and an initialization (trove summary, "How to use
+  it"); it never sees activations (daiwk note, "本地复现").
+* Activation side, eq. (1) second half: X W^T ~= (X D_b) Qhat^T D_a, i.e. the
+  activation is multiplied by b and then quantized (trove summary, "How to use
+  it": beta is applied inside the activation-quantization kernel).
+
+Readings taken where the pages are silent (each also listed in the design notes):
+* Inner copies equal the (synced) outer copies, so the grid input is W/(a b^T).
+* Pi_F is the nearest admissible value in linear distance: with the codes fixed
+  the objective in one scale is den * (x - x*)^2 + const, so the nearest value
+  of F is the exact constrained minimiser.  BF16: round to nearest even,
+  clamped to the normal range [2^-126, max].  E8M0: exponent in [-126, 126],
+  midpoint 1.5 * 2^k, an exact tie goes up.
+* Group quantizer Q: per row and group of G consecutive columns, m = max|Y|;
+  m == 0 gives the scale 1.0; else s = P_grp(m / qmax) with
+  - BF16: round to nearest even, clamped to [2^-126, max];
+  - E8M0: round up to a power of two (the smallest s with m/s <= qmax), clamp;
+  - E4M3: round to nearest even, saturating at 448; a positive value that
+    rounds to 0 becomes the smallest subnormal 2^-9.
+  Codes c = round(Y / (s * ts)) on the grid (INT4: half to even, clamp [-8,7];
+  E2M1: nearest, ties to even code, saturate 6).  Qhat = c * s * ts.
+* NVFP4 second-level (tensor) scale for weights: ts = 2^ceil(log2(amax(W) /
+  (448 * 6))), fixed from the input W at the start; ts = 1 for every other
+  format and for activations.
+* MSE = sum (W - D_a Qhat D_b)^2 / (rows * cols).  mse_trace[0] is the
+  initial state, mse_trace[t] the state after iteration t; mse_half[t-1] the
+  state right after the row half-step of iteration t.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import numpy as np
+
+from . import formats as F
+
+
+@dataclass(frozen=True)
+class Format:
+    codes: str            # "int4" | "e2m1"
+    group: int            # G, consecutive columns sharing a scale
+    gscale: str           # "bf16" | "e8m0" | "e4m3"
+    oscale: str           # "bf16" | "e8m0"   (set of the outer scales a, b)
+    tensor_scale_auto: bool = False
+
+    @property
+    def qmax(self) -> float:
+        return 7.0 if self.codes == "int4" else 6.0
+
+
+PRESETS = {
+    # daiwk note, 本地复现: signed INT4 [-8,7] with BF16 scales; Table 1 uses G64.
+    "int4_bf16": Format("int4", 64, "bf16", "bf16"),
+    # same codebook, E8M0 power-of-two scales, exponent in [-126, 126].
+    "mxint4": Format("int4", 32, "e8m0", "e8m0"),
+    # news article: MXFP4 = E2M1, 32-element blocks, E8M0 shared scale.
+    "mxfp4": Format("e2m1", 32, "e8m0", "e8m0"),
+    # news article: NVFP4 = E2M1, 16-element blocks, E4M3 scale; BF16 outer scales.
+    "nvfp4": Format("e2m1", 16, "e4m3", "bf16", tensor_scale_auto=True),
+}
+
+
+def preset(name: str, group: int | None = None) -> Format:
+    f = PRESETS[name]
+    if group is not None and group != f.group:
+        f = Format(f.codes, group, f.gscale, f.oscale, f.tensor_scale_auto)
+    return f
+
+
+# --------------------------------------------------------------------------- #
+# Projections
+# --------------------------------------------------------------------------- #
+
+def project_group_scale(g: np.ndarray, fmt: Format) -> np.ndarray:
+    """P_grp: admissible group scale for g = m / qmax (g > 0)."""
+    if fmt.gscale == "bf16":
+        return np.clip(F.round_bf16(g), F.BF16_MIN_NORMAL, F.BF16_MAX)
+    if fmt.gscale == "e8m0":
+        return F.e8m0_ceil(g)
+    if fmt.gscale == "e4m3":
+        s = F.round_e4m3(g)
+        return np.where(s == 0.0, F.E4M3_MIN_SUB, s)
+    raise ValueError(fmt.gscale)
+
+
+def project_outer(x: np.ndarray, fmt: Format) -> np.ndarray:
+    """Pi_F for the outer inverse scales (x > 0): nearest admissible value."""
+    if fmt.oscale == "bf16":
+        return np.clip(F.round_bf16(x), F.BF16_MIN_NORMAL, F.BF16_MAX)
+    if fmt.oscale == "e8m0":
+        return F.e8m0_nearest(x)
+    raise ValueError(fmt.oscale)
+
+
+def round_codes(q: np.ndarray, fmt: Format) -> np.ndarray:
+    return F.round_int4(q) if fmt.codes == "int4" else F.round_e2m1(q)
+
+
+def tensor_scale(W: np.ndarray, fmt: Format) -> float:
+    """NVFP4 weight tensor scale 2^ceil(log2(amax / (448 * qmax))); else 1."""
+    if not fmt.tensor_scale_auto:
+        return 1.0
+    amax = float(np.max(np.abs(W))) if W.size else 0.0
+    if amax == 0.0:
+        return 1.0
+    return float(F.e8m0_ceil(amax / (F.E4M3_MAX * fmt.qmax)))
+
+
+# --------------------------------------------------------------------------- #
+# The black-box group quantizer Q
+# --------------------------------------------------------------------------- #
+
+def quantize(Y: np.ndarray, fmt: Format, ts: float = 1.0):
+    """Q(Y) per row and group of G columns.
+
+    Returns (codes, scales): codes [rows, cols] as grid values, scales
+    [rows, cols/G] as the stored group scale values (without ts).
+    """
+    Y = np.asarray(Y, dtype=np.float64)
+    rows, cols = Y.shape
+    G = fmt.group
+    assert cols % G == 0
+    Yg = Y.reshape(rows, cols // G, G)
+    m = np.abs(Yg).max(axis=2)
+    pos = m > 0
+    s = np.where(pos, project_group_scale(np.where(pos, m / (fmt.qmax * ts), 1.0), fmt), 1.0)
+    c = round_codes(Yg / (s * ts)[..., None], fmt)
+    return c.reshape(rows, cols), s
+
+
+def dequantize(c: np.ndarray, s: np.ndarray, fmt: Format, ts: float = 1.0) -> np.ndarray:
+    rows, cols = c.shape
+    G = fmt.group
+    return (c.reshape(rows, cols // G, G) * (s * ts)[..., None]).reshape(rows, cols)
+
+
+def inner(W: np.ndarray, a: np.ndarray, b: np.ndarray) -> np.ndarray:
+    """Grid input D_a^-1 W D_b^-1 (inner copies equal to the outer ones)."""
+    return W / (a[:, None] * b[None, :])
+
+
+def qhat(W, a, b, fmt, ts=1.0):
+    c, s = quantize(inner(W, a, b), fmt, ts)
+    return dequantize(c, s, fmt, ts), c, s
+
+
+def mse(W, Qh, a, b) -> float:
+    R = W - a[:, None] * Qh * b[None, :]
+    return float(np.sum(R * R) / W.size)
+
+
+# --------------------------------------------------------------------------- #
+# Closed-form block updates (eq. (2))
+# --------------------------------------------------------------------------- #
+
+def row_update(W, Qh, b, fmt):
+    """a_i <- Pi(sum_j W_ij R_ij / sum_j R_ij^2), R = Qhat D_b; zero slice -> 1.
+
+    Returns (a_new, x_pre) with x_pre the unprojected ratio (nan on zero slices).
+    """
+    R = Qh * b[None, :]
+    num = np.sum(W * R, axis=1)
+    den = np.sum(R * R, axis=1)
+    pos = den > 0
+    x = np.where(pos, num / np.where(pos, den, 1.0), np.nan)
+    a = np.where(pos, project_outer(np.where(pos, x, 1.0), fmt), 1.0)
+    return a, x
+
+
+def col_update(W, Qh, a, fmt):
+    """b_j <- Pi(sum_i W_ij S_ij / sum_i S_ij^2), S = D_a Qhat; zero slice -> 1."""
+    S = a[:, None] * Qh
+    num = np.sum(W * S, axis=0)
+    den = np.sum(S * S, axis=0)
+    pos = den > 0
+    x = np.where(pos, num / np.where(pos, den, 1.0), np.nan)
+    b = np.where(pos, project_outer(np.where(pos, x, 1.0), fmt), 1.0)
+    return b, x
+
+
+# --------------------------------------------------------------------------- #
+# Block coordinate descent
+# --------------------------------------------------------------------------- #
+
+def solve(W, fmt: Format, T: int, a0=None, b0=None):
+    """DualQuant solve: T iterations of row update, re-quantize, column
+    update, re-quantize (the flowchart of the daiwk note and the trove summary).
+    """
+    W = np.asarray(W, dtype=np.float64)
+    rows, cols = W.shape
+    a = np.ones(rows) if a0 is None else np.asarray(a0, dtype=np.float64).copy()
+    b = np.ones(cols) if b0 is None else np.asarray(b0, dtype=np.float64).copy()
+    ts = tensor_scale(W, fmt)
+    Qh, c, s = qhat(W, a, b, fmt, ts)
+    trace, half = [mse(W, Qh, a, b)], []
+    for _ in range(T):
+        a, xa = row_update(W, Qh, b, fmt)
+        Qh, c, s = qhat(W, a, b, fmt, ts)
+        half.append(mse(W, Qh, a, b))
+        b, xb = col_update(W, Qh, a, fmt)
+        Qh, c, s = qhat(W, a, b, fmt, ts)
+        trace.append(mse(W, Qh, a, b))
+    return dict(a=a, b=b, codes=c, scales=s, ts=ts, qhat=Qh,
+                mse_trace=np.array(trace), mse_half=np.array(half))
+
+
+def act_rescale_quant(X, b, fmt: Format):
+    """Q_act(X D_b): multiply each input channel by b_j, then group-quantize
+    with ts = 1.  Returns (codes, scales) as values."""
+    X = np.asarray(X, dtype=np.float64)
+    return quantize(X * np.asarray(b, dtype=np.float64)[None, :], fmt, 1.0)
+
+
+# --------------------------------------------------------------------------- #
+# Stored form (what the library writes)
+# --------------------------------------------------------------------------- #
+
+def encode_codes(c: np.ndarray, fmt: Format) -> np.ndarray:
+    nib = F.encode_int4(c) if fmt.codes == "int4" else F.encode_e2m1(c)
+    return F.pack_nibbles(nib)
+
+
+def encode_scales(s: np.ndarray, fmt: Format) -> np.ndarray:
+    if fmt.gscale == "bf16":
+        return F.encode_bf16(s)
+    if fmt.gscale == "e8m0":
+        return F.encode_e8m0(s)
+    return F.encode_e4m3(s)
+
+
+def decode_codes(packed: np.ndarray, fmt: Format) -> np.ndarray:
+    nib = F.unpack_nibbles(packed)
+    return F.decode_int4(nib) if fmt.codes == "int4" else F.decode_e2m1(nib)
+
+
+def decode_scales(u: np.ndarray, fmt: Format) -> np.ndarray:
+    if fmt.gscale == "bf16":
+        return F.decode_bf16(u)
+    if fmt.gscale == "e8m0":
+        return F.decode_e8m0(u)
+    return F.decode_e4m3(u)

@@ -1,0 +1,359 @@
+"""Pins of the oracle's quantizer, closed-form updates and loop (no GPU).
+
+Each check rests on something other than the oracle itself: an exact
+rational re-derivation in pure Python, a brute-force scan over every
+admissible scale, a mathematical property of the method (least squares with
+fixed codes, power-of-two invariance) or a hand-derived case.
+"""
+from fractions import Fraction as Fr
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import synth
+
+FORMATS = ["int4_bf16", "mxint4", "mxfp4", "nvfp4"]
+E2M1 = [Fr(0), Fr(1, 2), Fr(1), Fr(3, 2), Fr(2), Fr(3), Fr(4), Fr(6)]
+
+
+# --------------------------------------------------------------------------- #
+# An exact rational restatement of Q, pure Python, for small matrices
+# --------------------------------------------------------------------------- #
+
+def _floor_log2(x: Fr) -> int:
+    e = 0
+    while Fr(2) ** e > x:
+        e -= 1
+    while Fr(2) ** (e + 1) <= x:
+        e += 1
+    return e
+
+
+def _rne(x: Fr, p: int, emin: int, maxval: Fr) -> Fr:
+    e = max(_floor_log2(x), emin)
+    quantum = Fr(2) ** (e - (p - 1))
+    v = round(x / quantum) * quantum           # round() on Fraction: half to even
+    return min(v, maxval)
+
+
+def py_group_scale(g: Fr, gscale: str) -> Fr:
+    if gscale == "bf16":
+        v = _rne(g, 8, -126, Fr(2) ** 127 * (2 - Fr(1, 128)))
+        return max(v, Fr(2) ** -126)
+    if gscale == "e8m0":
+        e = -126
+        while Fr(2) ** e < g and e < 126:
+            e += 1
+        return Fr(2) ** e
+    v = _rne(g, 4, -6, Fr(448))
+    return v if v > 0 else Fr(2) ** -9
+
+
+def py_code(q: Fr, codes: str) -> Fr:
+    if codes == "int4":
+        return Fr(min(7, max(-8, round(q))))
+    aq = min(abs(q), Fr(6))
+    d = [abs(aq - g) for g in E2M1]
+    best = min(d)
+    idx = [i for i in range(8) if d[i] == best]
+    i = idx[0] if len(idx) == 1 else [i for i in idx if i % 2 == 0][0]
+    return E2M1[i] if q >= 0 else -E2M1[i]
+
+
+def py_quantize(Y, fmt, ts=Fr(1)):
+    rows, cols = len(Y), len(Y[0])
+    G = fmt.group
+    C = [[None] * cols for _ in range(rows)]
+    S = [[None] * (cols // G) for _ in range(rows)]
+    for i in range(rows):
+        for g in range(cols // G):
+            grp = Y[i][g * G:(g + 1) * G]
+            m = max(abs(v) for v in grp)
+            s = Fr(1) if m == 0 else py_group_scale(m / (Fr(int(fmt.qmax)) * ts), fmt.gscale)
+            S[i][g] = s
+            for k, v in enumerate(grp):
+                C[i][g * G + k] = py_code(v / (s * ts), fmt.codes)
+    return C, S
+
+
+def _small_matrix(rows, cols, seed, outliers=True):
+    rng = np.random.default_rng(seed)
+    W = rng.standard_t(4, (rows, cols)) * 0.02
+    if outliers:
+        W[:, rng.choice(cols, 3, replace=False)] *= 10
+    return torch.from_numpy(W).to(torch.bfloat16).double().numpy()
+
+
+@pytest.mark.parametrize("name", FORMATS)
+@pytest.mark.parametrize("G", [16, 32, 64])
+def test_quantize_matches_exact_rational_restatement(name, G):
+    fmt = O.preset(name, G)
+    W = _small_matrix(3, 2 * G, seed=G)
+    rng = np.random.default_rng(3)
+    a = O.project_outer(np.exp(rng.uniform(-1, 1, 3)), fmt)
+    b = O.project_outer(np.exp(rng.uniform(-1, 1, 2 * G)), fmt)
+    ts = 2.0 ** -9 if fmt.tensor_scale_auto else 1.0
+    c, s = O.quantize(O.inner(W, a, b), fmt, ts)
+    Y = [[Fr(float(W[i, j])) / (Fr(float(a[i])) * Fr(float(b[j]))) for j in range(2 * G)]
+         for i in range(3)]
+    C, S = py_quantize(Y, fmt, Fr(ts))
+    assert np.array_equal(c, np.array([[float(v) for v in r] for r in C]))
+    assert np.array_equal(s, np.array([[float(v) for v in r] for r in S]))
+
+
+def test_quantize_hand_cases():
+    # INT4 with BF16 scale, G16: max 7/8 -> s = (7/8)/7 = 1/8 exactly; codes are
+    # Y*8 rounded half to even: 3.5->4, -3.5->-4, 2.5->2, 0.5->0, 1.5->2.
+    fmt = O.preset("int4_bf16", 16)
+    y = np.array([7, 3.5, -3.5, 2.5, 0.5, -0.5, 1.5, 0, 1, 2, 3, 4, 5, 6, -7, 6.5]) / 8.0
+    c, s = O.quantize(y[None, :], fmt)
+    assert s[0, 0] == 0.125
+    assert list(c[0]) == [7, 4, -4, 2, 0, 0, 2, 0, 1, 2, 3, 4, 5, 6, -7, 6]
+    # MXFP4, G32: max 1.5 -> 1.5/6 = 0.25 is a power of two -> s = 0.25; codes
+    # on the E2M1 grid: 0.25->0, 0.75->1, 1.25->1, 1.75->2, 2.5->2, 3.5->4, 5->4.
+    fmt = O.preset("mxfp4", 32)
+    q = np.array([6, 0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5] + [0] * 24, dtype=float)
+    c, s = O.quantize((q * 0.25)[None, :], fmt)
+    assert s[0, 0] == 0.25
+    assert list(c[0, :8]) == [6, 0, 1, 1, 2, 2, 4, 4]
+    # MXINT4: max 7.5/16 -> 7.5/16/7 is just above 1/16 -> rounds up to 1/8;
+    # then 7.5/16 / (1/8) = 3.75 -> 4.
+    fmt = O.preset("mxint4", 32)
+    c, s = O.quantize(np.array([[7.5 / 16] + [0.0] * 31]), fmt)
+    assert s[0, 0] == 0.125 and c[0, 0] == 4
+    # NVFP4 (ts=1): max 1.8 -> 1.8/6 = 0.3 -> E4M3 nearest 0.3125 (1.010b x 2^-2).
+    fmt = O.preset("nvfp4", 16)
+    c, s = O.quantize(np.array([[1.8] + [0.0] * 15]), fmt)
+    assert s[0, 0] == 0.3125 and c[0, 0] == 6     # 5.76 -> 6
+    # all-zero group: scale 1, codes 0
+    c, s = O.quantize(np.zeros((1, 16)), fmt)
+    assert s[0, 0] == 1.0 and np.all(c == 0)
+    # E4M3 saturation: max/6 above 448 -> s = 448, codes saturate at 6
+    c, s = O.quantize(np.array([[6000.0, -3000.0] + [0.0] * 14]), fmt)
+    assert s[0, 0] == 448.0 and c[0, 0] == 6 and c[0, 1] == -6
+
+
+@pytest.mark.parametrize("name", FORMATS)
+def test_quantizer_idempotent(name):
+    fmt = O.preset(name)
+    W = _small_matrix(16, 4 * fmt.group, seed=5)
+    # adversarial groups: maxima exactly on scale boundaries
+    W[0, :fmt.group] = np.linspace(-1, 1, fmt.group) * fmt.qmax * 2.0 ** -4
+    W[1, :fmt.group] *= 0.0
+    W[1, 0] = 1.5 * 2.0 ** -5
+    ts = O.tensor_scale(W, fmt)
+    c, s = O.quantize(W, fmt, ts)
+    Qh = O.dequantize(c, s, fmt, ts)
+    c2, s2 = O.quantize(Qh, fmt, ts)
+    assert np.array_equal(O.dequantize(c2, s2, fmt, ts), Qh)
+
+
+def test_tensor_scale():
+    fmt = O.preset("nvfp4")
+    W = np.zeros((1, 16))
+    W[0, 3] = 448 * 6 * 2.0 ** -3
+    assert O.tensor_scale(W, fmt) == 2.0 ** -3
+    W[0, 3] = np.nextafter(W[0, 3], np.inf)
+    assert O.tensor_scale(W, fmt) == 2.0 ** -2
+    assert O.tensor_scale(np.zeros((2, 16)), fmt) == 1.0
+    assert O.tensor_scale(W, O.preset("mxfp4")) == 1.0
+
+
+# --------------------------------------------------------------------------- #
+# Closed-form updates: brute force over every admissible scale
+# --------------------------------------------------------------------------- #
+
+def _admissible(fmt, x):
+    if fmt.oscale == "e8m0":
+        return 2.0 ** np.arange(-126, 127)
+    # every bf16 value within a factor 4 of x
+    u = np.arange(1 << 15, dtype=np.uint32)
+    v = (u << 16).view(np.float32)
+    v = v[np.isfinite(v)].astype(np.float64)
+    v = v[v >= 2.0 ** -126]
+    return v[(v > x / 4) & (v < x * 4)]
+
+
+@pytest.mark.parametrize("name", FORMATS)
+def test_row_and_column_updates_minimise_over_the_scale_set(name):
+    fmt = O.preset(name)
+    W = _small_matrix(6, 2 * fmt.group, seed=17)
+    rng = np.random.default_rng(2)
+    a0 = O.project_outer(np.exp(rng.uniform(-0.5, 0.5, 6)), fmt)
+    b0 = O.project_outer(np.exp(rng.uniform(-0.5, 0.5, 2 * fmt.group)), fmt)
+    ts = O.tensor_scale(W, fmt)
+    Qh, _, _ = O.qhat(W, a0, b0, fmt, ts)
+    a, xa = O.row_update(W, Qh, b0, fmt)
+    R = Qh * b0[None, :]
+    for i in range(6):
+        cand = _admissible(fmt, xa[i])
+        obj = ((W[i][None, :] - cand[:, None] * R[i][None, :]) ** 2).sum(1)
+        mine = ((W[i] - a[i] * R[i]) ** 2).sum()
+        assert mine <= obj.min() * (1 + 1e-12), (i, a[i], cand[obj.argmin()])
+    b, xb = O.col_update(W, Qh, a0, fmt)
+    S = a0[:, None] * Qh
+    for j in range(2 * fmt.group):
+        cand = _admissible(fmt, xb[j])
+        obj = ((W[:, j][None, :] - cand[:, None] * S[:, j][None, :]) ** 2).sum(1)
+        mine = ((W[:, j] - b[j] * S[:, j]) ** 2).sum()
+        assert mine <= obj.min() * (1 + 1e-12), (j, b[j], cand[obj.argmin()])
+
+
+def test_closed_form_ratio_direction():
+    # With Qhat fixed and one row, the unprojected a* is <W,R>/<R,R>
+    # (least squares of W ~ a R); a 2-element case worked by hand:
+    # W = [2, 1], R = [1, 1] -> a* = 3/2.
+    fmt = O.preset("int4_bf16", 16)
+    W = np.zeros((1, 16))
+    W[0, :2] = [2.0, 1.0]
+    Qh = np.zeros((1, 16))
+    Qh[0, :2] = [1.0, 1.0]
+    a, x = O.row_update(W, Qh, np.ones(16), fmt)
+    assert x[0] == 1.5 and a[0] == 1.5
+    b, xb = O.col_update(W, Qh, np.array([2.0]), fmt)
+    assert xb[0] == 1.0 and xb[1] == 0.5       # (2*2)/(2*2), (1*2)/(2*2)
+
+
+def test_zero_slices_keep_scale_one():
+    fmt = O.preset("int4_bf16", 32)
+    W = _small_matrix(4, 64, seed=3)
+    W[:, 5] = 1e-6                                 # tiny column: codes all zero
+    W[2, :] = 0.0                                  # all-zero row
+    Qh, c, _ = O.qhat(W, np.full(4, 0.5), np.full(64, 2.0), fmt)
+    assert np.all(c[:, 5] == 0) and np.all(c[2] == 0)
+    a, xa = O.row_update(W, Qh, np.full(64, 2.0), fmt)
+    b, xb = O.col_update(W, Qh, np.full(4, 0.5), fmt)
+    assert a[2] == 1.0 and np.isnan(xa[2])
+    assert b[5] == 1.0 and np.isnan(xb[5])
+
+
+@pytest.mark.parametrize("name", FORMATS)
+def test_outputs_are_representable(name):
+    fmt = O.preset(name)
+    W = _small_matrix(32, 4 * fmt.group, seed=23)
+    r = O.solve(W, fmt, 3)
+    O.encode_scales(r["scales"], fmt)                              # raises if not
+    O.encode_codes(r["codes"], fmt)
+    if fmt.oscale == "e8m0":
+        from oracle import formats as F
+        F.encode_e8m0(r["a"]), F.encode_e8m0(r["b"])
+    else:
+        assert np.array_equal(O.project_outer(r["a"], fmt), r["a"])
+        assert np.array_equal(O.project_outer(r["b"], fmt), r["b"])
+
+
+# --------------------------------------------------------------------------- #
+# The loop
+# --------------------------------------------------------------------------- #
+
+def test_initial_state_is_single_scale_rtn():
+    fmt = O.preset("int4_bf16", 16)
+    W = _small_matrix(4, 48, seed=31)
+    r = O.solve(W, fmt, 0)
+    C, S = py_quantize([[Fr(float(v)) for v in row] for row in W], fmt)
+    err = sum((Fr(float(W[i, j])) - C[i][j] * S[i][j // 16]) ** 2
+              for i in range(4) for j in range(48)) / (4 * 48)
+    assert r["mse_trace"][0] == pytest.approx(float(err), rel=1e-13)
+
+
+@pytest.mark.parametrize("name", FORMATS)
+def test_fixed_code_half_steps_never_increase_the_error(name):
+    # with the codes held fixed, each closed-form + nearest-projection step is
+    # the exact minimiser over the scale set, so it cannot raise the MSE
+    fmt = O.preset(name)
+    W = _small_matrix(24, 4 * fmt.group, seed=41)
+    ts = O.tensor_scale(W, fmt)
+    a, b = np.ones(24), np.ones(4 * fmt.group)
+    for _ in range(4):
+        Qh, _, _ = O.qhat(W, a, b, fmt, ts)
+        before = O.mse(W, Qh, a, b)
+        a2, _ = O.row_update(W, Qh, b, fmt)
+        assert O.mse(W, Qh, a2, b) <= before * (1 + 1e-13)
+        a = a2
+        Qh, _, _ = O.qhat(W, a, b, fmt, ts)
+        before = O.mse(W, Qh, a, b)
+        b2, _ = O.col_update(W, Qh, a, fmt)
+        assert O.mse(W, Qh, a, b2) <= before * (1 + 1e-13)
+        b = b2
+
+
+@pytest.mark.parametrize("name", ["mxint4", "mxfp4"])
+def test_power_of_two_row_step_leaves_mx_reconstruction_unchanged(name):
+    # E8M0 row scale with E8M0 group scales: a power of two only shifts every
+    # group exponent, so D_a Qhat is unchanged and the row half-step MSE equals
+    # the previous full-step MSE exactly.
+    fmt = O.preset(name)
+    W = _small_matrix(16, 4 * fmt.group, seed=43)
+    r = O.solve(W, fmt, 4)
+    assert np.array_equal(r["mse_half"], r["mse_trace"][:-1])
+
+
+@pytest.mark.parametrize("name", FORMATS)
+def test_dual_scale_beats_single_scale_on_outlier_matrices(name):
+    fmt = O.preset(name)
+    W = _small_matrix(64, 8 * fmt.group, seed=47)
+    r = O.solve(W, fmt, 5)
+    assert r["mse_trace"][-1] < r["mse_trace"][0]
+
+
+def test_toy_workload_trace():
+    wl = synth.WORKLOADS["toy256x512_int4_g32"]
+    W = synth.weight(wl, 0, 0).double().numpy()
+    assert (W == 0).all(axis=1).sum() == 1
+    r = O.solve(W, O.preset(wl.fmt, wl.group), wl.T)
+    zr = np.where((W == 0).all(axis=1))[0][0]
+    assert r["a"][zr] == 1.0
+    assert r["mse_trace"][-1] < 0.5 * r["mse_trace"][0]
+
+
+# --------------------------------------------------------------------------- #
+# Activation rescale + quantize
+# --------------------------------------------------------------------------- #
+
+@pytest.mark.parametrize("name", FORMATS)
+def test_activation_path(name):
+    fmt = O.preset(name)
+    rng = np.random.default_rng(5)
+    X = torch.from_numpy(rng.standard_normal((8, 4 * fmt.group))).to(torch.bfloat16).double().numpy()
+    c1, s1 = O.act_rescale_quant(X, np.ones(X.shape[1]), fmt)
+    c0, s0 = O.quantize(X, fmt, 1.0)
+    assert np.array_equal(c1, c0) and np.array_equal(s1, s0)
+    # b multiplies the channel: b = 2 on all channels is Q(2X)
+    c2, s2 = O.act_rescale_quant(X, np.full(X.shape[1], 2.0), fmt)
+    c3, s3 = O.quantize(2 * X, fmt, 1.0)
+    assert np.array_equal(c2, c3) and np.array_equal(s2, s3)
+
+
+def test_activation_identity():
+    # eq. (1): X W^T ~ (X D_b) Qhat^T D_a with What = D_a Qhat D_b
+    fmt = O.preset("int4_bf16", 16)
+    W = _small_matrix(5, 32, seed=8)
+    r = O.solve(W, fmt, 2)
+    What = r["a"][:, None] * r["qhat"] * r["b"][None, :]
+    X = np.random.default_rng(1).standard_normal((3, 32))
+    lhs = (X * r["b"][None, :]) @ r["qhat"].T * r["a"][None, :]
+    assert np.allclose(lhs, X @ What.T, rtol=1e-12, atol=1e-14)
+
+
+# --------------------------------------------------------------------------- #
+# The seeded generator
+# --------------------------------------------------------------------------- #
+
+def test_generator_matches_integer_splitmix64():
+    M = (1 << 64) - 1
+
+    def sm(z):
+        z = (z + synth.GOLDEN) & M
+        z = ((z ^ (z >> 30)) * synth.MIX1) & M
+        z = ((z ^ (z >> 27)) * synth.MIX2) & M
+        return z ^ (z >> 31)
+
+    key = synth.stream_key(3, 1, 4)
+    bits = synth.raw_bits(key, 50, offset=1000)
+    for i in range(50):
+        want = sm((key + (1000 + i) * synth.GOLDEN) & M)
+        assert (int(bits[i]) & M) == want
+    u = synth.uniform(key, 50, offset=1000)
+    assert float(u[0]) == ((sm((key + 1000 * synth.GOLDEN) & M) >> 11) + 0.5) * 2.0 ** -53
