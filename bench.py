@@ -1,0 +1,413 @@
+#!/usr/bin/env python
+"""Benchmark of the dual-scale solver hot path on B200.
+
+One step = one full DualQuant solve of every linear layer of the workload
+(T block-coordinate-descent iterations plus the final pack pass, all in one
+batched launch sequence) followed by the activation rescale + quantize of the
+workload's activation batch with the solved b of the first linear (q_proj).
+
+Metric: solver weight-elements per second per BCD iteration, i.e.
+(sum of rows*cols) * T / step time; the step time also includes the final
+pack pass and the activation kernel, so the figure is conservative.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME]
+    python bench.py --impl reference ...      # the fp64 CPU oracle arm
+
+With N > 1 (torchrun, one rank per GPU) every rank solves a different decoder
+of the same model (weak scaling); no collective touches the data path, only
+the max-over-ranks of the timings.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import glob
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+DEFAULT_CONFIG = "llama31_70b_decoder_mxfp4_g32"
+METRIC = "solver weight-elements/s per BCD iteration"
+UNIT = "weight-elements/s"
+
+
+def _args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=10)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--config", default=DEFAULT_CONFIG)
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-rows", type=int, default=256,
+                   help="rows of q_proj in the oracle's bounded sample")
+    p.add_argument("--only", type=int, default=-1,
+                   help="profiling case: keep only this linear of the decoder")
+    p.add_argument("--T", type=int, default=-1, help="profiling case: iterations override")
+    p.add_argument("--no-act", action="store_true", help="profiling case: skip activations")
+    return p.parse_args()
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return json.load(f), "measured"
+    except OSError:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}, "fallback"
+
+
+def _src_hash():
+    h = hashlib.sha256()
+    for p in sorted(glob.glob(os.path.join(ROOT, "dual_scale_solver_b200", "csrc", "*"))):
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def _traffic(kind_name):
+    """ncu DRAM bytes per launch for the kernel, if a committed capture of the
+    current source exists (profiles/traffic.json); else None."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            t = json.load(f)
+    except OSError:
+        return None
+    e = t.get(kind_name)
+    if not e or e.get("src_hash") != _src_hash():
+        return None
+    return e.get("bytes_per_launch_full")
+
+
+class Clocks:
+    """nvidia-smi sampling of SM clock and throttle reasons during timing."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------- #
+# CPU oracle (baseline leg and reference arm)
+# --------------------------------------------------------------------------- #
+
+def _oracle_sample(wl, rows):
+    import numpy as np
+    import synth
+    import oracle as O
+    W = synth.weight(wl, 0, 0, rows=rows).double().numpy()
+    fmt = O.preset(wl.fmt, wl.group)
+    return W, fmt, np, O
+
+
+def _oracle_iteration(W, fmt, np, O, a, b, ts):
+    """One BCD iteration of the oracle from (a, b): row update, re-quantize,
+    column update, re-quantize."""
+    Qh, _, _ = O.qhat(W, a, b, fmt, ts)
+    a, _ = O.row_update(W, Qh, b, fmt)
+    Qh, _, _ = O.qhat(W, a, b, fmt, ts)
+    b, _ = O.col_update(W, Qh, a, fmt)
+    return a, b
+
+
+def cpu_baseline(wl, rows, min_seconds=10.0):
+    W, fmt, np, O = _oracle_sample(wl, rows)
+    ts = O.tensor_scale(W, fmt)
+    a, b = np.ones(W.shape[0]), np.ones(W.shape[1])
+    its, t0 = 0, time.perf_counter()
+    while True:
+        a, b = _oracle_iteration(W, fmt, np, O, a, b, ts)
+        its += 1
+        el = time.perf_counter() - t0
+        if el >= min_seconds or its >= 50:
+            break
+    value = W.size * its / el
+    sample = (f"{its} BCD iterations (row update, re-quantize, column update, re-quantize) of "
+              f"the fp64 numpy oracle on the first {rows} rows of decoder-0 "
+              f"{wl.linears[0].name} ({W.shape[0]}x{W.shape[1]}, {wl.fmt} G{wl.group}); "
+              f"{el:.1f} s")
+    return {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample}
+
+
+def run_reference(args, wl, rank, world):
+    if rank != 0:
+        return 0
+    W, fmt, np, O = _oracle_sample(wl, args.cpu_rows)
+    ts = O.tensor_scale(W, fmt)
+    a, b = np.ones(W.shape[0]), np.ones(W.shape[1])
+    for _ in range(args.warmup):
+        a, b = _oracle_iteration(W, fmt, np, O, a, b, ts)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        a, b = _oracle_iteration(W, fmt, np, O, a, b, ts)
+    el = time.perf_counter() - t0
+    value = W.size * args.steps / el
+    sample = (f"each step one BCD iteration of the fp64 numpy oracle on the first "
+              f"{args.cpu_rows} rows of decoder-0 {wl.linears[0].name} "
+              f"({W.shape[0]}x{W.shape[1]}, {wl.fmt} G{wl.group})")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": el / args.steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "sample_rows": args.cpu_rows},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------------------- #
+# GPU arm
+# --------------------------------------------------------------------------- #
+
+def run_ours(args, wl, rank, world, local_rank):
+    import torch
+    import synth
+    import dual_scale_solver_b200 as dq
+    from dual_scale_solver_b200 import build
+
+    dist = world > 1
+    if dist:
+        import torch.distributed as tdist
+        from datetime import timedelta
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    build.build()
+
+    # weak scaling: rank r solves decoder r of the model (seeded per decoder)
+    decoder = rank
+    idx = [args.only] if args.only >= 0 else range(len(wl.linears))
+    Ws = [synth.weight(wl, decoder, i, device=dev) for i in idx]
+    fmt = dq.format_preset(wl.fmt, wl.group)
+    act = None if args.no_act else wl.act
+    X = synth.activation(wl, device=dev) if act else None
+    fmt_act = dq.format_preset(act["fmt"], act["group"]) if act else None
+    T = wl.T if args.T < 0 else args.T
+    E = sum(W.numel() for W in Ws)
+    ws = dq.workspace([tuple(W.shape) for W in Ws], fmt, dev)
+    outs = None
+    act_out = None
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        nonlocal outs, act_out
+        outs = dq.solve_dual_scale_batched(Ws, fmt, T, ws=ws, outs=outs)
+        if X is not None:
+            if act_out is None:
+                act_out = dq.act_rescale_quant(X, outs[0]["b"], fmt_act)
+            else:
+                dq.act_rescale_quant(X, outs[0]["b"], fmt_act, codes=act_out[0], gscales=act_out[1])
+
+    def barrier():
+        if dist:
+            tdist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if dq.last_device_status() != 0:
+        raise RuntimeError("device status flags raised during warm-up")
+
+    clocks = Clocks(local_rank)
+    barrier()
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    time.sleep(0.3)
+    dq.kernel_timing(True)
+    for k in range(4):
+        dq.kernel_time(k)                     # clear
+    n0 = dq.launch_count()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    ms = e0.elapsed_time(e1)
+    launches = dq.launch_count() - n0
+    kt = {k: dq.kernel_time(k) for k in range(4)}
+    dq.kernel_timing(False)
+    clk = clocks.stop()
+    if dist:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+        ms = float(t.item())
+
+    ms_step = ms / args.steps
+    value = world * E * T / (ms_step / 1e3)
+
+    # dominant tile kernel and its roofline (HBM: it streams W once per launch)
+    names = {0: "row_stats", 1: "col_stats", 2: "pack", 3: "act_quant"}
+    dom = max((0, 1), key=lambda k: kt[k][0])
+    tot_ms, nl = kt[dom]
+    avg_s = tot_ms / max(nl, 1) / 1e3
+    rows_sum = sum(W.shape[0] for W in Ws)
+    cols_sum = sum(W.shape[1] for W in Ws)
+    alg_bytes = E * Ws[0].element_size() + 4 * (rows_sum + cols_sum)
+    peaks, which = _peaks()
+    peak = float(peaks["hbm_gbs"])
+    achieved = alg_bytes / avg_s / 1e9
+    roofline = {"bound": "hbm", "kernel": names[dom], "achieved": achieved, "peak": peak,
+                "unit": "GB/s", "frac": achieved / peak, "peak_source": which,
+                "traffic": _traffic(names[dom]), "algorithmic_bytes_per_launch": alg_bytes,
+                "avg_launch_ms": avg_s * 1e3,
+                "kernel_ms_per_step": {names[k]: kt[k][0] / args.steps for k in kt}}
+
+    # end-to-end: host buffers in, results out, every step
+    e2e = None
+    if not args.no_e2e:
+        hW = [W.to("cpu").pin_memory() for W in Ws]
+        hX = X.to("cpu").pin_memory() if X is not None else None
+        dW = [torch.empty_like(W) for W in Ws]
+        dX = torch.empty_like(X) if X is not None else None
+        h2d = sum(w.numel() * w.element_size() for w in hW) + (
+            hX.numel() * hX.element_size() if hX is not None else 0)
+        res_h = None
+
+        def e2e_step():
+            nonlocal res_h, outs, act_out
+            for h, d in zip(hW, dW):
+                d.copy_(h, non_blocking=True)
+            if dX is not None:
+                dX.copy_(hX, non_blocking=True)
+            outs = dq.solve_dual_scale_batched(dW, fmt, T, ws=ws, outs=outs)
+            if dX is not None:
+                dq.act_rescale_quant(dX, outs[0]["b"], fmt_act, codes=act_out[0], gscales=act_out[1])
+            dev_res = []
+            for o in outs:
+                dev_res += [o["codes"], o["gscales"], o["a"], o["b"], o["tensor_scale"], o["mse_trace"]]
+            if act_out is not None:
+                dev_res += [act_out[0], act_out[1]]
+            if res_h is None:
+                res_h = [torch.empty(r.shape, dtype=r.dtype, pin_memory=True) for r in dev_res]
+            for h, d in zip(res_h, dev_res):
+                h.copy_(d, non_blocking=True)
+            return sum(r.numel() * r.element_size() for r in dev_res)
+
+        d2h = e2e_step()
+        torch.cuda.synchronize(dev)
+        barrier()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        f1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        ems = f0.elapsed_time(f1)
+        if dist:
+            t = torch.tensor([ems], dtype=torch.float64, device=dev)
+            tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+            ems = float(t.item())
+        e2e = {"value": world * E * T / (ems / args.steps / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": ems / args.steps}
+
+    if dq.last_device_status() != 0:
+        raise RuntimeError("device status flags raised during timing")
+
+    if args.only >= 0 or args.T >= 0 or args.no_act:
+        wl_name = f"{wl.name} (profiling subset: only={args.only} T={T} act={act is not None})"
+    else:
+        wl_name = wl.name
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": wl_name, "matrices": len(Ws), "elements_per_gpu": E, "T": T,
+                   "format": f"{wl.fmt} G{wl.group}",
+                   "activation": (f"{act['tokens']}x{act['K']} bf16 -> {act['fmt']} G{act['group']}"
+                                  if act else None),
+                   "l2": "inputs larger than L2 (no flush needed)",
+                   "parallelism": f"{world} independent decoders" if world > 1 else "1 GPU"},
+        "roofline": roofline,
+        "gpu_launches": launches,
+        "clocks": clk,
+        "e2e": e2e,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl, args.cpu_rows)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = _args()
+    import synth
+    wl = synth.WORKLOADS[args.config]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, wl, rank, world)
+    if world > 1:
+        import torch
+        import torch.distributed as tdist
+        from datetime import timedelta
+        torch.cuda.set_device(local_rank)
+        tdist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                 device_id=torch.device("cuda", local_rank))
+    try:
+        return run_ours(args, wl, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as tdist
+            tdist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,326 @@
+"""dual_scale_solver_b200 — Python binding of the ``dq`` C ABI (``include/dq.h``).
+
+Argument marshalling only: every step of the solver runs in the CUDA kernels
+of ``libdq.so``.  Torch tensors supply device memory and the current CUDA
+stream; outputs that the caller does not pass are allocated with torch.
+There is no CPU fallback: without the built library every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from ctypes import c_char_p, c_double, c_float, c_int32, c_int64, c_size_t, c_void_p, POINTER
+
+import torch
+
+__all__ = [
+    "DqError", "dq_format", "dq_matrix", "lib", "library_path", "version", "format_preset",
+    "workspace_size", "quantize", "dequantize", "solve_dual_scale", "solve_dual_scale_batched",
+    "row_update", "col_update", "act_rescale_quant", "last_device_status", "EXPORTS",
+    "kernel_timing", "kernel_time", "launch_count",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libdq.so")
+
+DQ_CODES_INT4, DQ_CODES_E2M1 = 0, 1
+DQ_SCALE_BF16, DQ_SCALE_E8M0, DQ_SCALE_E4M3 = 0, 1, 2
+DQ_DT_F32, DQ_DT_BF16 = 0, 1
+DQ_OK, DQ_ERR_NONFINITE, DQ_ERR_RANGE = 0, -4, -5
+
+EXPORTS = ("dq_version", "dq_strerror", "dq_format_preset", "dq_workspace_size", "dq_quantize",
+           "dq_dequantize", "dq_solve_dual_scale", "dq_solve_dual_scale_batched",
+           "dq_row_update", "dq_col_update", "dq_act_rescale_quant", "dq_last_device_status",
+           "dq_kernel_timing", "dq_kernel_time", "dq_launch_count")
+
+
+class DqError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {_strerror(status)} (status {status})")
+
+
+class dq_format(ctypes.Structure):
+    _fields_ = [("codes", c_int32), ("group", c_int32), ("group_scale", c_int32),
+                ("outer_scale", c_int32), ("tensor_scale_auto", c_int32)]
+
+    def __repr__(self):
+        return (f"dq_format(codes={self.codes}, group={self.group}, group_scale={self.group_scale}, "
+                f"outer_scale={self.outer_scale}, tensor_scale_auto={self.tensor_scale_auto})")
+
+
+class dq_matrix(ctypes.Structure):
+    _fields_ = [("W", c_void_p), ("rows", c_int64), ("cols", c_int64), ("a0", c_void_p),
+                ("b0", c_void_p), ("codes", c_void_p), ("gscales", c_void_p), ("a", c_void_p),
+                ("b", c_void_p), ("tensor_scale", c_void_p), ("mse_trace", c_void_p),
+                ("mse_half", c_void_p)]
+
+
+_lib = None
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded ``libdq.so``; raises if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(_LIB_PATH):
+        raise ImportError(f"libdq.so not built at {_LIB_PATH}; run "
+                          "`python -m dual_scale_solver_b200.build` (no CPU fallback exists)")
+    L = ctypes.CDLL(_LIB_PATH)
+    P = POINTER
+    sig = {
+        "dq_version": (c_char_p, []),
+        "dq_strerror": (c_char_p, [c_int32]),
+        "dq_format_preset": (c_int32, [c_char_p, c_int32, P(dq_format)]),
+        "dq_workspace_size": (c_int32, [c_int32, P(c_int64), P(c_int64), P(dq_format), P(c_size_t)]),
+        "dq_quantize": (c_int32, [c_void_p, c_int32, c_int64, c_int64, P(dq_format), c_void_p,
+                                  c_void_p, c_float, c_void_p, c_void_p, c_void_p]),
+        "dq_dequantize": (c_int32, [c_void_p, c_void_p, c_int64, c_int64, P(dq_format), c_float,
+                                    c_void_p, c_void_p, c_void_p, c_void_p]),
+        "dq_solve_dual_scale": (c_int32, [c_void_p, c_int32, c_int64, c_int64, P(dq_format),
+                                          c_int32, c_void_p, c_void_p, c_void_p, c_void_p,
+                                          c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                          c_void_p, c_size_t, c_void_p]),
+        "dq_solve_dual_scale_batched": (c_int32, [c_int32, P(dq_matrix), c_int32, P(dq_format),
+                                                  c_int32, c_void_p, c_size_t, c_void_p]),
+        "dq_row_update": (c_int32, [c_void_p, c_int32, c_int64, c_int64, P(dq_format), c_float,
+                                    c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                    c_size_t, c_void_p]),
+        "dq_col_update": (c_int32, [c_void_p, c_int32, c_int64, c_int64, P(dq_format), c_float,
+                                    c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                    c_size_t, c_void_p]),
+        "dq_act_rescale_quant": (c_int32, [c_void_p, c_int64, c_int64, c_void_p, P(dq_format),
+                                           c_void_p, c_void_p, c_void_p]),
+        "dq_last_device_status": (c_int32, [c_void_p]),
+        "dq_kernel_timing": (c_int32, [c_int32]),
+        "dq_kernel_time": (c_int32, [c_int32, P(c_double), P(c_int64)]),
+        "dq_launch_count": (c_int64, []),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(L, name)
+        f.restype = res
+        f.argtypes = args
+    _lib = L
+    return L
+
+
+def _strerror(s: int) -> str:
+    return lib().dq_strerror(s).decode()
+
+
+def _check(s: int, where: str):
+    if s != DQ_OK:
+        raise DqError(s, where)
+
+
+def version() -> str:
+    return lib().dq_version().decode()
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return DQ_DT_BF16
+    if t.dtype == torch.float32:
+        return DQ_DT_F32
+    raise TypeError(f"unsupported input dtype {t.dtype} (bfloat16 or float32)")
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("tensors must be CUDA tensors")
+
+
+def format_preset(name: str, group: int = 0) -> dq_format:
+    f = dq_format()
+    _check(lib().dq_format_preset(name.encode(), group, ctypes.byref(f)), "dq_format_preset")
+    return f
+
+
+def gscale_dtype(fmt: dq_format) -> torch.dtype:
+    return torch.int16 if fmt.group_scale == DQ_SCALE_BF16 else torch.uint8
+
+
+def workspace_size(shapes, fmt: dq_format) -> int:
+    n = len(shapes)
+    rows = (c_int64 * max(n, 1))(*[int(r) for r, _ in shapes])
+    cols = (c_int64 * max(n, 1))(*[int(c) for _, c in shapes])
+    out = c_size_t(0)
+    _check(lib().dq_workspace_size(n, rows, cols, ctypes.byref(fmt), ctypes.byref(out)),
+           "dq_workspace_size")
+    return out.value
+
+
+def workspace(shapes, fmt: dq_format, device=None) -> torch.Tensor:
+    return torch.empty(workspace_size(shapes, fmt), dtype=torch.uint8,
+                       device=device or torch.device("cuda"))
+
+
+def _outputs(rows, cols, fmt, device, codes=None, gscales=None):
+    if codes is None:
+        codes = torch.empty(rows, cols // 2, dtype=torch.uint8, device=device)
+    if gscales is None:
+        gscales = torch.empty(rows, cols // fmt.group, dtype=gscale_dtype(fmt), device=device)
+    return codes, gscales
+
+
+def quantize(X, fmt, a=None, b=None, tensor_scale: float = 1.0, codes=None, gscales=None,
+             stream=None):
+    """Q(X / (a b^T)) -> (codes [rows, cols/2] uint8, group scales [rows, cols/G])."""
+    _need_cuda(X, a, b)
+    rows, cols = X.shape
+    codes, gscales = _outputs(rows, cols, fmt, X.device, codes, gscales)
+    _check(lib().dq_quantize(_ptr(X), _dtype_code(X), rows, cols, ctypes.byref(fmt), _ptr(a),
+                             _ptr(b), float(tensor_scale), _ptr(codes), _ptr(gscales),
+                             _stream(stream)), "dq_quantize")
+    return codes, gscales
+
+
+def dequantize(codes, gscales, rows, cols, fmt, tensor_scale=1.0, a=None, b=None, out=None,
+               stream=None):
+    """a_i * c_ij * s_g * ts * b_j as float32 [rows, cols]."""
+    if out is None:
+        out = torch.empty(rows, cols, dtype=torch.float32, device=codes.device)
+    _check(lib().dq_dequantize(_ptr(codes), _ptr(gscales), rows, cols, ctypes.byref(fmt),
+                               float(tensor_scale), _ptr(a), _ptr(b), _ptr(out),
+                               _stream(stream)), "dq_dequantize")
+    return out
+
+
+def solve_dual_scale(W, fmt, T, a0=None, b0=None, ws=None, half=True, stream=None):
+    """Full DualQuant solve of one matrix.  Returns a dict of device tensors:
+    codes, gscales, a, b, tensor_scale, mse_trace (T+1), mse_half (T)."""
+    _need_cuda(W, a0, b0)
+    rows, cols = W.shape
+    dev = W.device
+    codes, gscales = _outputs(rows, cols, fmt, dev)
+    a = torch.empty(rows, dtype=torch.float32, device=dev)
+    b = torch.empty(cols, dtype=torch.float32, device=dev)
+    ts = torch.empty(1, dtype=torch.float32, device=dev)
+    trace = torch.empty(T + 1, dtype=torch.float64, device=dev)
+    mhalf = torch.empty(max(T, 1), dtype=torch.float64, device=dev) if half else None
+    if ws is None:
+        ws = workspace([(rows, cols)], fmt, dev)
+    _check(lib().dq_solve_dual_scale(_ptr(W), _dtype_code(W), rows, cols, ctypes.byref(fmt), T,
+                                     _ptr(a0), _ptr(b0), _ptr(codes), _ptr(gscales), _ptr(a),
+                                     _ptr(b), _ptr(ts), _ptr(trace), _ptr(mhalf), _ptr(ws),
+                                     ws.numel(), _stream(stream)), "dq_solve_dual_scale")
+    return dict(codes=codes, gscales=gscales, a=a, b=b, tensor_scale=ts, mse_trace=trace,
+                mse_half=mhalf[:T] if half else None)
+
+
+def solve_dual_scale_batched(Ws, fmt, T, ws=None, outs=None, half=False, stream=None):
+    """Solve a list of independent matrices (same dtype) in one launch sequence.
+    ``outs`` (optional) is a list of dicts as returned by this function, reused."""
+    n = len(Ws)
+    if n == 0:
+        return []
+    dt = _dtype_code(Ws[0])
+    dev = Ws[0].device
+    if outs is None:
+        outs = []
+        for W in Ws:
+            rows, cols = W.shape
+            codes, gscales = _outputs(rows, cols, fmt, dev)
+            outs.append(dict(
+                codes=codes, gscales=gscales,
+                a=torch.empty(rows, dtype=torch.float32, device=dev),
+                b=torch.empty(cols, dtype=torch.float32, device=dev),
+                tensor_scale=torch.empty(1, dtype=torch.float32, device=dev),
+                mse_trace=torch.empty(T + 1, dtype=torch.float64, device=dev),
+                mse_half=torch.empty(max(T, 1), dtype=torch.float64, device=dev) if half else None))
+    if ws is None:
+        ws = workspace([tuple(W.shape) for W in Ws], fmt, dev)
+    mats = (dq_matrix * n)()
+    for i, (W, o) in enumerate(zip(Ws, outs)):
+        if _dtype_code(W) != dt:
+            raise TypeError("all matrices of a batch share one dtype")
+        m = mats[i]
+        m.W, m.rows, m.cols = _ptr(W), W.shape[0], W.shape[1]
+        m.a0 = m.b0 = None
+        m.codes, m.gscales = _ptr(o["codes"]), _ptr(o["gscales"])
+        m.a, m.b, m.tensor_scale = _ptr(o["a"]), _ptr(o["b"]), _ptr(o["tensor_scale"])
+        m.mse_trace, m.mse_half = _ptr(o["mse_trace"]), _ptr(o.get("mse_half"))
+    _check(lib().dq_solve_dual_scale_batched(n, mats, dt, ctypes.byref(fmt), T, _ptr(ws),
+                                             ws.numel(), _stream(stream)),
+           "dq_solve_dual_scale_batched")
+    return outs
+
+
+def _step(fn, name, W, fmt, tensor_scale, a_in, b_in, out_len, ws, stream):
+    _need_cuda(W, a_in, b_in)
+    rows, cols = W.shape
+    dev = W.device
+    out = torch.empty(out_len, dtype=torch.float32, device=dev)
+    pre = torch.empty(out_len, dtype=torch.float32, device=dev)
+    mse = torch.empty(1, dtype=torch.float64, device=dev)
+    if ws is None:
+        ws = workspace([(rows, cols)], fmt, dev)
+    _check(fn(_ptr(W), _dtype_code(W), rows, cols, ctypes.byref(fmt), float(tensor_scale),
+              _ptr(a_in), _ptr(b_in), _ptr(out), _ptr(pre), _ptr(mse), _ptr(ws), ws.numel(),
+              _stream(stream)), name)
+    return out, pre, mse
+
+
+def row_update(W, fmt, a_in, b_in, tensor_scale=1.0, ws=None, stream=None):
+    """One row half-step: returns (a_out, a_pre, mse_of_input_state)."""
+    return _step(lib().dq_row_update, "dq_row_update", W, fmt, tensor_scale, a_in, b_in,
+                 W.shape[0], ws, stream)
+
+
+def col_update(W, fmt, a_in, b_in, tensor_scale=1.0, ws=None, stream=None):
+    """One column half-step: returns (b_out, b_pre, mse_of_input_state)."""
+    return _step(lib().dq_col_update, "dq_col_update", W, fmt, tensor_scale, a_in, b_in,
+                 W.shape[1], ws, stream)
+
+
+def act_rescale_quant(X, b, fmt, codes=None, gscales=None, stream=None):
+    """Q(X D_b): returns (codes [tokens, K/2], group scales [tokens, K/G])."""
+    _need_cuda(X, b)
+    if X.dtype != torch.bfloat16:
+        raise TypeError("activations are bfloat16")
+    tokens, K = X.shape
+    codes, gscales = _outputs(tokens, K, fmt, X.device, codes, gscales)
+    _check(lib().dq_act_rescale_quant(_ptr(X), tokens, K, _ptr(b), ctypes.byref(fmt), _ptr(codes),
+                                      _ptr(gscales), _stream(stream)), "dq_act_rescale_quant")
+    return codes, gscales
+
+
+KIND_ROW, KIND_COL, KIND_PACK, KIND_ACT = 0, 1, 2, 3
+
+
+def kernel_timing(enable: bool):
+    """Bracket every tile-kernel launch with CUDA events on its stream."""
+    _check(lib().dq_kernel_timing(1 if enable else 0), "dq_kernel_timing")
+
+
+def kernel_time(kind: int):
+    """(summed ms, launches) of one tile-kernel kind since the last read."""
+    ms, n = c_double(0), c_int64(0)
+    _check(lib().dq_kernel_time(kind, ctypes.byref(ms), ctypes.byref(n)), "dq_kernel_time")
+    return ms.value, n.value
+
+
+def launch_count() -> int:
+    """Kernels this library has launched in the process so far."""
+    return lib().dq_launch_count()
+
+
+def last_device_status(stream=None) -> int:
+    """Synchronise and return (and clear) the device flags as a dq status code."""
+    return lib().dq_last_device_status(_stream(stream))

@@ -1,0 +1,707 @@
+// dq_api.cu — the C ABI declared in include/dq.h: argument checks, tile
+// geometry, workspace layout, and the launch sequences of the solver.
+//
+// Launch sequence of a solve (DualQuant, daiwk.github.io reproduction note,
+// "核心公式" eq. (2) and the order stated under it; trove summary, flowchart
+// of "How it works"):
+//   [amax + tensor scale]  init a, b
+//   for t in 1..T:
+//     ROW tiles   -> per-row partial sums of <W,R>, <R,R>; residual of state t-1
+//     row finalize: a <- Pi(sum/sum), zero slice -> 1
+//     COL tiles   -> per-column partial sums of <W,S>, <S,S> with the new a
+//     col finalize: b <- Pi(sum/sum), zero slice -> 1
+//     mse finalize: mse_trace[t-1], mse_half[t-1]
+//   PACK tiles -> codes, group scales, residual; mse finalize -> mse_trace[T]
+// The re-quantization after each update is not a separate pass: every tile
+// pass quantizes W with the current (a, b) on the fly.
+#include <cuda_runtime.h>
+
+#include <cstdio>
+#include <cstring>
+#include <atomic>
+#include <mutex>
+#include <vector>
+
+#include "../../include/dq.h"
+#define DQ_DEFINE_HOST_KERNELS
+#include "dq_launch.h"
+
+using namespace dq;
+
+namespace {
+
+__device__ unsigned int g_dq_status_word;
+
+constexpr int kMaxDevices = 64;
+unsigned int *g_status_ptr[kMaxDevices];
+std::once_flag g_status_once[kMaxDevices];
+
+// Device address of the status word on the current device (looked up once
+// per device with that device current).
+unsigned int *status_ptr() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::call_once(g_status_once[dev], [dev]() {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_dq_status_word) == cudaSuccess)
+            g_status_ptr[dev] = static_cast<unsigned int *>(p);
+    });
+    return g_status_ptr[dev];
+}
+
+// ---- measurement support: launch counter and optional per-kind event timing
+std::atomic<int64_t> g_launches{0};
+std::mutex g_timing_mu;
+bool g_timing = false;
+struct TimedLaunch { cudaEvent_t beg, end; int kind; };
+std::vector<TimedLaunch> g_timed;       // recorded, not yet read
+std::vector<cudaEvent_t> g_event_pool;  // free events
+
+cudaEvent_t take_event() {
+    if (!g_event_pool.empty()) {
+        cudaEvent_t e = g_event_pool.back();
+        g_event_pool.pop_back();
+        return e;
+    }
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    return e;
+}
+
+void count_launches(int k) { g_launches.fetch_add(k, std::memory_order_relaxed); }
+
+struct FmtInfo {
+    int combo;
+    int G;
+    float qmax;
+};
+
+dq_status check_format(const dq_format *f, FmtInfo *out) {
+    if (!f) return DQ_ERR_ARG;
+    if (f->group != 16 && f->group != 32 && f->group != 64) return DQ_ERR_FORMAT;
+    if (f->tensor_scale_auto != 0 && f->tensor_scale_auto != 1) return DQ_ERR_FORMAT;
+    if (f->tensor_scale_auto && f->group_scale != DQ_SCALE_E4M3) return DQ_ERR_FORMAT;
+    int combo = -1;
+    const int c = f->codes, g = f->group_scale, o = f->outer_scale;
+    if (c == DQ_CODES_INT4 && g == DQ_SCALE_BF16 && o == DQ_SCALE_BF16) combo = COMBO_INT4_BF16_BF16;
+    if (c == DQ_CODES_INT4 && g == DQ_SCALE_E8M0 && o == DQ_SCALE_E8M0) combo = COMBO_INT4_E8M0_E8M0;
+    if (c == DQ_CODES_E2M1 && g == DQ_SCALE_E8M0 && o == DQ_SCALE_E8M0) combo = COMBO_E2M1_E8M0_E8M0;
+    if (c == DQ_CODES_E2M1 && g == DQ_SCALE_E4M3 && o == DQ_SCALE_BF16) combo = COMBO_E2M1_E4M3_BF16;
+    if (c == DQ_CODES_INT4 && g == DQ_SCALE_E8M0 && o == DQ_SCALE_BF16) combo = COMBO_INT4_E8M0_BF16;
+    if (c == DQ_CODES_E2M1 && g == DQ_SCALE_E8M0 && o == DQ_SCALE_BF16) combo = COMBO_E2M1_E8M0_BF16;
+    if (combo < 0) return DQ_ERR_FORMAT;
+    if (out) {
+        out->combo = combo;
+        out->G = f->group;
+        out->qmax = (c == DQ_CODES_INT4) ? 7.0f : 6.0f;
+    }
+    return DQ_OK;
+}
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Tile geometry of one matrix (see the tile kernel's description).
+struct Geom {
+    int wc, ncb;
+    int tr[3];
+    int64_t ntiles[3];
+    int64_t nrb_col;
+};
+
+Geom geometry(int64_t rows, int64_t cols, bool f32) {
+    Geom g{};
+    const int epc = f32 ? 4 : 8, seg = 32 * epc;
+    const int64_t nseg = (cols + seg - 1) / seg;
+    int wc = 1;
+    while (wc < 8 && wc < nseg) wc <<= 1;
+    g.wc = wc;
+    g.ncb = (int)((nseg + wc - 1) / wc);
+    const int wr = kWarps / wc;
+    const int rpw[3] = {16, 64, 16};
+    for (int m = 0; m < 3; ++m) {
+        g.tr[m] = rpw[m] * wr;
+        const int64_t nrb = (rows + g.tr[m] - 1) / g.tr[m];
+        g.ntiles[m] = (rows > 0 && cols > 0) ? nrb * g.ncb : 0;
+    }
+    g.nrb_col = (rows + g.tr[1] - 1) / g.tr[1];
+    return g;
+}
+
+// Workspace bytes of one matrix (each region 256-byte aligned).
+size_t matrix_ws(int64_t rows, int64_t cols, bool f32) {
+    const Geom g = geometry(rows, cols, f32);
+    size_t b = 0;
+    b += round_up((size_t)rows * g.ncb * sizeof(float2), 256);               // rowpart
+    b += round_up((size_t)g.nrb_col * cols * sizeof(float2), 256);           // colpart
+    b += round_up((size_t)std::max(g.ntiles[0], g.ntiles[2]) * 8, 256);      // res_row
+    b += round_up((size_t)g.ntiles[1] * 8, 256);                             // res_col
+    b += 256;                                                                // amax
+    return b;
+}
+
+size_t table_ws(int n) { return n > 1 ? round_up((size_t)n * sizeof(MatDesc), 256) : 0; }
+
+struct Carve {
+    char *p;
+    char *end;
+    template <class T> T *take(size_t bytes) {
+        T *r = reinterpret_cast<T *>(p);
+        p += round_up(bytes, 256);
+        return r;
+    }
+};
+
+// Fill geometry and workspace pointers of one descriptor.
+void place(MatDesc &d, bool f32, Carve &cv, int64_t tile_base[3], int64_t &row_base,
+           int64_t &col_base) {
+    const Geom g = geometry(d.rows, d.cols, f32);
+    d.wc = g.wc;
+    d.ncb = g.ncb;
+    for (int m = 0; m < 3; ++m) {
+        d.tr[m] = g.tr[m];
+        d.ntiles[m] = g.ntiles[m];
+        d.tile0[m] = tile_base[m];
+        tile_base[m] += g.ntiles[m];
+    }
+    d.row0 = row_base;
+    d.col0 = col_base;
+    row_base += d.rows;
+    col_base += d.cols;
+    if (cv.p) {
+        d.rowpart = cv.take<float2>((size_t)d.rows * g.ncb * sizeof(float2));
+        d.colpart = cv.take<float2>((size_t)g.nrb_col * d.cols * sizeof(float2));
+        d.res_row = cv.take<double>((size_t)std::max(g.ntiles[0], g.ntiles[2]) * 8);
+        d.res_col = cv.take<double>((size_t)g.ntiles[1] * 8);
+        d.amax = cv.take<unsigned int>(256);
+    }
+}
+
+cudaError_t launch_tiles(int combo, const TileLaunch &L) {
+    switch (combo) {
+        case 0: return launch_tile_c0(L);
+        case 1: return launch_tile_c1(L);
+        case 2: return launch_tile_c2(L);
+        case 3: return launch_tile_c3(L);
+        case 4: return launch_tile_c4(L);
+        case 5: return launch_tile_c5(L);
+    }
+    return cudaErrorInvalidValue;
+}
+
+int outer_of(int combo) {
+    return (combo == COMBO_INT4_E8M0_E8M0 || combo == COMBO_E2M1_E8M0_E8M0) ? SC_E8M0 : SC_BF16;
+}
+
+unsigned grid_for(int64_t n, int block) {
+    int64_t g = (n + block - 1) / block;
+    if (g > 148 * 32) g = 148 * 32;
+    return (unsigned)(g < 1 ? 1 : g);
+}
+
+#define DQ_CUDA(x)                                      \
+    do {                                                \
+        cudaError_t e_ = (x);                           \
+        if (e_ != cudaSuccess) return DQ_ERR_CUDA;      \
+    } while (0)
+
+struct Launcher {
+    Table tab;
+    int combo, G;
+    bool f32;
+    float qmax;
+    int64_t tiles[3] = {0, 0, 0};
+    int64_t total_rows = 0, total_cols = 0;
+    cudaStream_t st;
+
+    dq_status tiles_pass(int mode) {
+        TileLaunch L;
+        L.tab = tab;
+        L.mode = mode;
+        L.slot = (mode == MODE_ACT) ? 2 : mode;
+        L.grid = tiles[L.slot];
+        L.f32 = f32 ? 1 : 0;
+        L.G = G;
+        L.stream = st;
+        if (L.grid <= 0) return DQ_OK;
+        cudaEvent_t beg = nullptr, end = nullptr;
+        {
+            std::lock_guard<std::mutex> lk(g_timing_mu);
+            if (g_timing) { beg = take_event(); end = take_event(); }
+        }
+        if (beg && end) DQ_CUDA(cudaEventRecord(beg, st));
+        DQ_CUDA(launch_tiles(combo, L));
+        count_launches(1);
+        if (beg && end) {
+            DQ_CUDA(cudaEventRecord(end, st));
+            std::lock_guard<std::mutex> lk(g_timing_mu);
+            g_timed.push_back({beg, end, mode});
+        }
+        return DQ_OK;
+    }
+    dq_status row_finalize() {
+        if (total_rows == 0) return DQ_OK;
+        if (outer_of(combo) == SC_E8M0)
+            row_finalize_kernel<SC_E8M0><<<grid_for(total_rows, 256), 256, 0, st>>>(tab, total_rows);
+        else
+            row_finalize_kernel<SC_BF16><<<grid_for(total_rows, 256), 256, 0, st>>>(tab, total_rows);
+        DQ_CUDA(cudaGetLastError());
+        count_launches(1);
+        return DQ_OK;
+    }
+    dq_status col_finalize() {
+        if (total_cols == 0) return DQ_OK;
+        if (outer_of(combo) == SC_E8M0)
+            col_finalize_kernel<SC_E8M0><<<grid_for(total_cols, 256), 256, 0, st>>>(tab, total_cols);
+        else
+            col_finalize_kernel<SC_BF16><<<grid_for(total_cols, 256), 256, 0, st>>>(tab, total_cols);
+        DQ_CUDA(cudaGetLastError());
+        count_launches(1);
+        return DQ_OK;
+    }
+    dq_status mse(int row_slot, int idx_trace, int idx_half, double *out_row, double *out_col) {
+        mse_finalize_kernel<<<2 * tab.n, 256, 0, st>>>(tab, row_slot, idx_trace, idx_half, out_row,
+                                                      out_col);
+        DQ_CUDA(cudaGetLastError());
+        count_launches(1);
+        return DQ_OK;
+    }
+};
+
+thread_local std::vector<MatDesc> t_table;
+
+dq_status solve_impl(int32_t n, const dq_matrix *mats, int32_t dtype, const dq_format *fmt,
+                     int32_t T, void *workspace, size_t ws_bytes, cudaStream_t st) {
+    if (n < 0 || T < 0 || !mats) return DQ_ERR_ARG;
+    if (dtype != DQ_DT_F32 && dtype != DQ_DT_BF16) return DQ_ERR_ARG;
+    FmtInfo fi;
+    dq_status s = check_format(fmt, &fi);
+    if (s != DQ_OK) return s;
+    if (n == 0) return DQ_OK;
+    const bool f32 = dtype == DQ_DT_F32;
+    size_t need = table_ws(n);
+    for (int i = 0; i < n; ++i) {
+        const dq_matrix &m = mats[i];
+        if (m.rows < 0 || m.cols < 0) return DQ_ERR_SHAPE;
+        if (m.cols % fi.G) return DQ_ERR_SHAPE;
+        const bool empty = m.rows == 0 || m.cols == 0;
+        if (!empty && (!m.W || !m.codes || !m.gscales)) return DQ_ERR_ARG;
+        if (!m.a || !m.b || !m.tensor_scale) return DQ_ERR_ARG;
+        if (!aligned(m.W, 16) || !aligned(m.codes, 16) || !aligned(m.gscales, 16)) return DQ_ERR_ALIGN;
+        if (!aligned(m.a, 4) || !aligned(m.b, 4) || !aligned(m.tensor_scale, 4)) return DQ_ERR_ALIGN;
+        if (!aligned(m.a0, 4) || !aligned(m.b0, 4)) return DQ_ERR_ALIGN;
+        if (!aligned(m.mse_trace, 8) || !aligned(m.mse_half, 8)) return DQ_ERR_ALIGN;
+        need += matrix_ws(m.rows, m.cols, f32);
+    }
+    if (!workspace || ws_bytes < need) return DQ_ERR_WORKSPACE;
+    if (!aligned(workspace, 256)) return DQ_ERR_ALIGN;
+
+    unsigned int *status = status_ptr();
+    if (!status) return DQ_ERR_CUDA;
+
+    Carve cv{static_cast<char *>(workspace), static_cast<char *>(workspace) + ws_bytes};
+    MatDesc *dev_table = n > 1 ? cv.take<MatDesc>((size_t)n * sizeof(MatDesc)) : nullptr;
+    t_table.assign(n, MatDesc{});
+    int64_t tile_base[3] = {0, 0, 0}, row_base = 0, col_base = 0;
+    for (int i = 0; i < n; ++i) {
+        const dq_matrix &m = mats[i];
+        MatDesc &d = t_table[i];
+        d.W = m.W;
+        d.rows = m.rows;
+        d.cols = m.cols;
+        d.a = m.a;
+        d.b = m.b;
+        d.a_out = m.a;
+        d.b_out = m.b;
+        d.codes = m.codes;
+        d.gscales = m.gscales;
+        d.ts_ptr = m.tensor_scale;
+        d.ts_out = m.tensor_scale;
+        d.ts_val = 1.0f;
+        d.a0 = m.a0;
+        d.b0 = m.b0;
+        d.mse_trace = m.mse_trace;
+        d.mse_half = m.mse_half;
+        place(d, f32, cv, tile_base, row_base, col_base);
+    }
+    Launcher L;
+    L.tab.dev = dev_table;
+    L.tab.n = n;
+    L.tab.status = status;
+    if (n == 1) L.tab.one = t_table[0];
+    L.combo = fi.combo;
+    L.G = fi.G;
+    L.f32 = f32;
+    L.qmax = fi.qmax;
+    for (int m = 0; m < 3; ++m) L.tiles[m] = tile_base[m];
+    L.total_rows = row_base;
+    L.total_cols = col_base;
+    L.st = st;
+    if (dev_table)
+        DQ_CUDA(cudaMemcpyAsync(dev_table, t_table.data(), (size_t)n * sizeof(MatDesc),
+                                cudaMemcpyHostToDevice, st));
+
+    // tensor scale (NVFP4 weights: from amax of W; otherwise 1)
+    if (fmt->tensor_scale_auto) {
+        for (int i = 0; i < n; ++i)
+            DQ_CUDA(cudaMemsetAsync(t_table[i].amax, 0, sizeof(unsigned int), st));
+        if (L.tiles[2] > 0) {
+            if (f32) amax_kernel<float><<<(unsigned)L.tiles[2], kThreads, 0, st>>>(L.tab);
+            else amax_kernel<Bf16Tag><<<(unsigned)L.tiles[2], kThreads, 0, st>>>(L.tab);
+            DQ_CUDA(cudaGetLastError());
+            count_launches(1);
+        }
+    }
+    tensor_scale_kernel<<<(n + 127) / 128, 128, 0, st>>>(L.tab, fi.qmax, fmt->tensor_scale_auto);
+    DQ_CUDA(cudaGetLastError());
+    count_launches(1);
+    if (row_base + col_base > 0) {
+        init_state_kernel<<<grid_for(row_base + col_base, 256), 256, 0, st>>>(L.tab, row_base, col_base);
+        DQ_CUDA(cudaGetLastError());
+        count_launches(1);
+    }
+    for (int t = 0; t < T; ++t) {
+        if ((s = L.tiles_pass(MODE_ROW)) != DQ_OK) return s;
+        if ((s = L.row_finalize()) != DQ_OK) return s;
+        if ((s = L.tiles_pass(MODE_COL)) != DQ_OK) return s;
+        if ((s = L.col_finalize()) != DQ_OK) return s;
+        if ((s = L.mse(MODE_ROW, t, t, nullptr, nullptr)) != DQ_OK) return s;
+    }
+    if ((s = L.tiles_pass(MODE_PACK)) != DQ_OK) return s;
+    if ((s = L.mse(2, T, -1, nullptr, nullptr)) != DQ_OK) return s;
+    return DQ_OK;
+}
+
+// Single-matrix descriptor for the no-workspace / step entry points.
+dq_status single(const void *W, int32_t dtype, int64_t rows, int64_t cols, const dq_format *fmt,
+                 FmtInfo *fi, MatDesc &d) {
+    if (dtype != DQ_DT_F32 && dtype != DQ_DT_BF16) return DQ_ERR_ARG;
+    dq_status s = check_format(fmt, fi);
+    if (s != DQ_OK) return s;
+    if (rows < 0 || cols < 0) return DQ_ERR_SHAPE;
+    if (cols % fi->G) return DQ_ERR_SHAPE;
+    if (rows > 0 && cols > 0 && !W) return DQ_ERR_ARG;
+    if (!aligned(W, 16)) return DQ_ERR_ALIGN;
+    d = MatDesc{};
+    d.W = W;
+    d.rows = rows;
+    d.cols = cols;
+    d.ts_val = 1.0f;
+    return DQ_OK;
+}
+
+dq_status step_impl(bool row_step, const void *W, int32_t dtype, int64_t rows, int64_t cols,
+                    const dq_format *fmt, float ts, const float *a_in, const float *b_in,
+                    float *out, float *pre, double *mse_in, void *workspace, size_t ws_bytes,
+                    cudaStream_t st) {
+    FmtInfo fi;
+    MatDesc d;
+    dq_status s = single(W, dtype, rows, cols, fmt, &fi, d);
+    if (s != DQ_OK) return s;
+    if (!a_in || !b_in || !out) return DQ_ERR_ARG;
+    if (!(ts > 0.0f)) return DQ_ERR_ARG;
+    if (!aligned(a_in, 4) || !aligned(b_in, 4) || !aligned(out, 4) || !aligned(pre, 4) ||
+        !aligned(mse_in, 8))
+        return DQ_ERR_ALIGN;
+    const bool f32 = dtype == DQ_DT_F32;
+    if (!workspace || ws_bytes < matrix_ws(rows, cols, f32)) return DQ_ERR_WORKSPACE;
+    if (!aligned(workspace, 256)) return DQ_ERR_ALIGN;
+    unsigned int *status = status_ptr();
+    if (!status) return DQ_ERR_CUDA;
+    d.a = a_in;
+    d.b = b_in;
+    d.ts_val = ts;
+    if (row_step) { d.a_out = out; d.a_pre = pre; }
+    else { d.b_out = out; d.b_pre = pre; }
+    Carve cv{static_cast<char *>(workspace), static_cast<char *>(workspace) + ws_bytes};
+    int64_t tb[3] = {0, 0, 0}, rb = 0, cb = 0;
+    place(d, f32, cv, tb, rb, cb);
+    Launcher L;
+    L.tab.dev = nullptr;
+    L.tab.one = d;
+    L.tab.n = 1;
+    L.tab.status = status;
+    L.combo = fi.combo;
+    L.G = fi.G;
+    L.f32 = f32;
+    L.qmax = fi.qmax;
+    for (int m = 0; m < 3; ++m) L.tiles[m] = tb[m];
+    L.total_rows = rb;
+    L.total_cols = cb;
+    L.st = st;
+    if (row_step) {
+        if ((s = L.tiles_pass(MODE_ROW)) != DQ_OK) return s;
+        if ((s = L.row_finalize()) != DQ_OK) return s;
+        if (mse_in) return L.mse(MODE_ROW, -1, -1, mse_in, nullptr);
+    } else {
+        if ((s = L.tiles_pass(MODE_COL)) != DQ_OK) return s;
+        if ((s = L.col_finalize()) != DQ_OK) return s;
+        if (mse_in) return L.mse(-1, -1, -1, nullptr, mse_in);
+    }
+    return DQ_OK;
+}
+
+// out_ij = a_i * c_ij * s_g * ts * b_j
+__global__ void dequant_kernel(const uint8_t *codes, const void *gs, int64_t rows, int64_t cols,
+                               int G, int codes_kind, int gs_kind, float ts, const float *a,
+                               const float *b, float *out) {
+    const int64_t n = rows * cols;
+    for (int64_t k = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; k < n;
+         k += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t r = k / cols, c = k % cols;
+        const uint8_t byte = codes[r * (cols / 2) + c / 2];
+        const uint32_t nib = (c & 1) ? (byte >> 4) : (byte & 0xF);
+        float cv;
+        if (codes_kind == DQ_CODES_INT4) {
+            cv = (float)((int)(nib ^ 8u) - 8);
+        } else {
+            const float mag[8] = {0.f, 0.5f, 1.f, 1.5f, 2.f, 3.f, 4.f, 6.f};
+            cv = (nib & 8u) ? -mag[nib & 7u] : mag[nib & 7u];
+        }
+        const int64_t gi = r * (cols / G) + c / G;
+        float s;
+        if (gs_kind == DQ_SCALE_BF16) {
+            s = __uint_as_float((uint32_t)reinterpret_cast<const uint16_t *>(gs)[gi] << 16);
+        } else if (gs_kind == DQ_SCALE_E8M0) {
+            s = __uint_as_float((uint32_t)reinterpret_cast<const uint8_t *>(gs)[gi] << 23);
+        } else {
+            const uint32_t e = reinterpret_cast<const uint8_t *>(gs)[gi];
+            const uint32_t ex = (e >> 3) & 15u, m = e & 7u;
+            s = ex == 0 ? (float)m * 0.001953125f : __uint_as_float(((ex + 120u) << 23) | (m << 20));
+            if (e & 128u) s = -s;
+        }
+        const float av = a ? a[r] : 1.0f, bv = b ? b[c] : 1.0f;
+        out[k] = av * (cv * (s * ts)) * bv;
+    }
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *dq_version(void) { return "dq 0.1.0 (sm_100a)"; }
+
+const char *dq_strerror(dq_status s) {
+    switch (s) {
+        case DQ_OK: return "ok";
+        case DQ_ERR_ARG: return "invalid argument";
+        case DQ_ERR_SHAPE: return "invalid shape (cols must be a multiple of the group size)";
+        case DQ_ERR_FORMAT: return "unsupported format";
+        case DQ_ERR_NONFINITE: return "non-finite value in the input";
+        case DQ_ERR_RANGE: return "an outer scale was clamped at its set's bound";
+        case DQ_ERR_CUDA: return "CUDA runtime error";
+        case DQ_ERR_WORKSPACE: return "workspace missing or too small";
+        case DQ_ERR_NOT_IMPLEMENTED: return "not implemented";
+        case DQ_ERR_ALIGN: return "pointer alignment";
+    }
+    return "unknown status";
+}
+
+dq_status dq_format_preset(const char *name, int32_t group, dq_format *out) {
+    if (!name || !out) return DQ_ERR_ARG;
+    dq_format f{};
+    if (!strcmp(name, "int4_bf16")) f = {DQ_CODES_INT4, 64, DQ_SCALE_BF16, DQ_SCALE_BF16, 0};
+    else if (!strcmp(name, "mxint4")) f = {DQ_CODES_INT4, 32, DQ_SCALE_E8M0, DQ_SCALE_E8M0, 0};
+    else if (!strcmp(name, "mxfp4")) f = {DQ_CODES_E2M1, 32, DQ_SCALE_E8M0, DQ_SCALE_E8M0, 0};
+    else if (!strcmp(name, "nvfp4")) f = {DQ_CODES_E2M1, 16, DQ_SCALE_E4M3, DQ_SCALE_BF16, 1};
+    else return DQ_ERR_FORMAT;
+    if (group != 0) f.group = group;
+    dq_status s = check_format(&f, nullptr);
+    if (s != DQ_OK) return s;
+    *out = f;
+    return DQ_OK;
+}
+
+dq_status dq_workspace_size(int32_t n, const int64_t *rows, const int64_t *cols,
+                            const dq_format *fmt, size_t *bytes) {
+    if (n < 0 || !bytes || (n > 0 && (!rows || !cols))) return DQ_ERR_ARG;
+    FmtInfo fi;
+    dq_status s = check_format(fmt, &fi);
+    if (s != DQ_OK) return s;
+    size_t b = table_ws(n);
+    for (int i = 0; i < n; ++i) {
+        if (rows[i] < 0 || cols[i] < 0 || cols[i] % fi.G) return DQ_ERR_SHAPE;
+        // the larger of the bf16 and float32 layouts, so one size serves both
+        b += std::max(matrix_ws(rows[i], cols[i], false), matrix_ws(rows[i], cols[i], true));
+    }
+    *bytes = b + 256;
+    return DQ_OK;
+}
+
+dq_status dq_quantize(const void *X, int32_t dtype, int64_t rows, int64_t cols,
+                      const dq_format *fmt, const float *a, const float *b, float tensor_scale,
+                      uint8_t *codes, void *gscales, dq_stream stream) {
+    FmtInfo fi;
+    MatDesc d;
+    dq_status s = single(X, dtype, rows, cols, fmt, &fi, d);
+    if (s != DQ_OK) return s;
+    if (rows == 0 || cols == 0) return DQ_OK;
+    if (!codes || !gscales) return DQ_ERR_ARG;
+    if (!(tensor_scale > 0.0f)) return DQ_ERR_ARG;
+    if (!aligned(codes, 16) || !aligned(gscales, 16) || !aligned(a, 4) || !aligned(b, 4))
+        return DQ_ERR_ALIGN;
+    unsigned int *status = status_ptr();
+    if (!status) return DQ_ERR_CUDA;
+    const bool f32 = dtype == DQ_DT_F32;
+    d.a = a;
+    d.b = b;
+    d.codes = codes;
+    d.gscales = gscales;
+    d.ts_val = tensor_scale;
+    Carve none{nullptr, nullptr};
+    int64_t tb[3] = {0, 0, 0}, rb = 0, cb = 0;
+    place(d, f32, none, tb, rb, cb);
+    Launcher L;
+    L.tab.dev = nullptr;
+    L.tab.one = d;
+    L.tab.n = 1;
+    L.tab.status = status;
+    L.combo = fi.combo;
+    L.G = fi.G;
+    L.f32 = f32;
+    L.qmax = fi.qmax;
+    for (int m = 0; m < 3; ++m) L.tiles[m] = tb[m];
+    L.st = reinterpret_cast<cudaStream_t>(stream);
+    return L.tiles_pass(MODE_PACK);
+}
+
+dq_status dq_act_rescale_quant(const void *X, int64_t tokens, int64_t K, const float *b,
+                               const dq_format *fmt, uint8_t *codes, void *gscales,
+                               dq_stream stream) {
+    FmtInfo fi;
+    MatDesc d;
+    dq_status s = single(X, DQ_DT_BF16, tokens, K, fmt, &fi, d);
+    if (s != DQ_OK) return s;
+    if (tokens == 0 || K == 0) return DQ_OK;
+    if (!codes || !gscales || !b) return DQ_ERR_ARG;
+    if (!aligned(codes, 16) || !aligned(gscales, 16) || !aligned(b, 4)) return DQ_ERR_ALIGN;
+    unsigned int *status = status_ptr();
+    if (!status) return DQ_ERR_CUDA;
+    d.b = b;
+    d.codes = codes;
+    d.gscales = gscales;
+    Carve none{nullptr, nullptr};
+    int64_t tb[3] = {0, 0, 0}, rb = 0, cb = 0;
+    place(d, false, none, tb, rb, cb);
+    Launcher L;
+    L.tab.dev = nullptr;
+    L.tab.one = d;
+    L.tab.n = 1;
+    L.tab.status = status;
+    L.combo = fi.combo;
+    L.G = fi.G;
+    L.f32 = false;
+    L.qmax = fi.qmax;
+    for (int m = 0; m < 3; ++m) L.tiles[m] = tb[m];
+    L.st = reinterpret_cast<cudaStream_t>(stream);
+    return L.tiles_pass(MODE_ACT);
+}
+
+dq_status dq_dequantize(const uint8_t *codes, const void *gscales, int64_t rows, int64_t cols,
+                        const dq_format *fmt, float tensor_scale, const float *a, const float *b,
+                        float *out, dq_stream stream) {
+    FmtInfo fi;
+    dq_status s = check_format(fmt, &fi);
+    if (s != DQ_OK) return s;
+    if (rows < 0 || cols < 0 || cols % fi.G) return DQ_ERR_SHAPE;
+    if (rows == 0 || cols == 0) return DQ_OK;
+    if (!codes || !gscales || !out) return DQ_ERR_ARG;
+    const int64_t n = rows * cols;
+    dequant_kernel<<<grid_for(n, 256), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        codes, gscales, rows, cols, fi.G, fmt->codes, fmt->group_scale, tensor_scale, a, b, out);
+    DQ_CUDA(cudaGetLastError());
+    count_launches(1);
+    return DQ_OK;
+}
+
+dq_status dq_solve_dual_scale(const void *W, int32_t dtype, int64_t rows, int64_t cols,
+                              const dq_format *fmt, int32_t T, const float *a0, const float *b0,
+                              uint8_t *codes, void *gscales, float *a, float *b,
+                              float *tensor_scale, double *mse_trace, double *mse_half,
+                              void *workspace, size_t ws_bytes, dq_stream stream) {
+    dq_matrix m;
+    m.W = W;
+    m.rows = rows;
+    m.cols = cols;
+    m.a0 = a0;
+    m.b0 = b0;
+    m.codes = codes;
+    m.gscales = gscales;
+    m.a = a;
+    m.b = b;
+    m.tensor_scale = tensor_scale;
+    m.mse_trace = mse_trace;
+    m.mse_half = mse_half;
+    return solve_impl(1, &m, dtype, fmt, T, workspace, ws_bytes,
+                      reinterpret_cast<cudaStream_t>(stream));
+}
+
+dq_status dq_solve_dual_scale_batched(int32_t n, const dq_matrix *mats, int32_t dtype,
+                                      const dq_format *fmt, int32_t T, void *workspace,
+                                      size_t ws_bytes, dq_stream stream) {
+    return solve_impl(n, mats, dtype, fmt, T, workspace, ws_bytes,
+                      reinterpret_cast<cudaStream_t>(stream));
+}
+
+dq_status dq_row_update(const void *W, int32_t dtype, int64_t rows, int64_t cols,
+                        const dq_format *fmt, float tensor_scale, const float *a_in,
+                        const float *b_in, float *a_out, float *a_pre, double *mse_in,
+                        void *workspace, size_t ws_bytes, dq_stream stream) {
+    return step_impl(true, W, dtype, rows, cols, fmt, tensor_scale, a_in, b_in, a_out, a_pre,
+                     mse_in, workspace, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+dq_status dq_col_update(const void *W, int32_t dtype, int64_t rows, int64_t cols,
+                        const dq_format *fmt, float tensor_scale, const float *a_in,
+                        const float *b_in, float *b_out, float *b_pre, double *mse_in,
+                        void *workspace, size_t ws_bytes, dq_stream stream) {
+    return step_impl(false, W, dtype, rows, cols, fmt, tensor_scale, a_in, b_in, b_out, b_pre,
+                     mse_in, workspace, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+dq_status dq_last_device_status(dq_stream stream) {
+    unsigned int *p = status_ptr();
+    if (!p) return DQ_ERR_CUDA;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    DQ_CUDA(cudaStreamSynchronize(st));
+    unsigned int v = 0;
+    DQ_CUDA(cudaMemcpy(&v, p, sizeof(v), cudaMemcpyDeviceToHost));
+    const unsigned int zero = 0;
+    DQ_CUDA(cudaMemcpy(p, &zero, sizeof(zero), cudaMemcpyHostToDevice));
+    if (v & STATUS_NONFINITE) return DQ_ERR_NONFINITE;
+    if (v & STATUS_RANGE) return DQ_ERR_RANGE;
+    return DQ_OK;
+}
+
+dq_status dq_kernel_timing(int32_t enable) {
+    std::lock_guard<std::mutex> lk(g_timing_mu);
+    g_timing = enable != 0;
+    return DQ_OK;
+}
+
+dq_status dq_kernel_time(int32_t kind, double *ms, int64_t *launches) {
+    if (!ms || !launches || kind < 0 || kind > 3) return DQ_ERR_ARG;
+    std::lock_guard<std::mutex> lk(g_timing_mu);
+    double tot = 0.0;
+    int64_t cnt = 0;
+    std::vector<TimedLaunch> keep;
+    for (const TimedLaunch &t : g_timed) {
+        if (t.kind != kind) { keep.push_back(t); continue; }
+        float m = 0.0f;
+        DQ_CUDA(cudaEventSynchronize(t.end));
+        DQ_CUDA(cudaEventElapsedTime(&m, t.beg, t.end));
+        tot += m;
+        ++cnt;
+        g_event_pool.push_back(t.beg);
+        g_event_pool.push_back(t.end);
+    }
+    g_timed.swap(keep);
+    *ms = tot;
+    *launches = cnt;
+    return DQ_OK;
+}
+
+int64_t dq_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+}  // extern "C"

@@ -1,0 +1,825 @@
+// dq_device.cuh — device side of the dual-scale solver: format units, the
+// streaming tile kernel (row statistics, column statistics, pack, activation)
+// and the small finalize kernels.
+//
+// Method: DualQuant, daiwk.github.io reproduction note, section "核心公式":
+// eq. (1) W ~= D_a Q(D_a^-1 W D_b^-1) D_b, eq. (2) the closed-form row and
+// column updates, and the order stated under eq. (2) (row update, re-quantize,
+// column update, re-quantize; zero-code slice -> scale 1; projected inverse
+// scales).  Formats: same note, "本地复现" (INT4 [-8,7] with BF16 or E8M0
+// scales, exponent in [-126,126]); news.yiqijian.com article (MXFP4: E2M1 in
+// blocks of 32 with an E8M0 scale; NVFP4: E2M1 in blocks of 16 with an E4M3
+// scale).
+//
+// Exactness.  Every rounding decision (group scale, code) equals the decision
+// on the exact real value W_ij / (a_i b_j s ts).  The fast path computes it in
+// float32; when the float32 value lies within a few ulps of a decision
+// boundary the kernel settles the decision with an fma whose sign is exact
+// (the products a_i*b_j*s are exact in float32 for the formats here: at most
+// 8+8+8 significant bits).  Power-of-two scalings are exact and skip the check.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace dq {
+
+enum { CODES_INT4 = 0, CODES_E2M1 = 1 };
+enum { SC_BF16 = 0, SC_E8M0 = 1, SC_E4M3 = 2 };
+enum { MODE_ROW = 0, MODE_COL = 1, MODE_PACK = 2, MODE_ACT = 3 };
+enum { STATUS_NONFINITE = 1u, STATUS_RANGE = 2u };
+
+constexpr int kWarps = 8;            // warps per CTA of the tile kernel
+constexpr int kThreads = 32 * kWarps;
+constexpr int kRowsPerWarp[4] = {16, 64, 16, 16};   // per mode
+constexpr float kBf16Max = 3.38953138925153547590470800371487866880e+38f;  // (2-2^-7)*2^127
+constexpr float kMinNormal = 1.17549435082228750796873653722224568e-38f;    // 2^-126
+
+// One matrix of a launch.  Tiles of mode m of this matrix are the global
+// tiles [tile0[m], tile0[m] + ntiles[m]); a tile is tr[m] rows by
+// wc * 32 * EPC columns (EPC = 16 bytes of input per lane).
+struct MatDesc {
+    const void *W;
+    int64_t rows, cols;
+    const float *a;          // state a (NULL: ones)
+    const float *b;          // state b (NULL: ones)
+    float *a_out, *b_out;    // finalize outputs
+    float *a_pre, *b_pre;    // unprojected ratios (may be NULL)
+    uint8_t *codes;
+    void *gscales;
+    const float *ts_ptr;     // tensor scale (device) or NULL: use ts_val
+    float ts_val;
+    int32_t wc;              // warps across columns (1, 2, 4, 8)
+    int32_t ncb;             // column blocks
+    int32_t tr[3];           // rows per tile: ROW, COL, PACK/ACT
+    int64_t tile0[3];
+    int64_t ntiles[3];
+    int64_t row0, col0;      // global row / column offsets (finalize kernels)
+    float2 *rowpart;         // [rows][ncb]  (num, den)
+    float2 *colpart;         // [nrb_col][cols]  (P, E)
+    double *res_row;         // [ntiles ROW]  residual partials (also PACK)
+    double *res_col;         // [ntiles COL]
+    unsigned int *amax;      // 1 word (tensor-scale pass)
+    float *ts_out;           // tensor scale output
+    const float *a0, *b0;    // initial state (init kernel)
+    double *mse_trace, *mse_half;
+};
+
+struct Table {
+    const MatDesc *dev;      // n entries in device memory, or NULL when n == 1
+    MatDesc one;             // the single entry when dev == NULL
+    int n;
+    unsigned int *status;    // device flag word (STATUS_*)
+    __device__ __forceinline__ const MatDesc &get(int i) const { return dev ? dev[i] : one; }
+};
+
+// Index of the matrix owning global item `t` (tiles, rows or columns), given
+// a monotone per-matrix start offset.
+template <class F>
+__device__ __forceinline__ int find_owner(const Table &tab, int64_t t, F start) {
+    if (tab.dev == nullptr) return 0;
+    int lo = 0, hi = tab.n - 1;
+    while (lo < hi) {
+        int mid = (lo + hi + 1) >> 1;
+        if (start(tab.dev[mid]) <= t) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+}
+
+// ------------------------------------------------------------------------- //
+// small float helpers
+// ------------------------------------------------------------------------- //
+
+__device__ __forceinline__ float pow2f(int e) {            // 2^e, e in [-126, 127]
+    return __uint_as_float((uint32_t)(e + 127) << 23);
+}
+__device__ __forceinline__ int ilog2f(float x) {            // floor(log2 x), x normal > 0
+    return (int)((__float_as_uint(x) >> 23) & 0xFF) - 127;
+}
+__device__ __forceinline__ float max_nan(float a, float b) {
+    float r;
+    asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+    return r;
+}
+__device__ __forceinline__ uint32_t cvt_e2m1x2(float hi, float lo) {
+    uint16_t r;
+    asm("{ .reg .b8 t; cvt.rn.satfinite.e2m1x2.f32 t, %1, %2; cvt.u16.u8 %0, t; }"
+        : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+__device__ __forceinline__ float2 e2m1x2_to_f32(uint32_t byte) {  // .x = low nibble
+    uint32_t h2;
+    uint16_t b16 = (uint16_t)byte;
+    asm("{ .reg .b8 t; cvt.u8.u16 t, %1; cvt.rn.f16x2.e2m1x2 %0, t; }" : "=r"(h2) : "h"(b16));
+    float lo, hi;
+    asm("{ .reg .f16 l, h; mov.b32 {l, h}, %2; cvt.f32.f16 %0, l; cvt.f32.f16 %1, h; }"
+        : "=f"(lo), "=f"(hi) : "r"(h2));
+    return make_float2(lo, hi);
+}
+__device__ __forceinline__ uint32_t e4m3_bits(float x) {    // x exactly representable
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(x));
+    return r & 0xFF;
+}
+
+// 1/x for a normal power of two x (exact)
+__device__ __forceinline__ float recip_pow2(float x) {
+    return __uint_as_float(0x7F000000u - __float_as_uint(x));
+}
+// 1/x within about one ulp (only feeds estimates that are checked against
+// exact boundaries)
+__device__ __forceinline__ float recip_approx(float x) {
+    float r;
+    asm("rcp.approx.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+
+template <int LPG>
+__device__ __forceinline__ float grp_max(float v) {
+#pragma unroll
+    for (int o = 1; o < LPG; o <<= 1) v = max_nan(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+template <int LPG>
+__device__ __forceinline__ int grp_or(int v) {
+#pragma unroll
+    for (int o = 1; o < LPG; o <<= 1) v |= __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// ------------------------------------------------------------------------- //
+// Group-scale projection P_grp(m / (qmax ts)) with a boundary description
+// ------------------------------------------------------------------------- //
+
+struct ScaleChoice {
+    float s;          // fast-path choice
+    float s_lo, s_hi; // the two candidates around the nearby boundary
+    float s_tie;      // the choice when the exact value sits on the boundary
+    float thr;        // group max m at the boundary (exact float)
+    bool near;        // fast path within tolerance of the boundary
+};
+
+// m > 0 finite.  qts = qmax*ts (exact), rqts ~ 1/qts.
+template <int GS, int CODES>
+__device__ __forceinline__ ScaleChoice project_group(float m, float qts, float rqts, float inv_ts) {
+    ScaleChoice c;
+    c.near = false;
+    c.thr = 0.f;
+    if (GS == SC_E8M0) {
+        // smallest 2^e with qmax * 2^e >= m/ts, e in [-126, 126]
+        float mm = m * inv_ts;                         // exact (power of two)
+        int e;
+        if (mm < kMinNormal) {
+            e = -126;
+            c.s_lo = c.s_hi = c.s_tie = c.s = pow2f(e);
+            return c;
+        }
+        uint32_t u = __float_as_uint(mm);
+        int k = ilog2f(mm);
+        uint32_t mant = u & 0x7FFFFFu;
+        constexpr uint32_t MT = (CODES == CODES_INT4) ? 0x600000u : 0x400000u;  // 1.75 / 1.5
+        e = k - 2 + (mant > MT ? 1 : 0);
+        int elo = min(max(k - 2, -126), 126), ehi = min(max(k - 1, -126), 126);
+        e = min(max(e, -126), 126);
+        c.s = pow2f(e);
+        c.s_lo = pow2f(elo);
+        c.s_hi = pow2f(ehi);
+        c.s_tie = c.s_lo;                              // m == qmax*2^(k-2): ceil is exact
+        int d = (int)mant - (int)MT;
+        c.near = (d < 16 && d > -16);
+        c.thr = __uint_as_float((u & 0xFF800000u) | MT) * (1.0f / inv_ts);  // Q*2^k*ts
+        return c;
+    } else if (GS == SC_BF16) {
+        float g = m * rqts;
+        if (g < kMinNormal) { c.s = c.s_lo = c.s_hi = c.s_tie = kMinNormal; return c; }
+        if (g >= kBf16Max) { c.s = c.s_lo = c.s_hi = c.s_tie = kBf16Max; return c; }
+        uint32_t u = __float_as_uint(g);
+        uint32_t lo = u & 0xFFFF0000u, low = u & 0xFFFFu;
+        float flo = __uint_as_float(lo);
+        float fhi = fminf(__uint_as_float(lo + 0x10000u), kBf16Max);
+        bool odd = (lo & 0x10000u) != 0;
+        c.s_lo = flo;
+        c.s_hi = fhi;
+        c.s_tie = odd ? fhi : flo;
+        c.s = (low > 0x8000u || (low == 0x8000u && odd)) ? fhi : flo;
+        int d = (int)low - 0x8000;
+        c.near = (d < 16 && d > -16);
+        c.thr = __uint_as_float(lo | 0x8000u) * qts;   // 9 bits x qmax*ts: exact
+        return c;
+    } else {  // E4M3, round to nearest even, saturating at 448, 0 -> 2^-9
+        float g = m * rqts;
+        if (g >= 448.0f) { c.s = c.s_lo = c.s_hi = c.s_tie = 448.0f; return c; }
+        int E = (g < 0.015625f) ? -6 : ilog2f(g);      // 2^-6: smallest normal
+        float quant = pow2f(E - 3);
+        float t = g * pow2f(3 - E);                    // exact
+        float fl = floorf(t);
+        float frac = t - fl;
+        float slo = fl * quant, shi = (fl + 1.0f) * quant;
+        if (slo == 0.0f) slo = 0.001953125f;           // 2^-9
+        shi = fminf(shi, 448.0f);
+        c.s_lo = slo;
+        c.s_hi = shi;
+        bool odd = (((int)fl) & 1) != 0;
+        c.s_tie = odd ? shi : slo;
+        c.s = (frac > 0.5f || (frac == 0.5f && odd)) ? shi : slo;
+        c.near = fabsf(frac - 0.5f) <= t * 1.9073486e-06f;   // t * 2^-19
+        c.thr = (fl + 0.5f) * quant * qts;
+        return c;
+    }
+}
+
+// ------------------------------------------------------------------------- //
+// Quantization of one lane's chunk of EPC consecutive elements of one row
+// ------------------------------------------------------------------------- //
+
+template <int CODES, int GS, int OS, bool ACT, int EPC, int LPG>
+struct Quant {
+    // exact fast path: all scalings are powers of two
+    static constexpr bool kExactQ = ACT ? (GS == SC_E8M0) : (GS == SC_E8M0 && OS == SC_E8M0);
+    // exact group max (inner scaling by b, and by a, exact)
+    static constexpr bool kExactM = ACT ? true : (OS == SC_E8M0);
+    static constexpr float kQmax = CODES == CODES_INT4 ? 7.0f : 6.0f;
+
+    // In: w (input values), z = inner-scaled values before the row factor
+    // (w*ib_j for weights, x*b_j for activations), ab = a*b_j (weights, only
+    // read on the exact path), ia = 1/a (weights; 1 for ACT), ts.
+    // Out: c (code values), s (stored group scale), s_eff = s*ts, nib (packed
+    // nibbles of the chunk, element 0 in the low nibble).
+    __device__ __forceinline__ static void run(const float (&w)[EPC], const float (&z)[EPC],
+                                               const float (&ab)[EPC], float ia, float ts,
+                                               float inv_ts, unsigned int *status,
+                                               float (&c)[EPC], float &s, float &s_eff,
+                                               uint32_t &nib) {
+        const float qts = kQmax * ts;
+        const float rqts = 1.0f / qts;
+        // group max of |y|, y = z * ia
+        float mz = 0.0f;
+#pragma unroll
+        for (int j = 0; j < EPC; ++j) mz = max_nan(mz, fabsf(z[j]));
+        mz = grp_max<LPG>(mz);
+        float m = mz * ia;
+        const bool finite = isfinite(m);
+        if (!finite) atomicOr(status, STATUS_NONFINITE);
+        // every lane takes part in the warp votes and group shuffles below,
+        // whatever its group holds (all-zero and out-of-range groups included)
+        const bool pos = finite && (m > 0.0f);
+        ScaleChoice sc = project_group<GS, CODES>(pos ? m : 1.0f, qts, rqts, inv_ts);
+        s = sc.s;
+        const bool resolve = pos && ((GS == SC_E8M0 && kExactM) ? false : sc.near);
+        if (__any_sync(0xffffffffu, resolve)) {
+            // exact comparison of the true group max with sc.thr
+            int gt = 0, eq = 0;
+            if (resolve) {
+                if (kExactM) {
+                    float d = m - sc.thr;                       // both exact: sign exact
+                    gt = d > 0.0f;
+                    eq = d == 0.0f;
+                } else {
+#pragma unroll
+                    for (int j = 0; j < EPC; ++j) {
+                        float d = fmaf(-sc.thr, ab[j], fabsf(w[j]));
+                        gt |= d > 0.0f;
+                        eq |= d == 0.0f;
+                    }
+                }
+            }
+            if (!kExactM) {
+                gt = grp_or<LPG>(gt);
+                eq = grp_or<LPG>(eq);
+            }
+            if (resolve) s = gt ? sc.s_hi : (eq ? sc.s_tie : sc.s_lo);
+        }
+        if (!pos) s = 1.0f;
+        s_eff = s * ts;
+        // code decisions on q = y / s_eff
+        const float r = ia * ((GS == SC_E8M0) ? recip_pow2(s_eff) : recip_approx(s_eff));
+        float q[EPC];
+#pragma unroll
+        for (int j = 0; j < EPC; ++j) q[j] = z[j] * r;
+        if (CODES == CODES_INT4) {
+            nib = 0;
+            bool anynear = false;
+            bool nr[EPC];
+#pragma unroll
+            for (int j = 0; j < EPC; ++j) {
+                float rq = rintf(q[j]);
+                nr[j] = !kExactQ && (fabsf(q[j] - rq) > 0.5f - 1.52587890625e-05f);  // 2^-16
+                anynear |= nr[j];
+                c[j] = fminf(fmaxf(rq, -8.0f), 7.0f);
+            }
+            if (!kExactQ && anynear) {
+#pragma unroll
+                for (int j = 0; j < EPC; ++j) {
+                    if (nr[j]) {
+                        float aq = fabsf(q[j]);
+                        float lo = floorf(aq);
+                        float mid = lo + 0.5f;
+                        float d = ACT ? fmaf(-mid, s_eff, fabsf(z[j]))
+                                      : fmaf(-mid, ab[j] * s_eff, fabsf(w[j]));
+                        float mag = d > 0.0f ? lo + 1.0f
+                                  : (d < 0.0f ? lo : ((((int)lo) & 1) ? lo + 1.0f : lo));
+                        c[j] = fminf(fmaxf(copysignf(mag, q[j]), -8.0f), 7.0f);
+                    }
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < EPC; ++j) nib |= ((uint32_t)((int)c[j]) & 0xFu) << (4 * j);
+        } else {
+            uint32_t byte[EPC / 2];
+#pragma unroll
+            for (int j = 0; j < EPC; j += 2) byte[j / 2] = cvt_e2m1x2(q[j + 1], q[j]);
+            if (!kExactQ) {
+                const float up = 1.0f + 7.62939453125e-06f, dn = 1.0f - 7.62939453125e-06f;  // 2^-17
+#pragma unroll
+                for (int j = 0; j < EPC; j += 2) {
+                    uint32_t bh = cvt_e2m1x2(q[j + 1] * up, q[j] * up);
+                    uint32_t bl = cvt_e2m1x2(q[j + 1] * dn, q[j] * dn);
+                    if (bh != bl) {
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            uint32_t nh = (bh >> (4 * h)) & 0xF, nl = (bl >> (4 * h)) & 0xF;
+                            if (nh != nl) {
+                                int jj = j + h;
+                                float2 vh = e2m1x2_to_f32(nh), vl = e2m1x2_to_f32(nl);
+                                float mh = fabsf(vh.x), ml = fabsf(vl.x);
+                                float mid = 0.5f * (mh + ml);
+                                float d = ACT ? fmaf(-mid, s_eff, fabsf(z[jj]))
+                                              : fmaf(-mid, ab[jj] * s_eff, fabsf(w[jj]));
+                                // the even code of the two neighbours has mantissa bit 0
+                                float even = ((nh & 1u) == 0) ? mh : ml;
+                                float mag = d > 0.0f ? mh : (d < 0.0f ? ml : even);
+                                uint32_t nn = cvt_e2m1x2(0.0f, copysignf(mag, q[jj])) & 0xF;
+                                byte[j / 2] = (byte[j / 2] & ~(0xFu << (4 * h))) | (nn << (4 * h));
+                            }
+                        }
+                    }
+                }
+            }
+            nib = 0;
+#pragma unroll
+            for (int j = 0; j < EPC; j += 2) {
+                // sign of the code follows the sign bit of q (also for a zero result)
+                uint32_t bb = byte[j / 2];
+                bb |= (__float_as_uint(q[j]) >> 31) << 3;
+                bb |= (__float_as_uint(q[j + 1]) >> 31) << 7;
+                byte[j / 2] = bb;
+                float2 v = e2m1x2_to_f32(bb);
+                c[j] = v.x;
+                c[j + 1] = v.y;
+                nib |= bb << (4 * j);
+            }
+        }
+    }
+};
+
+// ------------------------------------------------------------------------- //
+// Loading one lane's chunk
+// ------------------------------------------------------------------------- //
+
+template <typename TIn> struct Chunk;
+template <> struct Chunk<float> {
+    static constexpr int EPC = 4;
+    uint4 raw;
+    __device__ __forceinline__ void load(const void *p) {
+        raw = __ldg(reinterpret_cast<const uint4 *>(p));
+    }
+    __device__ __forceinline__ void zero() { raw = make_uint4(0, 0, 0, 0); }
+    __device__ __forceinline__ void unpack(float (&w)[4]) const {
+        w[0] = __uint_as_float(raw.x); w[1] = __uint_as_float(raw.y);
+        w[2] = __uint_as_float(raw.z); w[3] = __uint_as_float(raw.w);
+    }
+};
+struct Bf16Tag {};
+template <> struct Chunk<Bf16Tag> {
+    static constexpr int EPC = 8;
+    uint4 raw;
+    __device__ __forceinline__ void load(const void *p) {
+        raw = __ldg(reinterpret_cast<const uint4 *>(p));
+    }
+    __device__ __forceinline__ void zero() { raw = make_uint4(0, 0, 0, 0); }
+    __device__ __forceinline__ void unpack(float (&w)[8]) const {
+        const uint32_t v[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            w[2 * k] = __uint_as_float(v[k] << 16);
+            w[2 * k + 1] = __uint_as_float(v[k] & 0xFFFF0000u);
+        }
+    }
+};
+
+__device__ __forceinline__ float tensor_scale_of(const MatDesc &md) {
+    return md.ts_ptr ? *md.ts_ptr : md.ts_val;
+}
+
+// Projection of an outer inverse scale onto its set (nearest value).
+template <int OS>
+__device__ __forceinline__ float project_outer(float x, bool &clamped) {
+    clamped = false;
+    if (OS == SC_E8M0) {
+        // nearest power of two, midpoint 1.5*2^k, tie up; exponent in [-126, 126]
+        if (x < kMinNormal) { clamped = true; return kMinNormal; }
+        uint32_t u = __float_as_uint(x);
+        int k = ilog2f(x) + (((u & 0x7FFFFFu) >= 0x400000u) ? 1 : 0);
+        if (k > 126) { clamped = true; k = 126; }
+        if (k < -126) { clamped = true; k = -126; }
+        return pow2f(k);
+    } else {
+        // bfloat16 round to nearest even, clamped to [2^-126, max]
+        if (!(x < kBf16Max)) { clamped = true; return kBf16Max; }
+        uint32_t u = __float_as_uint(x);
+        uint32_t r = (u + 0x7FFFu + ((u >> 16) & 1u)) & 0xFFFF0000u;
+        float v = __uint_as_float(r);
+        if (v < kMinNormal) { clamped = true; v = kMinNormal; }
+        if (!(v <= kBf16Max)) { clamped = true; v = kBf16Max; }
+        return v;
+    }
+}
+
+// ------------------------------------------------------------------------- //
+// The streaming tile kernel
+// ------------------------------------------------------------------------- //
+//
+// CTA = 8 warps = wr x wc (wc warps across columns).  Warp (r, c) handles the
+// tile's rows r, r + wr, r + 2 wr, ... of column segment c (32 lanes x EPC
+// columns).  Each lane keeps b_j and 1/b_j of its EPC columns in registers
+// for the whole tile.
+//   ROW : per row, sum_j W_ij R_ij and sum_j R_ij^2 (R = Qhat D_b) over the
+//         tile's columns -> rowpart[row][cb]; residual of the state -> res_row
+//   COL : per column, sum_i W_ij S_ij and sum_i S_ij^2 (S = D_a Qhat) over the
+//         tile's rows -> colpart[rb][col]; residual -> res_col
+//   PACK: codes and group scales of Q(W / (a b)); residual -> res_row
+//   ACT : codes and group scales of Q(X * b)
+template <int CODES, int GS, int OS, int MODE, typename TIn, int G>
+__global__ void __launch_bounds__(kThreads)
+tile_kernel(const __grid_constant__ Table tab, int mode_slot) {
+    using CK = Chunk<TIn>;
+    constexpr int EPC = CK::EPC;
+    constexpr int SEG = 32 * EPC;
+    constexpr int LPG = G / EPC;
+    constexpr bool ACT = MODE == MODE_ACT;
+    using Q = Quant<CODES, GS, OS, ACT, EPC, LPG>;
+    constexpr int RPW = kRowsPerWarp[MODE];
+    constexpr int ESZ = 16 / EPC;                    // bytes per element
+
+    __shared__ float2 sm_part[2048];
+    __shared__ double sm_res[kWarps];
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t t = blockIdx.x;
+    const int mi = find_owner(tab, t, [mode_slot](const MatDesc &d) { return d.tile0[mode_slot]; });
+    const MatDesc &md = tab.get(mi);
+    const int64_t lt = t - md.tile0[mode_slot];
+    if (lt >= md.ntiles[mode_slot]) return;          // (uniform per CTA)
+    const int wc = md.wc, wr = kWarps / wc;
+    const int tr = RPW * wr;
+    const int64_t rb = lt / md.ncb, cb = lt % md.ncb;
+    const int my_c = warp % wc, my_r = warp / wc;
+    const int64_t cols = md.cols, rows = md.rows;
+    const int64_t col = (cb * wc + my_c) * (int64_t)SEG + lane * EPC;
+    const bool col_ok = col < cols;
+    const int64_t row_first = rb * tr;
+
+    // per-lane column data
+    float bj[EPC], cm[EPC];
+#pragma unroll
+    for (int j = 0; j < EPC; ++j) { bj[j] = 1.0f; cm[j] = 1.0f; }
+    if (md.b != nullptr && col_ok) {
+#pragma unroll
+        for (int j = 0; j < EPC; ++j) bj[j] = __ldg(md.b + col + j);
+    }
+#pragma unroll
+    for (int j = 0; j < EPC; ++j)
+        cm[j] = ACT ? bj[j] : ((OS == SC_E8M0) ? recip_pow2(bj[j]) : recip_approx(bj[j]));
+
+    const float ts = ACT ? 1.0f : tensor_scale_of(md);
+    const float inv_ts = 1.0f / ts;                 // ts is a power of two
+    const char *Wb = reinterpret_cast<const char *>(md.W);
+
+    float acc_p[EPC], acc_e[EPC];                    // COL accumulators
+#pragma unroll
+    for (int j = 0; j < EPC; ++j) { acc_p[j] = 0.0f; acc_e[j] = 0.0f; }
+    float res = 0.0f;
+
+    constexpr int U = 4;
+    for (int k0 = 0; k0 < RPW; k0 += U) {
+        CK ck[U];
+        int64_t rr[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            rr[u] = row_first + my_r + (int64_t)(k0 + u) * wr;
+            if (rr[u] < rows && col_ok)
+                ck[u].load(Wb + (rr[u] * cols + col) * ESZ);
+            else
+                ck[u].zero();
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t r = rr[u];
+            if (r >= rows) break;                     // warp-uniform
+            float a = 1.0f, ia = 1.0f;
+            if (!ACT && md.a != nullptr) {
+                a = __ldg(md.a + r);
+                ia = (OS == SC_E8M0) ? recip_pow2(a) : recip_approx(a);
+            }
+            float w[EPC], z[EPC], ab[EPC], c[EPC];
+            ck[u].unpack(w);
+#pragma unroll
+            for (int j = 0; j < EPC; ++j) { z[j] = w[j] * cm[j]; ab[j] = a * bj[j]; }
+            float s, s_eff;
+            uint32_t nib;
+            Q::run(w, z, ab, ia, ts, inv_ts, tab.status, c, s, s_eff, nib);
+            if (MODE == MODE_ROW) {
+                float gn = 0.0f, gd = 0.0f;
+                const float as = a * s_eff;
+#pragma unroll
+                for (int j = 0; j < EPC; ++j) {
+                    float uq = c[j] * bj[j];
+                    gn = fmaf(w[j], uq, gn);
+                    gd = fmaf(uq, uq, gd);
+                    float d = fmaf(-as, uq, w[j]);
+                    res = fmaf(d, d, res);
+                }
+                float num = gn * s_eff, den = gd * (s_eff * s_eff);
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+                    num += __shfl_xor_sync(0xffffffffu, num, o);
+                    den += __shfl_xor_sync(0xffffffffu, den, o);
+                }
+                if (lane == 0) sm_part[(k0 + u) * kWarps + warp] = make_float2(num, den);
+            } else if (MODE == MODE_COL) {
+                const float as = a * s_eff;
+#pragma unroll
+                for (int j = 0; j < EPC; ++j) {
+                    float v = c[j] * as;
+                    acc_p[j] = fmaf(w[j], v, acc_p[j]);
+                    acc_e[j] = fmaf(v, v, acc_e[j]);
+                    float d = fmaf(-v, bj[j], w[j]);
+                    res = fmaf(d, d, res);
+                }
+            } else {
+                if (MODE == MODE_PACK) {
+                    const float as = a * s_eff;
+#pragma unroll
+                    for (int j = 0; j < EPC; ++j) {
+                        float d = fmaf(-as, c[j] * bj[j], w[j]);
+                        res = fmaf(d, d, res);
+                    }
+                }
+                if (col_ok) {
+                    uint8_t *cp = md.codes + r * (cols >> 1) + (col >> 1);
+                    if (EPC == 8) *reinterpret_cast<uint32_t *>(cp) = nib;
+                    else *reinterpret_cast<uint16_t *>(cp) = (uint16_t)nib;
+                    if ((lane % LPG) == 0) {
+                        const int64_t gi = r * (cols / G) + col / G;
+                        if (GS == SC_BF16)
+                            reinterpret_cast<uint16_t *>(md.gscales)[gi] = (uint16_t)(__float_as_uint(s) >> 16);
+                        else if (GS == SC_E8M0)
+                            reinterpret_cast<uint8_t *>(md.gscales)[gi] = (uint8_t)((__float_as_uint(s) >> 23) & 0xFF);
+                        else
+                            reinterpret_cast<uint8_t *>(md.gscales)[gi] = (uint8_t)e4m3_bits(s);
+                    }
+                }
+            }
+        }
+    }
+
+    // ---- tile epilogue ----
+    if (MODE == MODE_ROW) {
+        __syncthreads();
+        // rows of the tile: local row k*wr + r is warp-row r's k-th row
+        for (int lr = threadIdx.x; lr < tr; lr += kThreads) {
+            const int k = lr / wr, r = lr % wr;
+            const int64_t row = row_first + r + (int64_t)k * wr;
+            if (row < rows) {
+                float num = 0.0f, den = 0.0f;
+                for (int c2 = 0; c2 < wc; ++c2) {          // fixed order over segments
+                    float2 p = sm_part[k * kWarps + r * wc + c2];
+                    num += p.x;
+                    den += p.y;
+                }
+                md.rowpart[row * md.ncb + cb] = make_float2(num, den);
+            }
+        }
+    }
+    if (MODE == MODE_COL) {
+        if (wr == 1) {
+            if (col_ok) {
+                float2 *dst = md.colpart + rb * cols + col;
+#pragma unroll
+                for (int j = 0; j < EPC; ++j) dst[j] = make_float2(acc_p[j], acc_e[j]);
+            }
+        } else {
+            // reduce over the wr warp-rows of each segment in fixed order
+            const int seg_cols = wc * SEG;
+#pragma unroll
+            for (int j = 0; j < EPC; ++j)
+                sm_part[my_r * seg_cols + my_c * SEG + lane * EPC + j] = make_float2(acc_p[j], acc_e[j]);
+            __syncthreads();
+            for (int cc = threadIdx.x; cc < seg_cols; cc += kThreads) {
+                const int64_t gc = cb * seg_cols + cc;
+                if (gc < cols) {
+                    float p = 0.0f, e = 0.0f;
+                    for (int r = 0; r < wr; ++r) {
+                        float2 v = sm_part[r * seg_cols + cc];
+                        p += v.x;
+                        e += v.y;
+                    }
+                    md.colpart[rb * cols + gc] = make_float2(p, e);
+                }
+            }
+        }
+    }
+    if (MODE == MODE_ROW || MODE == MODE_COL || MODE == MODE_PACK) {
+        double rd = (double)res;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) rd += __shfl_xor_sync(0xffffffffu, rd, o);
+        if (lane == 0) sm_res[warp] = rd;
+        __syncthreads();
+        double *slot = (MODE == MODE_COL) ? md.res_col : md.res_row;
+        if (threadIdx.x == 0 && slot != nullptr) {
+            double tot = 0.0;
+            for (int k = 0; k < kWarps; ++k) tot += sm_res[k];
+            slot[lt] = tot;
+        }
+    }
+}
+
+// ------------------------------------------------------------------------- //
+// Finalize kernels
+// ------------------------------------------------------------------------- //
+
+// a_i <- Pi(sum num / sum den) over the row's column blocks (fixed order).
+template <int OS>
+__global__ void row_finalize_kernel(const __grid_constant__ Table tab, int64_t total_rows) {
+    for (int64_t g = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; g < total_rows;
+         g += (int64_t)gridDim.x * blockDim.x) {
+        const int mi = find_owner(tab, g, [](const MatDesc &d) { return d.row0; });
+        const MatDesc &md = tab.get(mi);
+        const int64_t r = g - md.row0;
+        double num = 0.0, den = 0.0;
+        const float2 *p = md.rowpart + r * md.ncb;
+        for (int k = 0; k < md.ncb; ++k) { num += p[k].x; den += p[k].y; }
+        float a = 1.0f, pre = __int_as_float(0x7fc00000);
+        if (den > 0.0) {
+            pre = (float)(num / den);
+            bool cl;
+            a = project_outer<OS>(pre, cl);
+            if (cl) atomicOr(tab.status, STATUS_RANGE);
+        }
+        if (!isfinite(num) || !isfinite(den)) atomicOr(tab.status, STATUS_NONFINITE);
+        md.a_out[r] = a;
+        if (md.a_pre) md.a_pre[r] = pre;
+    }
+}
+
+// b_j <- Pi(sum P / sum E) over the column's row blocks (fixed order).
+template <int OS>
+__global__ void col_finalize_kernel(const __grid_constant__ Table tab, int64_t total_cols) {
+    for (int64_t g = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; g < total_cols;
+         g += (int64_t)gridDim.x * blockDim.x) {
+        const int mi = find_owner(tab, g, [](const MatDesc &d) { return d.col0; });
+        const MatDesc &md = tab.get(mi);
+        const int64_t c = g - md.col0;
+        const int64_t nrb = md.ntiles[MODE_COL] / md.ncb;
+        double p = 0.0, e = 0.0;
+        for (int64_t k = 0; k < nrb; ++k) {
+            float2 v = md.colpart[k * md.cols + c];
+            p += v.x;
+            e += v.y;
+        }
+        float b = 1.0f, pre = __int_as_float(0x7fc00000);
+        if (e > 0.0) {
+            pre = (float)(p / e);
+            bool cl;
+            b = project_outer<OS>(pre, cl);
+            if (cl) atomicOr(tab.status, STATUS_RANGE);
+        }
+        if (!isfinite(p) || !isfinite(e)) atomicOr(tab.status, STATUS_NONFINITE);
+        md.b_out[c] = b;
+        if (md.b_pre) md.b_pre[c] = pre;
+    }
+}
+
+#ifdef DQ_DEFINE_HOST_KERNELS
+// Non-template kernels: defined in exactly one translation unit.
+
+// One block per (matrix, which): sum residual slots in a fixed order and
+// store sum / (rows * cols).  which = 0: res_row[ntiles[slot0]] -> dst0[idx0];
+// which = 1: res_col[ntiles[COL]] -> dst1[idx1].  Destinations are taken from
+// the descriptor's mse_trace / mse_half unless `out` is given.
+__global__ void mse_finalize_kernel(const __grid_constant__ Table tab, int row_slot, int idx_trace, int idx_half,
+                                    double *out_row, double *out_col) {
+    const int mi = blockIdx.x >> 1, which = blockIdx.x & 1;
+    const MatDesc &md = tab.get(mi);
+    double *dst;
+    const double *src;
+    int64_t n;
+    if (which == 0) {
+        dst = out_row ? out_row + mi : (md.mse_trace && idx_trace >= 0 ? md.mse_trace + idx_trace : nullptr);
+        src = md.res_row;
+        n = (row_slot >= 0) ? md.ntiles[row_slot] : 0;
+    } else {
+        dst = out_col ? out_col + mi : (md.mse_half && idx_half >= 0 ? md.mse_half + idx_half : nullptr);
+        src = md.res_col;
+        n = md.ntiles[MODE_COL];
+    }
+    if (dst == nullptr || (which == 0 && row_slot < 0)) return;
+    __shared__ double sm[256];
+    double acc = 0.0;
+    for (int64_t k = threadIdx.x; k < n; k += blockDim.x) acc += src[k];
+    sm[threadIdx.x] = acc;
+    __syncthreads();
+    for (int w = blockDim.x / 2; w > 0; w >>= 1) {
+        if (threadIdx.x < w) sm[threadIdx.x] += sm[threadIdx.x + w];
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) {
+        const double cnt = (double)md.rows * (double)md.cols;
+        *dst = cnt > 0 ? sm[0] / cnt : 0.0;
+    }
+}
+
+// Initial state: a <- a0 or 1, b <- b0 or 1 (rows then columns, all matrices).
+__global__ void init_state_kernel(const __grid_constant__ Table tab, int64_t total_rows, int64_t total_cols) {
+    for (int64_t g = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; g < total_rows + total_cols;
+         g += (int64_t)gridDim.x * blockDim.x) {
+        if (g < total_rows) {
+            const int mi = find_owner(tab, g, [](const MatDesc &d) { return d.row0; });
+            const MatDesc &md = tab.get(mi);
+            const int64_t r = g - md.row0;
+            md.a_out[r] = md.a0 ? md.a0[r] : 1.0f;
+        } else {
+            const int64_t gc = g - total_rows;
+            const int mi = find_owner(tab, gc, [](const MatDesc &d) { return d.col0; });
+            const MatDesc &md = tab.get(mi);
+            const int64_t c = gc - md.col0;
+            md.b_out[c] = md.b0 ? md.b0[c] : 1.0f;
+        }
+    }
+}
+
+#endif  // DQ_DEFINE_HOST_KERNELS
+
+// amax over each matrix (tiles of the PACK geometry), for the tensor scale.
+template <typename TIn>
+__global__ void __launch_bounds__(kThreads) amax_kernel(const __grid_constant__ Table tab) {
+    constexpr int EPC = Chunk<TIn>::EPC;
+    const int64_t t = blockIdx.x;
+    const int mi = find_owner(tab, t, [](const MatDesc &d) { return d.tile0[MODE_PACK]; });
+    const MatDesc &md = tab.get(mi);
+    const int64_t lt = t - md.tile0[MODE_PACK];
+    if (lt >= md.ntiles[MODE_PACK]) return;
+    // the tile's rows as a flat range of 16-byte chunks
+    // tile (rb, cb): the cb == 0 tiles scan their whole row block
+    const int64_t cpr = md.cols / EPC;
+    const int64_t tr = md.tr[MODE_PACK];
+    const int64_t rb = lt / md.ncb, cb = lt % md.ncb;
+    float m = 0.0f;
+    if (cb == 0) {
+        const int64_t r0 = rb * tr, r1 = min(md.rows, r0 + tr);
+        const uint4 *base = reinterpret_cast<const uint4 *>(md.W);
+        for (int64_t k = r0 * cpr + threadIdx.x; k < r1 * cpr; k += kThreads) {
+            Chunk<TIn> ck;
+            ck.raw = __ldg(base + k);
+            float w[EPC];
+            ck.unpack(w);
+#pragma unroll
+            for (int j = 0; j < EPC; ++j) m = max_nan(m, fabsf(w[j]));
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = max_nan(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if ((threadIdx.x & 31) == 0 && cb == 0) {
+        if (!isfinite(m)) atomicOr(tab.status, STATUS_NONFINITE);
+        else atomicMax(md.amax, __float_as_uint(m));   // non-negative floats order as uints
+    }
+}
+
+#ifdef DQ_DEFINE_HOST_KERNELS
+// ts = 2^ceil(log2(amax / (448 qmax))), exponent in [-126, 126]; 1 if amax == 0.
+__global__ void tensor_scale_kernel(const __grid_constant__ Table tab, float qmax, int enabled) {
+    const int mi = blockIdx.x * blockDim.x + threadIdx.x;
+    if (mi >= tab.n) return;
+    const MatDesc &md = tab.get(mi);
+    float ts = 1.0f;
+    if (enabled) {
+        float amax = __uint_as_float(*md.amax);
+        if (amax > 0.0f) {
+            // 448*qmax = C * 2^11 with C = 1.3125 (qmax 6) or 1.53125 (qmax 7)
+            const uint32_t CT = (qmax == 6.0f) ? 0x280000u : 0x440000u;
+            int e;
+            if (amax < kMinNormal) e = -126;
+            else {
+                int k = ilog2f(amax);
+                e = ((__float_as_uint(amax) & 0x7FFFFFu) <= CT) ? k - 11 : k - 10;
+            }
+            e = min(max(e, -126), 126);
+            ts = pow2f(e);
+        }
+    }
+    *md.ts_out = ts;
+}
+
+#endif  // DQ_DEFINE_HOST_KERNELS
+
+}  // namespace dq

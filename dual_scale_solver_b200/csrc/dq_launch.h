@@ -1,0 +1,72 @@
+// dq_launch.h — host-side launch entry points of the per-format kernel
+// translation units (one unit per (codes, group scale, outer scale) set, so
+// that they compile in parallel).
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "dq_device.cuh"
+
+namespace dq {
+
+struct TileLaunch {
+    Table tab;
+    int64_t grid;       // number of tiles (one CTA each)
+    int mode;           // MODE_*
+    int slot;           // tile table slot: 0 ROW, 1 COL, 2 PACK/ACT
+    int f32;            // 1: float32 input, 0: bfloat16
+    int G;              // 16, 32, 64
+    cudaStream_t stream;
+};
+
+// Format sets with compiled kernels.
+enum Combo {
+    COMBO_INT4_BF16_BF16 = 0,   // INT4, BF16 group, BF16 outer     ("int4_bf16")
+    COMBO_INT4_E8M0_E8M0 = 1,   // INT4, E8M0 group, E8M0 outer     ("mxint4")
+    COMBO_E2M1_E8M0_E8M0 = 2,   // E2M1, E8M0 group, E8M0 outer     ("mxfp4")
+    COMBO_E2M1_E4M3_BF16 = 3,   // E2M1, E4M3 group, BF16 outer     ("nvfp4")
+    COMBO_INT4_E8M0_BF16 = 4,   // INT4, E8M0 group, BF16 outer
+    COMBO_E2M1_E8M0_BF16 = 5,   // E2M1, E8M0 group, BF16 outer
+    COMBO_COUNT = 6
+};
+
+cudaError_t launch_tile_c0(const TileLaunch &L);
+cudaError_t launch_tile_c1(const TileLaunch &L);
+cudaError_t launch_tile_c2(const TileLaunch &L);
+cudaError_t launch_tile_c3(const TileLaunch &L);
+cudaError_t launch_tile_c4(const TileLaunch &L);
+cudaError_t launch_tile_c5(const TileLaunch &L);
+
+// Dispatch over mode, dtype and G for one format set (used by each unit).
+template <int CODES, int GS, int OS>
+cudaError_t launch_tile_combo(const TileLaunch &L) {
+    if (L.grid <= 0) return cudaSuccess;
+    dim3 grid((unsigned)L.grid), block(kThreads);
+#define DQ_TILE(MODE, TIN, GG) \
+    tile_kernel<CODES, GS, OS, MODE, TIN, GG><<<grid, block, 0, L.stream>>>(L.tab, L.slot)
+#define DQ_BY_G(MODE, TIN)                          \
+    switch (L.G) {                                  \
+        case 16: DQ_TILE(MODE, TIN, 16); break;     \
+        case 32: DQ_TILE(MODE, TIN, 32); break;     \
+        case 64: DQ_TILE(MODE, TIN, 64); break;     \
+        default: return cudaErrorInvalidValue;      \
+    }
+#define DQ_BY_T(MODE)                                      \
+    if (L.f32) { DQ_BY_G(MODE, float) } else { DQ_BY_G(MODE, Bf16Tag) }
+    switch (L.mode) {
+        case MODE_ROW: DQ_BY_T(MODE_ROW); break;
+        case MODE_COL: DQ_BY_T(MODE_COL); break;
+        case MODE_PACK: DQ_BY_T(MODE_PACK); break;
+        case MODE_ACT:
+            if (L.f32) return cudaErrorInvalidValue;
+            DQ_BY_G(MODE_ACT, Bf16Tag);
+            break;
+        default: return cudaErrorInvalidValue;
+    }
+#undef DQ_BY_T
+#undef DQ_BY_G
+#undef DQ_TILE
+    return cudaGetLastError();
+}
+
+}  // namespace dq

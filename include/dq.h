@@ -1,0 +1,216 @@
+/*
+ * dq.h — C ABI of the B200 dual-scale weight quantization library.
+ *
+ * The library solves the DualQuant dual-scale model of a weight matrix
+ * (DualQuant reproduction note, daiwk.github.io, section "核心公式", eq. (1)):
+ *
+ *     W  ~=  D_a · Q( D_a^-1 · W · D_b^-1 ) · D_b
+ *
+ * with one outer inverse scale a_i per row and b_j per column, and Q a group
+ * quantizer on a fixed grid whose group scales lie in the format's scale set.
+ * It runs the block coordinate descent of eq. (2) of the same section: with
+ * the codes fixed, a_i <- Pi(sum_j W_ij R_ij / sum_j R_ij^2) with R = Qhat D_b,
+ * re-quantize, then b_j <- Pi(sum_i W_ij S_ij / sum_i S_ij^2) with S = D_a Qhat,
+ * re-quantize; a slice with all-zero codes keeps scale 1.  The activation side
+ * (second half of eq. (1)) multiplies X by b per input channel and quantizes.
+ *
+ * Conventions for every entry point:
+ *  - W and X are row-major [rows, cols] (out-features x in-features; groups of
+ *    G consecutive columns share a group scale).
+ *  - Pointers are DEVICE pointers unless marked (host).  The caller owns every
+ *    buffer; the library allocates no device memory.
+ *  - Calls are asynchronous and ordered on `stream` (a cudaStream_t; NULL is
+ *    the legacy default stream).  Argument errors are reported synchronously
+ *    through the return value and launch nothing.  Input data errors found on
+ *    the device (non-finite values, scale-range clamps) set flags that
+ *    dq_last_device_status() reports; kernels never trap.
+ *  - Shapes: cols % G == 0, G in {16, 32, 64}; rows >= 0 (rows == 0 or
+ *    cols == 0 is a valid empty call).  W, X, codes and gscales must be
+ *    16-byte aligned (base pointers), a/b/scale vectors 4-byte aligned.
+ *  - Codes: two 4-bit codes per byte, the even column in the low nibble.
+ *    INT4 is two's complement in [-8, 7]; E2M1 is the nibble s|ee|m.
+ *    Row i of the codes starts at byte i * cols / 2.
+ *  - Group scales: [rows, cols / G] row-major; BF16 as its uint16 bit
+ *    pattern, E8M0 as a biased exponent byte (127 + e), E4M3 as its byte
+ *    (OCP FP8 E4M3 "fn").  A group whose values are all zero stores 1.0.
+ *  - a, b: float32 values that lie exactly in the outer scale set.
+ *  - MSE values are sum (W - D_a Qhat D_b)^2 / (rows * cols), in double.
+ */
+#ifndef DQ_H
+#define DQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define DQ_API __attribute__((visibility("default")))
+#else
+#define DQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *dq_stream; /* cudaStream_t */
+
+typedef enum dq_status {
+    DQ_OK = 0,
+    DQ_ERR_ARG = -1,            /* null pointer, bad enum, T < 0, n < 0 */
+    DQ_ERR_SHAPE = -2,          /* cols % G != 0, negative size */
+    DQ_ERR_FORMAT = -3,         /* unknown preset or unsupported combination */
+    DQ_ERR_NONFINITE = -4,      /* (device flag) NaN or Inf met in W or X */
+    DQ_ERR_RANGE = -5,          /* (device flag) an outer scale hit the set's bound */
+    DQ_ERR_CUDA = -6,           /* a CUDA runtime call failed */
+    DQ_ERR_WORKSPACE = -7,      /* workspace null or smaller than dq_workspace_size */
+    DQ_ERR_NOT_IMPLEMENTED = -8,
+    DQ_ERR_ALIGN = -9           /* a pointer misses its alignment */
+} dq_status;
+
+enum { DQ_CODES_INT4 = 0, DQ_CODES_E2M1 = 1 };
+enum { DQ_SCALE_BF16 = 0, DQ_SCALE_E8M0 = 1, DQ_SCALE_E4M3 = 2 };
+enum { DQ_DT_F32 = 0, DQ_DT_BF16 = 1 };
+
+/* Format descriptor.  Scale sets (DualQuant pages: daiwk note "本地复现";
+ * news.yiqijian.com article, MXFP4/NVFP4 block structure):
+ *   BF16  — bfloat16 values; as an outer or group scale clamped to the
+ *           normal range [2^-126, max].
+ *   E8M0  — powers of two 2^e, e in [-126, 126].
+ *   E4M3  — OCP FP8 E4M3 values (group scale only), saturating at 448.
+ * Group scales are the projection of (group absmax / qmax) onto the set:
+ * BF16 and E4M3 round to nearest even, E8M0 rounds up (the smallest power of
+ * two that keeps every code in range).  Outer scales a, b are the nearest
+ * value of their set (E8M0: an exact tie goes up).
+ * tensor_scale_auto = 1 gives weights a second-level scale
+ * ts = 2^ceil(log2(amax(W) / (448 * qmax))) (NVFP4); otherwise ts = 1. */
+typedef struct dq_format {
+    int32_t codes;             /* DQ_CODES_* ; qmax = 7 (INT4) or 6 (E2M1) */
+    int32_t group;             /* G in {16, 32, 64} */
+    int32_t group_scale;       /* DQ_SCALE_* */
+    int32_t outer_scale;       /* DQ_SCALE_BF16 or DQ_SCALE_E8M0 */
+    int32_t tensor_scale_auto; /* 0 or 1 */
+} dq_format;
+
+/* One matrix of a batched solve.  All pointers are device pointers. */
+typedef struct dq_matrix {
+    const void *W;             /* [rows, cols] of the call's dtype */
+    int64_t rows, cols;
+    const float *a0, *b0;      /* initial a [rows], b [cols]; NULL = all ones */
+    uint8_t *codes;            /* out: [rows, cols/2] packed codes */
+    void *gscales;             /* out: [rows, cols/G] group scales */
+    float *a, *b;              /* out: final outer inverse scales */
+    float *tensor_scale;       /* out: 1 float, the ts used (1.0 unless auto) */
+    double *mse_trace;         /* out: T+1 doubles ([0] initial state), or NULL */
+    double *mse_half;          /* out: T doubles (after each row step), or NULL */
+} dq_matrix;
+
+/* Library version string (static storage). */
+DQ_API const char *dq_version(void);
+
+/* Text of a status code (static storage). */
+DQ_API const char *dq_strerror(dq_status s);
+
+/* Fill `out` (host) with a named preset: "int4_bf16" (INT4 codes, BF16 group
+ * and outer scales, default G 64), "mxint4" (INT4, E8M0, E8M0, G 32),
+ * "mxfp4" (E2M1, E8M0, E8M0, G 32), "nvfp4" (E2M1, E4M3 group, BF16 outer,
+ * G 16, tensor_scale_auto).  group == 0 keeps the preset's G.  Presets follow
+ * the formats of Table 1 of the daiwk note and the news article's MXFP4/NVFP4
+ * description.  Errors: DQ_ERR_ARG (null), DQ_ERR_FORMAT (unknown name or G). */
+DQ_API dq_status dq_format_preset(const char *name, int32_t group, dq_format *out);
+
+/* Bytes of device workspace a solve or a single update of the listed
+ * matrices needs (host arrays rows[n], cols[n]; result in *bytes, host).
+ * Workspace holds per-tile partial sums; it needs no initialisation and no
+ * alignment beyond 256 bytes.  Errors: DQ_ERR_ARG, DQ_ERR_SHAPE, DQ_ERR_FORMAT. */
+DQ_API dq_status dq_workspace_size(int32_t n, const int64_t *rows, const int64_t *cols,
+                            const dq_format *fmt, size_t *bytes);
+
+/* Q(X ⊘ (a bᵀ)): the black-box group quantizer (daiwk note, "原始论文总结")
+ * applied to X / (a_i b_j) with second-level scale `tensor_scale` (host value,
+ * a power of two; 1.0 when the format has none).  a (rows) and b (cols) may be
+ * NULL (all ones).  Writes packed codes and group scales.  No workspace. */
+DQ_API dq_status dq_quantize(const void *X, int32_t dtype, int64_t rows, int64_t cols,
+                      const dq_format *fmt, const float *a, const float *b,
+                      float tensor_scale, uint8_t *codes, void *gscales,
+                      dq_stream stream);
+
+/* out_ij = a_i * c_ij * s_g * ts * b_j (float32), the reconstruction
+ * D_a Qhat D_b of eq. (1).  a or b may be NULL (ones). */
+DQ_API dq_status dq_dequantize(const uint8_t *codes, const void *gscales, int64_t rows,
+                        int64_t cols, const dq_format *fmt, float tensor_scale,
+                        const float *a, const float *b, float *out, dq_stream stream);
+
+/* Full DualQuant solve of one matrix: initialise (a0, b0 or ones), then T
+ * iterations of {row update, re-quantize, column update, re-quantize}
+ * (eq. (2) and the order stated under it), then write the codes and group
+ * scales of Q(W ⊘ (a bᵀ)) for the final a, b.  tensor_scale (1 float) receives
+ * the ts used.  mse_trace (T+1) and mse_half (T) may be NULL.  `workspace`
+ * must hold dq_workspace_size bytes for this one matrix. */
+DQ_API dq_status dq_solve_dual_scale(const void *W, int32_t dtype, int64_t rows, int64_t cols,
+                              const dq_format *fmt, int32_t T, const float *a0,
+                              const float *b0, uint8_t *codes, void *gscales, float *a,
+                              float *b, float *tensor_scale, double *mse_trace,
+                              double *mse_half, void *workspace, size_t ws_bytes,
+                              dq_stream stream);
+
+/* The same solve for n independent matrices (host array mats[n]) sharing one
+ * format, dtype and T, in one launch sequence (every kernel covers all
+ * matrices).  Workspace: dq_workspace_size over all n shapes.  The work table
+ * (one entry per matrix) is built in a host buffer the library keeps per
+ * thread and copied into the workspace with one cudaMemcpyAsync; the call
+ * returns once the table is staged, so `mats` may be reused at once. */
+DQ_API dq_status dq_solve_dual_scale_batched(int32_t n, const dq_matrix *mats, int32_t dtype,
+                                      const dq_format *fmt, int32_t T, void *workspace,
+                                      size_t ws_bytes, dq_stream stream);
+
+/* One row half-step of eq. (2) from the state (a_in, b_in):
+ * a_out_i = Pi_Fa(<W_i, R_i> / <R_i, R_i>), R = Q(W ⊘ a_in b_inᵀ) D_b, zero
+ * slice -> 1.  a_pre (rows, may be NULL) receives the unprojected ratio
+ * (NaN on zero slices); mse_in (1 double, may be NULL) the MSE of the input
+ * state.  a_out may alias a_in. */
+DQ_API dq_status dq_row_update(const void *W, int32_t dtype, int64_t rows, int64_t cols,
+                        const dq_format *fmt, float tensor_scale, const float *a_in,
+                        const float *b_in, float *a_out, float *a_pre, double *mse_in,
+                        void *workspace, size_t ws_bytes, dq_stream stream);
+
+/* One column half-step of eq. (2) from the state (a_in, b_in):
+ * b_out_j = Pi_Fb(<W_:j, S_:j> / <S_:j, S_:j>), S = D_a Q(W ⊘ a_in b_inᵀ).
+ * b_pre (cols, may be NULL): unprojected ratio; mse_in: MSE of the input
+ * state.  b_out may alias b_in. */
+DQ_API dq_status dq_col_update(const void *W, int32_t dtype, int64_t rows, int64_t cols,
+                        const dq_format *fmt, float tensor_scale, const float *a_in,
+                        const float *b_in, float *b_out, float *b_pre, double *mse_in,
+                        void *workspace, size_t ws_bytes, dq_stream stream);
+
+/* Activation side of eq. (1): Q(X D_b) with ts = 1 — each input channel j is
+ * multiplied by b_j, then quantized in groups of G along K (the trove summary,
+ * "How to use it": beta is applied inside the activation-quantization kernel).
+ * X is bf16 [tokens, K]; b float [K].  Writes packed codes [tokens, K/2] and
+ * group scales [tokens, K/G].  No workspace. */
+DQ_API dq_status dq_act_rescale_quant(const void *X, int64_t tokens, int64_t K, const float *b,
+                               const dq_format *fmt, uint8_t *codes, void *gscales,
+                               dq_stream stream);
+
+/* Synchronise `stream`, read and clear the device flags raised by earlier
+ * calls on this device: DQ_ERR_NONFINITE if an input held NaN/Inf,
+ * DQ_ERR_RANGE if an outer scale was clamped at its set's bound, DQ_OK
+ * otherwise (NONFINITE wins when both are set).  The flags are one word per
+ * device shared by all streams. */
+DQ_API dq_status dq_last_device_status(dq_stream stream);
+
+/* Measurement support (no counterpart in the method).  dq_kernel_timing(1)
+ * makes every tile-kernel launch of the library record a CUDA event pair on
+ * its own stream (kind 0 row statistics, 1 column statistics, 2 pack,
+ * 3 activation); dq_kernel_time synchronises those events and returns (and
+ * clears) the summed milliseconds and the launch count of one kind.
+ * dq_launch_count returns the number of kernels this library has launched in
+ * the process so far (all kinds, including finalize kernels). */
+DQ_API dq_status dq_kernel_timing(int32_t enable);
+DQ_API dq_status dq_kernel_time(int32_t kind, double *ms, int64_t *launches);
+DQ_API int64_t dq_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DQ_H */

@@ -1,0 +1,58 @@
+"""Shared helpers of the GPU parity tests (oracle side and conversions)."""
+import numpy as np
+import torch
+
+import oracle as O
+
+PRESET_COMBOS = {
+    # name -> (oracle Format factory); the library's presets carry the same sets
+    "int4_bf16": lambda G: O.preset("int4_bf16", G),
+    "mxint4": lambda G: O.preset("mxint4", G),
+    "mxfp4": lambda G: O.preset("mxfp4", G),
+    "nvfp4": lambda G: O.preset("nvfp4", G),
+    # BF16 outer scales with E8M0 group scales (descriptor variant)
+    "mxint4_bf16outer": lambda G: O.Format("int4", G, "e8m0", "bf16"),
+    "mxfp4_bf16outer": lambda G: O.Format("e2m1", G, "e8m0", "bf16"),
+}
+
+
+def lib_format(name, G):
+    import dual_scale_solver_b200 as dq
+    if name.endswith("_bf16outer"):
+        f = dq.format_preset(name.split("_")[0], G)
+        f.outer_scale = 0
+        return f
+    return dq.format_preset(name, G)
+
+
+def np64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().to("cpu", torch.float64).numpy()
+
+
+def gpu_scales_np(gs: torch.Tensor) -> np.ndarray:
+    g = gs.detach().cpu().numpy()
+    return g.view(np.uint16) if g.dtype == np.int16 else g
+
+
+def oracle_encoded(W64, a, b, fmt, ts=1.0):
+    """Packed codes and encoded group scales of Q(W / (a b^T)) by the oracle."""
+    c, s = O.quantize(O.inner(W64, a, b), fmt, ts)
+    return O.encode_codes(c, fmt), O.encode_scales(s, fmt)
+
+
+def random_outer(fmt, n, key, spread=0.7):
+    """Seeded outer scales in the format's set (inputs of a parity case)."""
+    import synth
+    u = synth.uniform(key, n).numpy()
+    return O.project_outer(np.exp((2 * u - 1) * spread), fmt)
+
+
+def near_outer_boundary(x, fmt, rel=1e-5):
+    """True where x is within `rel` of a decision boundary of the outer projection."""
+    x = np.asarray(x, dtype=np.float64)
+    if fmt.oscale == "e8m0":
+        m, e = np.frexp(x)                       # x = m 2^e, boundary at m = 0.75
+        return np.abs(m - 0.75) <= 0.75 * rel
+    lo = O.project_outer(x * (1 - rel), fmt)
+    hi = O.project_outer(x * (1 + rel), fmt)
+    return lo != hi

@@ -1,0 +1,92 @@
+"""The C-ABI library loads, exports every symbol include/dq.h declares, and
+validates arguments on the host (no kernel launches; runs without a GPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import dual_scale_solver_b200 as dq
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "dq.h")).read()
+    return sorted(set(re.findall(r"^DQ_API\s+[^(]*?\b(dq_\w+)\s*\(", src, flags=re.M)))
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    from dual_scale_solver_b200 import build
+    build.build()
+
+
+def test_exports_match_header():
+    names = _declared()
+    assert len(names) == 15
+    assert sorted(dq.EXPORTS) == names
+    L = dq.lib()
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_version_and_errors():
+    assert "sm_100a" in dq.version()
+    assert dq.lib().dq_strerror(-2).decode().startswith("invalid shape")
+
+
+@pytest.mark.parametrize("name,codes,gs,os_,G,auto", [
+    ("int4_bf16", 0, 0, 0, 64, 0), ("mxint4", 0, 1, 1, 32, 0),
+    ("mxfp4", 1, 1, 1, 32, 0), ("nvfp4", 1, 2, 0, 16, 1)])
+def test_presets(name, codes, gs, os_, G, auto):
+    f = dq.format_preset(name)
+    assert (f.codes, f.group_scale, f.outer_scale, f.group, f.tensor_scale_auto) == (codes, gs, os_, G, auto)
+    assert dq.format_preset(name, 32).group == 32
+
+
+def test_bad_preset_and_group():
+    with pytest.raises(dq.DqError) as e:
+        dq.format_preset("fp8")
+    assert e.value.status == -3
+    with pytest.raises(dq.DqError):
+        dq.format_preset("mxfp4", 48)
+
+
+def test_workspace_size_and_shape_checks():
+    f = dq.format_preset("mxfp4")
+    n1 = dq.workspace_size([(8192, 8192)], f)
+    n2 = dq.workspace_size([(8192, 8192), (1024, 8192)], f)
+    assert 0 < n1 < n2
+    # per-tile column partials stay small next to the matrix (8 B per column
+    # per 64-row tile: 1/16 of its bf16 bytes, plus row partials)
+    assert n1 < 0.07 * 8192 * 8192 * 2
+    with pytest.raises(dq.DqError) as e:
+        dq.workspace_size([(16, 40)], f)            # 40 % 32 != 0
+    assert e.value.status == -2
+    assert dq.workspace_size([], f) > 0 or dq.workspace_size([], f) == 256
+
+
+def test_host_side_argument_errors():
+    L = dq.lib()
+    f = dq.format_preset("int4_bf16")
+    bad = dq.dq_format(0, 48, 0, 0, 0)
+    # bad format, shape and missing pointers are refused before any launch
+    assert L.dq_quantize(None, 1, 4, 64, ctypes.byref(bad), None, None, 1.0, None, None, None) == -3
+    assert L.dq_quantize(None, 1, 4, 65, ctypes.byref(f), None, None, 1.0, None, None, None) == -2
+    assert L.dq_quantize(None, 1, 4, 64, ctypes.byref(f), None, None, 1.0, None, None, None) == -1
+    assert L.dq_quantize(None, 7, 4, 64, ctypes.byref(f), None, None, 1.0, None, None, None) == -1
+    # misaligned input pointer
+    assert L.dq_quantize(ctypes.c_void_p(8), 1, 4, 64, ctypes.byref(f), None, None, 1.0,
+                         ctypes.c_void_p(16), ctypes.c_void_p(16), None) == -9
+    # empty shapes are valid no-ops
+    assert L.dq_quantize(None, 1, 0, 64, ctypes.byref(f), None, None, 1.0, None, None, None) == 0
+    # a solve without workspace
+    assert L.dq_solve_dual_scale(ctypes.c_void_p(256), 1, 4, 64, ctypes.byref(f), 3, None, None,
+                                 ctypes.c_void_p(256), ctypes.c_void_p(256), ctypes.c_void_p(256),
+                                 ctypes.c_void_p(256), ctypes.c_void_p(256), None, None, None, 0,
+                                 None) == -7
+    # tensor_scale_auto only with E4M3 group scales
+    assert L.dq_workspace_size(0, None, None, ctypes.byref(dq.dq_format(1, 32, 1, 1, 1)),
+                               ctypes.byref(ctypes.c_size_t())) == -3
+    assert L.dq_solve_dual_scale_batched(-1, None, 1, ctypes.byref(f), 1, None, 0, None) == -1

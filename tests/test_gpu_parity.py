@@ -1,0 +1,339 @@
+"""GPU path versus the fp64 oracle, element by element, on seeded inputs.
+
+Bars (derived from the method's arithmetic):
+* codes and group scales of Q given identical (a, b, ts): bit-exact;
+* activation codes and scales given identical b: bit-exact;
+* one half-step from an identical state: unprojected ratios within 1e-5
+  relative (float32 sums over <= 28672 terms against fp64); projected scales
+  equal except where the ratio lies within 1e-5 of a projection boundary
+  (listed, at most 1e-3 of the scales);
+* after T iterations: every mse_trace entry within 1e-4 relative.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import synth
+from _helpers import (PRESET_COMBOS, gpu_scales_np, lib_format, near_outer_boundary, np64,
+                      oracle_encoded, random_outer)
+
+pytestmark = pytest.mark.gpu
+
+dq = pytest.importorskip("dual_scale_solver_b200")
+
+ALL = list(PRESET_COMBOS)
+DEFAULT_G = {"int4_bf16": 64, "mxint4": 32, "mxfp4": 32, "nvfp4": 16,
+             "mxint4_bf16outer": 32, "mxfp4_bf16outer": 32}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from dual_scale_solver_b200 import build
+    build.build()
+
+
+def _weights(rows, cols, dtype, key=7, scale=0.02, outliers=0.01):
+    n = rows * cols
+    w = synth.student_t4(synth.stream_key(90, key, rows, cols), n).view(rows, cols) * scale
+    k = max(1, int(round(outliers * cols)))
+    idx = synth.distinct_indices(synth.stream_key(91, key, cols), cols, k)
+    w[:, idx] *= 10
+    return w.to(dtype)
+
+
+# --------------------------------------------------------------------------- #
+# Q itself
+# --------------------------------------------------------------------------- #
+
+@pytest.mark.parametrize("name", ALL)
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("shape", [(300, 2240), (37, 576), (5, 64)])
+def test_quantize_bit_exact(name, dtype, shape):
+    G = DEFAULT_G[name]
+    rows, cols = shape
+    if cols % G:
+        pytest.skip("shape not a multiple of G")
+    fo = PRESET_COMBOS[name](G)
+    fl = lib_format(name, G)
+    W = _weights(rows, cols, dtype, key=ALL.index(name))
+    a = random_outer(fo, rows, synth.stream_key(92, rows))
+    b = random_outer(fo, cols, synth.stream_key(93, cols))
+    ts = 2.0 ** -10 if fo.tensor_scale_auto else 1.0
+    Wd = W.cuda()
+    codes, gs = dq.quantize(Wd, fl, torch.tensor(a, dtype=torch.float32, device="cuda"),
+                            torch.tensor(b, dtype=torch.float32, device="cuda"), ts)
+    torch.cuda.synchronize()
+    ec, es = oracle_encoded(np64(W), a, b, fo, ts)
+    gc, gsn = codes.cpu().numpy(), gpu_scales_np(gs)
+    bad_s = np.argwhere(gsn != es)
+    assert bad_s.size == 0, f"{len(bad_s)} group scales differ, first {bad_s[:5].tolist()}"
+    bad_c = np.argwhere(gc != ec)
+    assert bad_c.size == 0, f"{len(bad_c)} code bytes differ, first {bad_c[:5].tolist()}"
+
+
+def _tie_matrix(fo, kind):
+    """fp32 rows whose values sit exactly on decision boundaries of Q (and one
+    float32 ulp either side) for a = b = non-trivial BF16/E8M0 values."""
+    G = fo.group
+    rows = []
+    rng = np.random.default_rng(3)
+    # decision boundaries of the code grid: half-integers (INT4), E2M1 midpoints
+    grid = np.arange(0, 7) + 0.5 if fo.codes == "int4" else \
+        np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0])
+    for r in range(24):
+        s = 2.0 ** int(rng.integers(-9, -3))
+        if fo.gscale == "bf16":
+            s *= 1 + int(rng.integers(0, 8)) / 8.0
+        vals = [fo.qmax * s]                    # fixes the group max: g = s exactly
+        while len(vals) < G:
+            q = grid[int(rng.integers(0, len(grid)))]
+            v = q * s * (1 if rng.random() < 0.5 else -1)
+            if kind == 1:
+                v = float(np.nextafter(np.float32(v), np.float32(np.inf)))
+            elif kind == 2:
+                v = float(np.nextafter(np.float32(v), np.float32(-np.inf)))
+            vals.append(v)
+        rows.append(vals * 2)
+    return np.array(rows, dtype=np.float32).astype(np.float64)
+
+
+@pytest.mark.parametrize("name", ALL)
+@pytest.mark.parametrize("kind", [0, 1, 2])
+def test_quantize_ties_and_neighbours(name, kind):
+    G = DEFAULT_G[name]
+    fo = PRESET_COMBOS[name](G)
+    fl = lib_format(name, G)
+    Y = _tie_matrix(fo, kind)                        # quantizer input for a = b = 1
+    rows, cols = Y.shape
+    a_val = 1.0 if fo.oscale == "e8m0" else 1.125    # BF16 outer: exercise inexact paths
+    a = np.full(rows, a_val)
+    b = np.ones(cols)
+    W = (Y * a_val).astype(np.float32)
+    ts = 1.0
+    Wd = torch.from_numpy(W).cuda()
+    codes, gs = dq.quantize(Wd, fl, torch.tensor(a, dtype=torch.float32, device="cuda"),
+                            torch.tensor(b, dtype=torch.float32, device="cuda"), ts)
+    ec, es = oracle_encoded(W.astype(np.float64), a, b, fo, ts)
+    assert np.array_equal(gpu_scales_np(gs), es)
+    assert np.array_equal(codes.cpu().numpy(), ec)
+
+
+def test_group_scale_ties_bf16():
+    # group max exactly 7 * (bf16 midpoint) * a: the scale rounds to the even neighbour
+    fo = O.preset("int4_bf16", 16)
+    fl = dq.format_preset("int4_bf16", 16)
+    mids = []
+    for k in range(40):
+        lo = (1 + k / 128.0) * 2.0 ** -5
+        mids.append(lo + 2.0 ** -13)                  # half a bf16 ulp above lo
+    a = 1.0 + 3 / 128.0
+    W = np.zeros((len(mids), 16), dtype=np.float32)
+    for i, m in enumerate(mids):
+        W[i, 0] = 7 * m * a
+        W[i, 1] = np.nextafter(np.float32(7 * m * a), np.float32(0))
+    assert np.all(W[:, 0].astype(np.float64) == 7 * np.array(mids) * a)
+    av = np.full(len(mids), a)
+    codes, gs = dq.quantize(torch.from_numpy(W).cuda(), fl,
+                            torch.tensor(av, dtype=torch.float32, device="cuda"), None, 1.0)
+    ec, es = oracle_encoded(W.astype(np.float64), av, np.ones(16), fo)
+    assert np.array_equal(gpu_scales_np(gs), es)
+    assert np.array_equal(codes.cpu().numpy(), ec)
+
+
+# --------------------------------------------------------------------------- #
+# Activation rescale + quantize
+# --------------------------------------------------------------------------- #
+
+@pytest.mark.parametrize("name", ["int4_bf16", "nvfp4", "mxfp4", "mxint4"])
+@pytest.mark.parametrize("tokens", [1, 333])
+def test_act_rescale_quant_bit_exact(name, tokens):
+    G = DEFAULT_G[name]
+    fo = PRESET_COMBOS[name](G)
+    fl = dq.format_preset(name, G)
+    K = 4096
+    wl = synth.WORKLOADS["llama31_8b_int4_g64"]
+    X = synth.activation(wl, tokens=tokens)
+    b = random_outer(fo, K, synth.stream_key(94, K))
+    codes, gs = dq.act_rescale_quant(X.cuda(), torch.tensor(b, dtype=torch.float32, device="cuda"), fl)
+    c, s = O.act_rescale_quant(np64(X), b, fo)
+    assert np.array_equal(gpu_scales_np(gs), O.encode_scales(s, fo))
+    assert np.array_equal(codes.cpu().numpy(), O.encode_codes(c, fo))
+
+
+# --------------------------------------------------------------------------- #
+# One half-step from an identical state
+# --------------------------------------------------------------------------- #
+
+def _check_projected(gpu, orc, pre, fo, what):
+    diff = gpu != orc
+    near = near_outer_boundary(pre, fo)
+    unexplained = np.argwhere(diff & ~near)
+    assert unexplained.size == 0, f"{what}: {unexplained.size} differ away from a boundary"
+    assert diff.sum() <= max(1, 1e-3 * diff.size), f"{what}: {diff.sum()} near-boundary flips"
+
+
+@pytest.mark.parametrize("name", ALL)
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_half_steps_from_identical_state(name, dtype):
+    G = DEFAULT_G[name]
+    fo = PRESET_COMBOS[name](G)
+    fl = lib_format(name, G)
+    rows, cols = 333, 4160
+    W = _weights(rows, cols, dtype, key=11)
+    W64 = np64(W)
+    a = random_outer(fo, rows, synth.stream_key(95, 1), 0.3)
+    b = random_outer(fo, cols, synth.stream_key(95, 2), 0.3)
+    ts = O.tensor_scale(W64, fo)
+    Wd = W.cuda()
+    ad = torch.tensor(a, dtype=torch.float32, device="cuda")
+    bd = torch.tensor(b, dtype=torch.float32, device="cuda")
+    # row step
+    a_gpu, a_pre, mse0 = dq.row_update(Wd, fl, ad, bd, ts)
+    Qh, _, _ = O.qhat(W64, a, b, fo, ts)
+    a_or, x_or = O.row_update(W64, Qh, b, fo)
+    pre = np64(a_pre)
+    ok = ~np.isnan(x_or)
+    assert np.array_equal(np.isnan(pre), np.isnan(x_or))
+    assert np.max(np.abs(pre[ok] - x_or[ok]) / x_or[ok]) < 1e-5
+    _check_projected(np64(a_gpu), a_or, x_or, fo, "a")
+    assert abs(mse0.item() - O.mse(W64, Qh, a, b)) <= 1e-6 * O.mse(W64, Qh, a, b)
+    # column step from (a_gpu, b)
+    a1 = np64(a_gpu)
+    b_gpu, b_pre, mse1 = dq.col_update(Wd, fl, a_gpu, bd, ts)
+    Qh1, _, _ = O.qhat(W64, a1, b, fo, ts)
+    b_or, xb_or = O.col_update(W64, Qh1, a1, fo)
+    pre = np64(b_pre)
+    ok = ~np.isnan(xb_or)
+    assert np.array_equal(np.isnan(pre), np.isnan(xb_or))
+    assert np.max(np.abs(pre[ok] - xb_or[ok]) / xb_or[ok]) < 1e-5
+    _check_projected(np64(b_gpu), b_or, xb_or, fo, "b")
+    ref = O.mse(W64, Qh1, a1, b)
+    assert abs(mse1.item() - ref) <= 1e-6 * ref
+
+
+# --------------------------------------------------------------------------- #
+# Whole solves
+# --------------------------------------------------------------------------- #
+
+def _solve_and_compare(Ws, fo, fl, T, tol=1e-4):
+    outs = dq.solve_dual_scale_batched([W.cuda() for W in Ws], fl, T, half=True)
+    torch.cuda.synchronize()
+    worst = 0.0
+    for W, o in zip(Ws, outs):
+        W64 = np64(W)
+        r = O.solve(W64, fo, T)
+        tr = np64(o["mse_trace"])
+        rel = np.abs(tr - r["mse_trace"]) / r["mse_trace"]
+        worst = max(worst, rel.max())
+        assert rel.max() < tol, (rel, tr, r["mse_trace"])
+        hf = np64(o["mse_half"])[:T]
+        assert np.max(np.abs(hf - r["mse_half"]) / r["mse_half"]) < tol
+        assert float(o["tensor_scale"].item()) == r["ts"]
+        # the stored codes are Q at the GPU's own final state, bit for bit
+        a, b = np64(o["a"]), np64(o["b"])
+        ec, es = oracle_encoded(W64, a, b, fo, r["ts"])
+        assert np.array_equal(o["codes"].cpu().numpy(), ec)
+        assert np.array_equal(gpu_scales_np(o["gscales"]), es)
+        # most scales agree with the oracle's trajectory exactly
+        same = (np.mean(a == r["a"]) + np.mean(b == r["b"])) / 2
+        assert same > 0.97, same
+    return worst
+
+
+def test_solve_toy_workload():
+    wl = synth.WORKLOADS["toy256x512_int4_g32"]
+    W = synth.weight(wl, 0, 0)
+    fo = O.preset(wl.fmt, wl.group)
+    fl = dq.format_preset(wl.fmt, wl.group)
+    _solve_and_compare([W], fo, fl, wl.T)
+
+
+@pytest.mark.parametrize("name", ["int4_bf16", "nvfp4", "mxfp4"])
+def test_solve_single_matrix_entry_point(name):
+    G = DEFAULT_G[name]
+    fo, fl = PRESET_COMBOS[name](G), dq.format_preset(name, G)
+    W = _weights(200, 1536, torch.bfloat16, key=5)
+    o = dq.solve_dual_scale(W.cuda(), fl, 4)
+    torch.cuda.synchronize()
+    r = O.solve(np64(W), fo, 4)
+    tr = np64(o["mse_trace"])
+    assert np.max(np.abs(tr - r["mse_trace"]) / r["mse_trace"]) < 1e-4
+
+
+def test_solve_smollm2_decoder0_batched_with_all_30():
+    wl = synth.WORKLOADS["smollm2_135m_mxint4_g32"]
+    fo = O.preset(wl.fmt, wl.group)
+    fl = dq.format_preset(wl.fmt, wl.group)
+    mats = wl.matrices
+    Ws = [synth.weight(wl, d, i, device="cuda") for d, i, _ in mats]
+    outs = dq.solve_dual_scale_batched(Ws, fl, wl.T, half=True)
+    torch.cuda.synchronize()
+    assert len(outs) == 210
+    for k in range(7):                       # decoder 0 against the oracle
+        W64 = np64(Ws[k])
+        r = O.solve(W64, fo, wl.T)
+        tr = np64(outs[k]["mse_trace"])
+        assert np.max(np.abs(tr - r["mse_trace"]) / r["mse_trace"]) < 1e-4
+        ec, es = oracle_encoded(W64, np64(outs[k]["a"]), np64(outs[k]["b"]), fo)
+        assert np.array_equal(outs[k]["codes"].cpu().numpy(), ec)
+        assert np.array_equal(gpu_scales_np(outs[k]["gscales"]), es)
+    # dual-scale never ends above single-scale, and beats it on most matrices
+    # (with E8M0 outer scales a solve can stay at RTN when no b_j leaves 1)
+    final = np.array([np64(o["mse_trace"])[-1] for o in outs])
+    start = np.array([np64(o["mse_trace"])[0] for o in outs])
+    assert np.all(final <= start)
+    assert np.mean(final < start) > 0.5
+
+
+def test_solve_is_deterministic():
+    wl = synth.WORKLOADS["llama31_8b_nvfp4_g16"]
+    fl = dq.format_preset(wl.fmt, wl.group)
+    Ws = [synth.weight(wl, 0, i, device="cuda", rows=512, cols=1024) for i in range(3)]
+    o1 = dq.solve_dual_scale_batched(Ws, fl, 3)
+    o2 = dq.solve_dual_scale_batched(Ws, fl, 3)
+    torch.cuda.synchronize()
+    for x, y in zip(o1, o2):
+        for k in ("codes", "gscales", "a", "b", "mse_trace"):
+            assert torch.equal(x[k], y[k]), k
+
+
+# --------------------------------------------------------------------------- #
+# Edge cases and device status
+# --------------------------------------------------------------------------- #
+
+def test_empty_and_degenerate_shapes():
+    fl = dq.format_preset("mxfp4")
+    W = torch.zeros(0, 64, dtype=torch.bfloat16, device="cuda")
+    o = dq.solve_dual_scale(W, fl, 2)
+    torch.cuda.synchronize()
+    assert o["a"].numel() == 0
+    # all-zero matrix: scales stay 1, codes 0, mse 0
+    Z = torch.zeros(40, 96, dtype=torch.bfloat16, device="cuda")
+    o = dq.solve_dual_scale(Z, fl, 3)
+    torch.cuda.synchronize()
+    assert torch.all(o["a"] == 1) and torch.all(o["b"] == 1)
+    assert torch.all(o["codes"] == 0) and torch.all(o["mse_trace"] == 0)
+    assert torch.all(o["gscales"] == 127)
+    # one group wide, one row tall
+    W = _weights(1, 32, torch.bfloat16).cuda()
+    o = dq.solve_dual_scale(W, fl, 2)
+    torch.cuda.synchronize()
+    r = O.solve(np64(W), O.preset("mxfp4"), 2)
+    assert np.allclose(np64(o["mse_trace"]), r["mse_trace"], rtol=1e-4, atol=0)
+    assert dq.last_device_status() == 0
+
+
+@pytest.mark.parametrize("bad", [float("nan"), float("inf")])
+def test_nonfinite_input_sets_device_flag(bad):
+    fl = dq.format_preset("int4_bf16")
+    W = _weights(64, 128, torch.bfloat16).cuda()
+    W[3, 17] = bad
+    assert dq.last_device_status() == 0
+    dq.solve_dual_scale(W, fl, 1)
+    assert dq.last_device_status() == -4
+    assert dq.last_device_status() == 0      # read clears
+    dq.quantize(W, fl)
+    assert dq.last_device_status() == -4
