@@ -17,7 +17,7 @@ __all__ = [
     "DqError", "dq_format", "dq_matrix", "lib", "library_path", "version", "format_preset",
     "workspace_size", "quantize", "dequantize", "solve_dual_scale", "solve_dual_scale_batched",
     "row_update", "col_update", "act_rescale_quant", "last_device_status", "EXPORTS",
-    "kernel_timing", "kernel_time", "launch_count",
+    "kernel_timing", "kernel_time", "launch_count", "solve_dual_scale_noalloc",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -31,7 +31,8 @@ DQ_OK, DQ_ERR_NONFINITE, DQ_ERR_RANGE = 0, -4, -5
 EXPORTS = ("dq_version", "dq_strerror", "dq_format_preset", "dq_workspace_size", "dq_quantize",
            "dq_dequantize", "dq_solve_dual_scale", "dq_solve_dual_scale_batched",
            "dq_row_update", "dq_col_update", "dq_act_rescale_quant", "dq_last_device_status",
-           "dq_kernel_timing", "dq_kernel_time", "dq_launch_count")
+           "dq_kernel_timing", "dq_kernel_time", "dq_launch_count",
+           "dq_solve_dual_scale_noalloc")
 
 
 class DqError(RuntimeError):
@@ -100,6 +101,10 @@ def lib() -> ctypes.CDLL:
         "dq_kernel_timing": (c_int32, [c_int32]),
         "dq_kernel_time": (c_int32, [c_int32, P(c_double), P(c_int64)]),
         "dq_launch_count": (c_int64, []),
+        "dq_solve_dual_scale_noalloc": (c_int32, [c_void_p, c_int32, c_int64, c_int64,
+                                                  P(dq_format), c_int32, c_void_p, c_void_p,
+                                                  c_void_p, c_void_p, c_void_p, c_void_p,
+                                                  c_void_p, c_void_p, c_void_p, c_void_p]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -220,6 +225,32 @@ def solve_dual_scale(W, fmt, T, a0=None, b0=None, ws=None, half=True, stream=Non
                                      _ptr(a0), _ptr(b0), _ptr(codes), _ptr(gscales), _ptr(a),
                                      _ptr(b), _ptr(ts), _ptr(trace), _ptr(mhalf), _ptr(ws),
                                      ws.numel(), _stream(stream)), "dq_solve_dual_scale")
+    return dict(codes=codes, gscales=gscales, a=a, b=b, tensor_scale=ts, mse_trace=trace,
+                mse_half=mhalf[:T] if half else None)
+
+
+NOALLOC_SCRATCH_BYTES = 32 << 20
+
+
+def solve_dual_scale_noalloc(W, fmt, T, a0=None, b0=None, half=True, stream=None):
+    """The solve of ``solve_dual_scale`` without a workspace: for callers that
+    cannot allocate device scratch (the library keeps a 32 MiB buffer per
+    device for it; concurrent calls on one device race).  Outputs are
+    allocated here with torch; pass them to the C call yourself to avoid that."""
+    _need_cuda(W, a0, b0)
+    rows, cols = W.shape
+    dev = W.device
+    codes, gscales = _outputs(rows, cols, fmt, dev)
+    a = torch.empty(rows, dtype=torch.float32, device=dev)
+    b = torch.empty(cols, dtype=torch.float32, device=dev)
+    ts = torch.empty(1, dtype=torch.float32, device=dev)
+    trace = torch.empty(T + 1, dtype=torch.float64, device=dev)
+    mhalf = torch.empty(max(T, 1), dtype=torch.float64, device=dev) if half else None
+    _check(lib().dq_solve_dual_scale_noalloc(_ptr(W), _dtype_code(W), rows, cols,
+                                             ctypes.byref(fmt), T, _ptr(a0), _ptr(b0),
+                                             _ptr(codes), _ptr(gscales), _ptr(a), _ptr(b),
+                                             _ptr(ts), _ptr(trace), _ptr(mhalf), _stream(stream)),
+           "dq_solve_dual_scale_noalloc")
     return dict(codes=codes, gscales=gscales, a=a, b=b, tensor_scale=ts, mse_trace=trace,
                 mse_half=mhalf[:T] if half else None)
 

@@ -494,6 +494,9 @@ const char *dq_strerror(dq_status s) {
         case DQ_ERR_WORKSPACE: return "workspace missing or too small";
         case DQ_ERR_NOT_IMPLEMENTED: return "not implemented";
         case DQ_ERR_ALIGN: return "pointer alignment";
+        case DQ_ERR_SCRATCH:
+            return "matrix needs more scratch than the built-in 32 MiB buffer of "
+                   "dq_solve_dual_scale_noalloc holds";
     }
     return "unknown status";
 }
@@ -705,3 +708,134 @@ dq_status dq_kernel_time(int32_t kind, double *ms, int64_t *launches) {
 int64_t dq_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------------- //
+// Solve without any allocation: scratch in a built-in device buffer
+// ------------------------------------------------------------------------- //
+//
+// For callers that cannot allocate device memory.  The per-tile partial sums
+// that dq_solve_dual_scale keeps in the caller's workspace live here in one
+// static buffer per device (held for the life of the process).  In host code
+// the array's name is only a host-side stand-in: its device address comes
+// from cudaGetSymbolAddress, looked up once per device with that device
+// current (the first call on a device does this, so it should come before
+// any stream capture).  Calls that overlap on the GPU share the buffer and
+// race.  The only region that must start at zero (the amax word of the
+// tensor-scale pass) is cleared by the solve sequence itself.
+
+namespace {
+
+static __device__ __align__(256) unsigned char g_dq_noalloc_scratch[DQ_NOALLOC_SCRATCH_BYTES];
+
+unsigned char *g_scratch_ptr[kMaxDevices];
+cudaError_t g_scratch_err[kMaxDevices];
+std::once_flag g_scratch_once[kMaxDevices];
+
+// Device address of the scratch buffer on the current device, or NULL.
+unsigned char *noalloc_scratch() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::call_once(g_scratch_once[dev], [dev]() {
+        void *p = nullptr;
+        g_scratch_err[dev] = cudaGetSymbolAddress(&p, g_dq_noalloc_scratch);
+        g_scratch_ptr[dev] = (g_scratch_err[dev] == cudaSuccess)
+                                 ? static_cast<unsigned char *>(p) : nullptr;
+    });
+    return g_scratch_ptr[dev];
+}
+
+}  // namespace
+
+extern "C" dq_status dq_solve_dual_scale_noalloc(const void *W, int32_t dtype, int64_t rows,
+                                                 int64_t cols, const dq_format *fmt, int32_t T,
+                                                 const float *a0, const float *b0,
+                                                 uint8_t *codes, void *gscales, float *a,
+                                                 float *b, float *tensor_scale,
+                                                 double *mse_trace, double *mse_half,
+                                                 dq_stream stream) {
+    if (T < 0) return DQ_ERR_ARG;
+    if (dtype != DQ_DT_F32 && dtype != DQ_DT_BF16) return DQ_ERR_ARG;
+    FmtInfo fi;
+    dq_status s = check_format(fmt, &fi);
+    if (s != DQ_OK) return s;
+    if (rows < 0 || cols < 0 || cols % fi.G) return DQ_ERR_SHAPE;
+    const bool f32 = dtype == DQ_DT_F32;
+    const bool empty = rows == 0 || cols == 0;
+    if (!empty && (!W || !codes || !gscales)) return DQ_ERR_ARG;
+    if (!a || !b || !tensor_scale) return DQ_ERR_ARG;
+    if (!aligned(W, 16) || !aligned(codes, 16) || !aligned(gscales, 16)) return DQ_ERR_ALIGN;
+    if (!aligned(a, 4) || !aligned(b, 4) || !aligned(tensor_scale, 4)) return DQ_ERR_ALIGN;
+    if (!aligned(a0, 4) || !aligned(b0, 4)) return DQ_ERR_ALIGN;
+    if (!aligned(mse_trace, 8) || !aligned(mse_half, 8)) return DQ_ERR_ALIGN;
+    const size_t need = matrix_ws(rows, cols, f32);
+    if (need > (size_t)DQ_NOALLOC_SCRATCH_BYTES) return DQ_ERR_SCRATCH;
+    unsigned char *scratch = noalloc_scratch();
+    if (!scratch) return DQ_ERR_CUDA;
+    unsigned int *status = status_ptr();
+    if (!status) return DQ_ERR_CUDA;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+
+    // descriptor of the one matrix, on the stack (no table copy)
+    MatDesc d{};
+    d.W = W;
+    d.rows = rows;
+    d.cols = cols;
+    d.a = a;
+    d.b = b;
+    d.a_out = a;
+    d.b_out = b;
+    d.codes = codes;
+    d.gscales = gscales;
+    d.ts_ptr = tensor_scale;
+    d.ts_out = tensor_scale;
+    d.ts_val = 1.0f;
+    d.a0 = a0;
+    d.b0 = b0;
+    d.mse_trace = mse_trace;
+    d.mse_half = mse_half;
+    Carve cv{reinterpret_cast<char *>(scratch),
+             reinterpret_cast<char *>(scratch) + DQ_NOALLOC_SCRATCH_BYTES};
+    int64_t tb[3] = {0, 0, 0}, rb = 0, cb = 0;
+    place(d, f32, cv, tb, rb, cb);
+    Launcher L;
+    L.tab.dev = nullptr;
+    L.tab.one = d;
+    L.tab.n = 1;
+    L.tab.status = status;
+    L.combo = fi.combo;
+    L.G = fi.G;
+    L.f32 = f32;
+    L.qmax = fi.qmax;
+    for (int m = 0; m < 3; ++m) L.tiles[m] = tb[m];
+    L.total_rows = rb;
+    L.total_cols = cb;
+    L.st = st;
+
+    // same launch sequence as dq_solve_dual_scale for one matrix
+    if (fmt->tensor_scale_auto) {
+        DQ_CUDA(cudaMemsetAsync(d.amax, 0, sizeof(unsigned int), st));   // starts at zero
+        if (L.tiles[2] > 0) {
+            if (f32) amax_kernel<float><<<(unsigned)L.tiles[2], kThreads, 0, st>>>(L.tab);
+            else amax_kernel<Bf16Tag><<<(unsigned)L.tiles[2], kThreads, 0, st>>>(L.tab);
+            DQ_CUDA(cudaGetLastError());
+            count_launches(1);
+        }
+    }
+    tensor_scale_kernel<<<1, 128, 0, st>>>(L.tab, fi.qmax, fmt->tensor_scale_auto);
+    DQ_CUDA(cudaGetLastError());
+    count_launches(1);
+    if (rb + cb > 0) {
+        init_state_kernel<<<grid_for(rb + cb, 256), 256, 0, st>>>(L.tab, rb, cb);
+        DQ_CUDA(cudaGetLastError());
+        count_launches(1);
+    }
+    for (int t = 0; t < T; ++t) {
+        if ((s = L.tiles_pass(MODE_ROW)) != DQ_OK) return s;
+        if ((s = L.row_finalize()) != DQ_OK) return s;
+        if ((s = L.tiles_pass(MODE_COL)) != DQ_OK) return s;
+        if ((s = L.col_finalize()) != DQ_OK) return s;
+        if ((s = L.mse(MODE_ROW, t, t, nullptr, nullptr)) != DQ_OK) return s;
+    }
+    if ((s = L.tiles_pass(MODE_PACK)) != DQ_OK) return s;
+    return L.mse(2, T, -1, nullptr, nullptr);
+}

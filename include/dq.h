@@ -64,7 +64,8 @@ typedef enum dq_status {
     DQ_ERR_CUDA = -6,           /* a CUDA runtime call failed */
     DQ_ERR_WORKSPACE = -7,      /* workspace null or smaller than dq_workspace_size */
     DQ_ERR_NOT_IMPLEMENTED = -8,
-    DQ_ERR_ALIGN = -9           /* a pointer misses its alignment */
+    DQ_ERR_ALIGN = -9,          /* a pointer misses its alignment */
+    DQ_ERR_SCRATCH = -10        /* matrix needs more than the built-in scratch buffer */
 } dq_status;
 
 enum { DQ_CODES_INT4 = 0, DQ_CODES_E2M1 = 1 };
@@ -197,6 +198,33 @@ DQ_API dq_status dq_act_rescale_quant(const void *X, int64_t tokens, int64_t K, 
  * otherwise (NONFINITE wins when both are set).  The flags are one word per
  * device shared by all streams. */
 DQ_API dq_status dq_last_device_status(dq_stream stream);
+
+/* Variant of dq_solve_dual_scale for callers that cannot allocate device
+ * memory: code that runs inside another framework's memory pool or under a
+ * strict memory budget, plug-ins that may not call cudaMalloc, or C hosts
+ * without a device allocator at hand.  It takes no workspace argument; its
+ * per-tile partial sums live in one scratch buffer of DQ_NOALLOC_SCRATCH_BYTES
+ * (32 MiB) built into the library, which every GPU that loads the library
+ * holds until the process exits.  The paper has no counterpart of this call.
+ *  - The first call on a device looks up the buffer's device address with
+ *    that device current (cudaGetSymbolAddress); make that first call before
+ *    any stream capture.
+ *  - A matrix whose scratch need exceeds the buffer is refused with
+ *    DQ_ERR_SCRATCH (dq_workspace_size gives the need: 8192 x 28672 bf16
+ *    fits, for example).
+ *  - Every call shares the one buffer per device: calls that overlap on the
+ *    GPU (on different streams, or from several host threads) race and give
+ *    wrong results; serialise them.  The buffer keeps the last call's
+ *    contents; the call clears what it needs to start at zero.
+ *  - Allocates nothing (no cudaMalloc, cudaFree or allocating library call).
+ * Arguments, outputs and errors as dq_solve_dual_scale. */
+#define DQ_NOALLOC_SCRATCH_BYTES (32u << 20)
+DQ_API dq_status dq_solve_dual_scale_noalloc(const void *W, int32_t dtype, int64_t rows,
+                                             int64_t cols, const dq_format *fmt, int32_t T,
+                                             const float *a0, const float *b0, uint8_t *codes,
+                                             void *gscales, float *a, float *b,
+                                             float *tensor_scale, double *mse_trace,
+                                             double *mse_half, dq_stream stream);
 
 /* Measurement support (no counterpart in the method).  dq_kernel_timing(1)
  * makes every tile-kernel launch of the library record a CUDA event pair on
