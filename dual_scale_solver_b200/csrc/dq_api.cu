@@ -287,7 +287,7 @@ dq_status solve_impl(int32_t n, const dq_matrix *mats, int32_t dtype, const dq_f
         if (m.cols % fi.G) return DQ_ERR_SHAPE;
         const bool empty = m.rows == 0 || m.cols == 0;
         if (!empty && (!m.W || !m.codes || !m.gscales)) return DQ_ERR_ARG;
-        if (!m.a || !m.b || !m.tensor_scale) return DQ_ERR_ARG;
+        if ((m.rows > 0 && !m.a) || (m.cols > 0 && !m.b) || !m.tensor_scale) return DQ_ERR_ARG;
         if (!aligned(m.W, 16) || !aligned(m.codes, 16) || !aligned(m.gscales, 16)) return DQ_ERR_ALIGN;
         if (!aligned(m.a, 4) || !aligned(m.b, 4) || !aligned(m.tensor_scale, 4)) return DQ_ERR_ALIGN;
         if (!aligned(m.a0, 4) || !aligned(m.b0, 4)) return DQ_ERR_ALIGN;
@@ -762,7 +762,7 @@ extern "C" dq_status dq_solve_dual_scale_noalloc(const void *W, int32_t dtype, i
     const bool f32 = dtype == DQ_DT_F32;
     const bool empty = rows == 0 || cols == 0;
     if (!empty && (!W || !codes || !gscales)) return DQ_ERR_ARG;
-    if (!a || !b || !tensor_scale) return DQ_ERR_ARG;
+    if ((rows > 0 && !a) || (cols > 0 && !b) || !tensor_scale) return DQ_ERR_ARG;
     if (!aligned(W, 16) || !aligned(codes, 16) || !aligned(gscales, 16)) return DQ_ERR_ALIGN;
     if (!aligned(a, 4) || !aligned(b, 4) || !aligned(tensor_scale, 4)) return DQ_ERR_ALIGN;
     if (!aligned(a0, 4) || !aligned(b0, 4)) return DQ_ERR_ALIGN;
