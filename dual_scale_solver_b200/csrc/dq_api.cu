@@ -215,7 +215,7 @@ struct Launcher {
     int64_t total_rows = 0, total_cols = 0;
     cudaStream_t st;
 
-    dq_status tiles_pass(int mode) {
+    dq_status tiles_pass(int mode, bool want_res) {
         TileLaunch L;
         L.tab = tab;
         L.mode = mode;
@@ -223,6 +223,7 @@ struct Launcher {
         L.grid = tiles[L.slot];
         L.f32 = f32 ? 1 : 0;
         L.G = G;
+        L.want_res = want_res ? 1 : 0;
         L.stream = st;
         if (L.grid <= 0) return DQ_OK;
         cudaEvent_t beg = nullptr, end = nullptr;
@@ -361,14 +362,19 @@ dq_status solve_impl(int32_t n, const dq_matrix *mats, int32_t dtype, const dq_f
         DQ_CUDA(cudaGetLastError());
         count_launches(1);
     }
+    bool want_trace = false, want_half = false;
+    for (int i = 0; i < n; ++i) {
+        want_trace |= mats[i].mse_trace != nullptr;
+        want_half |= mats[i].mse_half != nullptr;
+    }
     for (int t = 0; t < T; ++t) {
-        if ((s = L.tiles_pass(MODE_ROW)) != DQ_OK) return s;
+        if ((s = L.tiles_pass(MODE_ROW, want_trace)) != DQ_OK) return s;
         if ((s = L.row_finalize()) != DQ_OK) return s;
-        if ((s = L.tiles_pass(MODE_COL)) != DQ_OK) return s;
+        if ((s = L.tiles_pass(MODE_COL, want_half)) != DQ_OK) return s;
         if ((s = L.col_finalize()) != DQ_OK) return s;
         if ((s = L.mse(MODE_ROW, t, t, nullptr, nullptr)) != DQ_OK) return s;
     }
-    if ((s = L.tiles_pass(MODE_PACK)) != DQ_OK) return s;
+    if ((s = L.tiles_pass(MODE_PACK, want_trace)) != DQ_OK) return s;
     if ((s = L.mse(2, T, -1, nullptr, nullptr)) != DQ_OK) return s;
     return DQ_OK;
 }
@@ -401,6 +407,7 @@ dq_status step_impl(bool row_step, const void *W, int32_t dtype, int64_t rows, i
     if (s != DQ_OK) return s;
     if (!a_in || !b_in || !out) return DQ_ERR_ARG;
     if (!(ts > 0.0f)) return DQ_ERR_ARG;
+    if (fmt->group_scale != DQ_SCALE_E4M3 && ts != 1.0f) return DQ_ERR_ARG;
     if (!aligned(a_in, 4) || !aligned(b_in, 4) || !aligned(out, 4) || !aligned(pre, 4) ||
         !aligned(mse_in, 8))
         return DQ_ERR_ALIGN;
@@ -431,11 +438,11 @@ dq_status step_impl(bool row_step, const void *W, int32_t dtype, int64_t rows, i
     L.total_cols = cb;
     L.st = st;
     if (row_step) {
-        if ((s = L.tiles_pass(MODE_ROW)) != DQ_OK) return s;
+        if ((s = L.tiles_pass(MODE_ROW, mse_in != nullptr)) != DQ_OK) return s;
         if ((s = L.row_finalize()) != DQ_OK) return s;
         if (mse_in) return L.mse(MODE_ROW, -1, -1, mse_in, nullptr);
     } else {
-        if ((s = L.tiles_pass(MODE_COL)) != DQ_OK) return s;
+        if ((s = L.tiles_pass(MODE_COL, mse_in != nullptr)) != DQ_OK) return s;
         if ((s = L.col_finalize()) != DQ_OK) return s;
         if (mse_in) return L.mse(-1, -1, -1, nullptr, mse_in);
     }
@@ -542,6 +549,7 @@ dq_status dq_quantize(const void *X, int32_t dtype, int64_t rows, int64_t cols,
     if (rows == 0 || cols == 0) return DQ_OK;
     if (!codes || !gscales) return DQ_ERR_ARG;
     if (!(tensor_scale > 0.0f)) return DQ_ERR_ARG;
+    if (fmt->group_scale != DQ_SCALE_E4M3 && tensor_scale != 1.0f) return DQ_ERR_ARG;
     if (!aligned(codes, 16) || !aligned(gscales, 16) || !aligned(a, 4) || !aligned(b, 4))
         return DQ_ERR_ALIGN;
     unsigned int *status = status_ptr();
@@ -566,7 +574,7 @@ dq_status dq_quantize(const void *X, int32_t dtype, int64_t rows, int64_t cols,
     L.qmax = fi.qmax;
     for (int m = 0; m < 3; ++m) L.tiles[m] = tb[m];
     L.st = reinterpret_cast<cudaStream_t>(stream);
-    return L.tiles_pass(MODE_PACK);
+    return L.tiles_pass(MODE_PACK, false);
 }
 
 dq_status dq_act_rescale_quant(const void *X, int64_t tokens, int64_t K, const float *b,
@@ -598,7 +606,7 @@ dq_status dq_act_rescale_quant(const void *X, int64_t tokens, int64_t K, const f
     L.qmax = fi.qmax;
     for (int m = 0; m < 3; ++m) L.tiles[m] = tb[m];
     L.st = reinterpret_cast<cudaStream_t>(stream);
-    return L.tiles_pass(MODE_ACT);
+    return L.tiles_pass(MODE_ACT, false);
 }
 
 dq_status dq_dequantize(const uint8_t *codes, const void *gscales, int64_t rows, int64_t cols,
@@ -830,12 +838,12 @@ extern "C" dq_status dq_solve_dual_scale_noalloc(const void *W, int32_t dtype, i
         count_launches(1);
     }
     for (int t = 0; t < T; ++t) {
-        if ((s = L.tiles_pass(MODE_ROW)) != DQ_OK) return s;
+        if ((s = L.tiles_pass(MODE_ROW, mse_trace != nullptr)) != DQ_OK) return s;
         if ((s = L.row_finalize()) != DQ_OK) return s;
-        if ((s = L.tiles_pass(MODE_COL)) != DQ_OK) return s;
+        if ((s = L.tiles_pass(MODE_COL, mse_half != nullptr)) != DQ_OK) return s;
         if ((s = L.col_finalize()) != DQ_OK) return s;
         if ((s = L.mse(MODE_ROW, t, t, nullptr, nullptr)) != DQ_OK) return s;
     }
-    if ((s = L.tiles_pass(MODE_PACK)) != DQ_OK) return s;
+    if ((s = L.tiles_pass(MODE_PACK, mse_trace != nullptr)) != DQ_OK) return s;
     return L.mse(2, T, -1, nullptr, nullptr);
 }

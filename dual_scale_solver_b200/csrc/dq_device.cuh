@@ -32,6 +32,7 @@ enum { STATUS_NONFINITE = 1u, STATUS_RANGE = 2u };
 constexpr int kWarps = 8;            // warps per CTA of the tile kernel
 constexpr int kThreads = 32 * kWarps;
 constexpr int kRowsPerWarp[4] = {16, 64, 16, 16};   // per mode
+constexpr int kRing = 4;             // cp.async ring slots per lane (rows in flight + 1)
 constexpr float kBf16Max = 3.38953138925153547590470800371487866880e+38f;  // (2-2^-7)*2^127
 constexpr float kMinNormal = 1.17549435082228750796873653722224568e-38f;    // 2^-126
 
@@ -115,6 +116,31 @@ __device__ __forceinline__ float2 e2m1x2_to_f32(uint32_t byte) {  // .x = low ni
     asm("{ .reg .f16 l, h; mov.b32 {l, h}, %2; cvt.f32.f16 %0, l; cvt.f32.f16 %1, h; }"
         : "=f"(lo), "=f"(hi) : "r"(h2));
     return make_float2(lo, hi);
+}
+// Round a pair to E2M1 (nearest even, saturating) and return the code values
+// as float32 (.x from lo, .y from hi), optionally with the code byte.
+__device__ __forceinline__ float2 e2m1_round2(float lo, float hi) {
+    float a, b;
+    asm("{ .reg .b8 t; .reg .b32 p; .reg .f16 l, h;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 t, %3, %2;\n\t"
+        "cvt.rn.f16x2.e2m1x2 p, t;\n\t"
+        "mov.b32 {l, h}, p;\n\t"
+        "cvt.f32.f16 %0, l;\n\t"
+        "cvt.f32.f16 %1, h; }"
+        : "=f"(a), "=f"(b) : "f"(lo), "f"(hi));
+    return make_float2(a, b);
+}
+__device__ __forceinline__ float2 e2m1_round2_byte(float lo, float hi, uint32_t &byte) {
+    float a, b;
+    asm("{ .reg .b8 t; .reg .b32 p; .reg .f16 l, h;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 t, %4, %3;\n\t"
+        "cvt.u32.u8 %2, t;\n\t"
+        "cvt.rn.f16x2.e2m1x2 p, t;\n\t"
+        "mov.b32 {l, h}, p;\n\t"
+        "cvt.f32.f16 %0, l;\n\t"
+        "cvt.f32.f16 %1, h; }"
+        : "=f"(a), "=f"(b), "=r"(byte) : "f"(lo), "f"(hi));
+    return make_float2(a, b);
 }
 __device__ __forceinline__ uint32_t e4m3_bits(float x) {    // x exactly representable
     uint16_t r;
@@ -229,151 +255,192 @@ __device__ __forceinline__ ScaleChoice project_group(float m, float qts, float r
 }
 
 // ------------------------------------------------------------------------- //
-// Quantization of one lane's chunk of EPC consecutive elements of one row
+// Packed float32x2 helpers (sm_100 FFMA2 / FMUL2)
 // ------------------------------------------------------------------------- //
 
-template <int CODES, int GS, int OS, bool ACT, int EPC, int LPG>
+typedef float2 f2;
+__device__ __forceinline__ f2 mul2(f2 a, f2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ f2 fma2(f2 a, f2 b, f2 c) { return __ffma2_rn(a, b, c); }
+__device__ __forceinline__ f2 bcast(float v) { return make_float2(v, v); }
+__device__ __forceinline__ f2 neg2(f2 v) { return make_float2(-v.x, -v.y); }
+__device__ __forceinline__ float max3_nan(float a, float b, float c) {
+    float r;
+    asm("max.NaN.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+// ------------------------------------------------------------------------- //
+// Quantization of one lane's chunk: NP pairs of consecutive elements of a row
+// ------------------------------------------------------------------------- //
+
+template <int CODES, int GS, int OS, bool ACT, int NP, int LPG>
 struct Quant {
+    // a second-level tensor scale exists only with E4M3 group scales (NVFP4)
+    static constexpr bool kHasTs = GS == SC_E4M3;
     // exact fast path: all scalings are powers of two
     static constexpr bool kExactQ = ACT ? (GS == SC_E8M0) : (GS == SC_E8M0 && OS == SC_E8M0);
-    // exact group max (inner scaling by b, and by a, exact)
+    // exact group max (the inner scaling by b, and by a, is exact)
     static constexpr bool kExactM = ACT ? true : (OS == SC_E8M0);
     static constexpr float kQmax = CODES == CODES_INT4 ? 7.0f : 6.0f;
 
     // In: w (input values), z = inner-scaled values before the row factor
-    // (w*ib_j for weights, x*b_j for activations), ab = a*b_j (weights, only
-    // read on the exact path), ia = 1/a (weights; 1 for ACT), ts.
-    // Out: c (code values), s (stored group scale), s_eff = s*ts, nib (packed
-    // nibbles of the chunk, element 0 in the low nibble).
-    __device__ __forceinline__ static void run(const float (&w)[EPC], const float (&z)[EPC],
-                                               const float (&ab)[EPC], float ia, float ts,
-                                               float inv_ts, unsigned int *status,
-                                               float (&c)[EPC], float &s, float &s_eff,
-                                               uint32_t &nib) {
-        const float qts = kQmax * ts;
-        const float rqts = 1.0f / qts;
-        // group max of |y|, y = z * ia
+    // (w/b_j for weights, x*b_j for activations), a and ia = 1/a (1 for ACT),
+    // bj (b_j; read on the exact path only), ts and 1/ts (E4M3 only).
+    // Out: c (code values), s (stored group scale), s_eff = s*ts, nib (the
+    // chunk's packed nibbles, element 0 lowest; only when NIB).
+    template <bool NIB>
+    __device__ __forceinline__ static void run(const f2 (&w)[NP], const f2 (&z)[NP], float a,
+                                               float ia, const f2 (&bj)[NP], float ts,
+                                               float inv_ts, unsigned int *status, f2 (&c)[NP],
+                                               float &s, float &s_eff, uint32_t &nib) {
         float mz = 0.0f;
 #pragma unroll
-        for (int j = 0; j < EPC; ++j) mz = max_nan(mz, fabsf(z[j]));
+        for (int k = 0; k < NP; ++k) mz = max3_nan(mz, fabsf(z[k].x), fabsf(z[k].y));
         mz = grp_max<LPG>(mz);
-        float m = mz * ia;
-        const bool finite = isfinite(m);
-        if (!finite) atomicOr(status, STATUS_NONFINITE);
-        // every lane takes part in the warp votes and group shuffles below,
-        // whatever its group holds (all-zero and out-of-range groups included)
-        const bool pos = finite && (m > 0.0f);
-        ScaleChoice sc = project_group<GS, CODES>(pos ? m : 1.0f, qts, rqts, inv_ts);
-        s = sc.s;
-        const bool resolve = pos && ((GS == SC_E8M0 && kExactM) ? false : sc.near);
-        if (__any_sync(0xffffffffu, resolve)) {
-            // exact comparison of the true group max with sc.thr
-            int gt = 0, eq = 0;
-            if (resolve) {
-                if (kExactM) {
-                    float d = m - sc.thr;                       // both exact: sign exact
-                    gt = d > 0.0f;
-                    eq = d == 0.0f;
-                } else {
-#pragma unroll
-                    for (int j = 0; j < EPC; ++j) {
-                        float d = fmaf(-sc.thr, ab[j], fabsf(w[j]));
-                        gt |= d > 0.0f;
-                        eq |= d == 0.0f;
-                    }
-                }
-            }
-            if (!kExactM) {
-                gt = grp_or<LPG>(gt);
-                eq = grp_or<LPG>(eq);
-            }
-            if (resolve) s = gt ? sc.s_hi : (eq ? sc.s_tie : sc.s_lo);
-        }
-        if (!pos) s = 1.0f;
-        s_eff = s * ts;
-        // code decisions on q = y / s_eff
-        const float r = ia * ((GS == SC_E8M0) ? recip_pow2(s_eff) : recip_approx(s_eff));
-        float q[EPC];
-#pragma unroll
-        for (int j = 0; j < EPC; ++j) q[j] = z[j] * r;
-        if (CODES == CODES_INT4) {
-            nib = 0;
-            bool anynear = false;
-            bool nr[EPC];
-#pragma unroll
-            for (int j = 0; j < EPC; ++j) {
-                float rq = rintf(q[j]);
-                nr[j] = !kExactQ && (fabsf(q[j] - rq) > 0.5f - 1.52587890625e-05f);  // 2^-16
-                anynear |= nr[j];
-                c[j] = fminf(fmaxf(rq, -8.0f), 7.0f);
-            }
-            if (!kExactQ && anynear) {
-#pragma unroll
-                for (int j = 0; j < EPC; ++j) {
-                    if (nr[j]) {
-                        float aq = fabsf(q[j]);
-                        float lo = floorf(aq);
-                        float mid = lo + 0.5f;
-                        float d = ACT ? fmaf(-mid, s_eff, fabsf(z[j]))
-                                      : fmaf(-mid, ab[j] * s_eff, fabsf(w[j]));
-                        float mag = d > 0.0f ? lo + 1.0f
-                                  : (d < 0.0f ? lo : ((((int)lo) & 1) ? lo + 1.0f : lo));
-                        c[j] = fminf(fmaxf(copysignf(mag, q[j]), -8.0f), 7.0f);
-                    }
-                }
-            }
-#pragma unroll
-            for (int j = 0; j < EPC; ++j) nib |= ((uint32_t)((int)c[j]) & 0xFu) << (4 * j);
+        const float m = ACT ? mz : mz * ia;
+        const uint32_t mb = __float_as_uint(m);
+        const bool finite = (mb & 0x7F800000u) != 0x7F800000u;
+        // row and column statistics carry a NaN/Inf into their sums, which the
+        // finalize kernels flag; the other modes flag it here
+        if (NIB && !finite) atomicOr(status, STATUS_NONFINITE);
+        const bool pos = finite && m > 0.0f;
+        if (GS == SC_E8M0 && kExactM) {
+            // smallest 2^e with qmax 2^e >= m (m exact): e = E(m) - 2, plus 1
+            // when m's significand exceeds qmax/4 (1.75 INT4, 1.5 E2M1);
+            // e >= -126 (also covers subnormal m); e <= 126 holds for finite m
+            constexpr uint32_t MT = (CODES == CODES_INT4) ? 0x600000u : 0x400000u;
+            const int e = max((int)(mb >> 23) - 129 + (((mb & 0x7FFFFFu) > MT) ? 1 : 0), -126);
+            s = pow2f(e);
+            if (NIB && !pos) s = 1.0f;                     // stored scale of an all-zero group
         } else {
-            uint32_t byte[EPC / 2];
+            // every lane takes part in the warp vote and group shuffles below,
+            // whatever its group holds (all-zero and out-of-range groups too)
+            const float qts = kHasTs ? kQmax * ts : kQmax;
+            const float rqts = kHasTs ? 1.0f / qts : 1.0f / kQmax;
+            ScaleChoice sc = project_group<GS, CODES>(pos ? m : 1.0f, qts, rqts,
+                                                      kHasTs ? inv_ts : 1.0f);
+            s = sc.s;
+            const bool resolve = pos && sc.near;
+            if (__any_sync(0xffffffffu, resolve)) {
+                // exact comparison of the true group max with sc.thr
+                int gt = 0, eq = 0;
+                if (resolve) {
+                    if (kExactM) {
+                        const float d = m - sc.thr;              // both exact: sign exact
+                        gt = d > 0.0f;
+                        eq = d == 0.0f;
+                    } else {
 #pragma unroll
-            for (int j = 0; j < EPC; j += 2) byte[j / 2] = cvt_e2m1x2(q[j + 1], q[j]);
+                        for (int k = 0; k < NP; ++k) {
+                            const float d0 = fmaf(-sc.thr, a * bj[k].x, fabsf(w[k].x));
+                            const float d1 = fmaf(-sc.thr, a * bj[k].y, fabsf(w[k].y));
+                            gt |= (d0 > 0.0f) | (d1 > 0.0f);
+                            eq |= (d0 == 0.0f) | (d1 == 0.0f);
+                        }
+                    }
+                }
+                if (!kExactM) {
+                    gt = grp_or<LPG>(gt);
+                    eq = grp_or<LPG>(eq);
+                }
+                if (resolve) s = gt ? sc.s_hi : (eq ? sc.s_tie : sc.s_lo);
+            }
+            if (!pos) s = 1.0f;
+        }
+        s_eff = kHasTs ? s * ts : s;
+        const float r = (GS == SC_E8M0) ? (ACT ? recip_pow2(s_eff) : ia * recip_pow2(s_eff))
+                                        : (ACT ? recip_approx(s_eff) : ia * recip_approx(s_eff));
+        f2 q[NP];
+#pragma unroll
+        for (int k = 0; k < NP; ++k) q[k] = mul2(z[k], bcast(r));
+        nib = 0;
+        if (CODES == CODES_INT4) {
+            // round half to even; |q| <= 7 (E8M0 round-up) or < 7.5 (BF16
+            // nearest) so the codebook clamp never binds for these sets
+#pragma unroll
+            for (int k = 0; k < NP; ++k) c[k] = make_float2(rintf(q[k].x), rintf(q[k].y));
             if (!kExactQ) {
-                const float up = 1.0f + 7.62939453125e-06f, dn = 1.0f - 7.62939453125e-06f;  // 2^-17
+                bool any = false;
 #pragma unroll
-                for (int j = 0; j < EPC; j += 2) {
-                    uint32_t bh = cvt_e2m1x2(q[j + 1] * up, q[j] * up);
-                    uint32_t bl = cvt_e2m1x2(q[j + 1] * dn, q[j] * dn);
-                    if (bh != bl) {
+                for (int k = 0; k < NP; ++k)
+                    any |= (fabsf(q[k].x - c[k].x) > 0.5f - 1.52587890625e-05f) |
+                           (fabsf(q[k].y - c[k].y) > 0.5f - 1.52587890625e-05f);   // 2^-16
+                if (any) {
+#pragma unroll
+                    for (int k = 0; k < NP; ++k)
 #pragma unroll
                         for (int h = 0; h < 2; ++h) {
-                            uint32_t nh = (bh >> (4 * h)) & 0xF, nl = (bl >> (4 * h)) & 0xF;
-                            if (nh != nl) {
-                                int jj = j + h;
-                                float2 vh = e2m1x2_to_f32(nh), vl = e2m1x2_to_f32(nl);
-                                float mh = fabsf(vh.x), ml = fabsf(vl.x);
-                                float mid = 0.5f * (mh + ml);
-                                float d = ACT ? fmaf(-mid, s_eff, fabsf(z[jj]))
-                                              : fmaf(-mid, ab[jj] * s_eff, fabsf(w[jj]));
-                                // the even code of the two neighbours has mantissa bit 0
-                                float even = ((nh & 1u) == 0) ? mh : ml;
-                                float mag = d > 0.0f ? mh : (d < 0.0f ? ml : even);
-                                uint32_t nn = cvt_e2m1x2(0.0f, copysignf(mag, q[jj])) & 0xF;
-                                byte[j / 2] = (byte[j / 2] & ~(0xFu << (4 * h))) | (nn << (4 * h));
+                            const float qq = h ? q[k].y : q[k].x;
+                            const float cc = h ? c[k].y : c[k].x;
+                            if (fabsf(qq - cc) > 0.5f - 1.52587890625e-05f) {
+                                const float aq = fabsf(qq), lo = floorf(aq), mid = lo + 0.5f;
+                                const float ww = h ? w[k].y : w[k].x, zz = h ? z[k].y : z[k].x;
+                                const float bb = h ? bj[k].y : bj[k].x;
+                                const float d = ACT ? fmaf(-mid, s_eff, fabsf(zz))
+                                                    : fmaf(-mid, (a * bb) * s_eff, fabsf(ww));
+                                const float mag = d > 0.0f ? lo + 1.0f
+                                                : (d < 0.0f ? lo : ((((int)lo) & 1) ? lo + 1.0f : lo));
+                                const float v = copysignf(mag, qq);
+                                if (h) c[k].y = v; else c[k].x = v;
+                            }
+                        }
+                }
+            }
+            if (NIB) {
+#pragma unroll
+                for (int k = 0; k < NP; ++k)
+                    nib |= ((((uint32_t)(int)c[k].x) & 0xFu) | ((((uint32_t)(int)c[k].y) & 0xFu) << 4))
+                           << (8 * k);
+            }
+        } else {
+            if (kExactQ && !NIB) {
+#pragma unroll
+                for (int k = 0; k < NP; ++k) c[k] = e2m1_round2(q[k].x, q[k].y);
+            } else {
+                uint32_t byte[NP];
+#pragma unroll
+                for (int k = 0; k < NP; ++k) c[k] = e2m1_round2_byte(q[k].x, q[k].y, byte[k]);
+                if (!kExactQ) {
+                    const f2 up = bcast(1.0f + 7.62939453125e-06f), dn = bcast(1.0f - 7.62939453125e-06f);
+#pragma unroll
+                    for (int k = 0; k < NP; ++k) {
+                        const f2 qh = mul2(q[k], up), ql = mul2(q[k], dn);
+                        const uint32_t bh = cvt_e2m1x2(qh.y, qh.x), bl = cvt_e2m1x2(ql.y, ql.x);
+                        if (bh != bl) {
+#pragma unroll
+                            for (int h = 0; h < 2; ++h) {
+                                const uint32_t nh = (bh >> (4 * h)) & 0xF, nl = (bl >> (4 * h)) & 0xF;
+                                if (nh != nl) {
+                                    const float2 vh = e2m1x2_to_f32(nh), vl = e2m1x2_to_f32(nl);
+                                    const float mh = fabsf(vh.x), ml = fabsf(vl.x);
+                                    const float mid = 0.5f * (mh + ml);
+                                    const float ww = h ? w[k].y : w[k].x, zz = h ? z[k].y : z[k].x;
+                                    const float bb = h ? bj[k].y : bj[k].x, qq = h ? q[k].y : q[k].x;
+                                    const float d = ACT ? fmaf(-mid, s_eff, fabsf(zz))
+                                                        : fmaf(-mid, (a * bb) * s_eff, fabsf(ww));
+                                    // the even code of the two neighbours has mantissa bit 0
+                                    const float even = ((nh & 1u) == 0) ? mh : ml;
+                                    const float mag = d > 0.0f ? mh : (d < 0.0f ? ml : even);
+                                    const float v = copysignf(mag, qq);
+                                    const uint32_t nn = cvt_e2m1x2(0.0f, v) & 0xF;
+                                    byte[k] = (byte[k] & ~(0xFu << (4 * h))) | (nn << (4 * h));
+                                    if (h) c[k].y = v; else c[k].x = v;
+                                }
                             }
                         }
                     }
                 }
-            }
-            nib = 0;
+                if (NIB) {
 #pragma unroll
-            for (int j = 0; j < EPC; j += 2) {
-                // sign of the code follows the sign bit of q (also for a zero result)
-                uint32_t bb = byte[j / 2];
-                bb |= (__float_as_uint(q[j]) >> 31) << 3;
-                bb |= (__float_as_uint(q[j + 1]) >> 31) << 7;
-                byte[j / 2] = bb;
-                float2 v = e2m1x2_to_f32(bb);
-                c[j] = v.x;
-                c[j + 1] = v.y;
-                nib |= bb << (4 * j);
+                    for (int k = 0; k < NP; ++k) nib |= byte[k] << (8 * k);
+                }
             }
         }
     }
 };
 
 // ------------------------------------------------------------------------- //
-// Loading one lane's chunk
+// Loading one lane's chunk (16 bytes)
 // ------------------------------------------------------------------------- //
 
 template <typename TIn> struct Chunk;
@@ -387,6 +454,10 @@ template <> struct Chunk<float> {
     __device__ __forceinline__ void unpack(float (&w)[4]) const {
         w[0] = __uint_as_float(raw.x); w[1] = __uint_as_float(raw.y);
         w[2] = __uint_as_float(raw.z); w[3] = __uint_as_float(raw.w);
+    }
+    __device__ __forceinline__ void unpack2(f2 (&w)[2]) const {
+        w[0] = make_float2(__uint_as_float(raw.x), __uint_as_float(raw.y));
+        w[1] = make_float2(__uint_as_float(raw.z), __uint_as_float(raw.w));
     }
 };
 struct Bf16Tag {};
@@ -404,6 +475,12 @@ template <> struct Chunk<Bf16Tag> {
             w[2 * k] = __uint_as_float(v[k] << 16);
             w[2 * k + 1] = __uint_as_float(v[k] & 0xFFFF0000u);
         }
+    }
+    __device__ __forceinline__ void unpack2(f2 (&w)[4]) const {
+        const uint32_t v[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+            w[k] = make_float2(__uint_as_float(v[k] << 16), __uint_as_float(v[k] & 0xFFFF0000u));
     }
 };
 
@@ -442,27 +519,46 @@ __device__ __forceinline__ float project_outer(float x, bool &clamped) {
 // CTA = 8 warps = wr x wc (wc warps across columns).  Warp (r, c) handles the
 // tile's rows r, r + wr, r + 2 wr, ... of column segment c (32 lanes x EPC
 // columns).  Each lane keeps b_j and 1/b_j of its EPC columns in registers
-// for the whole tile.
+// for the whole tile; arithmetic runs on float32 pairs (FFMA2/FMUL2).
 //   ROW : per row, sum_j W_ij R_ij and sum_j R_ij^2 (R = Qhat D_b) over the
 //         tile's columns -> rowpart[row][cb]; residual of the state -> res_row
 //   COL : per column, sum_i W_ij S_ij and sum_i S_ij^2 (S = D_a Qhat) over the
 //         tile's rows -> colpart[rb][col]; residual -> res_col
 //   PACK: codes and group scales of Q(W / (a b)); residual -> res_row
 //   ACT : codes and group scales of Q(X * b)
+// `want_res` = 0 skips the residual (its MSE output was not requested).
+// Shared memory of one tile CTA, by mode.
+template <int MODE, int EPC>
+struct TileSmem {
+    static constexpr int RPW = kRowsPerWarp[MODE];
+    // ROW: per (warp, row of the current batch of 8, lane) partial (num, den);
+    // row stride padded by one entry against bank conflicts
+    static constexpr int kRed = MODE == MODE_ROW ? kWarps * 8 * 33 : 1;
+    // ROW: per (row, warp) totals; COL: per (warp-row, column) partials
+    static constexpr int kPart = MODE == MODE_ROW ? RPW * kWarps
+                               : (MODE == MODE_COL ? kWarps * 32 * EPC : 1);
+    float2 red[kRed];
+    float2 part[kPart];
+    double res[kWarps];
+    uint4 ring[kWarps][kRing][32];
+};
+
 template <int CODES, int GS, int OS, int MODE, typename TIn, int G>
-__global__ void __launch_bounds__(kThreads)
-tile_kernel(const __grid_constant__ Table tab, int mode_slot) {
+__global__ void __launch_bounds__(kThreads, 3)
+tile_kernel(const __grid_constant__ Table tab, int mode_slot, int want_res) {
     using CK = Chunk<TIn>;
     constexpr int EPC = CK::EPC;
+    constexpr int NP = EPC / 2;
     constexpr int SEG = 32 * EPC;
     constexpr int LPG = G / EPC;
     constexpr bool ACT = MODE == MODE_ACT;
-    using Q = Quant<CODES, GS, OS, ACT, EPC, LPG>;
+    constexpr bool NIB = MODE == MODE_PACK || MODE == MODE_ACT;
+    using Q = Quant<CODES, GS, OS, ACT, NP, LPG>;
     constexpr int RPW = kRowsPerWarp[MODE];
+    static_assert(RPW <= 32 || MODE == MODE_COL, "row factors are held one row per lane");
     constexpr int ESZ = 16 / EPC;                    // bytes per element
 
-    __shared__ float2 sm_part[2048];
-    __shared__ double sm_res[kWarps];
+    __shared__ __align__(16) TileSmem<MODE, EPC> sm;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t t = blockIdx.x;
@@ -478,110 +574,159 @@ tile_kernel(const __grid_constant__ Table tab, int mode_slot) {
     const int64_t col = (cb * wc + my_c) * (int64_t)SEG + lane * EPC;
     const bool col_ok = col < cols;
     const int64_t row_first = rb * tr;
+    const int64_t row0 = row_first + my_r;           // this warp's first row
+    // rows of this tile that this warp handles (k = 0 .. nk-1 -> row0 + k*wr)
+    const int nk = (int)max((int64_t)0, min((int64_t)RPW, (rows - row0 + wr - 1) / wr));
+    const bool res_on = !ACT && want_res != 0;
 
-    // per-lane column data
-    float bj[EPC], cm[EPC];
+    // per-lane column data, as pairs: b_j and the inner factor (1/b_j, or b_j for ACT)
+    f2 bj[NP], cm[NP];
 #pragma unroll
-    for (int j = 0; j < EPC; ++j) { bj[j] = 1.0f; cm[j] = 1.0f; }
-    if (md.b != nullptr && col_ok) {
-#pragma unroll
-        for (int j = 0; j < EPC; ++j) bj[j] = __ldg(md.b + col + j);
+    for (int k = 0; k < NP; ++k) {
+        float b0 = 1.0f, b1 = 1.0f;
+        if (md.b != nullptr && col_ok) {
+            b0 = __ldg(md.b + col + 2 * k);
+            b1 = __ldg(md.b + col + 2 * k + 1);
+        }
+        bj[k] = make_float2(b0, b1);
+        if (ACT) cm[k] = bj[k];
+        else if (OS == SC_E8M0) cm[k] = make_float2(recip_pow2(b0), recip_pow2(b1));
+        else cm[k] = make_float2(recip_approx(b0), recip_approx(b1));
     }
-#pragma unroll
-    for (int j = 0; j < EPC; ++j)
-        cm[j] = ACT ? bj[j] : ((OS == SC_E8M0) ? recip_pow2(bj[j]) : recip_approx(bj[j]));
+    // row factors: lane k holds a and 1/a of the warp's k-th row (COL mode
+    // reads them per row instead, it has 64 rows per warp)
+    float a_lane = 1.0f, ia_lane = 1.0f;
+    const float *const pa = ACT ? nullptr : md.a;
+    if (MODE != MODE_COL && pa != nullptr && lane < nk) {
+        a_lane = __ldg(pa + row0 + (int64_t)lane * wr);
+        ia_lane = (OS == SC_E8M0) ? recip_pow2(a_lane) : recip_approx(a_lane);
+    }
 
-    const float ts = ACT ? 1.0f : tensor_scale_of(md);
+    const float ts = (GS == SC_E4M3 && !ACT) ? tensor_scale_of(md) : 1.0f;
     const float inv_ts = 1.0f / ts;                 // ts is a power of two
-    const char *Wb = reinterpret_cast<const char *>(md.W);
 
-    float acc_p[EPC], acc_e[EPC];                    // COL accumulators
+    f2 acc_p[NP], acc_e[NP];                         // COL accumulators
 #pragma unroll
-    for (int j = 0; j < EPC; ++j) { acc_p[j] = 0.0f; acc_e[j] = 0.0f; }
-    float res = 0.0f;
+    for (int k = 0; k < NP; ++k) { acc_p[k] = bcast(0.0f); acc_e[k] = bcast(0.0f); }
+    f2 res2 = bcast(0.0f);
 
-    constexpr int U = 4;
-    for (int k0 = 0; k0 < RPW; k0 += U) {
-        CK ck[U];
-        int64_t rr[U];
+    // Each lane streams its own 16-byte chunk of the warp's rows through a
+    // private ring of kRing shared-memory slots with cp.async (one commit
+    // group per row, kRing - 1 rows in flight); only the lane that copied a
+    // slot reads it, so no barrier is needed.  Lanes past the last column
+    // never copy: their slots hold zeros.
+    if (!col_ok) {
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-            rr[u] = row_first + my_r + (int64_t)(k0 + u) * wr;
-            if (rr[u] < rows && col_ok)
-                ck[u].load(Wb + (rr[u] * cols + col) * ESZ);
-            else
-                ck[u].zero();
+        for (int q = 0; q < kRing; ++q) sm.ring[warp][q][lane] = make_uint4(0, 0, 0, 0);
+    }
+    const int64_t row_step = (int64_t)wr * cols * ESZ;
+    const char *src = reinterpret_cast<const char *>(md.W) + (row0 * cols + col) * ESZ;
+    const uint32_t ring0 = (uint32_t)__cvta_generic_to_shared(&sm.ring[warp][0][lane]);
+    auto issue = [&](int k) {
+        if (k < nk && col_ok) {
+            const uint32_t dst = ring0 + (uint32_t)((k & (kRing - 1)) * 32 * 16);
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;"
+                         :: "r"(dst), "l"(src + (int64_t)k * row_step) : "memory");
         }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const int64_t r = rr[u];
-            if (r >= rows) break;                     // warp-uniform
-            float a = 1.0f, ia = 1.0f;
-            if (!ACT && md.a != nullptr) {
-                a = __ldg(md.a + r);
+    for (int k = 0; k < kRing - 1; ++k) issue(k);
+
+#pragma unroll 1
+    for (int k = 0; k < nk; ++k) {
+        issue(k + kRing - 1);
+        asm volatile("cp.async.wait_group %0;" :: "n"(kRing - 1) : "memory");
+        CK ck;
+        ck.raw = sm.ring[warp][k & (kRing - 1)][lane];
+        float a = 1.0f, ia = 1.0f;
+        if (!ACT && pa != nullptr) {
+            if (MODE == MODE_COL) {
+                a = __ldg(pa + row0 + (int64_t)k * wr);
                 ia = (OS == SC_E8M0) ? recip_pow2(a) : recip_approx(a);
-            }
-            float w[EPC], z[EPC], ab[EPC], c[EPC];
-            ck[u].unpack(w);
-#pragma unroll
-            for (int j = 0; j < EPC; ++j) { z[j] = w[j] * cm[j]; ab[j] = a * bj[j]; }
-            float s, s_eff;
-            uint32_t nib;
-            Q::run(w, z, ab, ia, ts, inv_ts, tab.status, c, s, s_eff, nib);
-            if (MODE == MODE_ROW) {
-                float gn = 0.0f, gd = 0.0f;
-                const float as = a * s_eff;
-#pragma unroll
-                for (int j = 0; j < EPC; ++j) {
-                    float uq = c[j] * bj[j];
-                    gn = fmaf(w[j], uq, gn);
-                    gd = fmaf(uq, uq, gd);
-                    float d = fmaf(-as, uq, w[j]);
-                    res = fmaf(d, d, res);
-                }
-                float num = gn * s_eff, den = gd * (s_eff * s_eff);
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) {
-                    num += __shfl_xor_sync(0xffffffffu, num, o);
-                    den += __shfl_xor_sync(0xffffffffu, den, o);
-                }
-                if (lane == 0) sm_part[(k0 + u) * kWarps + warp] = make_float2(num, den);
-            } else if (MODE == MODE_COL) {
-                const float as = a * s_eff;
-#pragma unroll
-                for (int j = 0; j < EPC; ++j) {
-                    float v = c[j] * as;
-                    acc_p[j] = fmaf(w[j], v, acc_p[j]);
-                    acc_e[j] = fmaf(v, v, acc_e[j]);
-                    float d = fmaf(-v, bj[j], w[j]);
-                    res = fmaf(d, d, res);
-                }
             } else {
-                if (MODE == MODE_PACK) {
-                    const float as = a * s_eff;
+                a = __shfl_sync(0xffffffffu, a_lane, k);
+                ia = __shfl_sync(0xffffffffu, ia_lane, k);
+            }
+        }
+        f2 w[NP], z[NP], c[NP];
+        ck.unpack2(w);
 #pragma unroll
-                    for (int j = 0; j < EPC; ++j) {
-                        float d = fmaf(-as, c[j] * bj[j], w[j]);
-                        res = fmaf(d, d, res);
-                    }
+        for (int j = 0; j < NP; ++j) z[j] = mul2(w[j], cm[j]);
+        float s, s_eff;
+        uint32_t nib;
+        Q::template run<NIB>(w, z, a, ia, bj, ts, inv_ts, tab.status, c, s, s_eff, nib);
+        if (MODE == MODE_ROW) {
+            f2 gn = bcast(0.0f), gd = bcast(0.0f);
+            const f2 nas = bcast(-(a * s_eff));
+#pragma unroll
+            for (int j = 0; j < NP; ++j) {
+                const f2 uq = mul2(c[j], bj[j]);
+                gn = fma2(w[j], uq, gn);
+                gd = fma2(uq, uq, gd);
+                if (res_on) {
+                    const f2 d = fma2(nas, uq, w[j]);
+                    res2 = fma2(d, d, res2);
                 }
-                if (col_ok) {
-                    uint8_t *cp = md.codes + r * (cols >> 1) + (col >> 1);
-                    if (EPC == 8) *reinterpret_cast<uint32_t *>(cp) = nib;
-                    else *reinterpret_cast<uint16_t *>(cp) = (uint16_t)nib;
-                    if ((lane % LPG) == 0) {
-                        const int64_t gi = r * (cols / G) + col / G;
-                        if (GS == SC_BF16)
-                            reinterpret_cast<uint16_t *>(md.gscales)[gi] = (uint16_t)(__float_as_uint(s) >> 16);
-                        else if (GS == SC_E8M0)
-                            reinterpret_cast<uint8_t *>(md.gscales)[gi] = (uint8_t)((__float_as_uint(s) >> 23) & 0xFF);
-                        else
-                            reinterpret_cast<uint8_t *>(md.gscales)[gi] = (uint8_t)e4m3_bits(s);
-                    }
+            }
+            // this lane's share of row k; every 8 rows the warp sums the shares
+            // of its rows: lane l adds 8 shares of row l/4, then 2 shuffles
+            sm.red[(warp * 8 + (k & 7)) * 33 + lane] =
+                make_float2((gn.x + gn.y) * s_eff, (gd.x + gd.y) * (s_eff * s_eff));
+            if ((k & 7) == 7 || k == nk - 1) {
+                __syncwarp();
+                const int rr = lane >> 2, pp = lane & 3;
+                const float2 *p = &sm.red[(warp * 8 + rr) * 33 + pp * 8];
+                f2 acc = p[0];
+#pragma unroll
+                for (int j = 1; j < 8; ++j) acc = __fadd2_rn(acc, p[j]);
+                acc.x += __shfl_xor_sync(0xffffffffu, acc.x, 1);
+                acc.y += __shfl_xor_sync(0xffffffffu, acc.y, 1);
+                acc.x += __shfl_xor_sync(0xffffffffu, acc.x, 2);
+                acc.y += __shfl_xor_sync(0xffffffffu, acc.y, 2);
+                const int kk = (k & ~7) + rr;
+                if (pp == 0 && kk <= k) sm.part[kk * kWarps + warp] = acc;
+                __syncwarp();
+            }
+        } else if (MODE == MODE_COL) {
+            const f2 as = bcast(a * s_eff);
+#pragma unroll
+            for (int j = 0; j < NP; ++j) {
+                const f2 v = mul2(c[j], as);
+                acc_p[j] = fma2(w[j], v, acc_p[j]);
+                acc_e[j] = fma2(v, v, acc_e[j]);
+                if (res_on) {
+                    const f2 d = fma2(v, bj[j], neg2(w[j]));
+                    res2 = fma2(d, d, res2);
+                }
+            }
+        } else {
+            const int64_t r = row0 + (int64_t)k * wr;
+            if (MODE == MODE_PACK && res_on) {
+                const f2 nas = bcast(-(a * s_eff));
+#pragma unroll
+                for (int j = 0; j < NP; ++j) {
+                    const f2 d = fma2(nas, mul2(c[j], bj[j]), w[j]);
+                    res2 = fma2(d, d, res2);
+                }
+            }
+            if (col_ok) {
+                uint8_t *cp = md.codes + r * (cols >> 1) + (col >> 1);
+                if (EPC == 8) *reinterpret_cast<uint32_t *>(cp) = nib;
+                else *reinterpret_cast<uint16_t *>(cp) = (uint16_t)nib;
+                if ((lane % LPG) == 0) {
+                    const int64_t gi = r * (cols / G) + col / G;
+                    if (GS == SC_BF16)
+                        reinterpret_cast<uint16_t *>(md.gscales)[gi] = (uint16_t)(__float_as_uint(s) >> 16);
+                    else if (GS == SC_E8M0)
+                        reinterpret_cast<uint8_t *>(md.gscales)[gi] = (uint8_t)((__float_as_uint(s) >> 23) & 0xFF);
+                    else
+                        reinterpret_cast<uint8_t *>(md.gscales)[gi] = (uint8_t)e4m3_bits(s);
                 }
             }
         }
     }
+    asm volatile("cp.async.wait_all;" ::: "memory");
 
     // ---- tile epilogue ----
     if (MODE == MODE_ROW) {
@@ -593,7 +738,7 @@ tile_kernel(const __grid_constant__ Table tab, int mode_slot) {
             if (row < rows) {
                 float num = 0.0f, den = 0.0f;
                 for (int c2 = 0; c2 < wc; ++c2) {          // fixed order over segments
-                    float2 p = sm_part[k * kWarps + r * wc + c2];
+                    float2 p = sm.part[k * kWarps + r * wc + c2];
                     num += p.x;
                     den += p.y;
                 }
@@ -606,21 +751,27 @@ tile_kernel(const __grid_constant__ Table tab, int mode_slot) {
             if (col_ok) {
                 float2 *dst = md.colpart + rb * cols + col;
 #pragma unroll
-                for (int j = 0; j < EPC; ++j) dst[j] = make_float2(acc_p[j], acc_e[j]);
+                for (int k = 0; k < NP; ++k) {
+                    dst[2 * k] = make_float2(acc_p[k].x, acc_e[k].x);
+                    dst[2 * k + 1] = make_float2(acc_p[k].y, acc_e[k].y);
+                }
             }
         } else {
             // reduce over the wr warp-rows of each segment in fixed order
             const int seg_cols = wc * SEG;
 #pragma unroll
-            for (int j = 0; j < EPC; ++j)
-                sm_part[my_r * seg_cols + my_c * SEG + lane * EPC + j] = make_float2(acc_p[j], acc_e[j]);
+            for (int k = 0; k < NP; ++k) {
+                const int base = my_r * seg_cols + my_c * SEG + lane * EPC + 2 * k;
+                sm.part[base] = make_float2(acc_p[k].x, acc_e[k].x);
+                sm.part[base + 1] = make_float2(acc_p[k].y, acc_e[k].y);
+            }
             __syncthreads();
             for (int cc = threadIdx.x; cc < seg_cols; cc += kThreads) {
                 const int64_t gc = cb * seg_cols + cc;
                 if (gc < cols) {
                     float p = 0.0f, e = 0.0f;
                     for (int r = 0; r < wr; ++r) {
-                        float2 v = sm_part[r * seg_cols + cc];
+                        float2 v = sm.part[r * seg_cols + cc];
                         p += v.x;
                         e += v.y;
                     }
@@ -629,16 +780,16 @@ tile_kernel(const __grid_constant__ Table tab, int mode_slot) {
             }
         }
     }
-    if (MODE == MODE_ROW || MODE == MODE_COL || MODE == MODE_PACK) {
-        double rd = (double)res;
+    if ((MODE == MODE_ROW || MODE == MODE_COL || MODE == MODE_PACK) && res_on) {
+        double rd = (double)res2.x + (double)res2.y;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) rd += __shfl_xor_sync(0xffffffffu, rd, o);
-        if (lane == 0) sm_res[warp] = rd;
+        if (lane == 0) sm.res[warp] = rd;
         __syncthreads();
         double *slot = (MODE == MODE_COL) ? md.res_col : md.res_row;
         if (threadIdx.x == 0 && slot != nullptr) {
             double tot = 0.0;
-            for (int k = 0; k < kWarps; ++k) tot += sm_res[k];
+            for (int k = 0; k < kWarps; ++k) tot += sm.res[k];
             slot[lt] = tot;
         }
     }

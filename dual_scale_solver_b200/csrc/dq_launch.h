@@ -16,6 +16,7 @@ struct TileLaunch {
     int slot;           // tile table slot: 0 ROW, 1 COL, 2 PACK/ACT
     int f32;            // 1: float32 input, 0: bfloat16
     int G;              // 16, 32, 64
+    int want_res;       // 1: accumulate the residual (an MSE output is wanted)
     cudaStream_t stream;
 };
 
@@ -43,7 +44,7 @@ cudaError_t launch_tile_combo(const TileLaunch &L) {
     if (L.grid <= 0) return cudaSuccess;
     dim3 grid((unsigned)L.grid), block(kThreads);
 #define DQ_TILE(MODE, TIN, GG) \
-    tile_kernel<CODES, GS, OS, MODE, TIN, GG><<<grid, block, 0, L.stream>>>(L.tab, L.slot)
+    tile_kernel<CODES, GS, OS, MODE, TIN, GG><<<grid, block, 0, L.stream>>>(L.tab, L.slot, L.want_res)
 #define DQ_BY_G(MODE, TIN)                          \
     switch (L.G) {                                  \
         case 16: DQ_TILE(MODE, TIN, 16); break;     \

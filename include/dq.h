@@ -128,7 +128,7 @@ DQ_API dq_status dq_workspace_size(int32_t n, const int64_t *rows, const int64_t
 
 /* Q(X ⊘ (a bᵀ)): the black-box group quantizer (daiwk note, "原始论文总结")
  * applied to X / (a_i b_j) with second-level scale `tensor_scale` (host value,
- * a power of two; 1.0 when the format has none).  a (rows) and b (cols) may be
+ * a power of two; it must be 1.0 unless the group scales are E4M3).  a (rows) and b (cols) may be
  * NULL (all ones).  Writes packed codes and group scales.  No workspace. */
 DQ_API dq_status dq_quantize(const void *X, int32_t dtype, int64_t rows, int64_t cols,
                       const dq_format *fmt, const float *a, const float *b,
