@@ -531,9 +531,9 @@ __device__ __forceinline__ float project_outer(float x, bool &clamped) {
 template <int MODE, int EPC>
 struct TileSmem {
     static constexpr int RPW = kRowsPerWarp[MODE];
-    // ROW: per (warp, row of the current batch of 8, lane) partial (num, den);
-    // row stride padded by one entry against bank conflicts
-    static constexpr int kRed = MODE == MODE_ROW ? kWarps * 8 * 33 : 1;
+    // ROW: per (warp, row of the warp, lane) partial (num, den), reduced once
+    // at the end of the tile; row stride padded by one entry
+    static constexpr int kRed = MODE == MODE_ROW ? kWarps * RPW * 33 : 1;
     // ROW: per (row, warp) totals; COL: per (warp-row, column) partials
     static constexpr int kPart = MODE == MODE_ROW ? RPW * kWarps
                                : (MODE == MODE_COL ? kWarps * 32 * EPC : 1);
@@ -558,7 +558,8 @@ tile_kernel(const __grid_constant__ Table tab, int mode_slot, int want_res) {
     static_assert(RPW <= 32 || MODE == MODE_COL, "row factors are held one row per lane");
     constexpr int ESZ = 16 / EPC;                    // bytes per element
 
-    __shared__ __align__(16) TileSmem<MODE, EPC> sm;
+    extern __shared__ __align__(16) unsigned char tile_smem[];
+    TileSmem<MODE, EPC> &sm = *reinterpret_cast<TileSmem<MODE, EPC> *>(tile_smem);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t t = blockIdx.x;
@@ -622,23 +623,29 @@ tile_kernel(const __grid_constant__ Table tab, int mode_slot, int want_res) {
     const int64_t row_step = (int64_t)wr * cols * ESZ;
     const char *src = reinterpret_cast<const char *>(md.W) + (row0 * cols + col) * ESZ;
     const uint32_t ring0 = (uint32_t)__cvta_generic_to_shared(&sm.ring[warp][0][lane]);
-    auto issue = [&](int k) {
+    // copy of row k into slot k % kRing (k < nk; lanes past the last column never copy)
+    auto issue = [&](int k, int slot) {
         if (k < nk && col_ok) {
-            const uint32_t dst = ring0 + (uint32_t)((k & (kRing - 1)) * 32 * 16);
             asm volatile("cp.async.cg.shared.global [%0], [%1], 16;"
-                         :: "r"(dst), "l"(src + (int64_t)k * row_step) : "memory");
+                         :: "r"(ring0 + (uint32_t)(slot * 32 * 16)),
+                            "l"(src + (int64_t)k * row_step) : "memory");
         }
         asm volatile("cp.async.commit_group;" ::: "memory");
     };
 #pragma unroll
-    for (int k = 0; k < kRing - 1; ++k) issue(k);
+    for (int k = 0; k < kRing - 1; ++k) issue(k, k);
 
+    // rows in groups of kRing: the ring slot of each row is a constant
 #pragma unroll 1
-    for (int k = 0; k < nk; ++k) {
-        issue(k + kRing - 1);
+    for (int k0 = 0; k0 < nk; k0 += kRing) {
+#pragma unroll
+    for (int u = 0; u < kRing; ++u) {
+        const int k = k0 + u;
+        if (k >= nk) break;                           // warp-uniform
+        issue(k + kRing - 1, (u + kRing - 1) % kRing);
         asm volatile("cp.async.wait_group %0;" :: "n"(kRing - 1) : "memory");
         CK ck;
-        ck.raw = sm.ring[warp][k & (kRing - 1)][lane];
+        ck.raw = sm.ring[warp][u][lane];
         float a = 1.0f, ia = 1.0f;
         if (!ACT && pa != nullptr) {
             if (MODE == MODE_COL) {
@@ -669,25 +676,9 @@ tile_kernel(const __grid_constant__ Table tab, int mode_slot, int want_res) {
                     res2 = fma2(d, d, res2);
                 }
             }
-            // this lane's share of row k; every 8 rows the warp sums the shares
-            // of its rows: lane l adds 8 shares of row l/4, then 2 shuffles
-            sm.red[(warp * 8 + (k & 7)) * 33 + lane] =
+            // this lane's share of row k, summed over lanes at the end of the tile
+            sm.red[(warp * RPW + k) * 33 + lane] =
                 make_float2((gn.x + gn.y) * s_eff, (gd.x + gd.y) * (s_eff * s_eff));
-            if ((k & 7) == 7 || k == nk - 1) {
-                __syncwarp();
-                const int rr = lane >> 2, pp = lane & 3;
-                const float2 *p = &sm.red[(warp * 8 + rr) * 33 + pp * 8];
-                f2 acc = p[0];
-#pragma unroll
-                for (int j = 1; j < 8; ++j) acc = __fadd2_rn(acc, p[j]);
-                acc.x += __shfl_xor_sync(0xffffffffu, acc.x, 1);
-                acc.y += __shfl_xor_sync(0xffffffffu, acc.y, 1);
-                acc.x += __shfl_xor_sync(0xffffffffu, acc.x, 2);
-                acc.y += __shfl_xor_sync(0xffffffffu, acc.y, 2);
-                const int kk = (k & ~7) + rr;
-                if (pp == 0 && kk <= k) sm.part[kk * kWarps + warp] = acc;
-                __syncwarp();
-            }
         } else if (MODE == MODE_COL) {
             const f2 as = bcast(a * s_eff);
 #pragma unroll
@@ -726,10 +717,28 @@ tile_kernel(const __grid_constant__ Table tab, int mode_slot, int want_res) {
             }
         }
     }
+    }
     asm volatile("cp.async.wait_all;" ::: "memory");
 
     // ---- tile epilogue ----
     if (MODE == MODE_ROW) {
+        // (warp, row) pair p = t / 2 sums 16 lane shares per thread, then the
+        // two halves; fixed order throughout
+        static_assert((2 * kWarps * RPW) % kThreads == 0, "every thread takes the same trips");
+        __syncthreads();
+        for (int p2 = threadIdx.x; p2 < 2 * kWarps * RPW; p2 += kThreads) {
+            const int pw = (p2 >> 1) / RPW, pk = (p2 >> 1) % RPW, h = p2 & 1;
+            const int64_t row = row_first + (pw / wc) + (int64_t)pk * wr;
+            f2 acc = bcast(0.0f);
+            if (row < rows) {
+                const float2 *p = &sm.red[(pw * RPW + pk) * 33 + 16 * h];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) acc = __fadd2_rn(acc, p[j]);
+            }
+            acc.x += __shfl_xor_sync(0xffffffffu, acc.x, 1);
+            acc.y += __shfl_xor_sync(0xffffffffu, acc.y, 1);
+            if (h == 0) sm.part[pk * kWarps + pw] = acc;
+        }
         __syncthreads();
         // rows of the tile: local row k*wr + r is warp-row r's k-th row
         for (int lr = threadIdx.x; lr < tr; lr += kThreads) {

@@ -38,36 +38,53 @@ cudaError_t launch_tile_c3(const TileLaunch &L);
 cudaError_t launch_tile_c4(const TileLaunch &L);
 cudaError_t launch_tile_c5(const TileLaunch &L);
 
+// One tile-kernel launch; the shared memory is dynamic (the row-statistics
+// layout needs more than the 48 KB default, opted in once per device).
+template <int CODES, int GS, int OS, int MODE, typename TIn, int G>
+cudaError_t launch_tile_one(const TileLaunch &L) {
+    constexpr size_t bytes = sizeof(TileSmem<MODE, Chunk<TIn>::EPC>);
+    auto kern = tile_kernel<CODES, GS, OS, MODE, TIn, G>;
+    if (bytes > 48 * 1024) {
+        static bool done[64] = {};
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+        if (!done[dev]) {
+            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 (int)bytes);
+            if (e != cudaSuccess) return e;
+            done[dev] = true;
+        }
+    }
+    kern<<<dim3((unsigned)L.grid), dim3(kThreads), bytes, L.stream>>>(L.tab, L.slot, L.want_res);
+    return cudaGetLastError();
+}
+
 // Dispatch over mode, dtype and G for one format set (used by each unit).
 template <int CODES, int GS, int OS>
 cudaError_t launch_tile_combo(const TileLaunch &L) {
     if (L.grid <= 0) return cudaSuccess;
-    dim3 grid((unsigned)L.grid), block(kThreads);
-#define DQ_TILE(MODE, TIN, GG) \
-    tile_kernel<CODES, GS, OS, MODE, TIN, GG><<<grid, block, 0, L.stream>>>(L.tab, L.slot, L.want_res)
+#define DQ_TILE(MODE, TIN, GG) return launch_tile_one<CODES, GS, OS, MODE, TIN, GG>(L)
 #define DQ_BY_G(MODE, TIN)                          \
     switch (L.G) {                                  \
-        case 16: DQ_TILE(MODE, TIN, 16); break;     \
-        case 32: DQ_TILE(MODE, TIN, 32); break;     \
-        case 64: DQ_TILE(MODE, TIN, 64); break;     \
+        case 16: DQ_TILE(MODE, TIN, 16);            \
+        case 32: DQ_TILE(MODE, TIN, 32);            \
+        case 64: DQ_TILE(MODE, TIN, 64);            \
         default: return cudaErrorInvalidValue;      \
     }
 #define DQ_BY_T(MODE)                                      \
     if (L.f32) { DQ_BY_G(MODE, float) } else { DQ_BY_G(MODE, Bf16Tag) }
     switch (L.mode) {
-        case MODE_ROW: DQ_BY_T(MODE_ROW); break;
-        case MODE_COL: DQ_BY_T(MODE_COL); break;
-        case MODE_PACK: DQ_BY_T(MODE_PACK); break;
+        case MODE_ROW: DQ_BY_T(MODE_ROW);
+        case MODE_COL: DQ_BY_T(MODE_COL);
+        case MODE_PACK: DQ_BY_T(MODE_PACK);
         case MODE_ACT:
             if (L.f32) return cudaErrorInvalidValue;
             DQ_BY_G(MODE_ACT, Bf16Tag);
-            break;
         default: return cudaErrorInvalidValue;
     }
 #undef DQ_BY_T
 #undef DQ_BY_G
 #undef DQ_TILE
-    return cudaGetLastError();
 }
 
 }  // namespace dq
