@@ -264,7 +264,7 @@ def run_ours(args, wl, rank, world, local_rank):
     clocks.start()
     time.sleep(0.3)
     dq.kernel_timing(True)
-    for k in range(4):
+    for k in range(5):
         dq.kernel_time(k)                     # clear
     n0 = dq.launch_count()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -278,7 +278,7 @@ def run_ours(args, wl, rank, world, local_rank):
     barrier()
     ms = e0.elapsed_time(e1)
     launches = dq.launch_count() - n0
-    kt = {k: dq.kernel_time(k) for k in range(4)}
+    kt = {k: dq.kernel_time(k) for k in range(5)}
     dq.kernel_timing(False)
     clk = clocks.stop()
     if dist:
@@ -290,8 +290,8 @@ def run_ours(args, wl, rank, world, local_rank):
     value = world * E * T / (ms_step / 1e3)
 
     # dominant tile kernel and its roofline (HBM: it streams W once per launch)
-    names = {0: "row_stats", 1: "col_stats", 2: "pack", 3: "act_quant"}
-    dom = max((0, 1), key=lambda k: kt[k][0])
+    names = {0: "row_stats", 1: "col_stats", 2: "pack", 3: "act_quant", 4: "fused_row_col_stats"}
+    dom = max((0, 1, 4), key=lambda k: kt[k][0])
     tot_ms, nl = kt[dom]
     avg_s = tot_ms / max(nl, 1) / 1e3
     rows_sum = sum(W.shape[0] for W in Ws)

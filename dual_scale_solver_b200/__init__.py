@@ -332,7 +332,7 @@ def act_rescale_quant(X, b, fmt, codes=None, gscales=None, stream=None):
     return codes, gscales
 
 
-KIND_ROW, KIND_COL, KIND_PACK, KIND_ACT = 0, 1, 2, 3
+KIND_ROW, KIND_COL, KIND_PACK, KIND_ACT, KIND_FUSED = 0, 1, 2, 3, 4
 
 
 def kernel_timing(enable: bool):

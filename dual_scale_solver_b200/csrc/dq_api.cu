@@ -215,15 +215,21 @@ struct Launcher {
     int64_t total_rows = 0, total_cols = 0;
     cudaStream_t st;
 
-    dq_status tiles_pass(int mode, bool want_res) {
+    // One tile pass.  A gated pass (the literal fallback of a fused
+    // iteration) launches a small grid that visits the tiles grid-stride and
+    // returns at once unless its flag is up.
+    dq_status tiles_pass(int mode, bool want_res, unsigned int *flags = nullptr, int gate = 0) {
         TileLaunch L;
         L.tab = tab;
         L.mode = mode;
-        L.slot = (mode == MODE_ACT) ? 2 : mode;
-        L.grid = tiles[L.slot];
+        L.slot = (mode == MODE_ACT) ? 2 : (mode == MODE_FUSED ? 1 : mode);
+        L.tiles = tiles[L.slot];
+        L.grid = gate ? std::min<int64_t>(L.tiles, 148 * 3) : L.tiles;
         L.f32 = f32 ? 1 : 0;
         L.G = G;
         L.want_res = want_res ? 1 : 0;
+        L.flags = flags;
+        L.gate = gate;
         L.stream = st;
         if (L.grid <= 0) return DQ_OK;
         cudaEvent_t beg = nullptr, end = nullptr;
@@ -241,12 +247,12 @@ struct Launcher {
         }
         return DQ_OK;
     }
-    dq_status row_finalize() {
+    dq_status row_finalize(unsigned int *flags = nullptr) {
         if (total_rows == 0) return DQ_OK;
         if (outer_of(combo) == SC_E8M0)
-            row_finalize_kernel<SC_E8M0><<<grid_for(total_rows, 256), 256, 0, st>>>(tab, total_rows);
+            row_finalize_kernel<SC_E8M0><<<grid_for(total_rows, 256), 256, 0, st>>>(tab, total_rows, flags);
         else
-            row_finalize_kernel<SC_BF16><<<grid_for(total_rows, 256), 256, 0, st>>>(tab, total_rows);
+            row_finalize_kernel<SC_BF16><<<grid_for(total_rows, 256), 256, 0, st>>>(tab, total_rows, flags);
         DQ_CUDA(cudaGetLastError());
         count_launches(1);
         return DQ_OK;
@@ -268,7 +274,40 @@ struct Launcher {
         count_launches(1);
         return DQ_OK;
     }
+
+    // One BCD iteration: row statistics, row update, column statistics,
+    // column update, MSE.  With power-of-two outer and group scales (MX
+    // formats) both statistics come from one pass over W (`fused`); the
+    // literal passes stand by behind the iteration's flags.
+    dq_status iteration(int t, bool fused, unsigned int *flag_slots, bool want_trace,
+                        bool want_half) {
+        dq_status s;
+        // iteration t uses flag slot t % 2; its MSE kernel clears the other slot
+        unsigned int *flags = flag_slots + 2 * (t & 1);
+        unsigned int *next = flag_slots + 2 * ((t + 1) & 1);
+        if (!fused) {
+            if ((s = tiles_pass(MODE_ROW, want_trace)) != DQ_OK) return s;
+            if ((s = row_finalize()) != DQ_OK) return s;
+            if ((s = tiles_pass(MODE_COL, want_half)) != DQ_OK) return s;
+            if ((s = col_finalize()) != DQ_OK) return s;
+            return mse(MODE_ROW, t, t, nullptr, nullptr);
+        }
+        if ((s = tiles_pass(MODE_FUSED, want_trace || want_half, flags, 0)) != DQ_OK) return s;
+        if ((s = tiles_pass(MODE_ROW, want_trace, flags, 1)) != DQ_OK) return s;
+        if ((s = row_finalize(flags)) != DQ_OK) return s;
+        if ((s = tiles_pass(MODE_COL, want_half, flags, 2)) != DQ_OK) return s;
+        if ((s = col_finalize()) != DQ_OK) return s;
+        mse_finalize_fused_kernel<<<2 * tab.n, 256, 0, st>>>(tab, flags, next, t);
+        DQ_CUDA(cudaGetLastError());
+        count_launches(1);
+        return DQ_OK;
+    }
 };
+
+// MX formats: power-of-two outer and group scales
+bool fused_ok(int combo) {
+    return combo == COMBO_INT4_E8M0_E8M0 || combo == COMBO_E2M1_E8M0_E8M0;
+}
 
 thread_local std::vector<MatDesc> t_table;
 
@@ -281,7 +320,7 @@ dq_status solve_impl(int32_t n, const dq_matrix *mats, int32_t dtype, const dq_f
     if (s != DQ_OK) return s;
     if (n == 0) return DQ_OK;
     const bool f32 = dtype == DQ_DT_F32;
-    size_t need = table_ws(n);
+    size_t need = table_ws(n) + 256;
     for (int i = 0; i < n; ++i) {
         const dq_matrix &m = mats[i];
         if (m.rows < 0 || m.cols < 0) return DQ_ERR_SHAPE;
@@ -303,6 +342,7 @@ dq_status solve_impl(int32_t n, const dq_matrix *mats, int32_t dtype, const dq_f
 
     Carve cv{static_cast<char *>(workspace), static_cast<char *>(workspace) + ws_bytes};
     MatDesc *dev_table = n > 1 ? cv.take<MatDesc>((size_t)n * sizeof(MatDesc)) : nullptr;
+    unsigned int *flags = cv.take<unsigned int>(256);     // fused-path flags: 2 slots x 2 words
     t_table.assign(n, MatDesc{});
     int64_t tile_base[3] = {0, 0, 0}, row_base = 0, col_base = 0;
     for (int i = 0; i < n; ++i) {
@@ -367,13 +407,10 @@ dq_status solve_impl(int32_t n, const dq_matrix *mats, int32_t dtype, const dq_f
         want_trace |= mats[i].mse_trace != nullptr;
         want_half |= mats[i].mse_half != nullptr;
     }
-    for (int t = 0; t < T; ++t) {
-        if ((s = L.tiles_pass(MODE_ROW, want_trace)) != DQ_OK) return s;
-        if ((s = L.row_finalize()) != DQ_OK) return s;
-        if ((s = L.tiles_pass(MODE_COL, want_half)) != DQ_OK) return s;
-        if ((s = L.col_finalize()) != DQ_OK) return s;
-        if ((s = L.mse(MODE_ROW, t, t, nullptr, nullptr)) != DQ_OK) return s;
-    }
+    const bool fused = fused_ok(fi.combo);
+    if (fused && T > 0) DQ_CUDA(cudaMemsetAsync(flags, 0, 4 * sizeof(unsigned int), st));
+    for (int t = 0; t < T; ++t)
+        if ((s = L.iteration(t, fused, flags, want_trace, want_half)) != DQ_OK) return s;
     if ((s = L.tiles_pass(MODE_PACK, want_trace)) != DQ_OK) return s;
     if ((s = L.mse(2, T, -1, nullptr, nullptr)) != DQ_OK) return s;
     return DQ_OK;
@@ -535,7 +572,7 @@ dq_status dq_workspace_size(int32_t n, const int64_t *rows, const int64_t *cols,
         // the larger of the bf16 and float32 layouts, so one size serves both
         b += std::max(matrix_ws(rows[i], cols[i], false), matrix_ws(rows[i], cols[i], true));
     }
-    *bytes = b + 256;
+    *bytes = b + 512;
     return DQ_OK;
 }
 
@@ -692,7 +729,7 @@ dq_status dq_kernel_timing(int32_t enable) {
 }
 
 dq_status dq_kernel_time(int32_t kind, double *ms, int64_t *launches) {
-    if (!ms || !launches || kind < 0 || kind > 3) return DQ_ERR_ARG;
+    if (!ms || !launches || kind < 0 || kind > 4) return DQ_ERR_ARG;
     std::lock_guard<std::mutex> lk(g_timing_mu);
     double tot = 0.0;
     int64_t cnt = 0;

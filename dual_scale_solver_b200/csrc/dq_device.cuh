@@ -26,12 +26,12 @@ namespace dq {
 
 enum { CODES_INT4 = 0, CODES_E2M1 = 1 };
 enum { SC_BF16 = 0, SC_E8M0 = 1, SC_E4M3 = 2 };
-enum { MODE_ROW = 0, MODE_COL = 1, MODE_PACK = 2, MODE_ACT = 3 };
+enum { MODE_ROW = 0, MODE_COL = 1, MODE_PACK = 2, MODE_ACT = 3, MODE_FUSED = 4 };
 enum { STATUS_NONFINITE = 1u, STATUS_RANGE = 2u };
 
 constexpr int kWarps = 8;            // warps per CTA of the tile kernel
 constexpr int kThreads = 32 * kWarps;
-constexpr int kRowsPerWarp[4] = {16, 64, 16, 16};   // per mode
+constexpr int kRowsPerWarp[5] = {16, 64, 16, 16, 64};   // per mode
 constexpr int kRing = 4;             // cp.async ring slots per lane (rows in flight + 1)
 constexpr float kBf16Max = 3.38953138925153547590470800371487866880e+38f;  // (2-2^-7)*2^127
 constexpr float kMinNormal = 1.17549435082228750796873653722224568e-38f;    // 2^-126
@@ -292,7 +292,8 @@ struct Quant {
     __device__ __forceinline__ static void run(const f2 (&w)[NP], const f2 (&z)[NP], float a,
                                                float ia, const f2 (&bj)[NP], float ts,
                                                float inv_ts, unsigned int *status, f2 (&c)[NP],
-                                               float &s, float &s_eff, uint32_t &nib) {
+                                               float &s, float &s_eff, uint32_t &nib,
+                                               bool &nonzero) {
         float mz = 0.0f;
 #pragma unroll
         for (int k = 0; k < NP; ++k) mz = max3_nan(mz, fabsf(z[k].x), fabsf(z[k].y));
@@ -304,6 +305,7 @@ struct Quant {
         // finalize kernels flag; the other modes flag it here
         if (NIB && !finite) atomicOr(status, STATUS_NONFINITE);
         const bool pos = finite && m > 0.0f;
+        nonzero = pos;
         if (GS == SC_E8M0 && kExactM) {
             // smallest 2^e with qmax 2^e >= m (m exact): e = E(m) - 2, plus 1
             // when m's significand exceeds qmax/4 (1.75 INT4, 1.5 E2M1);
@@ -532,20 +534,29 @@ template <int MODE, int EPC>
 struct TileSmem {
     static constexpr int RPW = kRowsPerWarp[MODE];
     // ROW: per (warp, row of the warp, lane) partial (num, den), reduced once
-    // at the end of the tile; row stride padded by one entry
-    static constexpr int kRed = MODE == MODE_ROW ? kWarps * RPW * 33 : 1;
-    // ROW: per (row, warp) totals; COL: per (warp-row, column) partials
-    static constexpr int kPart = MODE == MODE_ROW ? RPW * kWarps
-                               : (MODE == MODE_COL ? kWarps * 32 * EPC : 1);
+    // at the end of the tile; FUSED: the same for a batch of 8 rows, reduced
+    // every 8 rows.  Row stride padded by one entry.
+    static constexpr int kRed = MODE == MODE_ROW ? kWarps * RPW * 33
+                              : (MODE == MODE_FUSED ? kWarps * 8 * 33 : 1);
+    // ROW, FUSED: per (row, warp) totals
+    static constexpr int kRtot = (MODE == MODE_ROW || MODE == MODE_FUSED) ? RPW * kWarps : 1;
+    // COL, FUSED: per (warp-row, column) partials
+    static constexpr int kPart = (MODE == MODE_COL || MODE == MODE_FUSED) ? kWarps * 32 * EPC : 1;
     float2 red[kRed];
+    float2 rtot[kRtot];
     float2 part[kPart];
     double res[kWarps];
     uint4 ring[kWarps][kRing][32];
 };
 
+// Column statistics keep 2 x EPC accumulators per lane: those modes run 2
+// CTAs per SM (up to 128 registers), the others 3.
+template <int MODE> struct TileOcc { static constexpr int kMinBlocks = (MODE == MODE_COL || MODE == MODE_FUSED) ? 2 : 3; };
+
 template <int CODES, int GS, int OS, int MODE, typename TIn, int G>
-__global__ void __launch_bounds__(kThreads, 3)
-tile_kernel(const __grid_constant__ Table tab, int mode_slot, int want_res) {
+__global__ void __launch_bounds__(kThreads, TileOcc<MODE>::kMinBlocks)
+tile_kernel(const __grid_constant__ Table tab, int mode_slot, int want_res, int64_t total_tiles,
+            unsigned int *flags, int gate) {
     using CK = Chunk<TIn>;
     constexpr int EPC = CK::EPC;
     constexpr int NP = EPC / 2;
@@ -553,20 +564,31 @@ tile_kernel(const __grid_constant__ Table tab, int mode_slot, int want_res) {
     constexpr int LPG = G / EPC;
     constexpr bool ACT = MODE == MODE_ACT;
     constexpr bool NIB = MODE == MODE_PACK || MODE == MODE_ACT;
+    constexpr bool FUSED = MODE == MODE_FUSED;
+    constexpr bool ROWSTAT = MODE == MODE_ROW || FUSED;
+    constexpr bool COLSTAT = MODE == MODE_COL || FUSED;
     using Q = Quant<CODES, GS, OS, ACT, NP, LPG>;
     constexpr int RPW = kRowsPerWarp[MODE];
-    static_assert(RPW <= 32 || MODE == MODE_COL, "row factors are held one row per lane");
+    static_assert(RPW <= 32 || MODE == MODE_COL || FUSED, "row factors are held one row per lane");
+    static_assert(!FUSED || (GS == SC_E8M0 && OS == SC_E8M0), "fused statistics need power-of-two scales");
     constexpr int ESZ = 16 / EPC;                    // bytes per element
 
     extern __shared__ __align__(16) unsigned char tile_smem[];
     TileSmem<MODE, EPC> &sm = *reinterpret_cast<TileSmem<MODE, EPC> *>(tile_smem);
 
+    // gated launches (the literal fallback of a fused iteration) run only when
+    // an earlier kernel of the iteration raised the flag
+    if (gate == 1 && flags[0] == 0) return;
+    if (gate == 2 && (flags[0] | flags[1]) == 0) return;
+
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t t = blockIdx.x;
+    const bool res_on = !ACT && want_res != 0;
+
+    for (int64_t t = blockIdx.x; t < total_tiles; t += gridDim.x) {
     const int mi = find_owner(tab, t, [mode_slot](const MatDesc &d) { return d.tile0[mode_slot]; });
     const MatDesc &md = tab.get(mi);
     const int64_t lt = t - md.tile0[mode_slot];
-    if (lt >= md.ntiles[mode_slot]) return;          // (uniform per CTA)
+    if (lt >= md.ntiles[mode_slot]) continue;        // (uniform per CTA)
     const int wc = md.wc, wr = kWarps / wc;
     const int tr = RPW * wr;
     const int64_t rb = lt / md.ncb, cb = lt % md.ncb;
@@ -578,7 +600,6 @@ tile_kernel(const __grid_constant__ Table tab, int mode_slot, int want_res) {
     const int64_t row0 = row_first + my_r;           // this warp's first row
     // rows of this tile that this warp handles (k = 0 .. nk-1 -> row0 + k*wr)
     const int nk = (int)max((int64_t)0, min((int64_t)RPW, (rows - row0 + wr - 1) / wr));
-    const bool res_on = !ACT && want_res != 0;
 
     // per-lane column data, as pairs: b_j and the inner factor (1/b_j, or b_j for ACT)
     f2 bj[NP], cm[NP];
@@ -594,11 +615,12 @@ tile_kernel(const __grid_constant__ Table tab, int mode_slot, int want_res) {
         else if (OS == SC_E8M0) cm[k] = make_float2(recip_pow2(b0), recip_pow2(b1));
         else cm[k] = make_float2(recip_approx(b0), recip_approx(b1));
     }
-    // row factors: lane k holds a and 1/a of the warp's k-th row (COL mode
-    // reads them per row instead, it has 64 rows per warp)
+    // row factors: lane k holds a and 1/a of the warp's k-th row (modes with
+    // 64 rows per warp read them per row instead)
+    constexpr bool kRowFactorPerRow = RPW > 32;
     float a_lane = 1.0f, ia_lane = 1.0f;
     const float *const pa = ACT ? nullptr : md.a;
-    if (MODE != MODE_COL && pa != nullptr && lane < nk) {
+    if (!kRowFactorPerRow && pa != nullptr && lane < nk) {
         a_lane = __ldg(pa + row0 + (int64_t)lane * wr);
         ia_lane = (OS == SC_E8M0) ? recip_pow2(a_lane) : recip_approx(a_lane);
     }
@@ -606,10 +628,11 @@ tile_kernel(const __grid_constant__ Table tab, int mode_slot, int want_res) {
     const float ts = (GS == SC_E4M3 && !ACT) ? tensor_scale_of(md) : 1.0f;
     const float inv_ts = 1.0f / ts;                 // ts is a power of two
 
-    f2 acc_p[NP], acc_e[NP];                         // COL accumulators
+    f2 acc_p[NP], acc_e[NP];                         // column accumulators
 #pragma unroll
     for (int k = 0; k < NP; ++k) { acc_p[k] = bcast(0.0f); acc_e[k] = bcast(0.0f); }
     f2 res2 = bcast(0.0f);
+    bool clamp_risk = false;                         // FUSED: exponent margin check
 
     // Each lane streams its own 16-byte chunk of the warp's rows through a
     // private ring of kRing shared-memory slots with cp.async (one commit
@@ -648,7 +671,7 @@ tile_kernel(const __grid_constant__ Table tab, int mode_slot, int want_res) {
         ck.raw = sm.ring[warp][u][lane];
         float a = 1.0f, ia = 1.0f;
         if (!ACT && pa != nullptr) {
-            if (MODE == MODE_COL) {
+            if (kRowFactorPerRow) {
                 a = __ldg(pa + row0 + (int64_t)k * wr);
                 ia = (OS == SC_E8M0) ? recip_pow2(a) : recip_approx(a);
             } else {
@@ -662,10 +685,29 @@ tile_kernel(const __grid_constant__ Table tab, int mode_slot, int want_res) {
         for (int j = 0; j < NP; ++j) z[j] = mul2(w[j], cm[j]);
         float s, s_eff;
         uint32_t nib;
-        Q::template run<NIB>(w, z, a, ia, bj, ts, inv_ts, tab.status, c, s, s_eff, nib);
-        if (MODE == MODE_ROW) {
+        bool nonzero;
+        if (FUSED) {
+            // Q(W / b): with power-of-two scales D_a Q(W / (a b)) equals it
+            // exactly, for the row's a before and after its update
+            Q::template run<NIB>(w, z, 1.0f, 1.0f, bj, ts, inv_ts, tab.status, c, s, s_eff, nib,
+                                 nonzero);
+            // ... as long as no group exponent reaches the E8M0 bounds:
+            // require |e(s) - e(a)| <= 120 (the row update may move e(a) by at
+            // most 6 more, which the row finalize checks)
+            const int es = (int)(__float_as_uint(s) >> 23) - 127;
+            const int ea = (int)(__float_as_uint(a) >> 23) - 127;
+            clamp_risk |= nonzero && (es - ea > 120 || es - ea < -120);
+        } else {
+            Q::template run<NIB>(w, z, a, ia, bj, ts, inv_ts, tab.status, c, s, s_eff, nib,
+                                 nonzero);
+        }
+        if (ROWSTAT) {
+            // the row statistics of the literal row step: R = Qhat D_b with
+            // Qhat = Q(W / (a b)); in FUSED mode Qhat = c * (s / a)
+            const float s_row = FUSED ? s_eff * ia : s_eff;
+            const float as = FUSED ? s_eff : a * s_eff;     // a * s_row
             f2 gn = bcast(0.0f), gd = bcast(0.0f);
-            const f2 nas = bcast(-(a * s_eff));
+            const f2 nas = bcast(-as);
 #pragma unroll
             for (int j = 0; j < NP; ++j) {
                 const f2 uq = mul2(c[j], bj[j]);
@@ -676,22 +718,48 @@ tile_kernel(const __grid_constant__ Table tab, int mode_slot, int want_res) {
                     res2 = fma2(d, d, res2);
                 }
             }
-            // this lane's share of row k, summed over lanes at the end of the tile
-            sm.red[(warp * RPW + k) * 33 + lane] =
-                make_float2((gn.x + gn.y) * s_eff, (gd.x + gd.y) * (s_eff * s_eff));
-        } else if (MODE == MODE_COL) {
-            const f2 as = bcast(a * s_eff);
+            const float2 share = make_float2((gn.x + gn.y) * s_row, (gd.x + gd.y) * (s_row * s_row));
+            if (MODE == MODE_ROW) {
+                // this lane's share of row k, summed over lanes at the end of the tile
+                sm.red[(warp * RPW + k) * 33 + lane] = share;
+            } else {
+                // batches of 8 rows: lane 2r + h adds the 16 shares of half h of
+                // the batch's row r in order, then the halves are added -- the
+                // same order as the row-statistics epilogue, so both modes give
+                // the same bits
+                sm.red[(warp * 8 + (k & 7)) * 33 + lane] = share;
+                if ((k & 7) == 7 || k == nk - 1) {
+                    __syncwarp();
+                    const int rr = (lane >> 1) & 7, hh = lane & 1;
+                    const float2 *p = &sm.red[(warp * 8 + rr) * 33 + 16 * hh];
+                    f2 acc = bcast(0.0f);
+                    if (lane < 16) {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) acc = __fadd2_rn(acc, p[j]);
+                    }
+                    acc.x += __shfl_xor_sync(0xffffffffu, acc.x, 1);
+                    acc.y += __shfl_xor_sync(0xffffffffu, acc.y, 1);
+                    const int kk = (k & ~7) + rr;
+                    if (lane < 16 && hh == 0 && kk <= k) sm.rtot[kk * kWarps + warp] = acc;
+                    __syncwarp();
+                }
+            }
+        }
+        if (COLSTAT) {
+            // the column statistics of the literal column step: S = D_a Qhat
+            const f2 as = bcast(FUSED ? s_eff : a * s_eff);
 #pragma unroll
             for (int j = 0; j < NP; ++j) {
                 const f2 v = mul2(c[j], as);
                 acc_p[j] = fma2(w[j], v, acc_p[j]);
                 acc_e[j] = fma2(v, v, acc_e[j]);
-                if (res_on) {
+                if (!FUSED && res_on) {
                     const f2 d = fma2(v, bj[j], neg2(w[j]));
                     res2 = fma2(d, d, res2);
                 }
             }
-        } else {
+        }
+        if (NIB) {
             const int64_t r = row0 + (int64_t)k * wr;
             if (MODE == MODE_PACK && res_on) {
                 const f2 nas = bcast(-(a * s_eff));
@@ -719,12 +787,14 @@ tile_kernel(const __grid_constant__ Table tab, int mode_slot, int want_res) {
     }
     }
     asm volatile("cp.async.wait_all;" ::: "memory");
+    if (FUSED && clamp_risk) atomicOr(&flags[0], 1u);
 
     // ---- tile epilogue ----
     if (MODE == MODE_ROW) {
         // (warp, row) pair p = t / 2 sums 16 lane shares per thread, then the
         // two halves; fixed order throughout
-        static_assert((2 * kWarps * RPW) % kThreads == 0, "every thread takes the same trips");
+        static_assert((2 * kWarps * RPW) % kThreads == 0 || MODE != MODE_ROW,
+                      "every thread takes the same trips");
         __syncthreads();
         for (int p2 = threadIdx.x; p2 < 2 * kWarps * RPW; p2 += kThreads) {
             const int pw = (p2 >> 1) / RPW, pk = (p2 >> 1) % RPW, h = p2 & 1;
@@ -737,8 +807,10 @@ tile_kernel(const __grid_constant__ Table tab, int mode_slot, int want_res) {
             }
             acc.x += __shfl_xor_sync(0xffffffffu, acc.x, 1);
             acc.y += __shfl_xor_sync(0xffffffffu, acc.y, 1);
-            if (h == 0) sm.part[pk * kWarps + pw] = acc;
+            if (h == 0) sm.rtot[pk * kWarps + pw] = acc;
         }
+    }
+    if (ROWSTAT) {
         __syncthreads();
         // rows of the tile: local row k*wr + r is warp-row r's k-th row
         for (int lr = threadIdx.x; lr < tr; lr += kThreads) {
@@ -747,7 +819,7 @@ tile_kernel(const __grid_constant__ Table tab, int mode_slot, int want_res) {
             if (row < rows) {
                 float num = 0.0f, den = 0.0f;
                 for (int c2 = 0; c2 < wc; ++c2) {          // fixed order over segments
-                    float2 p = sm.part[k * kWarps + r * wc + c2];
+                    float2 p = sm.rtot[k * kWarps + r * wc + c2];
                     num += p.x;
                     den += p.y;
                 }
@@ -755,7 +827,7 @@ tile_kernel(const __grid_constant__ Table tab, int mode_slot, int want_res) {
             }
         }
     }
-    if (MODE == MODE_COL) {
+    if (COLSTAT) {
         if (wr == 1) {
             if (col_ok) {
                 float2 *dst = md.colpart + rb * cols + col;
@@ -789,7 +861,7 @@ tile_kernel(const __grid_constant__ Table tab, int mode_slot, int want_res) {
             }
         }
     }
-    if ((MODE == MODE_ROW || MODE == MODE_COL || MODE == MODE_PACK) && res_on) {
+    if (!ACT && res_on) {
         double rd = (double)res2.x + (double)res2.y;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) rd += __shfl_xor_sync(0xffffffffu, rd, o);
@@ -802,6 +874,8 @@ tile_kernel(const __grid_constant__ Table tab, int mode_slot, int want_res) {
             slot[lt] = tot;
         }
     }
+    __syncthreads();                                 // shared memory reused by the next tile
+    }
 }
 
 // ------------------------------------------------------------------------- //
@@ -809,8 +883,12 @@ tile_kernel(const __grid_constant__ Table tab, int mode_slot, int want_res) {
 // ------------------------------------------------------------------------- //
 
 // a_i <- Pi(sum num / sum den) over the row's column blocks (fixed order).
+// With `flags` (an iteration of the fused path), a row whose power-of-two
+// scale moves by more than 2^6 raises flags[1]: the column step of the
+// iteration is then redone literally.
 template <int OS>
-__global__ void row_finalize_kernel(const __grid_constant__ Table tab, int64_t total_rows) {
+__global__ void row_finalize_kernel(const __grid_constant__ Table tab, int64_t total_rows,
+                                    unsigned int *flags) {
     for (int64_t g = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; g < total_rows;
          g += (int64_t)gridDim.x * blockDim.x) {
         const int mi = find_owner(tab, g, [](const MatDesc &d) { return d.row0; });
@@ -827,6 +905,11 @@ __global__ void row_finalize_kernel(const __grid_constant__ Table tab, int64_t t
             if (cl) atomicOr(tab.status, STATUS_RANGE);
         }
         if (!isfinite(num) || !isfinite(den)) atomicOr(tab.status, STATUS_NONFINITE);
+        if (flags != nullptr) {
+            const float a_old = md.a ? md.a[r] : 1.0f;
+            const int d = (int)((__float_as_uint(a) >> 23) & 0xFF) - (int)((__float_as_uint(a_old) >> 23) & 0xFF);
+            if (d > 6 || d < -6) atomicOr(&flags[1], 1u);
+        }
         md.a_out[r] = a;
         if (md.a_pre) md.a_pre[r] = pre;
     }
@@ -884,6 +967,46 @@ __global__ void mse_finalize_kernel(const __grid_constant__ Table tab, int row_s
         n = md.ntiles[MODE_COL];
     }
     if (dst == nullptr || (which == 0 && row_slot < 0)) return;
+    __shared__ double sm[256];
+    double acc = 0.0;
+    for (int64_t k = threadIdx.x; k < n; k += blockDim.x) acc += src[k];
+    sm[threadIdx.x] = acc;
+    __syncthreads();
+    for (int w = blockDim.x / 2; w > 0; w >>= 1) {
+        if (threadIdx.x < w) sm[threadIdx.x] += sm[threadIdx.x + w];
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) {
+        const double cnt = (double)md.rows * (double)md.cols;
+        *dst = cnt > 0 ? sm[0] / cnt : 0.0;
+    }
+}
+
+// MSE of an iteration of the fused path: the residual of its state comes
+// from the fused tiles (res_row, column-tile geometry) unless the row step
+// was redone literally (res_row, row-tile geometry); the half-step residual
+// equals it (power-of-two row scales leave D_a Qhat unchanged) unless the
+// column step was redone literally (res_col).
+__global__ void mse_finalize_fused_kernel(const __grid_constant__ Table tab,
+                                          const unsigned int *flags, unsigned int *next_flags,
+                                          int idx) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) { next_flags[0] = 0u; next_flags[1] = 0u; }
+    const int mi = blockIdx.x >> 1, which = blockIdx.x & 1;
+    const MatDesc &md = tab.get(mi);
+    const bool lit_row = flags[0] != 0, lit_col = (flags[0] | flags[1]) != 0;
+    double *dst;
+    const double *src;
+    int64_t n;
+    if (which == 0) {
+        dst = md.mse_trace ? md.mse_trace + idx : nullptr;
+        src = md.res_row;
+        n = lit_row ? md.ntiles[MODE_ROW] : md.ntiles[MODE_COL];
+    } else {
+        dst = md.mse_half ? md.mse_half + idx : nullptr;
+        src = lit_col ? md.res_col : md.res_row;
+        n = md.ntiles[MODE_COL];
+    }
+    if (dst == nullptr) return;
     __shared__ double sm[256];
     double acc = 0.0;
     for (int64_t k = threadIdx.x; k < n; k += blockDim.x) acc += src[k];

@@ -11,12 +11,15 @@ namespace dq {
 
 struct TileLaunch {
     Table tab;
-    int64_t grid;       // number of tiles (one CTA each)
+    int64_t grid;       // CTAs launched (tiles are visited grid-stride)
+    int64_t tiles;      // number of tiles
     int mode;           // MODE_*
     int slot;           // tile table slot: 0 ROW, 1 COL, 2 PACK/ACT
     int f32;            // 1: float32 input, 0: bfloat16
     int G;              // 16, 32, 64
     int want_res;       // 1: accumulate the residual (an MSE output is wanted)
+    unsigned int *flags;  // fused-path flags of the iteration (or NULL)
+    int gate;           // 0 always run; 1 run if flags[0]; 2 run if flags[0] | flags[1]
     cudaStream_t stream;
 };
 
@@ -55,14 +58,15 @@ cudaError_t launch_tile_one(const TileLaunch &L) {
             done[dev] = true;
         }
     }
-    kern<<<dim3((unsigned)L.grid), dim3(kThreads), bytes, L.stream>>>(L.tab, L.slot, L.want_res);
+    kern<<<dim3((unsigned)L.grid), dim3(kThreads), bytes, L.stream>>>(L.tab, L.slot, L.want_res,
+                                                                      L.tiles, L.flags, L.gate);
     return cudaGetLastError();
 }
 
 // Dispatch over mode, dtype and G for one format set (used by each unit).
 template <int CODES, int GS, int OS>
 cudaError_t launch_tile_combo(const TileLaunch &L) {
-    if (L.grid <= 0) return cudaSuccess;
+    if (L.grid <= 0 || L.tiles <= 0) return cudaSuccess;
 #define DQ_TILE(MODE, TIN, GG) return launch_tile_one<CODES, GS, OS, MODE, TIN, GG>(L)
 #define DQ_BY_G(MODE, TIN)                          \
     switch (L.G) {                                  \
@@ -76,6 +80,9 @@ cudaError_t launch_tile_combo(const TileLaunch &L) {
     switch (L.mode) {
         case MODE_ROW: DQ_BY_T(MODE_ROW);
         case MODE_COL: DQ_BY_T(MODE_COL);
+        case MODE_FUSED:
+            if constexpr (GS == SC_E8M0 && OS == SC_E8M0) { DQ_BY_T(MODE_FUSED); }
+            return cudaErrorInvalidValue;
         case MODE_PACK: DQ_BY_T(MODE_PACK);
         case MODE_ACT:
             if (L.f32) return cudaErrorInvalidValue;

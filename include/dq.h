@@ -59,7 +59,8 @@ typedef enum dq_status {
     DQ_ERR_ARG = -1,            /* null pointer, bad enum, T < 0, n < 0 */
     DQ_ERR_SHAPE = -2,          /* cols % G != 0, negative size */
     DQ_ERR_FORMAT = -3,         /* unknown preset or unsupported combination */
-    DQ_ERR_NONFINITE = -4,      /* (device flag) NaN or Inf met in W or X */
+    DQ_ERR_NONFINITE = -4,      /* (device flag) NaN or Inf in W or X, or W/(a b)
+                                   beyond the float32 range */
     DQ_ERR_RANGE = -5,          /* (device flag) an outer scale hit the set's bound */
     DQ_ERR_CUDA = -6,           /* a CUDA runtime call failed */
     DQ_ERR_WORKSPACE = -7,      /* workspace null or smaller than dq_workspace_size */
@@ -193,7 +194,8 @@ DQ_API dq_status dq_act_rescale_quant(const void *X, int64_t tokens, int64_t K, 
                                dq_stream stream);
 
 /* Synchronise `stream`, read and clear the device flags raised by earlier
- * calls on this device: DQ_ERR_NONFINITE if an input held NaN/Inf,
+ * calls on this device: DQ_ERR_NONFINITE if an input held NaN/Inf (or
+ * scaling it by the outer scales left the float32 range),
  * DQ_ERR_RANGE if an outer scale was clamped at its set's bound, DQ_OK
  * otherwise (NONFINITE wins when both are set).  The flags are one word per
  * device shared by all streams. */
@@ -229,7 +231,7 @@ DQ_API dq_status dq_solve_dual_scale_noalloc(const void *W, int32_t dtype, int64
 /* Measurement support (no counterpart in the method).  dq_kernel_timing(1)
  * makes every tile-kernel launch of the library record a CUDA event pair on
  * its own stream (kind 0 row statistics, 1 column statistics, 2 pack,
- * 3 activation); dq_kernel_time synchronises those events and returns (and
+ * 3 activation, 4 row and column statistics in one pass); dq_kernel_time synchronises those events and returns (and
  * clears) the summed milliseconds and the launch count of one kind.
  * dq_launch_count returns the number of kernels this library has launched in
  * the process so far (all kinds, including finalize kernels). */

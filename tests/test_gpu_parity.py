@@ -284,8 +284,10 @@ def test_solve_smollm2_decoder0_batched_with_all_30():
     # these solves stay at RTN: no b_j leaves 1, in the oracle as well)
     final = np.array([np64(o["mse_trace"])[-1] for o in outs])
     start = np.array([np64(o["mse_trace"])[0] for o in outs])
-    assert np.all(final <= start)
-    assert np.any(final < start)
+    # (start and end residuals are summed over different tile shapes: allow
+    # float32 summation noise)
+    assert np.all(final <= start * (1 + 1e-6))
+    assert np.any(final < start * (1 - 1e-4))
 
 
 def test_solve_is_deterministic():
@@ -337,3 +339,67 @@ def test_nonfinite_input_sets_device_flag(bad):
     assert dq.last_device_status() == 0      # read clears
     dq.quantize(W, fl)
     assert dq.last_device_status() == -4
+
+
+# --------------------------------------------------------------------------- #
+# MX formats: one-pass iterations against the literal steps
+# --------------------------------------------------------------------------- #
+
+def _literal_sequence(W, fl, T, a0, b0):
+    """T iterations through the step entry points (literal row pass, then
+    literal column pass with the new a)."""
+    a, b = a0.clone(), b0.clone()
+    for _ in range(T):
+        a, _, _ = dq.row_update(W, fl, a, b)
+        b, _, _ = dq.col_update(W, fl, a, b)
+    return a, b
+
+
+@pytest.mark.parametrize("name", ["mxfp4", "mxint4"])
+@pytest.mark.parametrize("extreme", [None, -124, 126])
+def test_mx_solve_equals_the_literal_steps(name, extreme):
+    # With power-of-two scales the solve takes both statistics of an
+    # iteration from one pass; the result must equal the literal row and
+    # column steps bit for bit.  extreme = -124: rows whose a0 = 2^-124 still
+    # keep every group exponent in range (no fallback); extreme = 126: group
+    # exponents of those rows clamp, so the iteration falls back to the
+    # literal passes.
+    fl = dq.format_preset(name)
+    fo = PRESET_COMBOS[name](32)
+    rows, cols = 300, 2240
+    W = _weights(rows, cols, torch.bfloat16, key=23).cuda()
+    a0 = torch.ones(rows, device="cuda")
+    if extreme is not None:
+        a0[::7] = 2.0 ** extreme
+    b0 = torch.ones(cols, device="cuda")
+    T = 4
+    o = dq.solve_dual_scale(W, fl, T, a0=a0, b0=b0)
+    a, b = _literal_sequence(W, fl, T, a0, b0)
+    torch.cuda.synchronize()
+    assert torch.equal(o["a"], a)
+    assert torch.equal(o["b"], b)
+    tr, hf = np64(o["mse_trace"]), np64(o["mse_half"])
+    if extreme is None:
+        r = O.solve(np64(W), fo, T)
+        assert np.max(np.abs(tr - r["mse_trace"]) / r["mse_trace"]) < 1e-4
+        # a power-of-two row step leaves D_a Qhat unchanged: half == trace
+        assert np.array_equal(hf, tr[:T])
+        assert dq.last_device_status() == 0
+    else:
+        # extreme scales can push float32 statistics out of range; the device
+        # reports it (and the literal steps agree with the solve all the same)
+        assert dq.last_device_status() in (0, -4, -5)
+
+
+def test_batched_mx_solve_equals_single_solves():
+    wl = synth.WORKLOADS["llama31_70b_decoder_mxfp4_g32"]
+    fl = dq.format_preset(wl.fmt, wl.group)
+    Ws = [synth.weight(wl, 0, i, device="cuda", rows=r, cols=c)
+          for i, (r, c) in enumerate([(512, 1024), (96, 2048), (300, 512)])]
+    outs = dq.solve_dual_scale_batched(Ws, fl, 3)
+    for W, o in zip(Ws, outs):
+        s = dq.solve_dual_scale(W, fl, 3)
+        torch.cuda.synchronize()
+        for k in ("codes", "gscales", "a", "b"):
+            assert torch.equal(o[k], s[k]), k
+        assert torch.equal(o["mse_trace"], s["mse_trace"])
