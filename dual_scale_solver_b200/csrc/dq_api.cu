@@ -208,6 +208,7 @@ unsigned grid_for(int64_t n, int block) {
 
 struct Launcher {
     Table tab;
+    const MatDesc *host_table = nullptr;   // host copy of tab.dev's entries
     int combo, G;
     bool f32;
     float qmax;
@@ -259,10 +260,18 @@ struct Launcher {
     }
     dq_status col_finalize() {
         if (total_cols == 0) return DQ_OK;
+        // one block per 32-column slab (slabs of all matrices, in order)
+        int64_t slabs = 0;
+        for (int i = 0; i < tab.n; ++i) {
+            const MatDesc &d = tab.dev ? host_table[i] : tab.one;
+            slabs += (d.cols + kColFinCols - 1) / kColFinCols;
+        }
+        const unsigned grid = (unsigned)std::max<int64_t>(1, std::min<int64_t>(slabs, 148 * 16));
+        const int threads = kColFinCols * kColFinSlices;
         if (outer_of(combo) == SC_E8M0)
-            col_finalize_kernel<SC_E8M0><<<grid_for(total_cols, 256), 256, 0, st>>>(tab, total_cols);
+            col_finalize_kernel<SC_E8M0><<<grid, threads, 0, st>>>(tab, total_cols);
         else
-            col_finalize_kernel<SC_BF16><<<grid_for(total_cols, 256), 256, 0, st>>>(tab, total_cols);
+            col_finalize_kernel<SC_BF16><<<grid, threads, 0, st>>>(tab, total_cols);
         DQ_CUDA(cudaGetLastError());
         count_launches(1);
         return DQ_OK;
@@ -368,6 +377,7 @@ dq_status solve_impl(int32_t n, const dq_matrix *mats, int32_t dtype, const dq_f
     }
     Launcher L;
     L.tab.dev = dev_table;
+    L.host_table = t_table.data();
     L.tab.n = n;
     L.tab.status = status;
     if (n == 1) L.tab.one = t_table[0];

@@ -915,31 +915,61 @@ __global__ void row_finalize_kernel(const __grid_constant__ Table tab, int64_t t
     }
 }
 
-// b_j <- Pi(sum P / sum E) over the column's row blocks (fixed order).
+// b_j <- Pi(sum P / sum E) over the column's row blocks.  A block handles 32
+// consecutive columns of one matrix with 8 slices of row blocks (slice s
+// sums row blocks s, s+8, ... in order, in double); the slices are then
+// added in order: a fixed summation order, independent of the launch.
+constexpr int kColFinCols = 32, kColFinSlices = 8;
 template <int OS>
-__global__ void col_finalize_kernel(const __grid_constant__ Table tab, int64_t total_cols) {
-    for (int64_t g = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; g < total_cols;
-         g += (int64_t)gridDim.x * blockDim.x) {
-        const int mi = find_owner(tab, g, [](const MatDesc &d) { return d.col0; });
+__global__ void __launch_bounds__(kColFinCols * kColFinSlices)
+col_finalize_kernel(const __grid_constant__ Table tab, int64_t total_cols) {
+    __shared__ double sp[kColFinSlices][kColFinCols], se[kColFinSlices][kColFinCols];
+    const int cl = threadIdx.x % kColFinCols, sl = threadIdx.x / kColFinCols;
+    // blocks enumerate 32-column slabs of every matrix in turn
+    for (int64_t slab = blockIdx.x; ; slab += gridDim.x) {
+        // matrix of this slab: slabs of matrix i start at ceil-sum of cols / 32
+        int mi = -1;
+        int64_t c0 = 0;
+        {
+            int64_t acc = 0;
+            for (int i = 0; i < tab.n; ++i) {
+                const int64_t ns = (tab.get(i).cols + kColFinCols - 1) / kColFinCols;
+                if (slab < acc + ns) { mi = i; c0 = (slab - acc) * kColFinCols; break; }
+                acc += ns;
+            }
+        }
+        if (mi < 0) break;                                 // uniform per block
         const MatDesc &md = tab.get(mi);
-        const int64_t c = g - md.col0;
-        const int64_t nrb = md.ntiles[MODE_COL] / md.ncb;
+        const int64_t c = c0 + cl;
+        const bool ok = c < md.cols;
+        const int64_t nrb = md.ntiles[MODE_COL] / max(md.ncb, 1);
         double p = 0.0, e = 0.0;
-        for (int64_t k = 0; k < nrb; ++k) {
-            float2 v = md.colpart[k * md.cols + c];
-            p += v.x;
-            e += v.y;
+        if (ok) {
+#pragma unroll 4
+            for (int64_t k = sl; k < nrb; k += kColFinSlices) {
+                const float2 v = md.colpart[k * md.cols + c];
+                p += v.x;
+                e += v.y;
+            }
         }
-        float b = 1.0f, pre = __int_as_float(0x7fc00000);
-        if (e > 0.0) {
-            pre = (float)(p / e);
-            bool cl;
-            b = project_outer<OS>(pre, cl);
-            if (cl) atomicOr(tab.status, STATUS_RANGE);
+        sp[sl][cl] = p;
+        se[sl][cl] = e;
+        __syncthreads();
+        if (sl == 0 && ok) {
+            double pt = 0.0, et = 0.0;
+            for (int q = 0; q < kColFinSlices; ++q) { pt += sp[q][cl]; et += se[q][cl]; }
+            float b = 1.0f, pre = __int_as_float(0x7fc00000);
+            if (et > 0.0) {
+                pre = (float)(pt / et);
+                bool cl2;
+                b = project_outer<OS>(pre, cl2);
+                if (cl2) atomicOr(tab.status, STATUS_RANGE);
+            }
+            if (!isfinite(pt) || !isfinite(et)) atomicOr(tab.status, STATUS_NONFINITE);
+            md.b_out[c] = b;
+            if (md.b_pre) md.b_pre[c] = pre;
         }
-        if (!isfinite(p) || !isfinite(e)) atomicOr(tab.status, STATUS_NONFINITE);
-        md.b_out[c] = b;
-        if (md.b_pre) md.b_pre[c] = pre;
+        __syncthreads();
     }
 }
 
