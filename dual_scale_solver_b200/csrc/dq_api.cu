@@ -119,7 +119,7 @@ Geom geometry(int64_t rows, int64_t cols, bool f32) {
     g.wc = wc;
     g.ncb = (int)((nseg + wc - 1) / wc);
     const int wr = kWarps / wc;
-    const int rpw[3] = {16, 64, 16};
+    const int rpw[3] = {16, 128, 16};
     for (int m = 0; m < 3; ++m) {
         g.tr[m] = rpw[m] * wr;
         const int64_t nrb = (rows + g.tr[m] - 1) / g.tr[m];
@@ -225,7 +225,7 @@ struct Launcher {
         L.mode = mode;
         L.slot = (mode == MODE_ACT) ? 2 : (mode == MODE_FUSED ? 1 : mode);
         L.tiles = tiles[L.slot];
-        L.grid = gate ? std::min<int64_t>(L.tiles, 148 * 3) : L.tiles;
+        L.grid = gate ? std::min<int64_t>(L.tiles, 148) : L.tiles;
         L.f32 = f32 ? 1 : 0;
         L.G = G;
         L.want_res = want_res ? 1 : 0;

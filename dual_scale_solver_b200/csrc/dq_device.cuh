@@ -31,7 +31,7 @@ enum { STATUS_NONFINITE = 1u, STATUS_RANGE = 2u };
 
 constexpr int kWarps = 8;            // warps per CTA of the tile kernel
 constexpr int kThreads = 32 * kWarps;
-constexpr int kRowsPerWarp[5] = {16, 64, 16, 16, 64};   // per mode
+constexpr int kRowsPerWarp[5] = {16, 128, 16, 16, 128};   // per mode
 constexpr int kRing = 4;             // cp.async ring slots per lane (rows in flight + 1)
 constexpr float kBf16Max = 3.38953138925153547590470800371487866880e+38f;  // (2-2^-7)*2^127
 constexpr float kMinNormal = 1.17549435082228750796873653722224568e-38f;    // 2^-126
@@ -616,7 +616,7 @@ tile_kernel(const __grid_constant__ Table tab, int mode_slot, int want_res, int6
         else cm[k] = make_float2(recip_approx(b0), recip_approx(b1));
     }
     // row factors: lane k holds a and 1/a of the warp's k-th row (modes with
-    // 64 rows per warp read them per row instead)
+    // more than 32 rows per warp read them per row instead)
     constexpr bool kRowFactorPerRow = RPW > 32;
     float a_lane = 1.0f, ia_lane = 1.0f;
     const float *const pa = ACT ? nullptr : md.a;
