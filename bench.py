@@ -207,6 +207,32 @@ def run_reference(args, wl, rank, world):
 
 
 # --------------------------------------------------------------------------- #
+# Multi-GPU plumbing (weak scaling, no collective on the data path)
+# --------------------------------------------------------------------------- #
+
+def decoder_of(rank: int) -> int:
+    """Decoder of the model that rank `rank` solves: every rank a different
+    one, so per-GPU work is fixed as the number of GPUs grows."""
+    return rank
+
+
+def max_over_ranks(value: float, device=None) -> float:
+    """Max of a per-rank timing over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as tdist
+    if not (tdist.is_available() and tdist.is_initialized()) or tdist.get_world_size() == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(elements_per_rank: int, T: int, world: int, ms_per_step: float) -> float:
+    """Weight-elements per second per BCD iteration over all ranks."""
+    return world * elements_per_rank * T / (ms_per_step / 1e3)
+
+
+# --------------------------------------------------------------------------- #
 # GPU arm
 # --------------------------------------------------------------------------- #
 
@@ -225,7 +251,7 @@ def run_ours(args, wl, rank, world, local_rank):
     build.build()
 
     # weak scaling: rank r solves decoder r of the model (seeded per decoder)
-    decoder = rank
+    decoder = decoder_of(rank)
     idx = [args.only] if args.only >= 0 else range(len(wl.linears))
     Ws = [synth.weight(wl, decoder, i, device=dev) for i in idx]
     fmt = dq.format_preset(wl.fmt, wl.group)
@@ -281,13 +307,10 @@ def run_ours(args, wl, rank, world, local_rank):
     kt = {k: dq.kernel_time(k) for k in range(5)}
     dq.kernel_timing(False)
     clk = clocks.stop()
-    if dist:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, dev)
 
     ms_step = ms / args.steps
-    value = world * E * T / (ms_step / 1e3)
+    value = whole_job_rate(E, T, world, ms_step)
 
     # dominant tile kernel and its roofline (HBM: it streams W once per launch)
     names = {0: "row_stats", 1: "col_stats", 2: "pack", 3: "act_quant", 4: "fused_row_col_stats"}
@@ -347,12 +370,8 @@ def run_ours(args, wl, rank, world, local_rank):
         f1.record(stream)
         torch.cuda.synchronize(dev)
         barrier()
-        ems = f0.elapsed_time(f1)
-        if dist:
-            t = torch.tensor([ems], dtype=torch.float64, device=dev)
-            tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
-            ems = float(t.item())
-        e2e = {"value": world * E * T / (ems / args.steps / 1e3), "unit": UNIT,
+        ems = max_over_ranks(f0.elapsed_time(f1), dev)
+        e2e = {"value": whole_job_rate(E, T, world, ems / args.steps), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "ms_per_step": ems / args.steps}
 
