@@ -248,12 +248,14 @@ struct Launcher {
         }
         return DQ_OK;
     }
-    dq_status row_finalize(unsigned int *flags = nullptr) {
+    dq_status row_finalize(unsigned int *flags = nullptr, unsigned int *next_flags = nullptr) {
         if (total_rows == 0) return DQ_OK;
         if (outer_of(combo) == SC_E8M0)
-            row_finalize_kernel<SC_E8M0><<<grid_for(total_rows, 256), 256, 0, st>>>(tab, total_rows, flags);
+            row_finalize_kernel<SC_E8M0><<<grid_for(total_rows, 256), 256, 0, st>>>(tab, total_rows,
+                                                                                  flags, next_flags);
         else
-            row_finalize_kernel<SC_BF16><<<grid_for(total_rows, 256), 256, 0, st>>>(tab, total_rows, flags);
+            row_finalize_kernel<SC_BF16><<<grid_for(total_rows, 256), 256, 0, st>>>(tab, total_rows,
+                                                                                  flags, next_flags);
         DQ_CUDA(cudaGetLastError());
         count_launches(1);
         return DQ_OK;
@@ -291,9 +293,11 @@ struct Launcher {
     dq_status iteration(int t, bool fused, unsigned int *flag_slots, bool want_trace,
                         bool want_half) {
         dq_status s;
-        // iteration t uses flag slot t % 2; its MSE kernel clears the other slot
-        unsigned int *flags = flag_slots + 2 * (t & 1);
-        unsigned int *next = flag_slots + 2 * ((t + 1) & 1);
+        // iteration t uses flag slot t % 3; its row finalize may raise the
+        // next slot, its MSE kernel clears the slot after that
+        unsigned int *flags = flag_slots + 2 * (t % 3);
+        unsigned int *next = flag_slots + 2 * ((t + 1) % 3);
+        unsigned int *clear = flag_slots + 2 * ((t + 2) % 3);
         if (!fused) {
             if ((s = tiles_pass(MODE_ROW, want_trace)) != DQ_OK) return s;
             if ((s = row_finalize()) != DQ_OK) return s;
@@ -303,10 +307,10 @@ struct Launcher {
         }
         if ((s = tiles_pass(MODE_FUSED, want_trace || want_half, flags, 0)) != DQ_OK) return s;
         if ((s = tiles_pass(MODE_ROW, want_trace, flags, 1)) != DQ_OK) return s;
-        if ((s = row_finalize(flags)) != DQ_OK) return s;
+        if ((s = row_finalize(flags, next)) != DQ_OK) return s;
         if ((s = tiles_pass(MODE_COL, want_half, flags, 2)) != DQ_OK) return s;
         if ((s = col_finalize()) != DQ_OK) return s;
-        mse_finalize_fused_kernel<<<2 * tab.n, 256, 0, st>>>(tab, flags, next, t);
+        mse_finalize_fused_kernel<<<2 * tab.n, 256, 0, st>>>(tab, flags, clear, t);
         DQ_CUDA(cudaGetLastError());
         count_launches(1);
         return DQ_OK;
@@ -351,7 +355,7 @@ dq_status solve_impl(int32_t n, const dq_matrix *mats, int32_t dtype, const dq_f
 
     Carve cv{static_cast<char *>(workspace), static_cast<char *>(workspace) + ws_bytes};
     MatDesc *dev_table = n > 1 ? cv.take<MatDesc>((size_t)n * sizeof(MatDesc)) : nullptr;
-    unsigned int *flags = cv.take<unsigned int>(256);     // fused-path flags: 2 slots x 2 words
+    unsigned int *flags = cv.take<unsigned int>(256);     // fused-path flags: 3 slots x 2 words
     t_table.assign(n, MatDesc{});
     int64_t tile_base[3] = {0, 0, 0}, row_base = 0, col_base = 0;
     for (int i = 0; i < n; ++i) {
@@ -407,8 +411,11 @@ dq_status solve_impl(int32_t n, const dq_matrix *mats, int32_t dtype, const dq_f
     tensor_scale_kernel<<<(n + 127) / 128, 128, 0, st>>>(L.tab, fi.qmax, fmt->tensor_scale_auto);
     DQ_CUDA(cudaGetLastError());
     count_launches(1);
+    const bool fused = fused_ok(fi.combo) && T > 0;
+    if (fused) DQ_CUDA(cudaMemsetAsync(flags, 0, 6 * sizeof(unsigned int), st));
     if (row_base + col_base > 0) {
-        init_state_kernel<<<grid_for(row_base + col_base, 256), 256, 0, st>>>(L.tab, row_base, col_base);
+        init_state_kernel<<<grid_for(row_base + col_base, 256), 256, 0, st>>>(
+            L.tab, row_base, col_base, fused ? flags : nullptr);
         DQ_CUDA(cudaGetLastError());
         count_launches(1);
     }
@@ -417,8 +424,6 @@ dq_status solve_impl(int32_t n, const dq_matrix *mats, int32_t dtype, const dq_f
         want_trace |= mats[i].mse_trace != nullptr;
         want_half |= mats[i].mse_half != nullptr;
     }
-    const bool fused = fused_ok(fi.combo);
-    if (fused && T > 0) DQ_CUDA(cudaMemsetAsync(flags, 0, 4 * sizeof(unsigned int), st));
     for (int t = 0; t < T; ++t)
         if ((s = L.iteration(t, fused, flags, want_trace, want_half)) != DQ_OK) return s;
     if ((s = L.tiles_pass(MODE_PACK, want_trace)) != DQ_OK) return s;
@@ -880,7 +885,7 @@ extern "C" dq_status dq_solve_dual_scale_noalloc(const void *W, int32_t dtype, i
     DQ_CUDA(cudaGetLastError());
     count_launches(1);
     if (rb + cb > 0) {
-        init_state_kernel<<<grid_for(rb + cb, 256), 256, 0, st>>>(L.tab, rb, cb);
+        init_state_kernel<<<grid_for(rb + cb, 256), 256, 0, st>>>(L.tab, rb, cb, nullptr);
         DQ_CUDA(cudaGetLastError());
         count_launches(1);
     }

@@ -670,7 +670,7 @@ tile_kernel(const __grid_constant__ Table tab, int mode_slot, int want_res, int6
         CK ck;
         ck.raw = sm.ring[warp][u][lane];
         float a = 1.0f, ia = 1.0f;
-        if (!ACT && pa != nullptr) {
+        if (!ACT && !FUSED && pa != nullptr) {
             if (kRowFactorPerRow) {
                 a = __ldg(pa + row0 + (int64_t)k * wr);
                 ia = (OS == SC_E8M0) ? recip_pow2(a) : recip_approx(a);
@@ -688,24 +688,25 @@ tile_kernel(const __grid_constant__ Table tab, int mode_slot, int want_res, int6
         bool nonzero;
         if (FUSED) {
             // Q(W / b): with power-of-two scales D_a Q(W / (a b)) equals it
-            // exactly, for the row's a before and after its update
+            // exactly, for the row's a before and after its update, as long
+            // as no group exponent of either reaches the E8M0 bounds: here
+            // |e(s)| <= 100 for every non-zero group; the row finalize keeps
+            // |e(a)| <= 20 (old) and <= 26 (new)
             Q::template run<NIB>(w, z, 1.0f, 1.0f, bj, ts, inv_ts, tab.status, c, s, s_eff, nib,
                                  nonzero);
-            // ... as long as no group exponent reaches the E8M0 bounds:
-            // require |e(s) - e(a)| <= 120 (the row update may move e(a) by at
-            // most 6 more, which the row finalize checks)
             const int es = (int)(__float_as_uint(s) >> 23) - 127;
-            const int ea = (int)(__float_as_uint(a) >> 23) - 127;
-            clamp_risk |= nonzero && (es - ea > 120 || es - ea < -120);
+            clamp_risk |= nonzero && (es > 100 || es < -100);
         } else {
             Q::template run<NIB>(w, z, a, ia, bj, ts, inv_ts, tab.status, c, s, s_eff, nib,
                                  nonzero);
         }
         if (ROWSTAT) {
             // the row statistics of the literal row step: R = Qhat D_b with
-            // Qhat = Q(W / (a b)); in FUSED mode Qhat = c * (s / a)
-            const float s_row = FUSED ? s_eff * ia : s_eff;
-            const float as = FUSED ? s_eff : a * s_eff;     // a * s_row
+            // Qhat = Q(W / (a b)); FUSED writes them for a = 1 and the row
+            // finalize scales the sums by 1/a and 1/a^2 (exact: a is a power
+            // of two), which gives the literal bits
+            const float s_row = s_eff;
+            const float as = FUSED ? s_eff : a * s_eff;
             f2 gn = bcast(0.0f), gd = bcast(0.0f);
             const f2 nas = bcast(-as);
 #pragma unroll
@@ -883,12 +884,15 @@ tile_kernel(const __grid_constant__ Table tab, int mode_slot, int want_res, int6
 // ------------------------------------------------------------------------- //
 
 // a_i <- Pi(sum num / sum den) over the row's column blocks (fixed order).
-// With `flags` (an iteration of the fused path), a row whose power-of-two
-// scale moves by more than 2^6 raises flags[1]: the column step of the
-// iteration is then redone literally.
+// With `flags` (an iteration of the one-pass MX path): unless flags[0] says
+// the literal row pass ran, the sums were taken for a = 1 and are scaled by
+// 1/a_old and 1/a_old^2 here; a new scale with |e(a)| > 26 raises flags[1]
+// (the column step is redone literally) and one with |e(a)| > 20 raises the
+// next iteration's flags[0] (its row step is done literally).
 template <int OS>
 __global__ void row_finalize_kernel(const __grid_constant__ Table tab, int64_t total_rows,
-                                    unsigned int *flags) {
+                                    unsigned int *flags, unsigned int *next_flags) {
+    const bool scale_old = flags != nullptr && flags[0] == 0;
     for (int64_t g = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; g < total_rows;
          g += (int64_t)gridDim.x * blockDim.x) {
         const int mi = find_owner(tab, g, [](const MatDesc &d) { return d.row0; });
@@ -897,6 +901,11 @@ __global__ void row_finalize_kernel(const __grid_constant__ Table tab, int64_t t
         double num = 0.0, den = 0.0;
         const float2 *p = md.rowpart + r * md.ncb;
         for (int k = 0; k < md.ncb; ++k) { num += p[k].x; den += p[k].y; }
+        if (scale_old) {
+            const double ia = (double)recip_pow2(md.a ? md.a[r] : 1.0f);
+            num *= ia;
+            den *= ia * ia;
+        }
         float a = 1.0f, pre = __int_as_float(0x7fc00000);
         if (den > 0.0) {
             pre = (float)(num / den);
@@ -906,9 +915,9 @@ __global__ void row_finalize_kernel(const __grid_constant__ Table tab, int64_t t
         }
         if (!isfinite(num) || !isfinite(den)) atomicOr(tab.status, STATUS_NONFINITE);
         if (flags != nullptr) {
-            const float a_old = md.a ? md.a[r] : 1.0f;
-            const int d = (int)((__float_as_uint(a) >> 23) & 0xFF) - (int)((__float_as_uint(a_old) >> 23) & 0xFF);
-            if (d > 6 || d < -6) atomicOr(&flags[1], 1u);
+            const int ea = (int)((__float_as_uint(a) >> 23) & 0xFF) - 127;
+            if (ea > 26 || ea < -26) atomicOr(&flags[1], 1u);
+            if (ea > 20 || ea < -20) atomicOr(&next_flags[0], 1u);
         }
         md.a_out[r] = a;
         if (md.a_pre) md.a_pre[r] = pre;
@@ -1053,14 +1062,22 @@ __global__ void mse_finalize_fused_kernel(const __grid_constant__ Table tab,
 }
 
 // Initial state: a <- a0 or 1, b <- b0 or 1 (rows then columns, all matrices).
-__global__ void init_state_kernel(const __grid_constant__ Table tab, int64_t total_rows, int64_t total_cols) {
+// With `flags` (one-pass MX path): an initial |e(a)| > 20 makes iteration 0
+// take its row step literally.
+__global__ void init_state_kernel(const __grid_constant__ Table tab, int64_t total_rows,
+                                  int64_t total_cols, unsigned int *flags) {
     for (int64_t g = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; g < total_rows + total_cols;
          g += (int64_t)gridDim.x * blockDim.x) {
         if (g < total_rows) {
             const int mi = find_owner(tab, g, [](const MatDesc &d) { return d.row0; });
             const MatDesc &md = tab.get(mi);
             const int64_t r = g - md.row0;
-            md.a_out[r] = md.a0 ? md.a0[r] : 1.0f;
+            const float a = md.a0 ? md.a0[r] : 1.0f;
+            md.a_out[r] = a;
+            if (flags != nullptr) {
+                const int ea = (int)((__float_as_uint(a) >> 23) & 0xFF) - 127;
+                if (ea > 20 || ea < -20) atomicOr(&flags[0], 1u);
+            }
         } else {
             const int64_t gc = g - total_rows;
             const int mi = find_owner(tab, gc, [](const MatDesc &d) { return d.col0; });
