@@ -210,10 +210,11 @@ def run_reference(args, wl, rank, world):
 # Multi-GPU plumbing (weak scaling, no collective on the data path)
 # --------------------------------------------------------------------------- #
 
-def decoder_of(rank: int) -> int:
-    """Decoder of the model that rank `rank` solves: every rank a different
-    one, so per-GPU work is fixed as the number of GPUs grows."""
-    return rank
+def decoders_of(rank: int, per_rank: int) -> list:
+    """Decoders that rank `rank` solves: every rank its own block of
+    `per_rank` seeded decoders (the workload's decoder count), so per-GPU work
+    is fixed as the number of GPUs grows."""
+    return list(range(rank * per_rank, (rank + 1) * per_rank))
 
 
 def max_over_ranks(value: float, device=None) -> float:
@@ -250,10 +251,9 @@ def run_ours(args, wl, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     build.build()
 
-    # weak scaling: rank r solves decoder r of the model (seeded per decoder)
-    decoder = decoder_of(rank)
+    # weak scaling: rank r solves its own block of decoders (seeded per decoder)
     idx = [args.only] if args.only >= 0 else range(len(wl.linears))
-    Ws = [synth.weight(wl, decoder, i, device=dev) for i in idx]
+    Ws = [synth.weight(wl, d, i, device=dev) for d in decoders_of(rank, wl.decoders) for i in idx]
     fmt = dq.format_preset(wl.fmt, wl.group)
     act = None if args.no_act else wl.act
     X = synth.activation(wl, device=dev) if act else None

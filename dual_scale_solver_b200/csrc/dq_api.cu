@@ -119,7 +119,12 @@ Geom geometry(int64_t rows, int64_t cols, bool f32) {
     g.wc = wc;
     g.ncb = (int)((nseg + wc - 1) / wc);
     const int wr = kWarps / wc;
-    const int rpw[3] = {16, 128, 16};
+    // rows per warp: 16 for row statistics and packing; 128 for column
+    // statistics (fewer partial sums), reduced for short matrices so that
+    // they still make about 16 row blocks
+    int rpw_col = 16;
+    while (rpw_col < 128 && 2 * rpw_col <= rows / (wr * 16)) rpw_col *= 2;
+    const int rpw[3] = {16, rpw_col, 16};
     for (int m = 0; m < 3; ++m) {
         g.tr[m] = rpw[m] * wr;
         const int64_t nrb = (rows + g.tr[m] - 1) / g.tr[m];

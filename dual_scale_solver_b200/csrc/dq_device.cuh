@@ -362,12 +362,15 @@ struct Quant {
 #pragma unroll
             for (int k = 0; k < NP; ++k) c[k] = make_float2(rintf(q[k].x), rintf(q[k].y));
             if (!kExactQ) {
-                bool any = false;
+                // largest distance of q from its rounded value: near 0.5 only
+                // when some element sits within 2^-16 of a half-integer
+                float dmax = 0.0f;
 #pragma unroll
-                for (int k = 0; k < NP; ++k)
-                    any |= (fabsf(q[k].x - c[k].x) > 0.5f - 1.52587890625e-05f) |
-                           (fabsf(q[k].y - c[k].y) > 0.5f - 1.52587890625e-05f);   // 2^-16
-                if (any) {
+                for (int k = 0; k < NP; ++k) {
+                    const f2 d = __fadd2_rn(q[k], neg2(c[k]));
+                    dmax = max3_nan(dmax, fabsf(d.x), fabsf(d.y));
+                }
+                if (dmax > 0.5f - 1.52587890625e-05f) {
 #pragma unroll
                     for (int k = 0; k < NP; ++k)
 #pragma unroll
@@ -590,7 +593,10 @@ tile_kernel(const __grid_constant__ Table tab, int mode_slot, int want_res, int6
     const int64_t lt = t - md.tile0[mode_slot];
     if (lt >= md.ntiles[mode_slot]) continue;        // (uniform per CTA)
     const int wc = md.wc, wr = kWarps / wc;
-    const int tr = RPW * wr;
+    // tile rows: up to RPW per warp (fewer for short matrices, so that they
+    // still spread over many CTAs)
+    const int tr = md.tr[mode_slot];
+    const int rpw = tr / wr;
     const int64_t rb = lt / md.ncb, cb = lt % md.ncb;
     const int my_c = warp % wc, my_r = warp / wc;
     const int64_t cols = md.cols, rows = md.rows;
@@ -599,7 +605,7 @@ tile_kernel(const __grid_constant__ Table tab, int mode_slot, int want_res, int6
     const int64_t row_first = rb * tr;
     const int64_t row0 = row_first + my_r;           // this warp's first row
     // rows of this tile that this warp handles (k = 0 .. nk-1 -> row0 + k*wr)
-    const int nk = (int)max((int64_t)0, min((int64_t)RPW, (rows - row0 + wr - 1) / wr));
+    const int nk = (int)max((int64_t)0, min((int64_t)rpw, (rows - row0 + wr - 1) / wr));
 
     // per-lane column data, as pairs: b_j and the inner factor (1/b_j, or b_j for ACT)
     f2 bj[NP], cm[NP];
@@ -801,7 +807,7 @@ tile_kernel(const __grid_constant__ Table tab, int mode_slot, int want_res, int6
             const int pw = (p2 >> 1) / RPW, pk = (p2 >> 1) % RPW, h = p2 & 1;
             const int64_t row = row_first + (pw / wc) + (int64_t)pk * wr;
             f2 acc = bcast(0.0f);
-            if (row < rows) {
+            if (pk < rpw && row < rows) {
                 const float2 *p = &sm.red[(pw * RPW + pk) * 33 + 16 * h];
 #pragma unroll
                 for (int j = 0; j < 16; ++j) acc = __fadd2_rn(acc, p[j]);

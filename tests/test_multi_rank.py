@@ -30,11 +30,11 @@ def _worker(rank, world, port, q):
         import bench
         import synth
         wl = synth.WORKLOADS["llama31_70b_decoder_mxfp4_g32"]
-        d = bench.decoder_of(rank)
+        ds = bench.decoders_of(rank, 3)
         shards = [None] * world
-        dist.all_gather_object(shards, d)
-        # this rank's matrix (a reduced-size slice of its decoder's k_proj)
-        w = synth.weight(wl, d, 1, rows=4, cols=64)
+        dist.all_gather_object(shards, ds)
+        # this rank's matrix (a reduced-size slice of its first decoder's k_proj)
+        w = synth.weight(wl, ds[0], 1, rows=4, cols=64)
         ws = [None] * world
         dist.all_gather_object(ws, w)
         # per-rank step times meet in a max
@@ -60,7 +60,7 @@ def test_two_ranks_shard_by_decoder_and_reduce_timing():
         assert p.exitcode == 0
     res.sort()
     for rank, shards, ws, mx, rate in res:
-        assert shards == [0, 1]                       # one decoder per rank, distinct
+        assert shards == [[0, 1, 2], [3, 4, 5]]       # disjoint decoder blocks
         assert not torch.equal(ws[0], ws[1])          # different seeded weights
         assert mx == 15.0                             # the slowest rank's time
         assert rate == 2 * 1000 * 15 / (15.0 / 1e3)   # whole-job throughput
