@@ -335,9 +335,13 @@ def act_rescale_quant(X, b, fmt, codes=None, gscales=None, stream=None):
 KIND_ROW, KIND_COL, KIND_PACK, KIND_ACT, KIND_FUSED = 0, 1, 2, 3, 4
 
 
-def kernel_timing(enable: bool):
-    """Bracket every tile-kernel launch with CUDA events on its stream."""
-    _check(lib().dq_kernel_timing(1 if enable else 0), "dq_kernel_timing")
+def kernel_timing(enable: bool, kinds=None):
+    """Bracket the tile-kernel launches of the given kinds (all when None)
+    with CUDA events on their stream; enable=False turns timing off."""
+    mask = 0
+    if enable:
+        mask = 0x1F if kinds is None else sum(1 << int(k) for k in kinds)
+    _check(lib().dq_kernel_timing(mask), "dq_kernel_timing")
 
 
 def kernel_time(kind: int):

@@ -52,7 +52,7 @@ unsigned int *status_ptr() {
 // ---- measurement support: launch counter and optional per-kind event timing
 std::atomic<int64_t> g_launches{0};
 std::mutex g_timing_mu;
-bool g_timing = false;
+unsigned int g_timing_kinds = 0;   // bit k: time tile launches of kind k
 struct TimedLaunch { cudaEvent_t beg, end; int kind; };
 std::vector<TimedLaunch> g_timed;       // recorded, not yet read
 std::vector<cudaEvent_t> g_event_pool;  // free events
@@ -119,12 +119,14 @@ Geom geometry(int64_t rows, int64_t cols, bool f32) {
     g.wc = wc;
     g.ncb = (int)((nseg + wc - 1) / wc);
     const int wr = kWarps / wc;
-    // rows per warp: 16 for row statistics and packing; 128 for column
-    // statistics (fewer partial sums), reduced for short matrices so that
-    // they still make about 16 row blocks
-    int rpw_col = 16;
-    while (rpw_col < 128 && 2 * rpw_col <= rows / (wr * 16)) rpw_col *= 2;
-    const int rpw[3] = {16, rpw_col, 16};
+    // rows per warp: 256 for column statistics (fewer partial sums), 128 for
+    // the other modes (tile set-up spread over the rows), both reduced for
+    // short matrices so that they still make about 16 row blocks
+    int rpw_long = 16;
+    while (rpw_long < 128 && 2 * rpw_long <= rows / (wr * 16)) rpw_long *= 2;
+    int rpw_col = rpw_long;
+    while (rpw_col < 256 && 2 * rpw_col <= rows / (wr * 16)) rpw_col *= 2;
+    const int rpw[3] = {rpw_long, rpw_col, rpw_long};
     for (int m = 0; m < 3; ++m) {
         g.tr[m] = rpw[m] * wr;
         const int64_t nrb = (rows + g.tr[m] - 1) / g.tr[m];
@@ -241,7 +243,7 @@ struct Launcher {
         cudaEvent_t beg = nullptr, end = nullptr;
         {
             std::lock_guard<std::mutex> lk(g_timing_mu);
-            if (g_timing) { beg = take_event(); end = take_event(); }
+            if (g_timing_kinds & (1u << mode)) { beg = take_event(); end = take_event(); }
         }
         if (beg && end) DQ_CUDA(cudaEventRecord(beg, st));
         DQ_CUDA(launch_tiles(combo, L));
@@ -256,37 +258,36 @@ struct Launcher {
     dq_status row_finalize(unsigned int *flags = nullptr, unsigned int *next_flags = nullptr) {
         if (total_rows == 0) return DQ_OK;
         if (outer_of(combo) == SC_E8M0)
-            row_finalize_kernel<SC_E8M0><<<grid_for(total_rows, 256), 256, 0, st>>>(tab, total_rows,
-                                                                                  flags, next_flags);
+            DQ_CUDA(launch_k(row_finalize_kernel<SC_E8M0>, dim3(grid_for(total_rows, 256)),
+                             dim3(256), 0, st, tab, total_rows, flags, next_flags));
         else
-            row_finalize_kernel<SC_BF16><<<grid_for(total_rows, 256), 256, 0, st>>>(tab, total_rows,
-                                                                                  flags, next_flags);
-        DQ_CUDA(cudaGetLastError());
+            DQ_CUDA(launch_k(row_finalize_kernel<SC_BF16>, dim3(grid_for(total_rows, 256)),
+                             dim3(256), 0, st, tab, total_rows, flags, next_flags));
         count_launches(1);
         return DQ_OK;
     }
     dq_status col_finalize() {
         if (total_cols == 0) return DQ_OK;
-        // one block per 32-column slab (slabs of all matrices, in order)
+        // one block per 64-column slab (slabs of all matrices, in order)
         int64_t slabs = 0;
         for (int i = 0; i < tab.n; ++i) {
             const MatDesc &d = tab.dev ? host_table[i] : tab.one;
             slabs += (d.cols + kColFinCols - 1) / kColFinCols;
         }
         const unsigned grid = (unsigned)std::max<int64_t>(1, std::min<int64_t>(slabs, 148 * 16));
-        const int threads = kColFinCols * kColFinSlices;
+        const int threads = kColFinThreads;
         if (outer_of(combo) == SC_E8M0)
-            col_finalize_kernel<SC_E8M0><<<grid, threads, 0, st>>>(tab, total_cols);
+            DQ_CUDA(launch_k(col_finalize_kernel<SC_E8M0>, dim3(grid), dim3(threads), 0, st, tab,
+                             total_cols));
         else
-            col_finalize_kernel<SC_BF16><<<grid, threads, 0, st>>>(tab, total_cols);
-        DQ_CUDA(cudaGetLastError());
+            DQ_CUDA(launch_k(col_finalize_kernel<SC_BF16>, dim3(grid), dim3(threads), 0, st, tab,
+                             total_cols));
         count_launches(1);
         return DQ_OK;
     }
     dq_status mse(int row_slot, int idx_trace, int idx_half, double *out_row, double *out_col) {
-        mse_finalize_kernel<<<2 * tab.n, 256, 0, st>>>(tab, row_slot, idx_trace, idx_half, out_row,
-                                                      out_col);
-        DQ_CUDA(cudaGetLastError());
+        DQ_CUDA(launch_k(mse_finalize_kernel, dim3(2 * tab.n), dim3(256), 0, st, tab, row_slot,
+                         idx_trace, idx_half, out_row, out_col));
         count_launches(1);
         return DQ_OK;
     }
@@ -315,8 +316,8 @@ struct Launcher {
         if ((s = row_finalize(flags, next)) != DQ_OK) return s;
         if ((s = tiles_pass(MODE_COL, want_half, flags, 2)) != DQ_OK) return s;
         if ((s = col_finalize()) != DQ_OK) return s;
-        mse_finalize_fused_kernel<<<2 * tab.n, 256, 0, st>>>(tab, flags, clear, t);
-        DQ_CUDA(cudaGetLastError());
+        DQ_CUDA(launch_k(mse_finalize_fused_kernel, dim3(2 * tab.n), dim3(256), 0, st, tab, flags,
+                         clear, t));
         count_launches(1);
         return DQ_OK;
     }
@@ -407,21 +408,21 @@ dq_status solve_impl(int32_t n, const dq_matrix *mats, int32_t dtype, const dq_f
         for (int i = 0; i < n; ++i)
             DQ_CUDA(cudaMemsetAsync(t_table[i].amax, 0, sizeof(unsigned int), st));
         if (L.tiles[2] > 0) {
-            if (f32) amax_kernel<float><<<(unsigned)L.tiles[2], kThreads, 0, st>>>(L.tab);
-            else amax_kernel<Bf16Tag><<<(unsigned)L.tiles[2], kThreads, 0, st>>>(L.tab);
-            DQ_CUDA(cudaGetLastError());
+            if (f32) DQ_CUDA(launch_k(amax_kernel<float>, dim3((unsigned)L.tiles[2]),
+                                      dim3(kThreads), 0, st, L.tab));
+            else DQ_CUDA(launch_k(amax_kernel<Bf16Tag>, dim3((unsigned)L.tiles[2]), dim3(kThreads),
+                                  0, st, L.tab));
             count_launches(1);
         }
     }
-    tensor_scale_kernel<<<(n + 127) / 128, 128, 0, st>>>(L.tab, fi.qmax, fmt->tensor_scale_auto);
-    DQ_CUDA(cudaGetLastError());
+    DQ_CUDA(launch_k(tensor_scale_kernel, dim3((n + 127) / 128), dim3(128), 0, st, L.tab, fi.qmax,
+                     fmt->tensor_scale_auto));
     count_launches(1);
     const bool fused = fused_ok(fi.combo) && T > 0;
     if (fused) DQ_CUDA(cudaMemsetAsync(flags, 0, 6 * sizeof(unsigned int), st));
     if (row_base + col_base > 0) {
-        init_state_kernel<<<grid_for(row_base + col_base, 256), 256, 0, st>>>(
-            L.tab, row_base, col_base, fused ? flags : nullptr);
-        DQ_CUDA(cudaGetLastError());
+        DQ_CUDA(launch_k(init_state_kernel, dim3(grid_for(row_base + col_base, 256)), dim3(256), 0,
+                         st, L.tab, row_base, col_base, fused ? flags : nullptr));
         count_launches(1);
     }
     bool want_trace = false, want_half = false;
@@ -510,6 +511,7 @@ dq_status step_impl(bool row_step, const void *W, int32_t dtype, int64_t rows, i
 __global__ void dequant_kernel(const uint8_t *codes, const void *gs, int64_t rows, int64_t cols,
                                int G, int codes_kind, int gs_kind, float ts, const float *a,
                                const float *b, float *out) {
+    grid_dependency_begin();
     const int64_t n = rows * cols;
     for (int64_t k = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; k < n;
          k += (int64_t)gridDim.x * blockDim.x) {
@@ -676,9 +678,9 @@ dq_status dq_dequantize(const uint8_t *codes, const void *gscales, int64_t rows,
     if (rows == 0 || cols == 0) return DQ_OK;
     if (!codes || !gscales || !out) return DQ_ERR_ARG;
     const int64_t n = rows * cols;
-    dequant_kernel<<<grid_for(n, 256), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
-        codes, gscales, rows, cols, fi.G, fmt->codes, fmt->group_scale, tensor_scale, a, b, out);
-    DQ_CUDA(cudaGetLastError());
+    DQ_CUDA(launch_k(dequant_kernel, dim3(grid_for(n, 256)), dim3(256), 0,
+                     reinterpret_cast<cudaStream_t>(stream), codes, gscales, rows, cols, fi.G,
+                     fmt->codes, fmt->group_scale, tensor_scale, a, b, out));
     count_launches(1);
     return DQ_OK;
 }
@@ -742,9 +744,9 @@ dq_status dq_last_device_status(dq_stream stream) {
     return DQ_OK;
 }
 
-dq_status dq_kernel_timing(int32_t enable) {
+dq_status dq_kernel_timing(int32_t kinds) {
     std::lock_guard<std::mutex> lk(g_timing_mu);
-    g_timing = enable != 0;
+    g_timing_kinds = (unsigned int)kinds & 0x1Fu;
     return DQ_OK;
 }
 
@@ -880,18 +882,19 @@ extern "C" dq_status dq_solve_dual_scale_noalloc(const void *W, int32_t dtype, i
     if (fmt->tensor_scale_auto) {
         DQ_CUDA(cudaMemsetAsync(d.amax, 0, sizeof(unsigned int), st));   // starts at zero
         if (L.tiles[2] > 0) {
-            if (f32) amax_kernel<float><<<(unsigned)L.tiles[2], kThreads, 0, st>>>(L.tab);
-            else amax_kernel<Bf16Tag><<<(unsigned)L.tiles[2], kThreads, 0, st>>>(L.tab);
-            DQ_CUDA(cudaGetLastError());
+            if (f32) DQ_CUDA(launch_k(amax_kernel<float>, dim3((unsigned)L.tiles[2]),
+                                      dim3(kThreads), 0, st, L.tab));
+            else DQ_CUDA(launch_k(amax_kernel<Bf16Tag>, dim3((unsigned)L.tiles[2]), dim3(kThreads),
+                                  0, st, L.tab));
             count_launches(1);
         }
     }
-    tensor_scale_kernel<<<1, 128, 0, st>>>(L.tab, fi.qmax, fmt->tensor_scale_auto);
-    DQ_CUDA(cudaGetLastError());
+    DQ_CUDA(launch_k(tensor_scale_kernel, dim3(1), dim3(128), 0, st, L.tab, fi.qmax,
+                     fmt->tensor_scale_auto));
     count_launches(1);
     if (rb + cb > 0) {
-        init_state_kernel<<<grid_for(rb + cb, 256), 256, 0, st>>>(L.tab, rb, cb, nullptr);
-        DQ_CUDA(cudaGetLastError());
+        DQ_CUDA(launch_k(init_state_kernel, dim3(grid_for(rb + cb, 256)), dim3(256), 0, st, L.tab,
+                         rb, cb, nullptr));
         count_launches(1);
     }
     for (int t = 0; t < T; ++t) {

@@ -31,10 +31,21 @@ enum { STATUS_NONFINITE = 1u, STATUS_RANGE = 2u };
 
 constexpr int kWarps = 8;            // warps per CTA of the tile kernel
 constexpr int kThreads = 32 * kWarps;
-constexpr int kRowsPerWarp[5] = {16, 128, 16, 16, 128};   // per mode
+constexpr int kRowsPerWarp[5] = {128, 256, 128, 128, 256};   // per mode (at most)
 constexpr int kRing = 4;             // cp.async ring slots per lane (rows in flight + 1)
 constexpr float kBf16Max = 3.38953138925153547590470800371487866880e+38f;  // (2-2^-7)*2^127
 constexpr float kMinNormal = 1.17549435082228750796873653722224568e-38f;    // 2^-126
+
+// Programmatic dependent launch.  The library launches its kernels with
+// programmatic stream serialization, so a kernel may start while the one
+// before it on the stream is finishing.  Every kernel therefore first waits
+// for the grids it depends on to complete (their writes are then visible),
+// before it reads or writes global memory, and then lets the next kernel of
+// the stream launch early (its blocks wait in the same way).
+__device__ __forceinline__ void grid_dependency_begin() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
 
 // One matrix of a launch.  Tiles of mode m of this matrix are the global
 // tiles [tile0[m], tile0[m] + ntiles[m]); a tile is tr[m] rows by
@@ -311,8 +322,9 @@ struct Quant {
             // when m's significand exceeds qmax/4 (1.75 INT4, 1.5 E2M1);
             // e >= -126 (also covers subnormal m); e <= 126 holds for finite m
             constexpr uint32_t MT = (CODES == CODES_INT4) ? 0x600000u : 0x400000u;
-            const int e = max((int)(mb >> 23) - 129 + (((mb & 0x7FFFFFu) > MT) ? 1 : 0), -126);
-            s = pow2f(e);
+            // (the carry of the addition below adds that 1 to the exponent field)
+            const int sb = max((int)((mb + (0x7FFFFFu - MT)) & 0x7F800000u) - (2 << 23), 1 << 23);
+            s = __uint_as_float((uint32_t)sb);
             if (NIB && !pos) s = 1.0f;                     // stored scale of an all-zero group
         } else {
             // every lane takes part in the warp vote and group shuffles below,
@@ -529,18 +541,19 @@ __device__ __forceinline__ float project_outer(float x, bool &clamped) {
 //         tile's columns -> rowpart[row][cb]; residual of the state -> res_row
 //   COL : per column, sum_i W_ij S_ij and sum_i S_ij^2 (S = D_a Qhat) over the
 //         tile's rows -> colpart[rb][col]; residual -> res_col
+//   FUSED (power-of-two scales): ROW and COL from one quantization
 //   PACK: codes and group scales of Q(W / (a b)); residual -> res_row
 //   ACT : codes and group scales of Q(X * b)
-// `want_res` = 0 skips the residual (its MSE output was not requested).
+// Tiles have up to kRowsPerWarp[mode] rows per warp (the host picks fewer for
+// short matrices).  `want_res` = 0 skips the residual (its MSE output was
+// not requested).
 // Shared memory of one tile CTA, by mode.
 template <int MODE, int EPC>
 struct TileSmem {
     static constexpr int RPW = kRowsPerWarp[MODE];
-    // ROW: per (warp, row of the warp, lane) partial (num, den), reduced once
-    // at the end of the tile; FUSED: the same for a batch of 8 rows, reduced
-    // every 8 rows.  Row stride padded by one entry.
-    static constexpr int kRed = MODE == MODE_ROW ? kWarps * RPW * 33
-                              : (MODE == MODE_FUSED ? kWarps * 8 * 33 : 1);
+    // ROW, FUSED: per (warp, row of a batch of 8, lane) partial (num, den),
+    // reduced every 8 rows.  Row stride padded by one entry.
+    static constexpr int kRed = (MODE == MODE_ROW || MODE == MODE_FUSED) ? kWarps * 8 * 33 : 1;
     // ROW, FUSED: per (row, warp) totals
     static constexpr int kRtot = (MODE == MODE_ROW || MODE == MODE_FUSED) ? RPW * kWarps : 1;
     // COL, FUSED: per (warp-row, column) partials
@@ -560,6 +573,7 @@ template <int CODES, int GS, int OS, int MODE, typename TIn, int G>
 __global__ void __launch_bounds__(kThreads, TileOcc<MODE>::kMinBlocks)
 tile_kernel(const __grid_constant__ Table tab, int mode_slot, int want_res, int64_t total_tiles,
             unsigned int *flags, int gate) {
+    grid_dependency_begin();
     using CK = Chunk<TIn>;
     constexpr int EPC = CK::EPC;
     constexpr int NP = EPC / 2;
@@ -572,7 +586,6 @@ tile_kernel(const __grid_constant__ Table tab, int mode_slot, int want_res, int6
     constexpr bool COLSTAT = MODE == MODE_COL || FUSED;
     using Q = Quant<CODES, GS, OS, ACT, NP, LPG>;
     constexpr int RPW = kRowsPerWarp[MODE];
-    static_assert(RPW <= 32 || MODE == MODE_COL || FUSED, "row factors are held one row per lane");
     static_assert(!FUSED || (GS == SC_E8M0 && OS == SC_E8M0), "fused statistics need power-of-two scales");
     constexpr int ESZ = 16 / EPC;                    // bytes per element
 
@@ -621,15 +634,8 @@ tile_kernel(const __grid_constant__ Table tab, int mode_slot, int want_res, int6
         else if (OS == SC_E8M0) cm[k] = make_float2(recip_pow2(b0), recip_pow2(b1));
         else cm[k] = make_float2(recip_approx(b0), recip_approx(b1));
     }
-    // row factors: lane k holds a and 1/a of the warp's k-th row (modes with
-    // more than 32 rows per warp read them per row instead)
-    constexpr bool kRowFactorPerRow = RPW > 32;
-    float a_lane = 1.0f, ia_lane = 1.0f;
+    // row factors a_i are read per row (one cached load per lane)
     const float *const pa = ACT ? nullptr : md.a;
-    if (!kRowFactorPerRow && pa != nullptr && lane < nk) {
-        a_lane = __ldg(pa + row0 + (int64_t)lane * wr);
-        ia_lane = (OS == SC_E8M0) ? recip_pow2(a_lane) : recip_approx(a_lane);
-    }
 
     const float ts = (GS == SC_E4M3 && !ACT) ? tensor_scale_of(md) : 1.0f;
     const float inv_ts = 1.0f / ts;                 // ts is a power of two
@@ -664,26 +670,18 @@ tile_kernel(const __grid_constant__ Table tab, int mode_slot, int want_res, int6
 #pragma unroll
     for (int k = 0; k < kRing - 1; ++k) issue(k, k);
 
-    // rows in groups of kRing: the ring slot of each row is a constant
-#pragma unroll 1
-    for (int k0 = 0; k0 < nk; k0 += kRing) {
-#pragma unroll
-    for (int u = 0; u < kRing; ++u) {
-        const int k = k0 + u;
-        if (k >= nk) break;                           // warp-uniform
+    // One row of the warp: row k, in ring slot u % kRing (u is a constant
+    // where the loops below unroll); batch_end closes a batch of 8 rows of
+    // the row statistics.
+    auto one_row = [&](const int k, const int u, const bool batch_end) {
         issue(k + kRing - 1, (u + kRing - 1) % kRing);
         asm volatile("cp.async.wait_group %0;" :: "n"(kRing - 1) : "memory");
         CK ck;
-        ck.raw = sm.ring[warp][u][lane];
+        ck.raw = sm.ring[warp][u % kRing][lane];
         float a = 1.0f, ia = 1.0f;
         if (!ACT && !FUSED && pa != nullptr) {
-            if (kRowFactorPerRow) {
-                a = __ldg(pa + row0 + (int64_t)k * wr);
-                ia = (OS == SC_E8M0) ? recip_pow2(a) : recip_approx(a);
-            } else {
-                a = __shfl_sync(0xffffffffu, a_lane, k);
-                ia = __shfl_sync(0xffffffffu, ia_lane, k);
-            }
+            a = __ldg(pa + row0 + (int64_t)k * wr);
+            ia = (OS == SC_E8M0) ? recip_pow2(a) : recip_approx(a);
         }
         f2 w[NP], z[NP], c[NP];
         ck.unpack2(w);
@@ -700,8 +698,8 @@ tile_kernel(const __grid_constant__ Table tab, int mode_slot, int want_res, int6
             // |e(a)| <= 20 (old) and <= 26 (new)
             Q::template run<NIB>(w, z, 1.0f, 1.0f, bj, ts, inv_ts, tab.status, c, s, s_eff, nib,
                                  nonzero);
-            const int es = (int)(__float_as_uint(s) >> 23) - 127;
-            clamp_risk |= nonzero && (es > 100 || es < -100);
+            // s = 2^e with |e| <= 100: exponent field in [27, 227]
+            clamp_risk |= nonzero && (__float_as_uint(s) - (27u << 23)) > (200u << 23);
         } else {
             Q::template run<NIB>(w, z, a, ia, bj, ts, inv_ts, tab.status, c, s, s_eff, nib,
                                  nonzero);
@@ -726,30 +724,24 @@ tile_kernel(const __grid_constant__ Table tab, int mode_slot, int want_res, int6
                 }
             }
             const float2 share = make_float2((gn.x + gn.y) * s_row, (gd.x + gd.y) * (s_row * s_row));
-            if (MODE == MODE_ROW) {
-                // this lane's share of row k, summed over lanes at the end of the tile
-                sm.red[(warp * RPW + k) * 33 + lane] = share;
-            } else {
-                // batches of 8 rows: lane 2r + h adds the 16 shares of half h of
-                // the batch's row r in order, then the halves are added -- the
-                // same order as the row-statistics epilogue, so both modes give
-                // the same bits
-                sm.red[(warp * 8 + (k & 7)) * 33 + lane] = share;
-                if ((k & 7) == 7 || k == nk - 1) {
-                    __syncwarp();
-                    const int rr = (lane >> 1) & 7, hh = lane & 1;
-                    const float2 *p = &sm.red[(warp * 8 + rr) * 33 + 16 * hh];
-                    f2 acc = bcast(0.0f);
-                    if (lane < 16) {
+            // batches of 8 rows: lane 2r + h adds the 16 shares of half h of
+            // the batch's row r in order, then the halves are added (a fixed
+            // order, the same in every mode with row statistics)
+            sm.red[(warp * 8 + (k & 7)) * 33 + lane] = share;
+            if (batch_end) {
+                __syncwarp();
+                const int rr = (lane >> 1) & 7, hh = lane & 1;
+                const float2 *p = &sm.red[(warp * 8 + rr) * 33 + 16 * hh];
+                f2 acc = bcast(0.0f);
+                if (lane < 16) {
 #pragma unroll
-                        for (int j = 0; j < 16; ++j) acc = __fadd2_rn(acc, p[j]);
-                    }
-                    acc.x += __shfl_xor_sync(0xffffffffu, acc.x, 1);
-                    acc.y += __shfl_xor_sync(0xffffffffu, acc.y, 1);
-                    const int kk = (k & ~7) + rr;
-                    if (lane < 16 && hh == 0 && kk <= k) sm.rtot[kk * kWarps + warp] = acc;
-                    __syncwarp();
+                    for (int j = 0; j < 16; ++j) acc = __fadd2_rn(acc, p[j]);
                 }
+                acc.x += __shfl_xor_sync(0xffffffffu, acc.x, 1);
+                acc.y += __shfl_xor_sync(0xffffffffu, acc.y, 1);
+                const int kk = (k & ~7) + rr;
+                if (lane < 16 && hh == 0 && kk <= k) sm.rtot[kk * kWarps + warp] = acc;
+                __syncwarp();
             }
         }
         if (COLSTAT) {
@@ -791,32 +783,23 @@ tile_kernel(const __grid_constant__ Table tab, int mode_slot, int want_res, int6
                 }
             }
         }
+    };
+    // full groups of 8 rows as straight-line code, then the tail
+    int k0 = 0;
+#pragma unroll 1
+    for (; k0 + 8 <= nk; k0 += 8) {
+#pragma unroll
+        for (int u = 0; u < 8; ++u) one_row(k0 + u, u, u == 7);
     }
+#pragma unroll
+    for (int u = 0; u < 7; ++u) {
+        if (k0 + u >= nk) break;                     // warp-uniform
+        one_row(k0 + u, u, k0 + u == nk - 1);
     }
     asm volatile("cp.async.wait_all;" ::: "memory");
     if (FUSED && clamp_risk) atomicOr(&flags[0], 1u);
 
     // ---- tile epilogue ----
-    if (MODE == MODE_ROW) {
-        // (warp, row) pair p = t / 2 sums 16 lane shares per thread, then the
-        // two halves; fixed order throughout
-        static_assert((2 * kWarps * RPW) % kThreads == 0 || MODE != MODE_ROW,
-                      "every thread takes the same trips");
-        __syncthreads();
-        for (int p2 = threadIdx.x; p2 < 2 * kWarps * RPW; p2 += kThreads) {
-            const int pw = (p2 >> 1) / RPW, pk = (p2 >> 1) % RPW, h = p2 & 1;
-            const int64_t row = row_first + (pw / wc) + (int64_t)pk * wr;
-            f2 acc = bcast(0.0f);
-            if (pk < rpw && row < rows) {
-                const float2 *p = &sm.red[(pw * RPW + pk) * 33 + 16 * h];
-#pragma unroll
-                for (int j = 0; j < 16; ++j) acc = __fadd2_rn(acc, p[j]);
-            }
-            acc.x += __shfl_xor_sync(0xffffffffu, acc.x, 1);
-            acc.y += __shfl_xor_sync(0xffffffffu, acc.y, 1);
-            if (h == 0) sm.rtot[pk * kWarps + pw] = acc;
-        }
-    }
     if (ROWSTAT) {
         __syncthreads();
         // rows of the tile: local row k*wr + r is warp-row r's k-th row
@@ -898,6 +881,7 @@ tile_kernel(const __grid_constant__ Table tab, int mode_slot, int want_res, int6
 template <int OS>
 __global__ void row_finalize_kernel(const __grid_constant__ Table tab, int64_t total_rows,
                                     unsigned int *flags, unsigned int *next_flags) {
+    grid_dependency_begin();
     const bool scale_old = flags != nullptr && flags[0] == 0;
     for (int64_t g = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; g < total_rows;
          g += (int64_t)gridDim.x * blockDim.x) {
@@ -930,19 +914,22 @@ __global__ void row_finalize_kernel(const __grid_constant__ Table tab, int64_t t
     }
 }
 
-// b_j <- Pi(sum P / sum E) over the column's row blocks.  A block handles 32
-// consecutive columns of one matrix with 8 slices of row blocks (slice s
+// b_j <- Pi(sum P / sum E) over the column's row blocks.  A block handles 64
+// consecutive columns of one matrix (a lane reads the partials of two
+// adjacent columns as one 16-byte load) with 8 slices of row blocks (slice s
 // sums row blocks s, s+8, ... in order, in double); the slices are then
 // added in order: a fixed summation order, independent of the launch.
-constexpr int kColFinCols = 32, kColFinSlices = 8;
+constexpr int kColFinCols = 64, kColFinSlices = 8;
+constexpr int kColFinThreads = 32 * kColFinSlices;
 template <int OS>
-__global__ void __launch_bounds__(kColFinCols * kColFinSlices)
+__global__ void __launch_bounds__(kColFinThreads)
 col_finalize_kernel(const __grid_constant__ Table tab, int64_t total_cols) {
+    grid_dependency_begin();
     __shared__ double sp[kColFinSlices][kColFinCols], se[kColFinSlices][kColFinCols];
-    const int cl = threadIdx.x % kColFinCols, sl = threadIdx.x / kColFinCols;
-    // blocks enumerate 32-column slabs of every matrix in turn
+    const int lane = threadIdx.x & 31, sl = threadIdx.x >> 5;
+    // blocks enumerate 64-column slabs of every matrix in turn
     for (int64_t slab = blockIdx.x; ; slab += gridDim.x) {
-        // matrix of this slab: slabs of matrix i start at ceil-sum of cols / 32
+        // matrix of this slab: slabs of matrix i start at ceil-sum of cols / 64
         int mi = -1;
         int64_t c0 = 0;
         {
@@ -955,22 +942,31 @@ col_finalize_kernel(const __grid_constant__ Table tab, int64_t total_cols) {
         }
         if (mi < 0) break;                                 // uniform per block
         const MatDesc &md = tab.get(mi);
-        const int64_t c = c0 + cl;
+        // columns c and c + 1 (cols is even, so both or neither exist)
+        const int64_t c = c0 + 2 * lane;
         const bool ok = c < md.cols;
         const int64_t nrb = md.ntiles[MODE_COL] / max(md.ncb, 1);
-        double p = 0.0, e = 0.0;
+        double p0 = 0.0, e0 = 0.0, p1 = 0.0, e1 = 0.0;
         if (ok) {
+            const float4 *src = reinterpret_cast<const float4 *>(md.colpart + c);
+            const int64_t stride = md.cols / 2;              // float4 per row block
 #pragma unroll 4
             for (int64_t k = sl; k < nrb; k += kColFinSlices) {
-                const float2 v = md.colpart[k * md.cols + c];
-                p += v.x;
-                e += v.y;
+                const float4 v = __ldg(src + k * stride);
+                p0 += v.x;
+                e0 += v.y;
+                p1 += v.z;
+                e1 += v.w;
             }
         }
-        sp[sl][cl] = p;
-        se[sl][cl] = e;
+        sp[sl][2 * lane] = p0;
+        se[sl][2 * lane] = e0;
+        sp[sl][2 * lane + 1] = p1;
+        se[sl][2 * lane + 1] = e1;
         __syncthreads();
-        if (sl == 0 && ok) {
+        const int cl = threadIdx.x;
+        if (cl < kColFinCols && c0 + cl < md.cols) {
+            const int64_t cc = c0 + cl;
             double pt = 0.0, et = 0.0;
             for (int q = 0; q < kColFinSlices; ++q) { pt += sp[q][cl]; et += se[q][cl]; }
             float b = 1.0f, pre = __int_as_float(0x7fc00000);
@@ -981,8 +977,8 @@ col_finalize_kernel(const __grid_constant__ Table tab, int64_t total_cols) {
                 if (cl2) atomicOr(tab.status, STATUS_RANGE);
             }
             if (!isfinite(pt) || !isfinite(et)) atomicOr(tab.status, STATUS_NONFINITE);
-            md.b_out[c] = b;
-            if (md.b_pre) md.b_pre[c] = pre;
+            md.b_out[cc] = b;
+            if (md.b_pre) md.b_pre[cc] = pre;
         }
         __syncthreads();
     }
@@ -997,6 +993,7 @@ col_finalize_kernel(const __grid_constant__ Table tab, int64_t total_cols) {
 // the descriptor's mse_trace / mse_half unless `out` is given.
 __global__ void mse_finalize_kernel(const __grid_constant__ Table tab, int row_slot, int idx_trace, int idx_half,
                                     double *out_row, double *out_col) {
+    grid_dependency_begin();
     const int mi = blockIdx.x >> 1, which = blockIdx.x & 1;
     const MatDesc &md = tab.get(mi);
     double *dst;
@@ -1035,6 +1032,7 @@ __global__ void mse_finalize_kernel(const __grid_constant__ Table tab, int row_s
 __global__ void mse_finalize_fused_kernel(const __grid_constant__ Table tab,
                                           const unsigned int *flags, unsigned int *next_flags,
                                           int idx) {
+    grid_dependency_begin();
     if (blockIdx.x == 0 && threadIdx.x == 0) { next_flags[0] = 0u; next_flags[1] = 0u; }
     const int mi = blockIdx.x >> 1, which = blockIdx.x & 1;
     const MatDesc &md = tab.get(mi);
@@ -1072,6 +1070,7 @@ __global__ void mse_finalize_fused_kernel(const __grid_constant__ Table tab,
 // take its row step literally.
 __global__ void init_state_kernel(const __grid_constant__ Table tab, int64_t total_rows,
                                   int64_t total_cols, unsigned int *flags) {
+    grid_dependency_begin();
     for (int64_t g = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; g < total_rows + total_cols;
          g += (int64_t)gridDim.x * blockDim.x) {
         if (g < total_rows) {
@@ -1099,6 +1098,7 @@ __global__ void init_state_kernel(const __grid_constant__ Table tab, int64_t tot
 // amax over each matrix (tiles of the PACK geometry), for the tensor scale.
 template <typename TIn>
 __global__ void __launch_bounds__(kThreads) amax_kernel(const __grid_constant__ Table tab) {
+    grid_dependency_begin();
     constexpr int EPC = Chunk<TIn>::EPC;
     const int64_t t = blockIdx.x;
     const int mi = find_owner(tab, t, [](const MatDesc &d) { return d.tile0[MODE_PACK]; });
@@ -1134,6 +1134,7 @@ __global__ void __launch_bounds__(kThreads) amax_kernel(const __grid_constant__ 
 #ifdef DQ_DEFINE_HOST_KERNELS
 // ts = 2^ceil(log2(amax / (448 qmax))), exponent in [-126, 126]; 1 if amax == 0.
 __global__ void tensor_scale_kernel(const __grid_constant__ Table tab, float qmax, int enabled) {
+    grid_dependency_begin();
     const int mi = blockIdx.x * blockDim.x + threadIdx.x;
     if (mi >= tab.n) return;
     const MatDesc &md = tab.get(mi);

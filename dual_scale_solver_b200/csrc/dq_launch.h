@@ -5,6 +5,8 @@
 
 #include <cuda_runtime.h>
 
+#include <utility>
+
 #include "dq_device.cuh"
 
 namespace dq {
@@ -34,6 +36,26 @@ enum Combo {
     COMBO_COUNT = 6
 };
 
+// Launch with programmatic stream serialization: the kernel may start while
+// the previous kernel of the stream finishes; every kernel of the library
+// begins with grid_dependency_begin(), which keeps the stream's order of
+// memory accesses.
+template <typename... P, typename... A>
+cudaError_t launch_k(void (*kern)(P...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                     A &&...args) {
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<A>(args)...);
+}
+
 cudaError_t launch_tile_c0(const TileLaunch &L);
 cudaError_t launch_tile_c1(const TileLaunch &L);
 cudaError_t launch_tile_c2(const TileLaunch &L);
@@ -58,9 +80,8 @@ cudaError_t launch_tile_one(const TileLaunch &L) {
             done[dev] = true;
         }
     }
-    kern<<<dim3((unsigned)L.grid), dim3(kThreads), bytes, L.stream>>>(L.tab, L.slot, L.want_res,
-                                                                      L.tiles, L.flags, L.gate);
-    return cudaGetLastError();
+    return launch_k(kern, dim3((unsigned)L.grid), dim3(kThreads), bytes, L.stream, L.tab, L.slot,
+                    L.want_res, L.tiles, L.flags, L.gate);
 }
 
 // Dispatch over mode, dtype and G for one format set (used by each unit).

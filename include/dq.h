@@ -228,14 +228,17 @@ DQ_API dq_status dq_solve_dual_scale_noalloc(const void *W, int32_t dtype, int64
                                              float *tensor_scale, double *mse_trace,
                                              double *mse_half, dq_stream stream);
 
-/* Measurement support (no counterpart in the method).  dq_kernel_timing(1)
- * makes every tile-kernel launch of the library record a CUDA event pair on
- * its own stream (kind 0 row statistics, 1 column statistics, 2 pack,
- * 3 activation, 4 row and column statistics in one pass); dq_kernel_time synchronises those events and returns (and
- * clears) the summed milliseconds and the launch count of one kind.
+/* Measurement support (no counterpart in the method).  dq_kernel_timing(kinds)
+ * makes the tile-kernel launches of the kinds whose bit is set in `kinds`
+ * (bit k for kind k: 0 row statistics, 1 column statistics, 2 pack,
+ * 3 activation, 4 row and column statistics in one pass; 0 turns timing off)
+ * record a CUDA event pair on their own stream; dq_kernel_time synchronises
+ * those events and returns (and clears) the summed milliseconds and the
+ * launch count of one kind.  Each event pair separates its launch from the
+ * kernels around it on the stream, so time only the kinds of interest.
  * dq_launch_count returns the number of kernels this library has launched in
  * the process so far (all kinds, including finalize kernels). */
-DQ_API dq_status dq_kernel_timing(int32_t enable);
+DQ_API dq_status dq_kernel_timing(int32_t kinds);
 DQ_API dq_status dq_kernel_time(int32_t kind, double *ms, int64_t *launches);
 DQ_API int64_t dq_launch_count(void);
 
