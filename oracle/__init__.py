@@ -11,7 +11,7 @@ pinned by the tests listed in the design notes (closed forms, brute force,
 library casts, hand-derived cases).
 """
 from .formats import *          # noqa: F401,F403
-from .solver import (Format, PRESETS, preset, project_group_scale, project_outer,  # noqa: F401
+from .solver import (Format, PRESETS, QMAX, CODE_BITS, preset, project_group_scale, project_outer,  # noqa: F401
                      round_codes, tensor_scale, quantize, dequantize, inner, qhat, mse,
                      row_update, col_update, solve, act_rescale_quant, encode_codes,
                      encode_scales, decode_codes, decode_scales)

@@ -18,11 +18,21 @@ Sources (the DualQuant pages):
   the format's admissible set: daiwk note, section "原始论文总结"; trove summary,
   "What it claims".
 
+* The method claims support for the whole MX family (news.yiqijian.com
+  article, same section, and the trove summary, "What it claims"); the MX
+  element formats beyond MXFP4/MXINT4 are taken from the OCP Microscaling
+  format definition: MXFP8 (E4M3 or E5M2 elements), MXFP6 (E2M3 or E3M2),
+  MXINT8 (8-bit two's complement), all in blocks of 32 with an E8M0 scale.
+
 Rounding rules that the pages leave open (readings, not quotations):
 * BF16 and E4M3 values: round to nearest, ties to even (IEEE default).
 * E4M3 saturates at 448 (the OCP "fn" variant has no infinity).
 * E2M1 magnitudes {0, 0.5, 1, 1.5, 2, 3, 4, 6}: nearest, ties to the code with
   an even mantissa bit, saturating at 6; the sign follows the input's sign bit.
+* The other float element formats the same way (nearest, ties to even,
+  saturating at the largest finite value, sign of zero from the input):
+  E4M3 max 448, E5M2 max 57344, E2M3 max 7.5, E3M2 max 28 (all with
+  subnormals).  INT8 elements: round half to even, clamp to [-128, 127].
 """
 from __future__ import annotations
 
@@ -115,6 +125,44 @@ def round_int4(q) -> np.ndarray:
     return np.clip(np.rint(np.asarray(q, dtype=np.float64)), -8.0, 7.0)
 
 
+def round_int8(q) -> np.ndarray:
+    """Round half to even, clamp to the signed INT8 codebook [-128, 127]."""
+    return np.clip(np.rint(np.asarray(q, dtype=np.float64)), -128.0, 127.0)
+
+
+# Element float formats of the MX family: (exponent bits, mantissa bits, bias,
+# largest finite value).  Normal exponents run from 1 - bias; the field of all
+# ones is an ordinary exponent in E4M3 (save its NaN code), E2M3 and E3M2 and
+# holds Inf/NaN in E5M2.
+FP_ELEMENTS = {
+    "e4m3": (4, 3, 7, 448.0),
+    "e5m2": (5, 2, 15, 57344.0),
+    "e2m3": (2, 3, 1, 7.5),
+    "e3m2": (3, 2, 3, 28.0),
+}
+
+
+def round_fp_element(q, name: str) -> np.ndarray:
+    """Nearest value of an MX float element format, ties to even, saturating."""
+    eb, mb, bias, mx = FP_ELEMENTS[name]
+    return round_float_format(q, mb + 1, 1 - bias, mx, satfinite=True)
+
+
+def fp_element_values(name: str) -> np.ndarray:
+    """Value of every code of an element format with the sign bit clear
+    (index = code); codes beyond the largest finite value are NaN."""
+    eb, mb, bias, mx = FP_ELEMENTS[name]
+    vals = np.empty(1 << (eb + mb))
+    for code in range(1 << (eb + mb)):
+        e, m = code >> mb, code & ((1 << mb) - 1)
+        if e == 0:
+            v = (m / 2.0 ** mb) * 2.0 ** (1 - bias)
+        else:
+            v = (1.0 + m / 2.0 ** mb) * 2.0 ** (e - bias)
+        vals[code] = v if v <= mx else np.nan
+    return vals
+
+
 # --------------------------------------------------------------------------- #
 # Encodings of stored values (bit patterns the library writes)
 # --------------------------------------------------------------------------- #
@@ -193,6 +241,58 @@ def encode_e2m1(c) -> np.ndarray:
 def decode_e2m1(n) -> np.ndarray:
     n = np.asarray(n, dtype=np.int64)
     return np.where(n & 8, -1.0, 1.0) * E2M1_GRID[n & 7]
+
+
+def encode_fp_element(v, name: str) -> np.ndarray:
+    """Code (sign bit above the magnitude bits) of element-format values."""
+    eb, mb, _, _ = FP_ELEMENTS[name]
+    vals = fp_element_values(name)
+    n = int(np.sum(~np.isnan(vals)))           # finite magnitudes: codes 0 .. n-1
+    v = np.asarray(v, dtype=np.float64)
+    av = np.abs(v)
+    idx = np.minimum(np.searchsorted(vals[:n], av), n - 1)
+    if not np.all(vals[idx] == av):
+        raise ValueError(f"value not representable in {name}")
+    return (idx | np.where(np.signbit(v), 1 << (eb + mb), 0)).astype(np.uint8)
+
+
+def decode_fp_element(u, name: str) -> np.ndarray:
+    eb, mb, _, _ = FP_ELEMENTS[name]
+    u = np.asarray(u, dtype=np.int64)
+    sign = 1 << (eb + mb)
+    return np.where(u & sign, -1.0, 1.0) * fp_element_values(name)[u & (sign - 1)]
+
+
+def encode_int8(c) -> np.ndarray:
+    """Two's-complement byte of INT8 values."""
+    return (np.asarray(c).astype(np.int64) & 0xFF).astype(np.uint8)
+
+
+def decode_int8(u) -> np.ndarray:
+    u = np.asarray(u, dtype=np.int64) & 0xFF
+    return np.where(u >= 128, u - 256, u).astype(np.float64)
+
+
+def pack_sixbits(codes: np.ndarray) -> np.ndarray:
+    """Pack ``[..., 4k]`` 6-bit codes into ``[..., 3k]`` bytes: four
+    consecutive codes form one little-endian 24-bit word, the first code in
+    the lowest bits."""
+    c = np.asarray(codes, dtype=np.uint32)
+    w = c[..., 0::4] | (c[..., 1::4] << 6) | (c[..., 2::4] << 12) | (c[..., 3::4] << 18)
+    out = np.empty(w.shape[:-1] + (3 * w.shape[-1],), dtype=np.uint8)
+    out[..., 0::3] = w & 0xFF
+    out[..., 1::3] = (w >> 8) & 0xFF
+    out[..., 2::3] = (w >> 16) & 0xFF
+    return out
+
+
+def unpack_sixbits(b: np.ndarray) -> np.ndarray:
+    b = np.asarray(b, dtype=np.uint32)
+    w = b[..., 0::3] | (b[..., 1::3] << 8) | (b[..., 2::3] << 16)
+    out = np.empty(w.shape[:-1] + (4 * w.shape[-1],), dtype=np.uint8)
+    for k in range(4):
+        out[..., k::4] = (w >> (6 * k)) & 0x3F
+    return out
 
 
 def pack_nibbles(nib: np.ndarray) -> np.ndarray:

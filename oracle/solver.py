@@ -34,7 +34,9 @@ Readings taken where the pages are silent (each also listed in the design notes)
   - E4M3: round to nearest even, saturating at 448; a positive value that
     rounds to 0 becomes the smallest subnormal 2^-9.
   Codes c = round(Y / (s * ts)) on the grid (INT4: half to even, clamp [-8,7];
-  E2M1: nearest, ties to even code, saturate 6).  Qhat = c * s * ts.
+  E2M1: nearest, ties to even code, saturate 6; the other MX element formats
+  likewise: INT8 clamps to [-128,127], float elements saturate at their
+  largest finite value).  Qhat = c * s * ts.
 * NVFP4 second-level (tensor) scale for weights: ts = 2^ceil(log2(amax(W) /
   (448 * 6))), fixed from the input W at the start; ts = 1 for every other
   format and for activations.
@@ -51,9 +53,16 @@ import numpy as np
 from . import formats as F
 
 
+# largest code magnitude of each element format (the grid's qmax)
+QMAX = {"int4": 7.0, "e2m1": 6.0, "int8": 127.0, "e4m3": 448.0, "e5m2": 57344.0,
+        "e2m3": 7.5, "e3m2": 28.0}
+# stored bits per code
+CODE_BITS = {"int4": 4, "e2m1": 4, "int8": 8, "e4m3": 8, "e5m2": 8, "e2m3": 6, "e3m2": 6}
+
+
 @dataclass(frozen=True)
 class Format:
-    codes: str            # "int4" | "e2m1"
+    codes: str            # a key of QMAX
     group: int            # G, consecutive columns sharing a scale
     gscale: str           # "bf16" | "e8m0" | "e4m3"
     oscale: str           # "bf16" | "e8m0"   (set of the outer scales a, b)
@@ -61,7 +70,11 @@ class Format:
 
     @property
     def qmax(self) -> float:
-        return 7.0 if self.codes == "int4" else 6.0
+        return QMAX[self.codes]
+
+    @property
+    def code_bits(self) -> int:
+        return CODE_BITS[self.codes]
 
 
 PRESETS = {
@@ -73,6 +86,13 @@ PRESETS = {
     "mxfp4": Format("e2m1", 32, "e8m0", "e8m0"),
     # news article: NVFP4 = E2M1, 16-element blocks, E4M3 scale; BF16 outer scales.
     "nvfp4": Format("e2m1", 16, "e4m3", "bf16", tensor_scale_auto=True),
+    # the rest of the MX family (the pages claim it; element formats from the
+    # OCP Microscaling definition): 32-element blocks, E8M0 scales
+    "mxfp8_e4m3": Format("e4m3", 32, "e8m0", "e8m0"),
+    "mxfp8_e5m2": Format("e5m2", 32, "e8m0", "e8m0"),
+    "mxfp6_e2m3": Format("e2m3", 32, "e8m0", "e8m0"),
+    "mxfp6_e3m2": Format("e3m2", 32, "e8m0", "e8m0"),
+    "mxint8": Format("int8", 32, "e8m0", "e8m0"),
 }
 
 
@@ -109,7 +129,13 @@ def project_outer(x: np.ndarray, fmt: Format) -> np.ndarray:
 
 
 def round_codes(q: np.ndarray, fmt: Format) -> np.ndarray:
-    return F.round_int4(q) if fmt.codes == "int4" else F.round_e2m1(q)
+    if fmt.codes == "int4":
+        return F.round_int4(q)
+    if fmt.codes == "int8":
+        return F.round_int8(q)
+    if fmt.codes == "e2m1":
+        return F.round_e2m1(q)
+    return F.round_fp_element(q, fmt.codes)
 
 
 def tensor_scale(W: np.ndarray, fmt: Format) -> float:
@@ -232,8 +258,16 @@ def act_rescale_quant(X, b, fmt: Format):
 # --------------------------------------------------------------------------- #
 
 def encode_codes(c: np.ndarray, fmt: Format) -> np.ndarray:
-    nib = F.encode_int4(c) if fmt.codes == "int4" else F.encode_e2m1(c)
-    return F.pack_nibbles(nib)
+    """Stored codes: 4-bit codes two per byte (even column low), 8-bit codes
+    one per byte, 6-bit codes four per three bytes."""
+    if fmt.codes == "int4":
+        return F.pack_nibbles(F.encode_int4(c))
+    if fmt.codes == "e2m1":
+        return F.pack_nibbles(F.encode_e2m1(c))
+    if fmt.codes == "int8":
+        return F.encode_int8(c)
+    u = F.encode_fp_element(c, fmt.codes)
+    return F.pack_sixbits(u) if fmt.code_bits == 6 else u
 
 
 def encode_scales(s: np.ndarray, fmt: Format) -> np.ndarray:
@@ -245,8 +279,14 @@ def encode_scales(s: np.ndarray, fmt: Format) -> np.ndarray:
 
 
 def decode_codes(packed: np.ndarray, fmt: Format) -> np.ndarray:
-    nib = F.unpack_nibbles(packed)
-    return F.decode_int4(nib) if fmt.codes == "int4" else F.decode_e2m1(nib)
+    if fmt.codes == "int4":
+        return F.decode_int4(F.unpack_nibbles(packed))
+    if fmt.codes == "e2m1":
+        return F.decode_e2m1(F.unpack_nibbles(packed))
+    if fmt.codes == "int8":
+        return F.decode_int8(packed)
+    u = F.unpack_sixbits(packed) if fmt.code_bits == 6 else packed
+    return F.decode_fp_element(u, fmt.codes)
 
 
 def decode_scales(u: np.ndarray, fmt: Format) -> np.ndarray:

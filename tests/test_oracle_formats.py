@@ -129,3 +129,86 @@ def test_bf16_encoding_bit_pattern():
     for v in (0.015625, 3.140625, -0.0009765625):
         want = struct.unpack(">I", struct.pack(">f", v))[0] >> 16
         assert F.encode_bf16(np.array([v]))[0] == want
+
+
+# --------------------------------------------------------------------------- #
+# The other element formats of the MX family
+# --------------------------------------------------------------------------- #
+
+def _grid_from_bits(eb, mb, bias):
+    """Magnitudes of all codes of a float element format, written from the
+    bit layout independently of the oracle's table (NaN/Inf codes dropped by
+    the caller)."""
+    out = []
+    for e in range(1 << eb):
+        for m in range(1 << mb):
+            frac = m / (1 << mb)
+            out.append(math.ldexp(frac, 1 - bias) if e == 0 else math.ldexp(1 + frac, e - bias))
+    return np.array(out)
+
+
+@pytest.mark.parametrize("name,eb,mb,bias,top,nfinite", [
+    ("e4m3", 4, 3, 7, 448.0, 127), ("e5m2", 5, 2, 15, 57344.0, 124),
+    ("e2m3", 2, 3, 1, 7.5, 32), ("e3m2", 3, 2, 3, 28.0, 32)])
+def test_fp_element_rounding_brute_force(name, eb, mb, bias, top, nfinite):
+    grid = _grid_from_bits(eb, mb, bias)[:nfinite]
+    assert grid[-1] == top and np.all(np.diff(grid) > 0)
+    vals = F.fp_element_values(name)
+    assert np.array_equal(vals[:nfinite], grid) and np.all(np.isnan(vals[nfinite:]))
+    rng = np.random.default_rng(11)
+    mids = (grid[:-1] + grid[1:]) / 2
+    x = np.concatenate([grid, mids, np.nextafter(mids, 0), np.nextafter(mids, np.inf),
+                        rng.uniform(0, 1.3 * top, 4000), top * np.exp(rng.uniform(-30, 0, 4000)),
+                        [top * 1.01, top * 2, 1e30]])
+    x = np.concatenate([x, -x])
+    got = F.round_fp_element(x, name)
+    # brute force: nearest grid magnitude of min(|x|, top); ties to the even code
+    ax = np.minimum(np.abs(x), top)
+    d = np.abs(ax[:, None] - grid[None, :])
+    best = d.min(axis=1, keepdims=True)
+    cand = d == best
+    idx = np.where(cand & (np.arange(nfinite) % 2 == 0), np.arange(nfinite), 1 << 20).min(axis=1)
+    idx = np.where(idx == 1 << 20, np.argmax(cand, axis=1), idx)
+    want = np.copysign(grid[idx], x)
+    assert np.array_equal(got, want)
+    assert np.array_equal(np.signbit(got), np.signbit(x))
+    # codes: sign bit above the magnitude bits, round trip
+    enc = F.encode_fp_element(want, name)
+    assert np.array_equal(enc & ((1 << (eb + mb)) - 1), idx)
+    assert np.array_equal(F.decode_fp_element(enc, name), want)
+
+
+@pytest.mark.parametrize("name,dt", [("e4m3", torch.float8_e4m3fn), ("e5m2", torch.float8_e5m2)])
+def test_fp8_elements_match_torch(name, dt):
+    # every finite code decodes as torch decodes it
+    codes = np.arange(256, dtype=np.uint8)
+    tv = torch.from_numpy(codes).view(dt).to(torch.float64).numpy()
+    fin = np.isfinite(tv)
+    assert np.array_equal(F.decode_fp_element(codes[fin], name), tv[fin])
+    # rounding of float32 inputs inside the range matches torch's cast
+    top = F.FP_ELEMENTS[name][3]
+    rng = np.random.default_rng(12)
+    x = (rng.uniform(-top, top, 100000) * np.exp(rng.uniform(-25, 0, 100000))).astype(np.float32)
+    want = torch.from_numpy(x).to(dt).to(torch.float64).numpy()
+    assert np.array_equal(F.round_fp_element(x.astype(np.float64), name), want)
+
+
+def test_int8_elements():
+    q = np.array([2.5, -2.5, 3.5, 126.5, 127.4, 127.6, 300.0, -127.5, -128.4, -129.0, 0.49])
+    assert list(F.round_int8(q)) == [2, -2, 4, 126, 127, 127, 127, -128, -128, -128, 0]
+    for v in np.linspace(-200, 200, 801):
+        assert F.round_int8(np.array([v]))[0] == max(-128, min(127, round(v)))
+    c = np.arange(-128, 128, dtype=np.float64)
+    u = F.encode_int8(c)
+    assert list(u[:2]) == [0x80, 0x81] and u[128] == 0 and u[-1] == 0x7F
+    assert np.array_equal(F.decode_int8(u), c)
+
+
+def test_six_bit_packing():
+    # four codes in one little-endian 24-bit word, the first in the low bits
+    assert list(F.pack_sixbits(np.array([1, 2, 3, 4]))) == [0x81, 0x30, 0x10]
+    rng = np.random.default_rng(13)
+    c = rng.integers(0, 64, (3, 32)).astype(np.uint8)
+    p = F.pack_sixbits(c)
+    assert p.shape == (3, 24)
+    assert np.array_equal(F.unpack_sixbits(p), c)

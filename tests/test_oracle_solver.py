@@ -15,6 +15,12 @@ import oracle as O
 import synth
 
 FORMATS = ["int4_bf16", "mxint4", "mxfp4", "nvfp4"]
+# the rest of the MX family
+MX_MORE = ["mxfp8_e4m3", "mxfp8_e5m2", "mxfp6_e2m3", "mxfp6_e3m2", "mxint8"]
+ALL_FORMATS = FORMATS + MX_MORE
+# element float formats: (significant bits, lowest normal exponent, largest value)
+FP_ELEM = {"e4m3": (4, -6, Fr(448)), "e5m2": (3, -14, Fr(57344)),
+           "e2m3": (4, 0, Fr(15, 2)), "e3m2": (3, -2, Fr(28))}
 E2M1 = [Fr(0), Fr(1, 2), Fr(1), Fr(3, 2), Fr(2), Fr(3), Fr(4), Fr(6)]
 
 
@@ -54,6 +60,12 @@ def py_group_scale(g: Fr, gscale: str) -> Fr:
 def py_code(q: Fr, codes: str) -> Fr:
     if codes == "int4":
         return Fr(min(7, max(-8, round(q))))
+    if codes == "int8":
+        return Fr(min(127, max(-128, round(q))))
+    if codes in FP_ELEM:
+        p, emin, mx = FP_ELEM[codes]
+        v = Fr(0) if q == 0 else _rne(abs(q), p, emin, mx)
+        return v if q >= 0 else -v
     aq = min(abs(q), Fr(6))
     d = [abs(aq - g) for g in E2M1]
     best = min(d)
@@ -71,7 +83,7 @@ def py_quantize(Y, fmt, ts=Fr(1)):
         for g in range(cols // G):
             grp = Y[i][g * G:(g + 1) * G]
             m = max(abs(v) for v in grp)
-            s = Fr(1) if m == 0 else py_group_scale(m / (Fr(int(fmt.qmax)) * ts), fmt.gscale)
+            s = Fr(1) if m == 0 else py_group_scale(m / (Fr(fmt.qmax) * ts), fmt.gscale)
             S[i][g] = s
             for k, v in enumerate(grp):
                 C[i][g * G + k] = py_code(v / (s * ts), fmt.codes)
@@ -86,7 +98,7 @@ def _small_matrix(rows, cols, seed, outliers=True):
     return torch.from_numpy(W).to(torch.bfloat16).double().numpy()
 
 
-@pytest.mark.parametrize("name", FORMATS)
+@pytest.mark.parametrize("name", ALL_FORMATS)
 @pytest.mark.parametrize("G", [16, 32, 64])
 def test_quantize_matches_exact_rational_restatement(name, G):
     fmt = O.preset(name, G)
@@ -135,7 +147,7 @@ def test_quantize_hand_cases():
     assert s[0, 0] == 448.0 and c[0, 0] == 6 and c[0, 1] == -6
 
 
-@pytest.mark.parametrize("name", FORMATS)
+@pytest.mark.parametrize("name", ALL_FORMATS)
 def test_quantizer_idempotent(name):
     fmt = O.preset(name)
     W = _small_matrix(16, 4 * fmt.group, seed=5)
@@ -176,7 +188,7 @@ def _admissible(fmt, x):
     return v[(v > x / 4) & (v < x * 4)]
 
 
-@pytest.mark.parametrize("name", FORMATS)
+@pytest.mark.parametrize("name", ALL_FORMATS)
 def test_row_and_column_updates_minimise_over_the_scale_set(name):
     fmt = O.preset(name)
     W = _small_matrix(6, 2 * fmt.group, seed=17)
@@ -229,7 +241,7 @@ def test_zero_slices_keep_scale_one():
     assert b[5] == 1.0 and np.isnan(xb[5])
 
 
-@pytest.mark.parametrize("name", FORMATS)
+@pytest.mark.parametrize("name", ALL_FORMATS)
 def test_outputs_are_representable(name):
     fmt = O.preset(name)
     W = _small_matrix(32, 4 * fmt.group, seed=23)
@@ -258,7 +270,7 @@ def test_initial_state_is_single_scale_rtn():
     assert r["mse_trace"][0] == pytest.approx(float(err), rel=1e-13)
 
 
-@pytest.mark.parametrize("name", FORMATS)
+@pytest.mark.parametrize("name", ALL_FORMATS)
 def test_fixed_code_half_steps_never_increase_the_error(name):
     # with the codes held fixed, each closed-form + nearest-projection step is
     # the exact minimiser over the scale set, so it cannot raise the MSE
@@ -279,7 +291,7 @@ def test_fixed_code_half_steps_never_increase_the_error(name):
         b = b2
 
 
-@pytest.mark.parametrize("name", ["mxint4", "mxfp4"])
+@pytest.mark.parametrize("name", ["mxint4", "mxfp4"] + MX_MORE)
 def test_power_of_two_row_step_leaves_mx_reconstruction_unchanged(name):
     # E8M0 row scale with E8M0 group scales: a power of two only shifts every
     # group exponent, so D_a Qhat is unchanged and the row half-step MSE equals
@@ -312,7 +324,7 @@ def test_toy_workload_trace():
 # Activation rescale + quantize
 # --------------------------------------------------------------------------- #
 
-@pytest.mark.parametrize("name", FORMATS)
+@pytest.mark.parametrize("name", ALL_FORMATS)
 def test_activation_path(name):
     fmt = O.preset(name)
     rng = np.random.default_rng(5)
@@ -357,3 +369,20 @@ def test_generator_matches_integer_splitmix64():
         assert (int(bits[i]) & M) == want
     u = synth.uniform(key, 50, offset=1000)
     assert float(u[0]) == ((sm((key + 1000 * synth.GOLDEN) & M) >> 11) + 0.5) * 2.0 ** -53
+
+
+@pytest.mark.parametrize("name,s,c_max,c_03", [
+    # group max 1.0 and an element 0.3, G32, E8M0 scale = smallest 2^e >= 1/qmax
+    ("mxfp8_e4m3", 2.0 ** -8, 256.0, 80.0),      # 0.3*256 = 76.8 -> grid step 8 -> 80
+    ("mxfp8_e5m2", 2.0 ** -15, 32768.0, 10240.0),  # 9830.4 -> step 2048 -> 10240
+    ("mxfp6_e2m3", 2.0 ** -2, 4.0, 1.25),        # 1.2 -> step 0.125 -> 1.25
+    ("mxfp6_e3m2", 2.0 ** -4, 16.0, 5.0),        # 4.8 -> step 1 -> 5
+    ("mxint8", 2.0 ** -6, 64.0, 19.0),           # 19.2 -> 19
+])
+def test_quantize_hand_cases_mx_family(name, s, c_max, c_03):
+    fmt = O.preset(name)
+    y = np.zeros((1, 32))
+    y[0, 0], y[0, 1], y[0, 2] = 1.0, 0.3, -0.3
+    c, sc = O.quantize(y, fmt)
+    assert sc[0, 0] == s
+    assert c[0, 0] == c_max and c[0, 1] == c_03 and c[0, 2] == -c_03
