@@ -17,13 +17,14 @@ __all__ = [
     "DqError", "dq_format", "dq_matrix", "lib", "library_path", "version", "format_preset",
     "workspace_size", "quantize", "dequantize", "solve_dual_scale", "solve_dual_scale_batched",
     "row_update", "col_update", "act_rescale_quant", "last_device_status", "EXPORTS",
-    "kernel_timing", "kernel_time", "launch_count", "solve_dual_scale_noalloc",
+    "kernel_timing", "kernel_time", "launch_count", "solve_dual_scale_noalloc", "code_bytes",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libdq.so")
 
-DQ_CODES_INT4, DQ_CODES_E2M1 = 0, 1
+DQ_CODES_INT4, DQ_CODES_E2M1, DQ_CODES_INT8, DQ_CODES_E4M3 = 0, 1, 2, 3
+DQ_CODES_E5M2, DQ_CODES_E2M3, DQ_CODES_E3M2 = 4, 5, 6
 DQ_SCALE_BF16, DQ_SCALE_E8M0, DQ_SCALE_E4M3 = 0, 1, 2
 DQ_DT_F32, DQ_DT_BF16 = 0, 1
 DQ_OK, DQ_ERR_NONFINITE, DQ_ERR_RANGE = 0, -4, -5
@@ -32,7 +33,7 @@ EXPORTS = ("dq_version", "dq_strerror", "dq_format_preset", "dq_workspace_size",
            "dq_dequantize", "dq_solve_dual_scale", "dq_solve_dual_scale_batched",
            "dq_row_update", "dq_col_update", "dq_act_rescale_quant", "dq_last_device_status",
            "dq_kernel_timing", "dq_kernel_time", "dq_launch_count",
-           "dq_solve_dual_scale_noalloc")
+           "dq_solve_dual_scale_noalloc", "dq_code_bytes")
 
 
 class DqError(RuntimeError):
@@ -101,6 +102,7 @@ def lib() -> ctypes.CDLL:
         "dq_kernel_timing": (c_int32, [c_int32]),
         "dq_kernel_time": (c_int32, [c_int32, P(c_double), P(c_int64)]),
         "dq_launch_count": (c_int64, []),
+        "dq_code_bytes": (c_int64, [P(dq_format), c_int64, c_int64]),
         "dq_solve_dual_scale_noalloc": (c_int32, [c_void_p, c_int32, c_int64, c_int64,
                                                   P(dq_format), c_int32, c_void_p, c_void_p,
                                                   c_void_p, c_void_p, c_void_p, c_void_p,
@@ -176,9 +178,18 @@ def workspace(shapes, fmt: dq_format, device=None) -> torch.Tensor:
                        device=device or torch.device("cuda"))
 
 
+def code_bytes(fmt, rows, cols) -> int:
+    """Bytes of the codes of a rows x cols matrix (rows of cols*bits/8 bytes)."""
+    n = lib().dq_code_bytes(ctypes.byref(fmt), rows, cols)
+    if n < 0:
+        raise DqError(-3 if cols % max(fmt.group, 1) == 0 else -2, "dq_code_bytes")
+    return n
+
+
 def _outputs(rows, cols, fmt, device, codes=None, gscales=None):
     if codes is None:
-        codes = torch.empty(rows, cols // 2, dtype=torch.uint8, device=device)
+        per_row = code_bytes(fmt, 1, cols) if rows > 0 else 0
+        codes = torch.empty(rows, per_row, dtype=torch.uint8, device=device)
     if gscales is None:
         gscales = torch.empty(rows, cols // fmt.group, dtype=gscale_dtype(fmt), device=device)
     return codes, gscales
@@ -186,7 +197,7 @@ def _outputs(rows, cols, fmt, device, codes=None, gscales=None):
 
 def quantize(X, fmt, a=None, b=None, tensor_scale: float = 1.0, codes=None, gscales=None,
              stream=None):
-    """Q(X / (a b^T)) -> (codes [rows, cols/2] uint8, group scales [rows, cols/G])."""
+    """Q(X / (a b^T)) -> (codes [rows, cols*bits/8] uint8, group scales [rows, cols/G])."""
     _need_cuda(X, a, b)
     rows, cols = X.shape
     codes, gscales = _outputs(rows, cols, fmt, X.device, codes, gscales)
@@ -321,7 +332,7 @@ def col_update(W, fmt, a_in, b_in, tensor_scale=1.0, ws=None, stream=None):
 
 
 def act_rescale_quant(X, b, fmt, codes=None, gscales=None, stream=None):
-    """Q(X D_b): returns (codes [tokens, K/2], group scales [tokens, K/G])."""
+    """Q(X D_b): returns (codes [tokens, K*bits/8], group scales [tokens, K/G])."""
     _need_cuda(X, b)
     if X.dtype != torch.bfloat16:
         raise TypeError("activations are bfloat16")

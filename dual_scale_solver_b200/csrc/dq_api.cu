@@ -74,6 +74,7 @@ struct FmtInfo {
     int combo;
     int G;
     float qmax;
+    int bits;       // stored bits per code
 };
 
 dq_status check_format(const dq_format *f, FmtInfo *out) {
@@ -89,11 +90,21 @@ dq_status check_format(const dq_format *f, FmtInfo *out) {
     if (c == DQ_CODES_E2M1 && g == DQ_SCALE_E4M3 && o == DQ_SCALE_BF16) combo = COMBO_E2M1_E4M3_BF16;
     if (c == DQ_CODES_INT4 && g == DQ_SCALE_E8M0 && o == DQ_SCALE_BF16) combo = COMBO_INT4_E8M0_BF16;
     if (c == DQ_CODES_E2M1 && g == DQ_SCALE_E8M0 && o == DQ_SCALE_BF16) combo = COMBO_E2M1_E8M0_BF16;
+    // the other MX element formats: E8M0 group and outer scales only
+    const bool mx = g == DQ_SCALE_E8M0 && o == DQ_SCALE_E8M0;
+    if (mx && c == DQ_CODES_INT8) combo = COMBO_INT8_E8M0_E8M0;
+    if (mx && c == DQ_CODES_E4M3) combo = COMBO_E4M3_E8M0_E8M0;
+    if (mx && c == DQ_CODES_E5M2) combo = COMBO_E5M2_E8M0_E8M0;
+    if (mx && c == DQ_CODES_E2M3) combo = COMBO_E2M3_E8M0_E8M0;
+    if (mx && c == DQ_CODES_E3M2) combo = COMBO_E3M2_E8M0_E8M0;
     if (combo < 0) return DQ_ERR_FORMAT;
     if (out) {
+        static const float qmax[7] = {7.0f, 6.0f, 127.0f, 448.0f, 57344.0f, 7.5f, 28.0f};
+        static const int bits[7] = {4, 4, 8, 8, 8, 6, 6};
         out->combo = combo;
         out->G = f->group;
-        out->qmax = (c == DQ_CODES_INT4) ? 7.0f : 6.0f;
+        out->qmax = qmax[c];
+        out->bits = bits[c];
     }
     return DQ_OK;
 }
@@ -193,13 +204,22 @@ cudaError_t launch_tiles(int combo, const TileLaunch &L) {
         case 3: return launch_tile_c3(L);
         case 4: return launch_tile_c4(L);
         case 5: return launch_tile_c5(L);
+        case 6: return launch_tile_c6(L);
+        case 7: return launch_tile_c7(L);
+        case 8: return launch_tile_c8(L);
+        case 9: return launch_tile_c9(L);
+        case 10: return launch_tile_c10(L);
     }
     return cudaErrorInvalidValue;
 }
 
-int outer_of(int combo) {
-    return (combo == COMBO_INT4_E8M0_E8M0 || combo == COMBO_E2M1_E8M0_E8M0) ? SC_E8M0 : SC_BF16;
+// format sets whose group and outer scales are both E8M0 (the MX family)
+bool all_e8m0(int combo) {
+    return combo == COMBO_INT4_E8M0_E8M0 || combo == COMBO_E2M1_E8M0_E8M0 ||
+           combo >= COMBO_INT8_E8M0_E8M0;
 }
+
+int outer_of(int combo) { return all_e8m0(combo) ? SC_E8M0 : SC_BF16; }
 
 unsigned grid_for(int64_t n, int block) {
     int64_t g = (n + block - 1) / block;
@@ -324,9 +344,7 @@ struct Launcher {
 };
 
 // MX formats: power-of-two outer and group scales
-bool fused_ok(int combo) {
-    return combo == COMBO_INT4_E8M0_E8M0 || combo == COMBO_E2M1_E8M0_E8M0;
-}
+bool fused_ok(int combo) { return all_e8m0(combo); }
 
 thread_local std::vector<MatDesc> t_table;
 
@@ -507,6 +525,37 @@ dq_status step_impl(bool row_step, const void *W, int32_t dtype, int64_t rows, i
     return DQ_OK;
 }
 
+// Value of the stored code of element (r, c) (layouts as the tile kernel
+// writes them: 4-bit codes two per byte, 8-bit one per byte, 6-bit four per
+// 3 bytes).  Float element formats decode from their bit fields.
+__device__ float code_value(const uint8_t *codes, int64_t r, int64_t c, int64_t cols, int kind) {
+    if (kind == DQ_CODES_INT4 || kind == DQ_CODES_E2M1) {
+        const uint8_t byte = codes[r * (cols / 2) + c / 2];
+        const uint32_t nib = (c & 1) ? (byte >> 4) : (byte & 0xF);
+        if (kind == DQ_CODES_INT4) return (float)((int)(nib ^ 8u) - 8);
+        const float mag[8] = {0.f, 0.5f, 1.f, 1.5f, 2.f, 3.f, 4.f, 6.f};
+        return (nib & 8u) ? -mag[nib & 7u] : mag[nib & 7u];
+    }
+    if (kind == DQ_CODES_INT8) return (float)(int8_t)codes[r * cols + c];
+    uint32_t u;
+    int eb, mb, bias;
+    if (kind == DQ_CODES_E4M3 || kind == DQ_CODES_E5M2) {
+        u = codes[r * cols + c];
+        eb = kind == DQ_CODES_E4M3 ? 4 : 5;
+    } else {
+        const uint8_t *q = codes + r * (cols / 4 * 3) + (c / 4) * 3;
+        const uint32_t w = q[0] | ((uint32_t)q[1] << 8) | ((uint32_t)q[2] << 16);
+        u = (w >> (6 * (c % 4))) & 0x3Fu;
+        eb = kind == DQ_CODES_E2M3 ? 2 : 3;
+    }
+    mb = (kind == DQ_CODES_E4M3 || kind == DQ_CODES_E2M3) ? 3 : 2;
+    bias = (1 << (eb - 1)) - 1;
+    const uint32_t e = (u >> mb) & ((1u << eb) - 1), m = u & ((1u << mb) - 1);
+    const float v = e == 0 ? ldexpf((float)m, 1 - bias - mb)
+                           : ldexpf((float)((1u << mb) + m), (int)e - bias - mb);
+    return (u >> (eb + mb)) & 1u ? -v : v;
+}
+
 // out_ij = a_i * c_ij * s_g * ts * b_j
 __global__ void dequant_kernel(const uint8_t *codes, const void *gs, int64_t rows, int64_t cols,
                                int G, int codes_kind, int gs_kind, float ts, const float *a,
@@ -516,15 +565,7 @@ __global__ void dequant_kernel(const uint8_t *codes, const void *gs, int64_t row
     for (int64_t k = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; k < n;
          k += (int64_t)gridDim.x * blockDim.x) {
         const int64_t r = k / cols, c = k % cols;
-        const uint8_t byte = codes[r * (cols / 2) + c / 2];
-        const uint32_t nib = (c & 1) ? (byte >> 4) : (byte & 0xF);
-        float cv;
-        if (codes_kind == DQ_CODES_INT4) {
-            cv = (float)((int)(nib ^ 8u) - 8);
-        } else {
-            const float mag[8] = {0.f, 0.5f, 1.f, 1.5f, 2.f, 3.f, 4.f, 6.f};
-            cv = (nib & 8u) ? -mag[nib & 7u] : mag[nib & 7u];
-        }
+        const float cv = code_value(codes, r, c, cols, codes_kind);
         const int64_t gi = r * (cols / G) + c / G;
         float s;
         if (gs_kind == DQ_SCALE_BF16) {
@@ -574,12 +615,24 @@ dq_status dq_format_preset(const char *name, int32_t group, dq_format *out) {
     else if (!strcmp(name, "mxint4")) f = {DQ_CODES_INT4, 32, DQ_SCALE_E8M0, DQ_SCALE_E8M0, 0};
     else if (!strcmp(name, "mxfp4")) f = {DQ_CODES_E2M1, 32, DQ_SCALE_E8M0, DQ_SCALE_E8M0, 0};
     else if (!strcmp(name, "nvfp4")) f = {DQ_CODES_E2M1, 16, DQ_SCALE_E4M3, DQ_SCALE_BF16, 1};
+    else if (!strcmp(name, "mxint8")) f = {DQ_CODES_INT8, 32, DQ_SCALE_E8M0, DQ_SCALE_E8M0, 0};
+    else if (!strcmp(name, "mxfp8_e4m3")) f = {DQ_CODES_E4M3, 32, DQ_SCALE_E8M0, DQ_SCALE_E8M0, 0};
+    else if (!strcmp(name, "mxfp8_e5m2")) f = {DQ_CODES_E5M2, 32, DQ_SCALE_E8M0, DQ_SCALE_E8M0, 0};
+    else if (!strcmp(name, "mxfp6_e2m3")) f = {DQ_CODES_E2M3, 32, DQ_SCALE_E8M0, DQ_SCALE_E8M0, 0};
+    else if (!strcmp(name, "mxfp6_e3m2")) f = {DQ_CODES_E3M2, 32, DQ_SCALE_E8M0, DQ_SCALE_E8M0, 0};
     else return DQ_ERR_FORMAT;
     if (group != 0) f.group = group;
     dq_status s = check_format(&f, nullptr);
     if (s != DQ_OK) return s;
     *out = f;
     return DQ_OK;
+}
+
+int64_t dq_code_bytes(const dq_format *fmt, int64_t rows, int64_t cols) {
+    FmtInfo fi;
+    if (check_format(fmt, &fi) != DQ_OK) return -1;
+    if (rows < 0 || cols < 0 || cols % fi.G) return -1;
+    return rows * (cols * fi.bits / 8);
 }
 
 dq_status dq_workspace_size(int32_t n, const int64_t *rows, const int64_t *cols,

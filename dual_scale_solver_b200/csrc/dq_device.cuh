@@ -24,7 +24,8 @@
 
 namespace dq {
 
-enum { CODES_INT4 = 0, CODES_E2M1 = 1 };
+enum { CODES_INT4 = 0, CODES_E2M1 = 1, CODES_INT8 = 2, CODES_E4M3 = 3, CODES_E5M2 = 4,
+       CODES_E2M3 = 5, CODES_E3M2 = 6 };
 enum { SC_BF16 = 0, SC_E8M0 = 1, SC_E4M3 = 2 };
 enum { MODE_ROW = 0, MODE_COL = 1, MODE_PACK = 2, MODE_ACT = 3, MODE_FUSED = 4 };
 enum { STATUS_NONFINITE = 1u, STATUS_RANGE = 2u };
@@ -35,6 +36,26 @@ constexpr int kRowsPerWarp[5] = {128, 256, 128, 128, 256};   // per mode (at mos
 constexpr int kRing = 4;             // cp.async ring slots per lane (rows in flight + 1)
 constexpr float kBf16Max = 3.38953138925153547590470800371487866880e+38f;  // (2-2^-7)*2^127
 constexpr float kMinNormal = 1.17549435082228750796873653722224568e-38f;    // 2^-126
+
+// Element grid of each code type.  qmax = the largest code magnitude =
+// (1 + kMT / 2^23) * 2^kQE; kBits stored bits per code.  INT4 and E2M1 are
+// the pages' codebooks; INT8, E4M3, E5M2 (MXFP8), E2M3 and E3M2 (MXFP6) are
+// the other element formats of the MX family (OCP Microscaling definition).
+template <int CODES> struct CodeTraits;
+template <> struct CodeTraits<CODES_INT4> {
+    static constexpr float kQmax = 7.0f;   static constexpr int kQE = 2;  static constexpr uint32_t kMT = 0x600000u; static constexpr int kBits = 4; };
+template <> struct CodeTraits<CODES_E2M1> {
+    static constexpr float kQmax = 6.0f;   static constexpr int kQE = 2;  static constexpr uint32_t kMT = 0x400000u; static constexpr int kBits = 4; };
+template <> struct CodeTraits<CODES_INT8> {
+    static constexpr float kQmax = 127.0f; static constexpr int kQE = 6;  static constexpr uint32_t kMT = 0x7E0000u; static constexpr int kBits = 8; };
+template <> struct CodeTraits<CODES_E4M3> {
+    static constexpr float kQmax = 448.0f; static constexpr int kQE = 8;  static constexpr uint32_t kMT = 0x600000u; static constexpr int kBits = 8; };
+template <> struct CodeTraits<CODES_E5M2> {
+    static constexpr float kQmax = 57344.0f; static constexpr int kQE = 15; static constexpr uint32_t kMT = 0x600000u; static constexpr int kBits = 8; };
+template <> struct CodeTraits<CODES_E2M3> {
+    static constexpr float kQmax = 7.5f;   static constexpr int kQE = 2;  static constexpr uint32_t kMT = 0x700000u; static constexpr int kBits = 6; };
+template <> struct CodeTraits<CODES_E3M2> {
+    static constexpr float kQmax = 28.0f;  static constexpr int kQE = 4;  static constexpr uint32_t kMT = 0x600000u; static constexpr int kBits = 6; };
 
 // Programmatic dependent launch.  The library launches its kernels with
 // programmatic stream serialization, so a kernel may start while the one
@@ -153,6 +174,61 @@ __device__ __forceinline__ float2 e2m1_round2_byte(float lo, float hi, uint32_t 
         : "=f"(a), "=f"(b), "=r"(byte) : "f"(lo), "f"(hi));
     return make_float2(a, b);
 }
+
+// Round a pair to an MX float element format (nearest even, saturating at
+// the largest finite value) and return the values as float32 (.x from lo);
+// `pair` receives the two codes, lo's in bits 0-7 and hi's in bits 8-15 (a
+// 6-bit code sits in the low bits of its byte).
+template <int CODES>
+__device__ __forceinline__ float2 fp_elem_round2(float lo, float hi, uint32_t &pair) {
+    uint16_t b;
+    uint32_t h2;
+    if constexpr (CODES == CODES_E4M3) {
+        asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(b) : "f"(hi), "f"(lo));
+        asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(b));
+    } else if constexpr (CODES == CODES_E5M2) {
+        asm("cvt.rn.satfinite.e5m2x2.f32 %0, %1, %2;" : "=h"(b) : "f"(hi), "f"(lo));
+        asm("cvt.rn.f16x2.e5m2x2 %0, %1;" : "=r"(h2) : "h"(b));
+    } else if constexpr (CODES == CODES_E2M3) {
+        asm("cvt.rn.satfinite.e2m3x2.f32 %0, %1, %2;" : "=h"(b) : "f"(hi), "f"(lo));
+        asm("cvt.rn.f16x2.e2m3x2 %0, %1;" : "=r"(h2) : "h"(b));
+    } else {
+        static_assert(CODES == CODES_E3M2, "float element formats only");
+        asm("cvt.rn.satfinite.e3m2x2.f32 %0, %1, %2;" : "=h"(b) : "f"(hi), "f"(lo));
+        asm("cvt.rn.f16x2.e3m2x2 %0, %1;" : "=r"(h2) : "h"(b));
+    }
+    pair = b;
+    float x, y;
+    asm("{ .reg .f16 l, h; mov.b32 {l, h}, %2; cvt.f32.f16 %0, l; cvt.f32.f16 %1, h; }"
+        : "=f"(x), "=f"(y) : "r"(h2));
+    return make_float2(x, y);
+}
+
+// Pack NP code pairs (8-bit codes in bits 0-7 and 8-15) into the stored
+// code words: 8-bit codes one per byte; 6-bit codes four per 24-bit
+// little-endian word (the first in the low bits), 3 bytes per 4 codes.
+template <int BITS, int NP>
+__device__ __forceinline__ void pack_code_pairs(const uint32_t (&pair)[NP], uint32_t (&cw)[2]) {
+    if constexpr (BITS == 8) {
+#pragma unroll
+        for (int k = 0; k < NP; ++k) cw[k >> 1] |= pair[k] << (16 * (k & 1));
+    } else {
+        static_assert(BITS == 6 && (NP == 2 || NP == 4), "6-bit codes come in quads");
+        uint32_t wq[NP / 2];
+#pragma unroll
+        for (int k = 0; k < NP / 2; ++k) {
+            const uint32_t p0 = pair[2 * k], p1 = pair[2 * k + 1];
+            wq[k] = (p0 & 0x3Fu) | (((p0 >> 8) & 0x3Fu) << 6) | ((p1 & 0x3Fu) << 12) |
+                    (((p1 >> 8) & 0x3Fu) << 18);
+        }
+        if constexpr (NP == 4) {
+            cw[0] = wq[0] | (wq[1] << 24);
+            cw[1] = wq[1] >> 8;
+        } else {
+            cw[0] = wq[0];
+        }
+    }
+}
 __device__ __forceinline__ uint32_t e4m3_bits(float x) {    // x exactly representable
     uint16_t r;
     asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(x));
@@ -214,14 +290,15 @@ __device__ __forceinline__ ScaleChoice project_group(float m, float qts, float r
         uint32_t u = __float_as_uint(mm);
         int k = ilog2f(mm);
         uint32_t mant = u & 0x7FFFFFu;
-        constexpr uint32_t MT = (CODES == CODES_INT4) ? 0x600000u : 0x400000u;  // 1.75 / 1.5
-        e = k - 2 + (mant > MT ? 1 : 0);
-        int elo = min(max(k - 2, -126), 126), ehi = min(max(k - 1, -126), 126);
+        constexpr uint32_t MT = CodeTraits<CODES>::kMT;
+        constexpr int QE = CodeTraits<CODES>::kQE;
+        e = k - QE + (mant > MT ? 1 : 0);
+        int elo = min(max(k - QE, -126), 126), ehi = min(max(k - QE + 1, -126), 126);
         e = min(max(e, -126), 126);
         c.s = pow2f(e);
         c.s_lo = pow2f(elo);
         c.s_hi = pow2f(ehi);
-        c.s_tie = c.s_lo;                              // m == qmax*2^(k-2): ceil is exact
+        c.s_tie = c.s_lo;                              // m == qmax*2^(k-QE): ceil is exact
         int d = (int)mant - (int)MT;
         c.near = (d < 16 && d > -16);
         c.thr = __uint_as_float((u & 0xFF800000u) | MT) * (1.0f / inv_ts);  // Q*2^k*ts
@@ -292,18 +369,21 @@ struct Quant {
     static constexpr bool kExactQ = ACT ? (GS == SC_E8M0) : (GS == SC_E8M0 && OS == SC_E8M0);
     // exact group max (the inner scaling by b, and by a, is exact)
     static constexpr bool kExactM = ACT ? true : (OS == SC_E8M0);
-    static constexpr float kQmax = CODES == CODES_INT4 ? 7.0f : 6.0f;
+    static constexpr float kQmax = CodeTraits<CODES>::kQmax;
+    static constexpr int kBits = CodeTraits<CODES>::kBits;
 
     // In: w (input values), z = inner-scaled values before the row factor
     // (w/b_j for weights, x*b_j for activations), a and ia = 1/a (1 for ACT),
     // bj (b_j; read on the exact path only), ts and 1/ts (E4M3 only).
-    // Out: c (code values), s (stored group scale), s_eff = s*ts, nib (the
-    // chunk's packed nibbles, element 0 lowest; only when NIB).
+    // Out: c (code values), s (stored group scale), s_eff = s*ts, cw (the
+    // chunk's stored codes, element 0 lowest, kBits each -- 4-bit codes two
+    // per byte, 8-bit codes one per byte, 6-bit codes four per 3 bytes; only
+    // when NIB).
     template <bool NIB>
     __device__ __forceinline__ static void run(const f2 (&w)[NP], const f2 (&z)[NP], float a,
                                                float ia, const f2 (&bj)[NP], float ts,
                                                float inv_ts, unsigned int *status, f2 (&c)[NP],
-                                               float &s, float &s_eff, uint32_t &nib,
+                                               float &s, float &s_eff, uint32_t (&cw)[2],
                                                bool &nonzero) {
         float mz = 0.0f;
 #pragma unroll
@@ -318,12 +398,13 @@ struct Quant {
         const bool pos = finite && m > 0.0f;
         nonzero = pos;
         if (GS == SC_E8M0 && kExactM) {
-            // smallest 2^e with qmax 2^e >= m (m exact): e = E(m) - 2, plus 1
-            // when m's significand exceeds qmax/4 (1.75 INT4, 1.5 E2M1);
-            // e >= -126 (also covers subnormal m); e <= 126 holds for finite m
-            constexpr uint32_t MT = (CODES == CODES_INT4) ? 0x600000u : 0x400000u;
+            // smallest 2^e with qmax 2^e >= m (m exact): e = E(m) - E(qmax),
+            // plus 1 when m's significand exceeds qmax's; e >= -126 (also
+            // covers subnormal m); e <= 126 holds for finite m
+            constexpr uint32_t MT = CodeTraits<CODES>::kMT;
+            constexpr int QE = CodeTraits<CODES>::kQE;
             // (the carry of the addition below adds that 1 to the exponent field)
-            const int sb = max((int)((mb + (0x7FFFFFu - MT)) & 0x7F800000u) - (2 << 23), 1 << 23);
+            const int sb = max((int)((mb + (0x7FFFFFu - MT)) & 0x7F800000u) - (QE << 23), 1 << 23);
             s = __uint_as_float((uint32_t)sb);
             if (NIB && !pos) s = 1.0f;                     // stored scale of an all-zero group
         } else {
@@ -367,10 +448,11 @@ struct Quant {
         f2 q[NP];
 #pragma unroll
         for (int k = 0; k < NP; ++k) q[k] = mul2(z[k], bcast(r));
-        nib = 0;
-        if (CODES == CODES_INT4) {
-            // round half to even; |q| <= 7 (E8M0 round-up) or < 7.5 (BF16
-            // nearest) so the codebook clamp never binds for these sets
+        cw[0] = 0;
+        cw[1] = 0;
+        if constexpr (CODES == CODES_INT4 || CODES == CODES_INT8) {
+            // round half to even; |q| <= qmax (E8M0 round-up) or < qmax + 0.5
+            // (BF16 nearest, INT4 only) so the codebook clamp never binds
 #pragma unroll
             for (int k = 0; k < NP; ++k) c[k] = make_float2(rintf(q[k].x), rintf(q[k].y));
             if (!kExactQ) {
@@ -404,12 +486,21 @@ struct Quant {
                 }
             }
             if (NIB) {
+                if constexpr (kBits == 4) {
 #pragma unroll
-                for (int k = 0; k < NP; ++k)
-                    nib |= ((((uint32_t)(int)c[k].x) & 0xFu) | ((((uint32_t)(int)c[k].y) & 0xFu) << 4))
-                           << (8 * k);
+                    for (int k = 0; k < NP; ++k)
+                        cw[0] |= ((((uint32_t)(int)c[k].x) & 0xFu) |
+                                  ((((uint32_t)(int)c[k].y) & 0xFu) << 4)) << (8 * k);
+                } else {
+                    uint32_t pair[NP];
+#pragma unroll
+                    for (int k = 0; k < NP; ++k)
+                        pair[k] = (((uint32_t)(int)c[k].x) & 0xFFu) |
+                                  ((((uint32_t)(int)c[k].y) & 0xFFu) << 8);
+                    pack_code_pairs<kBits, NP>(pair, cw);
+                }
             }
-        } else {
+        } else if constexpr (CODES == CODES_E2M1) {
             if (kExactQ && !NIB) {
 #pragma unroll
                 for (int k = 0; k < NP; ++k) c[k] = e2m1_round2(q[k].x, q[k].y);
@@ -449,9 +540,17 @@ struct Quant {
                 }
                 if (NIB) {
 #pragma unroll
-                    for (int k = 0; k < NP; ++k) nib |= byte[k] << (8 * k);
+                    for (int k = 0; k < NP; ++k) cw[0] |= byte[k] << (8 * k);
                 }
             }
+        } else {
+            // MX float elements (E4M3, E5M2, E2M3, E3M2): with power-of-two
+            // scales q is exact, so the hardware conversion decides each code
+            static_assert(kExactQ, "float element codes need power-of-two scales");
+            uint32_t pair[NP];
+#pragma unroll
+            for (int k = 0; k < NP; ++k) c[k] = fp_elem_round2<CODES>(q[k].x, q[k].y, pair[k]);
+            if constexpr (NIB) pack_code_pairs<kBits, NP>(pair, cw);
         }
     }
 };
@@ -585,7 +684,6 @@ tile_kernel(const __grid_constant__ Table tab, int mode_slot, int want_res, int6
     constexpr bool ROWSTAT = MODE == MODE_ROW || FUSED;
     constexpr bool COLSTAT = MODE == MODE_COL || FUSED;
     using Q = Quant<CODES, GS, OS, ACT, NP, LPG>;
-    constexpr int RPW = kRowsPerWarp[MODE];
     static_assert(!FUSED || (GS == SC_E8M0 && OS == SC_E8M0), "fused statistics need power-of-two scales");
     constexpr int ESZ = 16 / EPC;                    // bytes per element
 
@@ -688,7 +786,7 @@ tile_kernel(const __grid_constant__ Table tab, int mode_slot, int want_res, int6
 #pragma unroll
         for (int j = 0; j < NP; ++j) z[j] = mul2(w[j], cm[j]);
         float s, s_eff;
-        uint32_t nib;
+        uint32_t cw[2];
         bool nonzero;
         if (FUSED) {
             // Q(W / b): with power-of-two scales D_a Q(W / (a b)) equals it
@@ -696,12 +794,12 @@ tile_kernel(const __grid_constant__ Table tab, int mode_slot, int want_res, int6
             // as no group exponent of either reaches the E8M0 bounds: here
             // |e(s)| <= 100 for every non-zero group; the row finalize keeps
             // |e(a)| <= 20 (old) and <= 26 (new)
-            Q::template run<NIB>(w, z, 1.0f, 1.0f, bj, ts, inv_ts, tab.status, c, s, s_eff, nib,
+            Q::template run<NIB>(w, z, 1.0f, 1.0f, bj, ts, inv_ts, tab.status, c, s, s_eff, cw,
                                  nonzero);
             // s = 2^e with |e| <= 100: exponent field in [27, 227]
             clamp_risk |= nonzero && (__float_as_uint(s) - (27u << 23)) > (200u << 23);
         } else {
-            Q::template run<NIB>(w, z, a, ia, bj, ts, inv_ts, tab.status, c, s, s_eff, nib,
+            Q::template run<NIB>(w, z, a, ia, bj, ts, inv_ts, tab.status, c, s, s_eff, cw,
                                  nonzero);
         }
         if (ROWSTAT) {
@@ -769,9 +867,28 @@ tile_kernel(const __grid_constant__ Table tab, int mode_slot, int want_res, int6
                 }
             }
             if (col_ok) {
-                uint8_t *cp = md.codes + r * (cols >> 1) + (col >> 1);
-                if (EPC == 8) *reinterpret_cast<uint32_t *>(cp) = nib;
-                else *reinterpret_cast<uint16_t *>(cp) = (uint16_t)nib;
+                // codes: cols * BITS / 8 bytes per row; this lane's EPC codes
+                // start at byte col * BITS / 8 (aligned to their size: 4 or
+                // 8 bytes for 4- and 8-bit codes, 2 bytes for 6-bit codes
+                // in bf16 chunks, 1 byte in float32 chunks)
+                constexpr int BITS = CodeTraits<CODES>::kBits;
+                uint8_t *cp = md.codes + r * (cols * BITS / 8) + col * BITS / 8;
+                if (BITS == 4) {
+                    if (EPC == 8) *reinterpret_cast<uint32_t *>(cp) = cw[0];
+                    else *reinterpret_cast<uint16_t *>(cp) = (uint16_t)cw[0];
+                } else if (BITS == 8) {
+                    if (EPC == 8) *reinterpret_cast<uint2 *>(cp) = make_uint2(cw[0], cw[1]);
+                    else *reinterpret_cast<uint32_t *>(cp) = cw[0];
+                } else if (EPC == 8) {                      // 6-bit codes: 6 bytes
+                    uint16_t *cp2 = reinterpret_cast<uint16_t *>(cp);
+                    cp2[0] = (uint16_t)cw[0];
+                    cp2[1] = (uint16_t)(cw[0] >> 16);
+                    cp2[2] = (uint16_t)cw[1];
+                } else {                                    // 6-bit codes: 3 bytes
+                    cp[0] = (uint8_t)cw[0];
+                    cp[1] = (uint8_t)(cw[0] >> 8);
+                    cp[2] = (uint8_t)(cw[0] >> 16);
+                }
                 if ((lane % LPG) == 0) {
                     const int64_t gi = r * (cols / G) + col / G;
                     if (GS == SC_BF16)

@@ -33,7 +33,12 @@ enum Combo {
     COMBO_E2M1_E4M3_BF16 = 3,   // E2M1, E4M3 group, BF16 outer     ("nvfp4")
     COMBO_INT4_E8M0_BF16 = 4,   // INT4, E8M0 group, BF16 outer
     COMBO_E2M1_E8M0_BF16 = 5,   // E2M1, E8M0 group, BF16 outer
-    COMBO_COUNT = 6
+    COMBO_INT8_E8M0_E8M0 = 6,   // INT8, E8M0, E8M0                 ("mxint8")
+    COMBO_E4M3_E8M0_E8M0 = 7,   // E4M3 elements, E8M0, E8M0        ("mxfp8_e4m3")
+    COMBO_E5M2_E8M0_E8M0 = 8,   // E5M2 elements, E8M0, E8M0        ("mxfp8_e5m2")
+    COMBO_E2M3_E8M0_E8M0 = 9,   // E2M3 elements, E8M0, E8M0        ("mxfp6_e2m3")
+    COMBO_E3M2_E8M0_E8M0 = 10,  // E3M2 elements, E8M0, E8M0        ("mxfp6_e3m2")
+    COMBO_COUNT = 11
 };
 
 // Launch with programmatic stream serialization: the kernel may start while
@@ -62,6 +67,11 @@ cudaError_t launch_tile_c2(const TileLaunch &L);
 cudaError_t launch_tile_c3(const TileLaunch &L);
 cudaError_t launch_tile_c4(const TileLaunch &L);
 cudaError_t launch_tile_c5(const TileLaunch &L);
+cudaError_t launch_tile_c6(const TileLaunch &L);
+cudaError_t launch_tile_c7(const TileLaunch &L);
+cudaError_t launch_tile_c8(const TileLaunch &L);
+cudaError_t launch_tile_c9(const TileLaunch &L);
+cudaError_t launch_tile_c10(const TileLaunch &L);
 
 // One tile-kernel launch; the shared memory is dynamic (the row-statistics
 // layout needs more than the 48 KB default, opted in once per device).

@@ -69,7 +69,13 @@ typedef enum dq_status {
     DQ_ERR_SCRATCH = -10        /* matrix needs more than the built-in scratch buffer */
 } dq_status;
 
-enum { DQ_CODES_INT4 = 0, DQ_CODES_E2M1 = 1 };
+/* Code (element) types: the pages' INT4 and E2M1 codebooks, and the other
+ * element formats of the MX family the pages claim (OCP Microscaling
+ * definition): INT8 (MXINT8), E4M3 and E5M2 (MXFP8), E2M3 and E3M2 (MXFP6).
+ * qmax = 7, 6, 127, 448, 57344, 7.5, 28.  The last five need E8M0 group and
+ * outer scales. */
+enum { DQ_CODES_INT4 = 0, DQ_CODES_E2M1 = 1, DQ_CODES_INT8 = 2, DQ_CODES_E4M3 = 3,
+       DQ_CODES_E5M2 = 4, DQ_CODES_E2M3 = 5, DQ_CODES_E3M2 = 6 };
 enum { DQ_SCALE_BF16 = 0, DQ_SCALE_E8M0 = 1, DQ_SCALE_E4M3 = 2 };
 enum { DQ_DT_F32 = 0, DQ_DT_BF16 = 1 };
 
@@ -86,7 +92,7 @@ enum { DQ_DT_F32 = 0, DQ_DT_BF16 = 1 };
  * tensor_scale_auto = 1 gives weights a second-level scale
  * ts = 2^ceil(log2(amax(W) / (448 * qmax))) (NVFP4); otherwise ts = 1. */
 typedef struct dq_format {
-    int32_t codes;             /* DQ_CODES_* ; qmax = 7 (INT4) or 6 (E2M1) */
+    int32_t codes;             /* DQ_CODES_* */
     int32_t group;             /* G in {16, 32, 64} */
     int32_t group_scale;       /* DQ_SCALE_* */
     int32_t outer_scale;       /* DQ_SCALE_BF16 or DQ_SCALE_E8M0 */
@@ -98,7 +104,7 @@ typedef struct dq_matrix {
     const void *W;             /* [rows, cols] of the call's dtype */
     int64_t rows, cols;
     const float *a0, *b0;      /* initial a [rows], b [cols]; NULL = all ones */
-    uint8_t *codes;            /* out: [rows, cols/2] packed codes */
+    uint8_t *codes;            /* out: dq_code_bytes(fmt, rows, cols) bytes of codes */
     void *gscales;             /* out: [rows, cols/G] group scales */
     float *a, *b;              /* out: final outer inverse scales */
     float *tensor_scale;       /* out: 1 float, the ts used (1.0 unless auto) */
@@ -115,10 +121,22 @@ DQ_API const char *dq_strerror(dq_status s);
 /* Fill `out` (host) with a named preset: "int4_bf16" (INT4 codes, BF16 group
  * and outer scales, default G 64), "mxint4" (INT4, E8M0, E8M0, G 32),
  * "mxfp4" (E2M1, E8M0, E8M0, G 32), "nvfp4" (E2M1, E4M3 group, BF16 outer,
- * G 16, tensor_scale_auto).  group == 0 keeps the preset's G.  Presets follow
- * the formats of Table 1 of the daiwk note and the news article's MXFP4/NVFP4
- * description.  Errors: DQ_ERR_ARG (null), DQ_ERR_FORMAT (unknown name or G). */
+ * G 16, tensor_scale_auto); the rest of the MX family, all E8M0/E8M0 and
+ * G 32: "mxint8", "mxfp8_e4m3", "mxfp8_e5m2", "mxfp6_e2m3", "mxfp6_e3m2".
+ * group == 0 keeps the preset's G.  Presets follow the formats of Table 1 of
+ * the daiwk note, the news article's MXFP4/NVFP4 description and its claim of
+ * the whole MX family.  Errors: DQ_ERR_ARG (null), DQ_ERR_FORMAT (unknown
+ * name or G). */
 DQ_API dq_status dq_format_preset(const char *name, int32_t group, dq_format *out);
+
+/* Size in bytes of the codes of a rows x cols matrix in format `fmt`: rows
+ * rows of cols * bits / 8 bytes each.  Layout of a row: 4-bit codes two per
+ * byte, the even column in the low nibble (INT4 two's complement, E2M1
+ * s|ee|m); 8-bit codes one per byte (INT8 two's complement, E4M3 s|eeee|mmm,
+ * E5M2 s|eeeee|mm); 6-bit codes (E2M3 s|ee|mmm, E3M2 s|eee|mm) four per 3
+ * bytes as one little-endian 24-bit word, the first column in the low bits.
+ * Returns -1 for an invalid format or shape (cols % G != 0). */
+DQ_API int64_t dq_code_bytes(const dq_format *fmt, int64_t rows, int64_t cols);
 
 /* Bytes of device workspace a solve or a single update of the listed
  * matrices needs (host arrays rows[n], cols[n]; result in *bytes, host).
@@ -130,7 +148,8 @@ DQ_API dq_status dq_workspace_size(int32_t n, const int64_t *rows, const int64_t
 /* Q(X ⊘ (a bᵀ)): the black-box group quantizer (daiwk note, "原始论文总结")
  * applied to X / (a_i b_j) with second-level scale `tensor_scale` (host value,
  * a power of two; it must be 1.0 unless the group scales are E4M3).  a (rows) and b (cols) may be
- * NULL (all ones).  Writes packed codes and group scales.  No workspace. */
+ * NULL (all ones).  Writes the codes (dq_code_bytes layout) and group scales.
+ * No workspace. */
 DQ_API dq_status dq_quantize(const void *X, int32_t dtype, int64_t rows, int64_t cols,
                       const dq_format *fmt, const float *a, const float *b,
                       float tensor_scale, uint8_t *codes, void *gscales,
@@ -187,8 +206,8 @@ DQ_API dq_status dq_col_update(const void *W, int32_t dtype, int64_t rows, int64
 /* Activation side of eq. (1): Q(X D_b) with ts = 1 — each input channel j is
  * multiplied by b_j, then quantized in groups of G along K (the trove summary,
  * "How to use it": beta is applied inside the activation-quantization kernel).
- * X is bf16 [tokens, K]; b float [K].  Writes packed codes [tokens, K/2] and
- * group scales [tokens, K/G].  No workspace. */
+ * X is bf16 [tokens, K]; b float [K].  Writes the codes (dq_code_bytes(fmt,
+ * tokens, K) bytes) and group scales [tokens, K/G].  No workspace. */
 DQ_API dq_status dq_act_rescale_quant(const void *X, int64_t tokens, int64_t K, const float *b,
                                const dq_format *fmt, uint8_t *codes, void *gscales,
                                dq_stream stream);

@@ -13,7 +13,28 @@ PRESET_COMBOS = {
     # BF16 outer scales with E8M0 group scales (descriptor variant)
     "mxint4_bf16outer": lambda G: O.Format("int4", G, "e8m0", "bf16"),
     "mxfp4_bf16outer": lambda G: O.Format("e2m1", G, "e8m0", "bf16"),
+    # the rest of the MX family
+    "mxint8": lambda G: O.preset("mxint8", G),
+    "mxfp8_e4m3": lambda G: O.preset("mxfp8_e4m3", G),
+    "mxfp8_e5m2": lambda G: O.preset("mxfp8_e5m2", G),
+    "mxfp6_e2m3": lambda G: O.preset("mxfp6_e2m3", G),
+    "mxfp6_e3m2": lambda G: O.preset("mxfp6_e3m2", G),
 }
+MX_MORE = ["mxint8", "mxfp8_e4m3", "mxfp8_e5m2", "mxfp6_e2m3", "mxfp6_e3m2"]
+
+
+def code_boundaries(fo):
+    """Decision boundaries of the code grid (code magnitudes' midpoints)."""
+    if fo.codes == "int4":
+        return np.arange(0, 7) + 0.5
+    if fo.codes == "int8":
+        return np.arange(0, 127) + 0.5
+    if fo.codes == "e2m1":
+        grid = O.E2M1_GRID
+    else:
+        v = O.fp_element_values(fo.codes)
+        grid = v[~np.isnan(v)]
+    return (grid[:-1] + grid[1:]) / 2
 
 
 def lib_format(name, G):

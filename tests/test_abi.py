@@ -24,7 +24,7 @@ def built():
 
 def test_exports_match_header():
     names = _declared()
-    assert len(names) == 16
+    assert len(names) == 17
     assert sorted(dq.EXPORTS) == names
     L = dq.lib()
     for n in names:
@@ -38,11 +38,27 @@ def test_version_and_errors():
 
 @pytest.mark.parametrize("name,codes,gs,os_,G,auto", [
     ("int4_bf16", 0, 0, 0, 64, 0), ("mxint4", 0, 1, 1, 32, 0),
-    ("mxfp4", 1, 1, 1, 32, 0), ("nvfp4", 1, 2, 0, 16, 1)])
+    ("mxfp4", 1, 1, 1, 32, 0), ("nvfp4", 1, 2, 0, 16, 1),
+    ("mxint8", 2, 1, 1, 32, 0), ("mxfp8_e4m3", 3, 1, 1, 32, 0), ("mxfp8_e5m2", 4, 1, 1, 32, 0),
+    ("mxfp6_e2m3", 5, 1, 1, 32, 0), ("mxfp6_e3m2", 6, 1, 1, 32, 0)])
 def test_presets(name, codes, gs, os_, G, auto):
     f = dq.format_preset(name)
     assert (f.codes, f.group_scale, f.outer_scale, f.group, f.tensor_scale_auto) == (codes, gs, os_, G, auto)
     assert dq.format_preset(name, 32).group == 32
+
+
+@pytest.mark.parametrize("name,per_row", [
+    ("int4_bf16", 32), ("mxfp4", 32), ("nvfp4", 32), ("mxint8", 64), ("mxfp8_e4m3", 64),
+    ("mxfp8_e5m2", 64), ("mxfp6_e2m3", 48), ("mxfp6_e3m2", 48)])
+def test_code_bytes(name, per_row):
+    # 64 columns: 4-bit codes 32 bytes, 8-bit 64, 6-bit 48 (four codes per 3 bytes)
+    f = dq.format_preset(name)
+    assert dq.code_bytes(f, 3, 64) == 3 * per_row
+    assert dq.lib().dq_code_bytes(ctypes.byref(f), 3, 65) == -1
+    # the float element formats need E8M0 group and outer scales
+    bad = dq.dq_format(f.codes, 32, 0, 0, 0)
+    if f.codes >= 2:
+        assert dq.lib().dq_code_bytes(ctypes.byref(bad), 3, 64) == -1
 
 
 def test_bad_preset_and_group():

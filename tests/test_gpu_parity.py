@@ -15,8 +15,8 @@ import torch
 
 import oracle as O
 import synth
-from _helpers import (PRESET_COMBOS, gpu_scales_np, lib_format, near_outer_boundary, np64,
-                      oracle_encoded, random_outer)
+from _helpers import (MX_MORE, PRESET_COMBOS, code_boundaries, gpu_scales_np, lib_format,
+                      near_outer_boundary, np64, oracle_encoded, random_outer)
 
 pytestmark = pytest.mark.gpu
 
@@ -24,7 +24,7 @@ dq = pytest.importorskip("dual_scale_solver_b200")
 
 ALL = list(PRESET_COMBOS)
 DEFAULT_G = {"int4_bf16": 64, "mxint4": 32, "mxfp4": 32, "nvfp4": 16,
-             "mxint4_bf16outer": 32, "mxfp4_bf16outer": 32}
+             "mxint4_bf16outer": 32, "mxfp4_bf16outer": 32, **{n: 32 for n in MX_MORE}}
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -80,9 +80,8 @@ def _tie_matrix(fo, kind):
     G = fo.group
     rows = []
     rng = np.random.default_rng(3)
-    # decision boundaries of the code grid: half-integers (INT4), E2M1 midpoints
-    grid = np.arange(0, 7) + 0.5 if fo.codes == "int4" else \
-        np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0])
+    # decision boundaries of the code grid (midpoints of code magnitudes)
+    grid = code_boundaries(fo)
     for r in range(24):
         s = 2.0 ** int(rng.integers(-9, -3))
         if fo.gscale == "bf16":
@@ -147,7 +146,7 @@ def test_group_scale_ties_bf16():
 # Activation rescale + quantize
 # --------------------------------------------------------------------------- #
 
-@pytest.mark.parametrize("name", ["int4_bf16", "nvfp4", "mxfp4", "mxint4"])
+@pytest.mark.parametrize("name", ["int4_bf16", "nvfp4", "mxfp4", "mxint4"] + MX_MORE)
 @pytest.mark.parametrize("tokens", [1, 333])
 def test_act_rescale_quant_bit_exact(name, tokens):
     G = DEFAULT_G[name]
@@ -251,7 +250,7 @@ def test_solve_toy_workload():
     _solve_and_compare([W], fo, fl, wl.T)
 
 
-@pytest.mark.parametrize("name", ["int4_bf16", "nvfp4", "mxfp4"])
+@pytest.mark.parametrize("name", ["int4_bf16", "nvfp4", "mxfp4"] + MX_MORE)
 def test_solve_single_matrix_entry_point(name):
     G = DEFAULT_G[name]
     fo, fl = PRESET_COMBOS[name](G), dq.format_preset(name, G)
@@ -261,6 +260,16 @@ def test_solve_single_matrix_entry_point(name):
     r = O.solve(np64(W), fo, 4)
     tr = np64(o["mse_trace"])
     assert np.max(np.abs(tr - r["mse_trace"]) / r["mse_trace"]) < 1e-4
+
+
+@pytest.mark.parametrize("name", MX_MORE)
+def test_solve_mx_family_batched(name):
+    # three matrices of one batch against the oracle's whole trajectory,
+    # codes and scales at the GPU's final state bit for bit
+    fo, fl = PRESET_COMBOS[name](32), dq.format_preset(name)
+    Ws = [_weights(r, c, torch.bfloat16, key=30 + k)
+          for k, (r, c) in enumerate([(300, 2240), (64, 576), (17, 1024)])]
+    _solve_and_compare(Ws, fo, fl, 4)
 
 
 def test_solve_smollm2_decoder0_batched_with_all_30():
@@ -355,7 +364,7 @@ def _literal_sequence(W, fl, T, a0, b0):
     return a, b
 
 
-@pytest.mark.parametrize("name", ["mxfp4", "mxint4"])
+@pytest.mark.parametrize("name", ["mxfp4", "mxint4"] + MX_MORE)
 @pytest.mark.parametrize("extreme", [None, -124, 126])
 def test_mx_solve_equals_the_literal_steps(name, extreme):
     # With power-of-two scales the solve takes both statistics of an
