@@ -21,7 +21,7 @@ stated distributions stand in for them.
 from __future__ import annotations
 
 import math
-from dataclasses import dataclass, field
+from dataclasses import dataclass, field, replace
 
 import torch
 
@@ -178,6 +178,15 @@ WORKLOADS = {
         0.01, 0, 10.0, 0, "mxfp4", 32, 15,
         dict(tokens=8 * 4096, K=8192, frac=0.005, factor=30.0, fmt="mxfp4", group=32)),
 }
+
+
+# The same 70B decoder weights and activations in the other formats of the
+# MX family (the pages claim the whole family; element formats from the OCP
+# Microscaling definition).
+for _f in ("mxint8", "mxfp8_e4m3", "mxfp8_e5m2", "mxfp6_e2m3", "mxfp6_e3m2"):
+    _base = WORKLOADS["llama31_70b_decoder_mxfp4_g32"]
+    WORKLOADS[f"llama31_70b_decoder_{_f}_g32"] = replace(
+        _base, name=f"llama31_70b_decoder_{_f}_g32", fmt=_f, act=dict(_base.act, fmt=_f))
 
 
 def outlier_count(n: int, frac: float) -> int:

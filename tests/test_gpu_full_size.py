@@ -89,12 +89,30 @@ _E2M1 = torch.tensor([0, .5, 1, 1.5, 2, 3, 4, 6, -0., -.5, -1, -1.5, -2, -3, -4,
                      dtype=torch.float64)
 
 
+def _code_values(codes, fo):
+    """Code values [rows, cols] (float64) of stored codes, by table lookup
+    (tables from the oracle's decoders)."""
+    rows = codes.shape[0]
+    if fo.code_bits == 4:
+        tab = (_INT4 if fo.codes == "int4" else _E2M1).to(codes.device)
+        idx = torch.stack([codes & 0xF, codes >> 4], dim=-1).view(rows, -1).long()
+    elif fo.code_bits == 8:
+        tab = torch.tensor(O.decode_codes(np.arange(256, dtype=np.uint8)[None, :], fo)[0],
+                           dtype=torch.float64, device=codes.device)
+        idx = codes.long()
+    else:                                            # four 6-bit codes per 3 bytes
+        tab = torch.tensor(O.decode_fp_element(np.arange(64), fo.codes), dtype=torch.float64,
+                           device=codes.device)
+        b3 = codes.view(rows, -1, 3).long()
+        w = b3[..., 0] | (b3[..., 1] << 8) | (b3[..., 2] << 16)
+        idx = torch.stack([(w >> (6 * k)) & 0x3F for k in range(4)], dim=-1).view(rows, -1)
+    return tab[idx]
+
+
 def _decode_fp64(codes, gscales, fo, ts, a, b):
     """a_i c_ij s_g ts b_j in float64 with torch (table lookups, exact casts)."""
     rows = codes.shape[0]
-    tab = (_INT4 if fo.codes == "int4" else _E2M1).to(codes.device)
-    nib = torch.stack([codes & 0xF, codes >> 4], dim=-1).view(rows, -1).long()
-    c = tab[nib]
+    c = _code_values(codes, fo)
     if fo.gscale == "bf16":
         sc = (gscales.view(torch.int16).to(torch.int32) << 16).view(torch.float32).double()
     elif fo.gscale == "e8m0":
@@ -125,8 +143,10 @@ def _trajectory_against_oracle(W, o, fo, T):
     assert float(o["tensor_scale"].item()) == r["ts"]
 
 
-def test_full_size_70b_decoder_mxfp4():
-    wl = synth.WORKLOADS["llama31_70b_decoder_mxfp4_g32"]
+@pytest.mark.parametrize("fmt", ["mxfp4", "mxint8", "mxfp8_e4m3", "mxfp8_e5m2", "mxfp6_e2m3",
+                                 "mxfp6_e3m2"])
+def test_full_size_70b_decoder_mx(fmt):
+    wl = synth.WORKLOADS[f"llama31_70b_decoder_{fmt}_g32"]
     fl, fo, mats, Ws, outs = _solve_workload(wl)
     assert sum(W.numel() for W in Ws) == 855638016
     for k, (W, o) in enumerate(zip(Ws, outs)):
@@ -137,8 +157,10 @@ def test_full_size_70b_decoder_mxfp4():
     assert dq.last_device_status() == 0
 
 
-def test_full_size_70b_activation_mxfp4():
-    wl = synth.WORKLOADS["llama31_70b_decoder_mxfp4_g32"]
+@pytest.mark.parametrize("fmt", ["mxfp4", "mxint8", "mxfp8_e4m3", "mxfp8_e5m2", "mxfp6_e2m3",
+                                 "mxfp6_e3m2"])
+def test_full_size_70b_activation_mx(fmt):
+    wl = synth.WORKLOADS[f"llama31_70b_decoder_{fmt}_g32"]
     act = wl.act
     fa, foa = dq.format_preset(act["fmt"], act["group"]), O.preset(act["fmt"], act["group"])
     X = synth.activation(wl, device="cuda")
