@@ -14,4 +14,5 @@ from .formats import *          # noqa: F401,F403
 from .solver import (Format, PRESETS, QMAX, CODE_BITS, preset, project_group_scale, project_outer,  # noqa: F401
                      round_codes, tensor_scale, quantize, dequantize, inner, qhat, mse,
                      row_update, col_update, solve, act_rescale_quant, encode_codes,
-                     encode_scales, decode_codes, decode_scales)
+                     encode_scales, decode_codes, decode_scales, two_level_quant,
+                     MXFP4_MAX_NORMAL)

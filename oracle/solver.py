@@ -295,3 +295,47 @@ def decode_scales(u: np.ndarray, fmt: Format) -> np.ndarray:
     if fmt.gscale == "e8m0":
         return F.decode_e8m0(u)
     return F.decode_e4m3(u)
+
+
+# --------------------------------------------------------------------------- #
+# Two-level absmax quantization (msModelSlim "DualScale" page)
+# --------------------------------------------------------------------------- #
+
+MXFP4_MAX_NORMAL = 6.0
+
+
+def two_level_quant(X, dual_block: int, inner: Format):
+    """Two-level absmax quant-dequant (msmodelslim.readthedocs.io, DualScale,
+    "算法原理" 1(a)-(c) and 2(a)-(b)).
+
+    Per row and block of ``dual_block`` consecutive columns (the last block
+    may be shorter): outer scale S = max|X_block| / MXFP4_MAX_NORMAL, the
+    block divided by S, quantized with the inner format (our Q: E8M0 group
+    scale rounded up, codes nearest-even) and multiplied back by S.
+
+    Readings (the page fixes no precision): S and X/S are float32 values
+    (IEEE float32 division, i.e. the correctly rounded quotient: float64
+    division followed by rounding to float32 gives the same value, since
+    53 >= 2*24 + 2); an all-zero block takes S = 1; the reconstruction is the
+    float32 product (c * s) * S.
+
+    Returns (codes, inner_scales, outer_scales [rows, ceil(cols/dual_block)],
+    qdq) with codes/scales as values and qdq as float64 holding float32
+    values.
+    """
+    X = np.asarray(X, dtype=np.float64)
+    rows, cols = X.shape
+    nb = -(-cols // dual_block)
+    S = np.ones((rows, nb))
+    Y = np.empty_like(X)
+    for k in range(nb):
+        blk = X[:, k * dual_block:(k + 1) * dual_block]
+        m = np.abs(blk).max(axis=1)
+        s = np.where(m > 0, (m / MXFP4_MAX_NORMAL).astype(np.float32).astype(np.float64), 1.0)
+        S[:, k] = s
+        Y[:, k * dual_block:(k + 1) * dual_block] = (blk / s[:, None]).astype(np.float32)
+    c, s_in = quantize(Y, inner, 1.0)
+    inner_vals = dequantize(c, s_in, inner, 1.0)             # c * s: exact
+    Sfull = np.repeat(S, dual_block, axis=1)[:, :cols]
+    qdq = (inner_vals * Sfull).astype(np.float32).astype(np.float64)
+    return c, s_in, S, qdq

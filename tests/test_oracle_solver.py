@@ -386,3 +386,65 @@ def test_quantize_hand_cases_mx_family(name, s, c_max, c_03):
     c, sc = O.quantize(y, fmt)
     assert sc[0, 0] == s
     assert c[0, 0] == c_max and c[0, 1] == c_03 and c[0, 2] == -c_03
+
+
+# --------------------------------------------------------------------------- #
+# Two-level absmax quantization (msModelSlim DualScale page)
+# --------------------------------------------------------------------------- #
+
+def _rn32(x: Fr) -> Fr:
+    """Exact rational rounding to the nearest float32, ties to even."""
+    if x == 0:
+        return Fr(0)
+    v = _rne(abs(x), 24, -126, Fr(2) ** 127 * (2 - Fr(2) ** -23))
+    return v if x > 0 else -v
+
+
+def test_two_level_quant_matches_rational_restatement():
+    fmt = O.preset("mxfp4")
+    rng = np.random.default_rng(21)
+    X = (rng.standard_normal((3, 1056)) * np.exp(rng.uniform(-3, 3, (3, 1)))).astype(np.float32)
+    X[1, 512:1024] = 0.0                                   # an all-zero block
+    X = X.astype(np.float64)
+    c, s_in, S, qdq = O.two_level_quant(X, 512, fmt)
+    assert S.shape == (3, 3)                               # ragged last block of 32 columns
+    for i in range(3):
+        Y = []
+        Sr = []
+        for k in range(3):
+            blk = [Fr(float(v)) for v in X[i, k * 512:(k + 1) * 512]]
+            m = max(abs(v) for v in blk)
+            s = Fr(1) if m == 0 else _rn32(m / 6)
+            Sr.append(s)
+            Y += [_rn32(v / s) for v in blk]
+        C, Sg = py_quantize([Y], fmt)
+        assert [float(v) for v in Sr] == list(S[i])
+        assert [float(v) for v in C[0]] == list(c[i])
+        assert [float(v) for v in Sg[0]] == list(s_in[i])
+        want = [float(_rn32(C[0][j] * Sg[0][j // 32] * Sr[j // 512])) for j in range(1056)]
+        assert want == list(qdq[i])
+
+
+def test_two_level_quant_special_cases():
+    fmt = O.preset("mxfp4")
+    rng = np.random.default_rng(22)
+    X = rng.standard_normal((4, 1024)).astype(np.float32).astype(np.float64)
+    # block maxima 6 * 2^k: the outer scales are powers of two, so the result
+    # is plain MXFP4 of X
+    for i in range(4):
+        for k in range(2):
+            blk = X[i, k * 512:(k + 1) * 512]
+            blk *= 1.0 / np.abs(blk).max()
+            blk[np.argmax(np.abs(blk))] = np.sign(blk[np.argmax(np.abs(blk))])
+            blk *= 6.0 * 2.0 ** (i - k)
+    c, s_in, S, qdq = O.two_level_quant(X, 512, fmt)
+    assert np.array_equal(S, np.ldexp(1.0, np.array([[i - k for k in range(2)] for i in range(4)])))
+    c0, s0 = O.quantize(X, fmt)
+    assert np.array_equal(qdq, O.dequantize(c0, s0, fmt))
+    # scaling X by a power of two scales S and keeps codes and inner scales
+    c2, s2, S2, q2 = O.two_level_quant(X * 8.0, 512, fmt)
+    assert np.array_equal(c2, c) and np.array_equal(s2, s_in) and np.array_equal(S2, 8 * S)
+    assert np.array_equal(q2, 8 * qdq)
+    # zero input: S = 1, codes 0, scales 1, reconstruction 0
+    c3, s3, S3, q3 = O.two_level_quant(np.zeros((2, 512)), 512, fmt)
+    assert np.all(S3 == 1) and np.all(c3 == 0) and np.all(s3 == 1) and np.all(q3 == 0)
