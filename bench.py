@@ -53,6 +53,9 @@ def _args():
                    help="profiling case: keep only this linear of the decoder")
     p.add_argument("--T", type=int, default=-1, help="profiling case: iterations override")
     p.add_argument("--no-act", action="store_true", help="profiling case: skip activations")
+    p.add_argument("--method", default="dualquant", choices=["dualquant", "two_level"],
+                   help="two_level: the two-level absmax quantization of the same weights "
+                        "and activations instead of the solve")
     return p.parse_args()
 
 
@@ -416,6 +419,106 @@ def run_ours(args, wl, rank, world, local_rank):
     return 0
 
 
+def run_two_level(args, wl, rank, world, local_rank):
+    """Two-level absmax quantization of the workload's weights (codes and
+    scales) and of its activation batch (codes, scales and the float32
+    reconstruction), one step = all of it, 1 GPU per rank (weak scaling)."""
+    import torch
+    import synth
+    import dual_scale_solver_b200 as dq
+    from dual_scale_solver_b200 import build
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    build.build()
+    D = 512
+    Ws = [synth.weight(wl, d, i, device=dev) for d in decoders_of(rank, wl.decoders)
+          for i in range(len(wl.linears))]
+    X = synth.activation(wl, device=dev) if wl.act and not args.no_act else None
+    stream = torch.cuda.current_stream(dev)
+    E = sum(W.numel() for W in Ws) + (X.numel() if X is not None else 0)
+
+    def step(time_w=None):
+        if time_w:
+            time_w[0].record(stream)
+        for W in Ws:
+            dq.two_level_quant(W, D, qdq=False)
+        if time_w:
+            time_w[1].record(stream)
+        if X is not None:
+            dq.two_level_quant(X, D, qdq=True)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    clocks = Clocks(local_rank)
+    clocks.start()
+    time.sleep(0.3)
+    n0 = dq.launch_count()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for k in range(args.steps):
+        step(ev[k])
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = max_over_ranks(e0.elapsed_time(e1), dev) / args.steps
+    launches = dq.launch_count() - n0
+    clk = clocks.stop()
+    w_ms = sum(a.elapsed_time(b) for a, b in ev) / args.steps
+    Ew = sum(W.numel() for W in Ws)
+    rows_nb = sum(W.shape[0] * -(-W.shape[1] // D) for W in Ws)
+    alg = Ew * 2 + Ew // 2 + Ew // 32 + 4 * rows_nb        # read W, write codes + scales
+    peaks, which = _peaks()
+    peak = float(peaks["hbm_gbs"])
+    achieved = alg / (w_ms / 1e3) / 1e9
+    unit = "quantized elements/s"
+    e2e = None
+    if not args.no_e2e:
+        hW = [W.to("cpu").pin_memory() for W in Ws]
+        dW = [torch.empty_like(W) for W in Ws]
+        outs = [(torch.empty(W.shape[0], W.shape[1] // 2, dtype=torch.uint8, pin_memory=True),
+                 torch.empty(W.shape[0], W.shape[1] // 32, dtype=torch.uint8, pin_memory=True))
+                for W in Ws]
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for _ in range(args.steps):
+            for h, d, (hc, hs) in zip(hW, dW, outs):
+                d.copy_(h, non_blocking=True)
+                c, si, so, _ = dq.two_level_quant(d, D, qdq=False)
+                hc.copy_(c, non_blocking=True)
+                hs.copy_(si, non_blocking=True)
+        f1.record(stream)
+        torch.cuda.synchronize(dev)
+        ems = max_over_ranks(f0.elapsed_time(f1), dev) / args.steps
+        e2e = {"value": world * Ew / (ems / 1e3), "unit": unit,
+               "h2d_bytes_per_step": sum(h.numel() * h.element_size() for h in hW),
+               "d2h_bytes_per_step": sum(c.numel() + s.numel() for c, s in outs),
+               "ms_per_step": ems, "scope": "weights only"}
+    if dq.last_device_status() != 0:
+        raise RuntimeError("device status flags raised during timing")
+    line = {
+        "metric": "two-level absmax quantized elements/s", "value": world * E / (ms / 1e3),
+        "unit": unit, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32", "data": "synthetic",
+        "config": {"workload": f"{wl.name} weights + activations, two-level absmax (outer "
+                               f"{D}-column blocks, inner MXFP4 G32)",
+                   "elements_per_gpu": E, "l2": "inputs larger than L2 (no flush needed)",
+                   "parallelism": f"{world} independent decoders" if world > 1 else "1 GPU"},
+        "roofline": {"bound": "hbm", "kernel": "two_level (weights: codes + scales)",
+                     "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "peak_source": which, "traffic": None, "algorithmic_bytes_per_step": alg,
+                     "weights_ms_per_step": w_ms},
+        "gpu_launches": launches, "clocks": clk, "e2e": e2e,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = _args()
     import synth
@@ -433,6 +536,8 @@ def main():
         tdist.init_process_group("nccl", timeout=timedelta(seconds=120),
                                  device_id=torch.device("cuda", local_rank))
     try:
+        if args.method == "two_level":
+            return run_two_level(args, wl, rank, world, local_rank)
         return run_ours(args, wl, rank, world, local_rank)
     finally:
         if world > 1:

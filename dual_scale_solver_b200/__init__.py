@@ -18,6 +18,7 @@ __all__ = [
     "workspace_size", "quantize", "dequantize", "solve_dual_scale", "solve_dual_scale_batched",
     "row_update", "col_update", "act_rescale_quant", "last_device_status", "EXPORTS",
     "kernel_timing", "kernel_time", "launch_count", "solve_dual_scale_noalloc", "code_bytes",
+    "two_level_quant",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -33,7 +34,7 @@ EXPORTS = ("dq_version", "dq_strerror", "dq_format_preset", "dq_workspace_size",
            "dq_dequantize", "dq_solve_dual_scale", "dq_solve_dual_scale_batched",
            "dq_row_update", "dq_col_update", "dq_act_rescale_quant", "dq_last_device_status",
            "dq_kernel_timing", "dq_kernel_time", "dq_launch_count",
-           "dq_solve_dual_scale_noalloc", "dq_code_bytes")
+           "dq_solve_dual_scale_noalloc", "dq_code_bytes", "dq_two_level_quant")
 
 
 class DqError(RuntimeError):
@@ -103,6 +104,9 @@ def lib() -> ctypes.CDLL:
         "dq_kernel_time": (c_int32, [c_int32, P(c_double), P(c_int64)]),
         "dq_launch_count": (c_int64, []),
         "dq_code_bytes": (c_int64, [P(dq_format), c_int64, c_int64]),
+        "dq_two_level_quant": (c_int32, [c_void_p, c_int32, c_int64, c_int64, c_int32,
+                                         P(dq_format), c_void_p, c_void_p, c_void_p, c_void_p,
+                                         c_void_p]),
         "dq_solve_dual_scale_noalloc": (c_int32, [c_void_p, c_int32, c_int64, c_int64,
                                                   P(dq_format), c_int32, c_void_p, c_void_p,
                                                   c_void_p, c_void_p, c_void_p, c_void_p,
@@ -341,6 +345,25 @@ def act_rescale_quant(X, b, fmt, codes=None, gscales=None, stream=None):
     _check(lib().dq_act_rescale_quant(_ptr(X), tokens, K, _ptr(b), ctypes.byref(fmt), _ptr(codes),
                                       _ptr(gscales), _stream(stream)), "dq_act_rescale_quant")
     return codes, gscales
+
+
+def two_level_quant(X, dual_block=512, inner=None, qdq=True, stream=None):
+    """Two-level absmax quantization: returns (codes [rows, cols/2], inner
+    E8M0 scales [rows, cols/32], outer float32 scales [rows, ceil(cols/D)],
+    reconstruction float32 [rows, cols] or None)."""
+    _need_cuda(X)
+    inner = format_preset("mxfp4") if inner is None else inner
+    rows, cols = X.shape
+    dev = X.device
+    nb = -(-cols // dual_block) if cols else 0
+    codes = torch.empty(rows, cols // 2, dtype=torch.uint8, device=dev)
+    isc = torch.empty(rows, cols // 32, dtype=torch.uint8, device=dev)
+    osc = torch.empty(rows, nb, dtype=torch.float32, device=dev)
+    out = torch.empty(rows, cols, dtype=torch.float32, device=dev) if qdq else None
+    _check(lib().dq_two_level_quant(_ptr(X), _dtype_code(X), rows, cols, int(dual_block),
+                                    ctypes.byref(inner), _ptr(codes), _ptr(isc), _ptr(osc),
+                                    _ptr(out), _stream(stream)), "dq_two_level_quant")
+    return codes, isc, osc, out
 
 
 KIND_ROW, KIND_COL, KIND_PACK, KIND_ACT, KIND_FUSED = 0, 1, 2, 3, 4

@@ -721,6 +721,42 @@ dq_status dq_act_rescale_quant(const void *X, int64_t tokens, int64_t K, const f
     return L.tiles_pass(MODE_ACT, false);
 }
 
+dq_status dq_two_level_quant(const void *X, int32_t dtype, int64_t rows, int64_t cols,
+                             int32_t dual_block, const dq_format *inner, uint8_t *codes,
+                             void *inner_scales, float *outer_scales, float *qdq,
+                             dq_stream stream) {
+    if (!inner) return DQ_ERR_ARG;
+    if (inner->codes != DQ_CODES_E2M1 || inner->group != 32 || inner->group_scale != DQ_SCALE_E8M0 ||
+        inner->tensor_scale_auto != 0)
+        return DQ_ERR_FORMAT;
+    if (dual_block != 256 && dual_block != 512 && dual_block != 1024) return DQ_ERR_ARG;
+    if (dtype != DQ_DT_F32 && dtype != DQ_DT_BF16) return DQ_ERR_ARG;
+    if (rows < 0 || cols < 0 || cols % 32) return DQ_ERR_SHAPE;
+    if (rows == 0 || cols == 0) return DQ_OK;
+    if (!X || !codes || !inner_scales || !outer_scales) return DQ_ERR_ARG;
+    if (!aligned(X, 16) || !aligned(codes, 16) || !aligned(inner_scales, 16) ||
+        !aligned(outer_scales, 4) || !aligned(qdq, 16))
+        return DQ_ERR_ALIGN;
+    unsigned int *status = status_ptr();
+    if (!status) return DQ_ERR_CUDA;
+    TwoLevelLaunch L;
+    L.X = X;
+    L.rows = rows;
+    L.cols = cols;
+    L.nblk = (cols + dual_block - 1) / dual_block;
+    L.dual_block = dual_block;
+    L.f32 = dtype == DQ_DT_F32;
+    L.codes = codes;
+    L.iscales = static_cast<uint8_t *>(inner_scales);
+    L.oscales = outer_scales;
+    L.qdq = qdq;
+    L.status = status;
+    L.stream = reinterpret_cast<cudaStream_t>(stream);
+    DQ_CUDA(launch_two_level(L));
+    count_launches(1);
+    return DQ_OK;
+}
+
 dq_status dq_dequantize(const uint8_t *codes, const void *gscales, int64_t rows, int64_t cols,
                         const dq_format *fmt, float tensor_scale, const float *a, const float *b,
                         float *out, dq_stream stream) {

@@ -5,6 +5,7 @@
 
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <utility>
 
 #include "dq_device.cuh"
@@ -60,6 +61,21 @@ cudaError_t launch_k(void (*kern)(P...), dim3 grid, dim3 block, size_t smem, cud
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, kern, std::forward<A>(args)...);
 }
+
+// Two-level absmax quantization (dq_twolevel.cu).
+struct TwoLevelLaunch {
+    const void *X;
+    int64_t rows, cols, nblk;
+    int dual_block;         // 256, 512 or 1024
+    int f32;                // 1: float32 input, 0: bfloat16
+    uint8_t *codes;         // [rows, cols/2] E2M1
+    uint8_t *iscales;       // [rows, cols/32] E8M0
+    float *oscales;         // [rows, nblk]
+    float *qdq;             // [rows, cols] or NULL
+    unsigned int *status;
+    cudaStream_t stream;
+};
+cudaError_t launch_two_level(const TwoLevelLaunch &L);
 
 cudaError_t launch_tile_c0(const TileLaunch &L);
 cudaError_t launch_tile_c1(const TileLaunch &L);

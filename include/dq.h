@@ -212,6 +212,26 @@ DQ_API dq_status dq_act_rescale_quant(const void *X, int64_t tokens, int64_t K, 
                                const dq_format *fmt, uint8_t *codes, void *gscales,
                                dq_stream stream);
 
+/* Two-level absmax quantization (msmodelslim.readthedocs.io, DualScale page,
+ * "算法原理" 1(a)-(c) and 2(a)-(b)) — a second, non-iterative method.  Per
+ * row and block of `dual_block` consecutive columns (256, 512 or 1024; the
+ * last block may be shorter): outer scale S = max|X_block| / 6 (6 = the
+ * largest normal E2M1 value; float32 division; S = 1 for an all-zero
+ * block), then the inner format (`inner` must be MXFP4: E2M1 codes, E8M0
+ * group scales, G = 32) quantizes X / S (float32 division) exactly as
+ * dq_quantize does, and the reconstruction is qdq = (c * s) * S (float32).
+ * X: [rows, cols] of `dtype`, cols a multiple of 32.  Outputs (device,
+ * caller-owned): codes [rows, cols/2] (dq_code_bytes layout), inner_scales
+ * [rows, cols/32] E8M0 bytes, outer_scales [rows, ceil(cols/dual_block)]
+ * float32, qdq [rows, cols] float32 or NULL (not written).  16-byte aligned
+ * X, codes, inner_scales and qdq.  Errors: DQ_ERR_FORMAT (inner not MXFP4),
+ * DQ_ERR_ARG (block size, dtype, null pointer), DQ_ERR_SHAPE, DQ_ERR_ALIGN;
+ * a non-finite input raises the device flag. */
+DQ_API dq_status dq_two_level_quant(const void *X, int32_t dtype, int64_t rows, int64_t cols,
+                                    int32_t dual_block, const dq_format *inner, uint8_t *codes,
+                                    void *inner_scales, float *outer_scales, float *qdq,
+                                    dq_stream stream);
+
 /* Synchronise `stream`, read and clear the device flags raised by earlier
  * calls on this device: DQ_ERR_NONFINITE if an input held NaN/Inf (or
  * scaling it by the outer scales left the float32 range),

@@ -24,7 +24,7 @@ def built():
 
 def test_exports_match_header():
     names = _declared()
-    assert len(names) == 17
+    assert len(names) == 18
     assert sorted(dq.EXPORTS) == names
     L = dq.lib()
     for n in names:
@@ -106,3 +106,16 @@ def test_host_side_argument_errors():
     assert L.dq_workspace_size(0, None, None, ctypes.byref(dq.dq_format(1, 32, 1, 1, 1)),
                                ctypes.byref(ctypes.c_size_t())) == -3
     assert L.dq_solve_dual_scale_batched(-1, None, 1, ctypes.byref(f), 1, None, 0, None) == -1
+
+
+def test_two_level_argument_errors():
+    L = dq.lib()
+    f = dq.format_preset("mxfp4")
+    nv = dq.format_preset("nvfp4")
+    args = lambda fmt, D, cols: (None, 1, 4, cols, D, ctypes.byref(fmt), None, None, None, None, None)
+    assert L.dq_two_level_quant(*args(nv, 512, 64)) == -3          # inner must be MXFP4
+    assert L.dq_two_level_quant(*args(f, 384, 64)) == -1           # block size
+    assert L.dq_two_level_quant(*args(f, 512, 48)) == -2           # cols % 32
+    assert L.dq_two_level_quant(*args(f, 512, 64)) == -1           # null pointers
+    assert L.dq_two_level_quant(None, 1, 0, 64, 512, ctypes.byref(f), None, None, None, None,
+                                None) == 0                         # empty: nothing to do
