@@ -18,7 +18,7 @@ __all__ = [
     "workspace_size", "quantize", "dequantize", "solve_dual_scale", "solve_dual_scale_batched",
     "row_update", "col_update", "act_rescale_quant", "last_device_status", "EXPORTS",
     "kernel_timing", "kernel_time", "launch_count", "solve_dual_scale_noalloc", "code_bytes",
-    "two_level_quant",
+    "two_level_quant", "w4a4_gemm",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -34,7 +34,7 @@ EXPORTS = ("dq_version", "dq_strerror", "dq_format_preset", "dq_workspace_size",
            "dq_dequantize", "dq_solve_dual_scale", "dq_solve_dual_scale_batched",
            "dq_row_update", "dq_col_update", "dq_act_rescale_quant", "dq_last_device_status",
            "dq_kernel_timing", "dq_kernel_time", "dq_launch_count",
-           "dq_solve_dual_scale_noalloc", "dq_code_bytes", "dq_two_level_quant")
+           "dq_solve_dual_scale_noalloc", "dq_code_bytes", "dq_two_level_quant", "dq_w4a4_gemm")
 
 
 class DqError(RuntimeError):
@@ -104,6 +104,8 @@ def lib() -> ctypes.CDLL:
         "dq_kernel_time": (c_int32, [c_int32, P(c_double), P(c_int64)]),
         "dq_launch_count": (c_int64, []),
         "dq_code_bytes": (c_int64, [P(dq_format), c_int64, c_int64]),
+        "dq_w4a4_gemm": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int64,
+                                   c_int64, c_int64, P(dq_format), c_void_p, c_void_p]),
         "dq_two_level_quant": (c_int32, [c_void_p, c_int32, c_int64, c_int64, c_int32,
                                          P(dq_format), c_void_p, c_void_p, c_void_p, c_void_p,
                                          c_void_p]),
@@ -364,6 +366,20 @@ def two_level_quant(X, dual_block=512, inner=None, qdq=True, stream=None):
                                     ctypes.byref(inner), _ptr(codes), _ptr(isc), _ptr(osc),
                                     _ptr(out), _stream(stream)), "dq_two_level_quant")
     return codes, isc, osc, out
+
+
+def w4a4_gemm(codes_x, scales_x, codes_w, scales_w, a, fmt=None, out=None, stream=None):
+    """out[M, N] = a_n * sum_k Qx[m, k] Qw[n, k] (float32) from MXFP4 codes and
+    E8M0 scales of the activations (M rows) and the weights (N rows)."""
+    _need_cuda(codes_x, scales_x, codes_w, scales_w, a)
+    fmt = format_preset("mxfp4") if fmt is None else fmt
+    M, N, K = codes_x.shape[0], codes_w.shape[0], 2 * codes_x.shape[1]
+    if out is None:
+        out = torch.empty(M, N, dtype=torch.float32, device=codes_x.device)
+    _check(lib().dq_w4a4_gemm(_ptr(codes_x), _ptr(scales_x), _ptr(codes_w), _ptr(scales_w),
+                              _ptr(a), M, N, K, ctypes.byref(fmt), _ptr(out), _stream(stream)),
+           "dq_w4a4_gemm")
+    return out
 
 
 KIND_ROW, KIND_COL, KIND_PACK, KIND_ACT, KIND_FUSED = 0, 1, 2, 3, 4

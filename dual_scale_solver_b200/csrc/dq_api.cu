@@ -604,6 +604,7 @@ const char *dq_strerror(dq_status s) {
         case DQ_ERR_SCRATCH:
             return "matrix needs more scratch than the built-in 32 MiB buffer of "
                    "dq_solve_dual_scale_noalloc holds";
+        case DQ_ERR_TIMEOUT: return "a kernel's bounded wait ran out (stalled pipeline)";
     }
     return "unknown status";
 }
@@ -757,6 +758,39 @@ dq_status dq_two_level_quant(const void *X, int32_t dtype, int64_t rows, int64_t
     return DQ_OK;
 }
 
+dq_status dq_w4a4_gemm(const uint8_t *codes_x, const void *scales_x, const uint8_t *codes_w,
+                       const void *scales_w, const float *a, int64_t M, int64_t N, int64_t K,
+                       const dq_format *fmt, float *out, dq_stream stream) {
+    if (!fmt) return DQ_ERR_ARG;
+    if (fmt->codes != DQ_CODES_E2M1 || fmt->group != 32 || fmt->group_scale != DQ_SCALE_E8M0 ||
+        fmt->tensor_scale_auto != 0)
+        return DQ_ERR_FORMAT;
+    if (M < 0 || N < 0 || K < 0 || M % 128 || N % 128 || K % 256) return DQ_ERR_SHAPE;
+    if (M == 0 || N == 0) return DQ_OK;
+    if (K == 0) return DQ_ERR_SHAPE;
+    if (!codes_x || !scales_x || !codes_w || !scales_w || !a || !out) return DQ_ERR_ARG;
+    if (!aligned(codes_x, 16) || !aligned(scales_x, 16) || !aligned(codes_w, 16) ||
+        !aligned(scales_w, 16) || !aligned(a, 16) || !aligned(out, 16))
+        return DQ_ERR_ALIGN;
+    unsigned int *status = status_ptr();
+    if (!status) return DQ_ERR_CUDA;
+    GemmLaunch L;
+    L.codes_x = codes_x;
+    L.scales_x = static_cast<const uint8_t *>(scales_x);
+    L.codes_w = codes_w;
+    L.scales_w = static_cast<const uint8_t *>(scales_w);
+    L.a = a;
+    L.out = out;
+    L.M = M;
+    L.N = N;
+    L.K = K;
+    L.status = status;
+    L.stream = reinterpret_cast<cudaStream_t>(stream);
+    DQ_CUDA(launch_w4a4_gemm(L));
+    count_launches(1);
+    return DQ_OK;
+}
+
 dq_status dq_dequantize(const uint8_t *codes, const void *gscales, int64_t rows, int64_t cols,
                         const dq_format *fmt, float tensor_scale, const float *a, const float *b,
                         float *out, dq_stream stream) {
@@ -828,6 +862,7 @@ dq_status dq_last_device_status(dq_stream stream) {
     DQ_CUDA(cudaMemcpy(&v, p, sizeof(v), cudaMemcpyDeviceToHost));
     const unsigned int zero = 0;
     DQ_CUDA(cudaMemcpy(p, &zero, sizeof(zero), cudaMemcpyHostToDevice));
+    if (v & STATUS_TIMEOUT) return DQ_ERR_TIMEOUT;  // a kernel's bounded wait ran out
     if (v & STATUS_NONFINITE) return DQ_ERR_NONFINITE;
     if (v & STATUS_RANGE) return DQ_ERR_RANGE;
     return DQ_OK;

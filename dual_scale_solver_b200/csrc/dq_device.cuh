@@ -28,7 +28,7 @@ enum { CODES_INT4 = 0, CODES_E2M1 = 1, CODES_INT8 = 2, CODES_E4M3 = 3, CODES_E5M
        CODES_E2M3 = 5, CODES_E3M2 = 6 };
 enum { SC_BF16 = 0, SC_E8M0 = 1, SC_E4M3 = 2 };
 enum { MODE_ROW = 0, MODE_COL = 1, MODE_PACK = 2, MODE_ACT = 3, MODE_FUSED = 4 };
-enum { STATUS_NONFINITE = 1u, STATUS_RANGE = 2u };
+enum { STATUS_NONFINITE = 1u, STATUS_RANGE = 2u, STATUS_TIMEOUT = 4u };
 
 constexpr int kWarps = 8;            // warps per CTA of the tile kernel
 constexpr int kThreads = 32 * kWarps;

@@ -1,0 +1,367 @@
+// dq_gemm.cu — block-scaled W4A4 GEMM on the 5th-generation tensor cores:
+// the inference step that consumes the solver's output (eq. (1) of the daiwk
+// note: X W^T ~= (X D_b) Qhat^T D_a; trove summary, "How to use it": beta is
+// applied in the activation-quantization kernel, the weights are stored with
+// their codes and scales).
+//
+//   out[m, n] = a_n * sum_k  Qx[m, k] * Qw[n, k]
+//
+// Qx = the MXFP4 codes and E8M0 group scales of Q(X D_b) (dq_act_rescale_quant),
+// Qw = the MXFP4 codes and E8M0 group scales of Q(W / (a b^T)) (the solve), a =
+// the outer row scales of W.  Both operands are K-major E2M1, two codes per
+// byte, with one E8M0 scale per 32 elements of K.
+//
+// One CTA computes a 128 x 128 tile of `out` with tcgen05.mma kind::mxf4
+// (M = 128, N = 128, K = 64 per instruction, block scales of 32 from TMEM),
+// accumulating in float32 in TMEM.  K advances in tiles of 256 elements (128
+// bytes per row) through a 4-stage shared-memory ring:
+//   warp 0     producer: TMA loads of the A and B tiles (128-byte swizzle,
+//              no multicast) and the two operands' scale factors, gathered
+//              from their row-major arrays into the 128-row x 4-scale chunk
+//              layout the tensor core reads;
+//   warp 1     TMEM allocation; lane 0 issues tcgen05.cp (scales to TMEM),
+//              the MMAs and the tcgen05.commit arrivals;
+//   warps 2-5  epilogue: TMEM -> registers (tcgen05.ld), times a_n, stores.
+// Every wait on an mbarrier is bounded: a wait that runs out raises a device
+// status bit, the CTA stops issuing work, waits (bounded) for its copies in
+// flight, frees its TMEM and returns.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include "dq_launch.h"
+
+namespace dq {
+
+namespace {
+
+constexpr int kBM = 128, kBN = 128;
+constexpr int kBK = 256;                       // K elements per stage (128 bytes per row)
+constexpr int kStages = 4;
+constexpr int kTileBytes = kBM * kBK / 2;      // 16 KB per operand tile
+constexpr int kSfBytes = kBM * kBK / 32;       // 1 KB: two 512-byte chunks of 4 scales per row
+constexpr uint32_t kStageTx = 2u * kTileBytes; // TMA bytes per stage (the scales are stored by threads)
+constexpr int kThreadsGemm = 192;
+constexpr uint32_t kTmemCols = 256;            // accumulator 128 + scales 16, rounded up
+constexpr uint64_t kWaitLimitNs = 1000000000ull;   // a wait gives up after 1 s
+
+struct __align__(1024) GemmSmem {
+    uint8_t a[kStages][kTileBytes];
+    uint8_t b[kStages][kTileBytes];
+    uint8_t sfa[kStages][kSfBytes];
+    uint8_t sfb[kStages][kSfBytes];
+    uint64_t full[kStages];
+    uint64_t empty[kStages];
+    uint64_t acc_full;
+    uint32_t tmem_base;
+    int abort;
+};
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t *b, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" :: "r"(smem_u32(b)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *b, uint32_t tx) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;"
+                 :: "r"(smem_u32(b)), "r"(tx) : "memory");
+}
+
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ bool mbar_test(uint32_t addr, uint32_t parity) {
+    uint32_t done;
+    asm volatile("{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; "
+                 "selp.u32 %0, 1, 0, p; }"
+                 : "=r"(done) : "r"(addr), "r"(parity) : "memory");
+    return done != 0;
+}
+
+// Bounded wait for the phase with the given parity to complete.  Returns
+// false if another thread of the CTA gave up, or (raising the status bit and
+// the CTA's abort flag) if this wait ran past its time limit.
+__device__ __forceinline__ bool mbar_wait(uint64_t *b, uint32_t parity, volatile int *abort,
+                                          unsigned int *status) {
+    const uint32_t addr = smem_u32(b);
+    if (mbar_test(addr, parity)) return true;
+    const uint64_t t0 = global_ns();
+    while (true) {
+        if (mbar_test(addr, parity)) return true;
+        if (*abort) return false;
+        if (global_ns() - t0 > kWaitLimitNs) break;
+    }
+    *abort = 1;
+    atomicOr(status, STATUS_TIMEOUT);
+    return false;
+}
+
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y,
+                                            uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];"
+        :: "r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y),
+           "r"(smem_u32(bar))
+        : "memory");
+}
+
+// UMMA shared-memory descriptor, K-major, 128-byte swizzle: rows of 128
+// bytes, 8-row atoms 1024 bytes apart (stride byte offset), version 1.
+__device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr) {
+    return (uint64_t)((saddr & 0x3FFFFu) >> 4) | (1ull << 16) | (64ull << 32) | (1ull << 46) |
+           (2ull << 61);
+}
+
+// Descriptor of one 512-byte scale chunk for tcgen05.cp 32x128b: 32 rows of
+// 16 bytes, 8-row groups 128 bytes apart, no swizzle.
+__device__ __forceinline__ uint64_t desc_sf(uint32_t saddr) {
+    return (uint64_t)((saddr & 0x3FFFFu) >> 4) | (1ull << 16) | (8ull << 32) | (1ull << 46);
+}
+
+// Instruction descriptor, kind::mxf4 with E8M0 block scales: A and B E2M1
+// (K-major), M = 128, N = 128, scale-factor byte ids of A and B.
+__device__ __forceinline__ uint32_t idesc_mxf4(uint32_t sfa_id, uint32_t sfb_id) {
+    return (sfb_id << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kBN >> 3) << 17) | (1u << 23) |
+           ((uint32_t)(kBM >> 4) << 24) | (sfa_id << 29);
+}
+
+__device__ __forceinline__ void mma_mxf4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                         uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
+                                         uint32_t accumulate) {
+    asm volatile(
+        "{ .reg .pred p; setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p; }"
+        :: "r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem),
+           "r"(sfb_tmem)
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_cp_sf(uint32_t taddr, uint64_t sdesc) {
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" :: "r"(taddr), "l"(sdesc)
+                 : "memory");
+}
+
+__device__ __forceinline__ void umma_commit(uint64_t *bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                 :: "r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// 32 consecutive float32 columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+          "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+}
+
+// Bounded wait used while draining at exit (no abort check).
+__device__ __forceinline__ void mbar_drain(uint64_t *b, uint32_t parity) {
+    const uint32_t addr = smem_u32(b);
+    const uint64_t t0 = global_ns();
+    while (!mbar_test(addr, parity) && global_ns() - t0 <= kWaitLimitNs) {
+    }
+}
+
+__global__ void __launch_bounds__(kThreadsGemm, 1)
+w4a4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
+                 const uint8_t *sf_a, const uint8_t *sf_b, const float *a_row, float *out, int M,
+                 int N, int K, unsigned int *status) {
+    grid_dependency_begin();
+    extern __shared__ uint8_t gemm_smem_raw[];
+    GemmSmem &sm = *reinterpret_cast<GemmSmem *>(
+        (reinterpret_cast<uintptr_t>(gemm_smem_raw) + 1023) & ~uintptr_t(1023));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n0 = blockIdx.x * kBN, m0 = blockIdx.y * kBM;
+    const int KT = K / kBK;
+    const int64_t sf_row = K / 32;                  // scale bytes per row
+    volatile int *abort = &sm.abort;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&sm.full[s], 1);
+            mbar_init(&sm.empty[s], 1);
+        }
+        mbar_init(&sm.acc_full, 1);
+        sm.abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                     :: "r"(smem_u32(&sm.tmem_base)), "r"(kTmemCols) : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;             // accumulator: columns [0, 128)
+    const uint32_t sfa_t = tmem + 128, sfb_t = tmem + 136;   // scales: 2 chunks of 4 columns each
+
+    if (warp == 0) {
+        // ---- producer ----
+        int issued = 0;
+        for (int kt = 0; kt < KT; ++kt) {
+            const int s = kt % kStages;
+            if (kt >= kStages) {
+                int ok = 1;
+                if (lane == 0) ok = mbar_wait(&sm.empty[s], ((kt / kStages) - 1) & 1, abort, status);
+                if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+            }
+            // scales of rows lane + 32 q (q = 0..3): 8 bytes per row and K tile;
+            // chunk c holds scales 4c..4c+3 of each row, row r at byte (r%32)*16 + (r/32)*4
+            uint2 va[4], vb[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int r = lane + 32 * q;
+                va[q] = __ldg(reinterpret_cast<const uint2 *>(sf_a + (int64_t)(m0 + r) * sf_row + kt * 8));
+                vb[q] = __ldg(reinterpret_cast<const uint2 *>(sf_b + (int64_t)(n0 + r) * sf_row + kt * 8));
+            }
+            *reinterpret_cast<uint4 *>(&sm.sfa[s][lane * 16]) = make_uint4(va[0].x, va[1].x, va[2].x, va[3].x);
+            *reinterpret_cast<uint4 *>(&sm.sfa[s][512 + lane * 16]) = make_uint4(va[0].y, va[1].y, va[2].y, va[3].y);
+            *reinterpret_cast<uint4 *>(&sm.sfb[s][lane * 16]) = make_uint4(vb[0].x, vb[1].x, vb[2].x, vb[3].x);
+            *reinterpret_cast<uint4 *>(&sm.sfb[s][512 + lane * 16]) = make_uint4(vb[0].y, vb[1].y, vb[2].y, vb[3].y);
+            // the tensor core reads them through the async proxy
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive_expect_tx(&sm.full[s], kStageTx);
+                tma_load_2d(sm.a[s], &map_a, kt * (kBK / 2), m0, &sm.full[s]);
+                tma_load_2d(sm.b[s], &map_b, kt * (kBK / 2), n0, &sm.full[s]);
+            }
+            issued = kt + 1;
+        }
+        // after an abort, let the copies already issued land before the CTA exits
+        if (lane == 0 && *abort) {
+            for (int kt = max(0, issued - kStages); kt < issued; ++kt)
+                mbar_drain(&sm.full[kt % kStages], (kt / kStages) & 1);
+        }
+    } else if (warp == 1) {
+        // ---- MMA issuer ----
+        if (lane == 0) {
+            for (int kt = 0; kt < KT; ++kt) {
+                const int s = kt % kStages;
+                if (!mbar_wait(&sm.full[s], (kt / kStages) & 1, abort, status)) break;
+                tc_fence_after();
+                tmem_cp_sf(sfa_t, desc_sf(smem_u32(&sm.sfa[s][0])));
+                tmem_cp_sf(sfa_t + 4, desc_sf(smem_u32(&sm.sfa[s][512])));
+                tmem_cp_sf(sfb_t, desc_sf(smem_u32(&sm.sfb[s][0])));
+                tmem_cp_sf(sfb_t + 4, desc_sf(smem_u32(&sm.sfb[s][512])));
+                const uint32_t a0 = smem_u32(sm.a[s]), b0 = smem_u32(sm.b[s]);
+#pragma unroll
+                for (int kb = 0; kb < kBK / 64; ++kb) {
+                    // K = 64 per instruction: 32 bytes of each row; scale blocks
+                    // 2kb, 2kb+1 = chunk kb/2, bytes 2(kb%2), 2(kb%2)+1 of the word
+                    const uint32_t c = kb >> 1, id = (kb & 1) * 2;
+                    mma_mxf4(tmem, desc_sw128(a0 + kb * 32), desc_sw128(b0 + kb * 32),
+                             idesc_mxf4(id, id), sfa_t + 4 * c, sfb_t + 4 * c, (kt | kb) != 0);
+                }
+                umma_commit(&sm.empty[s]);          // frees the stage once these MMAs are done
+            }
+            umma_commit(&sm.acc_full);              // also after an abort: the epilogue waits on it
+        }
+        __syncwarp();
+    } else {
+        // ---- epilogue: TMEM lane quadrant = warp % 4 ----
+        const int quad = warp & 3;
+        int ok = 1;
+        if (lane == 0) ok = mbar_wait(&sm.acc_full, 0, abort, status) && !*abort;
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        tc_fence_after();
+        if (ok) {
+            const int64_t row = m0 + quad * 32 + lane;
+#pragma unroll 1
+            for (int c0 = 0; c0 < kBN; c0 += 32) {
+                float v[32];
+                tmem_ld32(tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)c0, v);
+                const float4 *ap = reinterpret_cast<const float4 *>(a_row + n0 + c0);
+                float4 *op = reinterpret_cast<float4 *>(out + row * N + n0 + c0);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const float4 sc = __ldg(ap + j);
+                    op[j] = make_float4(v[4 * j] * sc.x, v[4 * j + 1] * sc.y, v[4 * j + 2] * sc.z,
+                                        v[4 * j + 3] * sc.w);
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;"
+                     :: "r"(tmem), "r"(kTmemCols) : "memory");
+    }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess && q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+// 2-D map over a [rows, K/2]-byte code matrix: 128 x 128-byte boxes, 128-byte swizzle.
+bool code_map(CUtensorMap *m, const uint8_t *codes, int64_t rows, int64_t K) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)(K / 2), (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)(K / 2)};
+    const cuuint32_t box[2] = {(cuuint32_t)(kBK / 2), (cuuint32_t)kBM};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(codes), dims, strides,
+               box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+cudaError_t launch_w4a4_gemm(const GemmLaunch &L) {
+    if (L.M == 0 || L.N == 0) return cudaSuccess;
+    CUtensorMap ma, mb;
+    if (!code_map(&ma, L.codes_x, L.M, L.K) || !code_map(&mb, L.codes_w, L.N, L.K))
+        return cudaErrorInvalidValue;
+    const size_t smem = sizeof(GemmSmem) + 1024;
+    static bool done[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!done[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(w4a4_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)smem);
+        if (e != cudaSuccess) return e;
+        done[dev] = true;
+    }
+    return launch_k(w4a4_gemm_kernel, dim3((unsigned)(L.N / kBN), (unsigned)(L.M / kBM)),
+                    dim3(kThreadsGemm), smem, L.stream, ma, mb, L.scales_x, L.scales_w, L.a, L.out,
+                    (int)L.M, (int)L.N, (int)L.K, L.status);
+}
+
+}  // namespace dq

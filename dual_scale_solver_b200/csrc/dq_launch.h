@@ -77,6 +77,18 @@ struct TwoLevelLaunch {
 };
 cudaError_t launch_two_level(const TwoLevelLaunch &L);
 
+// Block-scaled W4A4 GEMM (dq_gemm.cu): out[M, N] = a_n * Qx[M, K] . Qw[N, K]^T.
+struct GemmLaunch {
+    const uint8_t *codes_x, *scales_x;   // [M, K/2] E2M1, [M, K/32] E8M0
+    const uint8_t *codes_w, *scales_w;   // [N, K/2] E2M1, [N, K/32] E8M0
+    const float *a;                      // [N]
+    float *out;                          // [M, N]
+    int64_t M, N, K;                     // multiples of 128, 128, 256
+    unsigned int *status;
+    cudaStream_t stream;
+};
+cudaError_t launch_w4a4_gemm(const GemmLaunch &L);
+
 cudaError_t launch_tile_c0(const TileLaunch &L);
 cudaError_t launch_tile_c1(const TileLaunch &L);
 cudaError_t launch_tile_c2(const TileLaunch &L);

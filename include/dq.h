@@ -66,7 +66,8 @@ typedef enum dq_status {
     DQ_ERR_WORKSPACE = -7,      /* workspace null or smaller than dq_workspace_size */
     DQ_ERR_NOT_IMPLEMENTED = -8,
     DQ_ERR_ALIGN = -9,          /* a pointer misses its alignment */
-    DQ_ERR_SCRATCH = -10        /* matrix needs more than the built-in scratch buffer */
+    DQ_ERR_SCRATCH = -10,       /* matrix needs more than the built-in scratch buffer */
+    DQ_ERR_TIMEOUT = -11        /* (device flag) a bounded wait in a kernel ran out */
 } dq_status;
 
 /* Code (element) types: the pages' INT4 and E2M1 codebooks, and the other
@@ -231,6 +232,22 @@ DQ_API dq_status dq_two_level_quant(const void *X, int32_t dtype, int64_t rows, 
                                     int32_t dual_block, const dq_format *inner, uint8_t *codes,
                                     void *inner_scales, float *outer_scales, float *qdq,
                                     dq_stream stream);
+
+/* Block-scaled W4A4 GEMM on the tensor cores, the inference step of eq. (1)
+ * (daiwk note, "核心公式": X W^T ~= (X D_b) Qhat^T D_a; trove summary, "How to
+ * use it"):  out[m, n] = a_n * sum_k Qx[m, k] * Qw[n, k], float32, where Qx
+ * is given by codes_x [M, K/2] and scales_x [M, K/32] (dq_act_rescale_quant
+ * output) and Qw by codes_w [N, K/2] and scales_w [N, K/32] (the solve's
+ * codes and group scales), a [N] the outer row scales of W.  `fmt` must be
+ * MXFP4 (E2M1 codes, E8M0 group scales, G = 32).  M and N multiples of 128,
+ * K a multiple of 256; every pointer 16-byte aligned; out [M, N] row-major,
+ * caller-owned.  The products are accumulated in float32.  Errors:
+ * DQ_ERR_FORMAT, DQ_ERR_SHAPE, DQ_ERR_ARG, DQ_ERR_ALIGN; a stalled pipeline
+ * (a bounded wait that ran out) raises the device flag read by
+ * dq_last_device_status as DQ_ERR_TIMEOUT. */
+DQ_API dq_status dq_w4a4_gemm(const uint8_t *codes_x, const void *scales_x, const uint8_t *codes_w,
+                              const void *scales_w, const float *a, int64_t M, int64_t N,
+                              int64_t K, const dq_format *fmt, float *out, dq_stream stream);
 
 /* Synchronise `stream`, read and clear the device flags raised by earlier
  * calls on this device: DQ_ERR_NONFINITE if an input held NaN/Inf (or

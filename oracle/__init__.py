@@ -15,4 +15,4 @@ from .solver import (Format, PRESETS, QMAX, CODE_BITS, preset, project_group_sca
                      round_codes, tensor_scale, quantize, dequantize, inner, qhat, mse,
                      row_update, col_update, solve, act_rescale_quant, encode_codes,
                      encode_scales, decode_codes, decode_scales, two_level_quant,
-                     MXFP4_MAX_NORMAL)
+                     MXFP4_MAX_NORMAL, w4a4_gemm)

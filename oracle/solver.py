@@ -339,3 +339,16 @@ def two_level_quant(X, dual_block: int, inner: Format):
     Sfull = np.repeat(S, dual_block, axis=1)[:, :cols]
     qdq = (inner_vals * Sfull).astype(np.float32).astype(np.float64)
     return c, s_in, S, qdq
+
+
+# --------------------------------------------------------------------------- #
+# The inference step: block-scaled W4A4 product
+# --------------------------------------------------------------------------- #
+
+def w4a4_gemm(cx, sx, cw, sw, a, fmt: Format):
+    """out[m, n] = a_n * sum_k Qx[m, k] Qw[n, k] with Qx = dequantize(cx, sx),
+    Qw = dequantize(cw, sw) (eq. (1) of the daiwk note: X W^T ~= (X D_b)
+    Qhat^T D_a).  Codes and scales as values; float64."""
+    Xq = dequantize(np.asarray(cx, dtype=np.float64), np.asarray(sx, dtype=np.float64), fmt)
+    Wq = dequantize(np.asarray(cw, dtype=np.float64), np.asarray(sw, dtype=np.float64), fmt)
+    return (Xq @ Wq.T) * np.asarray(a, dtype=np.float64)[None, :]

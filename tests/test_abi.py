@@ -24,7 +24,7 @@ def built():
 
 def test_exports_match_header():
     names = _declared()
-    assert len(names) == 18
+    assert len(names) == 19
     assert sorted(dq.EXPORTS) == names
     L = dq.lib()
     for n in names:
@@ -119,3 +119,15 @@ def test_two_level_argument_errors():
     assert L.dq_two_level_quant(*args(f, 512, 64)) == -1           # null pointers
     assert L.dq_two_level_quant(None, 1, 0, 64, 512, ctypes.byref(f), None, None, None, None,
                                 None) == 0                         # empty: nothing to do
+
+
+def test_w4a4_gemm_argument_errors():
+    L = dq.lib()
+    f = dq.format_preset("mxfp4")
+    nv = dq.format_preset("nvfp4")
+    args = lambda fmt, M, N, K: (None, None, None, None, None, M, N, K, ctypes.byref(fmt), None, None)
+    assert L.dq_w4a4_gemm(*args(nv, 128, 128, 256)) == -3          # MXFP4 only
+    assert L.dq_w4a4_gemm(*args(f, 100, 128, 256)) == -2           # M % 128
+    assert L.dq_w4a4_gemm(*args(f, 128, 128, 320)) == -2           # K % 256
+    assert L.dq_w4a4_gemm(*args(f, 128, 128, 256)) == -1           # null pointers
+    assert L.dq_w4a4_gemm(*args(f, 0, 128, 256)) == 0              # empty

@@ -448,3 +448,29 @@ def test_two_level_quant_special_cases():
     # zero input: S = 1, codes 0, scales 1, reconstruction 0
     c3, s3, S3, q3 = O.two_level_quant(np.zeros((2, 512)), 512, fmt)
     assert np.all(S3 == 1) and np.all(c3 == 0) and np.all(s3 == 1) and np.all(q3 == 0)
+
+
+def test_w4a4_gemm_against_explicit_sums():
+    # out[m, n] = a_n sum_k (c_x s_x)(c_w s_w), written out with fractions
+    fmt = O.preset("mxfp4")
+    rng = np.random.default_rng(31)
+    M, N, K = 3, 2, 64
+    grid = np.concatenate([O.E2M1_GRID, -O.E2M1_GRID])
+    cx, cw = rng.choice(grid, (M, K)), rng.choice(grid, (N, K))
+    sx = np.ldexp(1.0, rng.integers(-8, 8, (M, K // 32)))
+    sw = np.ldexp(1.0, rng.integers(-8, 8, (N, K // 32)))
+    a = np.array([0.5, 4.0])
+    out = O.w4a4_gemm(cx, sx, cw, sw, a, fmt)
+    for m in range(M):
+        for n in range(N):
+            acc = sum(Fr(float(cx[m, k])) * Fr(float(sx[m, k // 32])) * Fr(float(cw[n, k])) *
+                      Fr(float(sw[n, k // 32])) for k in range(K))
+            assert out[m, n] == float(acc * Fr(float(a[n])))
+    # the eq. (1) identity: with the solver's state, the product approximates X W^T
+    W = _small_matrix(64, 128, seed=32)
+    r = O.solve(W, fmt, 3)
+    X = rng.standard_normal((16, 128))
+    cxa, sxa = O.act_rescale_quant(X, r["b"], fmt)
+    approx = O.w4a4_gemm(cxa, sxa, r["codes"], r["scales"], r["a"], fmt)
+    exact = X @ W.T
+    assert np.linalg.norm(approx - exact) < 0.25 * np.linalg.norm(exact)
