@@ -53,7 +53,8 @@ def _args():
                    help="profiling case: keep only this linear of the decoder")
     p.add_argument("--T", type=int, default=-1, help="profiling case: iterations override")
     p.add_argument("--no-act", action="store_true", help="profiling case: skip activations")
-    p.add_argument("--method", default="dualquant", choices=["dualquant", "two_level"],
+    p.add_argument("--tokens", type=int, default=32768, help="w4a4_gemm: activation rows")
+    p.add_argument("--method", default="dualquant", choices=["dualquant", "two_level", "w4a4_gemm"],
                    help="two_level: the two-level absmax quantization of the same weights "
                         "and activations instead of the solve")
     return p.parse_args()
@@ -519,6 +520,84 @@ def run_two_level(args, wl, rank, world, local_rank):
     return 0
 
 
+def run_gemm(args, wl, rank, world, local_rank):
+    """The inference step after the solve: every linear of the workload's
+    decoder(s) as a block-scaled W4A4 GEMM (MXFP4 x MXFP4, E8M0 scales) on a
+    batch of `tokens` activation rows; the weights' codes, scales and a come
+    from the solve, the activations' codes and scales from the activation
+    quantizer (one batch per input width)."""
+    import torch
+    import synth
+    import dual_scale_solver_b200 as dq
+    from dual_scale_solver_b200 import build
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    build.build()
+    fmt = dq.format_preset("mxfp4")
+    Ws = [synth.weight(wl, d, i, device=dev) for d in decoders_of(rank, wl.decoders)
+          for i in range(len(wl.linears))]
+    outs = dq.solve_dual_scale_batched(Ws, fmt, wl.T)
+    M = args.tokens
+    acts = {}
+    for W in Ws:                                  # one quantized activation batch per width K
+        K = W.shape[1]
+        if K not in acts:
+            X = synth.normal(synth.stream_key(70, K), M * K, device=dev).view(M, K).to(torch.bfloat16)
+            acts[K] = dq.act_rescale_quant(X, torch.ones(K, device=dev), fmt)
+            del X
+    res = [torch.empty(M, W.shape[0], dtype=torch.float32, device=dev) for W in Ws]
+    del Ws
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        for o, r in zip(outs, res):
+            cx, sx = acts[2 * o["codes"].shape[1]]
+            dq.w4a4_gemm(cx, sx, o["codes"], o["gscales"], o["a"], fmt, out=r)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    clocks = Clocks(local_rank)
+    clocks.start()
+    time.sleep(0.3)
+    n0 = dq.launch_count()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = max_over_ranks(e0.elapsed_time(e1), dev) / args.steps
+    launches = dq.launch_count() - n0
+    clk = clocks.stop()
+    if dq.last_device_status() != 0:
+        raise RuntimeError("device status flags raised during timing")
+    flops = sum(2.0 * M * o["codes"].shape[0] * 2 * o["codes"].shape[1] for o in outs)
+    peaks, which = _peaks()
+    # FP4 dense peak = the measured bf16 GEMM peak x the nominal fp4/bf16 ratio (9 / 2.25)
+    peak = float(peaks.get("bf16_tflops", 1590.0)) * 4.0
+    tflops = flops / (ms / 1e3) / 1e12
+    line = {
+        "metric": "W4A4 GEMM TFLOP/s (MXFP4 x MXFP4, E8M0 scales, fp32 accumulate)",
+        "value": world * tflops, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "fp4 (e2m1)", "data": "synthetic",
+        "config": {"workload": f"{wl.name}: its {len(outs)} linears x {M} tokens",
+                   "flops_per_step": flops, "tile": "128 x (256 if N % 256 == 0 else 128) x 256, 4 stages",
+                   "l2": "operands larger than L2 (no flush needed)",
+                   "parallelism": f"{world} independent decoders" if world > 1 else "1 GPU"},
+        "roofline": {"bound": "tensor", "achieved": tflops, "peak": peak, "unit": "TFLOP/s",
+                     "frac": tflops / peak,
+                     "peak_source": f"{which} bf16 x 4 (nominal fp4/bf16 ratio)",
+                     "traffic": None},
+        "gpu_launches": launches, "clocks": clk, "e2e": None,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = _args()
     import synth
@@ -538,6 +617,8 @@ def main():
     try:
         if args.method == "two_level":
             return run_two_level(args, wl, rank, world, local_rank)
+        if args.method == "w4a4_gemm":
+            return run_gemm(args, wl, rank, world, local_rank)
         return run_ours(args, wl, rank, world, local_rank)
     finally:
         if world > 1:

@@ -35,21 +35,27 @@ namespace dq {
 
 namespace {
 
-constexpr int kBM = 128, kBN = 128;
+constexpr int kBM = 128;
 constexpr int kBK = 256;                       // K elements per stage (128 bytes per row)
 constexpr int kStages = 4;
-constexpr int kTileBytes = kBM * kBK / 2;      // 16 KB per operand tile
-constexpr int kSfBytes = kBM * kBK / 32;       // 1 KB: two 512-byte chunks of 4 scales per row
-constexpr uint32_t kStageTx = 2u * kTileBytes; // TMA bytes per stage (the scales are stored by threads)
+constexpr int kTileBytesA = kBM * kBK / 2;     // 16 KB per A tile
+constexpr int kSfChunk = 512;                  // 128 rows x 4 scales
 constexpr int kThreadsGemm = 192;
-constexpr uint32_t kTmemCols = 256;            // accumulator 128 + scales 16, rounded up
 constexpr uint64_t kWaitLimitNs = 1000000000ull;   // a wait gives up after 1 s
 
+// BN = 128 or 256 output columns per CTA.
+template <int BN>
 struct __align__(1024) GemmSmem {
-    uint8_t a[kStages][kTileBytes];
-    uint8_t b[kStages][kTileBytes];
-    uint8_t sfa[kStages][kSfBytes];
-    uint8_t sfb[kStages][kSfBytes];
+    static constexpr int NB = BN / 128;                        // 128-row blocks of B
+    static constexpr int kTileBytesB = BN * kBK / 2;
+    static constexpr uint32_t kStageTx = kTileBytesA + kTileBytesB;   // TMA bytes per stage
+    // TMEM: accumulator BN columns, then A's scales (2 chunks x 4 columns),
+    // then B's (2 k-chunks x NB row blocks x 4 columns)
+    static constexpr uint32_t kTmemCols = BN == 128 ? 256 : 512;
+    uint8_t a[kStages][kTileBytesA];
+    uint8_t b[kStages][kTileBytesB];
+    uint8_t sfa[kStages][2 * kSfChunk];            // [k-chunk][512]
+    uint8_t sfb[kStages][2 * NB * kSfChunk];       // [k-chunk][row block][512]
     uint64_t full[kStages];
     uint64_t empty[kStages];
     uint64_t acc_full;
@@ -126,9 +132,10 @@ __device__ __forceinline__ uint64_t desc_sf(uint32_t saddr) {
 }
 
 // Instruction descriptor, kind::mxf4 with E8M0 block scales: A and B E2M1
-// (K-major), M = 128, N = 128, scale-factor byte ids of A and B.
+// (K-major), M = 128, N = BN, scale-factor byte ids of A and B.
+template <int BN>
 __device__ __forceinline__ uint32_t idesc_mxf4(uint32_t sfa_id, uint32_t sfb_id) {
-    return (sfb_id << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kBN >> 3) << 17) | (1u << 23) |
+    return (sfb_id << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | (1u << 23) |
            ((uint32_t)(kBM >> 4) << 24) | (sfa_id << 29);
 }
 
@@ -187,23 +194,26 @@ __device__ __forceinline__ void mbar_drain(uint64_t *b, uint32_t parity) {
     }
 }
 
+template <int BN>
 __global__ void __launch_bounds__(kThreadsGemm, 1)
 w4a4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                  const uint8_t *sf_a, const uint8_t *sf_b, const float *a_row, float *out, int M,
                  int N, int K, unsigned int *status) {
+    using Smem = GemmSmem<BN>;
+    constexpr int NB = Smem::NB;
     grid_dependency_begin();
     extern __shared__ uint8_t gemm_smem_raw[];
-    GemmSmem &sm = *reinterpret_cast<GemmSmem *>(
+    Smem &sm = *reinterpret_cast<Smem *>(
         (reinterpret_cast<uintptr_t>(gemm_smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int n0 = blockIdx.x * kBN, m0 = blockIdx.y * kBM;
+    const int n0 = blockIdx.x * BN, m0 = blockIdx.y * kBM;
     const int KT = K / kBK;
     const int64_t sf_row = K / 32;                  // scale bytes per row
     volatile int *abort = &sm.abort;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
-            mbar_init(&sm.full[s], 1);
+            mbar_init(&sm.full[s], 2);              // the TMA arrival and the scales' arrival
             mbar_init(&sm.empty[s], 1);
         }
         mbar_init(&sm.acc_full, 1);
@@ -212,17 +222,30 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
     }
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
-                     :: "r"(smem_u32(&sm.tmem_base)), "r"(kTmemCols) : "memory");
+                     :: "r"(smem_u32(&sm.tmem_base)), "r"(Smem::kTmemCols) : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem = sm.tmem_base;             // accumulator: columns [0, 128)
-    const uint32_t sfa_t = tmem + 128, sfb_t = tmem + 136;   // scales: 2 chunks of 4 columns each
+    const uint32_t tmem = sm.tmem_base;             // accumulator: columns [0, BN)
+    const uint32_t sfa_t = tmem + BN, sfb_t = tmem + BN + 8;
 
     if (warp == 0) {
-        // ---- producer ----
+        // ---- producer: TMA first, then the scales (gathered one stage ahead) ----
+        // lane gathers rows lane + 32 q: q < 4 of A, q < 4 NB of B; 8 scale
+        // bytes per row and K tile; chunk kc holds scales 4kc..4kc+3 of each
+        // row, row r of a 128-row block at byte (r%32)*16 + (r/32)*4
+        uint2 va[4], vb[4 * NB];
+        auto gather = [&](int kt) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                va[q] = __ldg(reinterpret_cast<const uint2 *>(sf_a + (int64_t)(m0 + lane + 32 * q) * sf_row + kt * 8));
+#pragma unroll
+            for (int q = 0; q < 4 * NB; ++q)
+                vb[q] = __ldg(reinterpret_cast<const uint2 *>(sf_b + (int64_t)(n0 + lane + 32 * q) * sf_row + kt * 8));
+        };
+        gather(0);
         int issued = 0;
         for (int kt = 0; kt < KT; ++kt) {
             const int s = kt % kStages;
@@ -231,28 +254,28 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
                 if (lane == 0) ok = mbar_wait(&sm.empty[s], ((kt / kStages) - 1) & 1, abort, status);
                 if (!__shfl_sync(0xffffffffu, ok, 0)) break;
             }
-            // scales of rows lane + 32 q (q = 0..3): 8 bytes per row and K tile;
-            // chunk c holds scales 4c..4c+3 of each row, row r at byte (r%32)*16 + (r/32)*4
-            uint2 va[4], vb[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const int r = lane + 32 * q;
-                va[q] = __ldg(reinterpret_cast<const uint2 *>(sf_a + (int64_t)(m0 + r) * sf_row + kt * 8));
-                vb[q] = __ldg(reinterpret_cast<const uint2 *>(sf_b + (int64_t)(n0 + r) * sf_row + kt * 8));
-            }
-            *reinterpret_cast<uint4 *>(&sm.sfa[s][lane * 16]) = make_uint4(va[0].x, va[1].x, va[2].x, va[3].x);
-            *reinterpret_cast<uint4 *>(&sm.sfa[s][512 + lane * 16]) = make_uint4(va[0].y, va[1].y, va[2].y, va[3].y);
-            *reinterpret_cast<uint4 *>(&sm.sfb[s][lane * 16]) = make_uint4(vb[0].x, vb[1].x, vb[2].x, vb[3].x);
-            *reinterpret_cast<uint4 *>(&sm.sfb[s][512 + lane * 16]) = make_uint4(vb[0].y, vb[1].y, vb[2].y, vb[3].y);
-            // the tensor core reads them through the async proxy
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            __syncwarp();
             if (lane == 0) {
-                mbar_arrive_expect_tx(&sm.full[s], kStageTx);
+                mbar_arrive_expect_tx(&sm.full[s], Smem::kStageTx);
                 tma_load_2d(sm.a[s], &map_a, kt * (kBK / 2), m0, &sm.full[s]);
                 tma_load_2d(sm.b[s], &map_b, kt * (kBK / 2), n0, &sm.full[s]);
             }
+            *reinterpret_cast<uint4 *>(&sm.sfa[s][lane * 16]) = make_uint4(va[0].x, va[1].x, va[2].x, va[3].x);
+            *reinterpret_cast<uint4 *>(&sm.sfa[s][kSfChunk + lane * 16]) = make_uint4(va[0].y, va[1].y, va[2].y, va[3].y);
+#pragma unroll
+            for (int nb = 0; nb < NB; ++nb) {
+                const uint2 *v = vb + 4 * nb;
+                *reinterpret_cast<uint4 *>(&sm.sfb[s][nb * kSfChunk + lane * 16]) =
+                    make_uint4(v[0].x, v[1].x, v[2].x, v[3].x);
+                *reinterpret_cast<uint4 *>(&sm.sfb[s][(NB + nb) * kSfChunk + lane * 16]) =
+                    make_uint4(v[0].y, v[1].y, v[2].y, v[3].y);
+            }
+            // the tensor core reads them through the async proxy
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncwarp();
+            if (lane == 0)
+                asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" :: "r"(smem_u32(&sm.full[s])) : "memory");
             issued = kt + 1;
+            if (kt + 1 < KT) gather(kt + 1);
         }
         // after an abort, let the copies already issued land before the CTA exits
         if (lane == 0 && *abort) {
@@ -267,17 +290,20 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
                 if (!mbar_wait(&sm.full[s], (kt / kStages) & 1, abort, status)) break;
                 tc_fence_after();
                 tmem_cp_sf(sfa_t, desc_sf(smem_u32(&sm.sfa[s][0])));
-                tmem_cp_sf(sfa_t + 4, desc_sf(smem_u32(&sm.sfa[s][512])));
-                tmem_cp_sf(sfb_t, desc_sf(smem_u32(&sm.sfb[s][0])));
-                tmem_cp_sf(sfb_t + 4, desc_sf(smem_u32(&sm.sfb[s][512])));
+                tmem_cp_sf(sfa_t + 4, desc_sf(smem_u32(&sm.sfa[s][kSfChunk])));
+#pragma unroll
+                for (int j = 0; j < 2 * NB; ++j)
+                    tmem_cp_sf(sfb_t + 4 * j, desc_sf(smem_u32(&sm.sfb[s][j * kSfChunk])));
                 const uint32_t a0 = smem_u32(sm.a[s]), b0 = smem_u32(sm.b[s]);
 #pragma unroll
                 for (int kb = 0; kb < kBK / 64; ++kb) {
                     // K = 64 per instruction: 32 bytes of each row; scale blocks
-                    // 2kb, 2kb+1 = chunk kb/2, bytes 2(kb%2), 2(kb%2)+1 of the word
+                    // 2kb, 2kb+1 = k-chunk kb/2, bytes 2(kb%2), 2(kb%2)+1 of the
+                    // word; B's scales of the k-chunk span NB x 4 columns
                     const uint32_t c = kb >> 1, id = (kb & 1) * 2;
                     mma_mxf4(tmem, desc_sw128(a0 + kb * 32), desc_sw128(b0 + kb * 32),
-                             idesc_mxf4(id, id), sfa_t + 4 * c, sfb_t + 4 * c, (kt | kb) != 0);
+                             idesc_mxf4<BN>(id, id), sfa_t + 4 * c, sfb_t + 4 * NB * c,
+                             (kt | kb) != 0);
                 }
                 umma_commit(&sm.empty[s]);          // frees the stage once these MMAs are done
             }
@@ -294,7 +320,7 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
         if (ok) {
             const int64_t row = m0 + quad * 32 + lane;
 #pragma unroll 1
-            for (int c0 = 0; c0 < kBN; c0 += 32) {
+            for (int c0 = 0; c0 < BN; c0 += 32) {
                 float v[32];
                 tmem_ld32(tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)c0, v);
                 const float4 *ap = reinterpret_cast<const float4 *>(a_row + n0 + c0);
@@ -313,7 +339,7 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
     if (warp == 1) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;"
-                     :: "r"(tmem), "r"(kTmemCols) : "memory");
+                     :: "r"(tmem), "r"(Smem::kTmemCols) : "memory");
     }
 }
 
@@ -329,39 +355,47 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
     return fn;
 }
 
-// 2-D map over a [rows, K/2]-byte code matrix: 128 x 128-byte boxes, 128-byte swizzle.
-bool code_map(CUtensorMap *m, const uint8_t *codes, int64_t rows, int64_t K) {
+// 2-D map over a [rows, K/2]-byte code matrix: boxes of box_rows x 128 bytes,
+// 128-byte swizzle.
+bool code_map(CUtensorMap *m, const uint8_t *codes, int64_t rows, int64_t K, int box_rows) {
     auto enc = tensor_map_encoder();
     if (!enc) return false;
     const cuuint64_t dims[2] = {(cuuint64_t)(K / 2), (cuuint64_t)rows};
     const cuuint64_t strides[1] = {(cuuint64_t)(K / 2)};
-    const cuuint32_t box[2] = {(cuuint32_t)(kBK / 2), (cuuint32_t)kBM};
+    const cuuint32_t box[2] = {(cuuint32_t)(kBK / 2), (cuuint32_t)box_rows};
     const cuuint32_t estr[2] = {1, 1};
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(codes), dims, strides,
                box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-}  // namespace
-
-cudaError_t launch_w4a4_gemm(const GemmLaunch &L) {
-    if (L.M == 0 || L.N == 0) return cudaSuccess;
+template <int BN>
+cudaError_t launch_bn(const GemmLaunch &L) {
     CUtensorMap ma, mb;
-    if (!code_map(&ma, L.codes_x, L.M, L.K) || !code_map(&mb, L.codes_w, L.N, L.K))
+    if (!code_map(&ma, L.codes_x, L.M, L.K, kBM) || !code_map(&mb, L.codes_w, L.N, L.K, BN))
         return cudaErrorInvalidValue;
-    const size_t smem = sizeof(GemmSmem) + 1024;
+    const size_t smem = sizeof(GemmSmem<BN>) + 1024;
     static bool done[64] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     if (!done[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(w4a4_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)smem);
+        cudaError_t e = cudaFuncSetAttribute(w4a4_gemm_kernel<BN>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
         done[dev] = true;
     }
-    return launch_k(w4a4_gemm_kernel, dim3((unsigned)(L.N / kBN), (unsigned)(L.M / kBM)),
+    return launch_k(w4a4_gemm_kernel<BN>, dim3((unsigned)(L.N / BN), (unsigned)(L.M / kBM)),
                     dim3(kThreadsGemm), smem, L.stream, ma, mb, L.scales_x, L.scales_w, L.a, L.out,
                     (int)L.M, (int)L.N, (int)L.K, L.status);
+}
+
+}  // namespace
+
+// 256 output columns per CTA when N allows it (A tiles reused twice as
+// often), else 128.
+cudaError_t launch_w4a4_gemm(const GemmLaunch &L) {
+    if (L.M == 0 || L.N == 0) return cudaSuccess;
+    return (L.N % 256 == 0) ? launch_bn<256>(L) : launch_bn<128>(L);
 }
 
 }  // namespace dq
