@@ -16,9 +16,9 @@
 // accumulating in float32 in TMEM.  K advances in tiles of 256 elements (128
 // bytes per row) through a 4-stage shared-memory ring:
 //   warp 0     producer: TMA loads of the A and B tiles (128-byte swizzle,
-//              no multicast) and the two operands' scale factors, gathered
-//              from their row-major arrays into the 128-row x 4-scale chunk
-//              layout the tensor core reads;
+//              no multicast) and 4-byte cp.async copies of the two operands'
+//              scale factors from their row-major arrays into the 128-row x
+//              4-scale chunk layout the tensor core reads;
 //   warp 1     TMEM allocation; lane 0 issues tcgen05.cp (scales to TMEM),
 //              the MMAs and the tcgen05.commit arrivals;
 //   warps 2-5  epilogue: TMEM -> registers (tcgen05.ld), times a_n, stores.
@@ -106,6 +106,11 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *b, uint32_t parity, volatile
     *abort = 1;
     atomicOr(status, STATUS_TIMEOUT);
     return false;
+}
+
+__device__ __forceinline__ void cp_async4(void *dst, const void *src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" :: "r"(smem_u32(dst)), "l"(src)
+                 : "memory");
 }
 
 __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y,
@@ -213,7 +218,7 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
-            mbar_init(&sm.full[s], 2);              // the TMA arrival and the scales' arrival
+            mbar_init(&sm.full[s], 33);             // the TMA arrival + 32 lanes' scale copies
             mbar_init(&sm.empty[s], 1);
         }
         mbar_init(&sm.acc_full, 1);
@@ -232,20 +237,12 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
     const uint32_t sfa_t = tmem + BN, sfb_t = tmem + BN + 8;
 
     if (warp == 0) {
-        // ---- producer: TMA first, then the scales (gathered one stage ahead) ----
-        // lane gathers rows lane + 32 q: q < 4 of A, q < 4 NB of B; 8 scale
-        // bytes per row and K tile; chunk kc holds scales 4kc..4kc+3 of each
-        // row, row r of a 128-row block at byte (r%32)*16 + (r/32)*4
-        uint2 va[4], vb[4 * NB];
-        auto gather = [&](int kt) {
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-                va[q] = __ldg(reinterpret_cast<const uint2 *>(sf_a + (int64_t)(m0 + lane + 32 * q) * sf_row + kt * 8));
-#pragma unroll
-            for (int q = 0; q < 4 * NB; ++q)
-                vb[q] = __ldg(reinterpret_cast<const uint2 *>(sf_b + (int64_t)(n0 + lane + 32 * q) * sf_row + kt * 8));
-        };
-        gather(0);
+        // ---- producer: TMA for the code tiles; the scales by 4-byte cp.async
+        // straight into the chunk layout (lane copies rows lane + 32 q: q < 4
+        // of A, q < 4 NB of B; chunk kc holds scales 4kc..4kc+3 of each row,
+        // row r of a 128-row block at byte (r%32)*16 + (r/32)*4).  Each lane's
+        // cp.async.mbarrier.arrive fires once its copies have landed, so the
+        // stage's barrier completes with the TMA bytes and 32 such arrivals. ----
         int issued = 0;
         for (int kt = 0; kt < KT; ++kt) {
             const int s = kt % kStages;
@@ -259,23 +256,22 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
                 tma_load_2d(sm.a[s], &map_a, kt * (kBK / 2), m0, &sm.full[s]);
                 tma_load_2d(sm.b[s], &map_b, kt * (kBK / 2), n0, &sm.full[s]);
             }
-            *reinterpret_cast<uint4 *>(&sm.sfa[s][lane * 16]) = make_uint4(va[0].x, va[1].x, va[2].x, va[3].x);
-            *reinterpret_cast<uint4 *>(&sm.sfa[s][kSfChunk + lane * 16]) = make_uint4(va[0].y, va[1].y, va[2].y, va[3].y);
 #pragma unroll
-            for (int nb = 0; nb < NB; ++nb) {
-                const uint2 *v = vb + 4 * nb;
-                *reinterpret_cast<uint4 *>(&sm.sfb[s][nb * kSfChunk + lane * 16]) =
-                    make_uint4(v[0].x, v[1].x, v[2].x, v[3].x);
-                *reinterpret_cast<uint4 *>(&sm.sfb[s][(NB + nb) * kSfChunk + lane * 16]) =
-                    make_uint4(v[0].y, v[1].y, v[2].y, v[3].y);
+            for (int q = 0; q < 4; ++q) {
+                const uint8_t *src = sf_a + (int64_t)(m0 + lane + 32 * q) * sf_row + kt * 8;
+                cp_async4(&sm.sfa[s][lane * 16 + q * 4], src);
+                cp_async4(&sm.sfa[s][kSfChunk + lane * 16 + q * 4], src + 4);
             }
-            // the tensor core reads them through the async proxy
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            __syncwarp();
-            if (lane == 0)
-                asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" :: "r"(smem_u32(&sm.full[s])) : "memory");
+#pragma unroll
+            for (int q = 0; q < 4 * NB; ++q) {
+                const uint8_t *src = sf_b + (int64_t)(n0 + lane + 32 * q) * sf_row + kt * 8;
+                const int nb = q >> 2, qq = q & 3;
+                cp_async4(&sm.sfb[s][nb * kSfChunk + lane * 16 + qq * 4], src);
+                cp_async4(&sm.sfb[s][(NB + nb) * kSfChunk + lane * 16 + qq * 4], src + 4);
+            }
+            asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];"
+                         :: "r"(smem_u32(&sm.full[s])) : "memory");
             issued = kt + 1;
-            if (kt + 1 < KT) gather(kt + 1);
         }
         // after an abort, let the copies already issued land before the CTA exits
         if (lane == 0 && *abort) {
@@ -288,6 +284,9 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
             for (int kt = 0; kt < KT; ++kt) {
                 const int s = kt % kStages;
                 if (!mbar_wait(&sm.full[s], (kt / kStages) & 1, abort, status)) break;
+                // the scales came through the generic proxy; tcgen05.cp reads
+                // them through the async proxy
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                 tc_fence_after();
                 tmem_cp_sf(sfa_t, desc_sf(smem_u32(&sm.sfa[s][0])));
                 tmem_cp_sf(sfa_t + 4, desc_sf(smem_u32(&sm.sfa[s][kSfChunk])));
