@@ -11,10 +11,12 @@
 // the outer row scales of W.  Both operands are K-major E2M1, two codes per
 // byte, with one E8M0 scale per 32 elements of K.
 //
-// One CTA computes a 128 x 128 tile of `out` with tcgen05.mma kind::mxf4
-// (M = 128, N = 128, K = 64 per instruction, block scales of 32 from TMEM),
+// A persistent CTA per SM walks 128 x BN tiles of `out` (BN = 256, or 128
+// when N is not a multiple of 256) with tcgen05.mma kind::mxf4 (M = 128,
+// N = BN, K = 64 per instruction, block scales of 32 from TMEM),
 // accumulating in float32 in TMEM.  K advances in tiles of 256 elements (128
-// bytes per row) through a 4-stage shared-memory ring:
+// bytes per row) through a 4-stage shared-memory ring that runs on across
+// output tiles:
 //   warp 0     producer: TMA loads of the A and B tiles (128-byte swizzle,
 //              no multicast) and 4-byte cp.async copies of the two operands'
 //              scale factors from their row-major arrays into the 128-row x
@@ -58,7 +60,8 @@ struct __align__(1024) GemmSmem {
     uint8_t sfb[kStages][2 * NB * kSfChunk];       // [k-chunk][row block][512]
     uint64_t full[kStages];
     uint64_t empty[kStages];
-    uint64_t acc_full;
+    uint64_t acc_full;      // MMA -> epilogue: the tile's accumulator is complete
+    uint64_t acc_empty;     // epilogue -> MMA: the accumulator has been read out
     uint32_t tmem_base;
     int abort;
 };
@@ -211,8 +214,9 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
     Smem &sm = *reinterpret_cast<Smem *>(
         (reinterpret_cast<uintptr_t>(gemm_smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int n0 = blockIdx.x * BN, m0 = blockIdx.y * kBM;
     const int KT = K / kBK;
+    const int n_tiles = N / BN;
+    const int tiles = (M / kBM) * n_tiles;
     const int64_t sf_row = K / 32;                  // scale bytes per row
     volatile int *abort = &sm.abort;
 
@@ -222,6 +226,7 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
             mbar_init(&sm.empty[s], 1);
         }
         mbar_init(&sm.acc_full, 1);
+        mbar_init(&sm.acc_empty, 4);                // one arrival per epilogue warp
         sm.abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -236,99 +241,127 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
     const uint32_t tmem = sm.tmem_base;             // accumulator: columns [0, BN)
     const uint32_t sfa_t = tmem + BN, sfb_t = tmem + BN + 8;
 
+    // The CTA walks the output tiles t = blockIdx.x, + gridDim.x, ...; tile t
+    // is (t / n_tiles, t % n_tiles), so CTAs running together share A rows.
     if (warp == 0) {
         // ---- producer: TMA for the code tiles; the scales by 4-byte cp.async
         // straight into the chunk layout (lane copies rows lane + 32 q: q < 4
         // of A, q < 4 NB of B; chunk kc holds scales 4kc..4kc+3 of each row,
         // row r of a 128-row block at byte (r%32)*16 + (r/32)*4).  Each lane's
         // cp.async.mbarrier.arrive fires once its copies have landed, so the
-        // stage's barrier completes with the TMA bytes and 32 such arrivals. ----
-        int issued = 0;
-        for (int kt = 0; kt < KT; ++kt) {
-            const int s = kt % kStages;
-            if (kt >= kStages) {
-                int ok = 1;
-                if (lane == 0) ok = mbar_wait(&sm.empty[s], ((kt / kStages) - 1) & 1, abort, status);
-                if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-            }
-            if (lane == 0) {
-                mbar_arrive_expect_tx(&sm.full[s], Smem::kStageTx);
-                tma_load_2d(sm.a[s], &map_a, kt * (kBK / 2), m0, &sm.full[s]);
-                tma_load_2d(sm.b[s], &map_b, kt * (kBK / 2), n0, &sm.full[s]);
-            }
+        // stage's barrier completes with the TMA bytes and 32 such arrivals.
+        // The ring runs on across tiles (g counts K tiles of all the CTA's
+        // output tiles), so the next tile's operands arrive during the
+        // current tile's last MMAs and epilogue. ----
+        int g = 0;
+        bool stop = false;
+        for (int t = blockIdx.x; t < tiles && !stop; t += gridDim.x) {
+            const int m0 = (t / n_tiles) * kBM, n0 = (t % n_tiles) * BN;
+            for (int kt = 0; kt < KT; ++kt, ++g) {
+                const int s = g % kStages;
+                if (g >= kStages) {
+                    int ok = 1;
+                    if (lane == 0) ok = mbar_wait(&sm.empty[s], ((g / kStages) - 1) & 1, abort, status);
+                    if (!__shfl_sync(0xffffffffu, ok, 0)) { stop = true; break; }
+                }
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(&sm.full[s], Smem::kStageTx);
+                    tma_load_2d(sm.a[s], &map_a, kt * (kBK / 2), m0, &sm.full[s]);
+                    tma_load_2d(sm.b[s], &map_b, kt * (kBK / 2), n0, &sm.full[s]);
+                }
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const uint8_t *src = sf_a + (int64_t)(m0 + lane + 32 * q) * sf_row + kt * 8;
-                cp_async4(&sm.sfa[s][lane * 16 + q * 4], src);
-                cp_async4(&sm.sfa[s][kSfChunk + lane * 16 + q * 4], src + 4);
-            }
+                for (int q = 0; q < 4; ++q) {
+                    const uint8_t *src = sf_a + (int64_t)(m0 + lane + 32 * q) * sf_row + kt * 8;
+                    cp_async4(&sm.sfa[s][lane * 16 + q * 4], src);
+                    cp_async4(&sm.sfa[s][kSfChunk + lane * 16 + q * 4], src + 4);
+                }
 #pragma unroll
-            for (int q = 0; q < 4 * NB; ++q) {
-                const uint8_t *src = sf_b + (int64_t)(n0 + lane + 32 * q) * sf_row + kt * 8;
-                const int nb = q >> 2, qq = q & 3;
-                cp_async4(&sm.sfb[s][nb * kSfChunk + lane * 16 + qq * 4], src);
-                cp_async4(&sm.sfb[s][(NB + nb) * kSfChunk + lane * 16 + qq * 4], src + 4);
+                for (int q = 0; q < 4 * NB; ++q) {
+                    const uint8_t *src = sf_b + (int64_t)(n0 + lane + 32 * q) * sf_row + kt * 8;
+                    const int nb = q >> 2, qq = q & 3;
+                    cp_async4(&sm.sfb[s][nb * kSfChunk + lane * 16 + qq * 4], src);
+                    cp_async4(&sm.sfb[s][(NB + nb) * kSfChunk + lane * 16 + qq * 4], src + 4);
+                }
+                asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];"
+                             :: "r"(smem_u32(&sm.full[s])) : "memory");
             }
-            asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];"
-                         :: "r"(smem_u32(&sm.full[s])) : "memory");
-            issued = kt + 1;
         }
         // after an abort, let the copies already issued land before the CTA exits
         if (lane == 0 && *abort) {
-            for (int kt = max(0, issued - kStages); kt < issued; ++kt)
-                mbar_drain(&sm.full[kt % kStages], (kt / kStages) & 1);
+            for (int k = max(0, g - kStages); k < g; ++k)
+                mbar_drain(&sm.full[k % kStages], (k / kStages) & 1);
         }
     } else if (warp == 1) {
         // ---- MMA issuer ----
         if (lane == 0) {
-            for (int kt = 0; kt < KT; ++kt) {
-                const int s = kt % kStages;
-                if (!mbar_wait(&sm.full[s], (kt / kStages) & 1, abort, status)) break;
-                // the scales came through the generic proxy; tcgen05.cp reads
-                // them through the async proxy
-                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            int g = 0, j = 0;
+            bool stop = false;
+            for (int t = blockIdx.x; t < tiles && !stop; t += gridDim.x, ++j) {
+                // the epilogue has read out the previous tile's accumulator
+                if (j > 0 && !mbar_wait(&sm.acc_empty, (j - 1) & 1, abort, status)) break;
                 tc_fence_after();
-                tmem_cp_sf(sfa_t, desc_sf(smem_u32(&sm.sfa[s][0])));
-                tmem_cp_sf(sfa_t + 4, desc_sf(smem_u32(&sm.sfa[s][kSfChunk])));
+                for (int kt = 0; kt < KT; ++kt, ++g) {
+                    const int s = g % kStages;
+                    if (!mbar_wait(&sm.full[s], (g / kStages) & 1, abort, status)) { stop = true; break; }
+                    // the scales came through the generic proxy; tcgen05.cp
+                    // reads them through the async proxy
+                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                    tc_fence_after();
+                    tmem_cp_sf(sfa_t, desc_sf(smem_u32(&sm.sfa[s][0])));
+                    tmem_cp_sf(sfa_t + 4, desc_sf(smem_u32(&sm.sfa[s][kSfChunk])));
 #pragma unroll
-                for (int j = 0; j < 2 * NB; ++j)
-                    tmem_cp_sf(sfb_t + 4 * j, desc_sf(smem_u32(&sm.sfb[s][j * kSfChunk])));
-                const uint32_t a0 = smem_u32(sm.a[s]), b0 = smem_u32(sm.b[s]);
+                    for (int q = 0; q < 2 * NB; ++q)
+                        tmem_cp_sf(sfb_t + 4 * q, desc_sf(smem_u32(&sm.sfb[s][q * kSfChunk])));
+                    const uint32_t a0 = smem_u32(sm.a[s]), b0 = smem_u32(sm.b[s]);
 #pragma unroll
-                for (int kb = 0; kb < kBK / 64; ++kb) {
-                    // K = 64 per instruction: 32 bytes of each row; scale blocks
-                    // 2kb, 2kb+1 = k-chunk kb/2, bytes 2(kb%2), 2(kb%2)+1 of the
-                    // word; B's scales of the k-chunk span NB x 4 columns
-                    const uint32_t c = kb >> 1, id = (kb & 1) * 2;
-                    mma_mxf4(tmem, desc_sw128(a0 + kb * 32), desc_sw128(b0 + kb * 32),
-                             idesc_mxf4<BN>(id, id), sfa_t + 4 * c, sfb_t + 4 * NB * c,
-                             (kt | kb) != 0);
+                    for (int kb = 0; kb < kBK / 64; ++kb) {
+                        // K = 64 per instruction: 32 bytes of each row; scale
+                        // blocks 2kb, 2kb+1 = k-chunk kb/2, bytes 2(kb%2),
+                        // 2(kb%2)+1 of the word; B's scales of the k-chunk
+                        // span NB x 4 columns
+                        const uint32_t c = kb >> 1, id = (kb & 1) * 2;
+                        mma_mxf4(tmem, desc_sw128(a0 + kb * 32), desc_sw128(b0 + kb * 32),
+                                 idesc_mxf4<BN>(id, id), sfa_t + 4 * c, sfb_t + 4 * NB * c,
+                                 (kt | kb) != 0);
+                    }
+                    umma_commit(&sm.empty[s]);      // frees the stage once these MMAs are done
                 }
-                umma_commit(&sm.empty[s]);          // frees the stage once these MMAs are done
+                umma_commit(&sm.acc_full);          // also after an abort: the epilogue waits on it
             }
-            umma_commit(&sm.acc_full);              // also after an abort: the epilogue waits on it
         }
         __syncwarp();
     } else {
         // ---- epilogue: TMEM lane quadrant = warp % 4 ----
         const int quad = warp & 3;
-        int ok = 1;
-        if (lane == 0) ok = mbar_wait(&sm.acc_full, 0, abort, status) && !*abort;
-        ok = __shfl_sync(0xffffffffu, ok, 0);
-        tc_fence_after();
-        if (ok) {
+        int j = 0;
+        for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++j) {
+            const int m0 = (t / n_tiles) * kBM, n0 = (t % n_tiles) * BN;
+            int ok = 1;
+            if (lane == 0) ok = mbar_wait(&sm.acc_full, j & 1, abort, status) && !*abort;
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) break;
+            tc_fence_after();
             const int64_t row = m0 + quad * 32 + lane;
 #pragma unroll 1
             for (int c0 = 0; c0 < BN; c0 += 32) {
                 float v[32];
                 tmem_ld32(tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)c0, v);
+                if (c0 + 32 == BN) {
+                    // the whole accumulator is in registers or stored: hand
+                    // TMEM back to the MMA warp before the last stores
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0)
+                        asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];"
+                                     :: "r"(smem_u32(&sm.acc_empty)) : "memory");
+                }
                 const float4 *ap = reinterpret_cast<const float4 *>(a_row + n0 + c0);
                 float4 *op = reinterpret_cast<float4 *>(out + row * N + n0 + c0);
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const float4 sc = __ldg(ap + j);
-                    op[j] = make_float4(v[4 * j] * sc.x, v[4 * j + 1] * sc.y, v[4 * j + 2] * sc.z,
-                                        v[4 * j + 3] * sc.w);
+                for (int q = 0; q < 8; ++q) {
+                    const float4 sc = __ldg(ap + q);
+                    op[q] = make_float4(v[4 * q] * sc.x, v[4 * q + 1] * sc.y, v[4 * q + 2] * sc.z,
+                                        v[4 * q + 3] * sc.w);
                 }
             }
         }
@@ -383,9 +416,13 @@ cudaError_t launch_bn(const GemmLaunch &L) {
         if (e != cudaSuccess) return e;
         done[dev] = true;
     }
-    return launch_k(w4a4_gemm_kernel<BN>, dim3((unsigned)(L.N / BN), (unsigned)(L.M / kBM)),
-                    dim3(kThreadsGemm), smem, L.stream, ma, mb, L.scales_x, L.scales_w, L.a, L.out,
-                    (int)L.M, (int)L.N, (int)L.K, L.status);
+    // persistent: one CTA per SM (the shared memory allows one), or fewer tiles
+    int sms = 148;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) sms = 148;
+    const int64_t tiles = (L.M / kBM) * (L.N / BN);
+    const unsigned grid = (unsigned)std::min<int64_t>(tiles, sms);
+    return launch_k(w4a4_gemm_kernel<BN>, dim3(grid), dim3(kThreadsGemm), smem, L.stream, ma, mb,
+                    L.scales_x, L.scales_w, L.a, L.out, (int)L.M, (int)L.N, (int)L.K, L.status);
 }
 
 }  // namespace
