@@ -147,6 +147,21 @@ __device__ __forceinline__ uint32_t idesc_mxf4(uint32_t sfa_id, uint32_t sfb_id)
            ((uint32_t)(kBM >> 4) << 24) | (sfa_id << 29);
 }
 
+// Output tile t -> (m0, n0).  Tiles go in bands of up to kBandTiles tile
+// columns: within a band every row of tiles is visited before the next band,
+// so the CTAs running together share the band's B tiles (which stay in L2)
+// and each A tile is read once per band.
+constexpr int kBandTiles = 16;
+__device__ __forceinline__ void tile_coords(int t, int m_tiles, int n_tiles, int bm, int bn,
+                                            int &m0, int &n0) {
+    const int band = t / (m_tiles * kBandTiles);
+    const int nb0 = band * kBandTiles;
+    const int width = min(kBandTiles, n_tiles - nb0);
+    const int r = t - band * (m_tiles * kBandTiles);
+    m0 = (r / width) * bm;
+    n0 = (nb0 + r % width) * bn;
+}
+
 __device__ __forceinline__ void mma_mxf4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
                                          uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
                                          uint32_t accumulate) {
@@ -215,8 +230,8 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
         (reinterpret_cast<uintptr_t>(gemm_smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int KT = K / kBK;
-    const int n_tiles = N / BN;
-    const int tiles = (M / kBM) * n_tiles;
+    const int n_tiles = N / BN, m_tiles = M / kBM;
+    const int tiles = m_tiles * n_tiles;
     const int64_t sf_row = K / 32;                  // scale bytes per row
     volatile int *abort = &sm.abort;
 
@@ -241,8 +256,8 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
     const uint32_t tmem = sm.tmem_base;             // accumulator: columns [0, BN)
     const uint32_t sfa_t = tmem + BN, sfb_t = tmem + BN + 8;
 
-    // The CTA walks the output tiles t = blockIdx.x, + gridDim.x, ...; tile t
-    // is (t / n_tiles, t % n_tiles), so CTAs running together share A rows.
+    // The CTA walks the output tiles t = blockIdx.x, + gridDim.x, ... in the
+    // band order of tile_coords.
     if (warp == 0) {
         // ---- producer: TMA for the code tiles; the scales by 4-byte cp.async
         // straight into the chunk layout (lane copies rows lane + 32 q: q < 4
@@ -256,7 +271,8 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
         int g = 0;
         bool stop = false;
         for (int t = blockIdx.x; t < tiles && !stop; t += gridDim.x) {
-            const int m0 = (t / n_tiles) * kBM, n0 = (t % n_tiles) * BN;
+            int m0, n0;
+            tile_coords(t, m_tiles, n_tiles, kBM, BN, m0, n0);
             for (int kt = 0; kt < KT; ++kt, ++g) {
                 const int s = g % kStages;
                 if (g >= kStages) {
@@ -335,7 +351,8 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
         const int quad = warp & 3;
         int j = 0;
         for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++j) {
-            const int m0 = (t / n_tiles) * kBM, n0 = (t % n_tiles) * BN;
+            int m0, n0;
+            tile_coords(t, m_tiles, n_tiles, kBM, BN, m0, n0);
             int ok = 1;
             if (lane == 0) ok = mbar_wait(&sm.acc_full, j & 1, abort, status) && !*abort;
             ok = __shfl_sync(0xffffffffu, ok, 0);
