@@ -901,17 +901,21 @@ tile_kernel(const __grid_constant__ Table tab, int mode_slot, int want_res, int6
             }
         }
     };
-    // full groups of 8 rows as straight-line code, then the tail
+    // full groups of GRP rows as straight-line code (8 in the fused mode; 4
+    // in the others, which run 3 CTAs per SM and have fewer registers), then
+    // the tail; a batch of the row statistics ends every 8 rows
+    constexpr int GRP = FUSED ? 8 : 4;
     int k0 = 0;
 #pragma unroll 1
-    for (; k0 + 8 <= nk; k0 += 8) {
+    for (; k0 + GRP <= nk; k0 += GRP) {
 #pragma unroll
-        for (int u = 0; u < 8; ++u) one_row(k0 + u, u, u == 7);
+        for (int u = 0; u < GRP; ++u)
+            one_row(k0 + u, u, ((k0 + u) & 7) == 7 || k0 + u == nk - 1);
     }
 #pragma unroll
-    for (int u = 0; u < 7; ++u) {
+    for (int u = 0; u < GRP - 1; ++u) {
         if (k0 + u >= nk) break;                     // warp-uniform
-        one_row(k0 + u, u, k0 + u == nk - 1);
+        one_row(k0 + u, u, k0 + u == nk - 1 || ((k0 + u) & 7) == 7);
     }
     asm volatile("cp.async.wait_all;" ::: "memory");
     if (FUSED && clamp_risk) atomicOr(&flags[0], 1u);
