@@ -198,3 +198,33 @@ def test_full_size_8b_all_decoders(name):
     assert np.array_equal(gpu_scales_np(gs[ti]), O.encode_scales(s, foa))
     del Ws, outs
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("fmt,T", [("mxfp4", 2), ("int4_bf16", 1)])
+def test_matrix_beyond_int32_elements(fmt, T):
+    # 65536 x 32832 = 2,151,677,952 elements (> 2^31): every flat offset of
+    # the last rows needs 64 bits; sampled rows include the last ones
+    wl = synth.WORKLOADS["llama31_70b_decoder_mxfp4_g32"]
+    rows, cols = 65536, 32832
+    W = synth.weight(wl, 0, 4, device="cuda", rows=rows, cols=cols)
+    assert W.numel() > 2 ** 31
+    fl = dq.format_preset(fmt, 32)
+    fo = O.preset(fmt, 32)
+    o = dq.solve_dual_scale(W, fl, T)
+    torch.cuda.synchronize()
+    assert dq.last_device_status() == 0
+    a, b = np64(o["a"]), np64(o["b"])
+    ri = np.concatenate([_sample(rows, 6, 77), np.arange(rows - 4, rows)])
+    c, s = O.quantize(O.inner(np64(W[ri]), a[ri], b), fo)
+    assert np.array_equal(o["codes"][ri].cpu().numpy(), O.encode_codes(c, fo))
+    assert np.array_equal(gpu_scales_np(o["gscales"][ri]), O.encode_scales(s, fo))
+    # the activation path on a batch of the same size
+    if fmt == "mxfp4":
+        X = W.view(rows, cols)                     # any bf16 [tokens, K] input
+        codes, gs = dq.act_rescale_quant(X, o["b"], fl)
+        torch.cuda.synchronize()
+        ca, sa = O.act_rescale_quant(np64(X[ri]), b, fo)
+        assert np.array_equal(codes[ri].cpu().numpy(), O.encode_codes(ca, fo))
+        assert np.array_equal(gs[ri].cpu().numpy(), O.encode_scales(sa, fo))
+    del W, o
+    torch.cuda.empty_cache()
