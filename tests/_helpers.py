@@ -13,6 +13,9 @@ PRESET_COMBOS = {
     # BF16 outer scales with E8M0 group scales (descriptor variant)
     "mxint4_bf16outer": lambda G: O.Format("int4", G, "e8m0", "bf16"),
     "mxfp4_bf16outer": lambda G: O.Format("e2m1", G, "e8m0", "bf16"),
+    # NVFP4 without the second-level tensor scale (the literal reading: E4M3
+    # group scales of small weights fall into E4M3's subnormal range)
+    "nvfp4_ts1": lambda G: O.Format("e2m1", G, "e4m3", "bf16", tensor_scale_auto=False),
     # the rest of the MX family
     "mxint8": lambda G: O.preset("mxint8", G),
     "mxfp8_e4m3": lambda G: O.preset("mxfp8_e4m3", G),
@@ -42,6 +45,10 @@ def lib_format(name, G):
     if name.endswith("_bf16outer"):
         f = dq.format_preset(name.split("_")[0], G)
         f.outer_scale = 0
+        return f
+    if name == "nvfp4_ts1":
+        f = dq.format_preset("nvfp4", G)
+        f.tensor_scale_auto = 0
         return f
     return dq.format_preset(name, G)
 

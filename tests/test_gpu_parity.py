@@ -24,7 +24,8 @@ dq = pytest.importorskip("dual_scale_solver_b200")
 
 ALL = list(PRESET_COMBOS)
 DEFAULT_G = {"int4_bf16": 64, "mxint4": 32, "mxfp4": 32, "nvfp4": 16,
-             "mxint4_bf16outer": 32, "mxfp4_bf16outer": 32, **{n: 32 for n in MX_MORE}}
+             "mxint4_bf16outer": 32, "mxfp4_bf16outer": 32, "nvfp4_ts1": 16,
+             **{n: 32 for n in MX_MORE}}
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -250,10 +251,10 @@ def test_solve_toy_workload():
     _solve_and_compare([W], fo, fl, wl.T)
 
 
-@pytest.mark.parametrize("name", ["int4_bf16", "nvfp4", "mxfp4"] + MX_MORE)
+@pytest.mark.parametrize("name", ["int4_bf16", "nvfp4", "nvfp4_ts1", "mxfp4"] + MX_MORE)
 def test_solve_single_matrix_entry_point(name):
     G = DEFAULT_G[name]
-    fo, fl = PRESET_COMBOS[name](G), dq.format_preset(name, G)
+    fo, fl = PRESET_COMBOS[name](G), lib_format(name, G)
     W = _weights(200, 1536, torch.bfloat16, key=5)
     o = dq.solve_dual_scale(W.cuda(), fl, 4)
     torch.cuda.synchronize()
