@@ -53,6 +53,8 @@ def _args():
                    help="profiling case: keep only this linear of the decoder")
     p.add_argument("--T", type=int, default=-1, help="profiling case: iterations override")
     p.add_argument("--no-act", action="store_true", help="profiling case: skip activations")
+    p.add_argument("--decoders", type=int, default=-1,
+                   help="profiling case: solve only this many of the workload's decoders")
     p.add_argument("--tokens", type=int, default=32768, help="w4a4_gemm: activation rows")
     p.add_argument("--method", default="dualquant", choices=["dualquant", "two_level", "w4a4_gemm"],
                    help="two_level: the two-level absmax quantization of the same weights "
@@ -257,7 +259,8 @@ def run_ours(args, wl, rank, world, local_rank):
 
     # weak scaling: rank r solves its own block of decoders (seeded per decoder)
     idx = [args.only] if args.only >= 0 else range(len(wl.linears))
-    Ws = [synth.weight(wl, d, i, device=dev) for d in decoders_of(rank, wl.decoders) for i in idx]
+    n_dec = wl.decoders if args.decoders < 0 else min(args.decoders, wl.decoders)
+    Ws = [synth.weight(wl, d, i, device=dev) for d in decoders_of(rank, n_dec) for i in idx]
     fmt = dq.format_preset(wl.fmt, wl.group)
     act = None if args.no_act else wl.act
     X = synth.activation(wl, device=dev) if act else None
@@ -394,8 +397,9 @@ def run_ours(args, wl, rank, world, local_rank):
     if dq.last_device_status() != 0:
         raise RuntimeError("device status flags raised during timing")
 
-    if args.only >= 0 or args.T >= 0 or args.no_act:
-        wl_name = f"{wl.name} (profiling subset: only={args.only} T={T} act={act is not None})"
+    if args.only >= 0 or args.T >= 0 or args.no_act or args.decoders >= 0:
+        wl_name = (f"{wl.name} (profiling subset: only={args.only} T={T} act={act is not None} "
+                   f"decoders={n_dec})")
     else:
         wl_name = wl.name
     line = {
