@@ -413,3 +413,26 @@ def test_batched_mx_solve_equals_single_solves():
         for k in ("codes", "gscales", "a", "b"):
             assert torch.equal(o[k], s[k]), k
         assert torch.equal(o["mse_trace"], s["mse_trace"])
+
+
+@pytest.mark.parametrize("name", ALL)
+def test_dequantize_reconstruction(name):
+    # D_a Qhat D_b from stored codes and scales: c * (s * ts) is exact in
+    # float32 for every code set; the products with a_i and b_j round twice
+    G = DEFAULT_G[name]
+    fo, fl = PRESET_COMBOS[name](G), lib_format(name, G)
+    rows, cols = 37, 8 * G
+    W = _weights(rows, cols, torch.float32, key=40)
+    a = random_outer(fo, rows, synth.stream_key(96, rows))
+    b = random_outer(fo, cols, synth.stream_key(96, cols))
+    ts = 2.0 ** -10 if fo.tensor_scale_auto else 1.0
+    ad = torch.tensor(a, dtype=torch.float32, device="cuda")
+    bd = torch.tensor(b, dtype=torch.float32, device="cuda")
+    codes, gs = dq.quantize(W.cuda(), fl, ad, bd, ts)
+    out = dq.dequantize(codes, gs, rows, cols, fl, ts, ad, bd)
+    torch.cuda.synchronize()
+    c = O.decode_codes(codes.cpu().numpy(), fo)
+    s = O.decode_scales(gpu_scales_np(gs), fo)
+    ref = a[:, None] * O.dequantize(c, s, fo, ts) * b[None, :]
+    got = np64(out)
+    assert np.all(np.abs(got - ref) <= 2.0 ** -22 * np.abs(ref))
