@@ -39,7 +39,6 @@ namespace {
 
 constexpr int kBM = 128;
 constexpr int kBK = 256;                       // K elements per stage (128 bytes per row)
-constexpr int kStages = 4;
 constexpr int kTileBytesA = kBM * kBK / 2;     // 16 KB per A tile
 constexpr int kSfChunk = 512;                  // 128 rows x 4 scales
 constexpr int kThreadsGemm = 192;
@@ -48,6 +47,10 @@ constexpr uint64_t kWaitLimitNs = 1000000000ull;   // a wait gives up after 1 s
 // BN = 128 or 256 output columns per CTA.
 template <int BN>
 struct __align__(1024) GemmSmem {
+    // 128-column tiles run two CTAs per SM (one's epilogue overlaps the
+    // other's MMAs) with a 3-stage ring; 256-column tiles one CTA, 4 stages
+    static constexpr int kCtasPerSm = BN == 128 ? 2 : 1;
+    static constexpr int kStages = BN == 128 ? 3 : 4;
     static constexpr int NB = BN / 128;                        // 128-row blocks of B
     static constexpr int kTileBytesB = BN * kBK / 2;
     static constexpr uint32_t kStageTx = kTileBytesA + kTileBytesB;   // TMA bytes per stage
@@ -218,11 +221,12 @@ __device__ __forceinline__ void mbar_drain(uint64_t *b, uint32_t parity) {
 }
 
 template <int BN>
-__global__ void __launch_bounds__(kThreadsGemm, 1)
+__global__ void __launch_bounds__(kThreadsGemm, GemmSmem<BN>::kCtasPerSm)
 w4a4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                  const uint8_t *sf_a, const uint8_t *sf_b, const float *a_row, float *out, int M,
                  int N, int K, unsigned int *status) {
     using Smem = GemmSmem<BN>;
+    constexpr int kStages = Smem::kStages;
     constexpr int NB = Smem::NB;
     grid_dependency_begin();
     extern __shared__ uint8_t gemm_smem_raw[];
@@ -437,7 +441,7 @@ cudaError_t launch_bn(const GemmLaunch &L) {
     int sms = 148;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) sms = 148;
     const int64_t tiles = (L.M / kBM) * (L.N / BN);
-    const unsigned grid = (unsigned)std::min<int64_t>(tiles, sms);
+    const unsigned grid = (unsigned)std::min<int64_t>(tiles, (int64_t)sms * GemmSmem<BN>::kCtasPerSm);
     return launch_k(w4a4_gemm_kernel<BN>, dim3(grid), dim3(kThreadsGemm), smem, L.stream, ma, mb,
                     L.scales_x, L.scales_w, L.a, L.out, (int)L.M, (int)L.N, (int)L.K, L.status);
 }

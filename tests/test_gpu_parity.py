@@ -436,3 +436,23 @@ def test_dequantize_reconstruction(name):
     ref = a[:, None] * O.dequantize(c, s, fo, ts) * b[None, :]
     got = np64(out)
     assert np.all(np.abs(got - ref) <= 2.0 ** -22 * np.abs(ref))
+
+
+def test_measurement_support():
+    # event timing of selected tile-kernel kinds and the launch counter
+    fl = dq.format_preset("mxfp4")
+    W = _weights(256, 1024, torch.bfloat16, key=41).cuda()
+    dq.solve_dual_scale(W, fl, 2)                # warm
+    torch.cuda.synchronize()
+    for k in range(5):
+        dq.kernel_time(k)
+    n0 = dq.launch_count()
+    dq.kernel_timing(True, kinds=[dq.KIND_FUSED])
+    dq.solve_dual_scale(W, fl, 3)
+    torch.cuda.synchronize()
+    ms, n = dq.kernel_time(dq.KIND_FUSED)
+    ms_pack, n_pack = dq.kernel_time(dq.KIND_PACK)
+    dq.kernel_timing(False)
+    assert n == 3 and ms > 0.0                   # one fused pass per iteration
+    assert n_pack == 0                            # kinds not selected are not timed
+    assert dq.launch_count() - n0 >= 3 * 5 + 1    # per iteration: fused, 2 gated, 2 finalize, mse
