@@ -38,29 +38,32 @@ namespace dq {
 namespace {
 
 constexpr int kBM = 128;
-constexpr int kBK = 256;                       // K elements per stage (128 bytes per row)
-constexpr int kTileBytesA = kBM * kBK / 2;     // 16 KB per A tile
 constexpr int kSfChunk = 512;                  // 128 rows x 4 scales
 constexpr int kThreadsGemm = 192;
 constexpr uint64_t kWaitLimitNs = 1000000000ull;   // a wait gives up after 1 s
 
-// BN = 128 or 256 output columns per CTA.
-template <int BN>
+// BN = 128 or 256 output columns per CTA; BK = 128 or 256 K elements per
+// stage (64- or 128-byte rows, 64- or 128-byte swizzle).
+template <int BN, int BK>
 struct __align__(1024) GemmSmem {
     // 128-column tiles run two CTAs per SM (one's epilogue overlaps the
-    // other's MMAs) with a 3-stage ring; 256-column tiles one CTA, 4 stages
+    // other's MMAs); the ring depth fills the shared memory
     static constexpr int kCtasPerSm = BN == 128 ? 2 : 1;
-    static constexpr int kStages = BN == 128 ? 3 : 4;
     static constexpr int NB = BN / 128;                        // 128-row blocks of B
-    static constexpr int kTileBytesB = BN * kBK / 2;
+    static constexpr int KC = BK / 128;                        // 4-scale chunks per row and stage
+    static constexpr int kRowBytes = BK / 2;
+    static constexpr int kTileBytesA = kBM * kRowBytes;
+    static constexpr int kTileBytesB = BN * kRowBytes;
+    static constexpr int kStageBytes = kTileBytesA + kTileBytesB + (1 + NB) * KC * kSfChunk;
+    static constexpr int kStages = (kCtasPerSm == 2 ? 102 * 1024 : 204 * 1024) / kStageBytes;
     static constexpr uint32_t kStageTx = kTileBytesA + kTileBytesB;   // TMA bytes per stage
-    // TMEM: accumulator BN columns, then A's scales (2 chunks x 4 columns),
-    // then B's (2 k-chunks x NB row blocks x 4 columns)
+    // TMEM: accumulator BN columns, then A's scales (KC chunks x 4 columns),
+    // then B's (KC k-chunks x NB row blocks x 4 columns)
     static constexpr uint32_t kTmemCols = BN == 128 ? 256 : 512;
     uint8_t a[kStages][kTileBytesA];
     uint8_t b[kStages][kTileBytesB];
-    uint8_t sfa[kStages][2 * kSfChunk];            // [k-chunk][512]
-    uint8_t sfb[kStages][2 * NB * kSfChunk];       // [k-chunk][row block][512]
+    uint8_t sfa[kStages][KC * kSfChunk];            // [k-chunk][512]
+    uint8_t sfb[kStages][KC * NB * kSfChunk];       // [k-chunk][row block][512]
     uint64_t full[kStages];
     uint64_t empty[kStages];
     uint64_t acc_full;      // MMA -> epilogue: the tile's accumulator is complete
@@ -129,11 +132,14 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, i
         : "memory");
 }
 
-// UMMA shared-memory descriptor, K-major, 128-byte swizzle: rows of 128
-// bytes, 8-row atoms 1024 bytes apart (stride byte offset), version 1.
-__device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr) {
-    return (uint64_t)((saddr & 0x3FFFFu) >> 4) | (1ull << 16) | (64ull << 32) | (1ull << 46) |
-           (2ull << 61);
+// UMMA shared-memory descriptor, K-major, ROWB-byte swizzle (128 or 64):
+// rows of ROWB bytes, 8-row atoms 8 * ROWB bytes apart (stride byte
+// offset), version 1; layout type 2 = 128-byte swizzle, 4 = 64-byte.
+template <int ROWB>
+__device__ __forceinline__ uint64_t desc_swz(uint32_t saddr) {
+    constexpr uint64_t kLayout = ROWB == 128 ? 2ull : 4ull;
+    return (uint64_t)((saddr & 0x3FFFFu) >> 4) | (1ull << 16) | ((uint64_t)(8 * ROWB / 16) << 32) |
+           (1ull << 46) | (kLayout << 61);
 }
 
 // Descriptor of one 512-byte scale chunk for tcgen05.cp 32x128b: 32 rows of
@@ -220,20 +226,21 @@ __device__ __forceinline__ void mbar_drain(uint64_t *b, uint32_t parity) {
     }
 }
 
-template <int BN>
-__global__ void __launch_bounds__(kThreadsGemm, GemmSmem<BN>::kCtasPerSm)
+template <int BN, int BK>
+__global__ void __launch_bounds__(kThreadsGemm, GemmSmem<BN, BK>::kCtasPerSm)
 w4a4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                  const uint8_t *sf_a, const uint8_t *sf_b, const float *a_row, float *out, int M,
                  int N, int K, unsigned int *status) {
-    using Smem = GemmSmem<BN>;
+    using Smem = GemmSmem<BN, BK>;
     constexpr int kStages = Smem::kStages;
+    constexpr int KC = Smem::KC;
     constexpr int NB = Smem::NB;
     grid_dependency_begin();
     extern __shared__ uint8_t gemm_smem_raw[];
     Smem &sm = *reinterpret_cast<Smem *>(
         (reinterpret_cast<uintptr_t>(gemm_smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int KT = K / kBK;
+    const int KT = K / BK;
     const int n_tiles = N / BN, m_tiles = M / kBM;
     const int tiles = m_tiles * n_tiles;
     const int64_t sf_row = K / 32;                  // scale bytes per row
@@ -258,7 +265,7 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;             // accumulator: columns [0, BN)
-    const uint32_t sfa_t = tmem + BN, sfb_t = tmem + BN + 8;
+    const uint32_t sfa_t = tmem + BN, sfb_t = tmem + BN + 4 * KC;
 
     // The CTA walks the output tiles t = blockIdx.x, + gridDim.x, ... in the
     // band order of tile_coords.
@@ -286,21 +293,23 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
                 }
                 if (lane == 0) {
                     mbar_arrive_expect_tx(&sm.full[s], Smem::kStageTx);
-                    tma_load_2d(sm.a[s], &map_a, kt * (kBK / 2), m0, &sm.full[s]);
-                    tma_load_2d(sm.b[s], &map_b, kt * (kBK / 2), n0, &sm.full[s]);
+                    tma_load_2d(sm.a[s], &map_a, kt * (BK / 2), m0, &sm.full[s]);
+                    tma_load_2d(sm.b[s], &map_b, kt * (BK / 2), n0, &sm.full[s]);
                 }
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
-                    const uint8_t *src = sf_a + (int64_t)(m0 + lane + 32 * q) * sf_row + kt * 8;
-                    cp_async4(&sm.sfa[s][lane * 16 + q * 4], src);
-                    cp_async4(&sm.sfa[s][kSfChunk + lane * 16 + q * 4], src + 4);
+                    const uint8_t *src = sf_a + (int64_t)(m0 + lane + 32 * q) * sf_row + kt * (BK / 32);
+#pragma unroll
+                    for (int kc = 0; kc < KC; ++kc)
+                        cp_async4(&sm.sfa[s][kc * kSfChunk + lane * 16 + q * 4], src + 4 * kc);
                 }
 #pragma unroll
                 for (int q = 0; q < 4 * NB; ++q) {
-                    const uint8_t *src = sf_b + (int64_t)(n0 + lane + 32 * q) * sf_row + kt * 8;
+                    const uint8_t *src = sf_b + (int64_t)(n0 + lane + 32 * q) * sf_row + kt * (BK / 32);
                     const int nb = q >> 2, qq = q & 3;
-                    cp_async4(&sm.sfb[s][nb * kSfChunk + lane * 16 + qq * 4], src);
-                    cp_async4(&sm.sfb[s][(NB + nb) * kSfChunk + lane * 16 + qq * 4], src + 4);
+#pragma unroll
+                    for (int kc = 0; kc < KC; ++kc)
+                        cp_async4(&sm.sfb[s][(kc * NB + nb) * kSfChunk + lane * 16 + qq * 4], src + 4 * kc);
                 }
                 asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];"
                              :: "r"(smem_u32(&sm.full[s])) : "memory");
@@ -327,20 +336,21 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
                     // reads them through the async proxy
                     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                     tc_fence_after();
-                    tmem_cp_sf(sfa_t, desc_sf(smem_u32(&sm.sfa[s][0])));
-                    tmem_cp_sf(sfa_t + 4, desc_sf(smem_u32(&sm.sfa[s][kSfChunk])));
 #pragma unroll
-                    for (int q = 0; q < 2 * NB; ++q)
+                    for (int kc = 0; kc < KC; ++kc)
+                        tmem_cp_sf(sfa_t + 4 * kc, desc_sf(smem_u32(&sm.sfa[s][kc * kSfChunk])));
+#pragma unroll
+                    for (int q = 0; q < KC * NB; ++q)
                         tmem_cp_sf(sfb_t + 4 * q, desc_sf(smem_u32(&sm.sfb[s][q * kSfChunk])));
                     const uint32_t a0 = smem_u32(sm.a[s]), b0 = smem_u32(sm.b[s]);
 #pragma unroll
-                    for (int kb = 0; kb < kBK / 64; ++kb) {
+                    for (int kb = 0; kb < BK / 64; ++kb) {
                         // K = 64 per instruction: 32 bytes of each row; scale
                         // blocks 2kb, 2kb+1 = k-chunk kb/2, bytes 2(kb%2),
                         // 2(kb%2)+1 of the word; B's scales of the k-chunk
                         // span NB x 4 columns
                         const uint32_t c = kb >> 1, id = (kb & 1) * 2;
-                        mma_mxf4(tmem, desc_sw128(a0 + kb * 32), desc_sw128(b0 + kb * 32),
+                        mma_mxf4(tmem, desc_swz<BK / 2>(a0 + kb * 32), desc_swz<BK / 2>(b0 + kb * 32),
                                  idesc_mxf4<BN>(id, id), sfa_t + 4 * c, sfb_t + 4 * NB * c,
                                  (kt | kb) != 0);
                     }
@@ -408,51 +418,56 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
     return fn;
 }
 
-// 2-D map over a [rows, K/2]-byte code matrix: boxes of box_rows x 128 bytes,
-// 128-byte swizzle.
-bool code_map(CUtensorMap *m, const uint8_t *codes, int64_t rows, int64_t K, int box_rows) {
+// 2-D map over a [rows, K/2]-byte code matrix: boxes of box_rows x row_bytes,
+// swizzled by row_bytes (128 or 64).
+bool code_map(CUtensorMap *m, const uint8_t *codes, int64_t rows, int64_t K, int box_rows,
+              int row_bytes) {
     auto enc = tensor_map_encoder();
     if (!enc) return false;
     const cuuint64_t dims[2] = {(cuuint64_t)(K / 2), (cuuint64_t)rows};
     const cuuint64_t strides[1] = {(cuuint64_t)(K / 2)};
-    const cuuint32_t box[2] = {(cuuint32_t)(kBK / 2), (cuuint32_t)box_rows};
+    const cuuint32_t box[2] = {(cuuint32_t)row_bytes, (cuuint32_t)box_rows};
     const cuuint32_t estr[2] = {1, 1};
+    const CUtensorMapSwizzle swz = row_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(codes), dims, strides,
-               box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+               box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int BN>
+template <int BN, int BK>
 cudaError_t launch_bn(const GemmLaunch &L) {
+    using Smem = GemmSmem<BN, BK>;
     CUtensorMap ma, mb;
-    if (!code_map(&ma, L.codes_x, L.M, L.K, kBM) || !code_map(&mb, L.codes_w, L.N, L.K, BN))
+    if (!code_map(&ma, L.codes_x, L.M, L.K, kBM, BK / 2) || !code_map(&mb, L.codes_w, L.N, L.K, BN, BK / 2))
         return cudaErrorInvalidValue;
-    const size_t smem = sizeof(GemmSmem<BN>) + 1024;
+    const size_t smem = sizeof(Smem) + 1024;
     static bool done[64] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     if (!done[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(w4a4_gemm_kernel<BN>,
+        cudaError_t e = cudaFuncSetAttribute(w4a4_gemm_kernel<BN, BK>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
         done[dev] = true;
     }
-    // persistent: one CTA per SM (the shared memory allows one), or fewer tiles
+    // persistent: kCtasPerSm CTAs per SM, or fewer tiles
     int sms = 148;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) sms = 148;
     const int64_t tiles = (L.M / kBM) * (L.N / BN);
-    const unsigned grid = (unsigned)std::min<int64_t>(tiles, (int64_t)sms * GemmSmem<BN>::kCtasPerSm);
-    return launch_k(w4a4_gemm_kernel<BN>, dim3(grid), dim3(kThreadsGemm), smem, L.stream, ma, mb,
+    const unsigned grid = (unsigned)std::min<int64_t>(tiles, (int64_t)sms * Smem::kCtasPerSm);
+    return launch_k(w4a4_gemm_kernel<BN, BK>, dim3(grid), dim3(kThreadsGemm), smem, L.stream, ma, mb,
                     L.scales_x, L.scales_w, L.a, L.out, (int)L.M, (int)L.N, (int)L.K, L.status);
 }
 
 }  // namespace
 
+constexpr int kGemmBK = 256;
+
 // 256 output columns per CTA when N allows it (A tiles reused twice as
 // often), else 128.
 cudaError_t launch_w4a4_gemm(const GemmLaunch &L) {
     if (L.M == 0 || L.N == 0) return cudaSuccess;
-    return (L.N % 256 == 0) ? launch_bn<256>(L) : launch_bn<128>(L);
+    return (L.N % 256 == 0) ? launch_bn<256, kGemmBK>(L) : launch_bn<128, kGemmBK>(L);
 }
 
 }  // namespace dq
