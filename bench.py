@@ -553,11 +553,15 @@ def run_gemm(args, wl, rank, world, local_rank):
     res = [torch.empty(M, W.shape[0], dtype=torch.float32, device=dev) for W in Ws]
     del Ws
     stream = torch.cuda.current_stream(dev)
+    # the GEMM reads E8M0 scales as scale tiles: the weights' once after the
+    # solve, the activation batches' once per batch
+    wtiles = [dq.scale_tiles(o["gscales"]) for o in outs]
+    acts = {K: (cx, dq.scale_tiles(sx)) for K, (cx, sx) in acts.items()}
 
     def step():
-        for o, r in zip(outs, res):
+        for o, r, sw in zip(outs, res, wtiles):
             cx, sx = acts[2 * o["codes"].shape[1]]
-            dq.w4a4_gemm(cx, sx, o["codes"], o["gscales"], o["a"], fmt, out=r)
+            dq.w4a4_gemm(cx, sx, o["codes"], sw, o["a"], fmt, out=r, tiled=True)
 
     for _ in range(args.warmup):
         step()

@@ -18,7 +18,7 @@ __all__ = [
     "workspace_size", "quantize", "dequantize", "solve_dual_scale", "solve_dual_scale_batched",
     "row_update", "col_update", "act_rescale_quant", "last_device_status", "EXPORTS",
     "kernel_timing", "kernel_time", "launch_count", "solve_dual_scale_noalloc", "code_bytes",
-    "two_level_quant", "w4a4_gemm",
+    "two_level_quant", "w4a4_gemm", "scale_tiles",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -34,7 +34,8 @@ EXPORTS = ("dq_version", "dq_strerror", "dq_format_preset", "dq_workspace_size",
            "dq_dequantize", "dq_solve_dual_scale", "dq_solve_dual_scale_batched",
            "dq_row_update", "dq_col_update", "dq_act_rescale_quant", "dq_last_device_status",
            "dq_kernel_timing", "dq_kernel_time", "dq_launch_count",
-           "dq_solve_dual_scale_noalloc", "dq_code_bytes", "dq_two_level_quant", "dq_w4a4_gemm")
+           "dq_solve_dual_scale_noalloc", "dq_code_bytes", "dq_two_level_quant", "dq_w4a4_gemm",
+           "dq_scale_tiles")
 
 
 class DqError(RuntimeError):
@@ -106,6 +107,7 @@ def lib() -> ctypes.CDLL:
         "dq_code_bytes": (c_int64, [P(dq_format), c_int64, c_int64]),
         "dq_w4a4_gemm": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int64,
                                    c_int64, c_int64, P(dq_format), c_void_p, c_void_p]),
+        "dq_scale_tiles": (c_int32, [c_void_p, c_int64, c_int64, c_void_p, c_void_p]),
         "dq_two_level_quant": (c_int32, [c_void_p, c_int32, c_int64, c_int64, c_int32,
                                          P(dq_format), c_void_p, c_void_p, c_void_p, c_void_p,
                                          c_void_p]),
@@ -368,12 +370,30 @@ def two_level_quant(X, dual_block=512, inner=None, qdq=True, stream=None):
     return codes, isc, osc, out
 
 
-def w4a4_gemm(codes_x, scales_x, codes_w, scales_w, a, fmt=None, out=None, stream=None):
+def scale_tiles(scales, K=None, out=None, stream=None):
+    """Row-major E8M0 scales [rows, K/32] -> the scale tiles dq_w4a4_gemm
+    reads (rows * K / 32 bytes, uint8)."""
+    _need_cuda(scales)
+    rows = scales.shape[0]
+    K = 32 * scales.shape[1] if K is None else K
+    if out is None:
+        out = torch.empty(rows * K // 32, dtype=torch.uint8, device=scales.device)
+    _check(lib().dq_scale_tiles(_ptr(scales), rows, K, _ptr(out), _stream(stream)), "dq_scale_tiles")
+    return out
+
+
+def w4a4_gemm(codes_x, scales_x, codes_w, scales_w, a, fmt=None, out=None, stream=None,
+              tiled=False):
     """out[M, N] = a_n * sum_k Qx[m, k] Qw[n, k] (float32) from MXFP4 codes and
-    E8M0 scales of the activations (M rows) and the weights (N rows)."""
+    E8M0 scales of the activations (M rows) and the weights (N rows).  The
+    scales are row-major [rows, K/32] (tiled=False: rewritten into scale tiles
+    first, one extra launch each) or already scale tiles (tiled=True)."""
     _need_cuda(codes_x, scales_x, codes_w, scales_w, a)
     fmt = format_preset("mxfp4") if fmt is None else fmt
     M, N, K = codes_x.shape[0], codes_w.shape[0], 2 * codes_x.shape[1]
+    if not tiled:
+        scales_x = scale_tiles(scales_x, K, stream=stream)
+        scales_w = scale_tiles(scales_w, K, stream=stream)
     if out is None:
         out = torch.empty(M, N, dtype=torch.float32, device=codes_x.device)
     _check(lib().dq_w4a4_gemm(_ptr(codes_x), _ptr(scales_x), _ptr(codes_w), _ptr(scales_w),

@@ -791,6 +791,18 @@ dq_status dq_w4a4_gemm(const uint8_t *codes_x, const void *scales_x, const uint8
     return DQ_OK;
 }
 
+dq_status dq_scale_tiles(const void *scales, int64_t rows, int64_t K, uint8_t *tiles,
+                         dq_stream stream) {
+    if (rows < 0 || K < 0 || rows % 128 || K % 128) return DQ_ERR_SHAPE;
+    if (rows == 0 || K == 0) return DQ_OK;
+    if (!scales || !tiles) return DQ_ERR_ARG;
+    if (!aligned(scales, 16) || !aligned(tiles, 16)) return DQ_ERR_ALIGN;
+    DQ_CUDA(launch_scale_tiles(static_cast<const uint8_t *>(scales), rows, K, tiles,
+                               reinterpret_cast<cudaStream_t>(stream)));
+    count_launches(1);
+    return DQ_OK;
+}
+
 dq_status dq_dequantize(const uint8_t *codes, const void *gscales, int64_t rows, int64_t cols,
                         const dq_format *fmt, float tensor_scale, const float *a, const float *b,
                         float *out, dq_stream stream) {

@@ -9,7 +9,10 @@
 // Qx = the MXFP4 codes and E8M0 group scales of Q(X D_b) (dq_act_rescale_quant),
 // Qw = the MXFP4 codes and E8M0 group scales of Q(W / (a b^T)) (the solve), a =
 // the outer row scales of W.  Both operands are K-major E2M1, two codes per
-// byte, with one E8M0 scale per 32 elements of K.
+// byte, with one E8M0 scale per 32 elements of K; the scales come in scale
+// tiles, the layout the tensor core reads (scale_tiles_kernel below): per
+// 128-row block and 128 elements of K one 512-byte chunk holding the scale
+// k (0..3) of row r at byte (r % 32) * 16 + (r / 32) * 4 + k.
 //
 // A persistent CTA per SM walks 128 x BN tiles of `out` (BN = 256, or 128
 // when N is not a multiple of 256) with tcgen05.mma kind::mxf4 (M = 128,
@@ -18,12 +21,11 @@
 // bytes per row) through a 4-stage shared-memory ring that runs on across
 // output tiles:
 //   warp 0     producer: TMA loads of the A and B tiles (128-byte swizzle,
-//              no multicast) and 4-byte cp.async copies of the two operands'
-//              scale factors from their row-major arrays into the 128-row x
-//              4-scale chunk layout the tensor core reads;
+//              no multicast) and bulk copies of their scale tiles;
 //   warp 1     TMEM allocation; lane 0 issues tcgen05.cp (scales to TMEM),
 //              the MMAs and the tcgen05.commit arrivals;
-//   warps 2-5  epilogue: TMEM -> registers (tcgen05.ld), times a_n, stores.
+//   warps 2-5  epilogue: TMEM -> registers (tcgen05.ld) -> shared memory ->
+//              row-contiguous float32 stores, times a_n.
 // Every wait on an mbarrier is bounded: a wait that runs out raises a device
 // status bit, the CTA stops issuing work, waits (bounded) for its copies in
 // flight, frees its TMEM and returns.
@@ -55,15 +57,22 @@ struct __align__(1024) GemmSmem {
     static constexpr int kTileBytesA = kBM * kRowBytes;
     static constexpr int kTileBytesB = BN * kRowBytes;
     static constexpr int kStageBytes = kTileBytesA + kTileBytesB + (1 + NB) * KC * kSfChunk;
-    static constexpr int kStages = (kCtasPerSm == 2 ? 102 * 1024 : 204 * 1024) / kStageBytes;
-    static constexpr uint32_t kStageTx = kTileBytesA + kTileBytesB;   // TMA bytes per stage
+    // epilogue staging: per epilogue warp 32 rows x EC float32 columns,
+    // 16-byte chunks swizzled so that a row-per-lane write and a
+    // row-contiguous read are both free of bank conflicts
+    static constexpr int EC = BN == 128 ? 16 : 32;
+    static constexpr int kStgBytes = 4 * 32 * EC * 4;
+    static constexpr int kStages =
+        ((kCtasPerSm == 2 ? 112 * 1024 : 226 * 1024) - kStgBytes - 1024) / kStageBytes;
+    static constexpr uint32_t kStageTx = kStageBytes;      // bytes that land per stage
     // TMEM: accumulator BN columns, then A's scales (KC chunks x 4 columns),
     // then B's (KC k-chunks x NB row blocks x 4 columns)
     static constexpr uint32_t kTmemCols = BN == 128 ? 256 : 512;
     uint8_t a[kStages][kTileBytesA];
     uint8_t b[kStages][kTileBytesB];
     uint8_t sfa[kStages][KC * kSfChunk];            // [k-chunk][512]
-    uint8_t sfb[kStages][KC * NB * kSfChunk];       // [k-chunk][row block][512]
+    uint8_t sfb[kStages][NB * KC * kSfChunk];       // [row block][k-chunk][512]
+    float4 stg[4][32 * EC / 4];
     uint64_t full[kStages];
     uint64_t empty[kStages];
     uint64_t acc_full;      // MMA -> epilogue: the tile's accumulator is complete
@@ -117,9 +126,13 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *b, uint32_t parity, volatile
     return false;
 }
 
-__device__ __forceinline__ void cp_async4(void *dst, const void *src) {
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" :: "r"(smem_u32(dst)), "l"(src)
-                 : "memory");
+// Untiled bulk copy global -> shared (no multicast), completion counted in
+// bytes on the mbarrier; both addresses 16-byte aligned, size a multiple of 16.
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        :: "r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
 }
 
 __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y,
@@ -243,12 +256,11 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
     const int KT = K / BK;
     const int n_tiles = N / BN, m_tiles = M / kBM;
     const int tiles = m_tiles * n_tiles;
-    const int64_t sf_row = K / 32;                  // scale bytes per row
     volatile int *abort = &sm.abort;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
-            mbar_init(&sm.full[s], 33);             // the TMA arrival + 32 lanes' scale copies
+            mbar_init(&sm.full[s], 1);              // the producer's arrival (+ the stage's bytes)
             mbar_init(&sm.empty[s], 1);
         }
         mbar_init(&sm.acc_full, 1);
@@ -270,17 +282,15 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
     // The CTA walks the output tiles t = blockIdx.x, + gridDim.x, ... in the
     // band order of tile_coords.
     if (warp == 0) {
-        // ---- producer: TMA for the code tiles; the scales by 4-byte cp.async
-        // straight into the chunk layout (lane copies rows lane + 32 q: q < 4
-        // of A, q < 4 NB of B; chunk kc holds scales 4kc..4kc+3 of each row,
-        // row r of a 128-row block at byte (r%32)*16 + (r/32)*4).  Each lane's
-        // cp.async.mbarrier.arrive fires once its copies have landed, so the
-        // stage's barrier completes with the TMA bytes and 32 such arrivals.
-        // The ring runs on across tiles (g counts K tiles of all the CTA's
-        // output tiles), so the next tile's operands arrive during the
-        // current tile's last MMAs and epilogue. ----
+        // ---- producer (lane 0): per K tile, TMA loads of the two code tiles
+        // and bulk copies of their scale tiles (KC consecutive 512-byte
+        // chunks per 128-row block), all counted in bytes on the stage's
+        // barrier.  The ring runs on across tiles (g counts K tiles of all
+        // the CTA's output tiles), so the next tile's operands arrive during
+        // the current tile's last MMAs and epilogue. ----
         int g = 0;
         bool stop = false;
+        const int64_t kblocks = K / 128;             // scale chunks per 128-row block
         for (int t = blockIdx.x; t < tiles && !stop; t += gridDim.x) {
             int m0, n0;
             tile_coords(t, m_tiles, n_tiles, kBM, BN, m0, n0);
@@ -295,24 +305,14 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
                     mbar_arrive_expect_tx(&sm.full[s], Smem::kStageTx);
                     tma_load_2d(sm.a[s], &map_a, kt * (BK / 2), m0, &sm.full[s]);
                     tma_load_2d(sm.b[s], &map_b, kt * (BK / 2), n0, &sm.full[s]);
+                    bulk_load(sm.sfa[s], sf_a + ((m0 / 128) * kblocks + (int64_t)kt * KC) * kSfChunk,
+                              KC * kSfChunk, &sm.full[s]);
+#pragma unroll
+                    for (int nb = 0; nb < NB; ++nb)
+                        bulk_load(sm.sfb[s] + nb * KC * kSfChunk,
+                                  sf_b + ((n0 / 128 + nb) * kblocks + (int64_t)kt * KC) * kSfChunk,
+                                  KC * kSfChunk, &sm.full[s]);
                 }
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const uint8_t *src = sf_a + (int64_t)(m0 + lane + 32 * q) * sf_row + kt * (BK / 32);
-#pragma unroll
-                    for (int kc = 0; kc < KC; ++kc)
-                        cp_async4(&sm.sfa[s][kc * kSfChunk + lane * 16 + q * 4], src + 4 * kc);
-                }
-#pragma unroll
-                for (int q = 0; q < 4 * NB; ++q) {
-                    const uint8_t *src = sf_b + (int64_t)(n0 + lane + 32 * q) * sf_row + kt * (BK / 32);
-                    const int nb = q >> 2, qq = q & 3;
-#pragma unroll
-                    for (int kc = 0; kc < KC; ++kc)
-                        cp_async4(&sm.sfb[s][(kc * NB + nb) * kSfChunk + lane * 16 + qq * 4], src + 4 * kc);
-                }
-                asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];"
-                             :: "r"(smem_u32(&sm.full[s])) : "memory");
             }
         }
         // after an abort, let the copies already issued land before the CTA exits
@@ -332,16 +332,14 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
                 for (int kt = 0; kt < KT; ++kt, ++g) {
                     const int s = g % kStages;
                     if (!mbar_wait(&sm.full[s], (g / kStages) & 1, abort, status)) { stop = true; break; }
-                    // the scales came through the generic proxy; tcgen05.cp
-                    // reads them through the async proxy
-                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                     tc_fence_after();
 #pragma unroll
                     for (int kc = 0; kc < KC; ++kc)
                         tmem_cp_sf(sfa_t + 4 * kc, desc_sf(smem_u32(&sm.sfa[s][kc * kSfChunk])));
 #pragma unroll
-                    for (int q = 0; q < KC * NB; ++q)
-                        tmem_cp_sf(sfb_t + 4 * q, desc_sf(smem_u32(&sm.sfb[s][q * kSfChunk])));
+                    for (int q = 0; q < KC * NB; ++q)     // TMEM: [k-chunk][row block]
+                        tmem_cp_sf(sfb_t + 4 * q,
+                                   desc_sf(smem_u32(&sm.sfb[s][((q % NB) * KC + q / NB) * kSfChunk])));
                     const uint32_t a0 = smem_u32(sm.a[s]), b0 = smem_u32(sm.b[s]);
 #pragma unroll
                     for (int kb = 0; kb < BK / 64; ++kb) {
@@ -361,8 +359,20 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
         }
         __syncwarp();
     } else {
-        // ---- epilogue: TMEM lane quadrant = warp % 4 ----
+        // ---- epilogue: TMEM lane quadrant = warp % 4.  Each 32-column slice
+        // of the warp's 32 accumulator rows goes TMEM -> registers (lane =
+        // row) -> the warp's staging block in shared memory (EC columns at a
+        // time) -> global memory with each store instruction covering whole
+        // row segments (CPR lanes per row), times a_n. ----
+        constexpr int EC = Smem::EC;
+        constexpr int CPR = EC / 4;                  // 16-byte chunks per staged row
+        constexpr int RPP = 32 / CPR;                // rows per store instruction
         const int quad = warp & 3;
+        float4 *stg = sm.stg[quad];
+        // chunk c of row r sits at chunk c ^ sw(r) of the row: 8 consecutive
+        // rows then cover all eight 16-byte bank groups
+        auto sw = [](int r) { return (r / (8 / CPR)) % CPR; };
+        const int rr = lane / CPR, cc = lane % CPR;  // this lane's row / chunk in the store pass
         int j = 0;
         for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++j) {
             int m0, n0;
@@ -372,27 +382,38 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok) break;
             tc_fence_after();
-            const int64_t row = m0 + quad * 32 + lane;
+            float *const orow = out + (int64_t)(m0 + quad * 32) * N + n0;
 #pragma unroll 1
             for (int c0 = 0; c0 < BN; c0 += 32) {
                 float v[32];
                 tmem_ld32(tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)c0, v);
                 if (c0 + 32 == BN) {
-                    // the whole accumulator is in registers or stored: hand
-                    // TMEM back to the MMA warp before the last stores
+                    // the whole accumulator has been read: hand TMEM back to
+                    // the MMA warp before the last stores
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0)
                         asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];"
                                      :: "r"(smem_u32(&sm.acc_empty)) : "memory");
                 }
-                const float4 *ap = reinterpret_cast<const float4 *>(a_row + n0 + c0);
-                float4 *op = reinterpret_cast<float4 *>(out + row * N + n0 + c0);
 #pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    const float4 sc = __ldg(ap + q);
-                    op[q] = make_float4(v[4 * q] * sc.x, v[4 * q + 1] * sc.y, v[4 * q + 2] * sc.z,
-                                        v[4 * q + 3] * sc.w);
+                for (int h = 0; h < 32 / EC; ++h) {
+#pragma unroll
+                    for (int c = 0; c < CPR; ++c)
+                        stg[lane * CPR + (c ^ sw(lane))] =
+                            make_float4(v[h * EC + 4 * c], v[h * EC + 4 * c + 1],
+                                        v[h * EC + 4 * c + 2], v[h * EC + 4 * c + 3]);
+                    __syncwarp();
+                    const int col = c0 + h * EC + 4 * cc;
+                    const float4 sc = __ldg(reinterpret_cast<const float4 *>(a_row + n0 + col));
+#pragma unroll
+                    for (int p = 0; p < CPR; ++p) {
+                        const int r = p * RPP + rr;
+                        const float4 x = stg[r * CPR + (cc ^ sw(r))];
+                        *reinterpret_cast<float4 *>(orow + (int64_t)r * N + col) =
+                            make_float4(x.x * sc.x, x.y * sc.y, x.z * sc.z, x.w * sc.w);
+                    }
+                    __syncwarp();
                 }
             }
         }
@@ -403,6 +424,23 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;"
                      :: "r"(tmem), "r"(Smem::kTmemCols) : "memory");
+    }
+}
+
+// Row-major E8M0 scales [rows, K/32] -> scale tiles: one thread per 4-byte
+// word (the 4 scales of one row in one 128-element K block); word w of chunk
+// (rb, kc) holds row rb*128 + (w % 4)*32 + w/4, so the writes are coalesced.
+__global__ void __launch_bounds__(256)
+scale_tiles_kernel(const uint8_t *scales, int64_t words, int64_t kblocks, uint8_t *tiles) {
+    grid_dependency_begin();
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < words;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t chunk = i >> 7;
+        const int w = (int)(i & 127);
+        const int64_t rb = chunk / kblocks, kc = chunk % kblocks;
+        const int64_t r = rb * 128 + (w & 3) * 32 + (w >> 2);
+        const uint32_t v = __ldg(reinterpret_cast<const uint32_t *>(scales + r * (kblocks * 4) + kc * 4));
+        reinterpret_cast<uint32_t *>(tiles)[i] = v;
     }
 }
 
@@ -437,6 +475,8 @@ bool code_map(CUtensorMap *m, const uint8_t *codes, int64_t rows, int64_t K, int
 template <int BN, int BK>
 cudaError_t launch_bn(const GemmLaunch &L) {
     using Smem = GemmSmem<BN, BK>;
+    static_assert(sizeof(Smem) + 1024 <= (Smem::kCtasPerSm == 2 ? 115712 : 232448),
+                  "shared memory of the GEMM CTA");
     CUtensorMap ma, mb;
     if (!code_map(&ma, L.codes_x, L.M, L.K, kBM, BK / 2) || !code_map(&mb, L.codes_w, L.N, L.K, BN, BK / 2))
         return cudaErrorInvalidValue;
@@ -465,6 +505,15 @@ constexpr int kGemmBK = 256;
 
 // 256 output columns per CTA when N allows it (A tiles reused twice as
 // often), else 128.
+cudaError_t launch_scale_tiles(const uint8_t *scales, int64_t rows, int64_t K, uint8_t *tiles,
+                               cudaStream_t stream) {
+    const int64_t words = rows * K / 128;
+    if (words == 0) return cudaSuccess;
+    const int64_t blocks = std::min<int64_t>((words + 255) / 256, 148 * 16);
+    return launch_k(scale_tiles_kernel, dim3((unsigned)blocks), dim3(256), 0, stream, scales, words,
+                    K / 128, tiles);
+}
+
 cudaError_t launch_w4a4_gemm(const GemmLaunch &L) {
     if (L.M == 0 || L.N == 0) return cudaSuccess;
     return (L.N % 256 == 0) ? launch_bn<256, kGemmBK>(L) : launch_bn<128, kGemmBK>(L);

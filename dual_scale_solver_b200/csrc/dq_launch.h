@@ -79,8 +79,8 @@ cudaError_t launch_two_level(const TwoLevelLaunch &L);
 
 // Block-scaled W4A4 GEMM (dq_gemm.cu): out[M, N] = a_n * Qx[M, K] . Qw[N, K]^T.
 struct GemmLaunch {
-    const uint8_t *codes_x, *scales_x;   // [M, K/2] E2M1, [M, K/32] E8M0
-    const uint8_t *codes_w, *scales_w;   // [N, K/2] E2M1, [N, K/32] E8M0
+    const uint8_t *codes_x, *scales_x;   // [M, K/2] E2M1, M*K/32 E8M0 in scale tiles
+    const uint8_t *codes_w, *scales_w;   // [N, K/2] E2M1, N*K/32 E8M0 in scale tiles
     const float *a;                      // [N]
     float *out;                          // [M, N]
     int64_t M, N, K;                     // multiples of 128, 128, 256
@@ -88,6 +88,10 @@ struct GemmLaunch {
     cudaStream_t stream;
 };
 cudaError_t launch_w4a4_gemm(const GemmLaunch &L);
+// Row-major E8M0 scales [rows, K/32] -> the GEMM's scale tiles (rows a
+// multiple of 128, K of 128).
+cudaError_t launch_scale_tiles(const uint8_t *scales, int64_t rows, int64_t K, uint8_t *tiles,
+                               cudaStream_t stream);
 
 cudaError_t launch_tile_c0(const TileLaunch &L);
 cudaError_t launch_tile_c1(const TileLaunch &L);

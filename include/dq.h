@@ -233,15 +233,30 @@ DQ_API dq_status dq_two_level_quant(const void *X, int32_t dtype, int64_t rows, 
                                     void *inner_scales, float *outer_scales, float *qdq,
                                     dq_stream stream);
 
+/* Scale tiles: the layout in which dq_w4a4_gemm takes E8M0 group scales
+ * (G = 32), the one the tensor core reads them in.  For every block of 128
+ * rows and every 128 elements of K (4 scales per row) one 512-byte chunk,
+ * chunks ordered [row block][K block]; inside a chunk the scale k (0..3) of
+ * row r (0..127 within the block) sits at byte (r % 32) * 16 + (r / 32) * 4
+ * + k.  rows * K / 32 bytes in all, like the row-major array.
+ * dq_scale_tiles rewrites row-major scales [rows, K/32] (the layout written
+ * by dq_solve_dual_scale, dq_quantize and dq_act_rescale_quant) into scale
+ * tiles: rows and K multiples of 128, both pointers 16-byte aligned, device,
+ * caller-owned, not overlapping.  Errors: DQ_ERR_SHAPE, DQ_ERR_ARG,
+ * DQ_ERR_ALIGN.  (No counterpart in the method: a data layout.) */
+DQ_API dq_status dq_scale_tiles(const void *scales, int64_t rows, int64_t K, uint8_t *tiles,
+                                dq_stream stream);
+
 /* Block-scaled W4A4 GEMM on the tensor cores, the inference step of eq. (1)
  * (daiwk note, "核心公式": X W^T ~= (X D_b) Qhat^T D_a; trove summary, "How to
  * use it"):  out[m, n] = a_n * sum_k Qx[m, k] * Qw[n, k], float32, where Qx
- * is given by codes_x [M, K/2] and scales_x [M, K/32] (dq_act_rescale_quant
- * output) and Qw by codes_w [N, K/2] and scales_w [N, K/32] (the solve's
- * codes and group scales), a [N] the outer row scales of W.  `fmt` must be
- * MXFP4 (E2M1 codes, E8M0 group scales, G = 32).  M and N multiples of 128,
- * K a multiple of 256; every pointer 16-byte aligned; out [M, N] row-major,
- * caller-owned.  The products are accumulated in float32.  Errors:
+ * is given by codes_x [M, K/2] and scales_x (M * K/32 bytes, scale tiles of
+ * the dq_act_rescale_quant scales) and Qw by codes_w [N, K/2] and scales_w
+ * (N * K/32 bytes, scale tiles of the solve's group scales), a [N] the outer
+ * row scales of W.  `fmt` must be MXFP4 (E2M1 codes, E8M0 group scales, G =
+ * 32).  M and N multiples of 128, K a multiple of 256; every pointer 16-byte
+ * aligned; out [M, N] row-major, caller-owned.  The products are
+ * accumulated in float32.  Errors:
  * DQ_ERR_FORMAT, DQ_ERR_SHAPE, DQ_ERR_ARG, DQ_ERR_ALIGN; a stalled pipeline
  * (a bounded wait that ran out) raises the device flag read by
  * dq_last_device_status as DQ_ERR_TIMEOUT. */

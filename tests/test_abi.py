@@ -24,7 +24,7 @@ def built():
 
 def test_exports_match_header():
     names = _declared()
-    assert len(names) == 19
+    assert len(names) == 20
     assert sorted(dq.EXPORTS) == names
     L = dq.lib()
     for n in names:
@@ -131,3 +131,12 @@ def test_w4a4_gemm_argument_errors():
     assert L.dq_w4a4_gemm(*args(f, 128, 128, 320)) == -2           # K % 256
     assert L.dq_w4a4_gemm(*args(f, 128, 128, 256)) == -1           # null pointers
     assert L.dq_w4a4_gemm(*args(f, 0, 128, 256)) == 0              # empty
+
+
+def test_scale_tiles_argument_errors():
+    L = dq.lib()
+    assert L.dq_scale_tiles(None, 100, 256, None, None) == -2       # rows % 128
+    assert L.dq_scale_tiles(None, 128, 96, None, None) == -2        # K % 128
+    assert L.dq_scale_tiles(None, 128, 256, None, None) == -1       # null pointers
+    assert L.dq_scale_tiles(None, 0, 256, None, None) == 0          # empty
+    assert L.dq_scale_tiles(ctypes.c_void_p(16), 128, 128, ctypes.c_void_p(24), None) == -9  # alignment

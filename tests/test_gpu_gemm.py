@@ -111,3 +111,36 @@ def test_w4a4_gemm_large_k_sampled_rows():
     rows = np.sort(synth.distinct_indices(synth.stream_key(88, M), M, 24).numpy())
     ref, bound = _reference(cx, sx, cw, sw, a, rows=rows)
     assert np.all(np.abs(np64(out)[rows] - ref) <= bound)
+
+
+def _tiles_expected(S):
+    """Scale tiles written out from their definition: chunk (row block rb, K
+    block kc) of 512 bytes, scale k of row r at (r % 32) * 16 + (r // 32) * 4 + k."""
+    rows, nk = S.shape
+    out = np.zeros((rows // 128, nk // 4, 512), dtype=np.uint8)
+    for rb in range(rows // 128):
+        for kc in range(nk // 4):
+            for r in range(128):
+                for k in range(4):
+                    out[rb, kc, (r % 32) * 16 + (r // 32) * 4 + k] = S[rb * 128 + r, 4 * kc + k]
+    return out.reshape(-1)
+
+
+@pytest.mark.parametrize("rows,K", [(128, 128), (384, 1024)])
+def test_scale_tiles_layout(rows, K):
+    _, S = _random_operand(rows, K, 40 + rows, e_lo=0, e_hi=256)
+    t = dq.scale_tiles(S.cuda(), K).cpu().numpy()
+    assert np.array_equal(t, _tiles_expected(S.numpy()))
+
+
+def test_w4a4_gemm_pretiled_scales_equal_row_major():
+    M, N, K = 256, 512, 1024
+    cx, sx = _random_operand(M, K, 31)
+    cw, sw = _random_operand(N, K, 32)
+    a = torch.ones(N).cuda()
+    cx, sx, cw, sw = cx.cuda(), sx.cuda(), cw.cuda(), sw.cuda()
+    y0 = dq.w4a4_gemm(cx, sx, cw, sw, a)
+    y1 = dq.w4a4_gemm(cx, dq.scale_tiles(sx), cw, dq.scale_tiles(sw), a, tiled=True)
+    torch.cuda.synchronize()
+    assert dq.last_device_status() == 0
+    assert torch.equal(y0, y1)
