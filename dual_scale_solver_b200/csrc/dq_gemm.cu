@@ -24,8 +24,9 @@
 //              no multicast) and bulk copies of their scale tiles;
 //   warp 1     TMEM allocation; lane 0 issues tcgen05.cp (scales to TMEM),
 //              the MMAs and the tcgen05.commit arrivals;
-//   warps 2-5  epilogue: TMEM -> registers (tcgen05.ld) -> shared memory ->
-//              row-contiguous float32 stores, times a_n.
+//   warps 2-9  epilogue: TMEM -> registers (tcgen05.ld; TMEM is handed back
+//              before the stores) -> shared memory -> row-contiguous float32
+//              stores, times a_n.
 // Every wait on an mbarrier is bounded: a wait that runs out raises a device
 // status bit, the CTA stops issuing work, waits (bounded) for its copies in
 // flight, frees its TMEM and returns.
@@ -41,7 +42,7 @@ namespace {
 
 constexpr int kBM = 128;
 constexpr int kSfChunk = 512;                  // 128 rows x 4 scales
-constexpr int kThreadsGemm = 192;
+constexpr int kThreadsGemm = 320;               // 10 warps: producer, MMA, 8 epilogue
 constexpr uint64_t kWaitLimitNs = 1000000000ull;   // a wait gives up after 1 s
 
 // BN = 128 or 256 output columns per CTA; BK = 128 or 256 K elements per
@@ -60,8 +61,8 @@ struct __align__(1024) GemmSmem {
     // epilogue staging: per epilogue warp 32 rows x EC float32 columns,
     // 16-byte chunks swizzled so that a row-per-lane write and a
     // row-contiguous read are both free of bank conflicts
-    static constexpr int EC = BN == 128 ? 16 : 32;
-    static constexpr int kStgBytes = 4 * 32 * EC * 4;
+    static constexpr int EC = BN == 128 ? 8 : 16;
+    static constexpr int kStgBytes = 8 * 32 * EC * 4;
     static constexpr int kStages =
         ((kCtasPerSm == 2 ? 112 * 1024 : 226 * 1024) - kStgBytes - 1024) / kStageBytes;
     static constexpr uint32_t kStageTx = kStageBytes;      // bytes that land per stage
@@ -72,7 +73,7 @@ struct __align__(1024) GemmSmem {
     uint8_t b[kStages][kTileBytesB];
     uint8_t sfa[kStages][KC * kSfChunk];            // [k-chunk][512]
     uint8_t sfb[kStages][NB * KC * kSfChunk];       // [row block][k-chunk][512]
-    float4 stg[4][32 * EC / 4];
+    float4 stg[8][32 * EC / 4];
     uint64_t full[kStages];
     uint64_t empty[kStages];
     uint64_t acc_full;      // MMA -> epilogue: the tile's accumulator is complete
@@ -212,23 +213,20 @@ __device__ __forceinline__ void tc_fence_after() {
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
-// 32 consecutive float32 columns of this thread's TMEM lane.
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
-    uint32_t r[32];
+// 32 consecutive 32-bit columns of this thread's TMEM lane; the registers
+// are valid after tmem_wait_ld on them.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
-        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
-          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
-          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
-          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
-          "=r"(r[31])
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
         : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-    for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+}
+
+// Waits for this thread's TMEM loads; passing the registers through makes
+// every later use of them depend on the wait.
+__device__ __forceinline__ void tmem_wait_ld(uint32_t (&r)[32]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;" : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31]) :: "memory");
 }
 
 // Bounded wait used while draining at exit (no abort check).
@@ -264,7 +262,7 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
             mbar_init(&sm.empty[s], 1);
         }
         mbar_init(&sm.acc_full, 1);
-        mbar_init(&sm.acc_empty, 4);                // one arrival per epilogue warp
+        mbar_init(&sm.acc_empty, 8);                // one arrival per epilogue warp
         sm.abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -359,16 +357,21 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
         }
         __syncwarp();
     } else {
-        // ---- epilogue: TMEM lane quadrant = warp % 4.  Each 32-column slice
-        // of the warp's 32 accumulator rows goes TMEM -> registers (lane =
-        // row) -> the warp's staging block in shared memory (EC columns at a
-        // time) -> global memory with each store instruction covering whole
-        // row segments (CPR lanes per row), times a_n. ----
+        // ---- epilogue: warps 2-9; a warp reads TMEM lane quadrant warp % 4
+        // (rows quad*32 .. +31 of the tile) and column half (warp - 2) / 4.
+        // It loads its whole share (BN/2 columns) into registers and hands
+        // TMEM back to the MMA warp at once, so the next tile's MMAs run
+        // while it stores: registers (lane = row) -> its staging block in
+        // shared memory (EC columns at a time) -> global memory with each
+        // store instruction covering whole row segments (CPR lanes per
+        // row), times a_n. ----
         constexpr int EC = Smem::EC;
         constexpr int CPR = EC / 4;                  // 16-byte chunks per staged row
         constexpr int RPP = 32 / CPR;                // rows per store instruction
-        const int quad = warp & 3;
-        float4 *stg = sm.stg[quad];
+        constexpr int HALF = BN / 2;                 // columns per warp
+        const int quad = warp & 3, ew = warp - 2;
+        const int cbase = (ew >> 2) * HALF;
+        float4 *stg = sm.stg[ew];
         // chunk c of row r sits at chunk c ^ sw(r) of the row: 8 consecutive
         // rows then cover all eight 16-byte bank groups
         auto sw = [](int r) { return (r / (8 / CPR)) % CPR; };
@@ -382,39 +385,38 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok) break;
             tc_fence_after();
-            float *const orow = out + (int64_t)(m0 + quad * 32) * N + n0;
-#pragma unroll 1
-            for (int c0 = 0; c0 < BN; c0 += 32) {
-                float v[32];
-                tmem_ld32(tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)c0, v);
-                if (c0 + 32 == BN) {
-                    // the whole accumulator has been read: hand TMEM back to
-                    // the MMA warp before the last stores
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0)
-                        asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];"
-                                     :: "r"(smem_u32(&sm.acc_empty)) : "memory");
+            uint32_t v[HALF / 32][32];
+            const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)cbase;
+#pragma unroll
+            for (int i = 0; i < HALF / 32; ++i) tmem_ld32(taddr + 32 * i, v[i]);
+#pragma unroll
+            for (int i = 0; i < HALF / 32; ++i) tmem_wait_ld(v[i]);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];"
+                             :: "r"(smem_u32(&sm.acc_empty)) : "memory");
+            float *const orow = out + (int64_t)(m0 + quad * 32) * N + n0 + cbase;
+#pragma unroll
+            for (int h = 0; h < HALF / EC; ++h) {
+#pragma unroll
+                for (int c = 0; c < CPR; ++c) {
+                    const int e = h * EC + 4 * c;
+                    stg[lane * CPR + (c ^ sw(lane))] = make_float4(
+                        __uint_as_float(v[e / 32][e % 32]), __uint_as_float(v[e / 32][e % 32 + 1]),
+                        __uint_as_float(v[e / 32][e % 32 + 2]), __uint_as_float(v[e / 32][e % 32 + 3]));
                 }
+                __syncwarp();
+                const int col = h * EC + 4 * cc;
+                const float4 sc = __ldg(reinterpret_cast<const float4 *>(a_row + n0 + cbase + col));
 #pragma unroll
-                for (int h = 0; h < 32 / EC; ++h) {
-#pragma unroll
-                    for (int c = 0; c < CPR; ++c)
-                        stg[lane * CPR + (c ^ sw(lane))] =
-                            make_float4(v[h * EC + 4 * c], v[h * EC + 4 * c + 1],
-                                        v[h * EC + 4 * c + 2], v[h * EC + 4 * c + 3]);
-                    __syncwarp();
-                    const int col = c0 + h * EC + 4 * cc;
-                    const float4 sc = __ldg(reinterpret_cast<const float4 *>(a_row + n0 + col));
-#pragma unroll
-                    for (int p = 0; p < CPR; ++p) {
-                        const int r = p * RPP + rr;
-                        const float4 x = stg[r * CPR + (cc ^ sw(r))];
-                        *reinterpret_cast<float4 *>(orow + (int64_t)r * N + col) =
-                            make_float4(x.x * sc.x, x.y * sc.y, x.z * sc.z, x.w * sc.w);
-                    }
-                    __syncwarp();
+                for (int p = 0; p < CPR; ++p) {
+                    const int r = p * RPP + rr;
+                    const float4 x = stg[r * CPR + (cc ^ sw(r))];
+                    *reinterpret_cast<float4 *>(orow + (int64_t)r * N + col) =
+                        make_float4(x.x * sc.x, x.y * sc.y, x.z * sc.z, x.w * sc.w);
                 }
+                __syncwarp();
             }
         }
     }
