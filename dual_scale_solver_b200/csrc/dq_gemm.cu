@@ -66,8 +66,8 @@ struct __align__(1024) GemmSmem {
     static constexpr int kStages =
         ((kCtasPerSm == 2 ? 112 * 1024 : 226 * 1024) - kStgBytes - 1024) / kStageBytes;
     static constexpr uint32_t kStageTx = kStageBytes;      // bytes that land per stage
-    // TMEM: accumulator BN columns, then A's scales (KC chunks x 4 columns),
-    // then B's (KC k-chunks x NB row blocks x 4 columns)
+    // TMEM: accumulator BN columns, then two slots of scales, each A's (KC
+    // chunks x 4 columns) then B's (KC k-chunks x NB row blocks x 4 columns)
     static constexpr uint32_t kTmemCols = BN == 128 ? 256 : 512;
     uint8_t a[kStages][kTileBytesA];
     uint8_t b[kStages][kTileBytesB];
@@ -163,11 +163,16 @@ __device__ __forceinline__ uint64_t desc_sf(uint32_t saddr) {
 }
 
 // Instruction descriptor, kind::mxf4 with E8M0 block scales: A and B E2M1
-// (K-major), M = 128, N = BN, scale-factor byte ids of A and B.
+// (K-major), M = BM (128, or 256 for a CTA pair), N = BN, scale-factor byte
+// ids of A and B.
+template <int BM, int BN>
+__device__ __forceinline__ uint32_t idesc_mxf4_m(uint32_t sfa_id, uint32_t sfb_id) {
+    return (sfb_id << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | (1u << 23) |
+           ((uint32_t)(BM >> 4) << 24) | (sfa_id << 29);
+}
 template <int BN>
 __device__ __forceinline__ uint32_t idesc_mxf4(uint32_t sfa_id, uint32_t sfb_id) {
-    return (sfb_id << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | (1u << 23) |
-           ((uint32_t)(kBM >> 4) << 24) | (sfa_id << 29);
+    return idesc_mxf4_m<kBM, BN>(sfa_id, sfb_id);
 }
 
 // Output tile t -> (m0, n0).  Tiles go in bands of up to kBandTiles tile
@@ -275,7 +280,10 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;             // accumulator: columns [0, BN)
-    const uint32_t sfa_t = tmem + BN, sfb_t = tmem + BN + 4 * KC;
+    // scales of even / odd K tiles in two slots, so that copying the next
+    // tile's scales never waits for the MMAs still reading the current ones
+    constexpr uint32_t kSfSlot = 4 * KC * (1 + NB);
+    const uint32_t sfa_t0 = tmem + BN, sfb_t0 = tmem + BN + 4 * KC;
 
     // The CTA walks the output tiles t = blockIdx.x, + gridDim.x, ... in the
     // band order of tile_coords.
@@ -331,6 +339,7 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
                     const int s = g % kStages;
                     if (!mbar_wait(&sm.full[s], (g / kStages) & 1, abort, status)) { stop = true; break; }
                     tc_fence_after();
+                    const uint32_t sfa_t = sfa_t0 + (g & 1) * kSfSlot, sfb_t = sfb_t0 + (g & 1) * kSfSlot;
 #pragma unroll
                     for (int kc = 0; kc < KC; ++kc)
                         tmem_cp_sf(sfa_t + 4 * kc, desc_sf(smem_u32(&sm.sfa[s][kc * kSfChunk])));
@@ -429,6 +438,293 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
     }
 }
 
+// ---------------------------------------------------------------------------
+// CTA-pair variant (M and N multiples of 256): a cluster of two CTAs on two
+// SMs computes a 256 x 256 tile with tcgen05.mma.cta_group::2 (M = 256, N =
+// 256): CTA rank r holds rows 128r..128r+127 of the A tile and rows
+// 128r..128r+127 of the B tile (its half of N) in its shared memory, the
+// A scales of its own rows and the B scales of all 256 rows; its TMEM holds
+// its 128 accumulator rows x 256 columns.  Per SM that is 32 KB of codes per
+// K tile of 256 instead of 48 KB, so the ring is 6 stages deep.
+//   both CTAs   warp 0 lane 0 loads its halves by TMA (.cta_group::2: the
+//               completion is counted on the barrier of CTA 0);
+//               warps 2-9 drain their own accumulator rows (as above) and
+//               release the accumulator on CTA 0's barrier;
+//               warp 1 allocates / frees TMEM (cta_group::2, both CTAs).
+//   CTA 0       warp 1 lane 0 waits for both halves of a stage, copies the
+//               scales to both TMEMs (tcgen05.cp.cta_group::2), issues the
+//               MMAs, and commits to the barriers of both CTAs.
+// ---------------------------------------------------------------------------
+template <int BK>
+struct __align__(1024) GemmPairSmem {
+    static constexpr int KC = BK / 128;
+    static constexpr int kRowBytes = BK / 2;
+    static constexpr int kTileBytes = 128 * kRowBytes;                 // A or B half, per CTA
+    static constexpr int kStageBytes = 2 * kTileBytes + 3 * KC * kSfChunk;
+    static constexpr int EC = 8;
+    static constexpr int kStgBytes = 8 * 32 * EC * 4;
+    static constexpr int kStages = (226 * 1024 - kStgBytes - 1024) / kStageBytes;
+    static constexpr uint32_t kPairTx = 2 * kStageBytes;              // both CTAs' bytes
+    static constexpr uint32_t kTmemCols = 512;
+    uint8_t a[kStages][kTileBytes];
+    uint8_t b[kStages][kTileBytes];
+    uint8_t sfa[kStages][KC * kSfChunk];            // [k-chunk][512], own rows
+    uint8_t sfb[kStages][2 * KC * kSfChunk];        // [row block][k-chunk][512], all 256 rows
+    float4 stg[8][32 * EC / 4];
+    uint64_t full[kStages];     // CTA 0: both CTAs' bytes of the stage have landed
+    uint64_t empty[kStages];    // the MMAs reading the stage are done (each CTA)
+    uint64_t acc_full;          // the tile's accumulator is complete (each CTA)
+    uint64_t acc_empty;         // CTA 0: both CTAs' epilogues have read it out
+    uint32_t tmem_base;
+    int abort;
+};
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+// Shared-memory address of the same variable in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t cluster_addr(const void *p, uint32_t rank) {
+    uint32_t a;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(smem_u32(p)), "r"(rank));
+    return a;
+}
+
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
+                 "barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// TMA load into this CTA's shared memory whose completion is counted on an
+// mbarrier of either CTA of the pair (bar: shared::cluster address).  No
+// multicast.
+__device__ __forceinline__ void tma_load_2d_pair(void *dst, const CUtensorMap *map, int x, int y,
+                                                 uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];"
+        :: "r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+        : "memory");
+}
+
+__device__ __forceinline__ void mma_mxf4_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                              uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
+                                              uint32_t accumulate) {
+    asm volatile(
+        "{ .reg .pred p; setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p; }"
+        :: "r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem),
+           "r"(sfb_tmem)
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_cp_sf_pair(uint32_t taddr, uint64_t sdesc) {
+    asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" :: "r"(taddr), "l"(sdesc)
+                 : "memory");
+}
+
+// Arrive on the mbarrier at this offset in both CTAs of the pair once the
+// tcgen05 operations issued so far by this thread are complete.
+__device__ __forceinline__ void umma_commit_pair(uint64_t *bar) {
+    asm volatile(
+        "{ .reg .b16 m; mov.b16 m, 3;\n\t"
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+        " [%0], m; }"
+        :: "r"(smem_u32(bar)) : "memory");
+}
+
+template <int BK>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsGemm, 1)
+w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
+                      const __grid_constant__ CUtensorMap map_sfa,
+                      const __grid_constant__ CUtensorMap map_sfb, const float *a_row, float *out,
+                      int M, int N, int K, unsigned int *status) {
+    using Smem = GemmPairSmem<BK>;
+    constexpr int kStages = Smem::kStages;
+    constexpr int KC = Smem::KC;
+    constexpr int BN = 256;
+    grid_dependency_begin();
+    extern __shared__ uint8_t gemm_smem_raw[];
+    Smem &sm = *reinterpret_cast<Smem *>(
+        (reinterpret_cast<uintptr_t>(gemm_smem_raw) + 1023) & ~uintptr_t(1023));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_rank();
+    const bool leader = rank == 0;
+    const int KT = K / BK;
+    const int n_tiles = N / BN, m_tiles = M / 256;
+    const int tiles = m_tiles * n_tiles;
+    const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+    const int64_t kblocks = K / 128;                // scale chunks per 128-row block
+    volatile int *abort = &sm.abort;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&sm.full[s], 1);              // CTA 0's producer (+ both CTAs' bytes)
+            mbar_init(&sm.empty[s], 1);             // CTA 0's commit
+        }
+        mbar_init(&sm.acc_full, 1);                 // CTA 0's commit
+        mbar_init(&sm.acc_empty, 16);               // 8 epilogue warps per CTA
+        sm.abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;"
+                     :: "r"(smem_u32(&sm.tmem_base)), "r"(Smem::kTmemCols) : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    cluster_sync_all();                             // barriers and TMEM ready in both CTAs
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;             // accumulator: columns [0, 256)
+    constexpr uint32_t kSfSlot = 4 * KC * 3;        // two scale slots, as above
+    const uint32_t sfa_t0 = tmem + BN, sfb_t0 = tmem + BN + 4 * KC;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ---- producer: this CTA's halves of every K tile ----
+            const uint32_t full0 = cluster_addr(&sm.full[0], 0);
+            int g = 0;
+            bool stop = false;
+            for (int t = pair; t < tiles && !stop; t += npairs) {
+                int m0, n0;
+                tile_coords(t, m_tiles, n_tiles, 256, BN, m0, n0);
+                const int ma = m0 + 128 * (int)rank, nb0 = n0 + 128 * (int)rank;
+                for (int kt = 0; kt < KT; ++kt, ++g) {
+                    const int s = g % kStages;
+                    if (g >= kStages && !mbar_wait(&sm.empty[s], ((g / kStages) - 1) & 1, abort, status)) {
+                        stop = true;
+                        break;
+                    }
+                    const uint32_t bar = full0 + (uint32_t)(s * sizeof(uint64_t));
+                    if (leader) mbar_arrive_expect_tx(&sm.full[s], Smem::kPairTx);
+                    tma_load_2d_pair(sm.a[s], &map_a, kt * (BK / 2), ma, bar);
+                    tma_load_2d_pair(sm.b[s], &map_b, kt * (BK / 2), nb0, bar);
+                    tma_load_2d_pair(sm.sfa[s], &map_sfa, 0, (int)((ma / 128) * kblocks + kt * KC), bar);
+#pragma unroll
+                    for (int nb = 0; nb < 2; ++nb)
+                        tma_load_2d_pair(sm.sfb[s] + nb * KC * kSfChunk, &map_sfb, 0,
+                                         (int)((n0 / 128 + nb) * kblocks + kt * KC), bar);
+                }
+            }
+            if (*abort) {
+                // let the copies already issued land before the CTA exits
+                if (leader) {
+                    for (int k = max(0, g - kStages); k < g; ++k)
+                        mbar_drain(&sm.full[k % kStages], (k / kStages) & 1);
+                } else {
+                    const uint64_t t0 = global_ns();
+                    while (global_ns() - t0 < 2000000ull) {
+                    }
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        if (leader && lane == 0) {
+            // ---- MMA issuer (CTA 0) ----
+            int g = 0, j = 0;
+            bool stop = false;
+            for (int t = pair; t < tiles && !stop; t += npairs, ++j) {
+                // both CTAs' epilogues have read out the previous accumulator
+                if (j > 0 && !mbar_wait(&sm.acc_empty, (j - 1) & 1, abort, status)) break;
+                tc_fence_after();
+                for (int kt = 0; kt < KT; ++kt, ++g) {
+                    const int s = g % kStages;
+                    if (!mbar_wait(&sm.full[s], (g / kStages) & 1, abort, status)) { stop = true; break; }
+                    tc_fence_after();
+                    const uint32_t sfa_t = sfa_t0 + (g & 1) * kSfSlot, sfb_t = sfb_t0 + (g & 1) * kSfSlot;
+#pragma unroll
+                    for (int kc = 0; kc < KC; ++kc)
+                        tmem_cp_sf_pair(sfa_t + 4 * kc, desc_sf(smem_u32(&sm.sfa[s][kc * kSfChunk])));
+#pragma unroll
+                    for (int q = 0; q < 2 * KC; ++q)      // TMEM: [k-chunk][row block]
+                        tmem_cp_sf_pair(sfb_t + 4 * q,
+                                        desc_sf(smem_u32(&sm.sfb[s][((q % 2) * KC + q / 2) * kSfChunk])));
+                    const uint32_t a0 = smem_u32(sm.a[s]), b0 = smem_u32(sm.b[s]);
+#pragma unroll
+                    for (int kb = 0; kb < BK / 64; ++kb) {
+                        const uint32_t c = kb >> 1, id = (kb & 1) * 2;
+                        mma_mxf4_pair(tmem, desc_swz<BK / 2>(a0 + kb * 32), desc_swz<BK / 2>(b0 + kb * 32),
+                                      idesc_mxf4_m<256, BN>(id, id), sfa_t + 4 * c, sfb_t + 8 * c,
+                                      (kt | kb) != 0);
+                    }
+                    umma_commit_pair(&sm.empty[s]);  // frees the stage in both CTAs
+                }
+                umma_commit_pair(&sm.acc_full);      // also after an abort: the epilogues wait on it
+            }
+        }
+        __syncwarp();
+    } else {
+        // ---- epilogue (both CTAs): rows m0 + 128 rank + quad*32 + lane ----
+        constexpr int EC = Smem::EC;
+        constexpr int CPR = EC / 4;
+        constexpr int RPP = 32 / CPR;
+        constexpr int HALF = BN / 2;
+        const int quad = warp & 3, ew = warp - 2;
+        const int cbase = (ew >> 2) * HALF;
+        float4 *stg = sm.stg[ew];
+        auto sw = [](int r) { return (r / (8 / CPR)) % CPR; };
+        const int rr = lane / CPR, cc = lane % CPR;
+        const uint32_t acc_empty0 = cluster_addr(&sm.acc_empty, 0);
+        int j = 0;
+        for (int t = pair; t < tiles; t += npairs, ++j) {
+            int m0, n0;
+            tile_coords(t, m_tiles, n_tiles, 256, BN, m0, n0);
+            int ok = 1;
+            if (lane == 0) ok = mbar_wait(&sm.acc_full, j & 1, abort, status) && !*abort;
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) break;
+            tc_fence_after();
+            uint32_t v[HALF / 32][32];
+            const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)cbase;
+#pragma unroll
+            for (int i = 0; i < HALF / 32; ++i) tmem_ld32(taddr + 32 * i, v[i]);
+#pragma unroll
+            for (int i = 0; i < HALF / 32; ++i) tmem_wait_ld(v[i]);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];"
+                             :: "r"(acc_empty0) : "memory");
+            float *const orow = out + (int64_t)(m0 + 128 * (int)rank + quad * 32) * N + n0 + cbase;
+#pragma unroll
+            for (int h = 0; h < HALF / EC; ++h) {
+#pragma unroll
+                for (int c = 0; c < CPR; ++c) {
+                    const int e = h * EC + 4 * c;
+                    stg[lane * CPR + (c ^ sw(lane))] = make_float4(
+                        __uint_as_float(v[e / 32][e % 32]), __uint_as_float(v[e / 32][e % 32 + 1]),
+                        __uint_as_float(v[e / 32][e % 32 + 2]), __uint_as_float(v[e / 32][e % 32 + 3]));
+                }
+                __syncwarp();
+                const int col = h * EC + 4 * cc;
+                const float4 sc = __ldg(reinterpret_cast<const float4 *>(a_row + n0 + cbase + col));
+#pragma unroll
+                for (int p = 0; p < CPR; ++p) {
+                    const int r = p * RPP + rr;
+                    const float4 x = stg[r * CPR + (cc ^ sw(r))];
+                    *reinterpret_cast<float4 *>(orow + (int64_t)r * N + col) =
+                        make_float4(x.x * sc.x, x.y * sc.y, x.z * sc.z, x.w * sc.w);
+                }
+                __syncwarp();
+            }
+        }
+    }
+    // every MMA of the pair has completed (each CTA's epilogue saw the last
+    // commit, or gave up): no CTA leaves while its partner may still signal
+    // its barriers or read its TMEM
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync_all();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;"
+                     :: "r"(tmem), "r"(Smem::kTmemCols) : "memory");
+    }
+}
+
 // Row-major E8M0 scales [rows, K/32] -> scale tiles: one thread per 4-byte
 // word (the 4 scales of one row in one 128-element K block); word w of chunk
 // (rb, kc) holds row rb*128 + (w % 4)*32 + w/4, so the writes are coalesced.
@@ -474,6 +770,48 @@ bool code_map(CUtensorMap *m, const uint8_t *codes, int64_t rows, int64_t K, int
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 2-D map over scale tiles as rows of one 512-byte chunk (256 x 16-bit
+// elements): boxes of KC consecutive chunks, no swizzle.
+bool scale_tile_map(CUtensorMap *m, const uint8_t *tiles, int64_t rows, int64_t K, int kc) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {256, (cuuint64_t)(rows / 128 * (K / 128))};
+    const cuuint64_t strides[1] = {512};
+    const cuuint32_t box[2] = {256, (cuuint32_t)kc};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<uint8_t *>(tiles), dims, strides,
+               box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int BK>
+cudaError_t launch_pair(const GemmLaunch &L) {
+    using Smem = GemmPairSmem<BK>;
+    static_assert(sizeof(Smem) + 1024 <= 232448, "shared memory of the GEMM CTA");
+    CUtensorMap ma, mb, msa, msb;
+    if (!code_map(&ma, L.codes_x, L.M, L.K, 128, BK / 2) || !code_map(&mb, L.codes_w, L.N, L.K, 128, BK / 2) ||
+        !scale_tile_map(&msa, L.scales_x, L.M, L.K, Smem::KC) ||
+        !scale_tile_map(&msb, L.scales_w, L.N, L.K, Smem::KC))
+        return cudaErrorInvalidValue;
+    const size_t smem = sizeof(Smem) + 1024;
+    static bool done[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!done[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(w4a4_gemm_pair_kernel<BK>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        done[dev] = true;
+    }
+    // persistent: one CTA pair per two SMs, or fewer tiles
+    int sms = 148;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) sms = 148;
+    const int64_t tiles = (L.M / 256) * (L.N / 256);
+    const unsigned grid = 2u * (unsigned)std::min<int64_t>(tiles, sms / 2);
+    return launch_k(w4a4_gemm_pair_kernel<BK>, dim3(grid), dim3(kThreadsGemm), smem, L.stream, ma, mb,
+                    msa, msb, L.a, L.out, (int)L.M, (int)L.N, (int)L.K, L.status);
+}
+
 template <int BN, int BK>
 cudaError_t launch_bn(const GemmLaunch &L) {
     using Smem = GemmSmem<BN, BK>;
@@ -505,8 +843,9 @@ cudaError_t launch_bn(const GemmLaunch &L) {
 
 constexpr int kGemmBK = 256;
 
-// 256 output columns per CTA when N allows it (A tiles reused twice as
-// often), else 128.
+// A CTA pair per 256 x 256 tile when M and N allow it; else one CTA per
+// 128 x 256 tile when N allows it (A tiles reused twice as often), else
+// 128 x 128.
 cudaError_t launch_scale_tiles(const uint8_t *scales, int64_t rows, int64_t K, uint8_t *tiles,
                                cudaStream_t stream) {
     const int64_t words = rows * K / 128;
@@ -518,6 +857,7 @@ cudaError_t launch_scale_tiles(const uint8_t *scales, int64_t rows, int64_t K, u
 
 cudaError_t launch_w4a4_gemm(const GemmLaunch &L) {
     if (L.M == 0 || L.N == 0) return cudaSuccess;
+    if (L.M % 256 == 0 && L.N % 256 == 0) return launch_pair<kGemmBK>(L);
     return (L.N % 256 == 0) ? launch_bn<256, kGemmBK>(L) : launch_bn<128, kGemmBK>(L);
 }
 

@@ -53,7 +53,11 @@ def _reference(cx, sx, cw, sw, a, rows=None):
     return ref, bound
 
 
-@pytest.mark.parametrize("M,N,K", [(128, 128, 256), (256, 384, 1024), (384, 256, 2048)])
+# (256, 256, 256), (512, 768, 1024), (768, 512, 2048): CTA pairs on 256 x 256
+# tiles; (128, 128, 256), (384, 256, 2048): one CTA per 128 x 256 tile;
+# (256, 384, 1024): 128 x 128 tiles
+@pytest.mark.parametrize("M,N,K", [(128, 128, 256), (256, 384, 1024), (384, 256, 2048),
+                                   (256, 256, 256), (512, 768, 1024), (768, 512, 2048)])
 def test_w4a4_gemm_random_operands(M, N, K):
     cx, sx = _random_operand(M, K, 1 + M)
     cw, sw = _random_operand(N, K, 2 + N)
@@ -144,3 +148,25 @@ def test_w4a4_gemm_pretiled_scales_equal_row_major():
     torch.cuda.synchronize()
     assert dq.last_device_status() == 0
     assert torch.equal(y0, y1)
+
+
+def test_w4a4_gemm_pair_tile_placement():
+    # a 256 x 256 tile is split over two CTAs: rows 128..255 of the output and
+    # rows 128..255 of the weights live in the second one
+    M, N, K = 256, 256, 512
+    cx = torch.zeros(M, K // 2, dtype=torch.uint8)
+    sx = torch.full((M, K // 32), 127, dtype=torch.uint8)
+    cw = torch.zeros(N, K // 2, dtype=torch.uint8)
+    sw = torch.full((N, K // 32), 127, dtype=torch.uint8)
+    cx[200, 150] = 0x02                                 # x[200, 300] = 1.0
+    sx[200, 9] = 128                                    # its group scale 2
+    cw[130, 150] = 0x07                                 # w[130, 300] = 6.0
+    cx[5, 100] = 0x02                                   # x[5, 200] = 1.0
+    cw[250, 100] = 0x06                                 # w[250, 200] = 4.0
+    a = torch.ones(N)
+    a[250] = 0.5
+    out = dq.w4a4_gemm(cx.cuda(), sx.cuda(), cw.cuda(), sw.cuda(), a.cuda()).cpu()
+    want = torch.zeros(M, N)
+    want[200, 130] = 12.0
+    want[5, 250] = 2.0
+    assert torch.equal(out, want)
