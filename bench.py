@@ -592,7 +592,7 @@ def run_gemm(args, wl, rank, world, local_rank):
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "fp4 (e2m1)", "data": "synthetic",
         "config": {"workload": f"{wl.name}: its {len(outs)} linears x {M} tokens",
-                   "flops_per_step": flops, "tile": "128 x (256 if N % 256 == 0 else 128) x 256, 4 stages",
+                   "flops_per_step": flops, "tile": "256 x 256 per CTA pair (tcgen05 cta_group::2), K tile 256, 6-stage ring (M, N multiples of 256; else 128 x 256 or 128 x 128 per CTA)",
                    "l2": "operands larger than L2 (no flush needed)",
                    "parallelism": f"{world} independent decoders" if world > 1 else "1 GPU"},
         "roofline": {"bound": "tensor", "achieved": tflops, "peak": peak, "unit": "TFLOP/s",
