@@ -18,7 +18,7 @@ __all__ = [
     "workspace_size", "quantize", "dequantize", "solve_dual_scale", "solve_dual_scale_batched",
     "row_update", "col_update", "act_rescale_quant", "last_device_status", "EXPORTS",
     "kernel_timing", "kernel_time", "launch_count", "solve_dual_scale_noalloc", "code_bytes",
-    "two_level_quant", "w4a4_gemm", "scale_tiles",
+    "two_level_quant", "w4a4_gemm", "scale_tiles", "solve_dual_scale_batched_host",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -35,7 +35,7 @@ EXPORTS = ("dq_version", "dq_strerror", "dq_format_preset", "dq_workspace_size",
            "dq_row_update", "dq_col_update", "dq_act_rescale_quant", "dq_last_device_status",
            "dq_kernel_timing", "dq_kernel_time", "dq_launch_count",
            "dq_solve_dual_scale_noalloc", "dq_code_bytes", "dq_two_level_quant", "dq_w4a4_gemm",
-           "dq_scale_tiles")
+           "dq_scale_tiles", "dq_solve_dual_scale_batched_host")
 
 
 class DqError(RuntimeError):
@@ -108,6 +108,9 @@ def lib() -> ctypes.CDLL:
         "dq_w4a4_gemm": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int64,
                                    c_int64, c_int64, P(dq_format), c_void_p, c_void_p]),
         "dq_scale_tiles": (c_int32, [c_void_p, c_int64, c_int64, c_void_p, c_void_p]),
+        "dq_solve_dual_scale_batched_host": (c_int32, [c_int32, P(dq_matrix), P(dq_matrix), c_int32,
+                                                       P(dq_format), c_int32, c_void_p, c_size_t,
+                                                       c_void_p, c_void_p, c_void_p]),
         "dq_two_level_quant": (c_int32, [c_void_p, c_int32, c_int64, c_int64, c_int32,
                                          P(dq_format), c_void_p, c_void_p, c_void_p, c_void_p,
                                          c_void_p]),
@@ -310,6 +313,80 @@ def solve_dual_scale_batched(Ws, fmt, T, ws=None, outs=None, half=False, stream=
                                              ws.numel(), _stream(stream)),
            "dq_solve_dual_scale_batched")
     return outs
+
+
+_COPY_STREAMS = {}
+
+
+def _copy_streams(device):
+    """One host-to-device and one device-to-host stream per device (kept)."""
+    idx = torch.device(device).index
+    idx = torch.cuda.current_device() if idx is None else idx
+    if idx not in _COPY_STREAMS:
+        _COPY_STREAMS[idx] = (torch.cuda.Stream(idx), torch.cuda.Stream(idx))
+    return _COPY_STREAMS[idx]
+
+
+def _solve_outputs(rows, cols, fmt, T, half, device, pin=False):
+    codes, gscales = _outputs(rows, cols, fmt, device)
+    kw = dict(device=device, pin_memory=pin)
+    if pin:
+        codes, gscales = codes.pin_memory(), gscales.pin_memory()
+    return dict(codes=codes, gscales=gscales,
+                a=torch.empty(rows, dtype=torch.float32, **kw),
+                b=torch.empty(cols, dtype=torch.float32, **kw),
+                tensor_scale=torch.empty(1, dtype=torch.float32, **kw),
+                mse_trace=torch.empty(T + 1, dtype=torch.float64, **kw),
+                mse_half=torch.empty(max(T, 1), dtype=torch.float64, **kw) if half else None)
+
+
+def _fill_matrix(m, W, o):
+    m.W, m.rows, m.cols = _ptr(W), W.shape[0], W.shape[1]
+    m.a0 = m.b0 = None
+    m.codes, m.gscales = _ptr(o["codes"]), _ptr(o["gscales"])
+    m.a, m.b, m.tensor_scale = _ptr(o["a"]), _ptr(o["b"]), _ptr(o["tensor_scale"])
+    m.mse_trace, m.mse_half = _ptr(o["mse_trace"]), _ptr(o.get("mse_half"))
+
+
+def solve_dual_scale_batched_host(Ws, fmt, T, outs=None, dev_outs=None, staging=None, ws=None,
+                                  half=False, device=None, stream=None):
+    """Solve matrices held in host memory (CPU tensors of one dtype; pin them
+    for the copies to overlap): matrix i+1 is copied in while matrix i is
+    solved and matrix i-1's results are copied back (dq_solve_dual_scale_batched_host).
+    Returns (outs, dev_outs): per matrix a dict of page-locked CPU tensors and
+    one of the device tensors holding the same results.  `stream` (default:
+    the current stream) runs the solves and, on return, also waits for the
+    copies back, so work ordered after it sees the host results.  `outs`,
+    `dev_outs`, `staging` (device copies of W) and `ws` may be passed back in
+    to reuse them."""
+    n = len(Ws)
+    if n == 0:
+        return [], []
+    dev = torch.device(device or "cuda")
+    dt = _dtype_code(Ws[0])
+    shapes = [tuple(W.shape) for W in Ws]
+    if outs is None:
+        outs = [_solve_outputs(r, c, fmt, T, half, "cpu", pin=True) for r, c in shapes]
+    if dev_outs is None:
+        dev_outs = [_solve_outputs(r, c, fmt, T, half, dev) for r, c in shapes]
+    if staging is None:
+        staging = [torch.empty(W.shape, dtype=W.dtype, device=dev) for W in Ws]
+    if ws is None:
+        ws = torch.empty(max(workspace_size([s], fmt) for s in shapes), dtype=torch.uint8, device=dev)
+    host, devm = (dq_matrix * n)(), (dq_matrix * n)()
+    for i in range(n):
+        if _dtype_code(Ws[i]) != dt or Ws[i].is_cuda:
+            raise TypeError("host matrices: CPU tensors of one dtype")
+        _fill_matrix(host[i], Ws[i], outs[i])
+        _fill_matrix(devm[i], staging[i], dev_outs[i])
+    compute = stream if stream is not None else torch.cuda.current_stream(dev)
+    h2d, d2h = _copy_streams(dev)
+    _check(lib().dq_solve_dual_scale_batched_host(n, host, devm, dt, ctypes.byref(fmt), T, _ptr(ws),
+                                                  ws.numel(), compute.cuda_stream, h2d.cuda_stream,
+                                                  d2h.cuda_stream),
+           "dq_solve_dual_scale_batched_host")
+    compute.wait_stream(d2h)
+    return outs, dev_outs
 
 
 def _step(fn, name, W, fmt, tensor_scale, a_in, b_in, out_len, ws, stream):

@@ -849,6 +849,100 @@ dq_status dq_solve_dual_scale_batched(int32_t n, const dq_matrix *mats, int32_t 
                       reinterpret_cast<cudaStream_t>(stream));
 }
 
+namespace {
+
+// Events of the host-streamed solve (created once, reused; calls serialised).
+std::mutex g_host_mu;
+std::vector<cudaEvent_t> g_host_events[kMaxDevices];
+
+dq_status host_events(int dev, size_t k, cudaEvent_t **out) {
+    std::vector<cudaEvent_t> &v = g_host_events[dev];
+    while (v.size() < k) {
+        cudaEvent_t e = nullptr;
+        if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return DQ_ERR_CUDA;
+        v.push_back(e);
+    }
+    *out = v.data();
+    return DQ_OK;
+}
+
+dq_status copy_async(void *dst, const void *src, size_t bytes, cudaMemcpyKind kind,
+                     cudaStream_t st) {
+    if (bytes == 0 || dst == nullptr) return DQ_OK;
+    if (src == nullptr) return DQ_ERR_ARG;
+    DQ_CUDA(cudaMemcpyAsync(dst, src, bytes, kind, st));
+    return DQ_OK;
+}
+
+}  // namespace
+
+dq_status dq_solve_dual_scale_batched_host(int32_t n, const dq_matrix *host, const dq_matrix *dev,
+                                           int32_t dtype, const dq_format *fmt, int32_t T,
+                                           void *workspace, size_t ws_bytes, dq_stream compute,
+                                           dq_stream h2d, dq_stream d2h) {
+    if (n < 0 || T < 0 || (n > 0 && (!host || !dev))) return DQ_ERR_ARG;
+    if (dtype != DQ_DT_F32 && dtype != DQ_DT_BF16) return DQ_ERR_ARG;
+    FmtInfo fi;
+    dq_status s = check_format(fmt, &fi);
+    if (s != DQ_OK) return s;
+    if (n == 0) return DQ_OK;
+    const size_t esz = dtype == DQ_DT_F32 ? 4 : 2;
+    const size_t gsz = fmt->group_scale == DQ_SCALE_BF16 ? 2 : 1;
+    for (int i = 0; i < n; ++i) {
+        const dq_matrix &h = host[i], &d = dev[i];
+        if (h.rows != d.rows || h.cols != d.cols) return DQ_ERR_SHAPE;
+        if (h.rows < 0 || h.cols < 0 || h.cols % fi.G) return DQ_ERR_SHAPE;
+        if (h.rows > 0 && h.cols > 0 && (!h.W || !d.W)) return DQ_ERR_ARG;
+        if ((h.a0 && !d.a0) || (h.b0 && !d.b0)) return DQ_ERR_ARG;
+        if ((h.mse_trace && !d.mse_trace) || (h.mse_half && !d.mse_half)) return DQ_ERR_ARG;
+    }
+    int devno = 0;
+    if (cudaGetDevice(&devno) != cudaSuccess || devno < 0 || devno >= kMaxDevices) return DQ_ERR_CUDA;
+    const cudaStream_t sc = reinterpret_cast<cudaStream_t>(compute);
+    const cudaStream_t sh = reinterpret_cast<cudaStream_t>(h2d);
+    const cudaStream_t sd = reinterpret_cast<cudaStream_t>(d2h);
+    std::lock_guard<std::mutex> lk(g_host_mu);
+    cudaEvent_t *ev = nullptr;
+    if ((s = host_events(devno, 2 + 2 * (size_t)n, &ev)) != DQ_OK) return s;
+    // an earlier call may still be solving from the staging buffers (h2d
+    // must not overwrite them yet) or copying out its results (compute must
+    // not overwrite those yet)
+    DQ_CUDA(cudaEventRecord(ev[0], sc));
+    DQ_CUDA(cudaStreamWaitEvent(sh, ev[0], 0));
+    DQ_CUDA(cudaEventRecord(ev[1], sd));
+    DQ_CUDA(cudaStreamWaitEvent(sc, ev[1], 0));
+    for (int i = 0; i < n; ++i) {
+        const dq_matrix &h = host[i], &d = dev[i];
+        const size_t rows = (size_t)h.rows, cols = (size_t)h.cols;
+        cudaEvent_t in = ev[2 + 2 * i], out = ev[3 + 2 * i];
+        // in: W (and the initial scales) of matrix i
+        if ((s = copy_async(const_cast<void *>(d.W), h.W, rows * cols * esz, cudaMemcpyHostToDevice, sh)) != DQ_OK) return s;
+        if (h.a0 && (s = copy_async(const_cast<float *>(d.a0), h.a0, rows * 4, cudaMemcpyHostToDevice, sh)) != DQ_OK) return s;
+        if (h.b0 && (s = copy_async(const_cast<float *>(d.b0), h.b0, cols * 4, cudaMemcpyHostToDevice, sh)) != DQ_OK) return s;
+        DQ_CUDA(cudaEventRecord(in, sh));
+        // solve it on the compute stream once its input has landed
+        DQ_CUDA(cudaStreamWaitEvent(sc, in, 0));
+        dq_matrix m = d;
+        if (!h.a0) m.a0 = nullptr;
+        if (!h.b0) m.b0 = nullptr;
+        if ((s = solve_impl(1, &m, dtype, fmt, T, workspace, ws_bytes, sc)) != DQ_OK) return s;
+        DQ_CUDA(cudaEventRecord(out, sc));
+        // out: the results the caller asked for in host memory
+        DQ_CUDA(cudaStreamWaitEvent(sd, out, 0));
+        const size_t code_bytes = rows * (cols * (size_t)fi.bits / 8);
+        const size_t gs_bytes = rows * (cols / (size_t)fi.G) * gsz;
+        if ((s = copy_async(h.codes, d.codes, code_bytes, cudaMemcpyDeviceToHost, sd)) != DQ_OK ||
+            (s = copy_async(h.gscales, d.gscales, gs_bytes, cudaMemcpyDeviceToHost, sd)) != DQ_OK ||
+            (s = copy_async(h.a, d.a, rows * 4, cudaMemcpyDeviceToHost, sd)) != DQ_OK ||
+            (s = copy_async(h.b, d.b, cols * 4, cudaMemcpyDeviceToHost, sd)) != DQ_OK ||
+            (s = copy_async(h.tensor_scale, d.tensor_scale, 4, cudaMemcpyDeviceToHost, sd)) != DQ_OK ||
+            (s = copy_async(h.mse_trace, d.mse_trace, ((size_t)T + 1) * 8, cudaMemcpyDeviceToHost, sd)) != DQ_OK ||
+            (s = copy_async(h.mse_half, d.mse_half, (size_t)T * 8, cudaMemcpyDeviceToHost, sd)) != DQ_OK)
+            return s;
+    }
+    return DQ_OK;
+}
+
 dq_status dq_row_update(const void *W, int32_t dtype, int64_t rows, int64_t cols,
                         const dq_format *fmt, float tensor_scale, const float *a_in,
                         const float *b_in, float *a_out, float *a_pre, double *mse_in,

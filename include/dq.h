@@ -299,6 +299,40 @@ DQ_API dq_status dq_solve_dual_scale_noalloc(const void *W, int32_t dtype, int64
                                              float *tensor_scale, double *mse_trace,
                                              double *mse_half, dq_stream stream);
 
+/* The batched solve for matrices whose inputs and outputs live in host
+ * memory, with the transfers overlapped with the solves (no counterpart in
+ * the pages: the way to feed the solver from the host).  host[i] and dev[i]
+ * describe matrix i twice, with equal rows and cols:
+ *  - host[i].W (and a0 / b0 when not NULL) are read from host memory; the
+ *    outputs whose host[i] pointer is not NULL (codes, gscales, a, b,
+ *    tensor_scale, mse_trace, mse_half) are written to host memory;
+ *  - dev[i] holds device buffers of the same sizes, caller-owned: W (and
+ *    a0 / b0 when host[i] has them) receive the copies of the inputs, the
+ *    outputs are written there as by dq_solve_dual_scale and stay there.
+ * For each i in order: the inputs are copied on stream `h2d`, the matrix is
+ * solved on `compute` once they have landed (one matrix at a time, in
+ * `workspace`, which must hold dq_workspace_size bytes for the largest
+ * single matrix), and the requested outputs are copied back on `d2h` once
+ * its solve is done; so matrix i+1 crosses the bus while matrix i is solved
+ * and matrix i-1's results return.  The call only enqueues: the host outputs
+ * are valid once the work queued on `d2h` has completed.  Host memory must
+ * be page-locked (cudaHostAlloc / cudaHostRegister) for the copies to
+ * overlap; pageable memory works but serialises.  Each call first orders
+ * `h2d` after the work already queued on `compute` and `compute` after the
+ * work already queued on `d2h`, so consecutive calls may reuse the same
+ * buffers.  Calls are serialised inside the library (one set of internal
+ * events per device).  One cudaMemcpyAsync per buffer.  Results equal
+ * dq_solve_dual_scale on each matrix.  Errors: as dq_solve_dual_scale_batched,
+ * plus DQ_ERR_SHAPE when host[i] and dev[i] disagree and DQ_ERR_ARG when a
+ * host input or requested output has no device counterpart; on an error the
+ * work already queued stays queued. */
+DQ_API dq_status dq_solve_dual_scale_batched_host(int32_t n, const dq_matrix *host,
+                                                  const dq_matrix *dev, int32_t dtype,
+                                                  const dq_format *fmt, int32_t T,
+                                                  void *workspace, size_t ws_bytes,
+                                                  dq_stream compute, dq_stream h2d,
+                                                  dq_stream d2h);
+
 /* Measurement support (no counterpart in the method).  dq_kernel_timing(kinds)
  * makes the tile-kernel launches of the kinds whose bit is set in `kinds`
  * (bit k for kind k: 0 row statistics, 1 column statistics, 2 pack,

@@ -24,7 +24,7 @@ def built():
 
 def test_exports_match_header():
     names = _declared()
-    assert len(names) == 20
+    assert len(names) == 21
     assert sorted(dq.EXPORTS) == names
     L = dq.lib()
     for n in names:
@@ -140,3 +140,20 @@ def test_scale_tiles_argument_errors():
     assert L.dq_scale_tiles(None, 128, 256, None, None) == -1       # null pointers
     assert L.dq_scale_tiles(None, 0, 256, None, None) == 0          # empty
     assert L.dq_scale_tiles(ctypes.c_void_p(16), 128, 128, ctypes.c_void_p(24), None) == -9  # alignment
+
+
+def test_host_solve_argument_errors():
+    L = dq.lib()
+    f = dq.format_preset("mxfp4")
+    h, d = (dq.dq_matrix * 1)(), (dq.dq_matrix * 1)()
+    h[0].rows, h[0].cols, d[0].rows, d[0].cols = 4, 64, 4, 64
+    call = lambda n, fmt, hh, dd: L.dq_solve_dual_scale_batched_host(n, hh, dd, 1, ctypes.byref(fmt),
+                                                                     3, None, 0, None, None, None)
+    assert call(-1, f, h, d) == -1                                  # n < 0
+    assert call(0, f, h, d) == 0                                    # nothing to do
+    d[0].cols = 96
+    assert call(1, f, h, d) == -2                                   # host / device shapes differ
+    d[0].cols = 64
+    assert call(1, f, h, d) == -1                                   # no W
+    bad = dq.dq_format(9, 32, 1, 1, 0)
+    assert call(1, bad, h, d) == -3                                 # format
