@@ -71,8 +71,14 @@ def _peaks():
 
 
 def _src_hash():
+    """Hash of the sources that fix the tile kernels and their launch geometry
+    (the device header, the launch header and the per-format tile units); the
+    host API, the GEMM and the two-level kernel do not change their traffic."""
     h = hashlib.sha256()
-    for p in sorted(glob.glob(os.path.join(ROOT, "dual_scale_solver_b200", "csrc", "*"))):
+    csrc = os.path.join(ROOT, "dual_scale_solver_b200", "csrc")
+    files = [os.path.join(csrc, "dq_device.cuh"), os.path.join(csrc, "dq_launch.h")]
+    files += sorted(glob.glob(os.path.join(csrc, "dq_tiles_c*.cu")))
+    for p in files:
         with open(p, "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -349,9 +355,9 @@ def run_ours(args, wl, rank, world, local_rank):
                 "kernel_ms_per_step_from": "one extra step after the timed region, every tile kind event-timed"}
 
     # end-to-end: host buffers in, results out, every step.  The weights go
-    # through the host-streamed solve (matrix i+1 crosses the bus while
-    # matrix i is solved and matrix i-1's results come back), largest first
-    # so that the last, small matrix leaves a short tail; the activation
+    # through the host-streamed solve (group g+1 of consecutive matrices
+    # crosses the bus while group g is solved and group g-1's results come
+    # back), largest first so that the last, small matrices leave a short tail; the activation
     # batch is copied on a stream of its own and quantized with q_proj's b
     # once the solves are done.  The step is bound by the bus: 2.25 GB in and
     # 0.6 GB out.
@@ -366,8 +372,7 @@ def run_ours(args, wl, rank, world, local_rank):
             hX.numel() * hX.element_size() if hX is not None else 0)
         x_stream = torch.cuda.Stream(dev)
         _, d2h_stream = dq._copy_streams(dev)
-        ws_h = torch.empty(max(dq.workspace_size([tuple(W.shape)], fmt) for W in Ws),
-                           dtype=torch.uint8, device=dev)
+        ws_h = dq.workspace([tuple(W.shape) for W in Ws], fmt, dev)
         staging = [torch.empty_like(Ws[i]) for i in order]
         host_outs = dev_outs = act_h = None
 

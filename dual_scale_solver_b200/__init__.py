@@ -353,6 +353,8 @@ def solve_dual_scale_batched_host(Ws, fmt, T, outs=None, dev_outs=None, staging=
     """Solve matrices held in host memory (CPU tensors of one dtype; pin them
     for the copies to overlap): matrix i+1 is copied in while matrix i is
     solved and matrix i-1's results are copied back (dq_solve_dual_scale_batched_host).
+    Consecutive matrices are solved in groups (one batched solve each), as
+    far as `ws` allows (default: room for all of them).
     Returns (outs, dev_outs): per matrix a dict of page-locked CPU tensors and
     one of the device tensors holding the same results.  `stream` (default:
     the current stream) runs the solves and, on return, also waits for the
@@ -371,8 +373,8 @@ def solve_dual_scale_batched_host(Ws, fmt, T, outs=None, dev_outs=None, staging=
         dev_outs = [_solve_outputs(r, c, fmt, T, half, dev) for r, c in shapes]
     if staging is None:
         staging = [torch.empty(W.shape, dtype=W.dtype, device=dev) for W in Ws]
-    if ws is None:
-        ws = torch.empty(max(workspace_size([s], fmt) for s in shapes), dtype=torch.uint8, device=dev)
+    if ws is None:                # room for every grouping the library may choose
+        ws = workspace(shapes, fmt, dev)
     host, devm = (dq_matrix * n)(), (dq_matrix * n)()
     for i in range(n):
         if _dtype_code(Ws[i]) != dt or Ws[i].is_cuda:

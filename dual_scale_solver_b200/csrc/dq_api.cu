@@ -114,39 +114,6 @@ bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // Tile geometry of one matrix (see the tile kernel's description).
-struct Geom {
-    int wc, ncb;
-    int tr[3];
-    int64_t ntiles[3];
-    int64_t nrb_col;
-};
-
-Geom geometry(int64_t rows, int64_t cols, bool f32) {
-    Geom g{};
-    const int epc = f32 ? 4 : 8, seg = 32 * epc;
-    const int64_t nseg = (cols + seg - 1) / seg;
-    int wc = 1;
-    while (wc < 8 && wc < nseg) wc <<= 1;
-    g.wc = wc;
-    g.ncb = (int)((nseg + wc - 1) / wc);
-    const int wr = kWarps / wc;
-    // rows per warp: 256 for column statistics (fewer partial sums), 128 for
-    // the other modes (tile set-up spread over the rows), both reduced for
-    // short matrices so that they still make about 16 row blocks
-    int rpw_long = 16;
-    while (rpw_long < 128 && 2 * rpw_long <= rows / (wr * 16)) rpw_long *= 2;
-    int rpw_col = rpw_long;
-    while (rpw_col < 256 && 2 * rpw_col <= rows / (wr * 16)) rpw_col *= 2;
-    const int rpw[3] = {rpw_long, rpw_col, rpw_long};
-    for (int m = 0; m < 3; ++m) {
-        g.tr[m] = rpw[m] * wr;
-        const int64_t nrb = (rows + g.tr[m] - 1) / g.tr[m];
-        g.ntiles[m] = (rows > 0 && cols > 0) ? nrb * g.ncb : 0;
-    }
-    g.nrb_col = (rows + g.tr[1] - 1) / g.tr[1];
-    return g;
-}
-
 // Workspace bytes of one matrix (each region 256-byte aligned).
 size_t matrix_ws(int64_t rows, int64_t cols, bool f32) {
     const Geom g = geometry(rows, cols, f32);
@@ -896,6 +863,14 @@ dq_status dq_solve_dual_scale_batched_host(int32_t n, const dq_matrix *host, con
         if ((h.a0 && !d.a0) || (h.b0 && !d.b0)) return DQ_ERR_ARG;
         if ((h.mse_trace && !d.mse_trace) || (h.mse_half && !d.mse_half)) return DQ_ERR_ARG;
     }
+    // Consecutive matrices are solved together, as one batched solve, up to
+    // about 1/8 of all the input bytes per group (at least 32 MiB) and as far
+    // as the workspace allows: enough groups for the copies to overlap, large
+    // enough groups that many small matrices still fill the GPU.
+    const bool f32 = dtype == DQ_DT_F32;
+    size_t total_in = 0;
+    for (int i = 0; i < n; ++i) total_in += (size_t)host[i].rows * (size_t)host[i].cols * esz;
+    const size_t target = std::max(total_in / 8, (size_t)32 << 20);
     int devno = 0;
     if (cudaGetDevice(&devno) != cudaSuccess || devno < 0 || devno >= kMaxDevices) return DQ_ERR_CUDA;
     const cudaStream_t sc = reinterpret_cast<cudaStream_t>(compute);
@@ -904,6 +879,11 @@ dq_status dq_solve_dual_scale_batched_host(int32_t n, const dq_matrix *host, con
     std::lock_guard<std::mutex> lk(g_host_mu);
     cudaEvent_t *ev = nullptr;
     if ((s = host_events(devno, 2 + 2 * (size_t)n, &ev)) != DQ_OK) return s;
+    std::vector<dq_matrix> dm(dev, dev + n);
+    for (int i = 0; i < n; ++i) {
+        if (!host[i].a0) dm[i].a0 = nullptr;
+        if (!host[i].b0) dm[i].b0 = nullptr;
+    }
     // an earlier call may still be solving from the staging buffers (h2d
     // must not overwrite them yet) or copying out its results (compute must
     // not overwrite those yet)
@@ -911,34 +891,51 @@ dq_status dq_solve_dual_scale_batched_host(int32_t n, const dq_matrix *host, con
     DQ_CUDA(cudaStreamWaitEvent(sh, ev[0], 0));
     DQ_CUDA(cudaEventRecord(ev[1], sd));
     DQ_CUDA(cudaStreamWaitEvent(sc, ev[1], 0));
-    for (int i = 0; i < n; ++i) {
-        const dq_matrix &h = host[i], &d = dev[i];
-        const size_t rows = (size_t)h.rows, cols = (size_t)h.cols;
-        cudaEvent_t in = ev[2 + 2 * i], out = ev[3 + 2 * i];
-        // in: W (and the initial scales) of matrix i
-        if ((s = copy_async(const_cast<void *>(d.W), h.W, rows * cols * esz, cudaMemcpyHostToDevice, sh)) != DQ_OK) return s;
-        if (h.a0 && (s = copy_async(const_cast<float *>(d.a0), h.a0, rows * 4, cudaMemcpyHostToDevice, sh)) != DQ_OK) return s;
-        if (h.b0 && (s = copy_async(const_cast<float *>(d.b0), h.b0, cols * 4, cudaMemcpyHostToDevice, sh)) != DQ_OK) return s;
+    int g = 0;
+    for (int i = 0; i < n; ++g) {
+        // the group: matrices i .. j-1
+        int j = i;
+        size_t in_bytes = 0, mat_ws = 0;           // the group's inputs and per-matrix workspace
+        while (j < n) {
+            const size_t ws_j = mat_ws + matrix_ws(host[j].rows, host[j].cols, f32);
+            const size_t need_j = 256 + table_ws(j - i + 1) + ws_j;   // as solve_impl needs
+            if (j > i && (in_bytes >= target || need_j > ws_bytes)) break;
+            if (need_j > ws_bytes) return DQ_ERR_WORKSPACE;        // not even matrix i alone
+            mat_ws = ws_j;
+            in_bytes += (size_t)host[j].rows * (size_t)host[j].cols * esz;
+            ++j;
+        }
+        cudaEvent_t in = ev[2 + 2 * g], out = ev[3 + 2 * g];
+        // in: W (and the initial scales) of the group's matrices
+        for (int k = i; k < j; ++k) {
+            const dq_matrix &h = host[k], &d = dev[k];
+            const size_t rows = (size_t)h.rows, cols = (size_t)h.cols;
+            if ((s = copy_async(const_cast<void *>(d.W), h.W, rows * cols * esz, cudaMemcpyHostToDevice, sh)) != DQ_OK) return s;
+            if (h.a0 && (s = copy_async(const_cast<float *>(d.a0), h.a0, rows * 4, cudaMemcpyHostToDevice, sh)) != DQ_OK) return s;
+            if (h.b0 && (s = copy_async(const_cast<float *>(d.b0), h.b0, cols * 4, cudaMemcpyHostToDevice, sh)) != DQ_OK) return s;
+        }
         DQ_CUDA(cudaEventRecord(in, sh));
-        // solve it on the compute stream once its input has landed
+        // solve them on the compute stream once their inputs have landed
         DQ_CUDA(cudaStreamWaitEvent(sc, in, 0));
-        dq_matrix m = d;
-        if (!h.a0) m.a0 = nullptr;
-        if (!h.b0) m.b0 = nullptr;
-        if ((s = solve_impl(1, &m, dtype, fmt, T, workspace, ws_bytes, sc)) != DQ_OK) return s;
+        if ((s = solve_impl(j - i, dm.data() + i, dtype, fmt, T, workspace, ws_bytes, sc)) != DQ_OK) return s;
         DQ_CUDA(cudaEventRecord(out, sc));
         // out: the results the caller asked for in host memory
         DQ_CUDA(cudaStreamWaitEvent(sd, out, 0));
-        const size_t code_bytes = rows * (cols * (size_t)fi.bits / 8);
-        const size_t gs_bytes = rows * (cols / (size_t)fi.G) * gsz;
-        if ((s = copy_async(h.codes, d.codes, code_bytes, cudaMemcpyDeviceToHost, sd)) != DQ_OK ||
-            (s = copy_async(h.gscales, d.gscales, gs_bytes, cudaMemcpyDeviceToHost, sd)) != DQ_OK ||
-            (s = copy_async(h.a, d.a, rows * 4, cudaMemcpyDeviceToHost, sd)) != DQ_OK ||
-            (s = copy_async(h.b, d.b, cols * 4, cudaMemcpyDeviceToHost, sd)) != DQ_OK ||
-            (s = copy_async(h.tensor_scale, d.tensor_scale, 4, cudaMemcpyDeviceToHost, sd)) != DQ_OK ||
-            (s = copy_async(h.mse_trace, d.mse_trace, ((size_t)T + 1) * 8, cudaMemcpyDeviceToHost, sd)) != DQ_OK ||
-            (s = copy_async(h.mse_half, d.mse_half, (size_t)T * 8, cudaMemcpyDeviceToHost, sd)) != DQ_OK)
-            return s;
+        for (int k = i; k < j; ++k) {
+            const dq_matrix &h = host[k], &d = dev[k];
+            const size_t rows = (size_t)h.rows, cols = (size_t)h.cols;
+            const size_t code_bytes = rows * (cols * (size_t)fi.bits / 8);
+            const size_t gs_bytes = rows * (cols / (size_t)fi.G) * gsz;
+            if ((s = copy_async(h.codes, d.codes, code_bytes, cudaMemcpyDeviceToHost, sd)) != DQ_OK ||
+                (s = copy_async(h.gscales, d.gscales, gs_bytes, cudaMemcpyDeviceToHost, sd)) != DQ_OK ||
+                (s = copy_async(h.a, d.a, rows * 4, cudaMemcpyDeviceToHost, sd)) != DQ_OK ||
+                (s = copy_async(h.b, d.b, cols * 4, cudaMemcpyDeviceToHost, sd)) != DQ_OK ||
+                (s = copy_async(h.tensor_scale, d.tensor_scale, 4, cudaMemcpyDeviceToHost, sd)) != DQ_OK ||
+                (s = copy_async(h.mse_trace, d.mse_trace, ((size_t)T + 1) * 8, cudaMemcpyDeviceToHost, sd)) != DQ_OK ||
+                (s = copy_async(h.mse_half, d.mse_half, (size_t)T * 8, cudaMemcpyDeviceToHost, sd)) != DQ_OK)
+                return s;
+        }
+        i = j;
     }
     return DQ_OK;
 }

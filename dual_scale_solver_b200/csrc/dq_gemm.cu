@@ -178,8 +178,10 @@ __device__ __forceinline__ uint32_t idesc_mxf4(uint32_t sfa_id, uint32_t sfb_id)
 // Output tile t -> (m0, n0).  Tiles go in bands of up to kBandTiles tile
 // columns: within a band every row of tiles is visited before the next band,
 // so the CTAs running together share the band's B tiles (which stay in L2)
-// and each A tile is read once per band.
-constexpr int kBandTiles = 16;
+// and each A tile is read once per band.  8 columns: the 74 CTA pairs (or
+// 148 CTAs on 128 x 256 tiles) running together then cover a roughly square
+// block of the output, which needs the fewest distinct A and B tiles.
+constexpr int kBandTiles = 8;
 __device__ __forceinline__ void tile_coords(int t, int m_tiles, int n_tiles, int bm, int bn,
                                             int &m0, int &n0) {
     const int band = t / (m_tiles * kBandTiles);

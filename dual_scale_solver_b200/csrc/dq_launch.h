@@ -12,6 +12,43 @@
 
 namespace dq {
 
+// Tile geometry of one matrix: wc warp columns of 256 bf16 (128 float32)
+// columns per CTA, ncb column blocks, tr[mode slot] rows per tile and the
+// tile counts; it fixes each tile kernel's traffic (the column partials are
+// one float2 per column per row block of the column statistics).
+struct Geom {
+    int wc, ncb;
+    int tr[3];
+    int64_t ntiles[3];
+    int64_t nrb_col;
+};
+
+inline Geom geometry(int64_t rows, int64_t cols, bool f32) {
+    Geom g{};
+    const int epc = f32 ? 4 : 8, seg = 32 * epc;
+    const int64_t nseg = (cols + seg - 1) / seg;
+    int wc = 1;
+    while (wc < 8 && wc < nseg) wc <<= 1;
+    g.wc = wc;
+    g.ncb = (int)((nseg + wc - 1) / wc);
+    const int wr = kWarps / wc;
+    // rows per warp: 256 for column statistics (fewer partial sums), 128 for
+    // the other modes (tile set-up spread over the rows), both reduced for
+    // short matrices so that they still make about 16 row blocks
+    int rpw_long = 16;
+    while (rpw_long < 128 && 2 * rpw_long <= rows / (wr * 16)) rpw_long *= 2;
+    int rpw_col = rpw_long;
+    while (rpw_col < 256 && 2 * rpw_col <= rows / (wr * 16)) rpw_col *= 2;
+    const int rpw[3] = {rpw_long, rpw_col, rpw_long};
+    for (int m = 0; m < 3; ++m) {
+        g.tr[m] = rpw[m] * wr;
+        const int64_t nrb = (rows + g.tr[m] - 1) / g.tr[m];
+        g.ntiles[m] = (rows > 0 && cols > 0) ? nrb * g.ncb : 0;
+    }
+    g.nrb_col = (rows + g.tr[1] - 1) / g.tr[1];
+    return g;
+}
+
 struct TileLaunch {
     Table tab;
     int64_t grid;       // CTAs launched (tiles are visited grid-stride)

@@ -309,12 +309,15 @@ DQ_API dq_status dq_solve_dual_scale_noalloc(const void *W, int32_t dtype, int64
  *  - dev[i] holds device buffers of the same sizes, caller-owned: W (and
  *    a0 / b0 when host[i] has them) receive the copies of the inputs, the
  *    outputs are written there as by dq_solve_dual_scale and stay there.
- * For each i in order: the inputs are copied on stream `h2d`, the matrix is
- * solved on `compute` once they have landed (one matrix at a time, in
- * `workspace`, which must hold dq_workspace_size bytes for the largest
- * single matrix), and the requested outputs are copied back on `d2h` once
- * its solve is done; so matrix i+1 crosses the bus while matrix i is solved
- * and matrix i-1's results return.  The call only enqueues: the host outputs
+ * The matrices are taken in order in groups of consecutive matrices (about
+ * 1/8 of all the input bytes per group, at least 32 MiB, and no more than
+ * `workspace` can hold as one batched solve; it must hold at least
+ * dq_workspace_size for the largest single matrix, and dq_workspace_size
+ * over all n shapes always lets the groups form fully).  For each group:
+ * its inputs are copied on stream `h2d`, it is solved on `compute` as one
+ * batched solve once they have landed, and the requested outputs are copied
+ * back on `d2h` once that solve is done; so group g+1 crosses the bus while
+ * group g is solved and group g-1's results return.  The call only enqueues: the host outputs
  * are valid once the work queued on `d2h` has completed.  Host memory must
  * be page-locked (cudaHostAlloc / cudaHostRegister) for the copies to
  * overlap; pageable memory works but serialises.  Each call first orders
@@ -322,7 +325,7 @@ DQ_API dq_status dq_solve_dual_scale_noalloc(const void *W, int32_t dtype, int64
  * work already queued on `d2h`, so consecutive calls may reuse the same
  * buffers.  Calls are serialised inside the library (one set of internal
  * events per device).  One cudaMemcpyAsync per buffer.  Results equal
- * dq_solve_dual_scale on each matrix.  Errors: as dq_solve_dual_scale_batched,
+ * dq_solve_dual_scale on each matrix, whatever the grouping.  Errors: as dq_solve_dual_scale_batched,
  * plus DQ_ERR_SHAPE when host[i] and dev[i] disagree and DQ_ERR_ARG when a
  * host input or requested output has no device counterpart; on an error the
  * work already queued stays queued. */

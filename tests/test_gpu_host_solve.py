@@ -34,7 +34,10 @@ def _same(o, r):
 
 @pytest.mark.parametrize("name", ["mxfp4", "int4_bf16", "nvfp4"])
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
-def test_host_solve_equals_device_batched(name, dtype):
+@pytest.mark.parametrize("grouping", ["all", "one"])
+def test_host_solve_equals_device_batched(name, dtype, grouping):
+    # "all": workspace for every shape (the matrices go as one group);
+    # "one": workspace for the largest single matrix (one matrix per group)
     G = {"mxfp4": 32, "int4_bf16": 64, "nvfp4": 16}[name]
     fmt = lib_format(name, G)
     shapes = [(300, 40 * G), (64, 8 * G), (1, G), (517, 24 * G)]
@@ -43,7 +46,11 @@ def test_host_solve_equals_device_batched(name, dtype):
     hW = [W.pin_memory() for W in Ws]
     T = 4
     ref = dq.solve_dual_scale_batched([W.cuda() for W in Ws], fmt, T, half=True)
-    outs, dev_outs = dq.solve_dual_scale_batched_host(hW, fmt, T, half=True)
+    ws = None
+    if grouping == "one":
+        ws = torch.empty(max(dq.workspace_size([s], fmt) for s in shapes), dtype=torch.uint8,
+                         device="cuda")
+    outs, dev_outs = dq.solve_dual_scale_batched_host(hW, fmt, T, half=True, ws=ws)
     torch.cuda.synchronize()
     assert dq.last_device_status() == 0
     for o, d, r in zip(outs, dev_outs, ref):
@@ -74,3 +81,25 @@ def test_host_solve_repeated_calls_reuse_buffers():
         _same(o, r)
     for o, r in zip(outs2, ref2):
         _same(o, r)
+
+
+def test_host_solve_many_small_matrices_in_groups():
+    # 40 small matrices (about 3 MB of inputs): fewer groups than matrices
+    fmt = dq.format_preset("mxint4")
+    g = torch.Generator().manual_seed(5)
+    Ws = [(torch.randn(96 + 32 * (i % 5), 576, generator=g) * 0.02).to(torch.bfloat16)
+          for i in range(40)]
+    ref = dq.solve_dual_scale_batched([W.cuda() for W in Ws], fmt, 5)
+    outs, _ = dq.solve_dual_scale_batched_host([W.pin_memory() for W in Ws], fmt, 5)
+    torch.cuda.synchronize()
+    for o, r in zip(outs, ref):
+        _same(o, r)
+
+
+def test_host_solve_workspace_too_small():
+    fmt = dq.format_preset("mxfp4")
+    W = torch.zeros(256, 1024, dtype=torch.bfloat16).pin_memory()
+    ws = torch.empty(256, dtype=torch.uint8, device="cuda")
+    with pytest.raises(dq.DqError) as e:
+        dq.solve_dual_scale_batched_host([W], fmt, 3, ws=ws)
+    assert e.value.status == -7
