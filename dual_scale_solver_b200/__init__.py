@@ -35,7 +35,7 @@ EXPORTS = ("dq_version", "dq_strerror", "dq_format_preset", "dq_workspace_size",
            "dq_row_update", "dq_col_update", "dq_act_rescale_quant", "dq_last_device_status",
            "dq_kernel_timing", "dq_kernel_time", "dq_launch_count",
            "dq_solve_dual_scale_noalloc", "dq_code_bytes", "dq_two_level_quant", "dq_w4a4_gemm",
-           "dq_scale_tiles", "dq_solve_dual_scale_batched_host")
+           "dq_scale_tiles", "dq_solve_dual_scale_batched_host", "dq_test_stall_next_gemm")
 
 
 class DqError(RuntimeError):
@@ -108,6 +108,7 @@ def lib() -> ctypes.CDLL:
         "dq_w4a4_gemm": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int64,
                                    c_int64, c_int64, P(dq_format), c_void_p, c_void_p]),
         "dq_scale_tiles": (c_int32, [c_void_p, c_int64, c_int64, c_void_p, c_void_p]),
+        "dq_test_stall_next_gemm": (c_int32, []),
         "dq_solve_dual_scale_batched_host": (c_int32, [c_int32, P(dq_matrix), P(dq_matrix), c_int32,
                                                        P(dq_format), c_int32, c_void_p, c_size_t,
                                                        c_void_p, c_void_p, c_void_p]),

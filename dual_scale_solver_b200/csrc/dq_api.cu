@@ -725,6 +725,15 @@ dq_status dq_two_level_quant(const void *X, int32_t dtype, int64_t rows, int64_t
     return DQ_OK;
 }
 
+namespace {
+std::atomic<int> g_stall_next_gemm{0};
+}  // namespace
+
+dq_status dq_test_stall_next_gemm(void) {
+    g_stall_next_gemm.store(1);
+    return DQ_OK;
+}
+
 dq_status dq_w4a4_gemm(const uint8_t *codes_x, const void *scales_x, const uint8_t *codes_w,
                        const void *scales_w, const float *a, int64_t M, int64_t N, int64_t K,
                        const dq_format *fmt, float *out, dq_stream stream) {
@@ -752,6 +761,7 @@ dq_status dq_w4a4_gemm(const uint8_t *codes_x, const void *scales_x, const uint8
     L.N = N;
     L.K = K;
     L.status = status;
+    L.stall = g_stall_next_gemm.exchange(0);
     L.stream = reinterpret_cast<cudaStream_t>(stream);
     DQ_CUDA(launch_w4a4_gemm(L));
     count_launches(1);

@@ -248,7 +248,7 @@ template <int BN, int BK>
 __global__ void __launch_bounds__(kThreadsGemm, GemmSmem<BN, BK>::kCtasPerSm)
 w4a4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                  const uint8_t *sf_a, const uint8_t *sf_b, const float *a_row, float *out, int M,
-                 int N, int K, unsigned int *status) {
+                 int N, int K, unsigned int *status, int stall) {
     using Smem = GemmSmem<BN, BK>;
     constexpr int kStages = Smem::kStages;
     constexpr int KC = Smem::KC;
@@ -289,6 +289,7 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
 
     // The CTA walks the output tiles t = blockIdx.x, + gridDim.x, ... in the
     // band order of tile_coords.
+    int issued = 0;                                 // K tiles the producer issued (warp 0)
     if (warp == 0) {
         // ---- producer (lane 0): per K tile, TMA loads of the two code tiles
         // and bulk copies of their scale tiles (KC consecutive 512-byte
@@ -309,7 +310,9 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
                     if (lane == 0) ok = mbar_wait(&sm.empty[s], ((g / kStages) - 1) & 1, abort, status);
                     if (!__shfl_sync(0xffffffffu, ok, 0)) { stop = true; break; }
                 }
-                if (lane == 0) {
+                // (test support: `stall` leaves the first K tile unloaded, so the
+                // MMA thread's bounded wait for it runs out)
+                if (lane == 0 && !(stall && g == 0)) {
                     mbar_arrive_expect_tx(&sm.full[s], Smem::kStageTx);
                     tma_load_2d(sm.a[s], &map_a, kt * (BK / 2), m0, &sm.full[s]);
                     tma_load_2d(sm.b[s], &map_b, kt * (BK / 2), n0, &sm.full[s]);
@@ -323,11 +326,7 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
                 }
             }
         }
-        // after an abort, let the copies already issued land before the CTA exits
-        if (lane == 0 && *abort) {
-            for (int k = max(0, g - kStages); k < g; ++k)
-                mbar_drain(&sm.full[k % kStages], (k / kStages) & 1);
-        }
+        issued = g;
     } else if (warp == 1) {
         // ---- MMA issuer ----
         if (lane == 0) {
@@ -432,6 +431,13 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
         }
     }
     tc_fence_before();
+    __syncthreads();
+    // after an abort (known to every thread by now), let the copies already
+    // issued land before the CTA frees its resources and exits
+    if (warp == 0 && lane == 0 && *abort) {
+        for (int k = max(0, issued - kStages); k < issued; ++k)
+            mbar_drain(&sm.full[k % kStages], (k / kStages) & 1);
+    }
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
@@ -542,7 +548,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsGemm, 1)
 w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                       const __grid_constant__ CUtensorMap map_sfa,
                       const __grid_constant__ CUtensorMap map_sfb, const float *a_row, float *out,
-                      int M, int N, int K, unsigned int *status) {
+                      int M, int N, int K, unsigned int *status, int stall) {
     using Smem = GemmPairSmem<BK>;
     constexpr int kStages = Smem::kStages;
     constexpr int KC = Smem::KC;
@@ -583,6 +589,7 @@ w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_co
     constexpr uint32_t kSfSlot = 4 * KC * 3;        // two scale slots, as above
     const uint32_t sfa_t0 = tmem + BN, sfb_t0 = tmem + BN + 4 * KC;
 
+    int issued = 0;                                 // K tiles the producer issued (warp 0)
     if (warp == 0) {
         if (lane == 0) {
             // ---- producer: this CTA's halves of every K tile ----
@@ -599,6 +606,7 @@ w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_co
                         stop = true;
                         break;
                     }
+                    if (stall && g == 0) continue;       // test support, as above
                     const uint32_t bar = full0 + (uint32_t)(s * sizeof(uint64_t));
                     if (leader) mbar_arrive_expect_tx(&sm.full[s], Smem::kPairTx);
                     tma_load_2d_pair(sm.a[s], &map_a, kt * (BK / 2), ma, bar);
@@ -610,17 +618,7 @@ w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_co
                                          (int)((n0 / 128 + nb) * kblocks + kt * KC), bar);
                 }
             }
-            if (*abort) {
-                // let the copies already issued land before the CTA exits
-                if (leader) {
-                    for (int k = max(0, g - kStages); k < g; ++k)
-                        mbar_drain(&sm.full[k % kStages], (k / kStages) & 1);
-                } else {
-                    const uint64_t t0 = global_ns();
-                    while (global_ns() - t0 < 2000000ull) {
-                    }
-                }
-            }
+            issued = g;
         }
         __syncwarp();
     } else if (warp == 1) {
@@ -719,6 +717,21 @@ w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_co
     // its barriers or read its TMEM
     tc_fence_before();
     __syncthreads();
+    // after an abort (known to every thread of this CTA by now), let the
+    // copies already issued land: CTA 0's barriers count both CTAs' bytes;
+    // CTA 1 only waits a little, its partner drains before the cluster
+    // barrier below
+    if (warp == 0 && lane == 0 && *abort) {
+        if (leader) {
+            for (int k = max(0, issued - kStages); k < issued; ++k)
+                mbar_drain(&sm.full[k % kStages], (k / kStages) & 1);
+        } else {
+            const uint64_t t0 = global_ns();
+            while (global_ns() - t0 < 2000000ull) {
+            }
+        }
+    }
+    __syncthreads();
     cluster_sync_all();
     if (warp == 1) {
         tc_fence_after();
@@ -811,7 +824,7 @@ cudaError_t launch_pair(const GemmLaunch &L) {
     const int64_t tiles = (L.M / 256) * (L.N / 256);
     const unsigned grid = 2u * (unsigned)std::min<int64_t>(tiles, sms / 2);
     return launch_k(w4a4_gemm_pair_kernel<BK>, dim3(grid), dim3(kThreadsGemm), smem, L.stream, ma, mb,
-                    msa, msb, L.a, L.out, (int)L.M, (int)L.N, (int)L.K, L.status);
+                    msa, msb, L.a, L.out, (int)L.M, (int)L.N, (int)L.K, L.status, L.stall);
 }
 
 template <int BN, int BK>
@@ -838,7 +851,7 @@ cudaError_t launch_bn(const GemmLaunch &L) {
     const int64_t tiles = (L.M / kBM) * (L.N / BN);
     const unsigned grid = (unsigned)std::min<int64_t>(tiles, (int64_t)sms * Smem::kCtasPerSm);
     return launch_k(w4a4_gemm_kernel<BN, BK>, dim3(grid), dim3(kThreadsGemm), smem, L.stream, ma, mb,
-                    L.scales_x, L.scales_w, L.a, L.out, (int)L.M, (int)L.N, (int)L.K, L.status);
+                    L.scales_x, L.scales_w, L.a, L.out, (int)L.M, (int)L.N, (int)L.K, L.status, L.stall);
 }
 
 }  // namespace

@@ -122,6 +122,7 @@ struct GemmLaunch {
     float *out;                          // [M, N]
     int64_t M, N, K;                     // multiples of 128, 128, 256
     unsigned int *status;
+    int stall;                           // test support: skip the loads of the first K tile
     cudaStream_t stream;
 };
 cudaError_t launch_w4a4_gemm(const GemmLaunch &L);

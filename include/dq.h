@@ -264,6 +264,15 @@ DQ_API dq_status dq_w4a4_gemm(const uint8_t *codes_x, const void *scales_x, cons
                               const void *scales_w, const float *a, int64_t M, int64_t N,
                               int64_t K, const dq_format *fmt, float *out, dq_stream stream);
 
+/* Test support for the failure path (no counterpart in the method): the
+ * next dq_w4a4_gemm call on any thread has its producer skip the loads of
+ * its first K tile, so the MMA thread's bounded wait for that tile runs out
+ * (after about 1 s); every CTA then stops issuing work, waits (bounded) for
+ * its copies in flight, frees its TMEM and returns, and the device flag reads
+ * DQ_ERR_TIMEOUT.  The output of that call is undefined.  Nothing faults or
+ * hangs; later calls run normally. */
+DQ_API dq_status dq_test_stall_next_gemm(void);
+
 /* Synchronise `stream`, read and clear the device flags raised by earlier
  * calls on this device: DQ_ERR_NONFINITE if an input held NaN/Inf (or
  * scaling it by the outer scales left the float32 range),

@@ -170,3 +170,24 @@ def test_w4a4_gemm_pair_tile_placement():
     want[200, 130] = 12.0
     want[5, 250] = 2.0
     assert torch.equal(out, want)
+
+
+@pytest.mark.parametrize("M,N", [(256, 256), (128, 128)])       # CTA pair, single CTA
+def test_w4a4_gemm_stalled_pipeline_reports_timeout(M, N):
+    # the producer leaves the first K tile unloaded: the MMA thread's bounded
+    # wait runs out, the kernel returns and raises the timeout flag; the
+    # context stays usable
+    K = 512
+    cx, sx = _random_operand(M, K, 51)
+    cw, sw = _random_operand(N, K, 52)
+    a = torch.ones(N)
+    args = (cx.cuda(), sx.cuda(), cw.cuda(), sw.cuda(), a.cuda())
+    assert dq.last_device_status() == 0
+    dq.lib().dq_test_stall_next_gemm()
+    dq.w4a4_gemm(*args)
+    assert dq.last_device_status() == -11
+    out = dq.w4a4_gemm(*args)
+    torch.cuda.synchronize()
+    assert dq.last_device_status() == 0
+    ref, bound = _reference(cx, sx, cw, sw, a)
+    assert np.all(np.abs(np64(out) - ref) <= bound)
