@@ -18,7 +18,7 @@ __all__ = [
     "workspace_size", "quantize", "dequantize", "solve_dual_scale", "solve_dual_scale_batched",
     "row_update", "col_update", "act_rescale_quant", "last_device_status", "EXPORTS",
     "kernel_timing", "kernel_time", "launch_count", "solve_dual_scale_noalloc", "code_bytes",
-    "two_level_quant", "w4a4_gemm", "scale_tiles", "solve_dual_scale_batched_host",
+    "two_level_quant", "w4a4_gemm", "scale_tiles", "solve_dual_scale_batched_host", "copy_streams",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -319,7 +319,7 @@ def solve_dual_scale_batched(Ws, fmt, T, ws=None, outs=None, half=False, stream=
 _COPY_STREAMS = {}
 
 
-def _copy_streams(device):
+def copy_streams(device):
     """One host-to-device and one device-to-host stream per device (kept)."""
     idx = torch.device(device).index
     idx = torch.cuda.current_device() if idx is None else idx
@@ -350,7 +350,7 @@ def _fill_matrix(m, W, o):
 
 
 def solve_dual_scale_batched_host(Ws, fmt, T, outs=None, dev_outs=None, staging=None, ws=None,
-                                  half=False, device=None, stream=None):
+                                  half=False, device=None, stream=None, wait_out=True):
     """Solve matrices held in host memory (CPU tensors of one dtype; pin them
     for the copies to overlap): matrix i+1 is copied in while matrix i is
     solved and matrix i-1's results are copied back (dq_solve_dual_scale_batched_host).
@@ -359,7 +359,9 @@ def solve_dual_scale_batched_host(Ws, fmt, T, outs=None, dev_outs=None, staging=
     Returns (outs, dev_outs): per matrix a dict of page-locked CPU tensors and
     one of the device tensors holding the same results.  `stream` (default:
     the current stream) runs the solves and, on return, also waits for the
-    copies back, so work ordered after it sees the host results.  `outs`,
+    copies back, so work ordered after it sees the host results (with
+    wait_out=False it does not: the caller orders its reads after
+    `copy_streams(device)[1]`, the copy-back stream).  `outs`,
     `dev_outs`, `staging` (device copies of W) and `ws` may be passed back in
     to reuse them."""
     n = len(Ws)
@@ -383,12 +385,13 @@ def solve_dual_scale_batched_host(Ws, fmt, T, outs=None, dev_outs=None, staging=
         _fill_matrix(host[i], Ws[i], outs[i])
         _fill_matrix(devm[i], staging[i], dev_outs[i])
     compute = stream if stream is not None else torch.cuda.current_stream(dev)
-    h2d, d2h = _copy_streams(dev)
+    h2d, d2h = copy_streams(dev)
     _check(lib().dq_solve_dual_scale_batched_host(n, host, devm, dt, ctypes.byref(fmt), T, _ptr(ws),
                                                   ws.numel(), compute.cuda_stream, h2d.cuda_stream,
                                                   d2h.cuda_stream),
            "dq_solve_dual_scale_batched_host")
-    compute.wait_stream(d2h)
+    if wait_out:
+        compute.wait_stream(d2h)
     return outs, dev_outs
 
 
