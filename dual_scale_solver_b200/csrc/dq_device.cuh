@@ -822,23 +822,24 @@ tile_kernel(const __grid_constant__ Table tab, int mode_slot, int want_res, int6
                 }
             }
             const float2 share = make_float2((gn.x + gn.y) * s_row, (gd.x + gd.y) * (s_row * s_row));
-            // batches of 8 rows: lane 2r + h adds the 16 shares of half h of
-            // the batch's row r in order, then the halves are added (a fixed
-            // order, the same in every mode with row statistics)
+            // batches of 8 rows: lane 4r + q adds the 8 shares of quarter q
+            // of the batch's row r as a fixed tree, then the quarters are
+            // added ((q0 + q1) + (q2 + q3), by two shuffle levels) -- one
+            // fixed order, the same in every mode with row statistics
             sm.red[(warp * 8 + (k & 7)) * 33 + lane] = share;
             if (batch_end) {
                 __syncwarp();
-                const int rr = (lane >> 1) & 7, hh = lane & 1;
-                const float2 *p = &sm.red[(warp * 8 + rr) * 33 + 16 * hh];
-                f2 acc = bcast(0.0f);
-                if (lane < 16) {
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) acc = __fadd2_rn(acc, p[j]);
-                }
+                const int rr = lane >> 2, qq = lane & 3;
+                const float2 *p = &sm.red[(warp * 8 + rr) * 33 + 8 * qq];
+                const f2 s01 = __fadd2_rn(p[0], p[1]), s23 = __fadd2_rn(p[2], p[3]);
+                const f2 s45 = __fadd2_rn(p[4], p[5]), s67 = __fadd2_rn(p[6], p[7]);
+                f2 acc = __fadd2_rn(__fadd2_rn(s01, s23), __fadd2_rn(s45, s67));
                 acc.x += __shfl_xor_sync(0xffffffffu, acc.x, 1);
                 acc.y += __shfl_xor_sync(0xffffffffu, acc.y, 1);
+                acc.x += __shfl_xor_sync(0xffffffffu, acc.x, 2);
+                acc.y += __shfl_xor_sync(0xffffffffu, acc.y, 2);
                 const int kk = (k & ~7) + rr;
-                if (lane < 16 && hh == 0 && kk <= k) sm.rtot[kk * kWarps + warp] = acc;
+                if (qq == 0 && kk <= k) sm.rtot[kk * kWarps + warp] = acc;
                 __syncwarp();
             }
         }
