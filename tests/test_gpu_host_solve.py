@@ -103,3 +103,18 @@ def test_host_solve_workspace_too_small():
     with pytest.raises(dq.DqError) as e:
         dq.solve_dual_scale_batched_host([W], fmt, 3, ws=ws)
     assert e.value.status == -7
+
+
+def test_host_solve_empty_and_zero_matrices():
+    # a matrix with no rows and an all-zero matrix among ordinary ones
+    fmt = dq.format_preset("mxfp4")
+    g = torch.Generator().manual_seed(9)
+    Ws = [torch.zeros(0, 64, dtype=torch.bfloat16), torch.zeros(40, 96, dtype=torch.bfloat16),
+          (torch.randn(64, 128, generator=g) * 0.02).to(torch.bfloat16)]
+    ref = dq.solve_dual_scale_batched([W.cuda() for W in Ws], fmt, 3)
+    outs, _ = dq.solve_dual_scale_batched_host([W.pin_memory() for W in Ws], fmt, 3)
+    torch.cuda.synchronize()
+    assert dq.last_device_status() == 0
+    for o, r in zip(outs, ref):
+        _same(o, r)
+    assert torch.all(outs[1]["codes"] == 0) and torch.all(outs[1]["mse_trace"] == 0)
