@@ -20,6 +20,7 @@ the max-over-ranks of the timings.
 from __future__ import annotations
 
 import argparse
+import datetime
 import hashlib
 import glob
 import json
@@ -41,7 +42,7 @@ UNIT = "weight-elements/s"
 def _args():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=10)
+    p.add_argument("--steps", type=int, default=50)
     p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--config", default=DEFAULT_CONFIG)
@@ -99,21 +100,29 @@ def _traffic(kind_name):
 
 
 class Clocks:
-    """nvidia-smi sampling of SM clock and throttle reasons during timing."""
+    """nvidia-smi sampling (every 50 ms) of SM clock and throttle reasons; the
+    samples whose timestamps fall inside the host-side window around the timed
+    loop (mark("t0") before it, mark("t1") after its final synchronize) are the
+    ones reported (window "timed"); a window too short to hold one sample
+    reports those within 0.25 s of it (window "near")."""
 
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    Q = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, index):
         self.index = index
         self.proc = None
+        self.t0 = self.t1 = None
+
+    def mark(self, which):
+        setattr(self, which, datetime.datetime.now())
 
     def start(self):
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
@@ -127,23 +136,33 @@ class Clocks:
         except subprocess.TimeoutExpired:
             self.proc.kill()
             out, _ = self.proc.communicate()
-        sm, mx, reasons = [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        rows = []
         for line in out.strip().splitlines():
             f = [x.strip() for x in line.split(",")]
-            if len(f) < 9:
+            if len(f) < 10:
                 continue
             try:
-                sm.append(float(f[1]))
-                mx.append(float(f[2]))
+                ts = datetime.datetime.strptime(f[0], "%Y/%m/%d %H:%M:%S.%f")
+                rows.append((ts, float(f[2]), float(f[3]),
+                             [n for n, v in zip(names, f[6:10]) if v.lower() == "active"]))
             except ValueError:
                 continue
-            for n, v in zip(names, f[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
+        window = "all"
+        if self.t0 is not None and self.t1 is not None:
+            inside = [r for r in rows if self.t0 <= r[0] <= self.t1]
+            pad = datetime.timedelta(seconds=0.25)
+            near = [r for r in rows if self.t0 - pad <= r[0] <= self.t1 + pad]
+            if inside:
+                rows, window = inside, "timed"
+            elif near:
+                rows, window = near, "near"
+        sm = [r[1] for r in rows]
+        mx = [r[2] for r in rows]
+        reasons = sorted({n for r in rows for n in r[3]})
         return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(sm), "window": window}
 
 
 # --------------------------------------------------------------------------- #
@@ -314,11 +333,13 @@ def run_ours(args, wl, rank, world, local_rank):
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize(dev)
+    clocks.mark("t0")
     e0.record(stream)
     for _ in range(args.steps):
         step()
     e1.record(stream)
     torch.cuda.synchronize(dev)
+    clocks.mark("t1")
     barrier()
     ms = e0.elapsed_time(e1)
     launches = dq.launch_count() - n0
@@ -488,11 +509,13 @@ def run_two_level(args, wl, rank, world, local_rank):
           for _ in range(args.steps)]
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize(dev)
+    clocks.mark("t0")
     e0.record(stream)
     for k in range(args.steps):
         step(ev[k])
     e1.record(stream)
     torch.cuda.synchronize(dev)
+    clocks.mark("t1")
     ms = max_over_ranks(e0.elapsed_time(e1), dev) / args.steps
     launches = dq.launch_count() - n0
     clk = clocks.stop()
@@ -595,11 +618,14 @@ def run_gemm(args, wl, rank, world, local_rank):
     time.sleep(0.3)
     n0 = dq.launch_count()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    clocks.mark("t0")
     e0.record(stream)
     for _ in range(args.steps):
         step()
     e1.record(stream)
     torch.cuda.synchronize(dev)
+    clocks.mark("t1")
     ms = max_over_ranks(e0.elapsed_time(e1), dev) / args.steps
     launches = dq.launch_count() - n0
     clk = clocks.stop()
