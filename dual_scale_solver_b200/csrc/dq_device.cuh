@@ -452,9 +452,16 @@ struct Quant {
         cw[1] = 0;
         if constexpr (CODES == CODES_INT4 || CODES == CODES_INT8) {
             // round half to even; |q| <= qmax (E8M0 round-up) or < qmax + 0.5
-            // (BF16 nearest, INT4 only) so the codebook clamp never binds
+            // (BF16 nearest, INT4 only) so the codebook clamp never binds.
+            // Adding and subtracting 1.5 * 2^23 rounds any |q| < 2^22 to the
+            // nearest integer, ties to even (the sum lies in [2^23, 2^24),
+            // where the spacing is 1; the subtraction is exact), on the FMA
+            // pipe; a negative q that rounds to zero gives +0, which encodes
+            // as the same integer code.
+            constexpr float kRound = 12582912.0f;   // 1.5 * 2^23
 #pragma unroll
-            for (int k = 0; k < NP; ++k) c[k] = make_float2(rintf(q[k].x), rintf(q[k].y));
+            for (int k = 0; k < NP; ++k)
+                c[k] = __fadd2_rn(__fadd2_rn(q[k], bcast(kRound)), bcast(-kRound));
             if (!kExactQ) {
                 // largest distance of q from its rounded value: near 0.5 only
                 // when some element sits within 2^-16 of a half-integer
