@@ -633,8 +633,12 @@ def run_gemm(args, wl, rank, world, local_rank):
         raise RuntimeError("device status flags raised during timing")
     flops = sum(2.0 * M * o["codes"].shape[0] * 2 * o["codes"].shape[1] for o in outs)
     peaks, which = _peaks()
-    # FP4 dense peak = the measured bf16 GEMM peak x the nominal fp4/bf16 ratio (9 / 2.25)
-    peak = float(peaks.get("bf16_tflops", 1590.0)) * 4.0
+    # FP4 dense peak = the measured bf16 GEMM peak x the nominal fp4/bf16 ratio (9 / 2.25);
+    # a timed region of more than half a second of back-to-back products runs
+    # under the power cap, so it is held against the sustained bf16 figure
+    sustained = ms * args.steps > 500.0 and "bf16_tflops_sustained" in peaks
+    peak_key = "bf16_tflops_sustained" if sustained else "bf16_tflops"
+    peak = float(peaks.get(peak_key, 1590.0)) * 4.0
     tflops = flops / (ms / 1e3) / 1e12
     line = {
         "metric": "W4A4 GEMM TFLOP/s (MXFP4 x MXFP4, E8M0 scales, fp32 accumulate)",
@@ -647,7 +651,8 @@ def run_gemm(args, wl, rank, world, local_rank):
                    "parallelism": f"{world} independent decoders" if world > 1 else "1 GPU"},
         "roofline": {"bound": "tensor", "achieved": tflops, "peak": peak, "unit": "TFLOP/s",
                      "frac": tflops / peak,
-                     "peak_source": f"{which} bf16 x 4 (nominal fp4/bf16 ratio)",
+                     "peak_source": f"{which} {'sustained' if sustained else 'burst'} bf16 x 4 "
+                                    f"(nominal fp4/bf16 ratio; timed region {ms * args.steps / 1e3:.2f} s)",
                      "traffic": None},
         "gpu_launches": launches, "clocks": clk, "e2e": None,
     }
