@@ -809,15 +809,11 @@ cudaError_t launch_pair(const GemmLaunch &L) {
         !scale_tile_map(&msb, L.scales_w, L.N, L.K, Smem::KC))
         return cudaErrorInvalidValue;
     const size_t smem = sizeof(Smem) + 1024;
-    static bool done[64] = {};
+    static std::atomic<bool> done[64];
+    cudaError_t e = smem_opt_in(w4a4_gemm_pair_kernel<BK>, smem, done);
+    if (e != cudaSuccess) return e;
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    if (!done[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(w4a4_gemm_pair_kernel<BK>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        done[dev] = true;
-    }
+    if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
     // persistent: one CTA pair per two SMs, or fewer tiles
     int sms = 148;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) sms = 148;
@@ -836,15 +832,11 @@ cudaError_t launch_bn(const GemmLaunch &L) {
     if (!code_map(&ma, L.codes_x, L.M, L.K, kBM, BK / 2) || !code_map(&mb, L.codes_w, L.N, L.K, BN, BK / 2))
         return cudaErrorInvalidValue;
     const size_t smem = sizeof(Smem) + 1024;
-    static bool done[64] = {};
+    static std::atomic<bool> done[64];
+    cudaError_t e = smem_opt_in(w4a4_gemm_kernel<BN, BK>, smem, done);
+    if (e != cudaSuccess) return e;
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    if (!done[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(w4a4_gemm_kernel<BN, BK>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        done[dev] = true;
-    }
+    if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
     // persistent: kCtasPerSm CTAs per SM, or fewer tiles
     int sms = 148;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) sms = 148;

@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <utility>
 
 #include "dq_device.cuh"
@@ -143,6 +144,22 @@ cudaError_t launch_tile_c8(const TileLaunch &L);
 cudaError_t launch_tile_c9(const TileLaunch &L);
 cudaError_t launch_tile_c10(const TileLaunch &L);
 
+// Raise a kernel's dynamic shared-memory limit on the current device, once
+// per device and kernel (`done`: one flag per device, owned by the caller's
+// instantiation).  Host threads racing on the first call both make the same
+// idempotent attribute call.
+template <typename K>
+cudaError_t smem_opt_in(K kern, size_t bytes, std::atomic<bool> (&done)[64]) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!done[dev].load(std::memory_order_acquire)) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+        if (e != cudaSuccess) return e;
+        done[dev].store(true, std::memory_order_release);
+    }
+    return cudaSuccess;
+}
+
 // One tile-kernel launch; the shared memory is dynamic (the row-statistics
 // layout needs more than the 48 KB default, opted in once per device).
 template <int CODES, int GS, int OS, int MODE, typename TIn, int G>
@@ -150,15 +167,9 @@ cudaError_t launch_tile_one(const TileLaunch &L) {
     constexpr size_t bytes = sizeof(TileSmem<MODE, Chunk<TIn>::EPC>);
     auto kern = tile_kernel<CODES, GS, OS, MODE, TIn, G>;
     if (bytes > 48 * 1024) {
-        static bool done[64] = {};
-        int dev = 0;
-        if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-        if (!done[dev]) {
-            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 (int)bytes);
-            if (e != cudaSuccess) return e;
-            done[dev] = true;
-        }
+        static std::atomic<bool> done[64];
+        cudaError_t e = smem_opt_in(kern, bytes, done);
+        if (e != cudaSuccess) return e;
     }
     return launch_k(kern, dim3((unsigned)L.grid), dim3(kThreads), bytes, L.stream, L.tab, L.slot,
                     L.want_res, L.tiles, L.flags, L.gate);
