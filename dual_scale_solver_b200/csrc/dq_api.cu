@@ -588,6 +588,8 @@ dq_status dq_format_preset(const char *name, int32_t group, dq_format *out) {
     else if (!strcmp(name, "mxfp8_e5m2")) f = {DQ_CODES_E5M2, 32, DQ_SCALE_E8M0, DQ_SCALE_E8M0, 0};
     else if (!strcmp(name, "mxfp6_e2m3")) f = {DQ_CODES_E2M3, 32, DQ_SCALE_E8M0, DQ_SCALE_E8M0, 0};
     else if (!strcmp(name, "mxfp6_e3m2")) f = {DQ_CODES_E3M2, 32, DQ_SCALE_E8M0, DQ_SCALE_E8M0, 0};
+    else if (!strcmp(name, "mxint4_bf16outer")) f = {DQ_CODES_INT4, 32, DQ_SCALE_E8M0, DQ_SCALE_BF16, 0};
+    else if (!strcmp(name, "mxfp4_bf16outer")) f = {DQ_CODES_E2M1, 32, DQ_SCALE_E8M0, DQ_SCALE_BF16, 0};
     else return DQ_ERR_FORMAT;
     if (group != 0) f.group = group;
     dq_status s = check_format(&f, nullptr);

@@ -123,8 +123,9 @@ DQ_API const char *dq_strerror(dq_status s);
  * and outer scales, default G 64), "mxint4" (INT4, E8M0, E8M0, G 32),
  * "mxfp4" (E2M1, E8M0, E8M0, G 32), "nvfp4" (E2M1, E4M3 group, BF16 outer,
  * G 16, tensor_scale_auto); the rest of the MX family, all E8M0/E8M0 and
- * G 32: "mxint8", "mxfp8_e4m3", "mxfp8_e5m2", "mxfp6_e2m3", "mxfp6_e3m2".
- * group == 0 keeps the preset's G.  Presets follow the formats of Table 1 of
+ * G 32: "mxint8", "mxfp8_e4m3", "mxfp8_e5m2", "mxfp6_e2m3", "mxfp6_e3m2";
+ * the MX block formats with BF16 outer scales (E8M0 group scales, G 32):
+ * "mxint4_bf16outer", "mxfp4_bf16outer".  group == 0 keeps the preset's G.  Presets follow the formats of Table 1 of
  * the daiwk note, the news article's MXFP4/NVFP4 description and its claim of
  * the whole MX family.  Errors: DQ_ERR_ARG (null), DQ_ERR_FORMAT (unknown
  * name or G). */

@@ -93,6 +93,11 @@ PRESETS = {
     "mxfp6_e2m3": Format("e2m3", 32, "e8m0", "e8m0"),
     "mxfp6_e3m2": Format("e3m2", 32, "e8m0", "e8m0"),
     "mxint8": Format("int8", 32, "e8m0", "e8m0"),
+    # the scale-set variant: MX blocks (E8M0 group scales) with BF16 outer
+    # scales (daiwk note, 本地复现: the reproduction selects the scale format
+    # with a command-line flag, so group and outer sets are a choice)
+    "mxint4_bf16outer": Format("int4", 32, "e8m0", "bf16"),
+    "mxfp4_bf16outer": Format("e2m1", 32, "e8m0", "bf16"),
 }
 
 

@@ -189,6 +189,13 @@ for _f in ("mxint8", "mxfp8_e4m3", "mxfp8_e5m2", "mxfp6_e2m3", "mxfp6_e3m2"):
         _base, name=f"llama31_70b_decoder_{_f}_g32", fmt=_f, act=dict(_base.act, fmt=_f))
 
 
+# The same weights with BF16 outer scales (the scale-set variant: E8M0
+# group scales, BF16 a and b); the activations stay MXFP4.
+WORKLOADS["llama31_70b_decoder_mxfp4_bf16outer_g32"] = replace(
+    WORKLOADS["llama31_70b_decoder_mxfp4_g32"], name="llama31_70b_decoder_mxfp4_bf16outer_g32",
+    fmt="mxfp4_bf16outer")
+
+
 def outlier_count(n: int, frac: float) -> int:
     return int(math.floor(n * frac + 0.5))
 

@@ -40,7 +40,8 @@ def test_version_and_errors():
     ("int4_bf16", 0, 0, 0, 64, 0), ("mxint4", 0, 1, 1, 32, 0),
     ("mxfp4", 1, 1, 1, 32, 0), ("nvfp4", 1, 2, 0, 16, 1),
     ("mxint8", 2, 1, 1, 32, 0), ("mxfp8_e4m3", 3, 1, 1, 32, 0), ("mxfp8_e5m2", 4, 1, 1, 32, 0),
-    ("mxfp6_e2m3", 5, 1, 1, 32, 0), ("mxfp6_e3m2", 6, 1, 1, 32, 0)])
+    ("mxfp6_e2m3", 5, 1, 1, 32, 0), ("mxfp6_e3m2", 6, 1, 1, 32, 0),
+    ("mxint4_bf16outer", 0, 1, 0, 32, 0), ("mxfp4_bf16outer", 1, 1, 0, 32, 0)])
 def test_presets(name, codes, gs, os_, G, auto):
     f = dq.format_preset(name)
     assert (f.codes, f.group_scale, f.outer_scale, f.group, f.tensor_scale_auto) == (codes, gs, os_, G, auto)
