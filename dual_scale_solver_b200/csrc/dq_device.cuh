@@ -372,25 +372,38 @@ struct Quant {
     static constexpr float kQmax = CodeTraits<CODES>::kQmax;
     static constexpr int kBits = CodeTraits<CODES>::kBits;
 
+    // Bits of the E8M0 group scale of an exact, finite group max with bits
+    // mb: the smallest 2^e with qmax 2^e >= m, e = E(m) - E(qmax), plus 1
+    // when m's significand exceeds qmax's (the carry of the addition adds it
+    // to the exponent field); at least 2^-126 (also for subnormal and zero
+    // m).  Non-decreasing in mb over finite values.
+    __device__ __forceinline__ static uint32_t e8m0_scale_bits(uint32_t mb) {
+        constexpr uint32_t MT = CodeTraits<CODES>::kMT;
+        constexpr int QE = CodeTraits<CODES>::kQE;
+        return (uint32_t)max((int)((mb + (0x7FFFFFu - MT)) & 0x7F800000u) - (QE << 23), 1 << 23);
+    }
+
     // In: w (input values), z = inner-scaled values before the row factor
     // (w/b_j for weights, x*b_j for activations), a and ia = 1/a (1 for ACT),
     // bj (b_j; read on the exact path only), ts and 1/ts (E4M3 only).
     // Out: c (code values), s (stored group scale), s_eff = s*ts, cw (the
     // chunk's stored codes, element 0 lowest, kBits each -- 4-bit codes two
     // per byte, 8-bit codes one per byte, 6-bit codes four per 3 bytes; only
-    // when NIB).
+    // when NIB), nonzero (the group max is positive and finite), mbits (the
+    // bits of the group max).
     template <bool NIB>
     __device__ __forceinline__ static void run(const f2 (&w)[NP], const f2 (&z)[NP], float a,
                                                float ia, const f2 (&bj)[NP], float ts,
                                                float inv_ts, unsigned int *status, f2 (&c)[NP],
                                                float &s, float &s_eff, uint32_t (&cw)[2],
-                                               bool &nonzero) {
+                                               bool &nonzero, uint32_t &mbits) {
         float mz = 0.0f;
 #pragma unroll
         for (int k = 0; k < NP; ++k) mz = max3_nan(mz, fabsf(z[k].x), fabsf(z[k].y));
         mz = grp_max<LPG>(mz);
         const float m = ACT ? mz : mz * ia;
         const uint32_t mb = __float_as_uint(m);
+        mbits = mb;
         const bool finite = (mb & 0x7F800000u) != 0x7F800000u;
         // row and column statistics carry a NaN/Inf into their sums, which the
         // finalize kernels flag; the other modes flag it here
@@ -398,14 +411,8 @@ struct Quant {
         const bool pos = finite && m > 0.0f;
         nonzero = pos;
         if (GS == SC_E8M0 && kExactM) {
-            // smallest 2^e with qmax 2^e >= m (m exact): e = E(m) - E(qmax),
-            // plus 1 when m's significand exceeds qmax's; e >= -126 (also
-            // covers subnormal m); e <= 126 holds for finite m
-            constexpr uint32_t MT = CodeTraits<CODES>::kMT;
-            constexpr int QE = CodeTraits<CODES>::kQE;
-            // (the carry of the addition below adds that 1 to the exponent field)
-            const int sb = max((int)((mb + (0x7FFFFFu - MT)) & 0x7F800000u) - (QE << 23), 1 << 23);
-            s = __uint_as_float((uint32_t)sb);
+            // (e <= 126 holds for finite m)
+            s = __uint_as_float(e8m0_scale_bits(mb));
             if (NIB && !pos) s = 1.0f;                     // stored scale of an all-zero group
         } else {
             // every lane takes part in the warp vote and group shuffles below,
@@ -749,7 +756,9 @@ tile_kernel(const __grid_constant__ Table tab, int mode_slot, int want_res, int6
 #pragma unroll
     for (int k = 0; k < NP; ++k) { acc_p[k] = bcast(0.0f); acc_e[k] = bcast(0.0f); }
     f2 res2 = bcast(0.0f);
-    bool clamp_risk = false;                         // FUSED: exponent margin check
+    // FUSED: smallest (bits - 1, unsigned: zero groups drop out) and largest
+    // bits of the lane's group maxima, for the exponent margin check
+    uint32_t m_lo = 0xFFFFFFFFu, m_hi = 0u;
 
     // Each lane streams its own 16-byte chunk of the warp's rows through a
     // private ring of kRing shared-memory slots with cp.async (one commit
@@ -793,34 +802,44 @@ tile_kernel(const __grid_constant__ Table tab, int mode_slot, int want_res, int6
 #pragma unroll
         for (int j = 0; j < NP; ++j) z[j] = mul2(w[j], cm[j]);
         float s, s_eff;
-        uint32_t cw[2];
+        uint32_t cw[2], mbits;
         bool nonzero;
         if (FUSED) {
             // Q(W / b): with power-of-two scales D_a Q(W / (a b)) equals it
             // exactly, for the row's a before and after its update, as long
             // as no group exponent of either reaches the E8M0 bounds: here
-            // |e(s)| <= 100 for every non-zero group; the row finalize keeps
-            // |e(a)| <= 20 (old) and <= 26 (new)
+            // |e(s)| <= 100 for every non-zero group (checked after the
+            // tile's rows on the extremes of the group maxima); the row
+            // finalize keeps |e(a)| <= 20 (old) and <= 26 (new)
             Q::template run<NIB>(w, z, 1.0f, 1.0f, bj, ts, inv_ts, tab.status, c, s, s_eff, cw,
-                                 nonzero);
-            // s = 2^e with |e| <= 100: exponent field in [27, 227]
-            clamp_risk |= nonzero && (__float_as_uint(s) - (27u << 23)) > (200u << 23);
+                                 nonzero, mbits);
+            m_lo = min(m_lo, mbits - 1u);
+            m_hi = max(m_hi, mbits);
         } else {
             Q::template run<NIB>(w, z, a, ia, bj, ts, inv_ts, tab.status, c, s, s_eff, cw,
-                                 nonzero);
+                                 nonzero, mbits);
+        }
+        // FUSED: S = Qhat s (a = 1), shared by both statistics
+        f2 v[NP];
+        if (FUSED) {
+#pragma unroll
+            for (int j = 0; j < NP; ++j) v[j] = mul2(c[j], bcast(s_eff));
         }
         if (ROWSTAT) {
             // the row statistics of the literal row step: R = Qhat D_b with
             // Qhat = Q(W / (a b)); FUSED writes them for a = 1 and the row
             // finalize scales the sums by 1/a and 1/a^2 (exact: a is a power
             // of two), which gives the literal bits
+            // (FUSED takes the group scale into R first: R = (Qhat s) b_j.
+            // Scaling by a power of two commutes with rounding, so the
+            // sums and the share are the same bits as the literal form's
+            // while every value stays in float32's normal range.)
             const float s_row = s_eff;
-            const float as = FUSED ? s_eff : a * s_eff;
             f2 gn = bcast(0.0f), gd = bcast(0.0f);
-            const f2 nas = bcast(-as);
+            const f2 nas = bcast(FUSED ? -1.0f : -(a * s_eff));
 #pragma unroll
             for (int j = 0; j < NP; ++j) {
-                const f2 uq = mul2(c[j], bj[j]);
+                const f2 uq = FUSED ? mul2(v[j], bj[j]) : mul2(c[j], bj[j]);
                 gn = fma2(w[j], uq, gn);
                 gd = fma2(uq, uq, gd);
                 if (res_on) {
@@ -828,7 +847,9 @@ tile_kernel(const __grid_constant__ Table tab, int mode_slot, int want_res, int6
                     res2 = fma2(d, d, res2);
                 }
             }
-            const float2 share = make_float2((gn.x + gn.y) * s_row, (gd.x + gd.y) * (s_row * s_row));
+            const float2 share =
+                FUSED ? make_float2(gn.x + gn.y, gd.x + gd.y)
+                      : make_float2((gn.x + gn.y) * s_row, (gd.x + gd.y) * (s_row * s_row));
             // batches of 8 rows: lane 4r + q adds the 8 shares of quarter q
             // of the batch's row r as a fixed tree, then the quarters are
             // added ((q0 + q1) + (q2 + q3), by two shuffle levels) -- one
@@ -852,14 +873,14 @@ tile_kernel(const __grid_constant__ Table tab, int mode_slot, int want_res, int6
         }
         if (COLSTAT) {
             // the column statistics of the literal column step: S = D_a Qhat
-            const f2 as = bcast(FUSED ? s_eff : a * s_eff);
+            const f2 as = bcast(a * s_eff);
 #pragma unroll
             for (int j = 0; j < NP; ++j) {
-                const f2 v = mul2(c[j], as);
-                acc_p[j] = fma2(w[j], v, acc_p[j]);
-                acc_e[j] = fma2(v, v, acc_e[j]);
+                const f2 sv = FUSED ? v[j] : mul2(c[j], as);
+                acc_p[j] = fma2(w[j], sv, acc_p[j]);
+                acc_e[j] = fma2(sv, sv, acc_e[j]);
                 if (!FUSED && res_on) {
-                    const f2 d = fma2(v, bj[j], neg2(w[j]));
+                    const f2 d = fma2(sv, bj[j], neg2(w[j]));
                     res2 = fma2(d, d, res2);
                 }
             }
@@ -916,9 +937,13 @@ tile_kernel(const __grid_constant__ Table tab, int mode_slot, int want_res, int6
     int k0 = 0;
 #pragma unroll 1
     for (; k0 + GRP <= nk; k0 += GRP) {
+        // FUSED: k0 is a multiple of 8 and row k0 + 7 exists, so the group's
+        // last row closes the batch and no other row does (a compile-time
+        // fact; the other modes keep the run-time test, which the compiler
+        // schedules with fewer registers live across rows)
 #pragma unroll
         for (int u = 0; u < GRP; ++u)
-            one_row(k0 + u, u, ((k0 + u) & 7) == 7 || k0 + u == nk - 1);
+            one_row(k0 + u, u, FUSED ? u == GRP - 1 : (((k0 + u) & 7) == 7 || k0 + u == nk - 1));
     }
 #pragma unroll
     for (int u = 0; u < GRP - 1; ++u) {
@@ -926,7 +951,14 @@ tile_kernel(const __grid_constant__ Table tab, int mode_slot, int want_res, int6
         one_row(k0 + u, u, k0 + u == nk - 1 || ((k0 + u) & 7) == 7);
     }
     asm volatile("cp.async.wait_all;" ::: "memory");
-    if (FUSED && clamp_risk) atomicOr(&flags[0], 1u);
+    if (FUSED && m_lo != 0xFFFFFFFFu) {
+        // some group max is non-zero: its scale must be 2^e with |e| <= 100
+        // (exponent field in [27, 227]); the scale bits grow with the max,
+        // so the extremes decide; a non-finite max also takes the literal
+        // passes (which carry it into the sums as well)
+        const uint32_t lo = Q::e8m0_scale_bits(m_lo + 1u), hi = Q::e8m0_scale_bits(m_hi);
+        if (lo < (27u << 23) || hi > (227u << 23) || m_hi >= 0x7F800000u) atomicOr(&flags[0], 1u);
+    }
 
     // ---- tile epilogue ----
     if (ROWSTAT) {
