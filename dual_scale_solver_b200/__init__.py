@@ -19,6 +19,7 @@ __all__ = [
     "row_update", "col_update", "act_rescale_quant", "last_device_status", "EXPORTS",
     "kernel_timing", "kernel_time", "launch_count", "solve_dual_scale_noalloc", "code_bytes",
     "two_level_quant", "w4a4_gemm", "scale_tiles", "solve_dual_scale_batched_host", "copy_streams",
+    "SolveGraph", "solve_dual_scale_batched_graph",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -35,7 +36,8 @@ EXPORTS = ("dq_version", "dq_strerror", "dq_format_preset", "dq_workspace_size",
            "dq_row_update", "dq_col_update", "dq_act_rescale_quant", "dq_last_device_status",
            "dq_kernel_timing", "dq_kernel_time", "dq_launch_count",
            "dq_solve_dual_scale_noalloc", "dq_code_bytes", "dq_two_level_quant", "dq_w4a4_gemm",
-           "dq_scale_tiles", "dq_solve_dual_scale_batched_host", "dq_test_stall_next_gemm")
+           "dq_scale_tiles", "dq_solve_dual_scale_batched_host", "dq_test_stall_next_gemm",
+           "dq_graph_solve_batched", "dq_graph_launch", "dq_graph_launches", "dq_graph_destroy")
 
 
 class DqError(RuntimeError):
@@ -109,6 +111,11 @@ def lib() -> ctypes.CDLL:
                                    c_int64, c_int64, P(dq_format), c_void_p, c_void_p]),
         "dq_scale_tiles": (c_int32, [c_void_p, c_int64, c_int64, c_void_p, c_void_p]),
         "dq_test_stall_next_gemm": (c_int32, []),
+        "dq_graph_solve_batched": (c_int32, [c_int32, P(dq_matrix), c_int32, P(dq_format), c_int32,
+                                             c_void_p, c_size_t, P(c_void_p)]),
+        "dq_graph_launch": (c_int32, [c_void_p, c_void_p]),
+        "dq_graph_launches": (c_int64, [c_void_p]),
+        "dq_graph_destroy": (c_int32, [c_void_p]),
         "dq_solve_dual_scale_batched_host": (c_int32, [c_int32, P(dq_matrix), P(dq_matrix), c_int32,
                                                        P(dq_format), c_int32, c_void_p, c_size_t,
                                                        c_void_p, c_void_p, c_void_p]),
@@ -278,12 +285,10 @@ def solve_dual_scale_noalloc(W, fmt, T, a0=None, b0=None, half=True, stream=None
                 mse_half=mhalf[:T] if half else None)
 
 
-def solve_dual_scale_batched(Ws, fmt, T, ws=None, outs=None, half=False, stream=None):
-    """Solve a list of independent matrices (same dtype) in one launch sequence.
-    ``outs`` (optional) is a list of dicts as returned by this function, reused."""
+def _batch(Ws, fmt, T, ws, outs, half):
+    """The dq_matrix array of a batch (outputs and workspace allocated when
+    not given): (mats, dtype code, outs, ws)."""
     n = len(Ws)
-    if n == 0:
-        return []
     dt = _dtype_code(Ws[0])
     dev = Ws[0].device
     if outs is None:
@@ -310,10 +315,63 @@ def solve_dual_scale_batched(Ws, fmt, T, ws=None, outs=None, half=False, stream=
         m.codes, m.gscales = _ptr(o["codes"]), _ptr(o["gscales"])
         m.a, m.b, m.tensor_scale = _ptr(o["a"]), _ptr(o["b"]), _ptr(o["tensor_scale"])
         m.mse_trace, m.mse_half = _ptr(o["mse_trace"]), _ptr(o.get("mse_half"))
-    _check(lib().dq_solve_dual_scale_batched(n, mats, dt, ctypes.byref(fmt), T, _ptr(ws),
+    return mats, dt, outs, ws
+
+
+def solve_dual_scale_batched(Ws, fmt, T, ws=None, outs=None, half=False, stream=None):
+    """Solve a list of independent matrices (same dtype) in one launch sequence.
+    ``outs`` (optional) is a list of dicts as returned by this function, reused."""
+    if len(Ws) == 0:
+        return []
+    mats, dt, outs, ws = _batch(Ws, fmt, T, ws, outs, half)
+    _check(lib().dq_solve_dual_scale_batched(len(Ws), mats, dt, ctypes.byref(fmt), T, _ptr(ws),
                                              ws.numel(), _stream(stream)),
            "dq_solve_dual_scale_batched")
     return outs
+
+
+class SolveGraph:
+    """A batched solve captured as a CUDA graph (dq_graph_solve_batched).
+    Holds the weights, outputs and workspace it was made with: ``launch``
+    solves the weights as they are at that time into ``outs``."""
+
+    def __init__(self, handle, Ws, outs, ws):
+        self._h, self.Ws, self.outs, self.ws = handle, Ws, outs, ws
+
+    @property
+    def launches(self):
+        return int(lib().dq_graph_launches(self._h)) if self._h else 0
+
+    def launch(self, stream=None):
+        if not self._h:
+            raise DqError(-1, "dq_graph_launch (graph closed)")
+        _check(lib().dq_graph_launch(self._h, _stream(stream)), "dq_graph_launch")
+        return self.outs
+
+    def close(self):
+        """Free the graph (a replay in flight completes first)."""
+        if self._h:
+            lib().dq_graph_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def solve_dual_scale_batched_graph(Ws, fmt, T, ws=None, outs=None, half=False):
+    """Capture the batched solve of ``Ws`` as a graph (nothing runs yet);
+    ``SolveGraph.launch`` replays it."""
+    if len(Ws) == 0:
+        raise ValueError("a graph needs at least one matrix")
+    mats, dt, outs, ws = _batch(Ws, fmt, T, ws, outs, half)
+    h = c_void_p()
+    _check(lib().dq_graph_solve_batched(len(Ws), mats, dt, ctypes.byref(fmt), T, _ptr(ws),
+                                        ws.numel(), ctypes.byref(h)),
+           "dq_graph_solve_batched")
+    return SolveGraph(h, list(Ws), outs, ws)
 
 
 _COPY_STREAMS = {}

@@ -20,6 +20,7 @@
 #include <cstring>
 #include <atomic>
 #include <mutex>
+#include <new>
 #include <vector>
 
 #include "../../include/dq.h"
@@ -68,7 +69,17 @@ cudaEvent_t take_event() {
     return e;
 }
 
-void count_launches(int k) { g_launches.fetch_add(k, std::memory_order_relaxed); }
+// Graph capture on this thread (dq_graph_solve_batched): launches are
+// counted into the graph, not the global counter, tile launches take no
+// timing events, and the work table is copied from the graph's pinned copy.
+thread_local bool t_capturing = false;
+thread_local int64_t t_captured_launches = 0;
+thread_local void *t_pinned_table = nullptr;
+
+void count_launches(int k) {
+    if (t_capturing) t_captured_launches += k;
+    else g_launches.fetch_add(k, std::memory_order_relaxed);
+}
 
 struct FmtInfo {
     int combo;
@@ -230,7 +241,7 @@ struct Launcher {
         cudaEvent_t beg = nullptr, end = nullptr;
         {
             std::lock_guard<std::mutex> lk(g_timing_mu);
-            if (g_timing_kinds & (1u << mode)) { beg = take_event(); end = take_event(); }
+            if (!t_capturing && (g_timing_kinds & (1u << mode))) { beg = take_event(); end = take_event(); }
         }
         if (beg && end) DQ_CUDA(cudaEventRecord(beg, st));
         DQ_CUDA(launch_tiles(combo, L));
@@ -315,13 +326,15 @@ bool fused_ok(int combo) { return all_e8m0(combo); }
 
 thread_local std::vector<MatDesc> t_table;
 
-dq_status solve_impl(int32_t n, const dq_matrix *mats, int32_t dtype, const dq_format *fmt,
-                     int32_t T, void *workspace, size_t ws_bytes, cudaStream_t st) {
+// Host-side checks of a batched solve's arguments (no CUDA call).
+dq_status check_batch(int32_t n, const dq_matrix *mats, int32_t dtype, const dq_format *fmt,
+                      int32_t T, void *workspace, size_t ws_bytes, FmtInfo *fi_out) {
     if (n < 0 || T < 0 || !mats) return DQ_ERR_ARG;
     if (dtype != DQ_DT_F32 && dtype != DQ_DT_BF16) return DQ_ERR_ARG;
     FmtInfo fi;
     dq_status s = check_format(fmt, &fi);
     if (s != DQ_OK) return s;
+    if (fi_out) *fi_out = fi;
     if (n == 0) return DQ_OK;
     const bool f32 = dtype == DQ_DT_F32;
     size_t need = table_ws(n) + 256;
@@ -340,6 +353,15 @@ dq_status solve_impl(int32_t n, const dq_matrix *mats, int32_t dtype, const dq_f
     }
     if (!workspace || ws_bytes < need) return DQ_ERR_WORKSPACE;
     if (!aligned(workspace, 256)) return DQ_ERR_ALIGN;
+    return DQ_OK;
+}
+
+dq_status solve_impl(int32_t n, const dq_matrix *mats, int32_t dtype, const dq_format *fmt,
+                     int32_t T, void *workspace, size_t ws_bytes, cudaStream_t st) {
+    FmtInfo fi;
+    dq_status s = check_batch(n, mats, dtype, fmt, T, workspace, ws_bytes, &fi);
+    if (s != DQ_OK || n == 0) return s;
+    const bool f32 = dtype == DQ_DT_F32;
 
     unsigned int *status = status_ptr();
     if (!status) return DQ_ERR_CUDA;
@@ -384,9 +406,17 @@ dq_status solve_impl(int32_t n, const dq_matrix *mats, int32_t dtype, const dq_f
     L.total_rows = row_base;
     L.total_cols = col_base;
     L.st = st;
-    if (dev_table)
-        DQ_CUDA(cudaMemcpyAsync(dev_table, t_table.data(), (size_t)n * sizeof(MatDesc),
+    if (dev_table) {
+        // (inside a graph capture the copy reads the graph's pinned table,
+        // which every replay uploads again)
+        const void *src = t_table.data();
+        if (t_pinned_table) {
+            std::memcpy(t_pinned_table, t_table.data(), (size_t)n * sizeof(MatDesc));
+            src = t_pinned_table;
+        }
+        DQ_CUDA(cudaMemcpyAsync(dev_table, src, (size_t)n * sizeof(MatDesc),
                                 cudaMemcpyHostToDevice, st));
+    }
 
     // tensor scale (NVFP4 weights: from amax of W; otherwise 1)
     if (fmt->tensor_scale_auto) {
@@ -826,6 +856,100 @@ dq_status dq_solve_dual_scale_batched(int32_t n, const dq_matrix *mats, int32_t 
                                       size_t ws_bytes, dq_stream stream) {
     return solve_impl(n, mats, dtype, fmt, T, workspace, ws_bytes,
                       reinterpret_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"
+
+struct dq_graph_s {
+    cudaGraph_t graph = nullptr;
+    cudaGraphExec_t exec = nullptr;
+    void *pinned = nullptr;      // host copy of the work table (n > 1)
+    int64_t launches = 0;        // kernels per replay
+    int device = -1;
+};
+
+namespace {
+// An executable graph still in flight is freed when it completes; the
+// pinned table it may still be reading is freed after the graph's device
+// has finished its work.
+void graph_free(dq_graph g) {
+    if (!g) return;
+    if (g->exec) cudaGraphExecDestroy(g->exec);
+    if (g->graph) cudaGraphDestroy(g->graph);
+    if (g->pinned) {
+        int cur = -1;
+        const bool switch_dev = cudaGetDevice(&cur) == cudaSuccess && cur != g->device && g->device >= 0;
+        if (switch_dev) cudaSetDevice(g->device);
+        cudaDeviceSynchronize();
+        if (switch_dev) cudaSetDevice(cur);
+        cudaFreeHost(g->pinned);
+    }
+    delete g;
+}
+}  // namespace
+
+extern "C" {
+
+dq_status dq_graph_solve_batched(int32_t n, const dq_matrix *mats, int32_t dtype,
+                                 const dq_format *fmt, int32_t T, void *workspace,
+                                 size_t ws_bytes, dq_graph *out) {
+    if (!out) return DQ_ERR_ARG;
+    *out = nullptr;
+    if (n == 0 || t_capturing) return DQ_ERR_ARG;      // empty batch; nested capture
+    dq_status s = check_batch(n, mats, dtype, fmt, T, workspace, ws_bytes, nullptr);
+    if (s != DQ_OK) return s;
+    dq_graph g = new (std::nothrow) dq_graph_s;
+    if (!g) return DQ_ERR_CUDA;
+    if (cudaGetDevice(&g->device) != cudaSuccess) { graph_free(g); return DQ_ERR_CUDA; }
+    if (n > 1 && cudaMallocHost(&g->pinned, (size_t)n * sizeof(MatDesc)) != cudaSuccess) {
+        g->pinned = nullptr;
+        graph_free(g);
+        return DQ_ERR_CUDA;
+    }
+    cudaStream_t cs = nullptr;
+    if (cudaStreamCreateWithFlags(&cs, cudaStreamNonBlocking) != cudaSuccess) { graph_free(g); return DQ_ERR_CUDA; }
+    if (cudaStreamBeginCapture(cs, cudaStreamCaptureModeRelaxed) != cudaSuccess) {
+        cudaStreamDestroy(cs);
+        graph_free(g);
+        return DQ_ERR_CUDA;
+    }
+    t_capturing = true;
+    t_captured_launches = 0;
+    t_pinned_table = g->pinned;
+    s = solve_impl(n, mats, dtype, fmt, T, workspace, ws_bytes, cs);
+    t_capturing = false;
+    t_pinned_table = nullptr;
+    g->launches = t_captured_launches;
+    const cudaError_t e = cudaStreamEndCapture(cs, &g->graph);
+    cudaStreamDestroy(cs);
+    if (s == DQ_OK && e != cudaSuccess) s = DQ_ERR_CUDA;
+    if (s == DQ_OK && cudaGraphInstantiate(&g->exec, g->graph, 0) != cudaSuccess) {
+        g->exec = nullptr;
+        s = DQ_ERR_CUDA;
+    }
+    if (s != DQ_OK) {
+        graph_free(g);
+        return s;
+    }
+    *out = g;
+    return DQ_OK;
+}
+
+dq_status dq_graph_launch(dq_graph g, dq_stream stream) {
+    if (!g || !g->exec) return DQ_ERR_ARG;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return DQ_ERR_CUDA;
+    if (dev != g->device) return DQ_ERR_ARG;
+    DQ_CUDA(cudaGraphLaunch(g->exec, reinterpret_cast<cudaStream_t>(stream)));
+    g_launches.fetch_add(g->launches, std::memory_order_relaxed);
+    return DQ_OK;
+}
+
+int64_t dq_graph_launches(dq_graph g) { return g ? g->launches : 0; }
+
+dq_status dq_graph_destroy(dq_graph g) {
+    graph_free(g);
+    return DQ_OK;
 }
 
 namespace {

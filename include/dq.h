@@ -186,6 +186,37 @@ DQ_API dq_status dq_solve_dual_scale_batched(int32_t n, const dq_matrix *mats, i
                                       const dq_format *fmt, int32_t T, void *workspace,
                                       size_t ws_bytes, dq_stream stream);
 
+/* The batched solve as a CUDA graph, for repeated solves of the same shapes
+ * (the launch sequence of dq_solve_dual_scale_batched, about 6 kernels per
+ * iteration, captured once and replayed with one launch; the solve is
+ * launch-bound on small matrices).  Arguments as dq_solve_dual_scale_batched;
+ * they are checked when the graph is made, and every device pointer in
+ * `mats` and the workspace is baked into the graph: they must stay
+ * allocated, and keep their shapes, until dq_graph_destroy.  Each replay
+ * reads W (and a0, b0) as they are at that time and writes every output
+ * again, so new weights of the same shapes take a replay, not a new graph.
+ * The graph owns a pinned host copy of the work table, uploaded by every
+ * replay (a caller may use the workspace for other calls between replays).
+ * Kernel timing (dq_kernel_timing) does not apply to graph launches.
+ * Errors: DQ_ERR_ARG (out NULL, n == 0), DQ_ERR_CUDA (capture or
+ * instantiation failed), and the argument codes of dq_solve_dual_scale_batched
+ * (checked before any CUDA call); *out is NULL then. */
+typedef struct dq_graph_s *dq_graph;
+DQ_API dq_status dq_graph_solve_batched(int32_t n, const dq_matrix *mats, int32_t dtype,
+                                        const dq_format *fmt, int32_t T, void *workspace,
+                                        size_t ws_bytes, dq_graph *out);
+/* One replay on `stream` (the device the graph was made on must be current:
+ * DQ_ERR_ARG otherwise, and for a NULL graph).  Replays on one stream run in
+ * order; replays of one graph on different streams must not overlap, since
+ * they share the workspace. */
+DQ_API dq_status dq_graph_launch(dq_graph g, dq_stream stream);
+/* Kernels one replay launches (0 for NULL). */
+DQ_API int64_t dq_graph_launches(dq_graph g);
+/* Frees the graph (NULL: no-op).  A replay still in flight completes; the
+ * pinned table is freed once the graph's device has finished its work (the
+ * call waits for that device when the graph has more than one matrix). */
+DQ_API dq_status dq_graph_destroy(dq_graph g);
+
 /* One row half-step of eq. (2) from the state (a_in, b_in):
  * a_out_i = Pi_Fa(<W_i, R_i> / <R_i, R_i>), R = Q(W ⊘ a_in b_inᵀ) D_b, zero
  * slice -> 1.  a_pre (rows, may be NULL) receives the unprojected ratio

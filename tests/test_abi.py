@@ -24,7 +24,7 @@ def built():
 
 def test_exports_match_header():
     names = _declared()
-    assert len(names) == 22
+    assert len(names) == 26
     assert sorted(dq.EXPORTS) == names
     L = dq.lib()
     for n in names:
@@ -158,3 +158,24 @@ def test_host_solve_argument_errors():
     assert call(1, f, h, d) == -1                                   # no W
     bad = dq.dq_format(9, 32, 1, 1, 0)
     assert call(1, bad, h, d) == -3                                 # format
+
+
+def test_graph_argument_errors():
+    # dq_graph_solve_batched checks its arguments before any CUDA call
+    L = dq.lib()
+    f = dq.format_preset("mxfp4")
+    m = (dq.dq_matrix * 1)()
+    m[0].rows, m[0].cols = 4, 64
+    h = ctypes.c_void_p(123)
+    call = lambda n, fmt, mm, out: L.dq_graph_solve_batched(n, mm, 1, ctypes.byref(fmt), 3, None, 0, out)
+    assert call(1, f, m, None) == -1                                # no out
+    assert call(0, f, m, ctypes.byref(h)) == -1 and h.value is None  # empty batch; *out cleared
+    assert call(-1, f, m, ctypes.byref(h)) == -1                    # n < 0
+    assert call(1, f, m, ctypes.byref(h)) == -1                     # no W
+    bad = dq.dq_format(9, 32, 1, 1, 0)
+    assert call(1, bad, m, ctypes.byref(h)) == -3                   # format
+    m[0].cols = 48
+    assert call(1, f, m, ctypes.byref(h)) == -2                     # cols % G
+    assert L.dq_graph_launch(None, None) == -1                      # no graph
+    assert L.dq_graph_launches(None) == 0
+    assert L.dq_graph_destroy(None) == 0                            # no-op
