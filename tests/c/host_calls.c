@@ -29,6 +29,21 @@ int main(void) {
     if (dq_quantize(NULL, DQ_DT_BF16, 4, 64, &f, NULL, NULL, 1.0f, NULL, NULL, NULL) != DQ_ERR_ARG)
         return fail("null input", 0);
     if (strlen(dq_strerror(DQ_ERR_TIMEOUT)) == 0) return fail("strerror", 0);
+    {
+        /* graph API: argument errors come back before any CUDA call */
+        dq_matrix m;
+        dq_graph g = (dq_graph)&m;
+        memset(&m, 0, sizeof(m));
+        m.rows = 4;
+        m.cols = 64;
+        if (dq_graph_solve_batched(1, &m, DQ_DT_BF16, &f, 3, NULL, 0, NULL) != DQ_ERR_ARG)
+            return fail("graph: no out", 0);
+        if (dq_graph_solve_batched(1, &m, DQ_DT_BF16, &f, 3, NULL, 0, &g) != DQ_ERR_ARG || g != NULL)
+            return fail("graph: no W", 0);
+        if (dq_graph_launch(NULL, NULL) != DQ_ERR_ARG) return fail("graph: launch NULL", 0);
+        if (dq_graph_launches(NULL) != 0) return fail("graph: launches NULL", 0);
+        if (dq_graph_destroy(NULL) != DQ_OK) return fail("graph: destroy NULL", 0);
+    }
     printf("ok %s\n", dq_version());
     return 0;
 }
