@@ -302,6 +302,53 @@ def test_power_of_two_row_step_leaves_mx_reconstruction_unchanged(name):
     assert np.array_equal(r["mse_half"], r["mse_trace"][:-1])
 
 
+@pytest.mark.parametrize("name", ALL_FORMATS)
+def test_solve_is_equivariant_under_row_and_group_permutations(name):
+    # Each row's update reads only that row (given b), each group's scale only
+    # that group (given a and b), each column's update only that column (given
+    # a): permuting the rows, the column groups and the columns inside each
+    # group of W permutes a, b, the codes and the group scales the same way
+    # and leaves the error unchanged.  An index slip or a transposed operand
+    # (a read by column, b by row) breaks this.
+    fmt = O.preset(name)
+    G, rows, ng = fmt.group, 20, 5
+    W = _small_matrix(rows, ng * G, seed=53)
+    rng = np.random.default_rng(7)
+    pr, pg = rng.permutation(rows), rng.permutation(ng)
+    pc = np.concatenate([g * G + rng.permutation(G) for g in pg])
+    r = O.solve(W, fmt, 4)
+    p = O.solve(W[pr][:, pc], fmt, 4)
+    assert np.array_equal(p["a"], r["a"][pr])
+    assert np.array_equal(p["b"], r["b"][pc])
+    assert np.array_equal(p["codes"], r["codes"][pr][:, pc])
+    assert np.array_equal(p["scales"], r["scales"][pr][:, pg])
+    assert p["ts"] == r["ts"]
+    assert np.allclose(p["mse_trace"], r["mse_trace"], rtol=1e-12, atol=0)
+
+
+@pytest.mark.parametrize("name", ALL_FORMATS)
+@pytest.mark.parametrize("k", [3, -5])
+def test_solve_scales_with_powers_of_two(name, k):
+    # W -> 2^k W moves every group maximum (and the NVFP4 tensor scale) by
+    # 2^k; every scale set is closed under that shift in this range and the
+    # projections commute with it, so the codes, a and b stay the same, the
+    # group scales (or, with a tensor scale, that scale) move by 2^k, and the
+    # error moves by exactly 4^k.
+    fmt = O.preset(name)
+    W = _small_matrix(16, 4 * fmt.group, seed=59)
+    r = O.solve(W, fmt, 4)
+    p = O.solve(W * 2.0 ** k, fmt, 4)
+    assert np.array_equal(p["a"], r["a"])
+    assert np.array_equal(p["b"], r["b"])
+    assert np.array_equal(p["codes"], r["codes"])
+    if fmt.tensor_scale_auto:
+        assert p["ts"] == r["ts"] * 2.0 ** k
+        assert np.array_equal(p["scales"], r["scales"])
+    else:
+        assert np.array_equal(p["scales"], r["scales"] * 2.0 ** k)
+    assert np.array_equal(p["mse_trace"], r["mse_trace"] * 4.0 ** k)
+
+
 @pytest.mark.parametrize("name", FORMATS)
 def test_dual_scale_beats_single_scale_on_outlier_matrices(name):
     fmt = O.preset(name)
