@@ -60,6 +60,41 @@ def _int4_clamp_7(q):                               # clamps to [-7, 7]
     return np.clip(_round_int4(q), -7, 7)
 
 
+def _solve_with(order):
+    """The oracle's loop with one slip in the order of its steps."""
+    def solve(W, fmt, T, a0=None, b0=None):
+        W = np.asarray(W, dtype=np.float64)
+        rows, cols = W.shape
+        a = np.ones(rows) if a0 is None else np.asarray(a0, dtype=np.float64).copy()
+        b = np.ones(cols) if b0 is None else np.asarray(b0, dtype=np.float64).copy()
+        ts = S.tensor_scale(W, fmt)
+        Qh, c, s = S.qhat(W, a, b, fmt, ts)
+        trace, half = [S.mse(W, Qh, a, b)], []
+        for _ in range(T):
+            if order == "column first":
+                b, _ = S.col_update(W, Qh, a, fmt)
+                Qh, c, s = S.qhat(W, a, b, fmt, ts)
+                half.append(S.mse(W, Qh, a, b))
+                a, _ = S.row_update(W, Qh, b, fmt)
+            else:
+                a, _ = S.row_update(W, Qh, b, fmt)
+                if order != "no re-quantize":
+                    Qh, c, s = S.qhat(W, a, b, fmt, ts)
+                if order != "half after column":
+                    half.append(S.mse(W, Qh, a, b))
+                b, _ = S.col_update(W, Qh, a, fmt)
+            Qh, c, s = S.qhat(W, a, b, fmt, ts)
+            if order == "half after column":
+                half.append(S.mse(W, Qh, a, b))
+            trace.append(S.mse(W, Qh, a, b))
+        return dict(a=a, b=b, codes=c, scales=s, ts=ts, qhat=Qh,
+                    mse_trace=np.array(trace), mse_half=np.array(half))
+    return solve
+
+
+_ORDER_PINS = [(TS.test_solve_follows_the_step_order_exactly, c) for c in TS.ORDER_CASES]
+
+
 MUTATIONS = {
     "row update without D_b": ([(S, "row_update", _row_no_db), (O, "row_update", _row_no_db)],
                                [(TS.test_row_and_column_updates_minimise_over_the_scale_set, ("int4_bf16",))]),
@@ -78,6 +113,13 @@ MUTATIONS = {
     "INT4 clamped to [-7, 7]": ([(F, "round_int4", _int4_clamp_7), (O, "round_int4", _int4_clamp_7)],
                                 [(TF.test_int4_half_even_matches_python_round, ()),
                                  (TS.test_quantize_matches_exact_rational_restatement, ("int4_bf16", 16))]),
+    # the order of the steps (text under eq. (2) of the daiwk note)
+    "column step first": ([(S, "solve", _solve_with("column first")),
+                           (O, "solve", _solve_with("column first"))], _ORDER_PINS),
+    "no re-quantize between the steps": ([(S, "solve", _solve_with("no re-quantize")),
+                                          (O, "solve", _solve_with("no re-quantize"))], _ORDER_PINS),
+    "mse_half after the column step": ([(S, "solve", _solve_with("half after column")),
+                                        (O, "solve", _solve_with("half after column"))], _ORDER_PINS),
 }
 
 

@@ -349,6 +349,104 @@ def test_solve_scales_with_powers_of_two(name, k):
     assert np.array_equal(p["mse_trace"], r["mse_trace"] * 4.0 ** k)
 
 
+# --------------------------------------------------------------------------- #
+# The order of the steps, against an exact restatement of whole iterations
+# --------------------------------------------------------------------------- #
+
+def _py_project_outer(x: Fr, oscale: str) -> Fr:
+    """Nearest admissible outer scale, exactly (BF16: nearest even in the
+    normal range; E8M0: midpoint 1.5 * 2^k, a tie goes up, |k| <= 126)."""
+    if oscale == "bf16":
+        return max(_rne(x, 8, -126, Fr(2) ** 127 * (2 - Fr(1, 128))), Fr(2) ** -126)
+    k = max(min(_floor_log2(x), 126), -127)
+    if x >= Fr(3, 2) * Fr(2) ** k:
+        k += 1
+    return Fr(2) ** max(min(k, 126), -126)
+
+
+def py_solve(W, fmt, T):
+    """T iterations of the dual-scale solve in exact rational arithmetic,
+    written from the text under eq. (2) of the daiwk note: update the row
+    scales from R = Qhat D_b with the codes fixed, re-quantize, update the
+    column scales from S = D_a Qhat with the codes fixed, re-quantize; a
+    slice with no non-zero code keeps scale 1.  Q is py_quantize; the NVFP4
+    tensor scale is 2^ceil(log2(amax / (448 qmax)))."""
+    rows, cols = len(W), len(W[0])
+    ts = Fr(1)
+    if fmt.tensor_scale_auto:
+        amax = max(abs(v) for r in W for v in r)
+        if amax > 0:
+            ts = py_group_scale(amax / (448 * Fr(fmt.qmax)), "e8m0")
+    a, b = [Fr(1)] * rows, [Fr(1)] * cols
+    G = fmt.group
+
+    def qhat():
+        C, S = py_quantize([[W[i][j] / (a[i] * b[j]) for j in range(cols)] for i in range(rows)],
+                           fmt, ts)
+        return [[C[i][j] * S[i][j // G] * ts for j in range(cols)] for i in range(rows)]
+
+    def err(Qh):
+        return sum((W[i][j] - a[i] * Qh[i][j] * b[j]) ** 2
+                   for i in range(rows) for j in range(cols)) / (rows * cols)
+
+    Qh = qhat()
+    trace, half = [err(Qh)], []
+    for _ in range(T):
+        for i in range(rows):
+            R = [Qh[i][j] * b[j] for j in range(cols)]
+            den = sum(v * v for v in R)
+            a[i] = _py_project_outer(sum(W[i][j] * R[j] for j in range(cols)) / den,
+                                     fmt.oscale) if den > 0 else Fr(1)
+        Qh = qhat()
+        half.append(err(Qh))
+        for j in range(cols):
+            S = [a[i] * Qh[i][j] for i in range(rows)]
+            den = sum(v * v for v in S)
+            b[j] = _py_project_outer(sum(W[i][j] * S[i] for i in range(rows)) / den,
+                                     fmt.oscale) if den > 0 else Fr(1)
+        Qh = qhat()
+        trace.append(err(Qh))
+    return a, b, trace, half
+
+
+def _order_matrix(seed):
+    # 3 x 32: one outlier column, one all-zero row (second row)
+    rng = np.random.default_rng(seed)
+    W = rng.standard_t(4, (3, 32)) * 0.02
+    W[:, rng.choice(32, 1, replace=False)] *= 10
+    W[1, :] = 0.0
+    return torch.from_numpy(W).to(torch.bfloat16).double().numpy()
+
+
+# (format, G, seed): inputs on which the first two iterations move scales --
+# with BF16 outer scales both a and b; with E8M0 outer scales b (a power-of-two
+# row scale only shifts the group exponents, so a stays)
+ORDER_CASES = [("int4_bf16", 16, 4), ("nvfp4", 16, 0), ("mxint4", 16, 1)]
+
+
+@pytest.mark.parametrize("name,G,seed", ORDER_CASES)
+def test_solve_follows_the_step_order_exactly(name, G, seed):
+    # The oracle's loop (row update, re-quantize, column update, re-quantize;
+    # mse_half right after the row half-step) against the exact restatement
+    # over two iterations.  Running the column step first, skipping the
+    # re-quantization between the steps, or recording mse_half after the
+    # column step each changes a, b or the traces here.
+    fmt = O.preset(name, G)
+    W = _order_matrix(seed)
+    r = O.solve(W, fmt, 2)
+    a, b, trace, half = py_solve([[Fr(float(v)) for v in row] for row in W], fmt, 2)
+    assert list(r["a"]) == [float(v) for v in a]
+    assert list(r["b"]) == [float(v) for v in b]
+    assert np.allclose(r["mse_trace"], [float(v) for v in trace], rtol=1e-12, atol=0)
+    assert np.allclose(r["mse_half"], [float(v) for v in half], rtol=1e-12, atol=0)
+    # the case is not at a fixed point: scales move in the first iteration
+    r1 = O.solve(W, fmt, 1)
+    assert np.any(r1["b"] != 1.0)
+    if fmt.oscale == "bf16":
+        assert np.any(r1["a"] != 1.0) and np.any(r["a"] != r1["a"])
+        assert half[0] != trace[0] and half[0] != trace[1]
+
+
 @pytest.mark.parametrize("name", FORMATS)
 def test_dual_scale_beats_single_scale_on_outlier_matrices(name):
     fmt = O.preset(name)
