@@ -175,11 +175,11 @@ class Clocks:
 # CPU oracle (baseline leg and reference arm)
 # --------------------------------------------------------------------------- #
 
-def _oracle_sample(wl, rows):
+def _oracle_sample(wl, rows, decoder=0):
     import numpy as np
     import synth
     import oracle as O
-    W = synth.weight(wl, 0, 0, rows=rows).double().numpy()
+    W = synth.weight(wl, decoder, 0, rows=rows).double().numpy()
     fmt = O.preset(wl.fmt, wl.group)
     return W, fmt, np, O
 
@@ -194,7 +194,92 @@ def _oracle_iteration(W, fmt, np, O, a, b, ts):
     return a, b
 
 
+def host_cores() -> int:
+    return len(os.sched_getaffinity(0))
+
+
+# Worker side of the all-cores oracle timing (spawned processes: numpy and
+# the oracle only).  Each worker holds its own row sample.
+_W_SAMPLE = None
+
+
+def _worker_init(sample, wl_fmt, wl_group):
+    global _W_SAMPLE
+    import numpy as np
+    import oracle as O
+    W = np.asarray(sample, dtype=np.float64)
+    fmt = O.preset(wl_fmt, wl_group)
+    _W_SAMPLE = (W, fmt, O.tensor_scale(W, fmt))
+
+
+def _worker_window(start_at, seconds):
+    """Whole BCD iterations of the oracle on this worker's sample from
+    `start_at` (wall clock) for about `seconds`; returns (elements x
+    iterations, elapsed seconds)."""
+    import numpy as np
+    import oracle as O
+    W, fmt, ts = _W_SAMPLE
+    while time.time() < start_at:
+        time.sleep(0.001)
+    a, b = np.ones(W.shape[0]), np.ones(W.shape[1])
+    its, t0 = 0, time.perf_counter()
+    while True:
+        a, b = _oracle_iteration(W, fmt, np, O, a, b, ts)
+        its += 1
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            return W.size * its, el
+
+
+def _worker_iteration(_):
+    """One BCD iteration of the oracle on this worker's sample from a = b = 1."""
+    import numpy as np
+    import oracle as O
+    W, fmt, ts = _W_SAMPLE
+    _oracle_iteration(W, fmt, np, O, np.ones(W.shape[0]), np.ones(W.shape[1]), ts)
+    return W.size
+
+
+class OraclePool:
+    """One spawned process per host core (os.sched_getaffinity), each with
+    its own seeded row sample of the workload: the first `rows` rows of
+    q_proj of decoder k for worker k (i.i.d. draws of the same shape and
+    distribution).  Spawned, not forked, so that it is safe after CUDA use."""
+
+    def __init__(self, wl, rows, n=None):
+        import multiprocessing as mp
+        self.n = n or host_cores()
+        self.rows = rows
+        os.environ.setdefault("OMP_NUM_THREADS", "1")
+        os.environ.setdefault("OPENBLAS_NUM_THREADS", "1")
+        ctx = mp.get_context("spawn")
+        samples = [_oracle_sample(wl, rows, decoder=k)[0].astype("float32") for k in range(self.n)]
+        self.shape = samples[0].shape
+        self.pool = [ctx.Pool(1, initializer=_worker_init, initargs=(samples[k], wl.fmt, wl.group))
+                     for k in range(self.n)]
+
+    def window(self, seconds):
+        """Aggregate rate (elements x iterations / s) of all workers running
+        iterations over the same wall-clock window."""
+        start_at = time.time() + 1.0
+        res = [p.apply_async(_worker_window, (start_at, seconds)) for p in self.pool]
+        out = [r.get() for r in res]
+        return sum(w / el for w, el in out), out
+
+    def step(self):
+        """One iteration on every worker's sample at once; returns elements."""
+        res = [p.apply_async(_worker_iteration, (0,)) for p in self.pool]
+        return sum(r.get() for r in res)
+
+    def close(self):
+        for p in self.pool:
+            p.close()
+            p.join()
+
+
 def cpu_baseline(wl, rows, min_seconds=10.0):
+    """The oracle on the host cores: one thread on a bounded sample, then one
+    process per core over a common window, each on its own sample."""
     W, fmt, np, O = _oracle_sample(wl, rows)
     ts = O.tensor_scale(W, fmt)
     a, b = np.ones(W.shape[0]), np.ones(W.shape[1])
@@ -205,37 +290,49 @@ def cpu_baseline(wl, rows, min_seconds=10.0):
         el = time.perf_counter() - t0
         if el >= min_seconds or its >= 50:
             break
-    value = W.size * its / el
-    sample = (f"{its} BCD iterations (row update, re-quantize, column update, re-quantize) of "
-              f"the fp64 numpy oracle on the first {rows} rows of decoder-0 "
-              f"{wl.linears[0].name} ({W.shape[0]}x{W.shape[1]}, {wl.fmt} G{wl.group}); "
-              f"{el:.1f} s")
-    return {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample}
+    single = W.size * its / el
+    pool = OraclePool(wl, rows)
+    try:
+        value, parts = pool.window(min_seconds)
+    finally:
+        pool.close()
+    its_all = sum(w for w, _ in parts) // W.size
+    sample = (f"the fp64 numpy oracle, whole BCD iterations (row update, re-quantize, column "
+              f"update, re-quantize) on the first {rows} rows of q_proj "
+              f"({W.shape[0]}x{W.shape[1]}, {wl.fmt} G{wl.group}): {pool.n} processes, one "
+              f"per host core, each on its own decoder's sample, {its_all} iterations in "
+              f"{min_seconds:.0f} s; one thread alone: {its} iterations on decoder 0 in "
+              f"{el:.1f} s ({single:.3g} el/s/iter)")
+    return {"value": value, "unit": UNIT, "cores": pool.n, "kind": "oracle", "sample": sample,
+            "single_thread_value": single}
 
 
 def run_reference(args, wl, rank, world):
     if rank != 0:
         return 0
-    W, fmt, np, O = _oracle_sample(wl, args.cpu_rows)
-    ts = O.tensor_scale(W, fmt)
-    a, b = np.ones(W.shape[0]), np.ones(W.shape[1])
-    for _ in range(args.warmup):
-        a, b = _oracle_iteration(W, fmt, np, O, a, b, ts)
-    t0 = time.perf_counter()
-    for _ in range(args.steps):
-        a, b = _oracle_iteration(W, fmt, np, O, a, b, ts)
-    el = time.perf_counter() - t0
-    value = W.size * args.steps / el
-    sample = (f"each step one BCD iteration of the fp64 numpy oracle on the first "
-              f"{args.cpu_rows} rows of decoder-0 {wl.linears[0].name} "
-              f"({W.shape[0]}x{W.shape[1]}, {wl.fmt} G{wl.group})")
+    pool = OraclePool(wl, args.cpu_rows)
+    try:
+        for _ in range(args.warmup):
+            pool.step()
+        t0 = time.perf_counter()
+        el_total = 0
+        for _ in range(args.steps):
+            el_total += pool.step()
+        el = time.perf_counter() - t0
+    finally:
+        pool.close()
+    value = el_total / el
+    sample = (f"each step one BCD iteration of the fp64 numpy oracle on each of {pool.n} "
+              f"row samples at once ({pool.n} processes, one per host core; sample k: the "
+              f"first {args.cpu_rows} rows of decoder k's {wl.linears[0].name}, "
+              f"{pool.shape[0]}x{pool.shape[1]}, {wl.fmt} G{wl.group})")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": el / args.steps * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": wl.name, "sample_rows": args.cpu_rows},
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+        "config": {"workload": wl.name, "sample_rows": args.cpu_rows, "processes": pool.n},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": pool.n, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }

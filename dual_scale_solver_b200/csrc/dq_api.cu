@@ -864,26 +864,23 @@ struct dq_graph_s {
     cudaGraph_t graph = nullptr;
     cudaGraphExec_t exec = nullptr;
     void *pinned = nullptr;      // host copy of the work table (n > 1)
+    cudaEvent_t done = nullptr;  // recorded after every replay
     int64_t launches = 0;        // kernels per replay
     int device = -1;
 };
 
 namespace {
 // An executable graph still in flight is freed when it completes; the
-// pinned table it may still be reading is freed after the graph's device
-// has finished its work.
+// pinned table it may still be reading is freed once the last replay has
+// finished (the replays of one executable graph run in launch order, so
+// the event recorded after the last one covers them all).
 void graph_free(dq_graph g) {
     if (!g) return;
+    if (g->done) cudaEventSynchronize(g->done);
     if (g->exec) cudaGraphExecDestroy(g->exec);
     if (g->graph) cudaGraphDestroy(g->graph);
-    if (g->pinned) {
-        int cur = -1;
-        const bool switch_dev = cudaGetDevice(&cur) == cudaSuccess && cur != g->device && g->device >= 0;
-        if (switch_dev) cudaSetDevice(g->device);
-        cudaDeviceSynchronize();
-        if (switch_dev) cudaSetDevice(cur);
-        cudaFreeHost(g->pinned);
-    }
+    if (g->done) cudaEventDestroy(g->done);
+    if (g->pinned) cudaFreeHost(g->pinned);
     delete g;
 }
 }  // namespace
@@ -901,6 +898,11 @@ dq_status dq_graph_solve_batched(int32_t n, const dq_matrix *mats, int32_t dtype
     dq_graph g = new (std::nothrow) dq_graph_s;
     if (!g) return DQ_ERR_CUDA;
     if (cudaGetDevice(&g->device) != cudaSuccess) { graph_free(g); return DQ_ERR_CUDA; }
+    if (cudaEventCreateWithFlags(&g->done, cudaEventDisableTiming) != cudaSuccess) {
+        g->done = nullptr;
+        graph_free(g);
+        return DQ_ERR_CUDA;
+    }
     if (n > 1 && cudaMallocHost(&g->pinned, (size_t)n * sizeof(MatDesc)) != cudaSuccess) {
         g->pinned = nullptr;
         graph_free(g);
@@ -941,6 +943,7 @@ dq_status dq_graph_launch(dq_graph g, dq_stream stream) {
     if (cudaGetDevice(&dev) != cudaSuccess) return DQ_ERR_CUDA;
     if (dev != g->device) return DQ_ERR_ARG;
     DQ_CUDA(cudaGraphLaunch(g->exec, reinterpret_cast<cudaStream_t>(stream)));
+    DQ_CUDA(cudaEventRecord(g->done, reinterpret_cast<cudaStream_t>(stream)));
     g_launches.fetch_add(g->launches, std::memory_order_relaxed);
     return DQ_OK;
 }
@@ -1150,8 +1153,9 @@ int64_t dq_launch_count(void) { return g_launches.load(std::memory_order_relaxed
 // from cudaGetSymbolAddress, looked up once per device with that device
 // current (the first call on a device does this, so it should come before
 // any stream capture).  Calls that overlap on the GPU share the buffer and
-// race.  The only region that must start at zero (the amax word of the
-// tensor-scale pass) is cleared by the solve sequence itself.
+// race.  The regions that must start at zero (the flag words of the
+// one-pass MX iteration and the amax word of the tensor-scale pass) are
+// cleared by the solve sequence itself.
 
 namespace {
 
@@ -1197,7 +1201,7 @@ extern "C" dq_status dq_solve_dual_scale_noalloc(const void *W, int32_t dtype, i
     if (!aligned(a, 4) || !aligned(b, 4) || !aligned(tensor_scale, 4)) return DQ_ERR_ALIGN;
     if (!aligned(a0, 4) || !aligned(b0, 4)) return DQ_ERR_ALIGN;
     if (!aligned(mse_trace, 8) || !aligned(mse_half, 8)) return DQ_ERR_ALIGN;
-    const size_t need = matrix_ws(rows, cols, f32);
+    const size_t need = 256 + matrix_ws(rows, cols, f32);        // flag words + partial sums
     if (need > (size_t)DQ_NOALLOC_SCRATCH_BYTES) return DQ_ERR_SCRATCH;
     unsigned char *scratch = noalloc_scratch();
     if (!scratch) return DQ_ERR_CUDA;
@@ -1225,6 +1229,7 @@ extern "C" dq_status dq_solve_dual_scale_noalloc(const void *W, int32_t dtype, i
     d.mse_half = mse_half;
     Carve cv{reinterpret_cast<char *>(scratch),
              reinterpret_cast<char *>(scratch) + DQ_NOALLOC_SCRATCH_BYTES};
+    unsigned int *flags = cv.take<unsigned int>(256);     // one-pass MX flags: 3 slots x 2 words
     int64_t tb[3] = {0, 0, 0}, rb = 0, cb = 0;
     place(d, f32, cv, tb, rb, cb);
     Launcher L;
@@ -1241,7 +1246,8 @@ extern "C" dq_status dq_solve_dual_scale_noalloc(const void *W, int32_t dtype, i
     L.total_cols = cb;
     L.st = st;
 
-    // same launch sequence as dq_solve_dual_scale for one matrix
+    // the launch sequence of dq_solve_dual_scale for one matrix (the MX
+    // formats take the one-pass iteration)
     if (fmt->tensor_scale_auto) {
         DQ_CUDA(cudaMemsetAsync(d.amax, 0, sizeof(unsigned int), st));   // starts at zero
         if (L.tiles[2] > 0) {
@@ -1255,18 +1261,16 @@ extern "C" dq_status dq_solve_dual_scale_noalloc(const void *W, int32_t dtype, i
     DQ_CUDA(launch_k(tensor_scale_kernel, dim3(1), dim3(128), 0, st, L.tab, fi.qmax,
                      fmt->tensor_scale_auto));
     count_launches(1);
+    const bool fused = fused_ok(fi.combo) && T > 0;
+    if (fused) DQ_CUDA(cudaMemsetAsync(flags, 0, 6 * sizeof(unsigned int), st));   // start at zero
     if (rb + cb > 0) {
         DQ_CUDA(launch_k(init_state_kernel, dim3(grid_for(rb + cb, 256)), dim3(256), 0, st, L.tab,
-                         rb, cb, nullptr));
+                         rb, cb, fused ? flags : nullptr));
         count_launches(1);
     }
-    for (int t = 0; t < T; ++t) {
-        if ((s = L.tiles_pass(MODE_ROW, mse_trace != nullptr)) != DQ_OK) return s;
-        if ((s = L.row_finalize()) != DQ_OK) return s;
-        if ((s = L.tiles_pass(MODE_COL, mse_half != nullptr)) != DQ_OK) return s;
-        if ((s = L.col_finalize()) != DQ_OK) return s;
-        if ((s = L.mse(MODE_ROW, t, t, nullptr, nullptr)) != DQ_OK) return s;
-    }
+    for (int t = 0; t < T; ++t)
+        if ((s = L.iteration(t, fused, flags, mse_trace != nullptr, mse_half != nullptr)) != DQ_OK)
+            return s;
     if ((s = L.tiles_pass(MODE_PACK, mse_trace != nullptr)) != DQ_OK) return s;
     return L.mse(2, T, -1, nullptr, nullptr);
 }

@@ -212,9 +212,9 @@ DQ_API dq_status dq_graph_solve_batched(int32_t n, const dq_matrix *mats, int32_
 DQ_API dq_status dq_graph_launch(dq_graph g, dq_stream stream);
 /* Kernels one replay launches (0 for NULL). */
 DQ_API int64_t dq_graph_launches(dq_graph g);
-/* Frees the graph (NULL: no-op).  A replay still in flight completes; the
- * pinned table is freed once the graph's device has finished its work (the
- * call waits for that device when the graph has more than one matrix). */
+/* Frees the graph (NULL: no-op).  The call waits for the graph's last
+ * replay to finish (only that: other work on the device is not waited
+ * for), then frees the graph and its pinned table. */
 DQ_API dq_status dq_graph_destroy(dq_graph g);
 
 /* One row half-step of eq. (2) from the state (a_in, b_in):
@@ -331,6 +331,8 @@ DQ_API dq_status dq_last_device_status(dq_stream stream);
  *    wrong results; serialise them.  The buffer keeps the last call's
  *    contents; the call clears what it needs to start at zero.
  *  - Allocates nothing (no cudaMalloc, cudaFree or allocating library call).
+ *  - Runs the launch sequence of dq_solve_dual_scale (the MX formats take
+ *    the one-pass iteration), so its results equal that call's bit for bit.
  * Arguments, outputs and errors as dq_solve_dual_scale. */
 #define DQ_NOALLOC_SCRATCH_BYTES (32u << 20)
 DQ_API dq_status dq_solve_dual_scale_noalloc(const void *W, int32_t dtype, int64_t rows,

@@ -4,10 +4,12 @@ Bars (derived from the method's arithmetic):
 * codes and group scales of Q given identical (a, b, ts): bit-exact;
 * activation codes and scales given identical b: bit-exact;
 * one half-step from an identical state: unprojected ratios within 1e-5
-  relative (float32 sums over <= 28672 terms against fp64); projected scales
-  equal except where the ratio lies within 1e-5 of a projection boundary
-  (listed, at most 1e-3 of the scales);
-* after T iterations: every mse_trace entry within 1e-4 relative.
+  relative (float32 sums over <= 28672 terms against fp64); projected E8M0
+  scales equal; projected BF16 scales equal except where the ratio lies
+  within 1e-5 of a bf16 rounding boundary (counted, at most 1e-3 of the
+  scales);
+* after T iterations: every mse_trace entry within 1e-4 relative; E8M0
+  scales of the whole trajectory equal to the oracle's.
 """
 import numpy as np
 import pytest
@@ -15,8 +17,8 @@ import torch
 
 import oracle as O
 import synth
-from _helpers import (MX_MORE, PRESET_COMBOS, code_boundaries, gpu_scales_np, lib_format,
-                      near_outer_boundary, np64, oracle_encoded, random_outer)
+from _helpers import (MX_MORE, PRESET_COMBOS, check_projected, code_boundaries, gpu_scales_np,
+                      lib_format, np64, oracle_encoded, random_outer)
 
 pytestmark = pytest.mark.gpu
 
@@ -167,14 +169,6 @@ def test_act_rescale_quant_bit_exact(name, tokens):
 # One half-step from an identical state
 # --------------------------------------------------------------------------- #
 
-def _check_projected(gpu, orc, pre, fo, what):
-    diff = gpu != orc
-    near = near_outer_boundary(pre, fo)
-    unexplained = np.argwhere(diff & ~near)
-    assert unexplained.size == 0, f"{what}: {unexplained.size} differ away from a boundary"
-    assert diff.sum() <= max(1, 1e-3 * diff.size), f"{what}: {diff.sum()} near-boundary flips"
-
-
 @pytest.mark.parametrize("name", ALL)
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
 def test_half_steps_from_identical_state(name, dtype):
@@ -198,7 +192,7 @@ def test_half_steps_from_identical_state(name, dtype):
     ok = ~np.isnan(x_or)
     assert np.array_equal(np.isnan(pre), np.isnan(x_or))
     assert np.max(np.abs(pre[ok] - x_or[ok]) / x_or[ok]) < 1e-5
-    _check_projected(np64(a_gpu), a_or, x_or, fo, "a")
+    check_projected(np64(a_gpu), a_or, x_or, fo, "a")
     assert abs(mse0.item() - O.mse(W64, Qh, a, b)) <= 1e-6 * O.mse(W64, Qh, a, b)
     # column step from (a_gpu, b)
     a1 = np64(a_gpu)
@@ -209,7 +203,7 @@ def test_half_steps_from_identical_state(name, dtype):
     ok = ~np.isnan(xb_or)
     assert np.array_equal(np.isnan(pre), np.isnan(xb_or))
     assert np.max(np.abs(pre[ok] - xb_or[ok]) / xb_or[ok]) < 1e-5
-    _check_projected(np64(b_gpu), b_or, xb_or, fo, "b")
+    check_projected(np64(b_gpu), b_or, xb_or, fo, "b")
     ref = O.mse(W64, Qh1, a1, b)
     assert abs(mse1.item() - ref) <= 1e-6 * ref
 
@@ -237,9 +231,15 @@ def _solve_and_compare(Ws, fo, fl, T, tol=1e-4):
         ec, es = oracle_encoded(W64, a, b, fo, r["ts"])
         assert np.array_equal(o["codes"].cpu().numpy(), ec)
         assert np.array_equal(gpu_scales_np(o["gscales"]), es)
-        # most scales agree with the oracle's trajectory exactly
-        same = (np.mean(a == r["a"]) + np.mean(b == r["b"])) / 2
-        assert same > 0.97, same
+        # E8M0 scales follow the oracle's trajectory exactly; BF16 scales
+        # may part from it after a flip at a rounding boundary (counted)
+        if fo.oscale == "e8m0":
+            assert np.array_equal(a, r["a"]) and np.array_equal(b, r["b"])
+        else:
+            same = (np.mean(a == r["a"]) + np.mean(b == r["b"])) / 2
+            print(f"trajectory: {np.sum(a != r['a'])} of {a.size} a and "
+                  f"{np.sum(b != r['b'])} of {b.size} b differ from the oracle's")
+            assert same > 0.97, same
     return worst
 
 
@@ -399,6 +399,79 @@ def test_mx_solve_equals_the_literal_steps(name, extreme):
         # extreme scales can push float32 statistics out of range; the device
         # reports it (and the literal steps agree with the solve all the same)
         assert dq.last_device_status() in (0, -4, -5)
+
+
+# spread of log(b0) per format, wide enough that some columns' values fall
+# where the element grid is coarse (fixed-point or subnormal codes), so that
+# column ratios leave [0.75, 1.5) and b moves; MXFP8 E5M2 would need a range
+# of 2^32, so only its zero columns move
+_MOVING_SPREAD = {"mxfp4": 1.5, "mxint4": 1.5, "mxint8": 6.0, "mxfp6_e2m3": 6.0,
+                  "mxfp6_e3m2": 6.0, "mxfp8_e4m3": 12.0, "mxfp8_e5m2": 1.5}
+
+
+def _moving_state(name, fo, rows=300, cols=2240):
+    """Weights and a seeded E8M0 starting state (a0, b0) from which the solve
+    moves.  Rows 0-3 repeat, per group of 32, one element at (113/32) 2^-6-r
+    and 31 at +-(33/64) 2^-6-r (times a0_r b0_j): MXINT4 codes 4 and +-1, a
+    row ratio of about 0.64, so a_r halves.  Row 4 and columns 7 and 1000
+    are zero and start away from 1: their scales return to 1."""
+    a0 = random_outer(fo, rows, synth.stream_key(98, 1), 1.5)
+    b0 = random_outer(fo, cols, synth.stream_key(98, 2), _MOVING_SPREAD[name])
+    a0[4], b0[7], b0[1000] = 4.0, 2.0, 0.25
+    W = _weights(rows, cols, torch.float32, key=23)
+    pat = torch.tensor([33 / 64 if k % 2 else -33 / 64 for k in range(32)])
+    pat[5] = 113 / 32
+    b0t = torch.tensor(b0, dtype=torch.float32)
+    for r in range(4):
+        W[r] = pat.repeat(cols // 32) * b0t * float(a0[r]) * 2.0 ** (-6 - r)
+    W[4] = 0.0
+    W[:, [7, 1000]] = 0.0
+    return W.to(torch.bfloat16), a0, b0
+
+
+@pytest.mark.parametrize("name", ["mxfp4", "mxint4"] + MX_MORE)
+def test_mx_solve_from_a_moving_state(name):
+    # The one-pass iteration from a seeded state with a != 1 and b != 1 whose
+    # scales are updated: equal to the literal row and column steps bit for
+    # bit, and to the oracle's whole trajectory (E8M0 scales exactly, MSE
+    # within 1e-4).  A slip in the fused path's row values (Qhat s) b_j or in
+    # the 1/a scaling of its row sums would show here.
+    fl = dq.format_preset(name)
+    fo = PRESET_COMBOS[name](32)
+    W, a0, b0 = _moving_state(name, fo)
+    Wd = W.cuda()
+    a0d = torch.tensor(a0, dtype=torch.float32, device="cuda")
+    b0d = torch.tensor(b0, dtype=torch.float32, device="cuda")
+    T = 4
+    o = dq.solve_dual_scale(Wd, fl, T, a0=a0d, b0=b0d)
+    # the literal steps, iteration by iteration, recording which scales move
+    a, b = a0d.clone(), b0d.clone()
+    moved_a, moved_b = [], []
+    for _ in range(T):
+        a1, _, _ = dq.row_update(Wd, fl, a, b)
+        b1, _, _ = dq.col_update(Wd, fl, a1, b)
+        moved_a.append(np.flatnonzero((a1 != a).cpu().numpy()))
+        moved_b.append(np.flatnonzero((b1 != b).cpu().numpy()))
+        a, b = a1, b1
+    torch.cuda.synchronize()
+    assert torch.equal(o["a"], a) and torch.equal(o["b"], b)
+    # the state moves: the zero row and columns in the first iteration, and
+    # (but for MXFP8 E5M2) other columns; MXINT4's constructed rows halve a
+    assert 4 in moved_a[0] and {7, 1000} <= set(moved_b[0].tolist())
+    if name != "mxfp8_e5m2":
+        assert len(set(np.concatenate(moved_b).tolist()) - {7, 1000}) > 0
+    if name == "mxint4":
+        assert {0, 1, 2, 3} <= set(moved_a[0].tolist())
+    # the oracle's trajectory from the same state
+    r = O.solve(np64(W), fo, T, a0=a0, b0=b0)
+    assert np.array_equal(np64(o["a"]), r["a"]) and np.array_equal(np64(o["b"]), r["b"])
+    tr, hf = np64(o["mse_trace"]), np64(o["mse_half"])
+    assert np.max(np.abs(tr - r["mse_trace"]) / r["mse_trace"]) < 1e-4
+    assert np.array_equal(hf, tr[:T])
+    ec, es = oracle_encoded(np64(W), r["a"], r["b"], fo)
+    assert np.array_equal(o["codes"].cpu().numpy(), ec)
+    assert np.array_equal(gpu_scales_np(o["gscales"]), es)
+    assert dq.last_device_status() == 0
 
 
 @pytest.mark.parametrize("name", ["mxfp4", "mxint8"])
