@@ -350,10 +350,13 @@ def two_level_quant(X, dual_block: int, inner: Format):
 # The inference step: block-scaled W4A4 product
 # --------------------------------------------------------------------------- #
 
-def w4a4_gemm(cx, sx, cw, sw, a, fmt: Format):
+def w4a4_gemm(cx, sx, cw, sw, a, fmt: Format, ts_w: float = 1.0):
     """out[m, n] = a_n * sum_k Qx[m, k] Qw[n, k] with Qx = dequantize(cx, sx),
-    Qw = dequantize(cw, sw) (eq. (1) of the daiwk note: X W^T ~= (X D_b)
-    Qhat^T D_a).  Codes and scales as values; float64."""
+    Qw = dequantize(cw, sw, ts_w) (eq. (1) of the daiwk note: X W^T ~= (X D_b)
+    Qhat^T D_a).  Codes and scales as values; float64.  ts_w is the weights'
+    tensor scale (NVFP4: E2M1 codes with an E4M3 scale per 16 elements, news
+    article "适配 MXFP4 与 NVFP4 块结构", times the per-matrix power of two the
+    solve takes; 1 otherwise); the activations are quantized with ts = 1."""
     Xq = dequantize(np.asarray(cx, dtype=np.float64), np.asarray(sx, dtype=np.float64), fmt)
-    Wq = dequantize(np.asarray(cw, dtype=np.float64), np.asarray(sw, dtype=np.float64), fmt)
+    Wq = dequantize(np.asarray(cw, dtype=np.float64), np.asarray(sw, dtype=np.float64), fmt, ts_w)
     return (Xq @ Wq.T) * np.asarray(a, dtype=np.float64)[None, :]

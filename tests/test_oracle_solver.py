@@ -619,3 +619,37 @@ def test_w4a4_gemm_against_explicit_sums():
     approx = O.w4a4_gemm(cxa, sxa, r["codes"], r["scales"], r["a"], fmt)
     exact = X @ W.T
     assert np.linalg.norm(approx - exact) < 0.25 * np.linalg.norm(exact)
+
+
+def test_w4a4_gemm_nvfp4_against_explicit_sums():
+    # NVFP4: E4M3 group scales per 16 elements and the weights' tensor scale,
+    # out[m, n] = a_n ts_w sum_k (c_x s_x)(c_w s_w), written out with fractions
+    fmt = O.preset("nvfp4")
+    rng = np.random.default_rng(33)
+    M, N, K = 3, 2, 48
+    grid = np.concatenate([O.E2M1_GRID, -O.E2M1_GRID])
+    e4m3 = O.decode_e4m3(np.arange(1, 127, dtype=np.uint8))       # positive finite values
+    cx, cw = rng.choice(grid, (M, K)), rng.choice(grid, (N, K))
+    sx, sw = rng.choice(e4m3, (M, K // 16)), rng.choice(e4m3, (N, K // 16))
+    a = np.array([0.75, 3.0])
+    ts = 2.0 ** -7
+    out = O.w4a4_gemm(cx, sx, cw, sw, a, fmt, ts)
+    for m in range(M):
+        for n in range(N):
+            acc = sum(Fr(float(cx[m, k])) * Fr(float(sx[m, k // 16])) * Fr(float(cw[n, k])) *
+                      Fr(float(sw[n, k // 16])) for k in range(K))
+            want = acc * Fr(ts) * Fr(float(a[n]))
+            assert abs(Fr(float(out[m, n])) - want) <= abs(want) * Fr(2) ** -50
+    # the eq. (1) identity with the NVFP4 solve (tensor scale from W) and
+    # activations quantized with ts = 1
+    W = _small_matrix(64, 128, seed=34)
+    r = O.solve(W, fmt, 3)
+    assert r["ts"] != 1.0
+    X = rng.standard_normal((16, 128))
+    cxa, sxa = O.act_rescale_quant(X, r["b"], fmt)
+    approx = O.w4a4_gemm(cxa, sxa, r["codes"], r["scales"], r["a"], fmt, r["ts"])
+    exact = X @ W.T
+    assert np.linalg.norm(approx - exact) < 0.2 * np.linalg.norm(exact)
+    # without the tensor scale the product is off by 1/ts
+    wrong = O.w4a4_gemm(cxa, sxa, r["codes"], r["scales"], r["a"], fmt)
+    assert np.linalg.norm(wrong - exact) > 0.9 * np.linalg.norm(exact)
