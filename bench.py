@@ -695,8 +695,10 @@ def run_two_level(args, wl, rank, world, local_rank):
 
 def run_gemm(args, wl, rank, world, local_rank):
     """The inference step after the solve: every linear of the workload's
-    decoder(s) as a block-scaled W4A4 GEMM (MXFP4 x MXFP4, E8M0 scales) on a
-    batch of `tokens` activation rows; the weights' codes, scales and a come
+    decoder(s) as a block-scaled W4A4 GEMM (MXFP4 x MXFP4 with E8M0 scales;
+    NVFP4 x NVFP4 with E4M3 scales and the weights' tensor scale for an NVFP4
+    workload) on a batch of `tokens` activation rows; the weights' codes,
+    scales, tensor scale and a come
     from the solve, the activations' codes and scales from the activation
     quantizer (one batch per input width)."""
     import torch
@@ -707,8 +709,12 @@ def run_gemm(args, wl, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     build.build()
-    fmt = dq.format_preset("mxfp4")
-    Ws = [synth.weight(wl, d, i, device=dev) for d in decoders_of(rank, wl.decoders)
+    nv = wl.fmt == "nvfp4"
+    fmt = dq.format_preset("nvfp4" if nv else "mxfp4")
+    # (--decoders caps the decoders per rank: the float32 outputs of all
+    # linears of the 32-decoder sets at 32768 tokens exceed the device memory)
+    n_dec = wl.decoders if args.decoders < 0 else min(args.decoders, wl.decoders)
+    Ws = [synth.weight(wl, d, i, device=dev) for d in decoders_of(rank, n_dec)
           for i in range(len(wl.linears))]
     outs = dq.solve_dual_scale_batched(Ws, fmt, wl.T)
     M = args.tokens
@@ -722,15 +728,16 @@ def run_gemm(args, wl, rank, world, local_rank):
     res = [torch.empty(M, W.shape[0], dtype=torch.float32, device=dev) for W in Ws]
     del Ws
     stream = torch.cuda.current_stream(dev)
-    # the GEMM reads E8M0 scales as scale tiles: the weights' once after the
+    # the GEMM reads group scales as scale tiles: the weights' once after the
     # solve, the activation batches' once per batch
-    wtiles = [dq.scale_tiles(o["gscales"]) for o in outs]
-    acts = {K: (cx, dq.scale_tiles(sx)) for K, (cx, sx) in acts.items()}
+    wtiles = [dq.scale_tiles(o["gscales"], group=fmt.group) for o in outs]
+    acts = {K: (cx, dq.scale_tiles(sx, group=fmt.group)) for K, (cx, sx) in acts.items()}
 
     def step():
         for o, r, sw in zip(outs, res, wtiles):
             cx, sx = acts[2 * o["codes"].shape[1]]
-            dq.w4a4_gemm(cx, sx, o["codes"], sw, o["a"], fmt, out=r, tiled=True)
+            dq.w4a4_gemm(cx, sx, o["codes"], sw, o["a"], fmt, out=r, tiled=True,
+                         tensor_scale=o["tensor_scale"] if nv else None)
 
     for _ in range(args.warmup):
         step()
@@ -763,7 +770,8 @@ def run_gemm(args, wl, rank, world, local_rank):
     peak = float(peaks.get(peak_key, 1590.0)) * 4.0
     tflops = flops / (ms / 1e3) / 1e12
     line = {
-        "metric": "W4A4 GEMM TFLOP/s (MXFP4 x MXFP4, E8M0 scales, fp32 accumulate)",
+        "metric": ("W4A4 GEMM TFLOP/s (NVFP4 x NVFP4, E4M3 scales per 16, fp32 accumulate)" if nv
+                   else "W4A4 GEMM TFLOP/s (MXFP4 x MXFP4, E8M0 scales, fp32 accumulate)"),
         "value": world * tflops, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "fp4 (e2m1)", "data": "synthetic",

@@ -19,7 +19,7 @@ __all__ = [
     "row_update", "col_update", "act_rescale_quant", "last_device_status", "EXPORTS",
     "kernel_timing", "kernel_time", "launch_count", "solve_dual_scale_noalloc", "code_bytes",
     "two_level_quant", "w4a4_gemm", "scale_tiles", "solve_dual_scale_batched_host", "copy_streams",
-    "SolveGraph", "solve_dual_scale_batched_graph",
+    "SolveGraph", "solve_dual_scale_batched_graph", "col_row_block", "col_partials", "col_finalize",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -29,7 +29,7 @@ DQ_CODES_INT4, DQ_CODES_E2M1, DQ_CODES_INT8, DQ_CODES_E4M3 = 0, 1, 2, 3
 DQ_CODES_E5M2, DQ_CODES_E2M3, DQ_CODES_E3M2 = 4, 5, 6
 DQ_SCALE_BF16, DQ_SCALE_E8M0, DQ_SCALE_E4M3 = 0, 1, 2
 DQ_DT_F32, DQ_DT_BF16 = 0, 1
-DQ_OK, DQ_ERR_NONFINITE, DQ_ERR_RANGE = 0, -4, -5
+DQ_OK, DQ_ERR_ARG, DQ_ERR_NONFINITE, DQ_ERR_RANGE = 0, -1, -4, -5
 
 EXPORTS = ("dq_version", "dq_strerror", "dq_format_preset", "dq_workspace_size", "dq_quantize",
            "dq_dequantize", "dq_solve_dual_scale", "dq_solve_dual_scale_batched",
@@ -37,7 +37,8 @@ EXPORTS = ("dq_version", "dq_strerror", "dq_format_preset", "dq_workspace_size",
            "dq_kernel_timing", "dq_kernel_time", "dq_launch_count",
            "dq_solve_dual_scale_noalloc", "dq_code_bytes", "dq_two_level_quant", "dq_w4a4_gemm",
            "dq_scale_tiles", "dq_solve_dual_scale_batched_host", "dq_test_stall_next_gemm",
-           "dq_graph_solve_batched", "dq_graph_launch", "dq_graph_launches", "dq_graph_destroy")
+           "dq_graph_solve_batched", "dq_graph_launch", "dq_graph_launches", "dq_graph_destroy",
+           "dq_col_row_block", "dq_col_partials", "dq_col_finalize")
 
 
 class DqError(RuntimeError):
@@ -100,6 +101,12 @@ def lib() -> ctypes.CDLL:
         "dq_col_update": (c_int32, [c_void_p, c_int32, c_int64, c_int64, P(dq_format), c_float,
                                     c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                     c_size_t, c_void_p]),
+        "dq_col_row_block": (c_int64, [c_int64, c_int64, c_int32]),
+        "dq_col_partials": (c_int32, [c_void_p, c_int32, c_int64, c_int64, P(dq_format), c_float,
+                                      c_void_p, c_void_p, c_int64, c_void_p, c_void_p, c_void_p,
+                                      c_size_t, c_void_p]),
+        "dq_col_finalize": (c_int32, [c_void_p, c_int64, c_int64, P(dq_format), c_void_p,
+                                      c_void_p, c_void_p]),
         "dq_act_rescale_quant": (c_int32, [c_void_p, c_int64, c_int64, c_void_p, P(dq_format),
                                            c_void_p, c_void_p, c_void_p]),
         "dq_last_device_status": (c_int32, [c_void_p]),
@@ -107,9 +114,9 @@ def lib() -> ctypes.CDLL:
         "dq_kernel_time": (c_int32, [c_int32, P(c_double), P(c_int64)]),
         "dq_launch_count": (c_int64, []),
         "dq_code_bytes": (c_int64, [P(dq_format), c_int64, c_int64]),
-        "dq_w4a4_gemm": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int64,
-                                   c_int64, c_int64, P(dq_format), c_void_p, c_void_p]),
-        "dq_scale_tiles": (c_int32, [c_void_p, c_int64, c_int64, c_void_p, c_void_p]),
+        "dq_w4a4_gemm": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                   c_int64, c_int64, c_int64, P(dq_format), c_void_p, c_void_p]),
+        "dq_scale_tiles": (c_int32, [c_void_p, c_int64, c_int64, c_int32, c_void_p, c_void_p]),
         "dq_test_stall_next_gemm": (c_int32, []),
         "dq_graph_solve_batched": (c_int32, [c_int32, P(dq_matrix), c_int32, P(dq_format), c_int32,
                                              c_void_p, c_size_t, P(c_void_p)]),
@@ -480,6 +487,46 @@ def col_update(W, fmt, a_in, b_in, tensor_scale=1.0, ws=None, stream=None):
                  W.shape[1], ws, stream)
 
 
+def col_row_block(rows, cols, dtype=torch.bfloat16) -> int:
+    """Rows per row block of the column statistics of a rows x cols matrix."""
+    v = lib().dq_col_row_block(rows, cols, DQ_DT_F32 if dtype == torch.float32 else DQ_DT_BF16)
+    if v < 0:
+        raise DqError(DQ_ERR_ARG, "dq_col_row_block")
+    return int(v)
+
+
+def col_partials(W, fmt, a, b, row_block, tensor_scale=1.0, out=None, ws=None, stream=None):
+    """Column partial sums of a row shard W (its rows' a, the matrix's b) per
+    block of `row_block` rows: returns (partials [ceil(rows/row_block), cols,
+    2] float32, mse of the input state over the shard)."""
+    _need_cuda(W, a, b)
+    rows, cols = W.shape
+    nrb = -(-rows // row_block)
+    if out is None:
+        out = torch.empty(nrb, cols, 2, dtype=torch.float32, device=W.device)
+    mse = torch.empty(1, dtype=torch.float64, device=W.device)
+    if ws is None:
+        ws = workspace([(rows, cols)], fmt, W.device)
+    _check(lib().dq_col_partials(_ptr(W), _dtype_code(W), rows, cols, ctypes.byref(fmt),
+                                 float(tensor_scale), _ptr(a), _ptr(b), row_block, _ptr(out),
+                                 _ptr(mse), _ptr(ws), ws.numel(), _stream(stream)),
+           "dq_col_partials")
+    return out, mse
+
+
+def col_finalize(partials, fmt, b_out=None, stream=None):
+    """b from column partial slabs [row_blocks, cols, 2] (fixed-order sums):
+    returns (b, b_pre)."""
+    _need_cuda(partials)
+    nrb, cols = partials.shape[0], partials.shape[1]
+    if b_out is None:
+        b_out = torch.empty(cols, dtype=torch.float32, device=partials.device)
+    pre = torch.empty(cols, dtype=torch.float32, device=partials.device)
+    _check(lib().dq_col_finalize(_ptr(partials), nrb, cols, ctypes.byref(fmt), _ptr(b_out),
+                                 _ptr(pre), _stream(stream)), "dq_col_finalize")
+    return b_out, pre
+
+
 def act_rescale_quant(X, b, fmt, codes=None, gscales=None, stream=None):
     """Q(X D_b): returns (codes [tokens, K*bits/8], group scales [tokens, K/G])."""
     _need_cuda(X, b)
@@ -511,34 +558,40 @@ def two_level_quant(X, dual_block=512, inner=None, qdq=True, stream=None):
     return codes, isc, osc, out
 
 
-def scale_tiles(scales, K=None, out=None, stream=None):
-    """Row-major E8M0 scales [rows, K/32] -> the scale tiles dq_w4a4_gemm
-    reads (rows * K / 32 bytes, uint8)."""
+def scale_tiles(scales, K=None, out=None, stream=None, group=32):
+    """Row-major group scales [rows, K/group] (E8M0 for MXFP4, group 32; E4M3
+    for NVFP4, group 16) -> the scale tiles dq_w4a4_gemm reads (rows * K /
+    group bytes, uint8)."""
     _need_cuda(scales)
     rows = scales.shape[0]
-    K = 32 * scales.shape[1] if K is None else K
+    K = group * scales.shape[1] if K is None else K
     if out is None:
-        out = torch.empty(rows * K // 32, dtype=torch.uint8, device=scales.device)
-    _check(lib().dq_scale_tiles(_ptr(scales), rows, K, _ptr(out), _stream(stream)), "dq_scale_tiles")
+        out = torch.empty(rows * K // group, dtype=torch.uint8, device=scales.device)
+    _check(lib().dq_scale_tiles(_ptr(scales), rows, K, group, _ptr(out), _stream(stream)),
+           "dq_scale_tiles")
     return out
 
 
 def w4a4_gemm(codes_x, scales_x, codes_w, scales_w, a, fmt=None, out=None, stream=None,
-              tiled=False):
-    """out[M, N] = a_n * sum_k Qx[m, k] Qw[n, k] (float32) from MXFP4 codes and
-    E8M0 scales of the activations (M rows) and the weights (N rows).  The
-    scales are row-major [rows, K/32] (tiled=False: rewritten into scale tiles
-    first, one extra launch each) or already scale tiles (tiled=True)."""
+              tiled=False, tensor_scale=None):
+    """out[M, N] = a_n * ts * sum_k Qx[m, k] Qw[n, k] (float32) from E2M1 codes
+    and group scales of the activations (M rows) and the weights (N rows):
+    MXFP4 (E8M0 scales per 32, the default) or NVFP4 (E4M3 scales per 16; ts
+    = the weights' tensor scale, a one-element device tensor as the solve
+    returns it, None for 1).  The scales are row-major [rows, K/G]
+    (tiled=False: rewritten into scale tiles first, one extra launch each) or
+    already scale tiles (tiled=True)."""
     _need_cuda(codes_x, scales_x, codes_w, scales_w, a)
     fmt = format_preset("mxfp4") if fmt is None else fmt
     M, N, K = codes_x.shape[0], codes_w.shape[0], 2 * codes_x.shape[1]
     if not tiled:
-        scales_x = scale_tiles(scales_x, K, stream=stream)
-        scales_w = scale_tiles(scales_w, K, stream=stream)
+        scales_x = scale_tiles(scales_x, K, stream=stream, group=fmt.group)
+        scales_w = scale_tiles(scales_w, K, stream=stream, group=fmt.group)
     if out is None:
         out = torch.empty(M, N, dtype=torch.float32, device=codes_x.device)
+    ts = None if tensor_scale is None else _ptr(tensor_scale)
     _check(lib().dq_w4a4_gemm(_ptr(codes_x), _ptr(scales_x), _ptr(codes_w), _ptr(scales_w),
-                              _ptr(a), M, N, K, ctypes.byref(fmt), _ptr(out), _stream(stream)),
+                              _ptr(a), ts, M, N, K, ctypes.byref(fmt), _ptr(out), _stream(stream)),
            "dq_w4a4_gemm")
     return out
 

@@ -522,6 +522,66 @@ dq_status step_impl(bool row_step, const void *W, int32_t dtype, int64_t rows, i
     return DQ_OK;
 }
 
+// Column statistics of a row shard with the whole matrix's row blocks
+// (dq_col_partials): the column pass of one matrix whose row blocks have
+// `row_block` rows, writing its partial sums to the caller's slab.
+dq_status col_partials_impl(const void *W, int32_t dtype, int64_t rows, int64_t cols,
+                            const dq_format *fmt, float ts, const float *a, const float *b,
+                            int64_t row_block, float *partials, double *mse, void *workspace,
+                            size_t ws_bytes, cudaStream_t st) {
+    FmtInfo fi;
+    MatDesc d;
+    dq_status s = single(W, dtype, rows, cols, fmt, &fi, d);
+    if (s != DQ_OK) return s;
+    if (!a || !b || !partials) return DQ_ERR_ARG;
+    if (!(ts > 0.0f)) return DQ_ERR_ARG;
+    if (fmt->group_scale != DQ_SCALE_E4M3 && ts != 1.0f) return DQ_ERR_ARG;
+    if (!aligned(a, 4) || !aligned(b, 4) || !aligned(partials, 16) || !aligned(mse, 8))
+        return DQ_ERR_ALIGN;
+    const bool f32 = dtype == DQ_DT_F32;
+    const Geom g = geometry(rows, cols, f32);
+    const int wr = kWarps / g.wc;
+    // (the residual slots in the workspace are sized for the shard's own row
+    // blocks: a row block below the shard's own is refused; the row block
+    // of a matrix never decreases with its rows, so a shard of it passes)
+    if (row_block <= 0 || row_block % wr || row_block / wr > kRowsPerWarp[MODE_COL] ||
+        row_block < g.tr[1])
+        return DQ_ERR_SHAPE;
+    if (!workspace || ws_bytes < matrix_ws(rows, cols, f32)) return DQ_ERR_WORKSPACE;
+    if (!aligned(workspace, 256)) return DQ_ERR_ALIGN;
+    if (rows == 0 || cols == 0) return DQ_OK;
+    unsigned int *status = status_ptr();
+    if (!status) return DQ_ERR_CUDA;
+    d.a = a;
+    d.b = b;
+    d.ts_val = ts;
+    Carve cv{static_cast<char *>(workspace), static_cast<char *>(workspace) + ws_bytes};
+    int64_t tb[3] = {0, 0, 0}, rb = 0, cb = 0;
+    place(d, f32, cv, tb, rb, cb);
+    // the column pass with the whole matrix's row blocks, into the caller's slab
+    d.tr[1] = (int32_t)row_block;
+    d.ntiles[1] = (rows + row_block - 1) / row_block * d.ncb;
+    d.colpart = reinterpret_cast<float2 *>(partials);
+    Launcher L;
+    L.tab.dev = nullptr;
+    L.tab.one = d;
+    L.tab.n = 1;
+    L.tab.status = status;
+    L.combo = fi.combo;
+    L.G = fi.G;
+    L.f32 = f32;
+    L.qmax = fi.qmax;
+    L.tiles[0] = d.ntiles[0];
+    L.tiles[1] = d.ntiles[1];
+    L.tiles[2] = d.ntiles[2];
+    L.total_rows = rb;
+    L.total_cols = cb;
+    L.st = st;
+    if ((s = L.tiles_pass(MODE_COL, mse != nullptr)) != DQ_OK) return s;
+    if (mse) return L.mse(-1, -1, -1, nullptr, mse);
+    return DQ_OK;
+}
+
 // Value of the stored code of element (r, c) (layouts as the tile kernel
 // writes them: 4-bit codes two per byte, 8-bit one per byte, 6-bit four per
 // 3 bytes).  Float element formats decode from their bit fields.
@@ -767,18 +827,20 @@ dq_status dq_test_stall_next_gemm(void) {
 }
 
 dq_status dq_w4a4_gemm(const uint8_t *codes_x, const void *scales_x, const uint8_t *codes_w,
-                       const void *scales_w, const float *a, int64_t M, int64_t N, int64_t K,
-                       const dq_format *fmt, float *out, dq_stream stream) {
+                       const void *scales_w, const float *a, const float *tensor_scale, int64_t M,
+                       int64_t N, int64_t K, const dq_format *fmt, float *out, dq_stream stream) {
     if (!fmt) return DQ_ERR_ARG;
-    if (fmt->codes != DQ_CODES_E2M1 || fmt->group != 32 || fmt->group_scale != DQ_SCALE_E8M0 ||
-        fmt->tensor_scale_auto != 0)
-        return DQ_ERR_FORMAT;
+    const bool mx = fmt->codes == DQ_CODES_E2M1 && fmt->group == 32 &&
+                    fmt->group_scale == DQ_SCALE_E8M0 && fmt->tensor_scale_auto == 0;
+    const bool nv = fmt->codes == DQ_CODES_E2M1 && fmt->group == 16 &&
+                    fmt->group_scale == DQ_SCALE_E4M3;
+    if (!mx && !nv) return DQ_ERR_FORMAT;
     if (M < 0 || N < 0 || K < 0 || M % 128 || N % 128 || K % 256) return DQ_ERR_SHAPE;
     if (M == 0 || N == 0) return DQ_OK;
     if (K == 0) return DQ_ERR_SHAPE;
     if (!codes_x || !scales_x || !codes_w || !scales_w || !a || !out) return DQ_ERR_ARG;
     if (!aligned(codes_x, 16) || !aligned(scales_x, 16) || !aligned(codes_w, 16) ||
-        !aligned(scales_w, 16) || !aligned(a, 16) || !aligned(out, 16))
+        !aligned(scales_w, 16) || !aligned(a, 16) || !aligned(out, 16) || !aligned(tensor_scale, 4))
         return DQ_ERR_ALIGN;
     unsigned int *status = status_ptr();
     if (!status) return DQ_ERR_CUDA;
@@ -788,10 +850,12 @@ dq_status dq_w4a4_gemm(const uint8_t *codes_x, const void *scales_x, const uint8
     L.codes_w = codes_w;
     L.scales_w = static_cast<const uint8_t *>(scales_w);
     L.a = a;
+    L.ts = tensor_scale;
     L.out = out;
     L.M = M;
     L.N = N;
     L.K = K;
+    L.nv = nv ? 1 : 0;
     L.status = status;
     L.stall = g_stall_next_gemm.exchange(0);
     L.stream = reinterpret_cast<cudaStream_t>(stream);
@@ -800,13 +864,14 @@ dq_status dq_w4a4_gemm(const uint8_t *codes_x, const void *scales_x, const uint8
     return DQ_OK;
 }
 
-dq_status dq_scale_tiles(const void *scales, int64_t rows, int64_t K, uint8_t *tiles,
-                         dq_stream stream) {
-    if (rows < 0 || K < 0 || rows % 128 || K % 128) return DQ_ERR_SHAPE;
+dq_status dq_scale_tiles(const void *scales, int64_t rows, int64_t K, int32_t group,
+                         uint8_t *tiles, dq_stream stream) {
+    if (group != 16 && group != 32) return DQ_ERR_ARG;
+    if (rows < 0 || K < 0 || rows % 128 || K % (4 * group)) return DQ_ERR_SHAPE;
     if (rows == 0 || K == 0) return DQ_OK;
     if (!scales || !tiles) return DQ_ERR_ARG;
     if (!aligned(scales, 16) || !aligned(tiles, 16)) return DQ_ERR_ALIGN;
-    DQ_CUDA(launch_scale_tiles(static_cast<const uint8_t *>(scales), rows, K, tiles,
+    DQ_CUDA(launch_scale_tiles(static_cast<const uint8_t *>(scales), rows, K, group, tiles,
                                reinterpret_cast<cudaStream_t>(stream)));
     count_launches(1);
     return DQ_OK;
@@ -1093,6 +1158,49 @@ dq_status dq_col_update(const void *W, int32_t dtype, int64_t rows, int64_t cols
                         void *workspace, size_t ws_bytes, dq_stream stream) {
     return step_impl(false, W, dtype, rows, cols, fmt, tensor_scale, a_in, b_in, b_out, b_pre,
                      mse_in, workspace, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int64_t dq_col_row_block(int64_t rows, int64_t cols, int32_t dtype) {
+    if (rows < 0 || cols < 0 || (dtype != DQ_DT_F32 && dtype != DQ_DT_BF16)) return -1;
+    return geometry(rows, cols, dtype == DQ_DT_F32).tr[1];
+}
+
+dq_status dq_col_partials(const void *W, int32_t dtype, int64_t rows, int64_t cols,
+                          const dq_format *fmt, float tensor_scale, const float *a, const float *b,
+                          int64_t row_block, float *partials, double *mse_in, void *workspace,
+                          size_t ws_bytes, dq_stream stream) {
+    return col_partials_impl(W, dtype, rows, cols, fmt, tensor_scale, a, b, row_block, partials,
+                             mse_in, workspace, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+dq_status dq_col_finalize(const float *partials, int64_t row_blocks, int64_t cols,
+                          const dq_format *fmt, float *b_out, float *b_pre, dq_stream stream) {
+    FmtInfo fi;
+    dq_status s = check_format(fmt, &fi);
+    if (s != DQ_OK) return s;
+    if (row_blocks < 0 || cols < 0 || cols % 2) return DQ_ERR_SHAPE;
+    if (cols == 0) return DQ_OK;
+    if (!b_out || (row_blocks > 0 && !partials)) return DQ_ERR_ARG;
+    if (!aligned(partials, 16) || !aligned(b_out, 4) || !aligned(b_pre, 4)) return DQ_ERR_ALIGN;
+    unsigned int *status = status_ptr();
+    if (!status) return DQ_ERR_CUDA;
+    MatDesc d{};
+    d.cols = cols;
+    d.ncb = 1;
+    d.ntiles[1] = row_blocks;
+    d.colpart = reinterpret_cast<float2 *>(const_cast<float *>(partials));
+    d.b_out = b_out;
+    d.b_pre = b_pre;
+    Launcher L;
+    L.tab.dev = nullptr;
+    L.tab.one = d;
+    L.tab.n = 1;
+    L.tab.status = status;
+    L.combo = fi.combo;
+    L.G = fi.G;
+    L.total_cols = cols;
+    L.st = reinterpret_cast<cudaStream_t>(stream);
+    return L.col_finalize();
 }
 
 dq_status dq_last_device_status(dq_stream stream) {

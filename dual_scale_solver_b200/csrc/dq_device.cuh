@@ -342,6 +342,45 @@ __device__ __forceinline__ ScaleChoice project_group(float m, float qts, float r
     }
 }
 
+// The fast-path choice of project_group alone: the same scale s and the
+// same `near` flag, without the boundary description (which project_group
+// computes when a group does sit near its boundary).
+template <int GS, int CODES>
+__device__ __forceinline__ float project_group_fast(float m, float rqts, float inv_ts, bool &near) {
+    near = false;
+    if (GS == SC_E8M0) {
+        const float mm = m * inv_ts;                   // exact (power of two)
+        if (mm < kMinNormal) return pow2f(-126);
+        const uint32_t u = __float_as_uint(mm);
+        constexpr uint32_t MT = CodeTraits<CODES>::kMT;
+        constexpr int QE = CodeTraits<CODES>::kQE;
+        const int mant = (int)(u & 0x7FFFFFu);
+        const int e = ilog2f(mm) - QE + (mant > (int)MT ? 1 : 0);
+        const int d = mant - (int)MT;
+        near = d < 16 && d > -16;
+        return pow2f(min(max(e, -126), 126));
+    } else if (GS == SC_BF16) {
+        const float g = m * rqts;
+        if (g < kMinNormal) return kMinNormal;
+        if (g >= kBf16Max) return kBf16Max;
+        // round to nearest even at the bfloat16 position (g < kBf16Max, so
+        // the rounded value stays finite and at most kBf16Max)
+        const uint32_t u = __float_as_uint(g);
+        const int d = (int)(u & 0xFFFFu) - 0x8000;
+        near = d < 16 && d > -16;
+        return __uint_as_float((u + 0x7FFFu + ((u >> 16) & 1u)) & 0xFFFF0000u);
+    } else {  // E4M3, round to nearest even, saturating at 448, 0 -> 2^-9
+        const float g = m * rqts;
+        if (g >= 448.0f) return 448.0f;
+        const int E = (g < 0.015625f) ? -6 : ilog2f(g);
+        const float t = g * pow2f(3 - E);              // exact
+        const float frac = t - floorf(t);
+        near = fabsf(frac - 0.5f) <= t * 1.9073486e-06f;
+        const float s = rintf(t) * pow2f(E - 3);       // ties to even, as project_group
+        return s == 0.0f ? 0.001953125f : fminf(s, 448.0f);
+    }
+}
+
 // ------------------------------------------------------------------------- //
 // Packed float32x2 helpers (sm_100 FFMA2 / FMUL2)
 // ------------------------------------------------------------------------- //
@@ -413,18 +452,23 @@ struct Quant {
         if (GS == SC_E8M0 && kExactM) {
             // (e <= 126 holds for finite m)
             s = __uint_as_float(e8m0_scale_bits(mb));
-            if (NIB && !pos) s = 1.0f;                     // stored scale of an all-zero group
+            // an all-zero group (also the zero chunks of lanes past the last
+            // column) takes scale 1: its stored scale, and the scale its codes
+            // are formed with -- with s at the 2^-126 floor, 1 / (a s) would
+            // overflow for a <= 1/4 and turn the zeros into NaN
+            if (!pos) s = 1.0f;
         } else {
             // every lane takes part in the warp vote and group shuffles below,
             // whatever its group holds (all-zero and out-of-range groups too)
             const float qts = kHasTs ? kQmax * ts : kQmax;
             const float rqts = kHasTs ? 1.0f / qts : 1.0f / kQmax;
-            ScaleChoice sc = project_group<GS, CODES>(pos ? m : 1.0f, qts, rqts,
-                                                      kHasTs ? inv_ts : 1.0f);
-            s = sc.s;
-            const bool resolve = pos && sc.near;
+            bool near;
+            s = project_group_fast<GS, CODES>(pos ? m : 1.0f, rqts, kHasTs ? inv_ts : 1.0f, near);
+            const bool resolve = pos && near;
             if (__any_sync(0xffffffffu, resolve)) {
                 // exact comparison of the true group max with sc.thr
+                const ScaleChoice sc = project_group<GS, CODES>(pos ? m : 1.0f, qts, rqts,
+                                                                kHasTs ? inv_ts : 1.0f);
                 int gt = 0, eq = 0;
                 if (resolve) {
                     if (kExactM) {
@@ -478,7 +522,9 @@ struct Quant {
                     const f2 d = __fadd2_rn(q[k], neg2(c[k]));
                     dmax = max3_nan(dmax, fabsf(d.x), fabsf(d.y));
                 }
-                if (dmax > 0.5f - 1.52587890625e-05f) {
+                // (rare: a warp-uniform branch, so that the fix-up below is
+                // not issued for every chunk)
+                if (__any_sync(0xffffffffu, dmax > 0.5f - 1.52587890625e-05f)) {
 #pragma unroll
                     for (int k = 0; k < NP; ++k)
 #pragma unroll
@@ -523,15 +569,26 @@ struct Quant {
 #pragma unroll
                 for (int k = 0; k < NP; ++k) c[k] = e2m1_round2_byte(q[k].x, q[k].y, byte[k]);
                 if (!kExactQ) {
+                    // a code is near a decision boundary when q scaled by
+                    // 1 +- 2^-17 rounds to two different codes; such codes
+                    // (rare) are settled exactly behind one warp-uniform branch
                     const f2 up = bcast(1.0f + 7.62939453125e-06f), dn = bcast(1.0f - 7.62939453125e-06f);
+                    uint32_t bh[NP], bl[NP];
+                    bool any_near = false;
 #pragma unroll
                     for (int k = 0; k < NP; ++k) {
                         const f2 qh = mul2(q[k], up), ql = mul2(q[k], dn);
-                        const uint32_t bh = cvt_e2m1x2(qh.y, qh.x), bl = cvt_e2m1x2(ql.y, ql.x);
-                        if (bh != bl) {
+                        bh[k] = cvt_e2m1x2(qh.y, qh.x);
+                        bl[k] = cvt_e2m1x2(ql.y, ql.x);
+                        any_near |= bh[k] != bl[k];
+                    }
+                    if (__any_sync(0xffffffffu, any_near)) {
+#pragma unroll
+                    for (int k = 0; k < NP; ++k) {
+                        if (bh[k] != bl[k]) {
 #pragma unroll
                             for (int h = 0; h < 2; ++h) {
-                                const uint32_t nh = (bh >> (4 * h)) & 0xF, nl = (bl >> (4 * h)) & 0xF;
+                                const uint32_t nh = (bh[k] >> (4 * h)) & 0xF, nl = (bl[k] >> (4 * h)) & 0xF;
                                 if (nh != nl) {
                                     const float2 vh = e2m1x2_to_f32(nh), vl = e2m1x2_to_f32(nl);
                                     const float mh = fabsf(vh.x), ml = fabsf(vl.x);
@@ -550,6 +607,7 @@ struct Quant {
                                 }
                             }
                         }
+                    }
                     }
                 }
                 if (NIB) {

@@ -6,13 +6,17 @@
 //
 //   out[m, n] = a_n * sum_k  Qx[m, k] * Qw[n, k]
 //
-// Qx = the MXFP4 codes and E8M0 group scales of Q(X D_b) (dq_act_rescale_quant),
-// Qw = the MXFP4 codes and E8M0 group scales of Q(W / (a b^T)) (the solve), a =
-// the outer row scales of W.  Both operands are K-major E2M1, two codes per
-// byte, with one E8M0 scale per 32 elements of K; the scales come in scale
-// tiles, the layout the tensor core reads (scale_tiles_kernel below): per
-// 128-row block and 128 elements of K one 512-byte chunk holding the scale
-// k (0..3) of row r at byte (r % 32) * 16 + (r / 32) * 4 + k.
+// Qx = the E2M1 codes and group scales of Q(X D_b) (dq_act_rescale_quant),
+// Qw = the E2M1 codes and group scales of Q(W / (a b^T)) (the solve), a = the
+// outer row scales of W.  Both operands are K-major E2M1, two codes per byte,
+// with one group scale per G elements of K: MXFP4, an E8M0 scale per 32
+// (kind::mxf4, block32); NVFP4, an E4M3 scale per 16 (kind::mxf4nvf4,
+// block16) and the weights' tensor scale ts (a power of two) applied with
+// a_n in the epilogue (news article, "适配 MXFP4 与 NVFP4 块结构").  The
+// scales come in scale tiles, the layout the tensor core reads
+// (scale_tiles_kernel below): per 128-row block and 4 G elements of K one
+// 512-byte chunk holding the scale k (0..3) of row r at byte (r % 32) * 16 +
+// (r / 32) * 4 + k.
 //
 // A persistent CTA per SM walks 128 x BN tiles of `out` (BN = 256, or 128
 // when N is not a multiple of 256) with tcgen05.mma kind::mxf4 (M = 128,
@@ -46,14 +50,15 @@ constexpr int kThreadsGemm = 320;               // 10 warps: producer, MMA, 8 ep
 constexpr uint64_t kWaitLimitNs = 1000000000ull;   // a wait gives up after 1 s
 
 // BN = 128 or 256 output columns per CTA; BK = 128 or 256 K elements per
-// stage (64- or 128-byte rows, 64- or 128-byte swizzle).
-template <int BN, int BK>
+// stage (64- or 128-byte rows, 64- or 128-byte swizzle); NV: NVFP4 (scale
+// chunks of 64 elements of K) rather than MXFP4 (128).
+template <int BN, int BK, bool NV>
 struct __align__(1024) GemmSmem {
     // 128-column tiles run two CTAs per SM (one's epilogue overlaps the
     // other's MMAs); the ring depth fills the shared memory
     static constexpr int kCtasPerSm = BN == 128 ? 2 : 1;
     static constexpr int NB = BN / 128;                        // 128-row blocks of B
-    static constexpr int KC = BK / 128;                        // 4-scale chunks per row and stage
+    static constexpr int KC = BK / (NV ? 64 : 128);            // 4-scale chunks per row and stage
     static constexpr int kRowBytes = BK / 2;
     static constexpr int kTileBytesA = kBM * kRowBytes;
     static constexpr int kTileBytesB = BN * kRowBytes;
@@ -162,17 +167,18 @@ __device__ __forceinline__ uint64_t desc_sf(uint32_t saddr) {
     return (uint64_t)((saddr & 0x3FFFFu) >> 4) | (1ull << 16) | (8ull << 32) | (1ull << 46);
 }
 
-// Instruction descriptor, kind::mxf4 with E8M0 block scales: A and B E2M1
-// (K-major), M = BM (128, or 256 for a CTA pair), N = BN, scale-factor byte
-// ids of A and B.
-template <int BM, int BN>
+// Instruction descriptor of the block-scaled E2M1 kinds: A and B E2M1
+// (format 1, K-major), M = BM (128, or 256 for a CTA pair), N = BN, the
+// scale type (bit 23: 1 = UE8M0 for MXFP4, 0 = UE4M3 for NVFP4) and the
+// scale-factor byte ids of A and B.
+template <int BM, int BN, bool NV>
 __device__ __forceinline__ uint32_t idesc_mxf4_m(uint32_t sfa_id, uint32_t sfb_id) {
-    return (sfb_id << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | (1u << 23) |
-           ((uint32_t)(BM >> 4) << 24) | (sfa_id << 29);
+    return (sfb_id << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
+           ((NV ? 0u : 1u) << 23) | ((uint32_t)(BM >> 4) << 24) | (sfa_id << 29);
 }
-template <int BN>
+template <int BN, bool NV>
 __device__ __forceinline__ uint32_t idesc_mxf4(uint32_t sfa_id, uint32_t sfb_id) {
-    return idesc_mxf4_m<kBM, BN>(sfa_id, sfb_id);
+    return idesc_mxf4_m<kBM, BN, NV>(sfa_id, sfb_id);
 }
 
 // Output tile t -> (m0, n0).  Tiles go in bands of up to kBandTiles tile
@@ -192,15 +198,26 @@ __device__ __forceinline__ void tile_coords(int t, int m_tiles, int n_tiles, int
     n0 = (nb0 + r % width) * bn;
 }
 
+// One MMA of K = 64: MXFP4 takes 2 E8M0 scales per row (bytes id, id + 1
+// of the scale column), NVFP4 4 E4M3 scales (the whole column, id 0).
+template <bool NV>
 __device__ __forceinline__ void mma_mxf4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
                                          uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
                                          uint32_t accumulate) {
-    asm volatile(
-        "{ .reg .pred p; setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p; }"
-        :: "r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem),
-           "r"(sfb_tmem)
-        : "memory");
+    if constexpr (NV)
+        asm volatile(
+            "{ .reg .pred p; setp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p; }"
+            :: "r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem),
+               "r"(sfb_tmem)
+            : "memory");
+    else
+        asm volatile(
+            "{ .reg .pred p; setp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p; }"
+            :: "r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem),
+               "r"(sfb_tmem)
+            : "memory");
 }
 
 __device__ __forceinline__ void tmem_cp_sf(uint32_t taddr, uint64_t sdesc) {
@@ -244,12 +261,12 @@ __device__ __forceinline__ void mbar_drain(uint64_t *b, uint32_t parity) {
     }
 }
 
-template <int BN, int BK>
-__global__ void __launch_bounds__(kThreadsGemm, GemmSmem<BN, BK>::kCtasPerSm)
+template <int BN, int BK, bool NV>
+__global__ void __launch_bounds__(kThreadsGemm, GemmSmem<BN, BK, NV>::kCtasPerSm)
 w4a4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
-                 const uint8_t *sf_a, const uint8_t *sf_b, const float *a_row, float *out, int M,
-                 int N, int K, unsigned int *status, int stall) {
-    using Smem = GemmSmem<BN, BK>;
+                 const uint8_t *sf_a, const uint8_t *sf_b, const float *a_row, const float *ts_w,
+                 float *out, int M, int N, int K, unsigned int *status, int stall) {
+    using Smem = GemmSmem<BN, BK, NV>;
     constexpr int kStages = Smem::kStages;
     constexpr int KC = Smem::KC;
     constexpr int NB = Smem::NB;
@@ -299,7 +316,7 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
         // the current tile's last MMAs and epilogue. ----
         int g = 0;
         bool stop = false;
-        const int64_t kblocks = K / 128;             // scale chunks per 128-row block
+        const int64_t kblocks = K / (NV ? 64 : 128);  // scale chunks per 128-row block
         for (int t = blockIdx.x; t < tiles && !stop; t += gridDim.x) {
             int m0, n0;
             tile_coords(t, m_tiles, n_tiles, kBM, BN, m0, n0);
@@ -351,14 +368,15 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
                     const uint32_t a0 = smem_u32(sm.a[s]), b0 = smem_u32(sm.b[s]);
 #pragma unroll
                     for (int kb = 0; kb < BK / 64; ++kb) {
-                        // K = 64 per instruction: 32 bytes of each row; scale
-                        // blocks 2kb, 2kb+1 = k-chunk kb/2, bytes 2(kb%2),
-                        // 2(kb%2)+1 of the word; B's scales of the k-chunk
-                        // span NB x 4 columns
-                        const uint32_t c = kb >> 1, id = (kb & 1) * 2;
-                        mma_mxf4(tmem, desc_swz<BK / 2>(a0 + kb * 32), desc_swz<BK / 2>(b0 + kb * 32),
-                                 idesc_mxf4<BN>(id, id), sfa_t + 4 * c, sfb_t + 4 * NB * c,
-                                 (kt | kb) != 0);
+                        // K = 64 per instruction: 32 bytes of each row.
+                        // MXFP4: scale blocks 2kb, 2kb+1 = k-chunk kb/2, bytes
+                        // 2(kb%2), 2(kb%2)+1 of the word; NVFP4: scale blocks
+                        // 4kb .. 4kb+3 = k-chunk kb, the whole word.  B's
+                        // scales of a k-chunk span NB x 4 columns
+                        const uint32_t c = NV ? kb : kb >> 1, id = NV ? 0 : (kb & 1) * 2;
+                        mma_mxf4<NV>(tmem, desc_swz<BK / 2>(a0 + kb * 32), desc_swz<BK / 2>(b0 + kb * 32),
+                                     idesc_mxf4<BN, NV>(id, id), sfa_t + 4 * c, sfb_t + 4 * NB * c,
+                                     (kt | kb) != 0);
                     }
                     umma_commit(&sm.empty[s]);      // frees the stage once these MMAs are done
                 }
@@ -386,6 +404,7 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
         // rows then cover all eight 16-byte bank groups
         auto sw = [](int r) { return (r / (8 / CPR)) % CPR; };
         const int rr = lane / CPR, cc = lane % CPR;  // this lane's row / chunk in the store pass
+        const float ts = ts_w ? __ldg(ts_w) : 1.0f;  // the weights' tensor scale
         int j = 0;
         for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++j) {
             int m0, n0;
@@ -418,7 +437,8 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
                 }
                 __syncwarp();
                 const int col = h * EC + 4 * cc;
-                const float4 sc = __ldg(reinterpret_cast<const float4 *>(a_row + n0 + cbase + col));
+                float4 sc = __ldg(reinterpret_cast<const float4 *>(a_row + n0 + cbase + col));
+                sc = make_float4(sc.x * ts, sc.y * ts, sc.z * ts, sc.w * ts);   // exact: ts = 2^k
 #pragma unroll
                 for (int p = 0; p < CPR; ++p) {
                     const int r = p * RPP + rr;
@@ -463,9 +483,9 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
 //               scales to both TMEMs (tcgen05.cp.cta_group::2), issues the
 //               MMAs, and commits to the barriers of both CTAs.
 // ---------------------------------------------------------------------------
-template <int BK>
+template <int BK, bool NV>
 struct __align__(1024) GemmPairSmem {
-    static constexpr int KC = BK / 128;
+    static constexpr int KC = BK / (NV ? 64 : 128);
     static constexpr int kRowBytes = BK / 2;
     static constexpr int kTileBytes = 128 * kRowBytes;                 // A or B half, per CTA
     static constexpr int kStageBytes = 2 * kTileBytes + 3 * KC * kSfChunk;
@@ -517,15 +537,24 @@ __device__ __forceinline__ void tma_load_2d_pair(void *dst, const CUtensorMap *m
         : "memory");
 }
 
+template <bool NV>
 __device__ __forceinline__ void mma_mxf4_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
                                               uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
                                               uint32_t accumulate) {
-    asm volatile(
-        "{ .reg .pred p; setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::2.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p; }"
-        :: "r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem),
-           "r"(sfb_tmem)
-        : "memory");
+    if constexpr (NV)
+        asm volatile(
+            "{ .reg .pred p; setp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p; }"
+            :: "r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem),
+               "r"(sfb_tmem)
+            : "memory");
+    else
+        asm volatile(
+            "{ .reg .pred p; setp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::2.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p; }"
+            :: "r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem),
+               "r"(sfb_tmem)
+            : "memory");
 }
 
 __device__ __forceinline__ void tmem_cp_sf_pair(uint32_t taddr, uint64_t sdesc) {
@@ -543,13 +572,14 @@ __device__ __forceinline__ void umma_commit_pair(uint64_t *bar) {
         :: "r"(smem_u32(bar)) : "memory");
 }
 
-template <int BK>
+template <int BK, bool NV>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsGemm, 1)
 w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                       const __grid_constant__ CUtensorMap map_sfa,
-                      const __grid_constant__ CUtensorMap map_sfb, const float *a_row, float *out,
-                      int M, int N, int K, unsigned int *status, int stall) {
-    using Smem = GemmPairSmem<BK>;
+                      const __grid_constant__ CUtensorMap map_sfb, const float *a_row,
+                      const float *ts_w, float *out, int M, int N, int K, unsigned int *status,
+                      int stall) {
+    using Smem = GemmPairSmem<BK, NV>;
     constexpr int kStages = Smem::kStages;
     constexpr int KC = Smem::KC;
     constexpr int BN = 256;
@@ -564,7 +594,7 @@ w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_co
     const int n_tiles = N / BN, m_tiles = M / 256;
     const int tiles = m_tiles * n_tiles;
     const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
-    const int64_t kblocks = K / 128;                // scale chunks per 128-row block
+    const int64_t kblocks = K / (NV ? 64 : 128);    // scale chunks per 128-row block
     volatile int *abort = &sm.abort;
 
     if (threadIdx.x == 0) {
@@ -645,10 +675,10 @@ w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_co
                     const uint32_t a0 = smem_u32(sm.a[s]), b0 = smem_u32(sm.b[s]);
 #pragma unroll
                     for (int kb = 0; kb < BK / 64; ++kb) {
-                        const uint32_t c = kb >> 1, id = (kb & 1) * 2;
-                        mma_mxf4_pair(tmem, desc_swz<BK / 2>(a0 + kb * 32), desc_swz<BK / 2>(b0 + kb * 32),
-                                      idesc_mxf4_m<256, BN>(id, id), sfa_t + 4 * c, sfb_t + 8 * c,
-                                      (kt | kb) != 0);
+                        const uint32_t c = NV ? kb : kb >> 1, id = NV ? 0 : (kb & 1) * 2;
+                        mma_mxf4_pair<NV>(tmem, desc_swz<BK / 2>(a0 + kb * 32), desc_swz<BK / 2>(b0 + kb * 32),
+                                          idesc_mxf4_m<256, BN, NV>(id, id), sfa_t + 4 * c, sfb_t + 8 * c,
+                                          (kt | kb) != 0);
                     }
                     umma_commit_pair(&sm.empty[s]);  // frees the stage in both CTAs
                 }
@@ -668,6 +698,7 @@ w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_co
         auto sw = [](int r) { return (r / (8 / CPR)) % CPR; };
         const int rr = lane / CPR, cc = lane % CPR;
         const uint32_t acc_empty0 = cluster_addr(&sm.acc_empty, 0);
+        const float ts = ts_w ? __ldg(ts_w) : 1.0f;  // the weights' tensor scale
         int j = 0;
         for (int t = pair; t < tiles; t += npairs, ++j) {
             int m0, n0;
@@ -700,7 +731,8 @@ w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_co
                 }
                 __syncwarp();
                 const int col = h * EC + 4 * cc;
-                const float4 sc = __ldg(reinterpret_cast<const float4 *>(a_row + n0 + cbase + col));
+                float4 sc = __ldg(reinterpret_cast<const float4 *>(a_row + n0 + cbase + col));
+                sc = make_float4(sc.x * ts, sc.y * ts, sc.z * ts, sc.w * ts);   // exact: ts = 2^k
 #pragma unroll
                 for (int p = 0; p < CPR; ++p) {
                     const int r = p * RPP + rr;
@@ -740,8 +772,8 @@ w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_co
     }
 }
 
-// Row-major E8M0 scales [rows, K/32] -> scale tiles: one thread per 4-byte
-// word (the 4 scales of one row in one 128-element K block); word w of chunk
+// Row-major group scales [rows, K/G] -> scale tiles: one thread per 4-byte
+// word (the 4 scales of one row in one 4G-element K block); word w of chunk
 // (rb, kc) holds row rb*128 + (w % 4)*32 + w/4, so the writes are coalesced.
 __global__ void __launch_bounds__(256)
 scale_tiles_kernel(const uint8_t *scales, int64_t words, int64_t kblocks, uint8_t *tiles) {
@@ -786,11 +818,12 @@ bool code_map(CUtensorMap *m, const uint8_t *codes, int64_t rows, int64_t K, int
 }
 
 // 2-D map over scale tiles as rows of one 512-byte chunk (256 x 16-bit
-// elements): boxes of KC consecutive chunks, no swizzle.
-bool scale_tile_map(CUtensorMap *m, const uint8_t *tiles, int64_t rows, int64_t K, int kc) {
+// elements): boxes of KC consecutive chunks, no swizzle; kblocks chunks per
+// 128-row block.
+bool scale_tile_map(CUtensorMap *m, const uint8_t *tiles, int64_t rows, int64_t kblocks, int kc) {
     auto enc = tensor_map_encoder();
     if (!enc) return false;
-    const cuuint64_t dims[2] = {256, (cuuint64_t)(rows / 128 * (K / 128))};
+    const cuuint64_t dims[2] = {256, (cuuint64_t)(rows / 128 * kblocks)};
     const cuuint64_t strides[1] = {512};
     const cuuint32_t box[2] = {256, (cuuint32_t)kc};
     const cuuint32_t estr[2] = {1, 1};
@@ -799,18 +832,19 @@ bool scale_tile_map(CUtensorMap *m, const uint8_t *tiles, int64_t rows, int64_t 
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int BK>
+template <int BK, bool NV>
 cudaError_t launch_pair(const GemmLaunch &L) {
-    using Smem = GemmPairSmem<BK>;
+    using Smem = GemmPairSmem<BK, NV>;
     static_assert(sizeof(Smem) + 1024 <= 232448, "shared memory of the GEMM CTA");
     CUtensorMap ma, mb, msa, msb;
+    const int64_t kblocks = L.K / (NV ? 64 : 128);
     if (!code_map(&ma, L.codes_x, L.M, L.K, 128, BK / 2) || !code_map(&mb, L.codes_w, L.N, L.K, 128, BK / 2) ||
-        !scale_tile_map(&msa, L.scales_x, L.M, L.K, Smem::KC) ||
-        !scale_tile_map(&msb, L.scales_w, L.N, L.K, Smem::KC))
+        !scale_tile_map(&msa, L.scales_x, L.M, kblocks, Smem::KC) ||
+        !scale_tile_map(&msb, L.scales_w, L.N, kblocks, Smem::KC))
         return cudaErrorInvalidValue;
     const size_t smem = sizeof(Smem) + 1024;
     static std::atomic<bool> done[64];
-    cudaError_t e = smem_opt_in(w4a4_gemm_pair_kernel<BK>, smem, done);
+    cudaError_t e = smem_opt_in(w4a4_gemm_pair_kernel<BK, NV>, smem, done);
     if (e != cudaSuccess) return e;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
@@ -819,13 +853,13 @@ cudaError_t launch_pair(const GemmLaunch &L) {
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) sms = 148;
     const int64_t tiles = (L.M / 256) * (L.N / 256);
     const unsigned grid = 2u * (unsigned)std::min<int64_t>(tiles, sms / 2);
-    return launch_k(w4a4_gemm_pair_kernel<BK>, dim3(grid), dim3(kThreadsGemm), smem, L.stream, ma, mb,
-                    msa, msb, L.a, L.out, (int)L.M, (int)L.N, (int)L.K, L.status, L.stall);
+    return launch_k(w4a4_gemm_pair_kernel<BK, NV>, dim3(grid), dim3(kThreadsGemm), smem, L.stream, ma,
+                    mb, msa, msb, L.a, L.ts, L.out, (int)L.M, (int)L.N, (int)L.K, L.status, L.stall);
 }
 
-template <int BN, int BK>
+template <int BN, int BK, bool NV>
 cudaError_t launch_bn(const GemmLaunch &L) {
-    using Smem = GemmSmem<BN, BK>;
+    using Smem = GemmSmem<BN, BK, NV>;
     static_assert(sizeof(Smem) + 1024 <= (Smem::kCtasPerSm == 2 ? 115712 : 232448),
                   "shared memory of the GEMM CTA");
     CUtensorMap ma, mb;
@@ -833,7 +867,7 @@ cudaError_t launch_bn(const GemmLaunch &L) {
         return cudaErrorInvalidValue;
     const size_t smem = sizeof(Smem) + 1024;
     static std::atomic<bool> done[64];
-    cudaError_t e = smem_opt_in(w4a4_gemm_kernel<BN, BK>, smem, done);
+    cudaError_t e = smem_opt_in(w4a4_gemm_kernel<BN, BK, NV>, smem, done);
     if (e != cudaSuccess) return e;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
@@ -842,8 +876,9 @@ cudaError_t launch_bn(const GemmLaunch &L) {
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) sms = 148;
     const int64_t tiles = (L.M / kBM) * (L.N / BN);
     const unsigned grid = (unsigned)std::min<int64_t>(tiles, (int64_t)sms * Smem::kCtasPerSm);
-    return launch_k(w4a4_gemm_kernel<BN, BK>, dim3(grid), dim3(kThreadsGemm), smem, L.stream, ma, mb,
-                    L.scales_x, L.scales_w, L.a, L.out, (int)L.M, (int)L.N, (int)L.K, L.status, L.stall);
+    return launch_k(w4a4_gemm_kernel<BN, BK, NV>, dim3(grid), dim3(kThreadsGemm), smem, L.stream, ma,
+                    mb, L.scales_x, L.scales_w, L.a, L.ts, L.out, (int)L.M, (int)L.N, (int)L.K,
+                    L.status, L.stall);
 }
 
 }  // namespace
@@ -853,19 +888,24 @@ constexpr int kGemmBK = 256;
 // A CTA pair per 256 x 256 tile when M and N allow it; else one CTA per
 // 128 x 256 tile when N allows it (A tiles reused twice as often), else
 // 128 x 128.
-cudaError_t launch_scale_tiles(const uint8_t *scales, int64_t rows, int64_t K, uint8_t *tiles,
+cudaError_t launch_scale_tiles(const uint8_t *scales, int64_t rows, int64_t K, int G, uint8_t *tiles,
                                cudaStream_t stream) {
-    const int64_t words = rows * K / 128;
+    const int64_t words = rows * K / (4 * G);
     if (words == 0) return cudaSuccess;
     const int64_t blocks = std::min<int64_t>((words + 255) / 256, 148 * 16);
     return launch_k(scale_tiles_kernel, dim3((unsigned)blocks), dim3(256), 0, stream, scales, words,
-                    K / 128, tiles);
+                    K / (4 * G), tiles);
+}
+
+template <bool NV>
+cudaError_t launch_w4a4_gemm_fmt(const GemmLaunch &L) {
+    if (L.M % 256 == 0 && L.N % 256 == 0) return launch_pair<kGemmBK, NV>(L);
+    return (L.N % 256 == 0) ? launch_bn<256, kGemmBK, NV>(L) : launch_bn<128, kGemmBK, NV>(L);
 }
 
 cudaError_t launch_w4a4_gemm(const GemmLaunch &L) {
     if (L.M == 0 || L.N == 0) return cudaSuccess;
-    if (L.M % 256 == 0 && L.N % 256 == 0) return launch_pair<kGemmBK>(L);
-    return (L.N % 256 == 0) ? launch_bn<256, kGemmBK>(L) : launch_bn<128, kGemmBK>(L);
+    return L.nv ? launch_w4a4_gemm_fmt<true>(L) : launch_w4a4_gemm_fmt<false>(L);
 }
 
 }  // namespace dq

@@ -115,21 +115,23 @@ struct TwoLevelLaunch {
 };
 cudaError_t launch_two_level(const TwoLevelLaunch &L);
 
-// Block-scaled W4A4 GEMM (dq_gemm.cu): out[M, N] = a_n * Qx[M, K] . Qw[N, K]^T.
+// Block-scaled W4A4 GEMM (dq_gemm.cu): out[M, N] = a_n ts * Qx[M, K] . Qw[N, K]^T.
 struct GemmLaunch {
-    const uint8_t *codes_x, *scales_x;   // [M, K/2] E2M1, M*K/32 E8M0 in scale tiles
-    const uint8_t *codes_w, *scales_w;   // [N, K/2] E2M1, N*K/32 E8M0 in scale tiles
+    const uint8_t *codes_x, *scales_x;   // [M, K/2] E2M1, M*K/G group scales in scale tiles
+    const uint8_t *codes_w, *scales_w;   // [N, K/2] E2M1, N*K/G group scales in scale tiles
     const float *a;                      // [N]
+    const float *ts;                     // the weights' tensor scale (1 float) or NULL (1)
     float *out;                          // [M, N]
     int64_t M, N, K;                     // multiples of 128, 128, 256
+    int nv;                              // 1: NVFP4 (E4M3 scales, G16); 0: MXFP4 (E8M0, G32)
     unsigned int *status;
     int stall;                           // test support: skip the loads of the first K tile
     cudaStream_t stream;
 };
 cudaError_t launch_w4a4_gemm(const GemmLaunch &L);
-// Row-major E8M0 scales [rows, K/32] -> the GEMM's scale tiles (rows a
-// multiple of 128, K of 128).
-cudaError_t launch_scale_tiles(const uint8_t *scales, int64_t rows, int64_t K, uint8_t *tiles,
+// Row-major group scales [rows, K/G] -> the GEMM's scale tiles (rows a
+// multiple of 128, K of 4 G).
+cudaError_t launch_scale_tiles(const uint8_t *scales, int64_t rows, int64_t K, int G, uint8_t *tiles,
                                cudaStream_t stream);
 
 cudaError_t launch_tile_c0(const TileLaunch &L);

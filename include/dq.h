@@ -236,6 +236,41 @@ DQ_API dq_status dq_col_update(const void *W, int32_t dtype, int64_t rows, int64
                         const float *b_in, float *b_out, float *b_pre, double *mse_in,
                         void *workspace, size_t ws_bytes, dq_stream stream);
 
+/* The column half-step split for a matrix whose rows are sharded (over
+ * GPUs, say): the column statistics of eq. (2) are sums over all rows, so
+ * each shard contributes partial sums and one fixed-order sum of all
+ * shards' partials gives the update.  No counterpart in the pages (the
+ * multi-GPU split of the closed form).
+ * dq_col_row_block: the number of rows per row block of the column
+ *   statistics of a rows x cols matrix (dtype DQ_DT_BF16 or DQ_DT_F32), as
+ *   dq_col_update and the solves use it; -1 on bad arguments.
+ * dq_col_partials: for the shard W [rows, cols] (its own rows, with their
+ *   row scales a [rows] and the matrix's b [cols]; tensor_scale as in
+ *   dq_col_update), the partial sums (sum_i W_ij S_ij, sum_i S_ij^2),
+ *   S = D_a Q(W ⊘ a bᵀ), over each block of `row_block` consecutive shard
+ *   rows: `partials` receives ceil(rows / row_block) x cols float pairs
+ *   (P, E), row block major, 16-byte aligned, caller-owned.  row_block is
+ *   the whole matrix's dq_col_row_block (a shard's own is never larger;
+ *   a smaller one is refused with DQ_ERR_SHAPE).  mse_in (1 double, may be
+ *   NULL) receives the shard's MSE sum / (rows cols) at the input state.
+ *   workspace as dq_col_update.
+ * dq_col_finalize: b_out_j = Pi_Fb(sum_k P[k][j] / sum_k E[k][j]) (zero
+ *   slice -> 1) over row_blocks slabs of cols float pairs (row block
+ *   major), summed in the fixed order of the solves' column update; b_pre
+ *   (may be NULL) the unprojected ratios.
+ * With shards whose first rows are multiples of row_block, the shards'
+ * partials concatenated in row order are the whole matrix's, so
+ * dq_col_finalize gives dq_col_update's b bit for bit. */
+DQ_API int64_t dq_col_row_block(int64_t rows, int64_t cols, int32_t dtype);
+DQ_API dq_status dq_col_partials(const void *W, int32_t dtype, int64_t rows, int64_t cols,
+                                 const dq_format *fmt, float tensor_scale, const float *a,
+                                 const float *b, int64_t row_block, float *partials,
+                                 double *mse_in, void *workspace, size_t ws_bytes,
+                                 dq_stream stream);
+DQ_API dq_status dq_col_finalize(const float *partials, int64_t row_blocks, int64_t cols,
+                                 const dq_format *fmt, float *b_out, float *b_pre,
+                                 dq_stream stream);
+
 /* Activation side of eq. (1): Q(X D_b) with ts = 1 — each input channel j is
  * multiplied by b_j, then quantized in groups of G along K (the trove summary,
  * "How to use it": beta is applied inside the activation-quantization kernel).
@@ -265,36 +300,42 @@ DQ_API dq_status dq_two_level_quant(const void *X, int32_t dtype, int64_t rows, 
                                     void *inner_scales, float *outer_scales, float *qdq,
                                     dq_stream stream);
 
-/* Scale tiles: the layout in which dq_w4a4_gemm takes E8M0 group scales
- * (G = 32), the one the tensor core reads them in.  For every block of 128
- * rows and every 128 elements of K (4 scales per row) one 512-byte chunk,
- * chunks ordered [row block][K block]; inside a chunk the scale k (0..3) of
- * row r (0..127 within the block) sits at byte (r % 32) * 16 + (r / 32) * 4
- * + k.  rows * K / 32 bytes in all, like the row-major array.
- * dq_scale_tiles rewrites row-major scales [rows, K/32] (the layout written
+/* Scale tiles: the layout in which dq_w4a4_gemm takes group scales (E8M0
+ * per 32 elements for MXFP4, E4M3 per 16 for NVFP4), the one the tensor core
+ * reads them in.  For every block of 128 rows and every 4 G elements of K (4
+ * scales per row) one 512-byte chunk, chunks ordered [row block][K block];
+ * inside a chunk the scale k (0..3) of row r (0..127 within the block) sits
+ * at byte (r % 32) * 16 + (r / 32) * 4 + k.  rows * K / G bytes in all, like
+ * the row-major array.
+ * dq_scale_tiles rewrites row-major scales [rows, K/G] (the layout written
  * by dq_solve_dual_scale, dq_quantize and dq_act_rescale_quant) into scale
- * tiles: rows and K multiples of 128, both pointers 16-byte aligned, device,
- * caller-owned, not overlapping.  Errors: DQ_ERR_SHAPE, DQ_ERR_ARG,
- * DQ_ERR_ALIGN.  (No counterpart in the method: a data layout.) */
-DQ_API dq_status dq_scale_tiles(const void *scales, int64_t rows, int64_t K, uint8_t *tiles,
-                                dq_stream stream);
+ * tiles: G = 16 or 32, rows a multiple of 128 and K of 4 G, both pointers
+ * 16-byte aligned, device, caller-owned, not overlapping.  Errors:
+ * DQ_ERR_SHAPE, DQ_ERR_ARG (also for another G), DQ_ERR_ALIGN.  (No
+ * counterpart in the method: a data layout.) */
+DQ_API dq_status dq_scale_tiles(const void *scales, int64_t rows, int64_t K, int32_t group,
+                                uint8_t *tiles, dq_stream stream);
 
 /* Block-scaled W4A4 GEMM on the tensor cores, the inference step of eq. (1)
  * (daiwk note, "核心公式": X W^T ~= (X D_b) Qhat^T D_a; trove summary, "How to
- * use it"):  out[m, n] = a_n * sum_k Qx[m, k] * Qw[n, k], float32, where Qx
- * is given by codes_x [M, K/2] and scales_x (M * K/32 bytes, scale tiles of
- * the dq_act_rescale_quant scales) and Qw by codes_w [N, K/2] and scales_w
- * (N * K/32 bytes, scale tiles of the solve's group scales), a [N] the outer
- * row scales of W.  `fmt` must be MXFP4 (E2M1 codes, E8M0 group scales, G =
- * 32).  M and N multiples of 128, K a multiple of 256; every pointer 16-byte
- * aligned; out [M, N] row-major, caller-owned.  The products are
- * accumulated in float32.  Errors:
- * DQ_ERR_FORMAT, DQ_ERR_SHAPE, DQ_ERR_ARG, DQ_ERR_ALIGN; a stalled pipeline
- * (a bounded wait that ran out) raises the device flag read by
+ * use it"):  out[m, n] = a_n * ts * sum_k Qx[m, k] * Qw[n, k], float32,
+ * where Qx is given by codes_x [M, K/2] and scales_x (M * K/G bytes, scale
+ * tiles of the dq_act_rescale_quant scales) and Qw by codes_w [N, K/2] and
+ * scales_w (N * K/G bytes, scale tiles of the solve's group scales), a [N]
+ * the outer row scales of W and ts the weights' tensor scale (device, one
+ * float as the solve wrote it; NULL reads as 1).  `fmt` is MXFP4 (E2M1
+ * codes, E8M0 group scales, G = 32) or NVFP4 (E2M1 codes, E4M3 group scales,
+ * G = 16; news article, "适配 MXFP4 与 NVFP4 块结构"); the activations are
+ * quantized with tensor scale 1.  M and N multiples of 128, K a multiple of
+ * 256; every pointer 16-byte aligned (tensor_scale 4-byte); out [M, N]
+ * row-major, caller-owned.  The products are accumulated in float32.
+ * Errors: DQ_ERR_FORMAT, DQ_ERR_SHAPE, DQ_ERR_ARG, DQ_ERR_ALIGN; a stalled
+ * pipeline (a bounded wait that ran out) raises the device flag read by
  * dq_last_device_status as DQ_ERR_TIMEOUT. */
 DQ_API dq_status dq_w4a4_gemm(const uint8_t *codes_x, const void *scales_x, const uint8_t *codes_w,
-                              const void *scales_w, const float *a, int64_t M, int64_t N,
-                              int64_t K, const dq_format *fmt, float *out, dq_stream stream);
+                              const void *scales_w, const float *a, const float *tensor_scale,
+                              int64_t M, int64_t N, int64_t K, const dq_format *fmt, float *out,
+                              dq_stream stream);
 
 /* Test support for the failure path (no counterpart in the method): the
  * next dq_w4a4_gemm call on any thread has its producer skip the loads of

@@ -126,21 +126,32 @@ def test_w4a4_gemm_argument_errors():
     L = dq.lib()
     f = dq.format_preset("mxfp4")
     nv = dq.format_preset("nvfp4")
-    args = lambda fmt, M, N, K: (None, None, None, None, None, M, N, K, ctypes.byref(fmt), None, None)
-    assert L.dq_w4a4_gemm(*args(nv, 128, 128, 256)) == -3          # MXFP4 only
+    mxi = dq.format_preset("mxint4")
+    nv32 = dq.format_preset("nvfp4", 32)
+    args = lambda fmt, M, N, K: (None, None, None, None, None, None, M, N, K, ctypes.byref(fmt),
+                                 None, None)
+    assert L.dq_w4a4_gemm(*args(mxi, 128, 128, 256)) == -3         # E2M1 codes only
+    assert L.dq_w4a4_gemm(*args(nv32, 128, 128, 256)) == -3        # NVFP4 blocks of 16 only
     assert L.dq_w4a4_gemm(*args(f, 100, 128, 256)) == -2           # M % 128
-    assert L.dq_w4a4_gemm(*args(f, 128, 128, 320)) == -2           # K % 256
+    assert L.dq_w4a4_gemm(*args(nv, 128, 128, 320)) == -2          # K % 256
     assert L.dq_w4a4_gemm(*args(f, 128, 128, 256)) == -1           # null pointers
+    assert L.dq_w4a4_gemm(*args(nv, 128, 128, 256)) == -1
     assert L.dq_w4a4_gemm(*args(f, 0, 128, 256)) == 0              # empty
+    p = ctypes.c_void_p(256)                                       # never dereferenced
+    assert L.dq_w4a4_gemm(p, p, p, p, p, ctypes.c_void_p(258), 128, 128, 256, ctypes.byref(nv),
+                          p, None) == -9                           # tensor_scale alignment
 
 
 def test_scale_tiles_argument_errors():
     L = dq.lib()
-    assert L.dq_scale_tiles(None, 100, 256, None, None) == -2       # rows % 128
-    assert L.dq_scale_tiles(None, 128, 96, None, None) == -2        # K % 128
-    assert L.dq_scale_tiles(None, 128, 256, None, None) == -1       # null pointers
-    assert L.dq_scale_tiles(None, 0, 256, None, None) == 0          # empty
-    assert L.dq_scale_tiles(ctypes.c_void_p(16), 128, 128, ctypes.c_void_p(24), None) == -9  # alignment
+    assert L.dq_scale_tiles(None, 100, 256, 32, None, None) == -2   # rows % 128
+    assert L.dq_scale_tiles(None, 128, 96, 32, None, None) == -2    # K % 128
+    assert L.dq_scale_tiles(None, 128, 96, 16, None, None) == -2    # K % 64
+    assert L.dq_scale_tiles(None, 128, 256, 64, None, None) == -1   # G 16 or 32 only
+    assert L.dq_scale_tiles(None, 128, 256, 32, None, None) == -1   # null pointers
+    assert L.dq_scale_tiles(None, 0, 256, 16, None, None) == 0      # empty
+    assert L.dq_scale_tiles(ctypes.c_void_p(16), 128, 128, 32, ctypes.c_void_p(24),
+                            None) == -9                             # alignment
 
 
 def test_host_solve_argument_errors():
@@ -179,3 +190,32 @@ def test_graph_argument_errors():
     assert L.dq_graph_launch(None, None) == -1                      # no graph
     assert L.dq_graph_launches(None) == 0
     assert L.dq_graph_destroy(None) == 0                            # no-op
+
+
+def test_sharded_column_entry_points_argument_errors():
+    L = dq.lib()
+    f = dq.format_preset("int4_bf16")
+    assert L.dq_col_row_block(-1, 64, 1) == -1
+    assert L.dq_col_row_block(64, 64, 7) == -1
+    assert L.dq_col_row_block(14336, 4096, 1) == 256        # 256 rows per warp, 1 warp row
+    assert L.dq_col_row_block(100, 4096, 1) % 1 == 0 and L.dq_col_row_block(100, 4096, 1) > 0
+    p = ctypes.c_void_p(256)                                 # never dereferenced
+    ws = ctypes.c_void_p(1 << 20)
+    # row block not a multiple of the warp rows / too large / null partials
+    assert L.dq_col_partials(p, 1, 64, 100 * 64, ctypes.byref(f), 1.0, p, p, 0, p, None, ws,
+                             1 << 30, None) == -2
+    assert L.dq_col_partials(p, 1, 64, 64, ctypes.byref(f), 1.0, p, p, 3, p, None, ws,
+                             1 << 30, None) == -2
+    assert L.dq_col_partials(p, 1, 64, 64, ctypes.byref(f), 1.0, p, p, 64, None, None, ws,
+                             1 << 30, None) == -1
+    assert L.dq_col_partials(p, 1, 64, 64, ctypes.byref(f), 2.0, p, p, 64, p, None, ws,
+                             1 << 30, None) == -1              # ts != 1 without a tensor scale
+    assert L.dq_col_row_block(64, 64, 1) == 128              # 16 rows per warp, 8 warp rows
+    assert L.dq_col_partials(p, 1, 64, 64, ctypes.byref(f), 1.0, p, p, 64, p, None, ws,
+                             1 << 30, None) == -2              # below the shard's own row block
+    assert L.dq_col_partials(p, 1, 64, 64, ctypes.byref(f), 1.0, p, p, 128, p, None, None,
+                             0, None) == -7                    # workspace
+    # finalize: odd columns, null output
+    assert L.dq_col_finalize(p, 4, 63, ctypes.byref(f), p, None, None) == -2
+    assert L.dq_col_finalize(p, 4, 64, ctypes.byref(f), None, None, None) == -1
+    assert L.dq_col_finalize(None, 0, 0, ctypes.byref(f), None, None, None) == 0

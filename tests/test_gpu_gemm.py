@@ -1,10 +1,12 @@
 """Block-scaled W4A4 GEMM on the tensor cores against the oracle's float64
 product of the decoded operands (eq. (1) of the daiwk note: X W^T ~= (X D_b)
-Qhat^T D_a).
+Qhat^T D_a), in MXFP4 (E8M0 scales per 32) and NVFP4 (E4M3 scales per 16
+and the weights' tensor scale; news article, "适配 MXFP4 与 NVFP4 块结构").
 
-Bar: the products of E2M1 codes and E8M0 scales are exact in float32, so the
-only error is the float32 accumulation over K terms and the final scaling:
-|gpu - ref| <= (K + 1) 2^-24 sum_k |x_k w_k| |a_n| for every element."""
+Bar: the products of E2M1 codes and E8M0 or E4M3 scales are exact in
+float32 (at most 2 + 4 significant bits per operand), so the only error is
+the float32 accumulation over K terms and the final scaling:
+|gpu - ref| <= (K + 1) 2^-24 sum_k |x_k w_k| |a_n| ts for every element."""
 import numpy as np
 import pytest
 import torch
@@ -191,3 +193,112 @@ def test_w4a4_gemm_stalled_pipeline_reports_timeout(M, N):
     assert dq.last_device_status() == 0
     ref, bound = _reference(cx, sx, cw, sw, a)
     assert np.all(np.abs(np64(out) - ref) <= bound)
+
+
+# --------------------------------------------------------------------------- #
+# NVFP4: E4M3 scales per 16 elements, the weights' tensor scale
+# --------------------------------------------------------------------------- #
+
+FNV = O.preset("nvfp4")
+
+
+def _random_operand_nv(rows, K, key):
+    # E4M3 scales between 2^-3 and 2^3 (bytes 0x20 .. 0x57, sign bit clear)
+    g = torch.Generator().manual_seed(key)
+    codes = torch.randint(0, 256, (rows, K // 2), generator=g, dtype=torch.uint8)
+    scales = torch.randint(0x20, 0x58, (rows, K // 16), generator=g, dtype=torch.uint8)
+    return codes, scales
+
+
+def _reference_nv(cx, sx, cw, sw, a, ts, rows=None):
+    cxn, sxn = cx.cpu().numpy(), sx.cpu().numpy()
+    if rows is not None:
+        cxn, sxn = cxn[rows], sxn[rows]
+    x_c, x_s = O.decode_codes(cxn, FNV), O.decode_scales(sxn, FNV)
+    w_c, w_s = O.decode_codes(cw.cpu().numpy(), FNV), O.decode_scales(sw.cpu().numpy(), FNV)
+    an = np64(a)
+    ref = O.w4a4_gemm(x_c, x_s, w_c, w_s, an, FNV, ts)
+    absx = np.abs(O.dequantize(x_c, x_s, FNV))
+    absw = np.abs(O.dequantize(w_c, w_s, FNV, ts))
+    K = x_c.shape[1]
+    bound = (K + 1) * 2.0 ** -24 * (absx @ absw.T) * np.abs(an)[None, :]
+    return ref, bound
+
+
+@pytest.mark.parametrize("M,N,K", [(128, 128, 256), (256, 384, 1024), (384, 256, 2048),
+                                   (256, 256, 256), (512, 768, 1024), (768, 512, 2048)])
+def test_w4a4_gemm_nvfp4_random_operands(M, N, K):
+    cx, sx = _random_operand_nv(M, K, 61 + M)
+    cw, sw = _random_operand_nv(N, K, 62 + N)
+    a = torch.tensor(np.ldexp(1.0, np.random.default_rng(K).integers(-3, 4, N)), dtype=torch.float32)
+    ts = 2.0 ** -9
+    tsd = torch.tensor([ts], dtype=torch.float32, device="cuda")
+    fl = dq.format_preset("nvfp4")
+    out = dq.w4a4_gemm(cx.cuda(), sx.cuda(), cw.cuda(), sw.cuda(), a.cuda(), fl, tensor_scale=tsd)
+    torch.cuda.synchronize()
+    assert dq.last_device_status() == 0
+    ref, bound = _reference_nv(cx, sx, cw, sw, a, ts)
+    err = np.abs(np64(out) - ref)
+    assert np.all(err <= bound), (err.max(), np.unravel_index(np.argmax(err - bound), err.shape))
+
+
+@pytest.mark.parametrize("M,N", [(128, 128), (256, 256)])         # single CTA, CTA pair
+def test_w4a4_gemm_nvfp4_block_placement(M, N):
+    # Scales apply per 16 elements of K: x[5, 200] = 1 with its block's scale
+    # 2 and w[9, 200] = 6 with its block's scale 1.5 (block 12 of 16), then
+    # x[5, 216] = 1.5 and w[9, 216] = 1 in block 13 with scale 1; a_9 = 2,
+    # ts = 1/4: out[5, 9] = (1*2*6*1.5 + 1.5*1) * 2 / 4 = 9.75.  (Scales read
+    # per 32 elements would give 3.75.)  Row M-1 of x and row N-1 of w repeat
+    # the pattern (with a_{N-1} = 2), so the four crossings are 9.75 and the
+    # rest 0; row M-1 and column N-1 live in the second CTA of a pair.
+    K = 512
+    cx = torch.zeros(M, K // 2, dtype=torch.uint8)
+    sx = torch.full((M, K // 16), 0x38, dtype=torch.uint8)        # E4M3 1.0
+    cw = torch.zeros(N, K // 2, dtype=torch.uint8)
+    sw = torch.full((N, K // 16), 0x38, dtype=torch.uint8)
+    for m, n in [(5, 9), (M - 1, N - 1)]:
+        cx[m, 100] = 0x02                                 # x[m, 200] = 1.0
+        sx[m, 12] = 0x40                                  # 2.0
+        cw[n, 100] = 0x07                                 # w[n, 200] = 6.0
+        sw[n, 12] = 0x3C                                  # 1.5
+        cx[m, 108] = 0x03                                 # x[m, 216] = 1.5
+        cw[n, 108] = 0x02                                 # w[n, 216] = 1.0
+    a = torch.ones(N)
+    a[9] = 2.0
+    a[N - 1] = 2.0
+    tsd = torch.tensor([0.25], device="cuda")
+    out = dq.w4a4_gemm(cx.cuda(), sx.cuda(), cw.cuda(), sw.cuda(), a.cuda(),
+                       dq.format_preset("nvfp4"), tensor_scale=tsd).cpu()
+    want = torch.zeros(M, N)
+    for m in (5, M - 1):
+        for n in (9, N - 1):
+            want[m, n] = 9.75
+    assert torch.equal(out, want)
+
+
+@pytest.mark.parametrize("rows,K", [(128, 64), (384, 1024)])
+def test_scale_tiles_layout_group16(rows, K):
+    _, S = _random_operand_nv(rows, K, 70 + rows)
+    t = dq.scale_tiles(S.cuda(), K, group=16).cpu().numpy()
+    assert np.array_equal(t, _tiles_expected(S.numpy()))
+
+
+def test_w4a4_gemm_nvfp4_after_solve_and_activation_quant():
+    # the NVFP4 pipeline: solve W (E4M3 group scales with the tensor scale),
+    # quantize X D_b to NVFP4 (tensor scale 1), multiply
+    wl = synth.WORKLOADS["llama31_8b_nvfp4_g16"]
+    fl = dq.format_preset("nvfp4")
+    W = synth.weight(wl, 0, 1, device="cuda", rows=512, cols=2048)
+    o = dq.solve_dual_scale(W, fl, 5)
+    X = synth.activation(wl, device="cuda", tokens=256)[:, :2048].contiguous()
+    cx, sx = dq.act_rescale_quant(X, o["b"], fl)
+    out = dq.w4a4_gemm(cx, sx, o["codes"], o["gscales"], o["a"], fl,
+                       tensor_scale=o["tensor_scale"])
+    torch.cuda.synchronize()
+    assert dq.last_device_status() == 0
+    ts = float(o["tensor_scale"].item())
+    assert ts != 1.0
+    ref, bound = _reference_nv(cx, sx, o["codes"], o["gscales"], o["a"], ts)
+    assert np.all(np.abs(np64(out) - ref) <= bound)
+    exact = np64(X) @ np64(W).T
+    assert np.linalg.norm(np64(out) - exact) < 0.35 * np.linalg.norm(exact)

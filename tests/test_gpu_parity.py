@@ -474,6 +474,36 @@ def test_mx_solve_from_a_moving_state(name):
     assert dq.last_device_status() == 0
 
 
+@pytest.mark.parametrize("name", ["mxint4", "mxint8", "mxfp8_e4m3", "mxfp6_e2m3", "mxfp4"])
+def test_literal_steps_small_row_scales_with_zero_groups(name):
+    # The literal row and column steps (also the fallback of the one-pass
+    # iteration) with row scales a = 2^-8 on a matrix whose last column block
+    # is partly past the last column (2240 columns) and with all-zero groups:
+    # an all-zero group (and a lane past the last column) takes scale 1, so
+    # 1 / (a s) stays finite; E8M0 scales exactly as the oracle's.
+    fl, fo = dq.format_preset(name), PRESET_COMBOS[name](32)
+    rows, cols = 64, 2240
+    W = _weights(rows, cols, torch.bfloat16, key=31)
+    W[3, 64:96] = 0.0                                  # one all-zero group
+    W[7] = 0.0                                         # an all-zero row
+    W64 = np64(W)
+    a = np.full(rows, 2.0 ** -8)
+    b = random_outer(fo, cols, synth.stream_key(95, 7), 0.7)
+    ad = torch.tensor(a, dtype=torch.float32, device="cuda")
+    bd = torch.tensor(b, dtype=torch.float32, device="cuda")
+    dq.last_device_status()
+    a1, a1pre, _ = dq.row_update(W.cuda(), fl, ad, bd)
+    b1, b1pre, _ = dq.col_update(W.cuda(), fl, a1, bd)
+    torch.cuda.synchronize()
+    assert dq.last_device_status() == 0
+    Qh, _, _ = O.qhat(W64, a, b, fo)
+    a_or, x_or = O.row_update(W64, Qh, b, fo)
+    check_projected(np64(a1), a_or, x_or, fo, "a")
+    Qh1, _, _ = O.qhat(W64, np64(a1), b, fo)
+    b_or, xb_or = O.col_update(W64, Qh1, np64(a1), fo)
+    check_projected(np64(b1), b_or, xb_or, fo, "b")
+
+
 @pytest.mark.parametrize("name", ["mxfp4", "mxint8"])
 def test_mx_group_exponent_out_of_range_falls_back(name):
     # Rows scaled by 2^-112 and 2^108 give group scales 2^e with |e| > 100 on
