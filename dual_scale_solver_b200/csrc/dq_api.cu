@@ -18,6 +18,7 @@
 
 #include <cstdio>
 #include <cstring>
+#include <algorithm>
 #include <atomic>
 #include <mutex>
 #include <new>
@@ -325,6 +326,7 @@ struct Launcher {
 bool fused_ok(int combo) { return all_e8m0(combo); }
 
 thread_local std::vector<MatDesc> t_table;
+thread_local std::vector<int> t_order;
 
 // Host-side checks of a batched solve's arguments (no CUDA call).
 dq_status check_batch(int32_t n, const dq_matrix *mats, int32_t dtype, const dq_format *fmt,
@@ -369,10 +371,21 @@ dq_status solve_impl(int32_t n, const dq_matrix *mats, int32_t dtype, const dq_f
     Carve cv{static_cast<char *>(workspace), static_cast<char *>(workspace) + ws_bytes};
     MatDesc *dev_table = n > 1 ? cv.take<MatDesc>((size_t)n * sizeof(MatDesc)) : nullptr;
     unsigned int *flags = cv.take<unsigned int>(256);     // fused-path flags: 3 slots x 2 words
+    // The work table lists the matrices by decreasing tile height (stable):
+    // CTAs are dispatched in tile order, so the short tiles of short matrices
+    // fill the last wave instead of leaving SMs idle behind full-size tiles.
+    // Each matrix's tiles and sums depend on its own shape alone, so the
+    // order changes no result.
+    t_order.resize(n);
+    for (int i = 0; i < n; ++i) t_order[i] = i;
+    std::stable_sort(t_order.begin(), t_order.end(), [&](int x, int y) {
+        return geometry(mats[x].rows, mats[x].cols, f32).tr[1] >
+               geometry(mats[y].rows, mats[y].cols, f32).tr[1];
+    });
     t_table.assign(n, MatDesc{});
     int64_t tile_base[3] = {0, 0, 0}, row_base = 0, col_base = 0;
     for (int i = 0; i < n; ++i) {
-        const dq_matrix &m = mats[i];
+        const dq_matrix &m = mats[t_order[i]];
         MatDesc &d = t_table[i];
         d.W = m.W;
         d.rows = m.rows;

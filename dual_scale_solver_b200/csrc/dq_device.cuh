@@ -429,8 +429,8 @@ struct Quant {
     // chunk's stored codes, element 0 lowest, kBits each -- 4-bit codes two
     // per byte, 8-bit codes one per byte, 6-bit codes four per 3 bytes; only
     // when NIB), nonzero (the group max is positive and finite), mbits (the
-    // bits of the group max).
-    template <bool NIB>
+    // bits of the group max).  UNIT_A: the row factor is 1 (a = ia = 1).
+    template <bool NIB, bool UNIT_A = false>
     __device__ __forceinline__ static void run(const f2 (&w)[NP], const f2 (&z)[NP], float a,
                                                float ia, const f2 (&bj)[NP], float ts,
                                                float inv_ts, unsigned int *status, f2 (&c)[NP],
@@ -453,10 +453,12 @@ struct Quant {
             // (e <= 126 holds for finite m)
             s = __uint_as_float(e8m0_scale_bits(mb));
             // an all-zero group (also the zero chunks of lanes past the last
-            // column) takes scale 1: its stored scale, and the scale its codes
-            // are formed with -- with s at the 2^-126 floor, 1 / (a s) would
-            // overflow for a <= 1/4 and turn the zeros into NaN
-            if (!pos) s = 1.0f;
+            // column) takes scale 1: its stored scale, and, with a row factor,
+            // the scale its codes are formed with -- with s at the 2^-126
+            // floor, 1 / (a s) would overflow for a <= 1/4 and turn the zeros
+            // into NaN (without a row factor 1/s = 2^126 stays finite and the
+            // zeros stay zeros)
+            if ((NIB || !(ACT || UNIT_A)) && !pos) s = 1.0f;
         } else {
             // every lane takes part in the warp vote and group shuffles below,
             // whatever its group holds (all-zero and out-of-range groups too)
@@ -869,8 +871,8 @@ tile_kernel(const __grid_constant__ Table tab, int mode_slot, int want_res, int6
             // |e(s)| <= 100 for every non-zero group (checked after the
             // tile's rows on the extremes of the group maxima); the row
             // finalize keeps |e(a)| <= 20 (old) and <= 26 (new)
-            Q::template run<NIB>(w, z, 1.0f, 1.0f, bj, ts, inv_ts, tab.status, c, s, s_eff, cw,
-                                 nonzero, mbits);
+            Q::template run<NIB, true>(w, z, 1.0f, 1.0f, bj, ts, inv_ts, tab.status, c, s, s_eff,
+                                       cw, nonzero, mbits);
             m_lo = min(m_lo, mbits - 1u);
             m_hi = max(m_hi, mbits);
         } else {

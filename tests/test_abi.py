@@ -24,7 +24,7 @@ def built():
 
 def test_exports_match_header():
     names = _declared()
-    assert len(names) == 26
+    assert len(names) == 29
     assert sorted(dq.EXPORTS) == names
     L = dq.lib()
     for n in names:

@@ -2,7 +2,9 @@
 shards of one matrix run in lockstep in this process, their column partial
 slabs concatenated in row order as the all-gather of a multi-GPU run would,
 and the result must be the unsharded solve's bit for bit (a, b, codes,
-group scales), its MSE trace within 1e-12."""
+group scales).  The MSE trace agrees within 1e-6 relative: each tile sums
+its residual in float32 per lane over its rows, so the shards' tile
+geometry changes the last bits of the trace (not the state)."""
 import numpy as np
 import pytest
 import torch
@@ -63,7 +65,7 @@ def test_row_shards_equal_the_unsharded_solve(name, G, nshards):
     assert torch.equal(torch.cat([p[0] for p in packs]), o["codes"])
     assert torch.equal(torch.cat([p[1] for p in packs]), o["gscales"])
     tr = torch.cat(trace).cpu().numpy()
-    assert np.allclose(tr, o["mse_trace"].cpu().numpy(), rtol=1e-12, atol=0)
+    assert np.allclose(tr, o["mse_trace"].cpu().numpy(), rtol=1e-6, atol=0)
 
 
 def test_col_partials_refuse_a_row_block_below_the_shards_own():
