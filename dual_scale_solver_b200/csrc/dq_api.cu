@@ -265,22 +265,27 @@ struct Launcher {
         count_launches(1);
         return DQ_OK;
     }
-    dq_status col_finalize() {
-        if (total_cols == 0) return DQ_OK;
+    // The column update of every matrix; with mse_mode the same launch also
+    // finishes the iteration's MSE (MSE_FUSED: flags / clear of the one-pass
+    // iteration; MSE_LITERAL: the row and column passes' residuals), entry idx.
+    dq_status col_finalize(int mse_mode = MSE_NONE, unsigned int *flags = nullptr,
+                           unsigned int *clear = nullptr, int idx = 0) {
+        if (total_cols == 0 && mse_mode == MSE_NONE) return DQ_OK;
         // one block per 64-column slab (slabs of all matrices, in order)
         int64_t slabs = 0;
         for (int i = 0; i < tab.n; ++i) {
             const MatDesc &d = tab.dev ? host_table[i] : tab.one;
             slabs += (d.cols + kColFinCols - 1) / kColFinCols;
         }
-        const unsigned grid = (unsigned)std::max<int64_t>(1, std::min<int64_t>(slabs, 148 * 16));
+        const int64_t gcols = total_cols == 0 ? 0 : std::max<int64_t>(1, std::min<int64_t>(slabs, 148 * 16));
+        const unsigned grid = (unsigned)(gcols + (mse_mode != MSE_NONE ? 2 * tab.n : 0));
         const int threads = kColFinThreads;
         if (outer_of(combo) == SC_E8M0)
             DQ_CUDA(launch_k(col_finalize_kernel<SC_E8M0>, dim3(grid), dim3(threads), 0, st, tab,
-                             total_cols));
+                             total_cols, mse_mode, flags, clear, idx));
         else
             DQ_CUDA(launch_k(col_finalize_kernel<SC_BF16>, dim3(grid), dim3(threads), 0, st, tab,
-                             total_cols));
+                             total_cols, mse_mode, flags, clear, idx));
         count_launches(1);
         return DQ_OK;
     }
@@ -307,18 +312,13 @@ struct Launcher {
             if ((s = tiles_pass(MODE_ROW, want_trace)) != DQ_OK) return s;
             if ((s = row_finalize()) != DQ_OK) return s;
             if ((s = tiles_pass(MODE_COL, want_half)) != DQ_OK) return s;
-            if ((s = col_finalize()) != DQ_OK) return s;
-            return mse(MODE_ROW, t, t, nullptr, nullptr);
+            return col_finalize(MSE_LITERAL, nullptr, nullptr, t);
         }
         if ((s = tiles_pass(MODE_FUSED, want_trace || want_half, flags, 0)) != DQ_OK) return s;
         if ((s = tiles_pass(MODE_ROW, want_trace, flags, 1)) != DQ_OK) return s;
         if ((s = row_finalize(flags, next)) != DQ_OK) return s;
         if ((s = tiles_pass(MODE_COL, want_half, flags, 2)) != DQ_OK) return s;
-        if ((s = col_finalize()) != DQ_OK) return s;
-        DQ_CUDA(launch_k(mse_finalize_fused_kernel, dim3(2 * tab.n), dim3(256), 0, st, tab, flags,
-                         clear, t));
-        count_launches(1);
-        return DQ_OK;
+        return col_finalize(MSE_FUSED, flags, clear, t);
     }
 };
 

@@ -1111,7 +1111,17 @@ __global__ void row_finalize_kernel(const __grid_constant__ Table tab, int64_t t
         const int64_t r = g - md.row0;
         double num = 0.0, den = 0.0;
         const float2 *p = md.rowpart + r * md.ncb;
-        for (int k = 0; k < md.ncb; ++k) { num += p[k].x; den += p[k].y; }
+        // the row's column blocks in order; loads issued a batch ahead of the
+        // sums (the order of the sums is unchanged)
+        for (int k0 = 0; k0 < md.ncb; k0 += 8) {
+            float2 v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                if (k0 + u < md.ncb) v[u] = __ldg(p + k0 + u);
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                if (k0 + u < md.ncb) { num += v[u].x; den += v[u].y; }
+        }
         if (scale_old) {
             const double ia = (double)recip_pow2(md.a ? md.a[r] : 1.0f);
             num *= ia;
@@ -1135,6 +1145,82 @@ __global__ void row_finalize_kernel(const __grid_constant__ Table tab, int64_t t
     }
 }
 
+// ------------------------------------------------------------------------- //
+// MSE reductions (one block of 256 threads per (matrix, which))
+// ------------------------------------------------------------------------- //
+
+// Sum n residual slots in a fixed order and store sum / (rows * cols).
+__device__ __forceinline__ void mse_reduce_block(const double *src, int64_t n, double *dst,
+                                                 const MatDesc &md) {
+    __shared__ double sm[256];
+    double acc = 0.0;
+    for (int64_t k = threadIdx.x; k < n; k += blockDim.x) acc += src[k];
+    sm[threadIdx.x] = acc;
+    __syncthreads();
+    for (int w = blockDim.x / 2; w > 0; w >>= 1) {
+        if (threadIdx.x < w) sm[threadIdx.x] += sm[threadIdx.x + w];
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) {
+        const double cnt = (double)md.rows * (double)md.cols;
+        *dst = cnt > 0 ? sm[0] / cnt : 0.0;
+    }
+}
+
+// Block blk = 2 mi + which of the MSE of the literal passes: which = 0:
+// res_row[ntiles[row_slot]] -> mse_trace[idx_trace] (or out_row[mi]);
+// which = 1: res_col[ntiles[COL]] -> mse_half[idx_half] (or out_col[mi]).
+__device__ __forceinline__ void mse_literal_block(const Table &tab, int blk, int row_slot,
+                                                  int idx_trace, int idx_half, double *out_row,
+                                                  double *out_col) {
+    const int mi = blk >> 1, which = blk & 1;
+    const MatDesc &md = tab.get(mi);
+    double *dst;
+    const double *src;
+    int64_t n;
+    if (which == 0) {
+        dst = out_row ? out_row + mi : (md.mse_trace && idx_trace >= 0 ? md.mse_trace + idx_trace : nullptr);
+        src = md.res_row;
+        n = (row_slot >= 0) ? md.ntiles[row_slot] : 0;
+    } else {
+        dst = out_col ? out_col + mi : (md.mse_half && idx_half >= 0 ? md.mse_half + idx_half : nullptr);
+        src = md.res_col;
+        n = md.ntiles[MODE_COL];
+    }
+    if (dst == nullptr || (which == 0 && row_slot < 0)) return;   // (uniform per block)
+    mse_reduce_block(src, n, dst, md);
+}
+
+// Block blk of the MSE of an iteration of the fused path: the residual of
+// its state comes from the fused tiles (res_row, column-tile geometry)
+// unless the row step was redone literally (res_row, row-tile geometry);
+// the half-step residual equals it (power-of-two row scales leave D_a Qhat
+// unchanged) unless the column step was redone literally (res_col).  Block
+// 0 also clears the flag slot the next iteration's row finalize may raise
+// after the one after it.
+__device__ __forceinline__ void mse_fused_block(const Table &tab, int blk,
+                                                const unsigned int *flags,
+                                                unsigned int *next_flags, int idx) {
+    if (blk == 0 && threadIdx.x == 0) { next_flags[0] = 0u; next_flags[1] = 0u; }
+    const int mi = blk >> 1, which = blk & 1;
+    const MatDesc &md = tab.get(mi);
+    const bool lit_row = flags[0] != 0, lit_col = (flags[0] | flags[1]) != 0;
+    double *dst;
+    const double *src;
+    int64_t n;
+    if (which == 0) {
+        dst = md.mse_trace ? md.mse_trace + idx : nullptr;
+        src = md.res_row;
+        n = lit_row ? md.ntiles[MODE_ROW] : md.ntiles[MODE_COL];
+    } else {
+        dst = md.mse_half ? md.mse_half + idx : nullptr;
+        src = lit_col ? md.res_col : md.res_row;
+        n = md.ntiles[MODE_COL];
+    }
+    if (dst == nullptr) return;                                   // (uniform per block)
+    mse_reduce_block(src, n, dst, md);
+}
+
 // b_j <- Pi(sum P / sum E) over the column's row blocks.  A block handles 64
 // consecutive columns of one matrix (a lane reads the partials of two
 // adjacent columns as one 16-byte load) with 8 slices of row blocks (slice s
@@ -1142,14 +1228,27 @@ __global__ void row_finalize_kernel(const __grid_constant__ Table tab, int64_t t
 // added in order: a fixed summation order, independent of the launch.
 constexpr int kColFinCols = 64, kColFinSlices = 8;
 constexpr int kColFinThreads = 32 * kColFinSlices;
+// With mse_mode != 0 the last 2n blocks of the grid finish the iteration's
+// MSE instead (1: mse_fused_block with flags / next_flags; 2:
+// mse_literal_block of the row and column passes), saving a launch.
+enum { MSE_NONE = 0, MSE_FUSED = 1, MSE_LITERAL = 2 };
 template <int OS>
 __global__ void __launch_bounds__(kColFinThreads)
-col_finalize_kernel(const __grid_constant__ Table tab, int64_t total_cols) {
+col_finalize_kernel(const __grid_constant__ Table tab, int64_t total_cols, int mse_mode,
+                    const unsigned int *flags, unsigned int *next_flags, int idx) {
     grid_dependency_begin();
+    const int nmse = mse_mode != MSE_NONE ? 2 * tab.n : 0;
+    const int gcols = (int)gridDim.x - nmse;            // blocks of the column update
+    if ((int)blockIdx.x >= gcols) {
+        const int blk = (int)blockIdx.x - gcols;
+        if (mse_mode == MSE_FUSED) mse_fused_block(tab, blk, flags, next_flags, idx);
+        else mse_literal_block(tab, blk, MODE_ROW, idx, idx, nullptr, nullptr);
+        return;
+    }
     __shared__ double sp[kColFinSlices][kColFinCols], se[kColFinSlices][kColFinCols];
     const int lane = threadIdx.x & 31, sl = threadIdx.x >> 5;
     // blocks enumerate 64-column slabs of every matrix in turn
-    for (int64_t slab = blockIdx.x; ; slab += gridDim.x) {
+    for (int64_t slab = blockIdx.x; ; slab += gcols) {
         // matrix of this slab: slabs of matrix i start at ceil-sum of cols / 64
         int mi = -1;
         int64_t c0 = 0;
@@ -1171,13 +1270,24 @@ col_finalize_kernel(const __grid_constant__ Table tab, int64_t total_cols) {
         if (ok) {
             const float4 *src = reinterpret_cast<const float4 *>(md.colpart + c);
             const int64_t stride = md.cols / 2;              // float4 per row block
-#pragma unroll 4
-            for (int64_t k = sl; k < nrb; k += kColFinSlices) {
-                const float4 v = __ldg(src + k * stride);
-                p0 += v.x;
-                e0 += v.y;
-                p1 += v.z;
-                e1 += v.w;
+            // this slice's row blocks in order; the loads of 8 of them are
+            // issued ahead of their sums (the order of the sums is unchanged)
+            for (int64_t k0 = sl; k0 < nrb; k0 += 8 * kColFinSlices) {
+                float4 v[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int64_t k = k0 + (int64_t)u * kColFinSlices;
+                    if (k < nrb) v[u] = __ldg(src + k * stride);
+                }
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    if (k0 + (int64_t)u * kColFinSlices < nrb) {
+                        p0 += v[u].x;
+                        e0 += v[u].y;
+                        p1 += v[u].z;
+                        e1 += v[u].w;
+                    }
+                }
             }
         }
         sp[sl][2 * lane] = p0;
@@ -1208,82 +1318,10 @@ col_finalize_kernel(const __grid_constant__ Table tab, int64_t total_cols) {
 #ifdef DQ_DEFINE_HOST_KERNELS
 // Non-template kernels: defined in exactly one translation unit.
 
-// One block per (matrix, which): sum residual slots in a fixed order and
-// store sum / (rows * cols).  which = 0: res_row[ntiles[slot0]] -> dst0[idx0];
-// which = 1: res_col[ntiles[COL]] -> dst1[idx1].  Destinations are taken from
-// the descriptor's mse_trace / mse_half unless `out` is given.
 __global__ void mse_finalize_kernel(const __grid_constant__ Table tab, int row_slot, int idx_trace, int idx_half,
                                     double *out_row, double *out_col) {
     grid_dependency_begin();
-    const int mi = blockIdx.x >> 1, which = blockIdx.x & 1;
-    const MatDesc &md = tab.get(mi);
-    double *dst;
-    const double *src;
-    int64_t n;
-    if (which == 0) {
-        dst = out_row ? out_row + mi : (md.mse_trace && idx_trace >= 0 ? md.mse_trace + idx_trace : nullptr);
-        src = md.res_row;
-        n = (row_slot >= 0) ? md.ntiles[row_slot] : 0;
-    } else {
-        dst = out_col ? out_col + mi : (md.mse_half && idx_half >= 0 ? md.mse_half + idx_half : nullptr);
-        src = md.res_col;
-        n = md.ntiles[MODE_COL];
-    }
-    if (dst == nullptr || (which == 0 && row_slot < 0)) return;
-    __shared__ double sm[256];
-    double acc = 0.0;
-    for (int64_t k = threadIdx.x; k < n; k += blockDim.x) acc += src[k];
-    sm[threadIdx.x] = acc;
-    __syncthreads();
-    for (int w = blockDim.x / 2; w > 0; w >>= 1) {
-        if (threadIdx.x < w) sm[threadIdx.x] += sm[threadIdx.x + w];
-        __syncthreads();
-    }
-    if (threadIdx.x == 0) {
-        const double cnt = (double)md.rows * (double)md.cols;
-        *dst = cnt > 0 ? sm[0] / cnt : 0.0;
-    }
-}
-
-// MSE of an iteration of the fused path: the residual of its state comes
-// from the fused tiles (res_row, column-tile geometry) unless the row step
-// was redone literally (res_row, row-tile geometry); the half-step residual
-// equals it (power-of-two row scales leave D_a Qhat unchanged) unless the
-// column step was redone literally (res_col).
-__global__ void mse_finalize_fused_kernel(const __grid_constant__ Table tab,
-                                          const unsigned int *flags, unsigned int *next_flags,
-                                          int idx) {
-    grid_dependency_begin();
-    if (blockIdx.x == 0 && threadIdx.x == 0) { next_flags[0] = 0u; next_flags[1] = 0u; }
-    const int mi = blockIdx.x >> 1, which = blockIdx.x & 1;
-    const MatDesc &md = tab.get(mi);
-    const bool lit_row = flags[0] != 0, lit_col = (flags[0] | flags[1]) != 0;
-    double *dst;
-    const double *src;
-    int64_t n;
-    if (which == 0) {
-        dst = md.mse_trace ? md.mse_trace + idx : nullptr;
-        src = md.res_row;
-        n = lit_row ? md.ntiles[MODE_ROW] : md.ntiles[MODE_COL];
-    } else {
-        dst = md.mse_half ? md.mse_half + idx : nullptr;
-        src = lit_col ? md.res_col : md.res_row;
-        n = md.ntiles[MODE_COL];
-    }
-    if (dst == nullptr) return;
-    __shared__ double sm[256];
-    double acc = 0.0;
-    for (int64_t k = threadIdx.x; k < n; k += blockDim.x) acc += src[k];
-    sm[threadIdx.x] = acc;
-    __syncthreads();
-    for (int w = blockDim.x / 2; w > 0; w >>= 1) {
-        if (threadIdx.x < w) sm[threadIdx.x] += sm[threadIdx.x + w];
-        __syncthreads();
-    }
-    if (threadIdx.x == 0) {
-        const double cnt = (double)md.rows * (double)md.cols;
-        *dst = cnt > 0 ? sm[0] / cnt : 0.0;
-    }
+    mse_literal_block(tab, blockIdx.x, row_slot, idx_trace, idx_half, out_row, out_col);
 }
 
 // Initial state: a <- a0 or 1, b <- b0 or 1 (rows then columns, all matrices).
