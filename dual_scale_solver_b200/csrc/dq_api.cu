@@ -152,7 +152,7 @@ struct Carve {
 
 // Fill geometry and workspace pointers of one descriptor.
 void place(MatDesc &d, bool f32, Carve &cv, int64_t tile_base[3], int64_t &row_base,
-           int64_t &col_base) {
+           int64_t &col_base, int64_t &slab_base) {
     const Geom g = geometry(d.rows, d.cols, f32);
     d.wc = g.wc;
     d.ncb = g.ncb;
@@ -164,6 +164,9 @@ void place(MatDesc &d, bool f32, Carve &cv, int64_t tile_base[3], int64_t &row_b
     }
     d.row0 = row_base;
     d.col0 = col_base;
+    // (64-column slabs of the matrices before this one: ceil per matrix)
+    d.slab0 = slab_base;
+    slab_base += (d.cols + kColFinCols - 1) / kColFinCols;
     row_base += d.rows;
     col_base += d.cols;
     if (cv.p) {
@@ -282,10 +285,10 @@ struct Launcher {
         const int threads = kColFinThreads;
         if (outer_of(combo) == SC_E8M0)
             DQ_CUDA(launch_k(col_finalize_kernel<SC_E8M0>, dim3(grid), dim3(threads), 0, st, tab,
-                             total_cols, mse_mode, flags, clear, idx));
+                             total_cols, slabs, mse_mode, flags, clear, idx));
         else
             DQ_CUDA(launch_k(col_finalize_kernel<SC_BF16>, dim3(grid), dim3(threads), 0, st, tab,
-                             total_cols, mse_mode, flags, clear, idx));
+                             total_cols, slabs, mse_mode, flags, clear, idx));
         count_launches(1);
         return DQ_OK;
     }
@@ -383,7 +386,7 @@ dq_status solve_impl(int32_t n, const dq_matrix *mats, int32_t dtype, const dq_f
                geometry(mats[y].rows, mats[y].cols, f32).tr[1];
     });
     t_table.assign(n, MatDesc{});
-    int64_t tile_base[3] = {0, 0, 0}, row_base = 0, col_base = 0;
+    int64_t tile_base[3] = {0, 0, 0}, row_base = 0, col_base = 0, slab_base = 0;
     for (int i = 0; i < n; ++i) {
         const dq_matrix &m = mats[t_order[i]];
         MatDesc &d = t_table[i];
@@ -403,7 +406,7 @@ dq_status solve_impl(int32_t n, const dq_matrix *mats, int32_t dtype, const dq_f
         d.b0 = m.b0;
         d.mse_trace = m.mse_trace;
         d.mse_half = m.mse_half;
-        place(d, f32, cv, tile_base, row_base, col_base);
+        place(d, f32, cv, tile_base, row_base, col_base, slab_base);
     }
     Launcher L;
     L.tab.dev = dev_table;
@@ -508,8 +511,8 @@ dq_status step_impl(bool row_step, const void *W, int32_t dtype, int64_t rows, i
     if (row_step) { d.a_out = out; d.a_pre = pre; }
     else { d.b_out = out; d.b_pre = pre; }
     Carve cv{static_cast<char *>(workspace), static_cast<char *>(workspace) + ws_bytes};
-    int64_t tb[3] = {0, 0, 0}, rb = 0, cb = 0;
-    place(d, f32, cv, tb, rb, cb);
+    int64_t tb[3] = {0, 0, 0}, rb = 0, cb = 0, sb = 0;
+    place(d, f32, cv, tb, rb, cb, sb);
     Launcher L;
     L.tab.dev = nullptr;
     L.tab.one = d;
@@ -569,8 +572,8 @@ dq_status col_partials_impl(const void *W, int32_t dtype, int64_t rows, int64_t 
     d.b = b;
     d.ts_val = ts;
     Carve cv{static_cast<char *>(workspace), static_cast<char *>(workspace) + ws_bytes};
-    int64_t tb[3] = {0, 0, 0}, rb = 0, cb = 0;
-    place(d, f32, cv, tb, rb, cb);
+    int64_t tb[3] = {0, 0, 0}, rb = 0, cb = 0, sb = 0;
+    place(d, f32, cv, tb, rb, cb, sb);
     // the column pass with the whole matrix's row blocks, into the caller's slab
     d.tr[1] = (int32_t)row_block;
     d.ntiles[1] = (rows + row_block - 1) / row_block * d.ncb;
@@ -746,8 +749,8 @@ dq_status dq_quantize(const void *X, int32_t dtype, int64_t rows, int64_t cols,
     d.gscales = gscales;
     d.ts_val = tensor_scale;
     Carve none{nullptr, nullptr};
-    int64_t tb[3] = {0, 0, 0}, rb = 0, cb = 0;
-    place(d, f32, none, tb, rb, cb);
+    int64_t tb[3] = {0, 0, 0}, rb = 0, cb = 0, sb = 0;
+    place(d, f32, none, tb, rb, cb, sb);
     Launcher L;
     L.tab.dev = nullptr;
     L.tab.one = d;
@@ -778,8 +781,8 @@ dq_status dq_act_rescale_quant(const void *X, int64_t tokens, int64_t K, const f
     d.codes = codes;
     d.gscales = gscales;
     Carve none{nullptr, nullptr};
-    int64_t tb[3] = {0, 0, 0}, rb = 0, cb = 0;
-    place(d, false, none, tb, rb, cb);
+    int64_t tb[3] = {0, 0, 0}, rb = 0, cb = 0, sb = 0;
+    place(d, false, none, tb, rb, cb, sb);
     Launcher L;
     L.tab.dev = nullptr;
     L.tab.one = d;
@@ -1351,8 +1354,8 @@ extern "C" dq_status dq_solve_dual_scale_noalloc(const void *W, int32_t dtype, i
     Carve cv{reinterpret_cast<char *>(scratch),
              reinterpret_cast<char *>(scratch) + DQ_NOALLOC_SCRATCH_BYTES};
     unsigned int *flags = cv.take<unsigned int>(256);     // one-pass MX flags: 3 slots x 2 words
-    int64_t tb[3] = {0, 0, 0}, rb = 0, cb = 0;
-    place(d, f32, cv, tb, rb, cb);
+    int64_t tb[3] = {0, 0, 0}, rb = 0, cb = 0, sb = 0;
+    place(d, f32, cv, tb, rb, cb, sb);
     Launcher L;
     L.tab.dev = nullptr;
     L.tab.one = d;

@@ -88,6 +88,7 @@ struct MatDesc {
     int64_t tile0[3];
     int64_t ntiles[3];
     int64_t row0, col0;      // global row / column offsets (finalize kernels)
+    int64_t slab0;           // global offset of its 64-column slabs (column finalize)
     float2 *rowpart;         // [rows][ncb]  (num, den)
     float2 *colpart;         // [nrb_col][cols]  (P, E)
     double *res_row;         // [ntiles ROW]  residual partials (also PACK)
@@ -1234,8 +1235,8 @@ constexpr int kColFinThreads = 32 * kColFinSlices;
 enum { MSE_NONE = 0, MSE_FUSED = 1, MSE_LITERAL = 2 };
 template <int OS>
 __global__ void __launch_bounds__(kColFinThreads)
-col_finalize_kernel(const __grid_constant__ Table tab, int64_t total_cols, int mse_mode,
-                    const unsigned int *flags, unsigned int *next_flags, int idx) {
+col_finalize_kernel(const __grid_constant__ Table tab, int64_t total_cols, int64_t total_slabs,
+                    int mse_mode, const unsigned int *flags, unsigned int *next_flags, int idx) {
     grid_dependency_begin();
     const int nmse = mse_mode != MSE_NONE ? 2 * tab.n : 0;
     const int gcols = (int)gridDim.x - nmse;            // blocks of the column update
@@ -1248,20 +1249,11 @@ col_finalize_kernel(const __grid_constant__ Table tab, int64_t total_cols, int m
     __shared__ double sp[kColFinSlices][kColFinCols], se[kColFinSlices][kColFinCols];
     const int lane = threadIdx.x & 31, sl = threadIdx.x >> 5;
     // blocks enumerate 64-column slabs of every matrix in turn
-    for (int64_t slab = blockIdx.x; ; slab += gcols) {
-        // matrix of this slab: slabs of matrix i start at ceil-sum of cols / 64
-        int mi = -1;
-        int64_t c0 = 0;
-        {
-            int64_t acc = 0;
-            for (int i = 0; i < tab.n; ++i) {
-                const int64_t ns = (tab.get(i).cols + kColFinCols - 1) / kColFinCols;
-                if (slab < acc + ns) { mi = i; c0 = (slab - acc) * kColFinCols; break; }
-                acc += ns;
-            }
-        }
-        if (mi < 0) break;                                 // uniform per block
+    for (int64_t slab = blockIdx.x; slab < total_slabs; slab += gcols) {
+        // matrix of this slab (slabs of matrix i start at its slab0)
+        const int mi = find_owner(tab, slab, [](const MatDesc &d) { return d.slab0; });
         const MatDesc &md = tab.get(mi);
+        const int64_t c0 = (slab - md.slab0) * kColFinCols;
         // columns c and c + 1 (cols is even, so both or neither exist)
         const int64_t c = c0 + 2 * lane;
         const bool ok = c < md.cols;

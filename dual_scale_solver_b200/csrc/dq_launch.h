@@ -28,8 +28,18 @@ inline Geom geometry(int64_t rows, int64_t cols, bool f32) {
     Geom g{};
     const int epc = f32 ? 4 : 8, seg = 32 * epc;
     const int64_t nseg = (cols + seg - 1) / seg;
-    int wc = 1;
-    while (wc < 8 && wc < nseg) wc <<= 1;
+    // warps across columns: of 8, 4, 2 and 1 the one whose column blocks
+    // (wc warp segments each) cover a row with the fewest segments, since a
+    // warp segment past the last column computes on zeros; ties go to the
+    // wider block (8 for 4096 columns; 1 for 576, in three column blocks,
+    // and 2 for 1536, where a power of two at least the segment count would
+    // leave a quarter or more of the lanes idle)
+    int wc = 8;
+    int64_t best = (nseg + 7) / 8 * 8;
+    for (int w = 4; w >= 1; w >>= 1) {
+        const int64_t segs = (nseg + w - 1) / w * w;
+        if (segs < best) { best = segs; wc = w; }
+    }
     g.wc = wc;
     g.ncb = (int)((nseg + wc - 1) / wc);
     const int wr = kWarps / wc;

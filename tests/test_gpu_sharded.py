@@ -41,7 +41,7 @@ def test_row_shards_equal_the_unsharded_solve(name, G, nshards):
     rows, cols, T = 1536, 2240, 3
     W = _weights(rows, cols, key=nshards)
     rb = dq.col_row_block(rows, cols)
-    assert rb == 64
+    assert rows // rb >= 6                              # shards span several row blocks
     # shard starts on multiples of the row block; the last shard is ragged
     starts = [0] + [((k * rows) // nshards) // rb * rb for k in range(1, nshards)] + [rows]
     shards = [sharded.RowShard(W[s0:s1], s0, rows, fl) for s0, s1 in zip(starts, starts[1:])]
