@@ -131,6 +131,8 @@ size_t matrix_ws(int64_t rows, int64_t cols, bool f32) {
     const Geom g = geometry(rows, cols, f32);
     size_t b = 0;
     b += round_up((size_t)rows * g.ncb * sizeof(float2), 256);               // rowpart
+    b += round_up((size_t)rows * g.ncb * sizeof(float), 256);                // rowsq
+    b += 2 * round_up((size_t)rows * sizeof(double), 256);                   // w2row, mse_row
     b += round_up((size_t)g.nrb_col * cols * sizeof(float2), 256);           // colpart
     b += round_up((size_t)std::max(g.ntiles[0], g.ntiles[2]) * 8, 256);      // res_row
     b += round_up((size_t)g.ntiles[1] * 8, 256);                             // res_col
@@ -171,6 +173,9 @@ void place(MatDesc &d, bool f32, Carve &cv, int64_t tile_base[3], int64_t &row_b
     col_base += d.cols;
     if (cv.p) {
         d.rowpart = cv.take<float2>((size_t)d.rows * g.ncb * sizeof(float2));
+        d.rowsq = cv.take<float>((size_t)d.rows * g.ncb * sizeof(float));
+        d.w2row = cv.take<double>((size_t)d.rows * sizeof(double));
+        d.mse_row = cv.take<double>((size_t)d.rows * sizeof(double));
         d.colpart = cv.take<float2>((size_t)g.nrb_col * d.cols * sizeof(float2));
         d.res_row = cv.take<double>((size_t)std::max(g.ntiles[0], g.ntiles[2]) * 8);
         d.res_col = cv.take<double>((size_t)g.ntiles[1] * 8);
@@ -224,6 +229,9 @@ struct Launcher {
     int64_t tiles[3] = {0, 0, 0};
     int64_t total_rows = 0, total_cols = 0;
     cudaStream_t st;
+    // one-pass iterations take each row's squared error from its row sums
+    // (4-bit MX formats; set when an MSE output is wanted)
+    bool row_mse = false;
 
     // One tile pass.  A gated pass (the literal fallback of a fused
     // iteration) launches a small grid that visits the tiles grid-stride and
@@ -232,7 +240,7 @@ struct Launcher {
         TileLaunch L;
         L.tab = tab;
         L.mode = mode;
-        L.slot = (mode == MODE_ACT) ? 2 : (mode == MODE_FUSED ? 1 : mode);
+        L.slot = (mode == MODE_ACT) ? 2 : ((mode == MODE_FUSED || mode == MODE_FUSED_W2) ? 1 : mode);
         L.tiles = tiles[L.slot];
         L.grid = gate ? std::min<int64_t>(L.tiles, 148) : L.tiles;
         L.f32 = f32 ? 1 : 0;
@@ -243,9 +251,11 @@ struct Launcher {
         L.stream = st;
         if (L.grid <= 0) return DQ_OK;
         cudaEvent_t beg = nullptr, end = nullptr;
+        // (the first one-pass iteration's variant is timed as the one-pass kind)
+        const int kind = mode == MODE_FUSED_W2 ? MODE_FUSED : mode;
         {
             std::lock_guard<std::mutex> lk(g_timing_mu);
-            if (!t_capturing && (g_timing_kinds & (1u << mode))) { beg = take_event(); end = take_event(); }
+            if (!t_capturing && (g_timing_kinds & (1u << kind))) { beg = take_event(); end = take_event(); }
         }
         if (beg && end) DQ_CUDA(cudaEventRecord(beg, st));
         DQ_CUDA(launch_tiles(combo, L));
@@ -253,18 +263,19 @@ struct Launcher {
         if (beg && end) {
             DQ_CUDA(cudaEventRecord(end, st));
             std::lock_guard<std::mutex> lk(g_timing_mu);
-            g_timed.push_back({beg, end, mode});
+            g_timed.push_back({beg, end, kind});
         }
         return DQ_OK;
     }
-    dq_status row_finalize(unsigned int *flags = nullptr, unsigned int *next_flags = nullptr) {
+    dq_status row_finalize(unsigned int *flags = nullptr, unsigned int *next_flags = nullptr,
+                           int rmse = 0) {
         if (total_rows == 0) return DQ_OK;
         if (outer_of(combo) == SC_E8M0)
             DQ_CUDA(launch_k(row_finalize_kernel<SC_E8M0>, dim3(grid_for(total_rows, 256)),
-                             dim3(256), 0, st, tab, total_rows, flags, next_flags));
+                             dim3(256), 0, st, tab, total_rows, flags, next_flags, rmse));
         else
             DQ_CUDA(launch_k(row_finalize_kernel<SC_BF16>, dim3(grid_for(total_rows, 256)),
-                             dim3(256), 0, st, tab, total_rows, flags, next_flags));
+                             dim3(256), 0, st, tab, total_rows, flags, next_flags, rmse));
         count_launches(1);
         return DQ_OK;
     }
@@ -317,16 +328,25 @@ struct Launcher {
             if ((s = tiles_pass(MODE_COL, want_half)) != DQ_OK) return s;
             return col_finalize(MSE_LITERAL, nullptr, nullptr, t);
         }
-        if ((s = tiles_pass(MODE_FUSED, want_trace || want_half, flags, 0)) != DQ_OK) return s;
+        // with row_mse the first iteration's pass also sums the rows' squares
+        const int fmode = (row_mse && t == 0) ? MODE_FUSED_W2 : MODE_FUSED;
+        if ((s = tiles_pass(fmode, want_trace || want_half, flags, 0)) != DQ_OK) return s;
         if ((s = tiles_pass(MODE_ROW, want_trace, flags, 1)) != DQ_OK) return s;
-        if ((s = row_finalize(flags, next)) != DQ_OK) return s;
+        if ((s = row_finalize(flags, next, row_mse ? (t == 0 ? 2 : 1) : 0)) != DQ_OK) return s;
         if ((s = tiles_pass(MODE_COL, want_half, flags, 2)) != DQ_OK) return s;
-        return col_finalize(MSE_FUSED, flags, clear, t);
+        return col_finalize(row_mse ? MSE_FUSED_ROWS : MSE_FUSED, flags, clear, t);
     }
 };
 
 // MX formats: power-of-two outer and group scales
 bool fused_ok(int combo) { return all_e8m0(combo); }
+// 4-bit MX formats: their one-pass iterations take the squared error per row
+// from the row sums (about 1% of sum W^2 for 4-bit codes, so the float32
+// row sums leave it correct to about 1e-5 relative; wider codes, whose error
+// is a far smaller share of sum W^2, sum (W - R)^2 directly)
+bool row_mse_ok(int combo) {
+    return combo == COMBO_INT4_E8M0_E8M0 || combo == COMBO_E2M1_E8M0_E8M0;
+}
 
 thread_local std::vector<MatDesc> t_table;
 thread_local std::vector<int> t_order;
@@ -461,6 +481,7 @@ dq_status solve_impl(int32_t n, const dq_matrix *mats, int32_t dtype, const dq_f
         want_trace |= mats[i].mse_trace != nullptr;
         want_half |= mats[i].mse_half != nullptr;
     }
+    L.row_mse = fused && row_mse_ok(fi.combo) && (want_trace || want_half);
     for (int t = 0; t < T; ++t)
         if ((s = L.iteration(t, fused, flags, want_trace, want_half)) != DQ_OK) return s;
     if ((s = L.tiles_pass(MODE_PACK, want_trace)) != DQ_OK) return s;
@@ -1392,6 +1413,7 @@ extern "C" dq_status dq_solve_dual_scale_noalloc(const void *W, int32_t dtype, i
                          rb, cb, fused ? flags : nullptr));
         count_launches(1);
     }
+    L.row_mse = fused && row_mse_ok(fi.combo) && (mse_trace != nullptr || mse_half != nullptr);
     for (int t = 0; t < T; ++t)
         if ((s = L.iteration(t, fused, flags, mse_trace != nullptr, mse_half != nullptr)) != DQ_OK)
             return s;

@@ -27,12 +27,14 @@ namespace dq {
 enum { CODES_INT4 = 0, CODES_E2M1 = 1, CODES_INT8 = 2, CODES_E4M3 = 3, CODES_E5M2 = 4,
        CODES_E2M3 = 5, CODES_E3M2 = 6 };
 enum { SC_BF16 = 0, SC_E8M0 = 1, SC_E4M3 = 2 };
-enum { MODE_ROW = 0, MODE_COL = 1, MODE_PACK = 2, MODE_ACT = 3, MODE_FUSED = 4 };
+// MODE_FUSED_W2: MODE_FUSED that also sums each row's squares (the first
+// one-pass iteration of the 4-bit MX formats; see the tile kernel)
+enum { MODE_ROW = 0, MODE_COL = 1, MODE_PACK = 2, MODE_ACT = 3, MODE_FUSED = 4, MODE_FUSED_W2 = 5 };
 enum { STATUS_NONFINITE = 1u, STATUS_RANGE = 2u, STATUS_TIMEOUT = 4u };
 
 constexpr int kWarps = 8;            // warps per CTA of the tile kernel
 constexpr int kThreads = 32 * kWarps;
-constexpr int kRowsPerWarp[5] = {128, 256, 128, 128, 256};   // per mode (at most)
+constexpr int kRowsPerWarp[6] = {128, 256, 128, 128, 256, 256};   // per mode (at most)
 constexpr int kRing = 4;             // cp.async ring slots per lane (rows in flight + 1)
 constexpr float kBf16Max = 3.38953138925153547590470800371487866880e+38f;  // (2-2^-7)*2^127
 constexpr float kMinNormal = 1.17549435082228750796873653722224568e-38f;    // 2^-126
@@ -90,6 +92,9 @@ struct MatDesc {
     int64_t row0, col0;      // global row / column offsets (finalize kernels)
     int64_t slab0;           // global offset of its 64-column slabs (column finalize)
     float2 *rowpart;         // [rows][ncb]  (num, den)
+    float *rowsq;            // [rows][ncb]  sum of W^2 (MODE_FUSED_W2)
+    double *w2row;           // [rows]  sum of W^2 per row (4-bit MX one-pass path)
+    double *mse_row;         // [rows]  squared error of each row (same)
     float2 *colpart;         // [nrb_col][cols]  (P, E)
     double *res_row;         // [ntiles ROW]  residual partials (also PACK)
     double *res_col;         // [ntiles COL]
@@ -725,23 +730,30 @@ __device__ __forceinline__ float project_outer(float x, bool &clamped) {
 template <int MODE, int EPC>
 struct TileSmem {
     static constexpr int RPW = kRowsPerWarp[MODE];
+    static constexpr bool kFused = MODE == MODE_FUSED || MODE == MODE_FUSED_W2;
+    static constexpr bool kW2 = MODE == MODE_FUSED_W2;
     // ROW, FUSED: per (warp, row of a batch of 8, lane) partial (num, den),
     // reduced every 8 rows.  Row stride padded by one entry.
-    static constexpr int kRed = (MODE == MODE_ROW || MODE == MODE_FUSED) ? kWarps * 8 * 33 : 1;
+    static constexpr int kRed = (MODE == MODE_ROW || kFused) ? kWarps * 8 * 33 : 1;
     // ROW, FUSED: per (row, warp) totals
-    static constexpr int kRtot = (MODE == MODE_ROW || MODE == MODE_FUSED) ? RPW * kWarps : 1;
+    static constexpr int kRtot = (MODE == MODE_ROW || kFused) ? RPW * kWarps : 1;
     // COL, FUSED: per (warp-row, column) partials
-    static constexpr int kPart = (MODE == MODE_COL || MODE == MODE_FUSED) ? kWarps * 32 * EPC : 1;
+    static constexpr int kPart = (MODE == MODE_COL || kFused) ? kWarps * 32 * EPC : 1;
     float2 red[kRed];
     float2 rtot[kRtot];
     float2 part[kPart];
+    // FUSED_W2: the same two stages for the sums of squares
+    float red2[kW2 ? kRed : 1];
+    float rtot2[kW2 ? kRtot : 1];
     double res[kWarps];
     uint4 ring[kWarps][kRing][32];
 };
 
 // Column statistics keep 2 x EPC accumulators per lane: those modes run 2
 // CTAs per SM (up to 128 registers), the others 3.
-template <int MODE> struct TileOcc { static constexpr int kMinBlocks = (MODE == MODE_COL || MODE == MODE_FUSED) ? 2 : 3; };
+template <int MODE> struct TileOcc {
+    static constexpr int kMinBlocks = (MODE == MODE_COL || MODE == MODE_FUSED || MODE == MODE_FUSED_W2) ? 2 : 3;
+};
 
 template <int CODES, int GS, int OS, int MODE, typename TIn, int G>
 __global__ void __launch_bounds__(kThreads, TileOcc<MODE>::kMinBlocks)
@@ -755,7 +767,12 @@ tile_kernel(const __grid_constant__ Table tab, int mode_slot, int want_res, int6
     constexpr int LPG = G / EPC;
     constexpr bool ACT = MODE == MODE_ACT;
     constexpr bool NIB = MODE == MODE_PACK || MODE == MODE_ACT;
-    constexpr bool FUSED = MODE == MODE_FUSED;
+    constexpr bool FUSED = MODE == MODE_FUSED || MODE == MODE_FUSED_W2;
+    constexpr bool W2 = MODE == MODE_FUSED_W2;
+    // 4-bit codes: the one-pass iteration's squared error is taken per row
+    // from its row sums (the row finalize), not summed here
+    constexpr bool kRowMse = FUSED && CodeTraits<CODES>::kBits == 4;
+    static_assert(!W2 || kRowMse, "row sums of squares serve the 4-bit one-pass path");
     constexpr bool ROWSTAT = MODE == MODE_ROW || FUSED;
     constexpr bool COLSTAT = MODE == MODE_COL || FUSED;
     using Q = Quant<CODES, GS, OS, ACT, NP, LPG>;
@@ -771,7 +788,7 @@ tile_kernel(const __grid_constant__ Table tab, int mode_slot, int want_res, int6
     if (gate == 2 && (flags[0] | flags[1]) == 0) return;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const bool res_on = !ACT && want_res != 0;
+    const bool res_on = !ACT && !kRowMse && want_res != 0;
 
     for (int64_t t = blockIdx.x; t < total_tiles; t += gridDim.x) {
     const int mi = find_owner(tab, t, [mode_slot](const MatDesc &d) { return d.tile0[mode_slot]; });
@@ -916,6 +933,15 @@ tile_kernel(const __grid_constant__ Table tab, int mode_slot, int want_res, int6
             // added ((q0 + q1) + (q2 + q3), by two shuffle levels) -- one
             // fixed order, the same in every mode with row statistics
             sm.red[(warp * 8 + (k & 7)) * 33 + lane] = share;
+            if (W2) {
+                // sum of squares of the row, in the order of the sums above
+                // (for a row that Q reproduces exactly, R = W and the three
+                // sums are the same bits)
+                f2 gq = bcast(0.0f);
+#pragma unroll
+                for (int j = 0; j < NP; ++j) gq = fma2(w[j], w[j], gq);
+                sm.red2[(warp * 8 + (k & 7)) * 33 + lane] = gq.x + gq.y;
+            }
             if (batch_end) {
                 __syncwarp();
                 const int rr = lane >> 2, qq = lane & 3;
@@ -929,6 +955,15 @@ tile_kernel(const __grid_constant__ Table tab, int mode_slot, int want_res, int6
                 acc.y += __shfl_xor_sync(0xffffffffu, acc.y, 2);
                 const int kk = (k & ~7) + rr;
                 if (qq == 0 && kk <= k) sm.rtot[kk * kWarps + warp] = acc;
+                if (W2) {
+                    const float *q2 = &sm.red2[(warp * 8 + rr) * 33 + 8 * qq];
+                    const float t01 = q2[0] + q2[1], t23 = q2[2] + q2[3];
+                    const float t45 = q2[4] + q2[5], t67 = q2[6] + q2[7];
+                    float sq = (t01 + t23) + (t45 + t67);
+                    sq += __shfl_xor_sync(0xffffffffu, sq, 1);
+                    sq += __shfl_xor_sync(0xffffffffu, sq, 2);
+                    if (qq == 0 && kk <= k) sm.rtot2[kk * kWarps + warp] = sq;
+                }
                 __syncwarp();
             }
         }
@@ -1036,6 +1071,11 @@ tile_kernel(const __grid_constant__ Table tab, int mode_slot, int want_res, int6
                     den += p.y;
                 }
                 md.rowpart[row * md.ncb + cb] = make_float2(num, den);
+                if (W2) {
+                    float sq = 0.0f;
+                    for (int c2 = 0; c2 < wc; ++c2) sq += sm.rtot2[k * kWarps + r * wc + c2];
+                    md.rowsq[row * md.ncb + cb] = sq;
+                }
             }
         }
     }
@@ -1100,9 +1140,13 @@ tile_kernel(const __grid_constant__ Table tab, int mode_slot, int want_res, int6
 // 1/a_old and 1/a_old^2 here; a new scale with |e(a)| > 26 raises flags[1]
 // (the column step is redone literally) and one with |e(a)| > 20 raises the
 // next iteration's flags[0] (its row step is done literally).
+// row_mse (the one-pass path of the 4-bit MX formats): the squared error of
+// each row of the state, sum_j (W_ij - R_ij)^2 = sum W^2 - 2 sum W R +
+// sum R^2 from the fused row sums (a = 1) -> mse_row; row_mse = 2 first
+// sums the row's squares from the fused pass (rowsq -> w2row), 1 reads them.
 template <int OS>
 __global__ void row_finalize_kernel(const __grid_constant__ Table tab, int64_t total_rows,
-                                    unsigned int *flags, unsigned int *next_flags) {
+                                    unsigned int *flags, unsigned int *next_flags, int row_mse) {
     grid_dependency_begin();
     const bool scale_old = flags != nullptr && flags[0] == 0;
     for (int64_t g = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; g < total_rows;
@@ -1122,6 +1166,19 @@ __global__ void row_finalize_kernel(const __grid_constant__ Table tab, int64_t t
 #pragma unroll
             for (int u = 0; u < 8; ++u)
                 if (k0 + u < md.ncb) { num += v[u].x; den += v[u].y; }
+        }
+        if (row_mse) {
+            double w2 = 0.0;
+            if (row_mse == 2) {
+                // the same order as num: for a row that Q reproduces exactly
+                // the three sums are equal and its error is exactly 0
+                const float *q = md.rowsq + r * md.ncb;
+                for (int k = 0; k < md.ncb; ++k) w2 += __ldg(q + k);
+                md.w2row[r] = w2;
+            } else {
+                w2 = md.w2row[r];
+            }
+            if (scale_old) md.mse_row[r] = (w2 - 2.0 * num) + den;
         }
         if (scale_old) {
             const double ia = (double)recip_pow2(md.a ? md.a[r] : 1.0f);
@@ -1164,7 +1221,10 @@ __device__ __forceinline__ void mse_reduce_block(const double *src, int64_t n, d
     }
     if (threadIdx.x == 0) {
         const double cnt = (double)md.rows * (double)md.cols;
-        *dst = cnt > 0 ? sm[0] / cnt : 0.0;
+        // (a sum of row errors taken from row sums can round below 0 only
+        // when the error is 0 up to rounding; a NaN passes)
+        const double tot = sm[0] < 0.0 ? 0.0 : sm[0];
+        *dst = cnt > 0 ? tot / cnt : 0.0;
     }
 }
 
@@ -1193,15 +1253,17 @@ __device__ __forceinline__ void mse_literal_block(const Table &tab, int blk, int
 }
 
 // Block blk of the MSE of an iteration of the fused path: the residual of
-// its state comes from the fused tiles (res_row, column-tile geometry)
-// unless the row step was redone literally (res_row, row-tile geometry);
-// the half-step residual equals it (power-of-two row scales leave D_a Qhat
-// unchanged) unless the column step was redone literally (res_col).  Block
-// 0 also clears the flag slot the next iteration's row finalize may raise
-// after the one after it.
+// its state comes from the fused tiles (res_row, column-tile geometry; or,
+// with rows_mse, the row finalize's per-row errors mse_row) unless the row
+// step was redone literally (res_row, row-tile geometry); the half-step
+// residual equals it (power-of-two row scales leave D_a Qhat unchanged)
+// unless the column step was redone literally (res_col).  Block 0 also
+// clears the flag slot the next iteration's row finalize may raise after
+// the one after it.
 __device__ __forceinline__ void mse_fused_block(const Table &tab, int blk,
                                                 const unsigned int *flags,
-                                                unsigned int *next_flags, int idx) {
+                                                unsigned int *next_flags, int idx,
+                                                bool rows_mse) {
     if (blk == 0 && threadIdx.x == 0) { next_flags[0] = 0u; next_flags[1] = 0u; }
     const int mi = blk >> 1, which = blk & 1;
     const MatDesc &md = tab.get(mi);
@@ -1209,14 +1271,17 @@ __device__ __forceinline__ void mse_fused_block(const Table &tab, int blk,
     double *dst;
     const double *src;
     int64_t n;
+    // the one-pass residual of the state
+    const double *src1 = rows_mse ? md.mse_row : md.res_row;
+    const int64_t n1 = rows_mse ? md.rows : md.ntiles[MODE_COL];
     if (which == 0) {
         dst = md.mse_trace ? md.mse_trace + idx : nullptr;
-        src = md.res_row;
-        n = lit_row ? md.ntiles[MODE_ROW] : md.ntiles[MODE_COL];
+        src = lit_row ? md.res_row : src1;
+        n = lit_row ? md.ntiles[MODE_ROW] : n1;
     } else {
         dst = md.mse_half ? md.mse_half + idx : nullptr;
-        src = lit_col ? md.res_col : md.res_row;
-        n = md.ntiles[MODE_COL];
+        src = lit_col ? md.res_col : src1;
+        n = lit_col ? md.ntiles[MODE_COL] : n1;
     }
     if (dst == nullptr) return;                                   // (uniform per block)
     mse_reduce_block(src, n, dst, md);
@@ -1230,9 +1295,10 @@ __device__ __forceinline__ void mse_fused_block(const Table &tab, int blk,
 constexpr int kColFinCols = 64, kColFinSlices = 8;
 constexpr int kColFinThreads = 32 * kColFinSlices;
 // With mse_mode != 0 the last 2n blocks of the grid finish the iteration's
-// MSE instead (1: mse_fused_block with flags / next_flags; 2:
-// mse_literal_block of the row and column passes), saving a launch.
-enum { MSE_NONE = 0, MSE_FUSED = 1, MSE_LITERAL = 2 };
+// MSE instead (1: mse_fused_block with flags / next_flags; 3: the same with
+// the per-row errors of the row finalize; 2: mse_literal_block of the row
+// and column passes), saving a launch.
+enum { MSE_NONE = 0, MSE_FUSED = 1, MSE_LITERAL = 2, MSE_FUSED_ROWS = 3 };
 template <int OS>
 __global__ void __launch_bounds__(kColFinThreads)
 col_finalize_kernel(const __grid_constant__ Table tab, int64_t total_cols, int64_t total_slabs,
@@ -1242,7 +1308,8 @@ col_finalize_kernel(const __grid_constant__ Table tab, int64_t total_cols, int64
     const int gcols = (int)gridDim.x - nmse;            // blocks of the column update
     if ((int)blockIdx.x >= gcols) {
         const int blk = (int)blockIdx.x - gcols;
-        if (mse_mode == MSE_FUSED) mse_fused_block(tab, blk, flags, next_flags, idx);
+        if (mse_mode == MSE_FUSED || mse_mode == MSE_FUSED_ROWS)
+            mse_fused_block(tab, blk, flags, next_flags, idx, mse_mode == MSE_FUSED_ROWS);
         else mse_literal_block(tab, blk, MODE_ROW, idx, idx, nullptr, nullptr);
         return;
     }

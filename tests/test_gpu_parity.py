@@ -429,6 +429,36 @@ def _moving_state(name, fo, rows=300, cols=2240):
     return W.to(torch.bfloat16), a0, b0
 
 
+@pytest.mark.parametrize("name", ["mxfp4", "mxint4"])
+def test_exactly_representable_matrix_has_zero_error(name):
+    # Every group is codes times a power of two with the top code in it, so Q
+    # reproduces W and a = b = 1 stay.  The one-pass iterations of the 4-bit
+    # formats take each row's error from its row sums, sum W^2 - 2 sum W R +
+    # sum R^2, with sum W^2 summed in the order of the other two: for such a
+    # row the three are the same bits and the error is exactly 0.
+    fl = dq.format_preset(name)
+    g = torch.Generator().manual_seed(41)
+    rows, cols = 200, 2240                      # ragged: 2240 = 8.75 x 256
+    if name == "mxfp4":
+        grid = torch.tensor([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+        top = 6.0
+    else:
+        grid = torch.arange(0.0, 8.0)
+        top = 7.0
+    vals = grid[torch.randint(0, len(grid), (rows, cols), generator=g)]
+    vals = vals * (torch.randint(0, 2, (rows, cols), generator=g) * 2.0 - 1.0)
+    v3 = vals.view(rows, cols // 32, 32)
+    v3[:, :, 5] = top * (torch.randint(0, 2, (rows, cols // 32), generator=g) * 2.0 - 1.0)
+    e = torch.randint(-12, 6, (rows, cols // 32), generator=g).double()
+    W = (v3.double() * torch.pow(2.0, e)[:, :, None]).reshape(rows, cols)
+    W[17] = 0.0
+    T = 3
+    o = dq.solve_dual_scale(W.to(torch.bfloat16).cuda(), fl, T)
+    torch.cuda.synchronize()
+    assert torch.all(o["mse_trace"] == 0) and torch.all(o["mse_half"] == 0)
+    assert torch.all(o["a"] == 1) and torch.all(o["b"] == 1)
+
+
 @pytest.mark.parametrize("name", ["mxfp4", "mxint4"] + MX_MORE)
 def test_mx_solve_from_a_moving_state(name):
     # The one-pass iteration from a seeded state with a != 1 and b != 1 whose
@@ -446,15 +476,21 @@ def test_mx_solve_from_a_moving_state(name):
     o = dq.solve_dual_scale(Wd, fl, T, a0=a0d, b0=b0d)
     # the literal steps, iteration by iteration, recording which scales move
     a, b = a0d.clone(), b0d.clone()
-    moved_a, moved_b = [], []
+    moved_a, moved_b, lit_mse = [], [], []
     for _ in range(T):
-        a1, _, _ = dq.row_update(Wd, fl, a, b)
+        a1, _, m = dq.row_update(Wd, fl, a, b)
         b1, _, _ = dq.col_update(Wd, fl, a1, b)
         moved_a.append(np.flatnonzero((a1 != a).cpu().numpy()))
         moved_b.append(np.flatnonzero((b1 != b).cpu().numpy()))
+        lit_mse.append(m.item())
         a, b = a1, b1
     torch.cuda.synchronize()
     assert torch.equal(o["a"], a) and torch.equal(o["b"], b)
+    # the one-pass squared error (for 4-bit codes from the row sums, sum W^2
+    # - 2 sum W R + sum R^2) against the literal row pass's sum of (W - R)^2
+    # at the same states
+    lit = np.array(lit_mse)
+    assert np.max(np.abs(np64(o["mse_trace"])[:T] - lit) / lit) < 2e-5
     # the state moves: the zero row and columns in the first iteration, and
     # (but for MXFP8 E5M2) other columns; MXINT4's constructed rows halve a
     assert 4 in moved_a[0] and {7, 1000} <= set(moved_b[0].tolist())

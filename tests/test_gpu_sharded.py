@@ -4,7 +4,10 @@ slabs concatenated in row order as the all-gather of a multi-GPU run would,
 and the result must be the unsharded solve's bit for bit (a, b, codes,
 group scales).  The MSE trace agrees within 1e-6 relative: each tile sums
 its residual in float32 per lane over its rows, so the shards' tile
-geometry changes the last bits of the trace (not the state)."""
+geometry changes the last bits of the trace (not the state).  For MXFP4 the
+unsharded solve's one-pass iterations take each row's error from its row
+sums (sum W^2 - 2 sum W R + sum R^2, float32 sums of terms about 100 times
+the error), so there the trace agrees within 2e-5."""
 import numpy as np
 import pytest
 import torch
@@ -65,7 +68,8 @@ def test_row_shards_equal_the_unsharded_solve(name, G, nshards):
     assert torch.equal(torch.cat([p[0] for p in packs]), o["codes"])
     assert torch.equal(torch.cat([p[1] for p in packs]), o["gscales"])
     tr = torch.cat(trace).cpu().numpy()
-    assert np.allclose(tr, o["mse_trace"].cpu().numpy(), rtol=1e-6, atol=0)
+    rtol = 2e-5 if name == "mxfp4" else 1e-6
+    assert np.allclose(tr, o["mse_trace"].cpu().numpy(), rtol=rtol, atol=0)
 
 
 def test_col_partials_refuse_a_row_block_below_the_shards_own():
