@@ -132,7 +132,8 @@ size_t matrix_ws(int64_t rows, int64_t cols, bool f32) {
     size_t b = 0;
     b += round_up((size_t)rows * g.ncb * sizeof(float2), 256);               // rowpart
     b += round_up((size_t)rows * g.ncb * sizeof(float), 256);                // rowsq
-    b += 2 * round_up((size_t)rows * sizeof(double), 256);                   // w2row, mse_row
+    b += round_up((size_t)rows * sizeof(double), 256);                       // w2row
+    b += round_up((size_t)((rows + kRowFinRows - 1) / kRowFinRows) * 8, 256); // mse_part
     b += round_up((size_t)g.nrb_col * cols * sizeof(float2), 256);           // colpart
     b += round_up((size_t)std::max(g.ntiles[0], g.ntiles[2]) * 8, 256);      // res_row
     b += round_up((size_t)g.ntiles[1] * 8, 256);                             // res_col
@@ -154,7 +155,7 @@ struct Carve {
 
 // Fill geometry and workspace pointers of one descriptor.
 void place(MatDesc &d, bool f32, Carve &cv, int64_t tile_base[3], int64_t &row_base,
-           int64_t &col_base, int64_t &slab_base) {
+           int64_t &col_base, int64_t &slab_base, int64_t &chunk_base) {
     const Geom g = geometry(d.rows, d.cols, f32);
     d.wc = g.wc;
     d.ncb = g.ncb;
@@ -169,13 +170,16 @@ void place(MatDesc &d, bool f32, Carve &cv, int64_t tile_base[3], int64_t &row_b
     // (64-column slabs of the matrices before this one: ceil per matrix)
     d.slab0 = slab_base;
     slab_base += (d.cols + kColFinCols - 1) / kColFinCols;
+    // (256-row chunks of the row finalize, likewise)
+    d.rchunk0 = chunk_base;
+    chunk_base += (d.rows + kRowFinRows - 1) / kRowFinRows;
     row_base += d.rows;
     col_base += d.cols;
     if (cv.p) {
         d.rowpart = cv.take<float2>((size_t)d.rows * g.ncb * sizeof(float2));
         d.rowsq = cv.take<float>((size_t)d.rows * g.ncb * sizeof(float));
         d.w2row = cv.take<double>((size_t)d.rows * sizeof(double));
-        d.mse_row = cv.take<double>((size_t)d.rows * sizeof(double));
+        d.mse_part = cv.take<double>((size_t)((d.rows + kRowFinRows - 1) / kRowFinRows) * sizeof(double));
         d.colpart = cv.take<float2>((size_t)g.nrb_col * d.cols * sizeof(float2));
         d.res_row = cv.take<double>((size_t)std::max(g.ntiles[0], g.ntiles[2]) * 8);
         d.res_col = cv.take<double>((size_t)g.ntiles[1] * 8);
@@ -270,12 +274,19 @@ struct Launcher {
     dq_status row_finalize(unsigned int *flags = nullptr, unsigned int *next_flags = nullptr,
                            int rmse = 0) {
         if (total_rows == 0) return DQ_OK;
+        // one block per 256-row chunk (chunks of all matrices, in order)
+        int64_t chunks = 0;
+        for (int i = 0; i < tab.n; ++i) {
+            const MatDesc &d = tab.dev ? host_table[i] : tab.one;
+            chunks += (d.rows + kRowFinRows - 1) / kRowFinRows;
+        }
+        const dim3 grid((unsigned)std::max<int64_t>(1, std::min<int64_t>(chunks, 148 * 32)));
         if (outer_of(combo) == SC_E8M0)
-            DQ_CUDA(launch_k(row_finalize_kernel<SC_E8M0>, dim3(grid_for(total_rows, 256)),
-                             dim3(256), 0, st, tab, total_rows, flags, next_flags, rmse));
+            DQ_CUDA(launch_k(row_finalize_kernel<SC_E8M0>, grid, dim3(kRowFinRows), 0, st, tab,
+                             chunks, flags, next_flags, rmse));
         else
-            DQ_CUDA(launch_k(row_finalize_kernel<SC_BF16>, dim3(grid_for(total_rows, 256)),
-                             dim3(256), 0, st, tab, total_rows, flags, next_flags, rmse));
+            DQ_CUDA(launch_k(row_finalize_kernel<SC_BF16>, grid, dim3(kRowFinRows), 0, st, tab,
+                             chunks, flags, next_flags, rmse));
         count_launches(1);
         return DQ_OK;
     }
@@ -406,7 +417,7 @@ dq_status solve_impl(int32_t n, const dq_matrix *mats, int32_t dtype, const dq_f
                geometry(mats[y].rows, mats[y].cols, f32).tr[1];
     });
     t_table.assign(n, MatDesc{});
-    int64_t tile_base[3] = {0, 0, 0}, row_base = 0, col_base = 0, slab_base = 0;
+    int64_t tile_base[3] = {0, 0, 0}, row_base = 0, col_base = 0, slab_base = 0, chunk_base = 0;
     for (int i = 0; i < n; ++i) {
         const dq_matrix &m = mats[t_order[i]];
         MatDesc &d = t_table[i];
@@ -426,7 +437,7 @@ dq_status solve_impl(int32_t n, const dq_matrix *mats, int32_t dtype, const dq_f
         d.b0 = m.b0;
         d.mse_trace = m.mse_trace;
         d.mse_half = m.mse_half;
-        place(d, f32, cv, tile_base, row_base, col_base, slab_base);
+        place(d, f32, cv, tile_base, row_base, col_base, slab_base, chunk_base);
     }
     Launcher L;
     L.tab.dev = dev_table;
@@ -532,8 +543,8 @@ dq_status step_impl(bool row_step, const void *W, int32_t dtype, int64_t rows, i
     if (row_step) { d.a_out = out; d.a_pre = pre; }
     else { d.b_out = out; d.b_pre = pre; }
     Carve cv{static_cast<char *>(workspace), static_cast<char *>(workspace) + ws_bytes};
-    int64_t tb[3] = {0, 0, 0}, rb = 0, cb = 0, sb = 0;
-    place(d, f32, cv, tb, rb, cb, sb);
+    int64_t tb[3] = {0, 0, 0}, rb = 0, cb = 0, sb = 0, hb = 0;
+    place(d, f32, cv, tb, rb, cb, sb, hb);
     Launcher L;
     L.tab.dev = nullptr;
     L.tab.one = d;
@@ -593,8 +604,8 @@ dq_status col_partials_impl(const void *W, int32_t dtype, int64_t rows, int64_t 
     d.b = b;
     d.ts_val = ts;
     Carve cv{static_cast<char *>(workspace), static_cast<char *>(workspace) + ws_bytes};
-    int64_t tb[3] = {0, 0, 0}, rb = 0, cb = 0, sb = 0;
-    place(d, f32, cv, tb, rb, cb, sb);
+    int64_t tb[3] = {0, 0, 0}, rb = 0, cb = 0, sb = 0, hb = 0;
+    place(d, f32, cv, tb, rb, cb, sb, hb);
     // the column pass with the whole matrix's row blocks, into the caller's slab
     d.tr[1] = (int32_t)row_block;
     d.ntiles[1] = (rows + row_block - 1) / row_block * d.ncb;
@@ -770,8 +781,8 @@ dq_status dq_quantize(const void *X, int32_t dtype, int64_t rows, int64_t cols,
     d.gscales = gscales;
     d.ts_val = tensor_scale;
     Carve none{nullptr, nullptr};
-    int64_t tb[3] = {0, 0, 0}, rb = 0, cb = 0, sb = 0;
-    place(d, f32, none, tb, rb, cb, sb);
+    int64_t tb[3] = {0, 0, 0}, rb = 0, cb = 0, sb = 0, hb = 0;
+    place(d, f32, none, tb, rb, cb, sb, hb);
     Launcher L;
     L.tab.dev = nullptr;
     L.tab.one = d;
@@ -802,8 +813,8 @@ dq_status dq_act_rescale_quant(const void *X, int64_t tokens, int64_t K, const f
     d.codes = codes;
     d.gscales = gscales;
     Carve none{nullptr, nullptr};
-    int64_t tb[3] = {0, 0, 0}, rb = 0, cb = 0, sb = 0;
-    place(d, false, none, tb, rb, cb, sb);
+    int64_t tb[3] = {0, 0, 0}, rb = 0, cb = 0, sb = 0, hb = 0;
+    place(d, false, none, tb, rb, cb, sb, hb);
     Launcher L;
     L.tab.dev = nullptr;
     L.tab.one = d;
@@ -1375,8 +1386,8 @@ extern "C" dq_status dq_solve_dual_scale_noalloc(const void *W, int32_t dtype, i
     Carve cv{reinterpret_cast<char *>(scratch),
              reinterpret_cast<char *>(scratch) + DQ_NOALLOC_SCRATCH_BYTES};
     unsigned int *flags = cv.take<unsigned int>(256);     // one-pass MX flags: 3 slots x 2 words
-    int64_t tb[3] = {0, 0, 0}, rb = 0, cb = 0, sb = 0;
-    place(d, f32, cv, tb, rb, cb, sb);
+    int64_t tb[3] = {0, 0, 0}, rb = 0, cb = 0, sb = 0, hb = 0;
+    place(d, f32, cv, tb, rb, cb, sb, hb);
     Launcher L;
     L.tab.dev = nullptr;
     L.tab.one = d;

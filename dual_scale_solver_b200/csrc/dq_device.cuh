@@ -35,6 +35,7 @@ enum { STATUS_NONFINITE = 1u, STATUS_RANGE = 2u, STATUS_TIMEOUT = 4u };
 constexpr int kWarps = 8;            // warps per CTA of the tile kernel
 constexpr int kThreads = 32 * kWarps;
 constexpr int kRowsPerWarp[6] = {128, 256, 128, 128, 256, 256};   // per mode (at most)
+constexpr int kRowFinRows = 256;     // rows per block of the row finalize
 constexpr int kRing = 4;             // cp.async ring slots per lane (rows in flight + 1)
 constexpr float kBf16Max = 3.38953138925153547590470800371487866880e+38f;  // (2-2^-7)*2^127
 constexpr float kMinNormal = 1.17549435082228750796873653722224568e-38f;    // 2^-126
@@ -91,10 +92,11 @@ struct MatDesc {
     int64_t ntiles[3];
     int64_t row0, col0;      // global row / column offsets (finalize kernels)
     int64_t slab0;           // global offset of its 64-column slabs (column finalize)
+    int64_t rchunk0;         // global offset of its 256-row chunks (row finalize)
     float2 *rowpart;         // [rows][ncb]  (num, den)
     float *rowsq;            // [rows][ncb]  sum of W^2 (MODE_FUSED_W2)
     double *w2row;           // [rows]  sum of W^2 per row (4-bit MX one-pass path)
-    double *mse_row;         // [rows]  squared error of each row (same)
+    double *mse_part;        // [ceil(rows / 256)]  squared error of each 256-row chunk (same)
     float2 *colpart;         // [nrb_col][cols]  (P, E)
     double *res_row;         // [ntiles ROW]  residual partials (also PACK)
     double *res_col;         // [ntiles COL]
@@ -1142,64 +1144,84 @@ tile_kernel(const __grid_constant__ Table tab, int mode_slot, int want_res, int6
 // next iteration's flags[0] (its row step is done literally).
 // row_mse (the one-pass path of the 4-bit MX formats): the squared error of
 // each row of the state, sum_j (W_ij - R_ij)^2 = sum W^2 - 2 sum W R +
-// sum R^2 from the fused row sums (a = 1) -> mse_row; row_mse = 2 first
-// sums the row's squares from the fused pass (rowsq -> w2row), 1 reads them.
+// sum R^2 from the fused row sums (a = 1), summed over the block's rows in
+// a fixed order -> mse_part[chunk]; row_mse = 2 first sums the row's
+// squares from the fused pass (rowsq -> w2row), 1 reads them.
+// A block handles one 256-row chunk of one matrix at a time (chunks of all
+// matrices in order, grid-stride).
 template <int OS>
-__global__ void row_finalize_kernel(const __grid_constant__ Table tab, int64_t total_rows,
-                                    unsigned int *flags, unsigned int *next_flags, int row_mse) {
+__global__ void __launch_bounds__(kRowFinRows)
+row_finalize_kernel(const __grid_constant__ Table tab, int64_t total_chunks, unsigned int *flags,
+                    unsigned int *next_flags, int row_mse) {
     grid_dependency_begin();
+    __shared__ double wsum[kRowFinRows / 32];
     const bool scale_old = flags != nullptr && flags[0] == 0;
-    for (int64_t g = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; g < total_rows;
-         g += (int64_t)gridDim.x * blockDim.x) {
-        const int mi = find_owner(tab, g, [](const MatDesc &d) { return d.row0; });
+    for (int64_t ch = blockIdx.x; ch < total_chunks; ch += gridDim.x) {
+        const int mi = find_owner(tab, ch, [](const MatDesc &d) { return d.rchunk0; });
         const MatDesc &md = tab.get(mi);
-        const int64_t r = g - md.row0;
-        double num = 0.0, den = 0.0;
-        const float2 *p = md.rowpart + r * md.ncb;
-        // the row's column blocks in order; loads issued a batch ahead of the
-        // sums (the order of the sums is unchanged)
-        for (int k0 = 0; k0 < md.ncb; k0 += 8) {
-            float2 v[8];
+        const int64_t r = (ch - md.rchunk0) * kRowFinRows + threadIdx.x;
+        double err = 0.0;
+        if (r < md.rows) {
+            double num = 0.0, den = 0.0;
+            const float2 *p = md.rowpart + r * md.ncb;
+            // the row's column blocks in order; loads issued a batch ahead of
+            // the sums (the order of the sums is unchanged)
+            for (int k0 = 0; k0 < md.ncb; k0 += 8) {
+                float2 v[8];
 #pragma unroll
-            for (int u = 0; u < 8; ++u)
-                if (k0 + u < md.ncb) v[u] = __ldg(p + k0 + u);
+                for (int u = 0; u < 8; ++u)
+                    if (k0 + u < md.ncb) v[u] = __ldg(p + k0 + u);
 #pragma unroll
-            for (int u = 0; u < 8; ++u)
-                if (k0 + u < md.ncb) { num += v[u].x; den += v[u].y; }
-        }
-        if (row_mse) {
-            double w2 = 0.0;
-            if (row_mse == 2) {
-                // the same order as num: for a row that Q reproduces exactly
-                // the three sums are equal and its error is exactly 0
-                const float *q = md.rowsq + r * md.ncb;
-                for (int k = 0; k < md.ncb; ++k) w2 += __ldg(q + k);
-                md.w2row[r] = w2;
-            } else {
-                w2 = md.w2row[r];
+                for (int u = 0; u < 8; ++u)
+                    if (k0 + u < md.ncb) { num += v[u].x; den += v[u].y; }
             }
-            if (scale_old) md.mse_row[r] = (w2 - 2.0 * num) + den;
+            if (row_mse) {
+                double w2 = 0.0;
+                if (row_mse == 2) {
+                    // the same order as num: for a row that Q reproduces
+                    // exactly the three sums are equal and its error is 0
+                    const float *q = md.rowsq + r * md.ncb;
+                    for (int k = 0; k < md.ncb; ++k) w2 += __ldg(q + k);
+                    md.w2row[r] = w2;
+                } else {
+                    w2 = md.w2row[r];
+                }
+                if (scale_old) err = (w2 - 2.0 * num) + den;
+            }
+            if (scale_old) {
+                const double ia = (double)recip_pow2(md.a ? md.a[r] : 1.0f);
+                num *= ia;
+                den *= ia * ia;
+            }
+            float a = 1.0f, pre = __int_as_float(0x7fc00000);
+            if (den > 0.0) {
+                pre = (float)(num / den);
+                bool cl;
+                a = project_outer<OS>(pre, cl);
+                if (cl) atomicOr(tab.status, STATUS_RANGE);
+            }
+            if (!isfinite(num) || !isfinite(den)) atomicOr(tab.status, STATUS_NONFINITE);
+            if (flags != nullptr) {
+                const int ea = (int)((__float_as_uint(a) >> 23) & 0xFF) - 127;
+                if (ea > 26 || ea < -26) atomicOr(&flags[1], 1u);
+                if (ea > 20 || ea < -20) atomicOr(&next_flags[0], 1u);
+            }
+            md.a_out[r] = a;
+            if (md.a_pre) md.a_pre[r] = pre;
         }
-        if (scale_old) {
-            const double ia = (double)recip_pow2(md.a ? md.a[r] : 1.0f);
-            num *= ia;
-            den *= ia * ia;
+        if (row_mse && scale_old) {                       // (uniform per block)
+            // the chunk's errors in a fixed order: lanes, then warps
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) err += __shfl_xor_sync(0xffffffffu, err, o);
+            if ((threadIdx.x & 31) == 0) wsum[threadIdx.x >> 5] = err;
+            __syncthreads();
+            if (threadIdx.x == 0) {
+                double t = 0.0;
+                for (int w = 0; w < kRowFinRows / 32; ++w) t += wsum[w];
+                md.mse_part[ch - md.rchunk0] = t;
+            }
+            __syncthreads();
         }
-        float a = 1.0f, pre = __int_as_float(0x7fc00000);
-        if (den > 0.0) {
-            pre = (float)(num / den);
-            bool cl;
-            a = project_outer<OS>(pre, cl);
-            if (cl) atomicOr(tab.status, STATUS_RANGE);
-        }
-        if (!isfinite(num) || !isfinite(den)) atomicOr(tab.status, STATUS_NONFINITE);
-        if (flags != nullptr) {
-            const int ea = (int)((__float_as_uint(a) >> 23) & 0xFF) - 127;
-            if (ea > 26 || ea < -26) atomicOr(&flags[1], 1u);
-            if (ea > 20 || ea < -20) atomicOr(&next_flags[0], 1u);
-        }
-        md.a_out[r] = a;
-        if (md.a_pre) md.a_pre[r] = pre;
     }
 }
 
@@ -1254,7 +1276,7 @@ __device__ __forceinline__ void mse_literal_block(const Table &tab, int blk, int
 
 // Block blk of the MSE of an iteration of the fused path: the residual of
 // its state comes from the fused tiles (res_row, column-tile geometry; or,
-// with rows_mse, the row finalize's per-row errors mse_row) unless the row
+// with rows_mse, the row finalize's per-chunk errors mse_part) unless the row
 // step was redone literally (res_row, row-tile geometry); the half-step
 // residual equals it (power-of-two row scales leave D_a Qhat unchanged)
 // unless the column step was redone literally (res_col).  Block 0 also
@@ -1272,8 +1294,8 @@ __device__ __forceinline__ void mse_fused_block(const Table &tab, int blk,
     const double *src;
     int64_t n;
     // the one-pass residual of the state
-    const double *src1 = rows_mse ? md.mse_row : md.res_row;
-    const int64_t n1 = rows_mse ? md.rows : md.ntiles[MODE_COL];
+    const double *src1 = rows_mse ? md.mse_part : md.res_row;
+    const int64_t n1 = rows_mse ? (md.rows + kRowFinRows - 1) / kRowFinRows : md.ntiles[MODE_COL];
     if (which == 0) {
         dst = md.mse_trace ? md.mse_trace + idx : nullptr;
         src = lit_row ? md.res_row : src1;
