@@ -167,9 +167,9 @@ void place(MatDesc &d, bool f32, Carve &cv, int64_t tile_base[3], int64_t &row_b
     }
     d.row0 = row_base;
     d.col0 = col_base;
-    // (64-column slabs of the matrices before this one: ceil per matrix)
-    d.slab0 = slab_base;
-    slab_base += (d.cols + kColFinCols - 1) / kColFinCols;
+    // (work units of the column finalize before this matrix)
+    d.cunit0 = slab_base;
+    slab_base += col_units(g.nrb_col, d.cols);
     // (256-row chunks of the row finalize, likewise)
     d.rchunk0 = chunk_base;
     chunk_base += (d.rows + kRowFinRows - 1) / kRowFinRows;
@@ -296,26 +296,27 @@ struct Launcher {
     dq_status col_finalize(int mse_mode = MSE_NONE, unsigned int *flags = nullptr,
                            unsigned int *clear = nullptr, int idx = 0) {
         if (total_cols == 0 && mse_mode == MSE_NONE) return DQ_OK;
-        // one block per 64-column slab (slabs of all matrices, in order)
-        int64_t slabs = 0;
+        // one block per work unit (units of all matrices, in order)
+        int64_t units = 0;
         for (int i = 0; i < tab.n; ++i) {
             const MatDesc &d = tab.dev ? host_table[i] : tab.one;
-            slabs += (d.cols + kColFinCols - 1) / kColFinCols;
+            units += col_units(d.ntiles[MODE_COL] / std::max(d.ncb, 1), d.cols);
         }
-        const int64_t gcols = total_cols == 0 ? 0 : std::max<int64_t>(1, std::min<int64_t>(slabs, 148 * 16));
-        const unsigned grid = (unsigned)(gcols + (mse_mode != MSE_NONE ? 2 * tab.n : 0));
+        const int64_t gcols = total_cols == 0 ? 0 : std::max<int64_t>(1, std::min<int64_t>(units, 148 * 16));
+        const unsigned grid = (unsigned)(gcols + (mse_mode != MSE_NONE ? (2 * tab.n + 7) / 8 : 0));
         const int threads = kColFinThreads;
         if (outer_of(combo) == SC_E8M0)
             DQ_CUDA(launch_k(col_finalize_kernel<SC_E8M0>, dim3(grid), dim3(threads), 0, st, tab,
-                             total_cols, slabs, mse_mode, flags, clear, idx));
+                             units, mse_mode, flags, clear, idx));
         else
             DQ_CUDA(launch_k(col_finalize_kernel<SC_BF16>, dim3(grid), dim3(threads), 0, st, tab,
-                             total_cols, slabs, mse_mode, flags, clear, idx));
+                             units, mse_mode, flags, clear, idx));
         count_launches(1);
         return DQ_OK;
     }
     dq_status mse(int row_slot, int idx_trace, int idx_half, double *out_row, double *out_col) {
-        DQ_CUDA(launch_k(mse_finalize_kernel, dim3(2 * tab.n), dim3(256), 0, st, tab, row_slot,
+        // a warp per (matrix, which), 8 per block
+        DQ_CUDA(launch_k(mse_finalize_kernel, dim3((2 * tab.n + 7) / 8), dim3(256), 0, st, tab, row_slot,
                          idx_trace, idx_half, out_row, out_col));
         count_launches(1);
         return DQ_OK;

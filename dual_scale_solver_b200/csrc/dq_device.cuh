@@ -91,7 +91,7 @@ struct MatDesc {
     int64_t tile0[3];
     int64_t ntiles[3];
     int64_t row0, col0;      // global row / column offsets (finalize kernels)
-    int64_t slab0;           // global offset of its 64-column slabs (column finalize)
+    int64_t cunit0;          // global offset of its work units (column finalize)
     int64_t rchunk0;         // global offset of its 256-row chunks (row finalize)
     float2 *rowpart;         // [rows][ncb]  (num, den)
     float *rowsq;            // [rows][ncb]  sum of W^2 (MODE_FUSED_W2)
@@ -1226,36 +1226,35 @@ row_finalize_kernel(const __grid_constant__ Table tab, int64_t total_chunks, uns
 }
 
 // ------------------------------------------------------------------------- //
-// MSE reductions (one block of 256 threads per (matrix, which))
+// MSE reductions (one warp per (matrix, which); 8 per block of 256 threads)
 // ------------------------------------------------------------------------- //
 
-// Sum n residual slots in a fixed order and store sum / (rows * cols).
-__device__ __forceinline__ void mse_reduce_block(const double *src, int64_t n, double *dst,
-                                                 const MatDesc &md) {
-    __shared__ double sm[256];
+// Sum n residual slots in a fixed order (lane l: slots l, l + 32, ... in
+// order; then the lanes by a fixed butterfly) and store sum / (rows * cols).
+// Called by a whole warp.
+__device__ __forceinline__ void mse_reduce_warp(const double *src, int64_t n, double *dst,
+                                                const MatDesc &md) {
+    const int lane = threadIdx.x & 31;
     double acc = 0.0;
-    for (int64_t k = threadIdx.x; k < n; k += blockDim.x) acc += src[k];
-    sm[threadIdx.x] = acc;
-    __syncthreads();
-    for (int w = blockDim.x / 2; w > 0; w >>= 1) {
-        if (threadIdx.x < w) sm[threadIdx.x] += sm[threadIdx.x + w];
-        __syncthreads();
-    }
-    if (threadIdx.x == 0) {
+    for (int64_t k = lane; k < n; k += 32) acc += src[k];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) {
         const double cnt = (double)md.rows * (double)md.cols;
         // (a sum of row errors taken from row sums can round below 0 only
         // when the error is 0 up to rounding; a NaN passes)
-        const double tot = sm[0] < 0.0 ? 0.0 : sm[0];
+        const double tot = acc < 0.0 ? 0.0 : acc;
         *dst = cnt > 0 ? tot / cnt : 0.0;
     }
 }
 
-// Block blk = 2 mi + which of the MSE of the literal passes: which = 0:
+// Item blk = 2 mi + which of the MSE of the literal passes: which = 0:
 // res_row[ntiles[row_slot]] -> mse_trace[idx_trace] (or out_row[mi]);
 // which = 1: res_col[ntiles[COL]] -> mse_half[idx_half] (or out_col[mi]).
-__device__ __forceinline__ void mse_literal_block(const Table &tab, int blk, int row_slot,
-                                                  int idx_trace, int idx_half, double *out_row,
-                                                  double *out_col) {
+// Called by a whole warp.
+__device__ __forceinline__ void mse_literal_item(const Table &tab, int blk, int row_slot,
+                                                 int idx_trace, int idx_half, double *out_row,
+                                                 double *out_col) {
     const int mi = blk >> 1, which = blk & 1;
     const MatDesc &md = tab.get(mi);
     double *dst;
@@ -1270,23 +1269,23 @@ __device__ __forceinline__ void mse_literal_block(const Table &tab, int blk, int
         src = md.res_col;
         n = md.ntiles[MODE_COL];
     }
-    if (dst == nullptr || (which == 0 && row_slot < 0)) return;   // (uniform per block)
-    mse_reduce_block(src, n, dst, md);
+    if (dst == nullptr || (which == 0 && row_slot < 0)) return;   // (uniform per warp)
+    mse_reduce_warp(src, n, dst, md);
 }
 
-// Block blk of the MSE of an iteration of the fused path: the residual of
+// Item blk of the MSE of an iteration of the fused path: the residual of
 // its state comes from the fused tiles (res_row, column-tile geometry; or,
 // with rows_mse, the row finalize's per-chunk errors mse_part) unless the row
 // step was redone literally (res_row, row-tile geometry); the half-step
 // residual equals it (power-of-two row scales leave D_a Qhat unchanged)
-// unless the column step was redone literally (res_col).  Block 0 also
+// unless the column step was redone literally (res_col).  Item 0 also
 // clears the flag slot the next iteration's row finalize may raise after
-// the one after it.
-__device__ __forceinline__ void mse_fused_block(const Table &tab, int blk,
-                                                const unsigned int *flags,
-                                                unsigned int *next_flags, int idx,
-                                                bool rows_mse) {
-    if (blk == 0 && threadIdx.x == 0) { next_flags[0] = 0u; next_flags[1] = 0u; }
+// the one after it.  Called by a whole warp.
+__device__ __forceinline__ void mse_fused_item(const Table &tab, int blk,
+                                               const unsigned int *flags,
+                                               unsigned int *next_flags, int idx,
+                                               bool rows_mse) {
+    if (blk == 0 && (threadIdx.x & 31) == 0) { next_flags[0] = 0u; next_flags[1] = 0u; }
     const int mi = blk >> 1, which = blk & 1;
     const MatDesc &md = tab.get(mi);
     const bool lit_row = flags[0] != 0, lit_col = (flags[0] | flags[1]) != 0;
@@ -1305,63 +1304,112 @@ __device__ __forceinline__ void mse_fused_block(const Table &tab, int blk,
         src = lit_col ? md.res_col : src1;
         n = lit_col ? md.ntiles[MODE_COL] : n1;
     }
-    if (dst == nullptr) return;                                   // (uniform per block)
-    mse_reduce_block(src, n, dst, md);
+    if (dst == nullptr) return;                                   // (uniform per warp)
+    mse_reduce_warp(src, n, dst, md);
 }
 
-// b_j <- Pi(sum P / sum E) over the column's row blocks.  A block handles 64
-// consecutive columns of one matrix (a lane reads the partials of two
-// adjacent columns as one 16-byte load) with 8 slices of row blocks (slice s
-// sums row blocks s, s+8, ... in order, in double); the slices are then
-// added in order: a fixed summation order, independent of the launch.
+// b_j <- Pi(sum P / sum E) over the column's row blocks, summed in double
+// in a fixed order that depends only on the matrix's shape: the column's row
+// blocks are split into 8 slices (slice s: row blocks s, s+8, ... added in
+// order), and the slices are added in order.  A matrix whose column pass has
+// more than 16 row blocks takes a block per 64 consecutive columns (a
+// "slab"; a lane reads the partials of two adjacent columns as one 16-byte
+// load), a warp per slice; a shorter one a warp per 32 columns, a lane per
+// column holding all of its row blocks in registers and forming the same
+// sums in the same order (a block: 256 columns).  Work units (a block's
+// columns) of all matrices in order.
 constexpr int kColFinCols = 64, kColFinSlices = 8;
 constexpr int kColFinThreads = 32 * kColFinSlices;
-// With mse_mode != 0 the last 2n blocks of the grid finish the iteration's
-// MSE instead (1: mse_fused_block with flags / next_flags; 3: the same with
-// the per-row errors of the row finalize; 2: mse_literal_block of the row
-// and column passes), saving a launch.
+constexpr int kColFinWarpRb = kColFinSlices;       // most row blocks of the lane-per-column form
+__host__ __device__ __forceinline__ int64_t col_units(int64_t rows_blocks, int64_t cols) {
+    return rows_blocks > kColFinWarpRb ? (cols + kColFinCols - 1) / kColFinCols
+                                       : (cols + 32 * kColFinSlices - 1) / (32 * kColFinSlices);
+}
+// Column cc's projection from its total sums.
+template <int OS>
+__device__ __forceinline__ void col_finish(const Table &tab, const MatDesc &md, int64_t cc,
+                                           double pt, double et) {
+    float b = 1.0f, pre = __int_as_float(0x7fc00000);
+    if (et > 0.0) {
+        pre = (float)(pt / et);
+        bool cl;
+        b = project_outer<OS>(pre, cl);
+        if (cl) atomicOr(tab.status, STATUS_RANGE);
+    }
+    if (!isfinite(pt) || !isfinite(et)) atomicOr(tab.status, STATUS_NONFINITE);
+    md.b_out[cc] = b;
+    if (md.b_pre) md.b_pre[cc] = pre;
+}
+// The lane-per-column form (a matrix with at most 8 row blocks in its
+// column pass, so that every slice holds at most one): lane l of warp w
+// takes column 256 (unit - cunit0) + 32 w + l and adds its row blocks in
+// order -- the sums of the block form, since its running sums are never -0.
+template <int OS>
+__device__ __forceinline__ void col_lane_unit(const Table &tab, const MatDesc &md, int64_t unit,
+                                              int64_t nrb) {
+    const int64_t c = (unit - md.cunit0) * (32 * kColFinSlices) + (threadIdx.x & ~31) +
+                      (threadIdx.x & 31);
+    if (c >= md.cols) return;
+    const float2 *src = md.colpart + c;
+    float2 v[kColFinSlices];
+#pragma unroll
+    for (int k = 0; k < kColFinSlices; ++k)
+        if (k < nrb) v[k] = __ldg(src + k * md.cols);
+    double pt = 0.0, et = 0.0;
+#pragma unroll
+    for (int k = 0; k < kColFinSlices; ++k)
+        if (k < nrb) { pt += v[k].x; et += v[k].y; }
+    col_finish<OS>(tab, md, c, pt, et);
+}
+
+// With mse_mode != 0 the last ceil(2n / 8) blocks of the grid finish the
+// iteration's MSE instead, a warp per item (1: mse_fused_item with flags /
+// next_flags; 3: the same with the per-row errors of the row finalize; 2:
+// mse_literal_item of the row and column passes), saving a launch.
 enum { MSE_NONE = 0, MSE_FUSED = 1, MSE_LITERAL = 2, MSE_FUSED_ROWS = 3 };
 template <int OS>
-__global__ void __launch_bounds__(kColFinThreads)
-col_finalize_kernel(const __grid_constant__ Table tab, int64_t total_cols, int64_t total_slabs,
-                    int mse_mode, const unsigned int *flags, unsigned int *next_flags, int idx) {
+__global__ void __launch_bounds__(kColFinThreads, 3)
+col_finalize_kernel(const __grid_constant__ Table tab, int64_t total_units, int mse_mode,
+                    const unsigned int *flags, unsigned int *next_flags, int idx) {
     grid_dependency_begin();
-    const int nmse = mse_mode != MSE_NONE ? 2 * tab.n : 0;
-    const int gcols = (int)gridDim.x - nmse;            // blocks of the column update
-    if ((int)blockIdx.x >= gcols) {
-        const int blk = (int)blockIdx.x - gcols;
+    const int nmse = mse_mode != MSE_NONE ? (2 * tab.n + kColFinSlices - 1) / kColFinSlices : 0;
+    const int gunits = (int)gridDim.x - nmse;           // blocks of the column update
+    if ((int)blockIdx.x >= gunits) {
+        const int blk = ((int)blockIdx.x - gunits) * kColFinSlices + (int)(threadIdx.x >> 5);
+        if (blk >= 2 * tab.n) return;                   // (uniform per warp)
         if (mse_mode == MSE_FUSED || mse_mode == MSE_FUSED_ROWS)
-            mse_fused_block(tab, blk, flags, next_flags, idx, mse_mode == MSE_FUSED_ROWS);
-        else mse_literal_block(tab, blk, MODE_ROW, idx, idx, nullptr, nullptr);
+            mse_fused_item(tab, blk, flags, next_flags, idx, mse_mode == MSE_FUSED_ROWS);
+        else mse_literal_item(tab, blk, MODE_ROW, idx, idx, nullptr, nullptr);
         return;
     }
     __shared__ double sp[kColFinSlices][kColFinCols], se[kColFinSlices][kColFinCols];
     const int lane = threadIdx.x & 31, sl = threadIdx.x >> 5;
-    // blocks enumerate 64-column slabs of every matrix in turn
-    for (int64_t slab = blockIdx.x; slab < total_slabs; slab += gcols) {
-        // matrix of this slab (slabs of matrix i start at its slab0)
-        const int mi = find_owner(tab, slab, [](const MatDesc &d) { return d.slab0; });
+    for (int64_t unit = blockIdx.x; unit < total_units; unit += gunits) {
+        const int mi = find_owner(tab, unit, [](const MatDesc &d) { return d.cunit0; });
         const MatDesc &md = tab.get(mi);
-        const int64_t c0 = (slab - md.slab0) * kColFinCols;
-        // columns c and c + 1 (cols is even, so both or neither exist)
+        const int64_t nrb = md.ntiles[MODE_COL] / max(md.ncb, 1);
+        const int64_t stride = md.cols / 2;                  // float4 per row block
+        if (nrb <= kColFinWarpRb) {                          // (uniform per block)
+            col_lane_unit<OS>(tab, md, unit, nrb);
+            continue;
+        }
+        const int64_t c0 = (unit - md.cunit0) * kColFinCols;
         const int64_t c = c0 + 2 * lane;
         const bool ok = c < md.cols;
-        const int64_t nrb = md.ntiles[MODE_COL] / max(md.ncb, 1);
         double p0 = 0.0, e0 = 0.0, p1 = 0.0, e1 = 0.0;
         if (ok) {
             const float4 *src = reinterpret_cast<const float4 *>(md.colpart + c);
-            const int64_t stride = md.cols / 2;              // float4 per row block
-            // this slice's row blocks in order; the loads of 8 of them are
+            // this slice's row blocks in order; the loads of 4 of them are
             // issued ahead of their sums (the order of the sums is unchanged)
-            for (int64_t k0 = sl; k0 < nrb; k0 += 8 * kColFinSlices) {
-                float4 v[8];
+            for (int64_t k0 = sl; k0 < nrb; k0 += 4 * kColFinSlices) {
+                float4 v[4];
 #pragma unroll
-                for (int u = 0; u < 8; ++u) {
+                for (int u = 0; u < 4; ++u) {
                     const int64_t k = k0 + (int64_t)u * kColFinSlices;
                     if (k < nrb) v[u] = __ldg(src + k * stride);
                 }
 #pragma unroll
-                for (int u = 0; u < 8; ++u) {
+                for (int u = 0; u < 4; ++u) {
                     if (k0 + (int64_t)u * kColFinSlices < nrb) {
                         p0 += v[u].x;
                         e0 += v[u].y;
@@ -1378,19 +1426,9 @@ col_finalize_kernel(const __grid_constant__ Table tab, int64_t total_cols, int64
         __syncthreads();
         const int cl = threadIdx.x;
         if (cl < kColFinCols && c0 + cl < md.cols) {
-            const int64_t cc = c0 + cl;
             double pt = 0.0, et = 0.0;
             for (int q = 0; q < kColFinSlices; ++q) { pt += sp[q][cl]; et += se[q][cl]; }
-            float b = 1.0f, pre = __int_as_float(0x7fc00000);
-            if (et > 0.0) {
-                pre = (float)(pt / et);
-                bool cl2;
-                b = project_outer<OS>(pre, cl2);
-                if (cl2) atomicOr(tab.status, STATUS_RANGE);
-            }
-            if (!isfinite(pt) || !isfinite(et)) atomicOr(tab.status, STATUS_NONFINITE);
-            md.b_out[cc] = b;
-            if (md.b_pre) md.b_pre[cc] = pre;
+            col_finish<OS>(tab, md, c0 + cl, pt, et);
         }
         __syncthreads();
     }
@@ -1402,7 +1440,9 @@ col_finalize_kernel(const __grid_constant__ Table tab, int64_t total_cols, int64
 __global__ void mse_finalize_kernel(const __grid_constant__ Table tab, int row_slot, int idx_trace, int idx_half,
                                     double *out_row, double *out_col) {
     grid_dependency_begin();
-    mse_literal_block(tab, blockIdx.x, row_slot, idx_trace, idx_half, out_row, out_col);
+    const int blk = (int)blockIdx.x * 8 + (int)(threadIdx.x >> 5);
+    if (blk >= 2 * tab.n) return;                       // (uniform per warp)
+    mse_literal_item(tab, blk, row_slot, idx_trace, idx_half, out_row, out_col);
 }
 
 // Initial state: a <- a0 or 1, b <- b0 or 1 (rows then columns, all matrices).
