@@ -155,8 +155,8 @@ struct Carve {
 
 // Fill geometry and workspace pointers of one descriptor.
 void place(MatDesc &d, bool f32, Carve &cv, int64_t tile_base[3], int64_t &row_base,
-           int64_t &col_base, int64_t &slab_base, int64_t &chunk_base) {
-    const Geom g = geometry(d.rows, d.cols, f32);
+           int64_t &col_base, int64_t &slab_base, int64_t &chunk_base, bool tall = false) {
+    const Geom g = geometry(d.rows, d.cols, f32, tall);
     d.wc = g.wc;
     d.ncb = g.ncb;
     for (int m = 0; m < 3; ++m) {
@@ -393,12 +393,25 @@ dq_status check_batch(int32_t n, const dq_matrix *mats, int32_t dtype, const dq_
     return DQ_OK;
 }
 
+// Whether a batch is tall (see geometry): its column passes make at least
+// kTallTiles tiles at the default geometry.
+bool tall_batch(int32_t n, const dq_matrix *mats, bool f32) {
+    int64_t tiles = 0;
+    for (int i = 0; i < n; ++i) tiles += geometry(mats[i].rows, mats[i].cols, f32).ntiles[1];
+    return tiles >= kTallTiles;
+}
+
+// tall_hint: -1 decides from this batch; 0 or 1 as given (a call that solves
+// a batch in parts passes the whole batch's choice, so that every part has
+// the geometry, and the sums, of the whole).
 dq_status solve_impl(int32_t n, const dq_matrix *mats, int32_t dtype, const dq_format *fmt,
-                     int32_t T, void *workspace, size_t ws_bytes, cudaStream_t st) {
+                     int32_t T, void *workspace, size_t ws_bytes, cudaStream_t st,
+                     int tall_hint = -1) {
     FmtInfo fi;
     dq_status s = check_batch(n, mats, dtype, fmt, T, workspace, ws_bytes, &fi);
     if (s != DQ_OK || n == 0) return s;
     const bool f32 = dtype == DQ_DT_F32;
+    const bool tall = tall_hint < 0 ? tall_batch(n, mats, f32) : tall_hint != 0;
 
     unsigned int *status = status_ptr();
     if (!status) return DQ_ERR_CUDA;
@@ -409,13 +422,13 @@ dq_status solve_impl(int32_t n, const dq_matrix *mats, int32_t dtype, const dq_f
     // The work table lists the matrices by decreasing tile height (stable):
     // CTAs are dispatched in tile order, so the short tiles of short matrices
     // fill the last wave instead of leaving SMs idle behind full-size tiles.
-    // Each matrix's tiles and sums depend on its own shape alone, so the
-    // order changes no result.
+    // Each matrix's tiles and sums depend on its own shape (and the batch's
+    // tall choice) alone, so the order changes no result.
     t_order.resize(n);
     for (int i = 0; i < n; ++i) t_order[i] = i;
     std::stable_sort(t_order.begin(), t_order.end(), [&](int x, int y) {
-        return geometry(mats[x].rows, mats[x].cols, f32).tr[1] >
-               geometry(mats[y].rows, mats[y].cols, f32).tr[1];
+        return geometry(mats[x].rows, mats[x].cols, f32, tall).tr[1] >
+               geometry(mats[y].rows, mats[y].cols, f32, tall).tr[1];
     });
     t_table.assign(n, MatDesc{});
     int64_t tile_base[3] = {0, 0, 0}, row_base = 0, col_base = 0, slab_base = 0, chunk_base = 0;
@@ -438,7 +451,7 @@ dq_status solve_impl(int32_t n, const dq_matrix *mats, int32_t dtype, const dq_f
         d.b0 = m.b0;
         d.mse_trace = m.mse_trace;
         d.mse_half = m.mse_half;
-        place(d, f32, cv, tile_base, row_base, col_base, slab_base, chunk_base);
+        place(d, f32, cv, tile_base, row_base, col_base, slab_base, chunk_base, tall);
     }
     Launcher L;
     L.tab.dev = dev_table;
@@ -1123,6 +1136,9 @@ dq_status dq_solve_dual_scale_batched_host(int32_t n, const dq_matrix *host, con
     const bool f32 = dtype == DQ_DT_F32;
     size_t total_in = 0;
     for (int i = 0; i < n; ++i) total_in += (size_t)host[i].rows * (size_t)host[i].cols * esz;
+    // every group takes the whole batch's geometry (the device batched
+    // solve's sums)
+    const int tall = tall_batch(n, host, f32) ? 1 : 0;
     const size_t target = std::max(total_in / 8, (size_t)32 << 20);
     int devno = 0;
     if (cudaGetDevice(&devno) != cudaSuccess || devno < 0 || devno >= kMaxDevices) return DQ_ERR_CUDA;
@@ -1170,7 +1186,7 @@ dq_status dq_solve_dual_scale_batched_host(int32_t n, const dq_matrix *host, con
         DQ_CUDA(cudaEventRecord(in, sh));
         // solve them on the compute stream once their inputs have landed
         DQ_CUDA(cudaStreamWaitEvent(sc, in, 0));
-        if ((s = solve_impl(j - i, dm.data() + i, dtype, fmt, T, workspace, ws_bytes, sc)) != DQ_OK) return s;
+        if ((s = solve_impl(j - i, dm.data() + i, dtype, fmt, T, workspace, ws_bytes, sc, tall)) != DQ_OK) return s;
         DQ_CUDA(cudaEventRecord(out, sc));
         // out: the results the caller asked for in host memory
         DQ_CUDA(cudaStreamWaitEvent(sd, out, 0));

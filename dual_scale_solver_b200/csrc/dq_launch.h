@@ -24,7 +24,12 @@ struct Geom {
     int64_t nrb_col;
 };
 
-inline Geom geometry(int64_t rows, int64_t cols, bool f32) {
+// tall: a batch with many tiles (kTallTiles at the default geometry) gives
+// every matrix at least 64 rows per warp: short matrices then take fewer,
+// longer tiles (a tile's set-up and drain cost about as much as 16 of its
+// rows), while alone they keep about 16 row blocks to spread over the GPU.
+constexpr int64_t kTallTiles = 8 * 2 * 148;      // 8 waves of the column pass (2 CTAs per SM)
+inline Geom geometry(int64_t rows, int64_t cols, bool f32, bool tall = false) {
     Geom g{};
     const int epc = f32 ? 4 : 8, seg = 32 * epc;
     const int64_t nseg = (cols + seg - 1) / seg;
@@ -45,8 +50,9 @@ inline Geom geometry(int64_t rows, int64_t cols, bool f32) {
     const int wr = kWarps / wc;
     // rows per warp: 256 for column statistics (fewer partial sums), 128 for
     // the other modes (tile set-up spread over the rows), both reduced for
-    // short matrices so that they still make about 16 row blocks
-    int rpw_long = 16;
+    // short matrices so that they still make about 16 row blocks (at least
+    // 16 rows, or 64 in a tall batch)
+    int rpw_long = tall ? 64 : 16;
     while (rpw_long < 128 && 2 * rpw_long <= rows / (wr * 16)) rpw_long *= 2;
     int rpw_col = rpw_long;
     while (rpw_col < 256 && 2 * rpw_col <= rows / (wr * 16)) rpw_col *= 2;

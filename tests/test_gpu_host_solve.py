@@ -118,3 +118,21 @@ def test_host_solve_empty_and_zero_matrices():
     for o, r in zip(outs, ref):
         _same(o, r)
     assert torch.all(outs[1]["codes"] == 0) and torch.all(outs[1]["mse_trace"] == 0)
+
+
+def test_host_solve_of_a_tall_batch_equals_device_batched():
+    # A batch of many short matrices (170 x 15 column-pass tiles at the
+    # default geometry) takes taller tiles; the host-streamed solve solves it
+    # in groups of about 50 matrices, each of which alone would not, and
+    # still gives the device batched solve's bits.
+    fmt = lib_format("mxfp4", 32)
+    g = torch.Generator().manual_seed(8)
+    Ws = [(torch.randn(576, 576, generator=g) * 0.02).to(torch.bfloat16) for _ in range(170)]
+    T = 2
+    ref = dq.solve_dual_scale_batched([W.cuda() for W in Ws], fmt, T, half=True)
+    outs, dev_outs = dq.solve_dual_scale_batched_host([W.pin_memory() for W in Ws], fmt, T,
+                                                      half=True)
+    torch.cuda.synchronize()
+    assert dq.last_device_status() == 0
+    for o, r in zip(outs, ref):
+        _same(o, r)
