@@ -167,8 +167,14 @@ DQ_API dq_status dq_dequantize(const uint8_t *codes, const void *gscales, int64_
  * iterations of {row update, re-quantize, column update, re-quantize}
  * (eq. (2) and the order stated under it), then write the codes and group
  * scales of Q(W ⊘ (a bᵀ)) for the final a, b.  tensor_scale (1 float) receives
- * the ts used.  mse_trace (T+1) and mse_half (T) may be NULL.  `workspace`
- * must hold dq_workspace_size bytes for this one matrix. */
+ * the ts used.  mse_trace (T+1) and mse_half (T) may be NULL; entry t is
+ * mean((W - D_a Qhat D_b)^2) of the state before iteration t's row step
+ * (mse_half: before its column step), the last entry that of the final
+ * state.  The last entry is summed as (W - R)^2; for MXFP4 and MXINT4 the
+ * others are taken per row as sum W^2 - 2 sum W R + sum R^2 from float32 row
+ * sums (correct to about 1e-5 relative, exactly 0 for rows that Q
+ * reproduces).  `workspace` must hold dq_workspace_size bytes for this one
+ * matrix. */
 DQ_API dq_status dq_solve_dual_scale(const void *W, int32_t dtype, int64_t rows, int64_t cols,
                               const dq_format *fmt, int32_t T, const float *a0,
                               const float *b0, uint8_t *codes, void *gscales, float *a,
