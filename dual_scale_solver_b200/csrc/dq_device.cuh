@@ -1162,6 +1162,10 @@ row_finalize_kernel(const __grid_constant__ Table tab, int64_t total_chunks, uns
         const int64_t r = (ch - md.rchunk0) * kRowFinRows + threadIdx.x;
         double err = 0.0;
         if (r < md.rows) {
+            // (the row's old scale and stored sum of squares are loaded ahead
+            // of its partial sums)
+            const float a_old = (scale_old && md.a) ? md.a[r] : 1.0f;
+            const double w2_old = row_mse == 1 ? md.w2row[r] : 0.0;
             double num = 0.0, den = 0.0;
             const float2 *p = md.rowpart + r * md.ncb;
             // the row's column blocks in order; loads issued a batch ahead of
@@ -1184,12 +1188,12 @@ row_finalize_kernel(const __grid_constant__ Table tab, int64_t total_chunks, uns
                     for (int k = 0; k < md.ncb; ++k) w2 += __ldg(q + k);
                     md.w2row[r] = w2;
                 } else {
-                    w2 = md.w2row[r];
+                    w2 = w2_old;
                 }
                 if (scale_old) err = (w2 - 2.0 * num) + den;
             }
             if (scale_old) {
-                const double ia = (double)recip_pow2(md.a ? md.a[r] : 1.0f);
+                const double ia = (double)recip_pow2(a_old);
                 num *= ia;
                 den *= ia * ia;
             }
