@@ -1243,7 +1243,7 @@ dq_status dq_col_finalize(const float *partials, int64_t row_blocks, int64_t col
     FmtInfo fi;
     dq_status s = check_format(fmt, &fi);
     if (s != DQ_OK) return s;
-    if (row_blocks < 0 || cols < 0 || cols % 2) return DQ_ERR_SHAPE;
+    if (row_blocks < 0 || cols < 0 || cols % fi.G) return DQ_ERR_SHAPE;   // (as the solves)
     if (cols == 0) return DQ_OK;
     if (!b_out || (row_blocks > 0 && !partials)) return DQ_ERR_ARG;
     if (!aligned(partials, 16) || !aligned(b_out, 4) || !aligned(b_pre, 4)) return DQ_ERR_ALIGN;

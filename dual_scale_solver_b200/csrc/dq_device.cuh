@@ -1316,13 +1316,14 @@ __device__ __forceinline__ void mse_fused_item(const Table &tab, int blk,
 // in a fixed order that depends only on the matrix's shape: the column's row
 // blocks are split into 8 slices (slice s: row blocks s, s+8, ... added in
 // order), and the slices are added in order.  A matrix whose column pass has
-// more than 16 row blocks takes a block per 64 consecutive columns (a
-// "slab"; a lane reads the partials of two adjacent columns as one 16-byte
-// load), a warp per slice; a shorter one a warp per 32 columns, a lane per
-// column holding all of its row blocks in registers and forming the same
-// sums in the same order (a block: 256 columns).  Work units (a block's
-// columns) of all matrices in order.
-constexpr int kColFinCols = 64, kColFinSlices = 8;
+// more than 8 row blocks takes a block per 128 consecutive columns (a lane
+// reads the partials of four adjacent columns as two 16-byte loads), a warp
+// per slice; a shorter one a warp per 32 columns, a lane per column holding
+// all of its row blocks in registers and forming the same sums in the same
+// order (a block: 256 columns).  Work units (a block's columns) of all
+// matrices in order.  (Columns come in multiples of 16: a lane's four are
+// all in or all out.)
+constexpr int kColFinCols = 128, kColFinSlices = 8;
 constexpr int kColFinThreads = 32 * kColFinSlices;
 constexpr int kColFinWarpRb = kColFinSlices;       // most row blocks of the lane-per-column form
 __host__ __device__ __forceinline__ int64_t col_units(int64_t rows_blocks, int64_t cols) {
@@ -1398,35 +1399,46 @@ col_finalize_kernel(const __grid_constant__ Table tab, int64_t total_units, int 
             continue;
         }
         const int64_t c0 = (unit - md.cunit0) * kColFinCols;
-        const int64_t c = c0 + 2 * lane;
+        const int64_t c = c0 + 4 * lane;
         const bool ok = c < md.cols;
-        double p0 = 0.0, e0 = 0.0, p1 = 0.0, e1 = 0.0;
+        double p0 = 0.0, e0 = 0.0, p1 = 0.0, e1 = 0.0, p2 = 0.0, e2 = 0.0, p3 = 0.0, e3 = 0.0;
         if (ok) {
             const float4 *src = reinterpret_cast<const float4 *>(md.colpart + c);
-            // this slice's row blocks in order; the loads of 4 of them are
+            // this slice's row blocks in order; the loads of 2 of them are
             // issued ahead of their sums (the order of the sums is unchanged)
-            for (int64_t k0 = sl; k0 < nrb; k0 += 4 * kColFinSlices) {
-                float4 v[4];
+            for (int64_t k0 = sl; k0 < nrb; k0 += 2 * kColFinSlices) {
+                float4 v[2], w[2];
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
+                for (int u = 0; u < 2; ++u) {
                     const int64_t k = k0 + (int64_t)u * kColFinSlices;
-                    if (k < nrb) v[u] = __ldg(src + k * stride);
+                    if (k < nrb) {
+                        v[u] = __ldg(src + k * stride);
+                        w[u] = __ldg(src + k * stride + 1);
+                    }
                 }
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
+                for (int u = 0; u < 2; ++u) {
                     if (k0 + (int64_t)u * kColFinSlices < nrb) {
                         p0 += v[u].x;
                         e0 += v[u].y;
                         p1 += v[u].z;
                         e1 += v[u].w;
+                        p2 += w[u].x;
+                        e2 += w[u].y;
+                        p3 += w[u].z;
+                        e3 += w[u].w;
                     }
                 }
             }
         }
-        sp[sl][2 * lane] = p0;
-        se[sl][2 * lane] = e0;
-        sp[sl][2 * lane + 1] = p1;
-        se[sl][2 * lane + 1] = e1;
+        sp[sl][4 * lane] = p0;
+        se[sl][4 * lane] = e0;
+        sp[sl][4 * lane + 1] = p1;
+        se[sl][4 * lane + 1] = e1;
+        sp[sl][4 * lane + 2] = p2;
+        se[sl][4 * lane + 2] = e2;
+        sp[sl][4 * lane + 3] = p3;
+        se[sl][4 * lane + 3] = e3;
         __syncthreads();
         const int cl = threadIdx.x;
         if (cl < kColFinCols && c0 + cl < md.cols) {

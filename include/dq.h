@@ -262,8 +262,9 @@ DQ_API dq_status dq_col_update(const void *W, int32_t dtype, int64_t rows, int64
  *   workspace as dq_col_update.
  * dq_col_finalize: b_out_j = Pi_Fb(sum_k P[k][j] / sum_k E[k][j]) (zero
  *   slice -> 1) over row_blocks slabs of cols float pairs (row block
- *   major), summed in the fixed order of the solves' column update; b_pre
- *   (may be NULL) the unprojected ratios.
+ *   major; cols a multiple of fmt's group size, as for the solves, else
+ *   DQ_ERR_SHAPE), summed in the fixed order of the solves' column update;
+ *   b_pre (may be NULL) the unprojected ratios.
  * With shards whose first rows are multiples of row_block, the shards'
  * partials concatenated in row order are the whole matrix's, so
  * dq_col_finalize gives dq_col_update's b bit for bit. */

@@ -215,7 +215,8 @@ def test_sharded_column_entry_points_argument_errors():
                              1 << 30, None) == -2              # below the shard's own row block
     assert L.dq_col_partials(p, 1, 64, 64, ctypes.byref(f), 1.0, p, p, 128, p, None, None,
                              0, None) == -7                    # workspace
-    # finalize: odd columns, null output
+    # finalize: columns not a multiple of the group size, null output
     assert L.dq_col_finalize(p, 4, 63, ctypes.byref(f), p, None, None) == -2
+    assert L.dq_col_finalize(p, 4, 66, ctypes.byref(f), p, None, None) == -2
     assert L.dq_col_finalize(p, 4, 64, ctypes.byref(f), None, None, None) == -1
     assert L.dq_col_finalize(None, 0, 0, ctypes.byref(f), None, None, None) == 0
