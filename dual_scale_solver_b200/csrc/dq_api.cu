@@ -155,7 +155,7 @@ struct Carve {
 
 // Fill geometry and workspace pointers of one descriptor.
 void place(MatDesc &d, bool f32, Carve &cv, int64_t tile_base[3], int64_t &row_base,
-           int64_t &col_base, int64_t &slab_base, int64_t &chunk_base, bool tall = false) {
+           int64_t &col_base, int64_t &unit_base, int64_t &chunk_base, bool tall = false) {
     const Geom g = geometry(d.rows, d.cols, f32, tall);
     d.wc = g.wc;
     d.ncb = g.ncb;
@@ -168,8 +168,8 @@ void place(MatDesc &d, bool f32, Carve &cv, int64_t tile_base[3], int64_t &row_b
     d.row0 = row_base;
     d.col0 = col_base;
     // (work units of the column finalize before this matrix)
-    d.cunit0 = slab_base;
-    slab_base += col_units(g.nrb_col, d.cols);
+    d.cunit0 = unit_base;
+    unit_base += col_units(g.nrb_col, d.cols);
     // (256-row chunks of the row finalize, likewise)
     d.rchunk0 = chunk_base;
     chunk_base += (d.rows + kRowFinRows - 1) / kRowFinRows;
@@ -431,7 +431,7 @@ dq_status solve_impl(int32_t n, const dq_matrix *mats, int32_t dtype, const dq_f
                geometry(mats[y].rows, mats[y].cols, f32, tall).tr[1];
     });
     t_table.assign(n, MatDesc{});
-    int64_t tile_base[3] = {0, 0, 0}, row_base = 0, col_base = 0, slab_base = 0, chunk_base = 0;
+    int64_t tile_base[3] = {0, 0, 0}, row_base = 0, col_base = 0, unit_base = 0, chunk_base = 0;
     for (int i = 0; i < n; ++i) {
         const dq_matrix &m = mats[t_order[i]];
         MatDesc &d = t_table[i];
@@ -451,7 +451,7 @@ dq_status solve_impl(int32_t n, const dq_matrix *mats, int32_t dtype, const dq_f
         d.b0 = m.b0;
         d.mse_trace = m.mse_trace;
         d.mse_half = m.mse_half;
-        place(d, f32, cv, tile_base, row_base, col_base, slab_base, chunk_base, tall);
+        place(d, f32, cv, tile_base, row_base, col_base, unit_base, chunk_base, tall);
     }
     Launcher L;
     L.tab.dev = dev_table;
