@@ -400,6 +400,11 @@ bool tall_batch(int32_t n, const dq_matrix *mats, bool f32) {
     for (int i = 0; i < n; ++i) tiles += geometry(mats[i].rows, mats[i].cols, f32).ntiles[1];
     return tiles >= kTallTiles;
 }
+// The same choice for one matrix alone (the single-matrix entry points take
+// it, so that their sums are those of dq_solve_dual_scale).
+bool tall_single(int64_t rows, int64_t cols, bool f32) {
+    return geometry(rows, cols, f32).ntiles[1] >= kTallTiles;
+}
 
 // tall_hint: -1 decides from this batch; 0 or 1 as given (a call that solves
 // a batch in parts passes the whole batch's choice, so that every part has
@@ -558,7 +563,7 @@ dq_status step_impl(bool row_step, const void *W, int32_t dtype, int64_t rows, i
     else { d.b_out = out; d.b_pre = pre; }
     Carve cv{static_cast<char *>(workspace), static_cast<char *>(workspace) + ws_bytes};
     int64_t tb[3] = {0, 0, 0}, rb = 0, cb = 0, sb = 0, hb = 0;
-    place(d, f32, cv, tb, rb, cb, sb, hb);
+    place(d, f32, cv, tb, rb, cb, sb, hb, tall_single(d.rows, d.cols, f32));
     Launcher L;
     L.tab.dev = nullptr;
     L.tab.one = d;
@@ -1227,7 +1232,8 @@ dq_status dq_col_update(const void *W, int32_t dtype, int64_t rows, int64_t cols
 
 int64_t dq_col_row_block(int64_t rows, int64_t cols, int32_t dtype) {
     if (rows < 0 || cols < 0 || (dtype != DQ_DT_F32 && dtype != DQ_DT_BF16)) return -1;
-    return geometry(rows, cols, dtype == DQ_DT_F32).tr[1];
+    const bool f32 = dtype == DQ_DT_F32;
+    return geometry(rows, cols, f32, tall_single(rows, cols, f32)).tr[1];
 }
 
 dq_status dq_col_partials(const void *W, int32_t dtype, int64_t rows, int64_t cols,
@@ -1404,7 +1410,7 @@ extern "C" dq_status dq_solve_dual_scale_noalloc(const void *W, int32_t dtype, i
              reinterpret_cast<char *>(scratch) + DQ_NOALLOC_SCRATCH_BYTES};
     unsigned int *flags = cv.take<unsigned int>(256);     // one-pass MX flags: 3 slots x 2 words
     int64_t tb[3] = {0, 0, 0}, rb = 0, cb = 0, sb = 0, hb = 0;
-    place(d, f32, cv, tb, rb, cb, sb, hb);
+    place(d, f32, cv, tb, rb, cb, sb, hb, tall_single(d.rows, d.cols, f32));
     Launcher L;
     L.tab.dev = nullptr;
     L.tab.one = d;
