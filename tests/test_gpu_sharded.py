@@ -85,3 +85,29 @@ def test_col_partials_refuse_a_row_block_below_the_shards_own():
     b2, _, _ = dq.col_update(W, fl, a, b)
     torch.cuda.synchronize()
     assert torch.equal(b1, b2)
+
+
+def test_row_shards_of_a_wide_tall_matrix_equal_the_unsharded_solve():
+    # 256 x 1,310,720: alone it makes more than 8 waves of column-pass tiles,
+    # so its tiles take at least 64 rows per warp (a "tall" geometry);
+    # dq_col_row_block and the step entry points take the same choice as
+    # the unsharded solve, and the two-shard solve stays bit-identical.
+    from dual_scale_solver_b200 import sharded
+    fl = lib_format("int4_bf16", 64)
+    rows, cols, T = 256, 1310720, 2
+    W = _weights(rows, cols, key=5)
+    rb = dq.col_row_block(rows, cols)
+    assert rb == 64                                     # 64 rows per warp, 1 warp row
+    starts = [0, 128, rows]
+    shards = [sharded.RowShard(W[s0:s1], s0, rows, fl) for s0, s1 in zip(starts, starts[1:])]
+    b = torch.ones(cols, device="cuda")
+    for _ in range(T):
+        for sh in shards:
+            sh.row_step(b)
+        parts = torch.cat([sh.col_partials(b)[0] for sh in shards])
+        b = shards[0].col_finalize(parts)
+    o = dq.solve_dual_scale(W, fl, T)
+    torch.cuda.synchronize()
+    assert dq.last_device_status() == 0
+    assert torch.equal(torch.cat([sh.a for sh in shards]), o["a"])
+    assert torch.equal(b, o["b"])
