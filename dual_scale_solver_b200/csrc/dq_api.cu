@@ -233,8 +233,8 @@ struct Launcher {
     int64_t tiles[3] = {0, 0, 0};
     int64_t total_rows = 0, total_cols = 0;
     cudaStream_t st;
-    // one-pass iterations take each row's squared error from its row sums
-    // (4-bit MX formats; set when an MSE output is wanted)
+    // the iterations take each row's squared error from its row sums (4-bit
+    // codes; set when an MSE output is wanted)
     bool row_mse = false;
 
     // One tile pass.  A gated pass (the literal fallback of a fused
@@ -244,7 +244,8 @@ struct Launcher {
         TileLaunch L;
         L.tab = tab;
         L.mode = mode;
-        L.slot = (mode == MODE_ACT) ? 2 : ((mode == MODE_FUSED || mode == MODE_FUSED_W2) ? 1 : mode);
+        L.slot = (mode == MODE_ACT) ? 2
+                 : ((mode == MODE_FUSED || mode == MODE_FUSED_W2) ? 1 : (mode == MODE_ROW_W2 ? 0 : mode));
         L.tiles = tiles[L.slot];
         L.grid = gate ? std::min<int64_t>(L.tiles, 148) : L.tiles;
         L.f32 = f32 ? 1 : 0;
@@ -255,8 +256,8 @@ struct Launcher {
         L.stream = st;
         if (L.grid <= 0) return DQ_OK;
         cudaEvent_t beg = nullptr, end = nullptr;
-        // (the first one-pass iteration's variant is timed as the one-pass kind)
-        const int kind = mode == MODE_FUSED_W2 ? MODE_FUSED : mode;
+        // (the variants that also sum each row's squares are timed as their kind)
+        const int kind = mode == MODE_FUSED_W2 ? MODE_FUSED : (mode == MODE_ROW_W2 ? MODE_ROW : mode);
         {
             std::lock_guard<std::mutex> lk(g_timing_mu);
             if (!t_capturing && (g_timing_kinds & (1u << kind))) { beg = take_event(); end = take_event(); }
@@ -335,10 +336,12 @@ struct Launcher {
         unsigned int *next = flag_slots + 2 * ((t + 1) % 3);
         unsigned int *clear = flag_slots + 2 * ((t + 2) % 3);
         if (!fused) {
-            if ((s = tiles_pass(MODE_ROW, want_trace)) != DQ_OK) return s;
-            if ((s = row_finalize()) != DQ_OK) return s;
+            // with row_mse the first iteration's row pass also sums the rows' squares
+            const int rmode = (row_mse && t == 0) ? MODE_ROW_W2 : MODE_ROW;
+            if ((s = tiles_pass(rmode, want_trace)) != DQ_OK) return s;
+            if ((s = row_finalize(nullptr, nullptr, row_mse ? (t == 0 ? 2 : 1) : 0)) != DQ_OK) return s;
             if ((s = tiles_pass(MODE_COL, want_half)) != DQ_OK) return s;
-            return col_finalize(MSE_LITERAL, nullptr, nullptr, t);
+            return col_finalize(row_mse ? MSE_LITERAL_ROWS : MSE_LITERAL, nullptr, nullptr, t);
         }
         // with row_mse the first iteration's pass also sums the rows' squares
         const int fmode = (row_mse && t == 0) ? MODE_FUSED_W2 : MODE_FUSED;
@@ -352,13 +355,12 @@ struct Launcher {
 
 // MX formats: power-of-two outer and group scales
 bool fused_ok(int combo) { return all_e8m0(combo); }
-// 4-bit MX formats: their one-pass iterations take the squared error per row
-// from the row sums (about 1% of sum W^2 for 4-bit codes, so the float32
-// row sums leave it correct to about 1e-5 relative; wider codes, whose error
-// is a far smaller share of sum W^2, sum (W - R)^2 directly)
-bool row_mse_ok(int combo) {
-    return combo == COMBO_INT4_E8M0_E8M0 || combo == COMBO_E2M1_E8M0_E8M0;
-}
+// Formats with 4-bit codes: their iterations take the squared error of the
+// state per row from the row sums (about 1% of sum W^2 for 4-bit codes, so
+// the float32 row sums leave it correct to about 1e-5 relative; wider
+// codes, whose error is a far smaller share of sum W^2, sum (W - R)^2
+// directly)
+bool row_mse_ok(int combo) { return combo <= COMBO_E2M1_E8M0_BF16; }
 
 thread_local std::vector<MatDesc> t_table;
 thread_local std::vector<int> t_order;
@@ -511,7 +513,7 @@ dq_status solve_impl(int32_t n, const dq_matrix *mats, int32_t dtype, const dq_f
         want_trace |= mats[i].mse_trace != nullptr;
         want_half |= mats[i].mse_half != nullptr;
     }
-    L.row_mse = fused && row_mse_ok(fi.combo) && (want_trace || want_half);
+    L.row_mse = T > 0 && row_mse_ok(fi.combo) && (want_trace || want_half);
     for (int t = 0; t < T; ++t)
         if ((s = L.iteration(t, fused, flags, want_trace, want_half)) != DQ_OK) return s;
     if ((s = L.tiles_pass(MODE_PACK, want_trace)) != DQ_OK) return s;
@@ -578,9 +580,12 @@ dq_status step_impl(bool row_step, const void *W, int32_t dtype, int64_t rows, i
     L.total_cols = cb;
     L.st = st;
     if (row_step) {
-        if ((s = L.tiles_pass(MODE_ROW, mse_in != nullptr)) != DQ_OK) return s;
-        if ((s = L.row_finalize()) != DQ_OK) return s;
-        if (mse_in) return L.mse(MODE_ROW, -1, -1, mse_in, nullptr);
+        // 4-bit codes: the state's squared error from the row sums, with the
+        // rows' squares summed by the same pass
+        const bool rows = mse_in != nullptr && row_mse_ok(fi.combo);
+        if ((s = L.tiles_pass(rows ? MODE_ROW_W2 : MODE_ROW, mse_in != nullptr)) != DQ_OK) return s;
+        if ((s = L.row_finalize(nullptr, nullptr, rows ? 2 : 0)) != DQ_OK) return s;
+        if (mse_in) return L.mse(rows ? kSlotRows : MODE_ROW, -1, -1, mse_in, nullptr);
     } else {
         if ((s = L.tiles_pass(MODE_COL, mse_in != nullptr)) != DQ_OK) return s;
         if ((s = L.col_finalize()) != DQ_OK) return s;
@@ -1447,7 +1452,7 @@ extern "C" dq_status dq_solve_dual_scale_noalloc(const void *W, int32_t dtype, i
                          rb, cb, fused ? flags : nullptr));
         count_launches(1);
     }
-    L.row_mse = fused && row_mse_ok(fi.combo) && (mse_trace != nullptr || mse_half != nullptr);
+    L.row_mse = T > 0 && row_mse_ok(fi.combo) && (mse_trace != nullptr || mse_half != nullptr);
     for (int t = 0; t < T; ++t)
         if ((s = L.iteration(t, fused, flags, mse_trace != nullptr, mse_half != nullptr)) != DQ_OK)
             return s;

@@ -27,14 +27,16 @@ namespace dq {
 enum { CODES_INT4 = 0, CODES_E2M1 = 1, CODES_INT8 = 2, CODES_E4M3 = 3, CODES_E5M2 = 4,
        CODES_E2M3 = 5, CODES_E3M2 = 6 };
 enum { SC_BF16 = 0, SC_E8M0 = 1, SC_E4M3 = 2 };
-// MODE_FUSED_W2: MODE_FUSED that also sums each row's squares (the first
-// one-pass iteration of the 4-bit MX formats; see the tile kernel)
-enum { MODE_ROW = 0, MODE_COL = 1, MODE_PACK = 2, MODE_ACT = 3, MODE_FUSED = 4, MODE_FUSED_W2 = 5 };
+// MODE_FUSED_W2 / MODE_ROW_W2: MODE_FUSED / MODE_ROW that also sum each
+// row's squares (the first iteration of a solve with 4-bit codes, and the
+// row step entry point; see the tile kernel)
+enum { MODE_ROW = 0, MODE_COL = 1, MODE_PACK = 2, MODE_ACT = 3, MODE_FUSED = 4, MODE_FUSED_W2 = 5,
+       MODE_ROW_W2 = 6 };
 enum { STATUS_NONFINITE = 1u, STATUS_RANGE = 2u, STATUS_TIMEOUT = 4u };
 
 constexpr int kWarps = 8;            // warps per CTA of the tile kernel
 constexpr int kThreads = 32 * kWarps;
-constexpr int kRowsPerWarp[6] = {128, 256, 128, 128, 256, 256};   // per mode (at most)
+constexpr int kRowsPerWarp[7] = {128, 256, 128, 128, 256, 256, 128};   // per mode (at most)
 constexpr int kRowFinRows = 256;     // rows per block of the row finalize
 constexpr int kRing = 4;             // cp.async ring slots per lane (rows in flight + 1)
 constexpr float kBf16Max = 3.38953138925153547590470800371487866880e+38f;  // (2-2^-7)*2^127
@@ -733,12 +735,13 @@ template <int MODE, int EPC>
 struct TileSmem {
     static constexpr int RPW = kRowsPerWarp[MODE];
     static constexpr bool kFused = MODE == MODE_FUSED || MODE == MODE_FUSED_W2;
-    static constexpr bool kW2 = MODE == MODE_FUSED_W2;
+    static constexpr bool kRowM = MODE == MODE_ROW || MODE == MODE_ROW_W2;
+    static constexpr bool kW2 = MODE == MODE_FUSED_W2 || MODE == MODE_ROW_W2;
     // ROW, FUSED: per (warp, row of a batch of 8, lane) partial (num, den),
     // reduced every 8 rows.  Row stride padded by one entry.
-    static constexpr int kRed = (MODE == MODE_ROW || kFused) ? kWarps * 8 * 33 : 1;
+    static constexpr int kRed = (kRowM || kFused) ? kWarps * 8 * 33 : 1;
     // ROW, FUSED: per (row, warp) totals
-    static constexpr int kRtot = (MODE == MODE_ROW || kFused) ? RPW * kWarps : 1;
+    static constexpr int kRtot = (kRowM || kFused) ? RPW * kWarps : 1;
     // COL, FUSED: per (warp-row, column) partials
     static constexpr int kPart = (MODE == MODE_COL || kFused) ? kWarps * 32 * EPC : 1;
     float2 red[kRed];
@@ -754,7 +757,7 @@ struct TileSmem {
 // Column statistics keep 2 x EPC accumulators per lane: those modes run 2
 // CTAs per SM (up to 128 registers), the others 3.
 template <int MODE> struct TileOcc {
-    static constexpr int kMinBlocks = (MODE == MODE_COL || MODE == MODE_FUSED || MODE == MODE_FUSED_W2) ? 2 : 3;
+    static constexpr int kMinBlocks = (MODE == MODE_COL || MODE == MODE_FUSED || MODE == MODE_FUSED_W2) ? 2 : 3;   // (ROW_W2: 3)
 };
 
 template <int CODES, int GS, int OS, int MODE, typename TIn, int G>
@@ -770,12 +773,13 @@ tile_kernel(const __grid_constant__ Table tab, int mode_slot, int want_res, int6
     constexpr bool ACT = MODE == MODE_ACT;
     constexpr bool NIB = MODE == MODE_PACK || MODE == MODE_ACT;
     constexpr bool FUSED = MODE == MODE_FUSED || MODE == MODE_FUSED_W2;
-    constexpr bool W2 = MODE == MODE_FUSED_W2;
-    // 4-bit codes: the one-pass iteration's squared error is taken per row
-    // from its row sums (the row finalize), not summed here
-    constexpr bool kRowMse = FUSED && CodeTraits<CODES>::kBits == 4;
-    static_assert(!W2 || kRowMse, "row sums of squares serve the 4-bit one-pass path");
-    constexpr bool ROWSTAT = MODE == MODE_ROW || FUSED;
+    constexpr bool ROWM = MODE == MODE_ROW || MODE == MODE_ROW_W2;
+    constexpr bool W2 = MODE == MODE_FUSED_W2 || MODE == MODE_ROW_W2;
+    // 4-bit codes: the squared error of the state is taken per row from its
+    // row sums (the row finalize), not summed by the passes with row sums
+    constexpr bool kRowMse = (FUSED || ROWM) && CodeTraits<CODES>::kBits == 4;
+    static_assert(!W2 || kRowMse, "row sums of squares serve the 4-bit codes");
+    constexpr bool ROWSTAT = ROWM || FUSED;
     constexpr bool COLSTAT = MODE == MODE_COL || FUSED;
     using Q = Quant<CODES, GS, OS, ACT, NP, LPG>;
     static_assert(!FUSED || (GS == SC_E8M0 && OS == SC_E8M0), "fused statistics need power-of-two scales");
@@ -1142,11 +1146,11 @@ tile_kernel(const __grid_constant__ Table tab, int mode_slot, int want_res, int6
 // 1/a_old and 1/a_old^2 here; a new scale with |e(a)| > 26 raises flags[1]
 // (the column step is redone literally) and one with |e(a)| > 20 raises the
 // next iteration's flags[0] (its row step is done literally).
-// row_mse (the one-pass path of the 4-bit MX formats): the squared error of
-// each row of the state, sum_j (W_ij - R_ij)^2 = sum W^2 - 2 sum W R +
-// sum R^2 from the fused row sums (a = 1), summed over the block's rows in
-// a fixed order -> mse_part[chunk]; row_mse = 2 first sums the row's
-// squares from the fused pass (rowsq -> w2row), 1 reads them.
+// row_mse (the formats with 4-bit codes): the squared error of each row of
+// the state, sum_j (W_ij - a_i R_ij)^2 = sum W^2 - 2 a sum W R + a^2 sum
+// R^2 from its row sums (the one-pass sums are for a = 1), summed over the
+// block's rows in a fixed order -> mse_part[chunk]; row_mse = 2 first sums
+// the row's squares from the pass's (rowsq -> w2row), 1 reads them.
 // A block handles one 256-row chunk of one matrix at a time (chunks of all
 // matrices in order, grid-stride).
 template <int OS>
@@ -1164,7 +1168,7 @@ row_finalize_kernel(const __grid_constant__ Table tab, int64_t total_chunks, uns
         if (r < md.rows) {
             // (the row's old scale and stored sum of squares are loaded ahead
             // of its partial sums)
-            const float a_old = (scale_old && md.a) ? md.a[r] : 1.0f;
+            const float a_old = ((scale_old || row_mse) && md.a) ? md.a[r] : 1.0f;
             const double w2_old = row_mse == 1 ? md.w2row[r] : 0.0;
             double num = 0.0, den = 0.0;
             const float2 *p = md.rowpart + r * md.ncb;
@@ -1190,7 +1194,14 @@ row_finalize_kernel(const __grid_constant__ Table tab, int64_t total_chunks, uns
                 } else {
                     w2 = w2_old;
                 }
-                if (scale_old) err = (w2 - 2.0 * num) + den;
+                // the one-pass sums are for a = 1 (R = D_a Qhat D_b); the
+                // literal ones for R = Qhat D_b, whose state is a R
+                if (scale_old) {
+                    err = (w2 - 2.0 * num) + den;
+                } else {
+                    const double as = (double)a_old;
+                    err = (w2 - 2.0 * as * num) + (as * as) * den;
+                }
             }
             if (scale_old) {
                 const double ia = (double)recip_pow2(a_old);
@@ -1213,7 +1224,7 @@ row_finalize_kernel(const __grid_constant__ Table tab, int64_t total_chunks, uns
             md.a_out[r] = a;
             if (md.a_pre) md.a_pre[r] = pre;
         }
-        if (row_mse && scale_old) {                       // (uniform per block)
+        if (row_mse) {                                    // (uniform per block)
             // the chunk's errors in a fixed order: lanes, then warps
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) err += __shfl_xor_sync(0xffffffffu, err, o);
@@ -1253,9 +1264,11 @@ __device__ __forceinline__ void mse_reduce_warp(const double *src, int64_t n, do
 }
 
 // Item blk = 2 mi + which of the MSE of the literal passes: which = 0:
-// res_row[ntiles[row_slot]] -> mse_trace[idx_trace] (or out_row[mi]);
-// which = 1: res_col[ntiles[COL]] -> mse_half[idx_half] (or out_col[mi]).
-// Called by a whole warp.
+// res_row[ntiles[row_slot]] (or, with row_slot = kSlotRows, the row
+// finalize's per-chunk errors mse_part) -> mse_trace[idx_trace] (or
+// out_row[mi]); which = 1: res_col[ntiles[COL]] -> mse_half[idx_half] (or
+// out_col[mi]).  Called by a whole warp.
+constexpr int kSlotRows = 3;
 __device__ __forceinline__ void mse_literal_item(const Table &tab, int blk, int row_slot,
                                                  int idx_trace, int idx_half, double *out_row,
                                                  double *out_col) {
@@ -1266,8 +1279,9 @@ __device__ __forceinline__ void mse_literal_item(const Table &tab, int blk, int 
     int64_t n;
     if (which == 0) {
         dst = out_row ? out_row + mi : (md.mse_trace && idx_trace >= 0 ? md.mse_trace + idx_trace : nullptr);
-        src = md.res_row;
-        n = (row_slot >= 0) ? md.ntiles[row_slot] : 0;
+        src = row_slot == kSlotRows ? md.mse_part : md.res_row;
+        n = row_slot == kSlotRows ? (md.rows + kRowFinRows - 1) / kRowFinRows
+                                  : ((row_slot >= 0) ? md.ntiles[row_slot] : 0);
     } else {
         dst = out_col ? out_col + mi : (md.mse_half && idx_half >= 0 ? md.mse_half + idx_half : nullptr);
         src = md.res_col;
@@ -1300,9 +1314,10 @@ __device__ __forceinline__ void mse_fused_item(const Table &tab, int blk,
     const double *src1 = rows_mse ? md.mse_part : md.res_row;
     const int64_t n1 = rows_mse ? (md.rows + kRowFinRows - 1) / kRowFinRows : md.ntiles[MODE_COL];
     if (which == 0) {
+        // (with rows_mse a literal row step's error comes from its row sums too)
         dst = md.mse_trace ? md.mse_trace + idx : nullptr;
-        src = lit_row ? md.res_row : src1;
-        n = lit_row ? md.ntiles[MODE_ROW] : n1;
+        src = (lit_row && !rows_mse) ? md.res_row : src1;
+        n = (lit_row && !rows_mse) ? md.ntiles[MODE_ROW] : n1;
     } else {
         dst = md.mse_half ? md.mse_half + idx : nullptr;
         src = lit_col ? md.res_col : src1;
@@ -1370,8 +1385,9 @@ __device__ __forceinline__ void col_lane_unit(const Table &tab, const MatDesc &m
 // With mse_mode != 0 the last ceil(2n / 8) blocks of the grid finish the
 // iteration's MSE instead, a warp per item (1: mse_fused_item with flags /
 // next_flags; 3: the same with the per-row errors of the row finalize; 2:
-// mse_literal_item of the row and column passes), saving a launch.
-enum { MSE_NONE = 0, MSE_FUSED = 1, MSE_LITERAL = 2, MSE_FUSED_ROWS = 3 };
+// mse_literal_item of the row and column passes; 4: the same with the
+// per-row errors), saving a launch.
+enum { MSE_NONE = 0, MSE_FUSED = 1, MSE_LITERAL = 2, MSE_FUSED_ROWS = 3, MSE_LITERAL_ROWS = 4 };
 template <int OS>
 __global__ void __launch_bounds__(kColFinThreads, 3)
 col_finalize_kernel(const __grid_constant__ Table tab, int64_t total_units, int mse_mode,
@@ -1384,7 +1400,8 @@ col_finalize_kernel(const __grid_constant__ Table tab, int64_t total_units, int 
         if (blk >= 2 * tab.n) return;                   // (uniform per warp)
         if (mse_mode == MSE_FUSED || mse_mode == MSE_FUSED_ROWS)
             mse_fused_item(tab, blk, flags, next_flags, idx, mse_mode == MSE_FUSED_ROWS);
-        else mse_literal_item(tab, blk, MODE_ROW, idx, idx, nullptr, nullptr);
+        else mse_literal_item(tab, blk, mse_mode == MSE_LITERAL_ROWS ? kSlotRows : MODE_ROW, idx, idx,
+                              nullptr, nullptr);
         return;
     }
     __shared__ double sp[kColFinSlices][kColFinCols], se[kColFinSlices][kColFinCols];

@@ -213,6 +213,9 @@ cudaError_t launch_tile_combo(const TileLaunch &L) {
         case MODE_FUSED:
             if constexpr (GS == SC_E8M0 && OS == SC_E8M0) { DQ_BY_T(MODE_FUSED); }
             return cudaErrorInvalidValue;
+        case MODE_ROW_W2:
+            if constexpr (CodeTraits<CODES>::kBits == 4) { DQ_BY_T(MODE_ROW_W2); }
+            return cudaErrorInvalidValue;
         case MODE_FUSED_W2:
             if constexpr (GS == SC_E8M0 && OS == SC_E8M0 && CodeTraits<CODES>::kBits == 4) {
                 DQ_BY_T(MODE_FUSED_W2);

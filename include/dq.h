@@ -170,10 +170,11 @@ DQ_API dq_status dq_dequantize(const uint8_t *codes, const void *gscales, int64_
  * the ts used.  mse_trace (T+1) and mse_half (T) may be NULL; entry t is
  * mean((W - D_a Qhat D_b)^2) of the state before iteration t's row step
  * (mse_half: before its column step), the last entry that of the final
- * state.  The last entry is summed as (W - R)^2; for MXFP4 and MXINT4 the
- * others are taken per row as sum W^2 - 2 sum W R + sum R^2 from float32 row
- * sums (correct to about 1e-5 relative, exactly 0 for rows that Q
- * reproduces).  `workspace` must hold dq_workspace_size bytes for this one
+ * state.  The last entry is summed as (W - R)^2; for the formats with 4-bit
+ * codes (INT4, E2M1) the others are taken per row as sum W^2 - 2 a sum W R
+ * + a^2 sum R^2 from float32 row sums (correct to about 1e-5 relative; for
+ * MXFP4 and MXINT4, whose sums are taken for a = 1, exactly 0 for rows that
+ * Q reproduces); mse_half entries of the literal formats sum (W - R)^2.  `workspace` must hold dq_workspace_size bytes for this one
  * matrix. */
 DQ_API dq_status dq_solve_dual_scale(const void *W, int32_t dtype, int64_t rows, int64_t cols,
                               const dq_format *fmt, int32_t T, const float *a0,
@@ -227,7 +228,8 @@ DQ_API dq_status dq_graph_destroy(dq_graph g);
  * a_out_i = Pi_Fa(<W_i, R_i> / <R_i, R_i>), R = Q(W ⊘ a_in b_inᵀ) D_b, zero
  * slice -> 1.  a_pre (rows, may be NULL) receives the unprojected ratio
  * (NaN on zero slices); mse_in (1 double, may be NULL) the MSE of the input
- * state.  a_out may alias a_in. */
+ * state (for 4-bit codes formed per row from the row sums, as in the
+ * solves; see dq_solve_dual_scale).  a_out may alias a_in. */
 DQ_API dq_status dq_row_update(const void *W, int32_t dtype, int64_t rows, int64_t cols,
                         const dq_format *fmt, float tensor_scale, const float *a_in,
                         const float *b_in, float *a_out, float *a_pre, double *mse_in,

@@ -193,7 +193,11 @@ def test_half_steps_from_identical_state(name, dtype):
     assert np.array_equal(np.isnan(pre), np.isnan(x_or))
     assert np.max(np.abs(pre[ok] - x_or[ok]) / x_or[ok]) < 1e-5
     check_projected(np64(a_gpu), a_or, x_or, fo, "a")
-    assert abs(mse0.item() - O.mse(W64, Qh, a, b)) <= 1e-6 * O.mse(W64, Qh, a, b)
+    # (4-bit codes: the state's error is formed per row as sum W^2 - 2 a sum
+    # W R + a^2 sum R^2 from float32 row sums, each about 100 times the
+    # error; wider codes sum (W - a R)^2 directly)
+    tol0 = 1e-6 if name in MX_MORE else 2e-5
+    assert abs(mse0.item() - O.mse(W64, Qh, a, b)) <= tol0 * O.mse(W64, Qh, a, b)
     # column step from (a_gpu, b)
     a1 = np64(a_gpu)
     b_gpu, b_pre, mse1 = dq.col_update(Wd, fl, a_gpu, bd, ts)

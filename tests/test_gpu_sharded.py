@@ -2,12 +2,12 @@
 shards of one matrix run in lockstep in this process, their column partial
 slabs concatenated in row order as the all-gather of a multi-GPU run would,
 and the result must be the unsharded solve's bit for bit (a, b, codes,
-group scales).  The MSE trace agrees within 1e-6 relative: each tile sums
-its residual in float32 per lane over its rows, so the shards' tile
-geometry changes the last bits of the trace (not the state).  For MXFP4 the
-unsharded solve's one-pass iterations take each row's error from its row
-sums (sum W^2 - 2 sum W R + sum R^2, float32 sums of terms about 100 times
-the error), so there the trace agrees within 2e-5."""
+group scales).  The MSE trace agrees within 1e-6 relative: the row errors
+of these 4-bit formats come from the row sums (sum W^2 - 2 a sum W R + a^2
+sum R^2), the same per row in both, summed in another grouping.  For MXFP4
+the unsharded solve's one-pass iterations form them from their a = 1 sums
+(float32 sums of terms about 100 times the error), so there the trace
+agrees within 2e-5."""
 import numpy as np
 import pytest
 import torch
