@@ -23,6 +23,7 @@ from __future__ import annotations
 import argparse
 import datetime
 import hashlib
+import re
 import glob
 import json
 import math
@@ -77,17 +78,30 @@ def _peaks():
         return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}, "fallback"
 
 
+def _code_only(text):
+    """C++ source without its comments and blank lines (a change to a comment
+    changes no kernel)."""
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    out = []
+    for line in text.splitlines():
+        line = re.sub(r"//.*$", "", line).rstrip()
+        if line.strip():
+            out.append(line)
+    return "\n".join(out)
+
+
 def _src_hash():
-    """Hash of the sources that fix the tile kernels and their launch geometry
-    (the device header, the launch header and the per-format tile units); the
-    host API, the GEMM and the two-level kernel do not change their traffic."""
+    """Hash of the code (comments left out) of the sources that fix the tile
+    kernels and their launch geometry (the device header, the launch header
+    and the per-format tile units); the host API, the GEMM and the two-level
+    kernel do not change their traffic."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "dual_scale_solver_b200", "csrc")
     files = [os.path.join(csrc, "dq_device.cuh"), os.path.join(csrc, "dq_launch.h")]
     files += sorted(glob.glob(os.path.join(csrc, "dq_tiles_c*.cu")))
     for p in files:
-        with open(p, "rb") as f:
-            h.update(f.read())
+        with open(p, encoding="utf-8") as f:
+            h.update(_code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

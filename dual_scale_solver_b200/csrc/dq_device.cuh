@@ -722,9 +722,12 @@ __device__ __forceinline__ float project_outer(float x, bool &clamped) {
 // for the whole tile; arithmetic runs on float32 pairs (FFMA2/FMUL2).
 //   ROW : per row, sum_j W_ij R_ij and sum_j R_ij^2 (R = Qhat D_b) over the
 //         tile's columns -> rowpart[row][cb]; residual of the state -> res_row
+//         (wider than 4-bit codes; for 4-bit codes the row finalize forms
+//         it from the row sums)
 //   COL : per column, sum_i W_ij S_ij and sum_i S_ij^2 (S = D_a Qhat) over the
 //         tile's rows -> colpart[rb][col]; residual -> res_col
 //   FUSED (power-of-two scales): ROW and COL from one quantization
+//   ROW_W2, FUSED_W2 (4-bit codes): also sum_j W_ij^2 per row -> rowsq[row][cb]
 //   PACK: codes and group scales of Q(W / (a b)); residual -> res_row
 //   ACT : codes and group scales of Q(X * b)
 // Tiles have up to kRowsPerWarp[mode] rows per warp (the host picks fewer for
