@@ -24,8 +24,8 @@
 // accumulating in float32 in TMEM.  K advances in tiles of 256 elements (128
 // bytes per row) through a 4-stage shared-memory ring that runs on across
 // output tiles:
-//   warp 0     producer: TMA loads of the A and B tiles (128-byte swizzle,
-//              no multicast) and bulk copies of their scale tiles;
+//   warp 0     producer: TMA loads of the A and B tiles (128-byte swizzle;
+//              every CTA loads its own) and bulk copies of their scale tiles;
 //   warp 1     TMEM allocation; lane 0 issues tcgen05.cp (scales to TMEM),
 //              the MMAs and the tcgen05.commit arrivals;
 //   warps 2-9  epilogue: TMEM -> registers (tcgen05.ld; TMEM is handed back
@@ -132,7 +132,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *b, uint32_t parity, volatile
     return false;
 }
 
-// Untiled bulk copy global -> shared (no multicast), completion counted in
+// Untiled bulk copy global -> this CTA's shared memory, completion counted in
 // bytes on the mbarrier; both addresses 16-byte aligned, size a multiple of 16.
 __device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
     asm volatile(
@@ -525,9 +525,9 @@ __device__ __forceinline__ void cluster_sync_all() {
                  "barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
-// TMA load into this CTA's shared memory whose completion is counted on an
-// mbarrier of either CTA of the pair (bar: shared::cluster address).  No
-// multicast.
+// TMA load into this CTA's shared memory (and no other CTA's) whose
+// completion is counted on an mbarrier of either CTA of the pair (bar:
+// shared::cluster address).
 __device__ __forceinline__ void tma_load_2d_pair(void *dst, const CUtensorMap *map, int x, int y,
                                                  uint32_t bar) {
     asm volatile(
