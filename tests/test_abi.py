@@ -198,6 +198,10 @@ def test_sharded_column_entry_points_argument_errors():
     assert L.dq_col_row_block(-1, 64, 1) == -1
     assert L.dq_col_row_block(64, 64, 7) == -1
     assert L.dq_col_row_block(14336, 4096, 1) == 256        # 256 rows per warp, 1 warp row
+    # a matrix whose column pass alone makes 8 waves of tiles takes at least
+    # 64 rows per warp (the "tall" geometry); a smaller one 16
+    assert L.dq_col_row_block(256, 1310720, 1) == 64         # 1 warp row, 64 rows per warp
+    assert L.dq_col_row_block(1536, 2240, 1) == 128          # 8 warp rows, 16 rows per warp
     assert L.dq_col_row_block(100, 4096, 1) % 1 == 0 and L.dq_col_row_block(100, 4096, 1) > 0
     p = ctypes.c_void_p(256)                                 # never dereferenced
     ws = ctypes.c_void_p(1 << 20)
