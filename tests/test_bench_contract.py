@@ -83,3 +83,13 @@ def test_traffic_guarded_by_tile_source_hash(tmp_path, monkeypatch):
     monkeypatch.setattr(bench, "_src_hash", lambda: h)
     assert bench._traffic("k") == 123.0
     assert bench._traffic("old") is None and bench._traffic("missing") is None
+
+
+def test_source_hash_ignores_comments_only():
+    # the hash that ties profiles/traffic.json to the tile sources sees code,
+    # not comments or blank lines
+    a = "int f(int x) {  // one\n    return x + 1;  /* two\n three */\n}\n"
+    b = "int f(int x) {\n\n    return x + 1;\n}  // other words\n"
+    c = "int f(int x) {\n    return x + 2;\n}\n"
+    assert bench._code_only(a) == bench._code_only(b)
+    assert bench._code_only(a) != bench._code_only(c)
